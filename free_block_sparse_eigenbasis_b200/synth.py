@@ -1,0 +1,199 @@
+"""Seeded synthetic Q/K/V generators and the named workloads.
+
+This module is shared by the CUDA path's tests/bench and by the fp64 oracle's
+tests. It holds only input recipes (shapes, seeds, value distributions); none
+of the method's arithmetic lives here.
+
+Workloads (video-DiT-shaped attention layers; the sizes are those of the
+layers the SparsePR and SVOO pages evaluate on, the values are synthetic
+because trained weights and prompts are not available):
+
+    tiny              1 head,  d=64,  fp32, N=256 on a 4x8x8 grid
+    wan13b_480p      12 heads, d=128, bf16, N=32,760 on 21x30x52
+    wan13b_720p      12 heads, d=128, bf16, N=75,600 on 21x45x80
+    wan14b_720p      40 heads, d=128, bf16, N=75,600, per-head keep in [0.15,0.35]
+    hunyuan13b_720p  24 heads, d=128, bf16, N=118,800 video + 256 text tokens
+
+Value recipe per head (all draws from numpy PCG64 seeded with (seed, head)):
+  * a smooth spatio-temporal field F_c(t,h,w) = sin(2*pi*(a_c t/T + b_c h/Hh
+    + c_c w/W) + phi_c) per channel c, a,b,c integers in {0,1,2},
+    phi ~ U[0, 2*pi), amplitude 1, shared by Q and K of the head;
+  * a Gaussian mixture: one component label per token, shared by Q and K,
+    with separate component means mu^Q, mu^K ~ N(0, I) and spread sigma;
+  * optional white noise of the stated variance;
+  * Q and K are then standardised per channel (zero mean, unit variance
+    over the video tokens); V ~ N(0, 1);
+  * text tokens (if any) are the trailing indices: N(0,1) values plus one
+    N(0, I) offset vector per head added to all text Q and K rows.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    H: int
+    grid: tuple  # (T, Hh, W) latent grid of the video tokens
+    d: int
+    dtype: str  # "bf16" | "f32"
+    n_comp: int  # mixture components
+    sigma: float  # mixture spread
+    noise_var: float  # extra white-noise variance
+    n_text: int
+    # method parameters
+    Ck: int
+    Cq: int
+    Ms: int
+    n_eig: int
+    kmeans_iters: int
+    keep: tuple  # per-head keep fraction of key groups
+    M: int
+    r: int
+    lam: float
+    scale: float  # 0 -> 1/sqrt(d)
+    seed: int
+
+    @property
+    def Nv(self) -> int:
+        T, Hh, W = self.grid
+        return T * Hh * W
+
+    @property
+    def N(self) -> int:
+        return self.Nv + self.n_text
+
+    def params(self) -> dict:
+        """Method parameters as a plain dict (the form both sides accept)."""
+        return dict(H=self.H, N=self.N, d=self.d, n_text=self.n_text,
+                    Ck=self.Ck, Cq=self.Cq, Ms=self.Ms, n_eig=self.n_eig,
+                    kmeans_iters=self.kmeans_iters, keep=list(self.keep),
+                    M=self.M, r=self.r, lam=self.lam, scale=self.scale,
+                    seed=self.seed)
+
+
+def _keep_uniform(seed: int, H: int, lo: float, hi: float) -> tuple:
+    rng = np.random.default_rng([seed, 1_000_003])
+    return tuple(float(lo + (hi - lo) * u) for u in rng.random(H))
+
+
+def _keep_beta12(seed: int, H: int, lo: float, hi: float) -> tuple:
+    # lo + (hi-lo) * Beta(1,2): support [lo, hi], mean lo + (hi-lo)/3
+    rng = np.random.default_rng([seed, 1_000_003])
+    return tuple(float(lo + (hi - lo) * (1.0 - math.sqrt(1.0 - u)))
+                 for u in rng.random(H))
+
+
+def workload(name: str, heads: Optional[int] = None) -> Workload:
+    """Return a named workload. ``heads`` truncates the head count (the
+    per-head values of the first ``heads`` heads are unchanged)."""
+    if name == "tiny":
+        w = Workload(name, 1, (4, 8, 8), 64, "f32", 8, 0.3, 0.0, 0,
+                     Ck=16, Cq=8, Ms=64, n_eig=2, kmeans_iters=10,
+                     keep=(0.25,), M=16, r=8, lam=1e-3, scale=0.0, seed=0)
+    elif name == "wan13b_480p":
+        w = Workload(name, 12, (21, 30, 52), 128, "bf16", 64, 0.5, 0.1, 0,
+                     Ck=500, Cq=100, Ms=512, n_eig=16, kmeans_iters=10,
+                     keep=(0.25,) * 12, M=256, r=32, lam=1e-2, scale=0.0,
+                     seed=1)
+    elif name == "wan13b_720p":
+        w = Workload(name, 12, (21, 45, 80), 128, "bf16", 128, 0.5, 0.1, 0,
+                     Ck=1000, Cq=200, Ms=1024, n_eig=16, kmeans_iters=10,
+                     keep=(0.22,) * 12, M=512, r=32, lam=1e-2, scale=0.0,
+                     seed=2)
+    elif name == "wan14b_720p":
+        w = Workload(name, 40, (21, 45, 80), 128, "bf16", 128, 0.5, 0.1, 0,
+                     Ck=1000, Cq=200, Ms=1024, n_eig=16, kmeans_iters=10,
+                     keep=_keep_uniform(3, 40, 0.15, 0.35), M=512, r=32,
+                     lam=1e-2, scale=0.0, seed=3)
+    elif name == "hunyuan13b_720p":
+        w = Workload(name, 24, (33, 45, 80), 128, "bf16", 128, 0.5, 0.1, 256,
+                     Ck=1500, Cq=300, Ms=1024, n_eig=16, kmeans_iters=10,
+                     keep=_keep_beta12(4, 24, 0.18, 0.30), M=768, r=48,
+                     lam=1e-2, scale=0.0, seed=4)
+    else:
+        raise KeyError(name)
+    if heads is not None:
+        w = dataclasses.replace(w, H=heads, keep=w.keep[:heads])
+    return w
+
+
+def custom(name: str, H: int, grid: tuple, d: int, dtype: str, **kw) -> Workload:
+    """A small workload of the same recipe (for parity cases between the
+    named sizes)."""
+    base = dict(n_comp=16, sigma=0.5, noise_var=0.1, n_text=0, Ck=32, Cq=8,
+                Ms=128, n_eig=8, kmeans_iters=10, M=32, r=16, lam=1e-2,
+                scale=0.0, seed=7)
+    base.update(kw)
+    keep = base.pop("keep", 0.25)
+    if not isinstance(keep, (tuple, list)):
+        keep = (keep,) * H
+    return Workload(name, H, tuple(grid), d, dtype, keep=tuple(keep), **base)
+
+
+def _head_values(w: Workload, h: int):
+    """fp64 Q, K, V of one head, [N, d] each."""
+    T, Hh, W = w.grid
+    Nv, d = w.Nv, w.d
+    rng = np.random.default_rng([w.seed, h])
+    # spatio-temporal field, shared by Q and K
+    abc = rng.integers(0, 3, size=(3, d)).astype(np.float64)
+    phi = rng.random(d) * 2.0 * np.pi
+    t = np.repeat(np.arange(T), Hh * W).astype(np.float64) / T
+    hh = np.tile(np.repeat(np.arange(Hh), W), T).astype(np.float64) / Hh
+    ww = np.tile(np.arange(W), T * Hh).astype(np.float64) / W
+    arg = (t[:, None] * abc[0][None, :] + hh[:, None] * abc[1][None, :]
+           + ww[:, None] * abc[2][None, :])
+    field = np.sin(2.0 * np.pi * arg + phi[None, :])
+    # mixture
+    comp = rng.integers(0, w.n_comp, size=Nv)
+    mu_q = rng.standard_normal((w.n_comp, d))
+    mu_k = rng.standard_normal((w.n_comp, d))
+    q = field + mu_q[comp] + w.sigma * rng.standard_normal((Nv, d))
+    k = field + mu_k[comp] + w.sigma * rng.standard_normal((Nv, d))
+    if w.noise_var > 0:
+        s = math.sqrt(w.noise_var)
+        q += s * rng.standard_normal((Nv, d))
+        k += s * rng.standard_normal((Nv, d))
+    for x in (q, k):
+        x -= x.mean(axis=0, keepdims=True)
+        x /= x.std(axis=0, keepdims=True)
+    v = rng.standard_normal((w.N, d))
+    if w.n_text:
+        off = rng.standard_normal(d)
+        qt = rng.standard_normal((w.n_text, d)) + off
+        kt = rng.standard_normal((w.n_text, d)) + off
+        q = np.concatenate([q, qt], axis=0)
+        k = np.concatenate([k, kt], axis=0)
+    return q, k, v
+
+
+def torch_dtype(w: Workload):
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+def generate(w: Workload, heads=None):
+    """Q, K, V as CPU torch tensors [H', N, d] in the workload's dtype, for the
+    heads listed in ``heads`` (default: all). Values are generated in fp64 and
+    rounded by torch's conversion to the workload dtype."""
+    hs = range(w.H) if heads is None else list(heads)
+    dt = torch_dtype(w)
+    out = []
+    for x_idx in range(3):
+        out.append(torch.empty((len(hs), w.N, w.d), dtype=dt))
+    for i, h in enumerate(hs):
+        vals = _head_values(w, h)
+        for x_idx in range(3):
+            out[x_idx][i].copy_(torch.from_numpy(vals[x_idx]).to(dt))
+    return tuple(out)
+
+
+def as_f64(x: torch.Tensor) -> np.ndarray:
+    """Widen a (bf16/fp32) tensor exactly to a float64 numpy array."""
+    return x.to(torch.float64).numpy()

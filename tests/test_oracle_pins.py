@@ -1,0 +1,373 @@
+"""Pins of the fp64 oracle against things other than itself: published
+generator outputs, closed forms, hand-worked examples (tests/golden), brute
+force on tiny inputs, invariants the pages fix, and library re-derivations
+through a different formula or routine. CPU only."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import sparsepr_oracle as O
+from free_block_sparse_eigenbasis_b200 import synth
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")))
+
+
+# -- random draws -----------------------------------------------------------
+
+def test_splitmix64_published_outputs():
+    g = O.splitmix64_stream(0)
+    assert [next(g) for _ in range(3)] == [int(h, 16) for h in GOLD["splitmix64"]["seed0_hex"]]
+    g = O.splitmix64_stream(1234567)
+    assert [next(g) for _ in range(3)] == GOLD["splitmix64"]["seed1234567"]
+
+
+def test_init_indices_distinct_and_seeded():
+    a = O.init_indices(1000, 200, 5, 3, 0)
+    assert len(set(a.tolist())) == 200 and a.min() >= 0 and a.max() < 1000
+    assert not np.array_equal(a, O.init_indices(1000, 200, 5, 3, 1))
+    assert np.array_equal(a, O.init_indices(1000, 200, 5, 3, 0))
+    # C = n is a full permutation
+    assert sorted(O.init_indices(17, 17, 1, 0, 0).tolist()) == list(range(17))
+
+
+def test_init_indices_first_draw_uniform():
+    # the first slot is a uniform draw over range(n): chi-square over seeds
+    n = 8
+    counts = np.zeros(n)
+    for s in range(4000):
+        counts[O.init_indices(n, 1, s, 0, 0)[0]] += 1
+    chi2 = ((counts - 500.0) ** 2 / 500.0).sum()
+    assert chi2 < 30.0  # 7 dof, p ~ 1e-4
+
+
+# -- stage 1 ----------------------------------------------------------------
+
+def test_sample_rows_hand_example():
+    gs = GOLD["sample_rows"]
+    assert O.sample_rows(gs["Nv"], gs["Ms"]).tolist() == gs["rows"]
+    assert O.sample_rows(37, 37).tolist() == list(range(37))
+
+
+def test_metric_quadratic_form_is_response_energy():
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((300, 6))
+    MK = O.metric_MK(q, 50)
+    Qs = q[O.sample_rows(300, 50)]
+    for _ in range(5):
+        x = rng.standard_normal(6)
+        # x^T M_K x = mean_s (q_s . x)^2
+        direct = sum(float(Qs[s] @ x) ** 2 for s in range(50)) / 50
+        assert abs(x @ MK @ x - direct) < 1e-10 * max(1.0, direct)
+    assert np.allclose(MK, MK.T)
+
+
+def test_eigenbasis_closed_form_and_residuals():
+    A = np.array(GOLD["eigen_2x2"]["A"])
+    lam, U = O.eigenbasis(A, 2)
+    assert np.allclose(lam, GOLD["eigen_2x2"]["lam"], atol=1e-14)
+    assert abs(abs(U[0, 0]) - 1 / math.sqrt(2)) < 1e-14
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((40, 12))
+    MK = X.T @ X / 40
+    lam, U = O.eigenbasis(MK, 5)
+    assert np.all(np.diff(lam) <= 0)
+    assert np.allclose(U.T @ U, np.eye(5), atol=1e-12)
+    assert np.abs(MK @ U - U * lam).max() < 1e-12
+    # the full spectrum sums to the trace
+    lam_all, _ = O.eigenbasis(MK, 12)
+    assert abs(lam_all.sum() - np.trace(MK)) < 1e-12
+
+
+def test_key_coordinates_give_response_profile_distance():
+    """With e = d, ||z1 - z2||^2 = ||Q_s (k1 - k2)||^2 / M_s."""
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((200, 8))
+    k = rng.standard_normal((30, 8))
+    Ms = 64
+    lam, U = O.eigenbasis(O.metric_MK(q, Ms), 8)
+    Z = O.key_coordinates(k, lam, U)
+    Qs = q[O.sample_rows(200, Ms)]
+    for i, j in [(0, 1), (3, 17), (29, 5)]:
+        resp = ((Qs @ (k[i] - k[j])) ** 2).sum() / Ms
+        assert abs(((Z[i] - Z[j]) ** 2).sum() - resp) < 1e-10 * resp
+
+
+def test_nearest_brute_force_and_ties():
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((50, 3))
+    C = rng.standard_normal((7, 3))
+    got = O.nearest(X, C, chunk=16)
+    for i in range(50):
+        d = [sum((X[i, t] - C[j, t]) ** 2 for t in range(3)) for j in range(7)]
+        assert got[i] == min(range(7), key=lambda j: (d[j], j))
+    # exact tie: the lower index wins
+    C2 = np.array([[1.0, 0.0], [-1.0, 0.0], [1.0, 0.0]])
+    assert O.nearest(np.array([[0.0, 0.0], [2.0, 0.0]]), C2).tolist() == [0, 0]
+
+
+def test_lloyd_fixed_point_and_planted_recovery():
+    rng = np.random.default_rng(4)
+    centers = rng.standard_normal((5, 4)) * 20
+    lab = rng.integers(0, 5, 400)
+    X = centers[lab] + 1e-3 * rng.standard_normal((400, 4))
+    init = O.init_indices(400, 5, 9, 0, 0)
+    labels, mu, passes = O.lloyd(X, init, 50)
+    # converged: labels equal the assignment to the group means
+    assert passes < 50
+    assert np.array_equal(O.nearest(X, O.group_means(X, labels, 5, prev=mu)), labels)
+    # planted clusters recovered up to relabelling when all 5 were seeded
+    if len(set(lab[init].tolist())) == 5:
+        for c in range(5):
+            assert len(set(labels[lab == c].tolist())) == 1
+
+
+def test_lloyd_empty_group_keeps_centroid():
+    X = np.array([[0.0], [0.1], [10.0]])
+    # centroids start at rows 0 and 1; row 2 joins group 1, row 0 group 0
+    labels, mu, _ = O.lloyd(X, np.array([0, 1]), 1)
+    assert labels.tolist() == [0, 1, 1]
+    m = O.group_means(X, np.array([0, 0, 0]), 2, prev=np.array([[5.0], [7.0]]))
+    assert m[1, 0] == 7.0 and abs(m[0, 0] - 10.1 / 3) < 1e-15
+
+
+def test_query_profile_distance_equals_metric_form():
+    """||p_i - pbar_g||^2 = (q_i - qbar_g)^T G (q_i - qbar_g), G = s^2 C_K^T C_K:
+    the oracle's literal Ck-dim profile distance against the d-dim form."""
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((60, 8))
+    CK = rng.standard_normal((20, 8))
+    s = 0.3
+    P = O.query_profiles(q, CK, s)
+    G = s * s * CK.T @ CK
+    lab = rng.integers(0, 4, 60)
+    pbar = O.group_means(P, lab, 4)
+    qbar = O.group_means(q, lab, 4)
+    D_lit = O.sqdist(P, pbar)
+    for i in range(0, 60, 7):
+        for g in range(4):
+            x = q[i] - qbar[g]
+            assert abs(D_lit[i, g] - x @ G @ x) < 1e-9 * max(1.0, D_lit[i, g])
+
+
+# -- stage 2 ----------------------------------------------------------------
+
+def test_group_major_round_trip_and_stability():
+    rng = np.random.default_rng(6)
+    lab = rng.integers(0, 9, 500)
+    perm, inv, off = O.group_major(lab, 9)
+    assert np.array_equal(perm[inv], np.arange(500))
+    assert np.array_equal(inv[perm], np.arange(500))
+    assert np.array_equal(np.diff(off), np.bincount(lab, minlength=9))
+    for c in range(9):
+        seg = perm[off[c]:off[c + 1]]
+        assert np.all(lab[seg] == c) and np.all(np.diff(seg) > 0)
+    X = rng.standard_normal((500, 3))
+    assert np.array_equal(X[perm][inv], X)
+
+
+# -- stage 3 ----------------------------------------------------------------
+
+def test_keep_budget_cases():
+    for keep, Ck, k in GOLD["keep_budget"]["cases"]:
+        assert O.keep_budget(keep, Ck) == k, (keep, Ck)
+
+
+def test_route_hand_example():
+    ge = GOLD["route_example"]
+    for k, want in ge["k_to_csr"]:
+        assert O.route(np.array(ge["CQ"]), np.array(ge["CK"]), k, 1.0)[0].tolist() == want
+
+
+def test_route_brute_force_all_subsets():
+    """On 16 key groups and k=4: the kept set maximises the summed score, with
+    ties broken towards the lexicographically smallest set -- all C(16,4)."""
+    rng = np.random.default_rng(7)
+    CQ = rng.standard_normal((8, 5))
+    CK = rng.standard_normal((16, 5))
+    CK[5] = CK[2]  # an exact tie
+    A = 0.5 * CQ @ CK.T
+    csr = O.route(CQ, CK, 4, 0.5)
+    for g in range(8):
+        best = max(itertools.combinations(range(16), 4),
+                   key=lambda s: (sorted(A[g, list(s)].tolist(), reverse=True), [-c for c in s]))
+        assert list(best) == csr[g].tolist()
+
+
+def test_masked_attention_matches_pseudo_code_and_closed_form():
+    # two kept keys: logistic weights
+    Qp = np.array([[1.0, 0.0]])
+    Kp = np.array([[1.0, 0.0], [0.0, 0.0], [5.0, 5.0]])
+    Vp = np.array([[1.0, 0.0], [0.0, 1.0], [100.0, 100.0]])
+    mask = np.array([True, True, False])
+    o = O.masked_attention_rows(Qp, Kp, Vp, [0], lambda i: 0, lambda g: mask, 1.0)
+    w1 = GOLD["two_key_attention"]["w1"]
+    assert np.allclose(o[0], [w1, 1 - w1], atol=1e-15)
+    # random case against an explicit loop over kept keys
+    rng = np.random.default_rng(8)
+    Q = rng.standard_normal((5, 4))
+    K = rng.standard_normal((30, 4))
+    V = rng.standard_normal((30, 3))
+    m = rng.random(30) < 0.4
+    o = O.masked_attention_rows(Q, K, V, range(5), lambda i: 0, lambda g: m, 0.7)
+    for i in range(5):
+        kept = [j for j in range(30) if m[j]]
+        logits = [0.7 * sum(Q[i, t] * K[j, t] for t in range(4)) for j in kept]
+        mx = max(logits)
+        ws = [math.exp(l - mx) for l in logits]
+        tot = sum(ws)
+        ref = [sum(ws[a] * V[j, c] for a, j in enumerate(kept)) / tot for c in range(3)]
+        assert np.allclose(o[i], ref, atol=1e-13)
+
+
+def test_dense_attention_explicit_loop():
+    rng = np.random.default_rng(9)
+    Q = rng.standard_normal((4, 3))
+    K = rng.standard_normal((6, 3))
+    V = rng.standard_normal((6, 2))
+    o = O.dense_attention(Q, K, V, 0.5)
+    for i in range(4):
+        ws = [math.exp(0.5 * float(Q[i] @ K[j])) for j in range(6)]
+        ref = [sum(ws[j] * V[j, c] for j in range(6)) / sum(ws) for c in range(2)]
+        assert np.allclose(o[i], ref, atol=1e-14)
+
+
+# -- stage 4 ----------------------------------------------------------------
+
+def test_probe_counts_hand_examples():
+    for n, M, want in GOLD["probe_counts"]["cases"]:
+        assert O.probe_counts(np.array(n), M).tolist() == want
+
+
+def test_probe_counts_properties():
+    rng = np.random.default_rng(10)
+    for _ in range(50):
+        n = rng.integers(0, 40, rng.integers(1, 12))
+        if n.sum() == 0:
+            continue
+        M = int(rng.integers(0, n.sum() + 1))
+        m = O.probe_counts(n, M)
+        assert m.sum() == M and np.all(m <= n) and np.all(m >= 0)
+        quota = M * n / n.sum()
+        assert np.all(np.abs(m - quota) < 1.0)
+
+
+def test_probe_rows_hand_example():
+    gp = GOLD["probe_rows"]
+    assert O.probe_rows(np.array(gp["off"]), gp["M"]).tolist() == gp["rows"]
+
+
+def test_ridge_recovers_exact_affine_map():
+    rng = np.random.default_rng(11)
+    M, d = 40, 6
+    X = rng.standard_normal((M, d))
+    B0 = rng.standard_normal((d, d))
+    b0 = rng.standard_normal(d)
+    R = b0 + X @ B0
+    B, b = O.ridge_fit(X, R, 1e-12)
+    assert np.abs(B - B0).max() < 1e-8 and np.abs(b - b0).max() < 1e-8
+
+
+def test_ridge_matches_lstsq_and_limits():
+    rng = np.random.default_rng(12)
+    X = rng.standard_normal((30, 5))
+    R = rng.standard_normal((30, 5))
+    # lam = 0: ordinary least squares on [1, X] (a different routine)
+    B, b = O.ridge_fit(X, R, 0.0)
+    sol, *_ = np.linalg.lstsq(np.hstack([np.ones((30, 1)), X]), R, rcond=None)
+    assert np.abs(b - sol[0]).max() < 1e-10 and np.abs(B - sol[1:]).max() < 1e-10
+    # huge lam: B -> 0, b -> mean residual
+    B, b = O.ridge_fit(X, R, 1e12)
+    assert np.abs(B).max() < 1e-9 and np.abs(b - R.mean(0)).max() < 1e-9
+    # ridge optimality: gradient of the penalised loss vanishes
+    lam = 0.3
+    B, b = O.ridge_fit(X, R, lam)
+    E = R - b - X @ B
+    assert np.abs(X.T @ E - lam * B).max() < 1e-10 and np.abs(E.sum(0)).max() < 1e-10
+
+
+def test_subspace_projection_noop_at_full_rank_and_matches_eig():
+    rng = np.random.default_rng(13)
+    M, d, rank = 50, 8, 5
+    X = rng.standard_normal((M, d))
+    R = rng.standard_normal((M, rank)) @ rng.standard_normal((rank, d))
+    B, b = O.ridge_fit(X, R, 0.1)
+    Vr = O.residual_subspace(R, rank)
+    Bp, bp = O.project_map(B, b, Vr)
+    assert np.abs(Bp - B).max() < 1e-10 and np.abs(bp - b).max() < 1e-10
+    # leading subspace equals the top eigenvectors of R^T R
+    R2 = rng.standard_normal((M, d))
+    Vr = O.residual_subspace(R2, 3)
+    w, U = np.linalg.eigh(R2.T @ R2)
+    U3 = U[:, np.argsort(-w)[:3]]
+    assert np.abs(Vr @ Vr.T - U3 @ U3.T).max() < 1e-10
+    # R = 0 gives a zero correction
+    B, b = O.ridge_fit(X, np.zeros((M, d)), 0.1)
+    assert np.abs(B).max() == 0 and np.abs(b).max() == 0
+
+
+# -- whole head -------------------------------------------------------------
+
+def _tiny_head(keep=None, **kw):
+    w = synth.workload("tiny")
+    if keep is not None:
+        w = synth.custom("tiny_k", 1, w.grid, w.d, w.dtype, n_comp=8, sigma=0.3,
+                         noise_var=0.0, Ck=16, Cq=8, Ms=64, n_eig=2, M=16,
+                         r=8, lam=1e-3, seed=0, keep=keep, **kw)
+    q, k, v = synth.generate(w)
+    return w, synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0])
+
+
+def test_keep_one_is_dense_with_zero_residual():
+    w, q, k, v = _tiny_head(keep=1.0)
+    res = O.run_head(q, k, v, w.params(), 0)
+    D = O.dense_attention(q, k, v, 1 / math.sqrt(w.d))
+    out = O.output_original_order(res, w.N, w.d)
+    assert np.abs(out - D).max() < 1e-12
+    Os = np.zeros_like(D)
+    Os[res.perm_q] = res.o_sparse
+    assert np.abs(Os - D).max() < 1e-12
+    assert np.abs(res.o_dense_probe - res.o_sparse_probe).max() < 1e-12
+    assert np.abs(res.B).max() < 1e-9 and np.abs(res.b).max() < 1e-9
+    assert res.pairs_exec == w.N * w.N + w.M * w.N  # rho = 1 + M/N
+
+
+def test_tiny_head_invariants():
+    w, q, k, v = _tiny_head()
+    res = O.run_head(q, k, v, w.params(), 0)
+    N = w.N
+    assert res.k == 4 and res.csr.shape == (w.Cq, 4)
+    assert np.all(np.diff(res.csr, axis=1) > 0)
+    assert res.probes.size == w.M and np.all(np.diff(res.probes) > 0)
+    # pair count equals the number of kept (row, key) pairs of the masks
+    n_k = np.diff(res.off_k)
+    tot = 0
+    for g in range(w.Cq):
+        m = O.kept_key_mask(res.csr[g], res.off_k, N)
+        assert m.sum() == n_k[res.csr[g]].sum()
+        tot += (res.off_q[g + 1] - res.off_q[g]) * int(m.sum())
+    assert tot == res.pairs_sparse and res.pairs_exec == tot + w.M * N
+    assert np.all(np.isfinite(res.out))
+    # probe rows carry the dense output
+    D = O.dense_attention(q[res.perm_q], k, v, 1 / math.sqrt(w.d))
+    assert np.abs(res.out[res.probes] - D[res.probes]).max() < 1e-12
+    # labels are consistent with the permutation
+    assert np.array_equal(np.sort(res.label_q[res.perm_q]), res.label_q[res.perm_q])
+
+
+def test_text_tokens_reading():
+    w = synth.custom("txt", 1, (2, 4, 8), 32, "f32", n_text=8, Ck=8, Cq=4,
+                     Ms=32, n_eig=4, M=8, r=4, keep=0.25)
+    q, k, v = synth.generate(w)
+    q, k, v = synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0])
+    res = O.run_head(q, k, v, w.params(), 0)
+    Nv = w.Nv
+    assert np.all(res.label_k[Nv:] == w.Ck) and np.all(res.label_q[Nv:] == w.Cq)
+    assert np.all(res.probes < res.off_q[w.Cq])  # no text probes
+    # text rows are exact dense attention
+    D = O.dense_attention(q[res.perm_q], k[res.perm_k], v[res.perm_k], 1 / math.sqrt(w.d))
+    trows = np.arange(res.off_q[w.Cq], w.N)
+    assert np.abs(res.out[trows] - D[trows]).max() < 1e-12
