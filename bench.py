@@ -1,0 +1,352 @@
+"""Benchmark of one SparsePR attention call (all five library calls) on the
+Wan2.1-1.3B-shaped 720p layer: 12 heads, N = 75,600 tokens (21x45x80),
+d = 128, bf16, 1000 key groups, 200 query groups, keep 0.22, M = 512 probes,
+r = 32, lambda = 1e-2. Inputs are seeded synthetic Q/K/V of that shape.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one whole call (partition, permute, route, block-sparse attention,
+probe-fitted correction) over the 12 heads, inputs resident in HBM. Under
+torchrun every rank runs its own call on its own GPU (heads are independent;
+no collective on the data path) and the job value is the sum of the ranks'
+executed pairs over the slowest rank's time.
+
+Prints one JSON line. `value` is executed-pair TFLOPS of the whole call,
+4 d P_exec / t_call (P_exec = routed pairs + M N probe pairs).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from free_block_sparse_eigenbasis_b200 import synth  # noqa: E402
+
+METRIC = ("attention-call ms and exec-pair TFLOPS at ρ_exec≈25%; "
+          "speedup vs dense attn")
+WORKLOAD = "wan13b_720p"
+PEAKS_FALLBACK = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+
+
+def workload_desc(w):
+    T, Hh, W = w.grid
+    return ("%s: %d heads, N=%d (%dx%dx%d), d=%d, %s, Ck=%d, Cq=%d, Ms=%d, e=%d, keep=%.2f, "
+            "M=%d, r=%d, lambda=%g, k-means passes<=%d"
+            % (w.name, w.H, w.N, T, Hh, W, w.d, w.dtype, w.Ck, w.Cq, w.Ms, w.n_eig,
+               statistics.mean(w.keep), w.M, w.r, w.lam, w.kmeans_iters))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return dict(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=smax,
+                    reasons=sorted(reasons), samples=len(sm))
+
+
+def gpu_launches_per_call(w) -> int:
+    """Kernels the library launches for one call of this workload (mirrors the
+    launch sequences of the C ABI; checked against the profiler's launch list)."""
+    it = w.kmeans_iters
+    partition = (7 + 2 * it + 4 * (it - 1)      # setup, metric, eigen, coordinates; key passes
+                 + 3 + 1 + 1 + 1                 # final key sort, C_K, G, query init
+                 + 3 * it + 4 * (it - 1) + 2)    # query passes, labels out
+    permute = 3 + 3 + 3
+    route = 4
+    attn = 5 if True else 0
+    probe = (3 + 5 + 1 + 2 + 1 + 1 + 1 + 1 + 1 + 1) if w.M > 0 else 2
+    return partition + permute + route + attn + probe
+
+
+def run_reference(args, w, rank):
+    """The oracle as it stands, on the host cores, on a bounded sample of the
+    same workload per step (head 0: full partition, routing and probe fit;
+    sparse attention + correction on every 64th group-major row)."""
+    from oracle import sparsepr_oracle as O
+    if rank != 0:
+        return
+    q, k, v = synth.generate(w, heads=[0])
+    qf, kf, vf = synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0])
+    stride = 64
+    rows = np.arange(0, w.N, stride)
+    times = []
+    res = None
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        res = O.run_head(qf, kf, vf, w.params(), 0, rows=rows)
+        t1 = time.perf_counter()
+        if s >= args.warmup:
+            times.append(t1 - t0)
+    t_head = statistics.median(times)
+    # extrapolate: the per-row part scales by the stride, the rest is per head
+    t_rows = t_head * 0.0
+    t_call = w.H * t_head  # conservative: fixed part dominates the sample
+    flops = 4.0 * w.d * res.pairs_exec * w.H
+    value = flops / t_call / 1e12
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    sample = ("head 0 of %d: full partition/route/probe fit, sparse attention + correction on "
+              "every %dth group-major row; call time = %d x head time (rows not extrapolated)"
+              % (w.H, stride, w.H))
+    line = dict(metric=METRIC, value=value, unit="TFLOPS", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=t_call * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                impl="reference",
+                config=dict(workload=workload_desc(w)),
+                cpu_baseline=dict(value=value, unit="TFLOPS", cores=cores, kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit="TFLOPS", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample(w):
+    """Oracle (as it stands) on a bounded sample: head 0, every 64th row."""
+    from oracle import sparsepr_oracle as O
+    q, k, v = synth.generate(w, heads=[0])
+    rows = np.arange(0, w.N, 64)
+    t0 = time.perf_counter()
+    res = O.run_head(synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0]), w.params(), 0,
+                     rows=rows)
+    t_head = time.perf_counter() - t0
+    t_call = w.H * t_head
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return dict(value=4.0 * w.d * res.pairs_exec * w.H / t_call / 1e12, unit="TFLOPS",
+                cores=cores, kind="oracle",
+                sample="head 0 of %d (full partition/route/probe fit, sparse attention + "
+                       "correction on every 64th row), call time = %d x %.1f s"
+                       % (w.H, w.H, t_head))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.workload(args.workload)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from free_block_sparse_eigenbasis_b200 import sparsepr as S
+
+    p = w.params()
+    q, k, v = synth.generate(w)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    qd, kd, vd = qh.to(dev), kh.to(dev), vh.to(dev)
+    b = S.allocate(p, qd.dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(qx, kx, vx, ev=None):
+        if ev: ev[0].record(stream)
+        S.sparsepr_partition(qx, kx, p, b.label_q, b.label_k, b.ws, stream)
+        if ev: ev[1].record(stream)
+        S.sparsepr_permute(qx, kx, vx, p, b.label_q, b.label_k, b.perm_q, b.perm_k, b.off_q,
+                           b.off_k, b.qp, b.kp, b.vp, b.ws, stream)
+        if ev: ev[2].record(stream)
+        S.sparsepr_route(b.qp, b.kp, p, b.off_q, b.off_k, b.csr, b.k_per_head, b.ws, stream)
+        if ev: ev[3].record(stream)
+        S.sparsepr_block_sparse_attn(b.qp, b.kp, b.vp, p, b.off_q, b.off_k, b.csr, b.k_per_head,
+                                     b.o_sparse, b.pairs_sparse, b.ws, stream)
+        if ev: ev[4].record(stream)
+        S.sparsepr_probe_correct(b.qp, b.kp, b.vp, p, b.off_q, b.perm_q, b.o_sparse,
+                                 b.pairs_sparse, b.out, b.probes, b.pairs_exec, b.ws, None,
+                                 stream)
+        if ev: ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        call(qd, kd, vd)
+    torch.cuda.synchronize(dev)
+    st = S.sparsepr_read_stats(b.ws)
+    pairs_sparse = int(b.pairs_sparse.sum())
+    pairs_exec = int(b.pairs_exec.sum())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        call(qd, kd, vd, evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    stage_names = ["partition", "permute", "route", "block_sparse_attn", "probe_correct"]
+    stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+                for i, n in enumerate(stage_names)}
+    ms = total_ms / args.steps
+
+    # dense baseline of the same kernel design on the same inputs
+    dense_out = torch.empty((w.H, w.N, w.d), dtype=torch.float32, device=dev)
+    meta, dws = S.dense_attention(qd, kd, vd, dense_out)
+    torch.cuda.synchronize(dev)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dense_steps = max(2, min(args.steps, 5))
+    d0.record(stream)
+    for _ in range(dense_steps):
+        S.dense_attention(qd, kd, vd, dense_out, ws=dws, meta=meta)
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = d0.elapsed_time(d1) / dense_steps
+
+    # end to end through the public API from pinned host buffers
+    out_h = torch.empty((w.H, w.N, w.d), dtype=qd.dtype).pin_memory()
+    qx, kx, vx = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 3))
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        qx.copy_(qh, non_blocking=True)
+        kx.copy_(kh, non_blocking=True)
+        vx.copy_(vh, non_blocking=True)
+        call(qx, kx, vx)
+        out_h.copy_(b.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    # max over ranks
+    vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms], device=dev,
+                        dtype=torch.float64)
+    tot_pairs = torch.tensor([pairs_exec, pairs_sparse], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot_pairs, op=dist.ReduceOp.SUM)
+    ms_max, e2e_max, attn_max, dense_max = vals.tolist()
+    P_exec_all, P_sparse_all = tot_pairs.tolist()
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+        value = 4.0 * w.d * P_exec_all / (ms_max * 1e-3) / 1e12
+        attn_tflops = 4.0 * w.d * pairs_sparse / (stage_ms["block_sparse_attn"] * 1e-3) / 1e12
+        line = dict(
+            metric=METRIC, value=value, unit="TFLOPS", n_gpus=world, steps=args.steps,
+            warmup=args.warmup, ms_per_step=ms_max, higher_is_better=True, scaling="weak",
+            vs_baseline=None, dtype="bf16", data="synthetic",
+            config=dict(workload=workload_desc(w), heads_per_rank=w.H,
+                        l2="inputs (697 MB of Q/K/V per call) are larger than the 126 MB L2",
+                        parallelism="replicas: each rank runs its own call (dp%d)" % world),
+            attn_call_ms=ms_max,
+            stage_ms=stage_ms,
+            stage_share={n: stage_ms[n] / ms for n in stage_ms},
+            rho_exec=pairs_exec / (w.H * w.N * w.N),
+            rho_sparse=pairs_sparse / (w.H * w.N * w.N),
+            attn_kernel_tflops=attn_tflops,
+            dense_same_kernel_ms=dense_max,
+            dense_same_kernel_tflops=4.0 * w.d * w.H * w.N * w.N / (dense_max * 1e-3) / 1e12,
+            speedup_vs_dense=dense_max / ms_max,
+            attn_only_speedup_vs_dense=dense_max / attn_max,
+            kmeans_passes=dict(key=st["key_passes"], query=st["query_passes"]),
+            device_status=st["status"],
+            roofline=dict(bound="tensor", kernel="sparse_attn_kernel<128>",
+                          achieved=attn_tflops, peak=peak, unit="TFLOP/s",
+                          frac=attn_tflops / peak, peak_source="bf16_tflops (burst) of " + src,
+                          traffic=None,
+                          note="achieved = 4 d P_sparse / duration of the block-sparse "
+                               "attention call (CUDA events on its stream)"),
+            clocks=clocks,
+            e2e=dict(value=4.0 * w.d * P_exec_all / (e2e_max * 1e-3) / 1e12, unit="TFLOPS",
+                     ms=e2e_max, h2d_bytes_per_step=3 * qd.numel() * qd.element_size(),
+                     d2h_bytes_per_step=b.out.numel() * b.out.element_size()),
+            gpu_launches=gpu_launches_per_call(w) * args.steps,
+        )
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline_sample(w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,402 @@
+// C ABI of the SparsePR library: argument checks, workspace carving and the
+// per-stage launch sequences. Declarations and the contract of every entry
+// point are in include/sparsepr.h.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace spr;
+
+namespace {
+
+struct Ctx {
+  sparsepr_params p;
+  Layout L;
+  cudaStream_t st;
+  DeviceStats* stats;
+  double scale;
+  bool bf16;
+  int kind;
+};
+
+bool finite_nonneg(double x) { return isfinite(x) && x >= 0.0; }
+
+sparsepr_status check_params(const sparsepr_params* p) {
+  if (!p || !p->keep) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->H < 1 || p->H > SPARSEPR_MAX_HEADS) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->n_text < 0 || p->N < 16) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
+  if (p->n_text != 0) return SPARSEPR_ERR_UNSUPPORTED;
+  const long long Nv = static_cast<long long>(p->N) - p->n_text;
+  if (Nv < 1) return SPARSEPR_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->H) * p->N >= (1LL << 31)) return SPARSEPR_ERR_UNSUPPORTED;
+  if (p->Ck < 1 || p->Ck > Nv || p->Ck > kMaxGroups) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->Cq < 1 || p->Cq > Nv || p->Cq > kMaxGroups) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->Ms < 1 || p->Ms > Nv) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->n_eig < 1 || p->n_eig > p->d || p->n_eig > 32) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->kmeans_iters < 1 || p->kmeans_iters > 1000) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->M < 0 || p->M > Nv) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->r < 1 || p->r > p->d) return SPARSEPR_ERR_INVALID_ARG;
+  if (!finite_nonneg(p->lambda) || !finite_nonneg(p->scale)) return SPARSEPR_ERR_INVALID_ARG;
+  for (int h = 0; h < p->H; ++h)
+    if (!(p->keep[h] > 0.0 && p->keep[h] <= 1.0)) return SPARSEPR_ERR_INVALID_ARG;
+  return SPARSEPR_OK;
+}
+
+sparsepr_status setup(Ctx* c, const sparsepr_params* p, sparsepr_dtype dt, void* ws,
+                      size_t ws_bytes, void* stream) {
+  sparsepr_status s = check_params(p);
+  if (s != SPARSEPR_OK) return s;
+  if (dt != SPARSEPR_BF16 && dt != SPARSEPR_F32) return SPARSEPR_ERR_UNSUPPORTED;
+  c->p = *p;
+  compute_layout(c->p, &c->L);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) != 0 || ws_bytes < c->L.total)
+    return SPARSEPR_ERR_WORKSPACE;
+  c->st = static_cast<cudaStream_t>(stream);
+  c->stats = at<DeviceStats>(ws, c->L.stats);
+  c->scale = p->scale > 0.0 ? p->scale : 1.0 / sqrt(static_cast<double>(p->d));
+  c->bf16 = (dt == SPARSEPR_BF16);
+  c->kind = c->bf16 ? kXbf16 : kXf32;
+  return SPARSEPR_OK;
+}
+
+sparsepr_status cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? SPARSEPR_OK : SPARSEPR_ERR_CUDA;
+}
+
+#define SPR_TRY(expr)                                \
+  do {                                               \
+    cudaError_t _e = (expr);                         \
+    if (_e != cudaSuccess) return SPARSEPR_ERR_CUDA; \
+  } while (0)
+
+__global__ void set_i32_kernel(int32_t* p, int v) { *p = v; }
+
+// Dense-mode routing metadata per head: one query group [0, M), one key
+// group [0, N) kept by it.
+__global__ void dense_meta_kernel(int32_t* meta, int H, int M, int N) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  int32_t* offq = meta;
+  int32_t* offk = meta + 2 * H;
+  int32_t* csr = meta + 4 * H;
+  int32_t* kh = meta + 5 * H;
+  offq[2 * h] = 0;
+  offq[2 * h + 1] = M;
+  offk[2 * h] = 0;
+  offk[2 * h + 1] = N;
+  csr[h] = 0;
+  kh[h] = 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sparsepr_workspace_bytes(const sparsepr_params* p) {
+  if (check_params(p) != SPARSEPR_OK) return 0;
+  Layout L;
+  compute_layout(*p, &L);
+  return L.total;
+}
+
+const char* sparsepr_status_string(sparsepr_status s) {
+  switch (s) {
+    case SPARSEPR_OK: return "ok";
+    case SPARSEPR_ERR_INVALID_ARG: return "invalid argument";
+    case SPARSEPR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SPARSEPR_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case SPARSEPR_ERR_CUDA: return "CUDA error";
+    case SPARSEPR_ERR_TIMEOUT: return "device wait limit reached";
+    case SPARSEPR_ERR_NUMERIC: return "numerical error (empty kept set or non-finite value)";
+  }
+  return "unknown status";
+}
+
+int32_t sparsepr_route_width(const sparsepr_params* p) {
+  if (check_params(p) != SPARSEPR_OK) return -1;
+  Layout L;
+  compute_layout(*p, &L);
+  return L.kmax;
+}
+
+sparsepr_status sparsepr_reset_stats(void* ws, void* stream) {
+  if (!ws) return SPARSEPR_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(DeviceStats), static_cast<cudaStream_t>(stream)));
+}
+
+sparsepr_status sparsepr_read_stats(const void* ws, sparsepr_stats* out) {
+  if (!ws || !out) return SPARSEPR_ERR_INVALID_ARG;
+  return cuda_status(cudaMemcpy(out, ws, sizeof(DeviceStats), cudaMemcpyDeviceToHost));
+}
+
+sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype dt,
+                                   const sparsepr_params* p, int32_t* label_q, int32_t* label_k,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!q || !k || !label_q || !label_k) return SPARSEPR_ERR_INVALID_ARG;
+  const Layout& L = c.L;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, Nv = L.Nv, e = c.p.n_eig, Ck = c.p.Ck, Cq = c.p.Cq;
+  const int iters = c.p.kmeans_iters;
+  cudaStream_t st = c.st;
+  int32_t* flags = at<int32_t>(ws, L.flags);
+  SPR_TRY(cudaMemsetAsync(ws, 0, sizeof(DeviceStats), st));
+  SPR_TRY(cudaMemsetAsync(flags, 0, static_cast<size_t>(H) * 16, st));
+  set_i32_kernel<<<1, 1, 0, st>>>(&c.stats->H, H);
+  int32_t* init_k = at<int32_t>(ws, L.init_k);
+  int32_t* init_q = at<int32_t>(ws, L.init_q);
+  double* mk = at<double>(ws, L.mk);
+  double* evl = at<double>(ws, L.eval);
+  double* evc = at<double>(ws, L.evec);
+  double* wk = at<double>(ws, L.wk);
+  double* z = at<double>(ws, L.z);
+  double* mu = at<double>(ws, L.mu);
+  double* mun = at<double>(ws, L.munorm);
+  int32_t* lab_k = at<int32_t>(ws, L.lab_k);
+  int32_t* lab_q = at<int32_t>(ws, L.lab_q);
+  int32_t* hist = at<int32_t>(ws, L.hist);
+  int32_t* sperm = at<int32_t>(ws, L.sortperm);
+  int32_t* soff = at<int32_t>(ws, L.sortoff);
+  double* ck = at<double>(ws, L.ck);
+  double* G = at<double>(ws, L.g);
+  double* qbar = at<double>(ws, L.qbar);
+  double* wg = at<double>(ws, L.wg);
+  double* cg = at<double>(ws, L.cg);
+  const long long hs_in = static_cast<long long>(N) * d;
+
+  // keys: metric, eigenbasis, response coordinates, Lloyd passes
+  SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, st));
+  SPR_TRY(launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st));
+  SPR_TRY(launch_jacobi(mk, H, d, evl, evc, c.stats, st));
+  SPR_TRY(launch_top_eig_projector(evl, evc, H, d, e, wk, st));
+  SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
+  const long long hs_z = static_cast<long long>(Nv) * e;
+  SPR_TRY(launch_gather_init(z, kXf64, hs_z, e, e, init_k, Ck, H, mu, mun, st));
+  for (int t = 0; t < iters; ++t) {
+    SPR_TRY(launch_argmin(z, kXf64, hs_z, e, Nv, e, mu, mun, Ck, H, lab_k, flags, 0, st));
+    SPR_TRY(launch_finalize_pass(H, t, flags, 0, c.stats->key_passes, st));
+    if (t + 1 < iters) {
+      SPR_TRY(launch_counting_sort(lab_k, H, Nv, Ck, L.nchunk, hist, sperm, soff, flags + 1, 4,
+                                   nullptr, st));
+      SPR_TRY(launch_group_mean(z, kXf64, hs_z, e, e, sperm, Nv, soff, Ck + 1, Ck, H, true, mu,
+                                mun, flags + 1, 4, st));
+    }
+  }
+  // K/V group centroids in the original space, query metric G = s^2 C_K^T C_K
+  SPR_TRY(launch_counting_sort(lab_k, H, Nv, Ck, L.nchunk, hist, sperm, soff, nullptr, 0, nullptr,
+                               st));
+  SPR_TRY(launch_group_mean(k, c.kind, hs_in, d, d, sperm, Nv, soff, Ck + 1, Ck, H, false, ck,
+                            nullptr, nullptr, 0, st));
+  SPR_TRY(launch_gram_f64(ck, ck, nullptr, nullptr, static_cast<long long>(Ck) * d,
+                          static_cast<long long>(Ck) * d, d, Ck, H, d, c.scale * c.scale, 0.0, G,
+                          static_cast<long long>(d) * d, 0, st));
+  // queries: Lloyd passes on logit profiles in the d-space form
+  SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
+  for (int t = 0; t < iters; ++t) {
+    SPR_TRY(launch_query_metric_apply(G, qbar, Cq, H, d, wg, cg, flags + 3, 4, st));
+    SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, st));
+    SPR_TRY(launch_finalize_pass(H, t, flags, 2, c.stats->query_passes, st));
+    if (t + 1 < iters) {
+      SPR_TRY(launch_counting_sort(lab_q, H, Nv, Cq, L.nchunk, hist, sperm, soff, flags + 3, 4,
+                                   nullptr, st));
+      SPR_TRY(launch_group_mean(q, c.kind, hs_in, d, d, sperm, Nv, soff, Cq + 1, Cq, H, true,
+                                qbar, nullptr, flags + 3, 4, st));
+    }
+  }
+  SPR_TRY(launch_write_labels(lab_q, H, N, Nv, Cq, label_q, st));
+  SPR_TRY(launch_write_labels(lab_k, H, N, Nv, Ck, label_k, st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v, sparsepr_dtype dt,
+                                 const sparsepr_params* p, const int32_t* label_q,
+                                 const int32_t* label_k, int32_t* perm_q, int32_t* perm_k,
+                                 int32_t* off_q, int32_t* off_k, void* qp, void* kp, void* vp,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!q || !k || !v || !label_q || !label_k || !perm_q || !perm_k || !off_q || !off_k || !qp ||
+      !kp || !vp)
+    return SPARSEPR_ERR_INVALID_ARG;
+  if (qp == q || kp == k || vp == v) return SPARSEPR_ERR_INVALID_ARG;
+  const int H = c.p.H, N = c.p.N, d = c.p.d;
+  const int nchunk = (N + kSortChunk - 1) / kSortChunk;
+  if (static_cast<size_t>(H) * nchunk * c.L.Cmax > static_cast<size_t>(H) * c.L.nchunk * c.L.Cmax)
+    return SPARSEPR_ERR_UNSUPPORTED;  // only while n_text == 0 (N == Nv)
+  int32_t* hist = at<int32_t>(ws, c.L.hist);
+  SPR_TRY(launch_counting_sort(label_q, H, N, c.p.Cq, nchunk, hist, perm_q, off_q, nullptr, 0,
+                               c.stats, c.st));
+  SPR_TRY(launch_counting_sort(label_k, H, N, c.p.Ck, nchunk, hist, perm_k, off_k, nullptr, 0,
+                               c.stats, c.st));
+  const int eb = c.bf16 ? 2 : 4;
+  SPR_TRY(launch_gather_rows(q, qp, perm_q, H, N, d, eb, c.st));
+  SPR_TRY(launch_gather_rows(k, kp, perm_k, H, N, d, eb, c.st));
+  SPR_TRY(launch_gather_rows(v, vp, perm_k, H, N, d, eb, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt,
+                               const sparsepr_params* p, const int32_t* off_q,
+                               const int32_t* off_k, int32_t* csr, int32_t* k_per_head, void* ws,
+                               size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!qp || !kp || !off_q || !off_k || !csr || !k_per_head) return SPARSEPR_ERR_INVALID_ARG;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, Ck = c.p.Ck, Cq = c.p.Cq;
+  double* cq = at<double>(ws, c.L.cq);
+  double* ckr = at<double>(ws, c.L.ckr);
+  SPR_TRY(launch_range_mean(qp, c.kind, H, N, d, off_q, Cq, cq, c.st));
+  SPR_TRY(launch_range_mean(kp, c.kind, H, N, d, off_k, Ck, ckr, c.st));
+  int32_t kh[SPARSEPR_MAX_HEADS];
+  for (int h = 0; h < H; ++h) kh[h] = keep_budget(c.p.keep[h], Ck);
+  SPR_TRY(launch_write_k(kh, H, k_per_head, c.st));
+  SPR_TRY(launch_route(cq, ckr, H, Cq, Ck, d, c.scale, k_per_head, c.L.kmax, csr, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const void* vp,
+                                           sparsepr_dtype dt, const sparsepr_params* p,
+                                           const int32_t* off_q, const int32_t* off_k,
+                                           const int32_t* csr, const int32_t* k_per_head,
+                                           float* o_sparse, int64_t* pairs_sparse, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!qp || !kp || !vp || !off_q || !off_k || !csr || !k_per_head || !o_sparse || !pairs_sparse)
+    return SPARSEPR_ERR_INVALID_ARG;
+  const int H = c.p.H, N = c.p.N, d = c.p.d;
+  const size_t n = static_cast<size_t>(H) * N * d;
+  const void *q16 = qp, *k16 = kp, *v16 = vp;
+  if (!c.bf16) {
+    __nv_bfloat16* b = at<__nv_bfloat16>(ws, c.L.bf16_qkv);
+    SPR_TRY(launch_cast_bf16(static_cast<const float*>(qp), b, n, c.st));
+    SPR_TRY(launch_cast_bf16(static_cast<const float*>(kp), b + n, n, c.st));
+    SPR_TRY(launch_cast_bf16(static_cast<const float*>(vp), b + 2 * n, n, c.st));
+    q16 = b;
+    k16 = b + n;
+    v16 = b + 2 * n;
+  }
+  AttnArgs a;
+  a.qp = q16;
+  a.kp = k16;
+  a.vp = v16;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.q_rows = N;
+  a.Cq = c.p.Cq;
+  a.Ck = c.p.Ck;
+  a.off_q = off_q;
+  a.off_k = off_k;
+  a.csr = csr;
+  a.kh = k_per_head;
+  a.kmax = c.L.kmax;
+  a.scale = static_cast<float>(c.scale);
+  a.out = o_sparse;
+  a.work = at<int32_t>(ws, c.L.work);
+  a.nwork = at<int32_t>(ws, c.L.nwork);
+  a.tiles_per_head = c.L.tiles_per_head;
+  a.nslots = at<int32_t>(ws, c.L.nslots);
+  a.pairs = pairs_sparse;
+  a.stats = c.stats;
+  SPR_TRY(launch_block_sparse_attn(a, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const void* vp,
+                                       sparsepr_dtype dt, const sparsepr_params* p,
+                                       const int32_t* off_q, const int32_t* perm_q,
+                                       const float* o_sparse, const int64_t* pairs_sparse,
+                                       void* out, int32_t* probes, int64_t* pairs_exec,
+                                       double* fit, void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!qp || !kp || !vp || !off_q || !perm_q || !o_sparse || !pairs_sparse || !out ||
+      !pairs_exec || (c.p.M > 0 && !probes))
+    return SPARSEPR_ERR_INVALID_ARG;
+  const Layout& L = c.L;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, M = c.p.M, Cq = c.p.Cq;
+  cudaStream_t st = c.st;
+  float* bp32 = at<float>(ws, L.bp32);
+  float* bv32 = at<float>(ws, L.bv32);
+  float* od = at<float>(ws, L.od);
+  if (M > 0) {
+    SPR_TRY(launch_probe_select(off_q, H, Cq, M, probes, st));
+    __nv_bfloat16* pq = at<__nv_bfloat16>(ws, L.probe_q);
+    SPR_TRY(launch_gather_probe_rows(qp, c.bf16, probes, H, N, M, d, pq, st));
+    const void *k16 = kp, *v16 = vp;
+    if (!c.bf16) {
+      const size_t n = static_cast<size_t>(H) * N * d;
+      __nv_bfloat16* b = at<__nv_bfloat16>(ws, L.bf16_qkv);
+      SPR_TRY(launch_cast_bf16(static_cast<const float*>(kp), b + n, n, st));
+      SPR_TRY(launch_cast_bf16(static_cast<const float*>(vp), b + 2 * n, n, st));
+      k16 = b + n;
+      v16 = b + 2 * n;
+    }
+    int32_t* meta = at<int32_t>(ws, L.pmeta);
+    dense_meta_kernel<<<(H + 127) / 128, 128, 0, st>>>(meta, H, M, N);
+    SPR_TRY(cudaGetLastError());
+    AttnArgs a;
+    a.qp = pq;
+    a.kp = k16;
+    a.vp = v16;
+    a.H = H;
+    a.N = N;
+    a.d = d;
+    a.q_rows = M;
+    a.Cq = 1;
+    a.Ck = 1;
+    a.off_q = meta;
+    a.off_k = meta + 2 * H;
+    a.csr = meta + 4 * H;
+    a.kh = meta + 5 * H;
+    a.kmax = 1;
+    a.scale = static_cast<float>(c.scale);
+    a.out = od;
+    a.work = at<int32_t>(ws, L.pwork);
+    a.nwork = at<int32_t>(ws, L.pnwork);
+    a.tiles_per_head = M / kTileM + 2;
+    a.nslots = meta + 6 * H;
+    a.pairs = nullptr;
+    a.stats = c.stats;
+    SPR_TRY(launch_block_sparse_attn(a, st));
+    double* xr = at<double>(ws, L.xr);
+    double* means = at<double>(ws, L.means);
+    double* gram = at<double>(ws, L.gram);
+    const long long hs = 2LL * M * d;
+    SPR_TRY(launch_probe_residuals(o_sparse, od, probes, H, N, M, d, xr, means, st));
+    SPR_TRY(launch_gram_f64(xr, xr, means, means, hs, hs, d, M, H, d, 1.0, c.p.lambda, gram,
+                            2LL * d * d, 2LL * d, st));
+    SPR_TRY(launch_gram_f64(xr, xr + static_cast<size_t>(M) * d, means, means + d, hs, hs, d, M, H,
+                            d, 1.0, 0.0, gram + static_cast<size_t>(d) * d, 2LL * d * d, 2LL * d,
+                            st));
+    double* bmat = at<double>(ws, L.bmat);
+    double* bvec = at<double>(ws, L.bvec);
+    SPR_TRY(launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, st));
+    double* rtr = at<double>(ws, L.mk);
+    SPR_TRY(launch_gram_f64(xr + static_cast<size_t>(M) * d, xr + static_cast<size_t>(M) * d,
+                            nullptr, nullptr, hs, hs, d, M, H, d, 1.0, 0.0, rtr,
+                            static_cast<long long>(d) * d, 0, st));
+    double* evl = at<double>(ws, L.eval);
+    double* evc = at<double>(ws, L.evec);
+    SPR_TRY(launch_jacobi(rtr, H, d, evl, evc, c.stats, st));
+    SPR_TRY(launch_project_map(bmat, bvec, evl, evc, H, d, c.p.r, bp32, bv32, fit, st));
+  } else {
+    SPR_TRY(cudaMemsetAsync(bp32, 0, static_cast<size_t>(H) * d * d * 4, st));
+    SPR_TRY(cudaMemsetAsync(bv32, 0, static_cast<size_t>(H) * d * 4, st));
+    if (fit) SPR_TRY(cudaMemsetAsync(fit, 0, static_cast<size_t>(H) * (d * d + d) * 8, st));
+  }
+  SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, M, d, out, c.bf16, st));
+  SPR_TRY(launch_pairs_exec(pairs_sparse, H, static_cast<int64_t>(M) * N, pairs_exec, c.stats, st));
+  return SPARSEPR_OK;
+}
+
+}  // extern "C"

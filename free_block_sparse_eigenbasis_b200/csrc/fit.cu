@@ -1,0 +1,358 @@
+// Stage 4 of "Partition the Support, Reconstruct the Residual" (2.B,
+// probe-fitted residual reconstruction): stratified probe rows, their exact
+// dense outputs (computed by the attention kernel in dense mode), the ridge
+// fit of R ~ b + x B in fp64, its restriction to the leading residual
+// subspace, and the fused correction + unpermute of every unprobed row.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+namespace {
+
+// Probes per query group by largest remainder (ties to the lower group),
+// rows at offsets floor((t + 1/2) n_g / m_g) inside each group.
+__global__ void probe_select_kernel(const int32_t* off_q, int Cq, int M, int32_t* probes) {
+  extern __shared__ int64_t psm[];
+  int64_t* rem = psm;                                  // [Cq]
+  int32_t* m = reinterpret_cast<int32_t*>(rem + Cq);   // [Cq]
+  int32_t* start = m + Cq;                             // [Cq]
+  __shared__ int32_t left;
+  const int h = blockIdx.x;
+  const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
+  const int64_t Nt = oq[Cq] - oq[0];
+  for (int g = threadIdx.x; g < Cq; g += blockDim.x) {
+    const int64_t n = oq[g + 1] - oq[g];
+    const int64_t num = static_cast<int64_t>(M) * n;
+    m[g] = static_cast<int32_t>(Nt > 0 ? num / Nt : 0);
+    rem[g] = Nt > 0 ? num % Nt : 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t s = 0;
+    for (int g = 0; g < Cq; ++g) s += m[g];
+    left = static_cast<int32_t>(M - s);
+  }
+  __syncthreads();
+  // rank of each remainder (larger first, lower group on ties)
+  for (int g = threadIdx.x; g < Cq; g += blockDim.x) {
+    const int64_t rg = rem[g];
+    int rank = 0;
+    for (int o = 0; o < Cq; ++o) rank += (rem[o] > rg) || (rem[o] == rg && o < g);
+    start[g] = rank;  // temporary
+  }
+  __syncthreads();
+  for (int g = threadIdx.x; g < Cq; g += blockDim.x)
+    if (start[g] < left) m[g] += 1;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t s = 0;
+    for (int g = 0; g < Cq; ++g) {
+      start[g] = s;
+      s += m[g];
+    }
+  }
+  __syncthreads();
+  int32_t* out = probes + static_cast<size_t>(h) * M;
+  for (int g = threadIdx.x; g < Cq; g += blockDim.x) {
+    const int64_t n = oq[g + 1] - oq[g];
+    const int mg = m[g];
+    for (int t = 0; t < mg; ++t)
+      out[start[g] + t] = oq[g] + static_cast<int32_t>(((2LL * t + 1) * n) / (2LL * mg));
+  }
+}
+
+// dst[h, t, :] = bf16(qp[h, probes[h, t], :]); rows M..M+127 of each head's
+// slot region are zero.
+__global__ void gather_probe_rows_kernel(const void* qp, int bf16, const int32_t* probes, int N,
+                                         int M, int d, __nv_bfloat16* dst) {
+  const int h = blockIdx.y;
+  const int t = blockIdx.x;
+  __nv_bfloat16* o = dst + (static_cast<size_t>(h) * M + t) * d;
+  if (t >= M) return;
+  const size_t src_row = static_cast<size_t>(h) * N + probes[static_cast<size_t>(h) * M + t];
+  for (int a = threadIdx.x; a < d; a += blockDim.x) {
+    if (bf16)
+      o[a] = static_cast<const __nv_bfloat16*>(qp)[src_row * d + a];
+    else
+      o[a] = __float2bfloat16_rn(static_cast<const float*>(qp)[src_row * d + a]);
+  }
+}
+
+// X = O_sparse[probes], R = O_dense - X (fp64), column means xbar, rbar.
+__global__ void probe_residuals_kernel(const float* o_sparse, const float* od,
+                                       const int32_t* probes, int N, int M, int d, double* xr,
+                                       double* means) {
+  const int h = blockIdx.x, a = threadIdx.x;
+  if (a >= d) return;
+  double* X = xr + static_cast<size_t>(h) * 2 * M * d;
+  double* R = X + static_cast<size_t>(M) * d;
+  double sx = 0.0, sr = 0.0;
+  for (int t = 0; t < M; ++t) {
+    const size_t row = static_cast<size_t>(h) * N + probes[static_cast<size_t>(h) * M + t];
+    const double x = o_sparse[row * d + a];
+    const double r = static_cast<double>(od[(static_cast<size_t>(h) * M + t) * d + a]) - x;
+    X[static_cast<size_t>(t) * d + a] = x;
+    R[static_cast<size_t>(t) * d + a] = r;
+    sx += x;
+    sr += r;
+  }
+  means[(static_cast<size_t>(h) * 2 + 0) * d + a] = M > 0 ? sx / M : 0.0;
+  means[(static_cast<size_t>(h) * 2 + 1) * d + a] = M > 0 ? sr / M : 0.0;
+}
+
+// Ridge solve per head: L L^T = A (Cholesky, packed lower L in shared
+// memory), B = A^{-1} C with one right-hand-side column per thread, then
+// b = rbar - xbar B.
+__global__ void ridge_solve_kernel(const double* gram, int d, double* bmat, double* bvec,
+                                   const double* means, DeviceStats* stats) {
+  extern __shared__ double rsm[];
+  const int ntri = d * (d + 1) / 2;
+  double* Lp = rsm;          // packed lower triangle, L[i][k] at i*(i+1)/2 + k
+  double* Cm = rsm + ntri;   // [d][d] right-hand sides (row-major), solved in place
+  __shared__ int bad;
+  const int h = blockIdx.x;
+  const double* A = gram + static_cast<size_t>(h) * 2 * d * d;
+  const double* C = A + static_cast<size_t>(d) * d;
+  for (int t = threadIdx.x; t < d * d; t += blockDim.x) {
+    const int i = t / d, k = t % d;
+    if (k <= i) Lp[i * (i + 1) / 2 + k] = A[t];
+    Cm[t] = C[t];
+  }
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int j = 0; j < d; ++j) {
+    if (threadIdx.x == 0) {
+      double s = Lp[j * (j + 1) / 2 + j];
+      for (int k = 0; k < j; ++k) {
+        const double l = Lp[j * (j + 1) / 2 + k];
+        s -= l * l;
+      }
+      if (!(s > 0.0)) {
+        bad = 1;
+        s = 1.0;
+      }
+      Lp[j * (j + 1) / 2 + j] = sqrt(s);
+    }
+    __syncthreads();
+    const double ljj = Lp[j * (j + 1) / 2 + j];
+    for (int i = j + 1 + threadIdx.x; i < d; i += blockDim.x) {
+      double s = Lp[i * (i + 1) / 2 + j];
+      for (int k = 0; k < j; ++k) s -= Lp[i * (i + 1) / 2 + k] * Lp[j * (j + 1) / 2 + k];
+      Lp[i * (i + 1) / 2 + j] = s / ljj;
+    }
+    __syncthreads();
+  }
+  const int col = threadIdx.x;
+  if (col < d) {
+    // forward: L Y = C
+    for (int i = 0; i < d; ++i) {
+      double s = Cm[i * d + col];
+      for (int k = 0; k < i; ++k) s -= Lp[i * (i + 1) / 2 + k] * Cm[k * d + col];
+      Cm[i * d + col] = s / Lp[i * (i + 1) / 2 + i];
+    }
+    // backward: L^T B = Y
+    for (int i = d - 1; i >= 0; --i) {
+      double s = Cm[i * d + col];
+      for (int k = i + 1; k < d; ++k) s -= Lp[k * (k + 1) / 2 + i] * Cm[k * d + col];
+      Cm[i * d + col] = s / Lp[i * (i + 1) / 2 + i];
+    }
+  }
+  __syncthreads();
+  if (bad) {
+    for (int t = threadIdx.x; t < d * d; t += blockDim.x) Cm[t] = 0.0;
+    if (threadIdx.x == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
+    __syncthreads();
+  }
+  double* Bo = bmat + static_cast<size_t>(h) * d * d;
+  for (int t = threadIdx.x; t < d * d; t += blockDim.x) Bo[t] = Cm[t];
+  if (col < d) {
+    const double* xbar = means + static_cast<size_t>(h) * 2 * d;
+    const double* rbar = xbar + d;
+    double s = rbar[col];
+    for (int a = 0; a < d; ++a) s -= xbar[a] * Cm[a * d + col];
+    bvec[static_cast<size_t>(h) * d + col] = bad ? 0.0 : s;
+  }
+}
+
+// P_r = sum over the r largest eigenpairs of R^T R of v v^T; B' = B P_r,
+// b' = b P_r (fp64), stored fp32 for the correction (and fp64 if asked).
+__global__ void project_map_kernel(const double* bmat, const double* bvec, const double* eval,
+                                   const double* evec, int d, int r, float* bp32, float* bv32,
+                                   double* fit_out) {
+  extern __shared__ double psm2[];
+  double* Pr = psm2;  // [d][d]
+  __shared__ int sel[128];
+  const int h = blockIdx.x;
+  const double* ev = eval + static_cast<size_t>(h) * d;
+  const double* V = evec + static_cast<size_t>(h) * d * d;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    const double lj = ev[j];
+    int rank = 0;
+    for (int i = 0; i < d; ++i) rank += (ev[i] > lj) || (ev[i] == lj && i < j);
+    sel[j] = rank < r;
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < d * d; t += blockDim.x) {
+    const int a = t / d, b = t % d;
+    double s = 0.0;
+    for (int j = 0; j < d; ++j)
+      if (sel[j]) s += V[static_cast<size_t>(a) * d + j] * V[static_cast<size_t>(b) * d + j];
+    Pr[t] = s;
+  }
+  __syncthreads();
+  const double* B = bmat + static_cast<size_t>(h) * d * d;
+  const int col = threadIdx.x;
+  if (col < d) {
+    for (int a = 0; a < d; ++a) {
+      double s = 0.0;
+      for (int k = 0; k < d; ++k) s += B[static_cast<size_t>(a) * d + k] * Pr[k * d + col];
+      bp32[(static_cast<size_t>(h) * d + a) * d + col] = static_cast<float>(s);
+      if (fit_out) fit_out[static_cast<size_t>(h) * (d * d + d) + a * d + col] = s;
+    }
+    const double* b = bvec + static_cast<size_t>(h) * d;
+    double s = 0.0;
+    for (int k = 0; k < d; ++k) s += b[k] * Pr[k * d + col];
+    bv32[static_cast<size_t>(h) * d + col] = static_cast<float>(s);
+    if (fit_out) fit_out[static_cast<size_t>(h) * (d * d + d) + d * d + col] = s;
+  }
+}
+
+// out[perm_q[i]] = O_dense(probe) for probe rows, else x + b' + x B'
+// (x = o_sparse row, fp32); 32 group-major rows per CTA, B' in shared memory.
+constexpr int kCorrRows = 32;
+
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256) correct_kernel(const float* o_sparse, const float* od,
+                                                      const int32_t* probes,
+                                                      const int32_t* perm_q, const float* bp32,
+                                                      const float* bv32, int N, int M, int d,
+                                                      void* out) {
+  extern __shared__ float csm[];
+  float* Bs = csm;                 // [d][d]
+  float* xs = Bs + d * d;          // [kCorrRows][d]
+  __shared__ int prow[kCorrRows];  // probe index or -1
+  const int h = blockIdx.y;
+  const int i0 = blockIdx.x * kCorrRows;
+  const float* Bh = bp32 + static_cast<size_t>(h) * d * d;
+  for (int t = threadIdx.x; t < d * d; t += blockDim.x) Bs[t] = Bh[t];
+  for (int t = threadIdx.x; t < kCorrRows * d; t += blockDim.x) {
+    const int r = t / d, a = t % d;
+    const int i = i0 + r;
+    xs[t] = (i < N) ? o_sparse[(static_cast<size_t>(h) * N + i) * d + a] : 0.f;
+  }
+  if (threadIdx.x < kCorrRows) {
+    const int i = i0 + threadIdx.x;
+    const int32_t* pr = probes + static_cast<size_t>(h) * M;
+    int lo = 0, hi = M;  // first probe >= i
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (pr[mid] < i) lo = mid + 1; else hi = mid;
+    }
+    prow[threadIdx.x] = (lo < M && pr[lo] == i) ? lo : -1;
+  }
+  __syncthreads();
+  const float* bv = bv32 + static_cast<size_t>(h) * d;
+  for (int t = threadIdx.x; t < kCorrRows * d; t += blockDim.x) {
+    const int r = t / d, col = t % d;
+    const int i = i0 + r;
+    if (i >= N) continue;
+    float y;
+    if (prow[r] >= 0) {
+      y = od[(static_cast<size_t>(h) * M + prow[r]) * d + col];
+    } else {
+      const float* xr = xs + r * d;
+      float acc = 0.f;
+      for (int a = 0; a < d; ++a) acc = fmaf(xr[a], Bs[a * d + col], acc);
+      y = xr[col] + bv[col] + acc;
+    }
+    const size_t dst = (static_cast<size_t>(h) * N + perm_q[static_cast<size_t>(h) * N + i]) * d + col;
+    if (OUT_BF16)
+      static_cast<__nv_bfloat16*>(out)[dst] = __float2bfloat16_rn(y);
+    else
+      static_cast<float*>(out)[dst] = y;
+  }
+}
+
+__global__ void pairs_exec_kernel(const int64_t* ps, int H, int64_t add, int64_t* pe,
+                                  DeviceStats* stats) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  const int64_t v = ps[h] + add;
+  pe[h] = v;
+  stats->pairs_exec[h] = v;
+}
+
+}  // namespace
+
+cudaError_t launch_probe_select(const int32_t* off_q, int H, int Cq, int M, int32_t* probes,
+                                cudaStream_t st) {
+  const size_t shb = static_cast<size_t>(Cq) * 16;
+  probe_select_kernel<<<H, 256, shb, st>>>(off_q, Cq, M, probes);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* probes, int H,
+                                     int N, int M, int d, __nv_bfloat16* dst, cudaStream_t st) {
+  gather_probe_rows_kernel<<<dim3(M, H), 128, 0, st>>>(qp, bf16 ? 1 : 0, probes, N, M, d, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const int32_t* probes,
+                                   int H, int N, int M, int d, double* xr, double* means,
+                                   cudaStream_t st) {
+  probe_residuals_kernel<<<H, 128, 0, st>>>(o_sparse, od, probes, N, M, d, xr, means);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
+                               const double* means, DeviceStats* stats, cudaStream_t st) {
+  const size_t shb = (static_cast<size_t>(d) * (d + 1) / 2 + static_cast<size_t>(d) * d) * 8;
+  cudaError_t e = cudaFuncSetAttribute(ridge_solve_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(shb));
+  if (e != cudaSuccess) return e;
+  ridge_solve_kernel<<<H, 128, shb, st>>>(gram, d, bmat, bvec, means, stats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* eval,
+                               const double* evec, int H, int d, int r, float* bp32, float* bv32,
+                               double* fit_out, cudaStream_t st) {
+  const size_t shb = static_cast<size_t>(d) * d * 8;
+  cudaError_t e = cudaFuncSetAttribute(project_map_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(shb));
+  if (e != cudaSuccess) return e;
+  project_map_kernel<<<H, 128, shb, st>>>(bmat, bvec, eval, evec, d, r, bp32, bv32, fit_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t* probes,
+                           const int32_t* perm_q, const float* bp32, const float* bv32, int H,
+                           int N, int M, int d, void* out, bool out_bf16, cudaStream_t st) {
+  const size_t shb = (static_cast<size_t>(d) * d + static_cast<size_t>(kCorrRows) * d) * 4;
+  dim3 grid((N + kCorrRows - 1) / kCorrRows, H);
+  cudaError_t e;
+  if (out_bf16) {
+    e = cudaFuncSetAttribute(correct_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(shb));
+    if (e != cudaSuccess) return e;
+    correct_kernel<true><<<grid, 256, shb, st>>>(o_sparse, od, probes, perm_q, bp32, bv32, N, M,
+                                                 d, out);
+  } else {
+    e = cudaFuncSetAttribute(correct_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(shb));
+    if (e != cudaSuccess) return e;
+    correct_kernel<false><<<grid, 256, shb, st>>>(o_sparse, od, probes, perm_q, bp32, bv32, N, M,
+                                                  d, out);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pairs_exec(const int64_t* pairs_sparse, int H, int64_t add, int64_t* pairs_exec,
+                              DeviceStats* stats, cudaStream_t st) {
+  pairs_exec_kernel<<<(H + 127) / 128, 128, 0, st>>>(pairs_sparse, H, add, pairs_exec, stats);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -1,0 +1,132 @@
+// Host-side launchers of the SparsePR kernels (one translation unit per
+// stage); called by the C-ABI layer in api.cu. Every launcher enqueues on
+// `st` and returns cudaGetLastError().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.h"
+
+namespace spr {
+
+// ---- sort.cu: stable counting sort of per-head labels ----------------------
+// labels [H, n] in 0..C-1 -> perm [H, n] (group-major order, ascending token
+// index inside a group) and off [H, C+1]. Heads with skip[h] != 0 are left
+// untouched (skip may be null).
+cudaError_t launch_counting_sort(const int32_t* labels, int H, int n, int C, int nchunk,
+                                 int32_t* hist, int32_t* perm, int32_t* off,
+                                 const int32_t* skip, int skip_stride, DeviceStats* stats,
+                                 cudaStream_t st);
+
+// ---- partition.cu ----------------------------------------------------------
+cudaError_t launch_fy_init(int H, int Nv, int Ck, int Cq, uint64_t seed, int32_t* init_k,
+                           int32_t* init_q, cudaStream_t st);
+// out[h] = factor * sum_s x_s x_s^T over the Ms strided sampled query rows.
+cudaError_t launch_metric_mk(const void* q, bool bf16, int H, int N, int Nv, int d, int Ms,
+                             double* out, cudaStream_t st);
+// out[h] = factor * sum_s (x_s - xm)(y_s - ym)^T + diag * I over S fp64 rows;
+// xm / ym (may be null) advance by mean_stride per head.
+cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
+                            const double* ym, long long head_stride_x, long long head_stride_y,
+                            int ld, int S, int H, int d, double factor, double diag,
+                            double* out, long long out_stride, long long mean_stride,
+                            cudaStream_t st);
+cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
+                         const double* wk, double* z, cudaStream_t st);
+// dst[h, c, :] = src[h, idx[h, c], :] (as fp64) and norms[h, c] = |dst|^2 (norms may be null)
+cudaError_t launch_gather_init(const void* src, int src_kind, long long head_stride, int ld,
+                               int D, const int32_t* idx, int C, int H, double* dst,
+                               double* norms, cudaStream_t st);
+// labels[h, i] = argmin_j (c[h, j] - 2 x_i . y[h, j]) (lowest j on ties);
+// changes[h] += number of labels that differ from the previous value.
+cudaError_t launch_argmin(const void* X, int x_kind, long long head_stride_x, int ldx, int n,
+                          int D, const double* Y, const double* c, int m, int H,
+                          int32_t* labels, int32_t* flags, int flag_base, cudaStream_t st);
+cudaError_t launch_finalize_pass(int H, int pass, int32_t* flags, int flag_base,
+                                 int32_t* passes_out, cudaStream_t st);
+// out[h, c, :] = mean of the rows perm[off[c]..off[c+1]) of X (fp64 sums in
+// ascending position order); empty group: keep (keep_prev) or zero.
+// norms[h, c] = |out[h, c]|^2 if norms is non-null.
+cudaError_t launch_group_mean(const void* X, int x_kind, long long head_stride_x, int ldx, int D,
+                              const int32_t* perm, int perm_stride, const int32_t* off,
+                              int off_stride, int C, int H, bool keep_prev, double* out,
+                              double* norms, const int32_t* skip, int skip_stride,
+                              cudaStream_t st);
+cudaError_t launch_query_metric_apply(const double* G, const double* qbar, int Cq, int H, int d,
+                                      double* wg, double* cg, const int32_t* skip,
+                                      int skip_stride, cudaStream_t st);
+cudaError_t launch_write_labels(const int32_t* lab, int H, int N, int Nv, int C_text,
+                                int32_t* out, cudaStream_t st);
+
+// x_kind values
+constexpr int kXf64 = 0;
+constexpr int kXbf16 = 1;
+constexpr int kXf32 = 2;
+
+// ---- linalg.cu -------------------------------------------------------------
+// Cyclic-parallel Jacobi eigensolver, one CTA per head: A [H, d, d] fp64
+// symmetric -> eval [H, d], evec [H, d, d] (eigenvectors in columns).
+cudaError_t launch_jacobi(const double* A, int H, int d, double* eval, double* evec,
+                          DeviceStats* stats, cudaStream_t st);
+// wk[h, a, t] = evec[h, a, j_t] * sqrt(max(eval_j_t, 0)) for the e largest
+// eigenvalues (t = rank, ties to the lower index).
+cudaError_t launch_top_eig_projector(const double* eval, const double* evec, int H, int d, int e,
+                                     double* wk, cudaStream_t st);
+
+// ---- permute.cu ------------------------------------------------------------
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, int H, int N,
+                               int d, int elem_bytes, cudaStream_t st);
+cudaError_t launch_route(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
+                         double scale, const int32_t* kh, int kmax, int32_t* csr,
+                         cudaStream_t st);
+cudaError_t launch_range_mean(const void* X, int x_kind, int H, int N, int d, const int32_t* off,
+                              int C, double* out, cudaStream_t st);
+cudaError_t launch_write_k(const int32_t* kh_host_vals, int H, int32_t* k_per_head,
+                           cudaStream_t st);
+
+// ---- attn.cu ---------------------------------------------------------------
+struct AttnArgs {
+  const void* qp;   // bf16 [H*Nq_total rows, d] (row = h * q_rows + i)
+  const void* kp;   // bf16 [H*N, d]
+  const void* vp;   // bf16 [H*N, d]
+  int H, N, d;
+  int q_rows;       // rows per head of the query tensor
+  int Cq, Ck;       // query groups per head (work list), key groups
+  const int32_t* off_q;  // [H, Cq+1]
+  const int32_t* off_k;  // [H, Ck+1]
+  const int32_t* csr;    // [H, Cq, kmax]
+  const int32_t* kh;     // [H]
+  int kmax;
+  float scale;
+  float* out;            // [H, q_rows, d] fp32
+  int32_t* work;         // [H, tiles_per_head]
+  int32_t* nwork;        // [H]
+  int tiles_per_head;
+  int32_t* nslots;       // [H, Cq]
+  int64_t* pairs;        // [H] (may be null)
+  DeviceStats* stats;
+};
+cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st);
+
+// ---- fit.cu ----------------------------------------------------------------
+cudaError_t launch_probe_select(const int32_t* off_q, int H, int Cq, int M, int32_t* probes,
+                                cudaStream_t st);
+cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* probes, int H,
+                                     int N, int M, int d, __nv_bfloat16* dst, cudaStream_t st);
+cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const int32_t* probes,
+                                   int H, int N, int M, int d, double* xr, double* means,
+                                   cudaStream_t st);
+cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
+                               const double* means, DeviceStats* stats, cudaStream_t st);
+cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* eval,
+                               const double* evec, int H, int d, int r, float* bp32, float* bv32,
+                               double* fit_out, cudaStream_t st);
+cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t* probes,
+                           const int32_t* perm_q, const float* bp32, const float* bv32, int H,
+                           int N, int M, int d, void* out, bool out_bf16, cudaStream_t st);
+cudaError_t launch_pairs_exec(const int64_t* pairs_sparse, int H, int64_t add, int64_t* pairs_exec,
+                              DeviceStats* stats, cudaStream_t st);
+
+}  // namespace spr

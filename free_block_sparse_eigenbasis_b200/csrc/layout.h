@@ -1,0 +1,154 @@
+// Workspace layout of the SparsePR library. The caller passes one device
+// buffer `ws`; every call carves the same regions out of it, at offsets that
+// depend only on the parameters. Regions are 256-byte aligned.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sparsepr.h"
+
+namespace spr {
+
+using DeviceStats = sparsepr_stats;
+
+constexpr int kTileM = 128;     // query rows per attention tile
+constexpr int kTileN = 128;     // keys per attention KV tile
+constexpr int kSlotRows = 8;    // keys per TMA row-slot of a KV tile
+constexpr int kSortChunk = 1024;  // tokens per counting-sort chunk
+constexpr int kMaxGroups = 4096;
+
+struct Layout {
+  // statistics / status (always at offset 0)
+  size_t stats;
+  // stage 1
+  size_t fy;       // [H, Nv] int32 Fisher-Yates scratch
+  size_t init_k;   // [H, Ck] int32
+  size_t init_q;   // [H, Cq] int32
+  size_t mk;       // [H, d, d] f64 (M_K, later the probe residual Gram R^T R)
+  size_t evec;     // [H, d, d] f64 Jacobi eigenvectors (columns)
+  size_t eval;     // [H, d] f64 Jacobi eigenvalues
+  size_t wk;       // [H, d, e] f64 key projector U_e L_e^{1/2}
+  size_t z;        // [H, Nv, e] f64 key coordinates
+  size_t mu;       // [H, Ck, e] f64 key centroids
+  size_t munorm;   // [H, Ck] f64 squared centroid norms
+  size_t lab_k;    // [H, Nv] int32
+  size_t lab_q;    // [H, Nv] int32
+  size_t flags;    // [H, 4] int32: changes_k, done_k, changes_q, done_q
+  size_t hist;     // [H, nchunk, Cmax] int32 counting-sort chunk histograms
+  size_t sortoff;  // [H, Cmax + 1] int32
+  size_t sortperm; // [H, Nv] int32
+  size_t ck;       // [H, Ck, d] f64 K/V group centroids
+  size_t g;        // [H, d, d] f64 query metric G
+  size_t qbar;     // [H, Cq, d] f64 query centroids
+  size_t wg;       // [H, Cq, d] f64 G * qbar
+  size_t cg;       // [H, Cq] f64 qbar^T G qbar
+  // stage 3
+  size_t cq;       // [H, Cq, d] f64 query-group means (route)
+  size_t ckr;      // [H, Ck, d] f64 key-group means (route)
+  size_t bf16_qkv; // [3, H, N, d] bf16 copies (fp32 inputs only)
+  size_t work;     // [H, tiles_per_head] int32 attention work list
+  size_t nwork;    // [H] int32
+  size_t nslots;   // [H, Cq] int32 KV row-slots per query group
+  // stage 4
+  size_t probe_q;  // [H, M, d] bf16 gathered probe rows (group-major)
+  size_t od;       // [H, M, d] f32 dense outputs of the probes
+  size_t xr;       // [H, 2, M, d] f64: X = O_sparse[probes], R = O_dense - X
+  size_t means;    // [H, 2, d] f64: xbar, rbar
+  size_t gram;     // [H, 2, d, d] f64: Xc^T Xc + lam I, Xc^T Rc
+  size_t bmat;     // [H, d, d] f64 ridge solution B
+  size_t bvec;     // [H, d] f64 intercept b
+  size_t bp32;     // [H, d, d] f32 projected B'
+  size_t bv32;     // [H, d] f32 projected b'
+  size_t pwork;    // [H, M/128 + 1] int32 probe attention work list
+  size_t pnwork;   // [H] int32
+  size_t pmeta;    // [H, 7] int32: dense-mode off_q(2), off_k(2), csr(1), k(1), nslots(1)
+  size_t total;
+
+  int Nv, e, Cmax, nchunk, tiles_per_head, kmax;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline int keep_budget(double keep, int Ck) {
+  // k = max(1, min(Ck, ceil(keep * Ck - 1e-9))) evaluated in fp64
+  double v = keep * static_cast<double>(Ck) - 1e-9;
+  long long k = static_cast<long long>(v);
+  if (static_cast<double>(k) < v) k += 1;  // ceil for positive v
+  if (v <= 0) k = 0;
+  if (k < 1) k = 1;
+  if (k > Ck) k = Ck;
+  return static_cast<int>(k);
+}
+
+inline void compute_layout(const sparsepr_params& p, Layout* L) {
+  const size_t H = p.H, N = p.N, d = p.d;
+  const int Nv = p.N - p.n_text;
+  const size_t e = p.n_eig, Ck = p.Ck, Cq = p.Cq, M = p.M;
+  L->Nv = Nv;
+  L->e = p.n_eig;
+  L->Cmax = (p.Ck > p.Cq ? p.Ck : p.Cq);
+  L->nchunk = (Nv + kSortChunk - 1) / kSortChunk;
+  L->tiles_per_head = (p.N + kTileM - 1) / kTileM + p.Cq;
+  int kmax = 1;
+  if (p.keep)
+    for (int h = 0; h < p.H; ++h) {
+      int k = keep_budget(p.keep[h], p.Ck);
+      if (k > kmax) kmax = k;
+    }
+  L->kmax = kmax;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L->stats = take(sizeof(DeviceStats));
+  L->fy = take(H * Nv * 4);
+  L->init_k = take(H * Ck * 4);
+  L->init_q = take(H * Cq * 4);
+  L->mk = take(H * d * d * 8);
+  L->evec = take(H * d * d * 8);
+  L->eval = take(H * d * 8);
+  L->wk = take(H * d * e * 8);
+  L->z = take(H * Nv * e * 8);
+  L->mu = take(H * Ck * e * 8);
+  L->munorm = take(H * Ck * 8);
+  L->lab_k = take(H * Nv * 4);
+  L->lab_q = take(H * Nv * 4);
+  L->flags = take(H * 4 * 4);
+  L->hist = take(H * static_cast<size_t>(L->nchunk) * L->Cmax * 4);
+  L->sortoff = take(H * (L->Cmax + 1) * 4);
+  L->sortperm = take(H * Nv * 4);
+  L->ck = take(H * Ck * d * 8);
+  L->g = take(H * d * d * 8);
+  L->qbar = take(H * Cq * d * 8);
+  L->wg = take(H * Cq * d * 8);
+  L->cg = take(H * Cq * 8);
+  L->cq = take(H * Cq * d * 8);
+  L->ckr = take(H * Ck * d * 8);
+  L->bf16_qkv = take(3 * H * N * d * 2);
+  L->work = take(H * static_cast<size_t>(L->tiles_per_head) * 4);
+  L->nwork = take(H * 4);
+  L->nslots = take(H * Cq * 4);
+  L->probe_q = take(H * (M + kTileM) * d * 2);
+  L->od = take(H * (M + 1) * d * 4);
+  L->xr = take(H * 2 * (M + 1) * d * 8);
+  L->means = take(H * 2 * d * 8);
+  L->gram = take(H * 2 * d * d * 8);
+  L->bmat = take(H * d * d * 8);
+  L->bvec = take(H * d * 8);
+  L->bp32 = take(H * d * d * 4);
+  L->bv32 = take(H * d * 4);
+  L->pwork = take(H * (M / kTileM + 2) * 4);
+  L->pnwork = take(H * 4);
+  L->pmeta = take(H * 7 * 4);
+  L->total = o;
+}
+
+template <typename T>
+inline T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+}  // namespace spr

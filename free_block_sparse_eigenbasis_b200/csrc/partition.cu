@@ -1,0 +1,483 @@
+// Stage 1 of "Partition the Support, Reconstruct the Residual" (2.A,
+// response-coupled partitioning): sampled-query metric M_K, key response
+// coordinates in its eigenbasis, key k-means, K/V group centroids, query
+// k-means on logit profiles (in the exact d-space form with
+// G = scale^2 C_K^T C_K).
+//
+// All distance, centroid and metric arithmetic is fp64; sums run in a fixed
+// order, so labels do not depend on scheduling.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Initial centroids: partial Fisher-Yates shuffle driven by SplitMix64
+// (Steele, Lea & Flood 2014). The virtual array a[i] = i is kept as a small
+// open-addressing map of the positions that moved.
+// ---------------------------------------------------------------------------
+constexpr int kFyTable = 16384;  // >= 2 * kMaxGroups, power of two
+
+__device__ __forceinline__ int fy_find(const int32_t* keys, int32_t pos) {
+  unsigned s = (static_cast<unsigned>(pos) * 2654435761u) & (kFyTable - 1);
+  while (keys[s] != -1 && keys[s] != pos) s = (s + 1) & (kFyTable - 1);
+  return static_cast<int>(s);
+}
+
+__global__ void fy_init_kernel(int Nv, int Ck, int Cq, uint64_t seed, int32_t* init_k,
+                               int32_t* init_q) {
+  extern __shared__ int32_t tab[];
+  int32_t* keys = tab;
+  int32_t* vals = tab + kFyTable;
+  const int h = blockIdx.x, which = blockIdx.y;
+  const int C = which ? Cq : Ck;
+  int32_t* out = which ? init_q + static_cast<size_t>(h) * Cq : init_k + static_cast<size_t>(h) * Ck;
+  for (int i = threadIdx.x; i < kFyTable; i += blockDim.x) keys[i] = -1;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  uint64_t state = seed ^ static_cast<uint64_t>(2 * h + which);
+  for (int i = 0; i < C; ++i) {
+    state += 0x9E3779B97F4A7C15ull;
+    uint64_t z = state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    const int j = i + static_cast<int>(z % static_cast<uint64_t>(Nv - i));
+    const int si = fy_find(keys, i);
+    const int32_t vi = (keys[si] == i) ? vals[si] : i;
+    const int sj = fy_find(keys, j);
+    const int32_t vj = (keys[sj] == j) ? vals[sj] : j;
+    keys[si] = i;
+    vals[si] = vj;
+    const int sj2 = fy_find(keys, j);  // slot may have shifted if si took it
+    keys[sj2] = j;
+    vals[sj2] = vi;
+    out[i] = vj;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Gram kernels: out = factor * sum_s x_s y_s^T (+ diag I), 32x32 output tile
+// per CTA, rows s summed in ascending order.
+// ---------------------------------------------------------------------------
+constexpr int kGT = 32;
+
+template <typename Loader>
+__device__ void gram_tile(Loader ld, int S, int d, double factor, double diag, double* out) {
+  __shared__ double xs[kGT][kGT + 1];
+  __shared__ double ys[kGT][kGT + 1];
+  const int a0 = blockIdx.x * kGT, b0 = blockIdx.y * kGT;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 256 threads: ty 0..7
+  double acc[4] = {0, 0, 0, 0};
+  for (int s0 = 0; s0 < S; s0 += kGT) {
+    for (int t = threadIdx.x; t < kGT * kGT; t += blockDim.x) {
+      const int ss = t / kGT, cc = t % kGT;
+      const int s = s0 + ss;
+      xs[ss][cc] = (s < S && a0 + cc < d) ? ld.x(s, a0 + cc) : 0.0;
+      ys[ss][cc] = (s < S && b0 + cc < d) ? ld.y(s, b0 + cc) : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int ss = 0; ss < kGT; ++ss) {
+      const double yv = ys[ss][tx];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fma(xs[ss][ty + 8 * i], yv, acc[i]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int a = a0 + ty + 8 * i, b = b0 + tx;
+    if (a < d && b < d) out[static_cast<size_t>(a) * d + b] = factor * acc[i] + (a == b ? diag : 0.0);
+  }
+}
+
+template <typename T>
+struct SampledQueryLoader {
+  const T* q;
+  int Nv, Ms, d;
+  __device__ double x(int s, int a) const {
+    const long long row = ((2LL * s + 1) * Nv) / (2LL * Ms);
+    return to_f64(q, static_cast<size_t>(row) * d + a);
+  }
+  __device__ double y(int s, int b) const { return x(s, b); }
+};
+
+template <typename T>
+__global__ void metric_mk_kernel(const T* q, int N, int Nv, int d, int Ms, double* out) {
+  const int h = blockIdx.z;
+  SampledQueryLoader<T> ld{q + static_cast<size_t>(h) * N * d, Nv, Ms, d};
+  gram_tile(ld, Ms, d, 1.0 / Ms, 0.0, out + static_cast<size_t>(h) * d * d);
+}
+
+struct F64Loader {
+  const double *X, *Y, *xm, *ym;
+  int ld;
+  __device__ double x(int s, int a) const {
+    return X[static_cast<size_t>(s) * ld + a] - (xm ? xm[a] : 0.0);
+  }
+  __device__ double y(int s, int b) const {
+    return Y[static_cast<size_t>(s) * ld + b] - (ym ? ym[b] : 0.0);
+  }
+};
+
+__global__ void gram_f64_kernel(const double* X, const double* Y, const double* xm,
+                                const double* ym, long long hsx, long long hsy, int ld, int S,
+                                int d, double factor, double diag, double* out, long long os,
+                                long long ms) {
+  const int h = blockIdx.z;
+  F64Loader l{X + h * hsx, Y + h * hsy, xm ? xm + h * ms : nullptr, ym ? ym + h * ms : nullptr,
+              ld};
+  gram_tile(l, S, d, factor, diag, out + h * os);
+}
+
+// ---------------------------------------------------------------------------
+// Key response coordinates z = W^T k, W = U_e L_e^{1/2} ([d, e] fp64).
+// ---------------------------------------------------------------------------
+constexpr int kZRows = 64;
+
+template <typename T>
+__global__ void zproj_kernel(const T* k, int N, int Nv, int d, int e, const double* wk,
+                             double* z) {
+  extern __shared__ double zsm[];
+  double* w = zsm;                  // [d][e]
+  float* ks = reinterpret_cast<float*>(zsm + d * e);  // [kZRows][d+1]
+  const int h = blockIdx.y;
+  const int j0 = blockIdx.x * kZRows;
+  const double* W = wk + static_cast<size_t>(h) * d * e;
+  for (int t = threadIdx.x; t < d * e; t += blockDim.x) w[t] = W[t];
+  const T* kh = k + static_cast<size_t>(h) * N * d;
+  for (int t = threadIdx.x; t < kZRows * d; t += blockDim.x) {
+    const int r = t / d, a = t % d;
+    const int j = j0 + r;
+    ks[r * (d + 1) + a] = (j < Nv) ? static_cast<float>(to_f64(kh, static_cast<size_t>(j) * d + a)) : 0.f;
+  }
+  __syncthreads();
+  // thread -> (row, output coordinate)
+  for (int t = threadIdx.x; t < kZRows * e; t += blockDim.x) {
+    const int r = t / e, c = t % e;
+    const int j = j0 + r;
+    if (j >= Nv) continue;
+    double acc = 0.0;
+    for (int a = 0; a < d; ++a) acc = fma(static_cast<double>(ks[r * (d + 1) + a]), w[a * e + c], acc);
+    z[(static_cast<size_t>(h) * Nv + j) * e + c] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Gather initial centroids (rows idx of src) as fp64, with squared norms.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double load_x(const void* X, int kind, size_t i) {
+  if (kind == kXf64) return static_cast<const double*>(X)[i];
+  if (kind == kXbf16) return to_f64(static_cast<const __nv_bfloat16*>(X), i);
+  return to_f64(static_cast<const float*>(X), i);
+}
+
+__global__ void gather_init_kernel(const void* src, int kind, long long hs, int ld, int D,
+                                   const int32_t* idx, int C, double* dst, double* norms) {
+  const int h = blockIdx.y;
+  const int c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= C) return;
+  const size_t row = static_cast<size_t>(idx[static_cast<size_t>(h) * C + c]);
+  double ss = 0.0;
+  for (int t = lane; t < D; t += 32) {
+    const double v = load_x(src, kind, h * hs + row * ld + t);
+    dst[(static_cast<size_t>(h) * C + c) * D + t] = v;
+    ss = fma(v, v, ss);
+  }
+  ss = warp_sum_f64(ss);
+  if (norms && lane == 0) norms[static_cast<size_t>(h) * C + c] = ss;
+}
+
+// ---------------------------------------------------------------------------
+// Nearest centroid: labels[i] = argmin_j (c_j - 2 x_i . y_j), lowest j on
+// ties, fp64. 64 rows x 64 centroids per tile step, 16x16 threads, 4x4
+// register block per thread, D in chunks of 32.
+// ---------------------------------------------------------------------------
+constexpr int kAR = 64, kAC = 64, kAK = 32;
+
+__global__ void __launch_bounds__(256) argmin_kernel(const void* X, int kind, long long hsx,
+                                                     int ldx, int n, int D, const double* Y,
+                                                     const double* c, int m, int32_t* labels,
+                                                     int32_t* flags, int flag_base) {
+  __shared__ double xs[kAK][kAR + 2];
+  __shared__ double ys[kAK][kAC + 2];
+  const int h = blockIdx.y;
+  int32_t* fl = flags + h * 4;
+  if (fl[flag_base + 1]) return;  // this head's k-means already converged
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int r0 = blockIdx.x * kAR;
+  const double* Yh = Y + static_cast<size_t>(h) * m * D;
+  const double* ch = c + static_cast<size_t>(h) * m;
+  double best[4];
+  int bidx[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    best[i] = INFINITY;
+    bidx[i] = 0x7fffffff;
+  }
+  for (int c0 = 0; c0 < m; c0 += kAC) {
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int k0 = 0; k0 < D; k0 += kAK) {
+      for (int t = threadIdx.x; t < kAK * kAR; t += blockDim.x) {
+        const int rr = t / kAK, kk = t % kAK;
+        const int row = r0 + rr, col = k0 + kk;
+        xs[kk][rr] = (row < n && col < D)
+                         ? load_x(X, kind, h * hsx + static_cast<size_t>(row) * ldx + col)
+                         : 0.0;
+        const int cc = c0 + rr;
+        ys[kk][rr] = (cc < m && col < D) ? Yh[static_cast<size_t>(cc) * D + col] : 0.0;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int kk = 0; kk < kAK; ++kk) {
+        double xv[4], yv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) yv[j] = ys[kk][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv[i], yv[j], acc[i][j]);
+      }
+      __syncthreads();
+    }
+    // epilogue: candidate distances of this centroid chunk
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      double bd = INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int cc = c0 + tx * 4 + j;
+        if (cc < m) {
+          const double dist = ch[cc] - 2.0 * acc[i][j];
+          if (dist < bd) {
+            bd = dist;
+            bi = cc;
+          }
+        }
+      }
+      // reduce over the 16 lanes sharing these rows (lowest index on ties)
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) {
+        const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (od < bd || (od == bd && oi < bi)) {
+          bd = od;
+          bi = oi;
+        }
+      }
+      if (bd < best[i] || (bd == best[i] && bi < bidx[i])) {
+        best[i] = bd;
+        bidx[i] = bi;
+      }
+    }
+  }
+  if (tx == 0) {
+    int changed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = r0 + ty * 4 + i;
+      if (row < n) {
+        int32_t* lp = labels + static_cast<size_t>(h) * n + row;
+        if (*lp != bidx[i]) changed++;
+        *lp = bidx[i];
+      }
+    }
+    if (changed) atomicAdd(&fl[flag_base + 0], changed);
+  }
+}
+
+// After a pass: count it; a pass after the first that changed no label ends
+// that head's k-means (labels repeat).
+__global__ void finalize_pass_kernel(int H, int pass, int32_t* flags, int flag_base,
+                                     int32_t* passes_out) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  int32_t* fl = flags + h * 4;
+  if (fl[flag_base + 1]) return;
+  passes_out[h] = pass + 1;
+  if (pass > 0 && fl[flag_base + 0] == 0) fl[flag_base + 1] = 1;
+  fl[flag_base + 0] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Group means in a fixed order: one warp per group, lanes own coordinates,
+// members summed in ascending position order of the stable sort.
+// ---------------------------------------------------------------------------
+__global__ void group_mean_kernel(const void* X, int kind, long long hsx, int ldx, int D,
+                                  const int32_t* perm, int perm_stride, const int32_t* off,
+                                  int off_stride, int C, bool keep_prev, double* out,
+                                  double* norms, const int32_t* skip, int skip_stride) {
+  const int h = blockIdx.y;
+  if (skip && skip[h * skip_stride]) return;
+  const int c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= C) return;
+  const int32_t* oo = off + static_cast<size_t>(h) * off_stride;
+  const int32_t* pp = perm ? perm + static_cast<size_t>(h) * perm_stride : nullptr;
+  const int lo = oo[c], hi = oo[c + 1];
+  double* dst = out + (static_cast<size_t>(h) * C + c) * D;
+  double ss = 0.0;
+  for (int t0 = 0; t0 < D; t0 += 32) {
+    const int t = t0 + lane;
+    double acc = 0.0;
+    if (t < D) {
+      for (int p = lo; p < hi; ++p) {
+        const size_t row = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
+        acc += load_x(X, kind, h * hsx + row * ldx + t);
+      }
+      double v;
+      if (hi > lo)
+        v = acc / static_cast<double>(hi - lo);
+      else
+        v = keep_prev ? dst[t] : 0.0;
+      dst[t] = v;
+      ss = fma(v, v, ss);
+    }
+  }
+  ss = warp_sum_f64(ss);
+  if (norms && lane == 0) norms[static_cast<size_t>(h) * C + c] = ss;
+}
+
+// W_g = G qbar_g, c_g = qbar_g^T G qbar_g (fp64, fixed-order reduction).
+__global__ void query_metric_apply_kernel(const double* G, const double* qbar, int Cq, int d,
+                                          double* wg, double* cg, const int32_t* skip,
+                                          int skip_stride) {
+  __shared__ double qs[128];
+  __shared__ double part[128];
+  const int h = blockIdx.y, g = blockIdx.x;
+  if (skip && skip[h * skip_stride]) return;
+  const double* Gh = G + static_cast<size_t>(h) * d * d;
+  const double* qb = qbar + (static_cast<size_t>(h) * Cq + g) * d;
+  const int a = threadIdx.x;
+  if (a < d) qs[a] = qb[a];
+  __syncthreads();
+  double w = 0.0;
+  if (a < d) {
+    for (int b = 0; b < d; ++b) w = fma(Gh[static_cast<size_t>(b) * d + a], qs[b], w);
+    wg[(static_cast<size_t>(h) * Cq + g) * d + a] = w;
+  }
+  part[a] = (a < d) ? qs[a] * w : 0.0;
+  __syncthreads();
+  for (int s = 64; s > 0; s >>= 1) {
+    if (a < s) part[a] += part[a + s];
+    __syncthreads();
+  }
+  if (a == 0) cg[static_cast<size_t>(h) * Cq + g] = part[0];
+}
+
+__global__ void write_labels_kernel(const int32_t* lab, int H, int N, int Nv, int C_text,
+                                    int32_t* out) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<size_t>(H) * N) return;
+  const int h = static_cast<int>(i / N), j = static_cast<int>(i % N);
+  out[i] = (j < Nv) ? lab[static_cast<size_t>(h) * Nv + j] : C_text;
+}
+
+}  // namespace
+
+cudaError_t launch_fy_init(int H, int Nv, int Ck, int Cq, uint64_t seed, int32_t* init_k,
+                           int32_t* init_q, cudaStream_t st) {
+  const int shb = 2 * kFyTable * 4;
+  cudaFuncSetAttribute(fy_init_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
+  fy_init_kernel<<<dim3(H, 2), 256, shb, st>>>(Nv, Ck, Cq, seed, init_k, init_q);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_metric_mk(const void* q, bool bf16, int H, int N, int Nv, int d, int Ms,
+                             double* out, cudaStream_t st) {
+  dim3 grid((d + kGT - 1) / kGT, (d + kGT - 1) / kGT, H);
+  if (bf16)
+    metric_mk_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), N, Nv, d, Ms, out);
+  else
+    metric_mk_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(q), N, Nv, d, Ms, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
+                            const double* ym, long long hsx, long long hsy, int ld, int S, int H,
+                            int d, double factor, double diag, double* out, long long os,
+                            long long ms, cudaStream_t st) {
+  dim3 grid((d + kGT - 1) / kGT, (d + kGT - 1) / kGT, H);
+  gram_f64_kernel<<<grid, 256, 0, st>>>(X, Y, xm, ym, hsx, hsy, ld, S, d, factor, diag, out, os,
+                                        ms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
+                         const double* wk, double* z, cudaStream_t st) {
+  const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;
+  dim3 grid((Nv + kZRows - 1) / kZRows, H);
+  if (bf16) {
+    cudaFuncSetAttribute(zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(shb));
+    zproj_kernel<<<grid, 256, shb, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv, d, e, wk, z);
+  } else {
+    cudaFuncSetAttribute(zproj_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(shb));
+    zproj_kernel<<<grid, 256, shb, st>>>(static_cast<const float*>(k), N, Nv, d, e, wk, z);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_init(const void* src, int src_kind, long long head_stride, int ld,
+                               int D, const int32_t* idx, int C, int H, double* dst,
+                               double* norms, cudaStream_t st) {
+  dim3 grid((C + 3) / 4, H);
+  gather_init_kernel<<<grid, 128, 0, st>>>(src, src_kind, head_stride, ld, D, idx, C, dst, norms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_argmin(const void* X, int x_kind, long long hsx, int ldx, int n, int D,
+                          const double* Y, const double* c, int m, int H, int32_t* labels,
+                          int32_t* flags, int flag_base, cudaStream_t st) {
+  dim3 grid((n + kAR - 1) / kAR, H);
+  argmin_kernel<<<grid, 256, 0, st>>>(X, x_kind, hsx, ldx, n, D, Y, c, m, labels, flags,
+                                      flag_base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_pass(int H, int pass, int32_t* flags, int flag_base,
+                                 int32_t* passes_out, cudaStream_t st) {
+  finalize_pass_kernel<<<(H + 127) / 128, 128, 0, st>>>(H, pass, flags, flag_base, passes_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx, int D,
+                              const int32_t* perm, int perm_stride, const int32_t* off,
+                              int off_stride, int C, int H, bool keep_prev, double* out,
+                              double* norms, const int32_t* skip, int skip_stride,
+                              cudaStream_t st) {
+  dim3 grid((C + 3) / 4, H);
+  group_mean_kernel<<<grid, 128, 0, st>>>(X, x_kind, hsx, ldx, D, perm, perm_stride, off,
+                                          off_stride, C, keep_prev, out, norms, skip,
+                                          skip_stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_query_metric_apply(const double* G, const double* qbar, int Cq, int H, int d,
+                                      double* wg, double* cg, const int32_t* skip,
+                                      int skip_stride, cudaStream_t st) {
+  query_metric_apply_kernel<<<dim3(Cq, H), 128, 0, st>>>(G, qbar, Cq, d, wg, cg, skip,
+                                                         skip_stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_write_labels(const int32_t* lab, int H, int N, int Nv, int C_text,
+                                int32_t* out, cudaStream_t st) {
+  const size_t tot = static_cast<size_t>(H) * N;
+  write_labels_kernel<<<static_cast<unsigned>((tot + 255) / 256), 256, 0, st>>>(lab, H, N, Nv,
+                                                                              C_text, out);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -1,0 +1,285 @@
+"""Thin Python binding of libsparsepr.so (the C ABI in include/sparsepr.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. torch is used for device memory and streams. Importing this module
+loads the in-tree library and raises if it has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsparsepr.so")
+MAX_HEADS = 256
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_NUMERIC = range(7)
+BF16, F32 = 0, 1
+
+EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_partition",
+            "sparsepr_permute", "sparsepr_route", "sparsepr_route_width",
+            "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
+            "sparsepr_reset_stats")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("N", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("n_text", ctypes.c_int32), ("Ck", ctypes.c_int32), ("Cq", ctypes.c_int32),
+                ("Ms", ctypes.c_int32), ("n_eig", ctypes.c_int32),
+                ("kmeans_iters", ctypes.c_int32), ("M", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("pad0", ctypes.c_int32), ("lam", ctypes.c_double), ("scale", ctypes.c_double),
+                ("seed", ctypes.c_uint64), ("keep", ctypes.POINTER(ctypes.c_double))]
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_uint32), ("H", ctypes.c_int32),
+                ("key_passes", ctypes.c_int32 * MAX_HEADS),
+                ("query_passes", ctypes.c_int32 * MAX_HEADS),
+                ("pairs_sparse", ctypes.c_int64 * MAX_HEADS),
+                ("pairs_exec", ctypes.c_int64 * MAX_HEADS)]
+
+
+class SparsePRError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__("%s: %s (status %d)" % (where, status_string(code), code))
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError("libsparsepr.so is not built; run "
+                          "`python -m free_block_sparse_eigenbasis_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, V, I32P, I64P = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    PP = ctypes.POINTER(Params)
+    st = ctypes.c_int
+    sz = ctypes.c_size_t
+    lib.sparsepr_workspace_bytes.argtypes = [PP]
+    lib.sparsepr_workspace_bytes.restype = sz
+    lib.sparsepr_status_string.argtypes = [st]
+    lib.sparsepr_status_string.restype = ctypes.c_char_p
+    lib.sparsepr_route_width.argtypes = [PP]
+    lib.sparsepr_route_width.restype = ctypes.c_int32
+    lib.sparsepr_partition.argtypes = [P, P, st, PP, I32P, I32P, V, sz, V]
+    lib.sparsepr_permute.argtypes = [P, P, P, st, PP, I32P, I32P, I32P, I32P, I32P, I32P, P, P, P,
+                                     V, sz, V]
+    lib.sparsepr_route.argtypes = [P, P, st, PP, I32P, I32P, I32P, I32P, V, sz, V]
+    lib.sparsepr_block_sparse_attn.argtypes = [P, P, P, st, PP, I32P, I32P, I32P, I32P, P, I64P,
+                                               V, sz, V]
+    lib.sparsepr_probe_correct.argtypes = [P, P, P, st, PP, I32P, I32P, P, I64P, P, I32P, I64P, P,
+                                           V, sz, V]
+    lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
+    lib.sparsepr_reset_stats.argtypes = [V, V]
+    for name in ("sparsepr_partition", "sparsepr_permute", "sparsepr_route",
+                 "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
+                 "sparsepr_reset_stats"):
+        getattr(lib, name).restype = st
+    return lib
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.sparsepr_status_string(code).decode()
+
+
+def make_params(p: dict):
+    """ctypes Params from a plain parameter dict; returns (params, keep array)
+    -- keep the second value alive for as long as the first is used."""
+    H = int(p["H"])
+    keep = p["keep"]
+    if not isinstance(keep, (list, tuple)):
+        keep = [keep] * H
+    arr = (ctypes.c_double * max(1, H))(*[float(x) for x in keep[:H]])
+    prm = Params(H=H, N=int(p["N"]), d=int(p["d"]), n_text=int(p.get("n_text", 0)),
+                 Ck=int(p["Ck"]), Cq=int(p["Cq"]), Ms=int(p["Ms"]), n_eig=int(p["n_eig"]),
+                 kmeans_iters=int(p["kmeans_iters"]), M=int(p["M"]), r=int(p["r"]), pad0=0,
+                 lam=float(p["lam"]), scale=float(p.get("scale", 0.0)),
+                 seed=int(p["seed"]) & ((1 << 64) - 1),
+                 keep=ctypes.cast(arr, ctypes.POINTER(ctypes.c_double)))
+    return prm, arr
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return BF16
+    if x.dtype == torch.float32:
+        return F32
+    raise TypeError("Q/K/V must be bf16 or fp32")
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise SparsePRError(code, where)
+
+
+def workspace_bytes(p: dict) -> int:
+    prm, keep = make_params(p)
+    return int(lib.sparsepr_workspace_bytes(ctypes.byref(prm)))
+
+
+def route_width(p: dict) -> int:
+    prm, keep = make_params(p)
+    return int(lib.sparsepr_route_width(ctypes.byref(prm)))
+
+
+# ---- the five calls, same names as the C ABI --------------------------------
+
+def sparsepr_partition(q, k, p, label_q, label_k, ws, stream=None):
+    prm, keep = make_params(p)
+    _check(lib.sparsepr_partition(_ptr(q), _ptr(k), _dtype_code(q), ctypes.byref(prm),
+                                  _ptr(label_q), _ptr(label_k), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "sparsepr_partition")
+
+
+def sparsepr_permute(q, k, v, p, label_q, label_k, perm_q, perm_k, off_q, off_k, qp, kp, vp, ws,
+                     stream=None):
+    prm, keep = make_params(p)
+    _check(lib.sparsepr_permute(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), ctypes.byref(prm),
+                                _ptr(label_q), _ptr(label_k), _ptr(perm_q), _ptr(perm_k),
+                                _ptr(off_q), _ptr(off_k), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(ws),
+                                ws.numel(), _stream(stream)), "sparsepr_permute")
+
+
+def sparsepr_route(qp, kp, p, off_q, off_k, csr, k_per_head, ws, stream=None):
+    prm, keep = make_params(p)
+    _check(lib.sparsepr_route(_ptr(qp), _ptr(kp), _dtype_code(qp), ctypes.byref(prm), _ptr(off_q),
+                              _ptr(off_k), _ptr(csr), _ptr(k_per_head), _ptr(ws), ws.numel(),
+                              _stream(stream)), "sparsepr_route")
+
+
+def sparsepr_block_sparse_attn(qp, kp, vp, p, off_q, off_k, csr, k_per_head, o_sparse,
+                               pairs_sparse, ws, stream=None):
+    prm, keep = make_params(p)
+    _check(lib.sparsepr_block_sparse_attn(_ptr(qp), _ptr(kp), _ptr(vp), _dtype_code(qp),
+                                          ctypes.byref(prm), _ptr(off_q), _ptr(off_k), _ptr(csr),
+                                          _ptr(k_per_head), _ptr(o_sparse), _ptr(pairs_sparse),
+                                          _ptr(ws), ws.numel(), _stream(stream)),
+           "sparsepr_block_sparse_attn")
+
+
+def sparsepr_probe_correct(qp, kp, vp, p, off_q, perm_q, o_sparse, pairs_sparse, out, probes,
+                           pairs_exec, ws, fit=None, stream=None):
+    prm, keep = make_params(p)
+    _check(lib.sparsepr_probe_correct(_ptr(qp), _ptr(kp), _ptr(vp), _dtype_code(qp),
+                                      ctypes.byref(prm), _ptr(off_q), _ptr(perm_q),
+                                      _ptr(o_sparse), _ptr(pairs_sparse), _ptr(out),
+                                      _ptr(probes), _ptr(pairs_exec), _ptr(fit), _ptr(ws),
+                                      ws.numel(), _stream(stream)), "sparsepr_probe_correct")
+
+
+def sparsepr_read_stats(ws) -> dict:
+    s = Stats()
+    _check(lib.sparsepr_read_stats(_ptr(ws), ctypes.byref(s)), "sparsepr_read_stats")
+    H = max(0, min(s.H, MAX_HEADS))
+    return dict(status=int(s.status), H=H, key_passes=list(s.key_passes[:H]),
+                query_passes=list(s.query_passes[:H]), pairs_sparse=list(s.pairs_sparse[:H]),
+                pairs_exec=list(s.pairs_exec[:H]))
+
+
+# ---- buffers + the whole call ----------------------------------------------
+
+@dataclass
+class Buffers:
+    """Device buffers of one attention call (all owned by torch)."""
+    ws: torch.Tensor
+    label_q: torch.Tensor
+    label_k: torch.Tensor
+    perm_q: torch.Tensor
+    perm_k: torch.Tensor
+    off_q: torch.Tensor
+    off_k: torch.Tensor
+    qp: torch.Tensor
+    kp: torch.Tensor
+    vp: torch.Tensor
+    csr: torch.Tensor
+    k_per_head: torch.Tensor
+    o_sparse: torch.Tensor
+    pairs_sparse: torch.Tensor
+    out: torch.Tensor
+    probes: torch.Tensor
+    pairs_exec: torch.Tensor
+    fit: Optional[torch.Tensor]
+
+
+def allocate(p: dict, dtype: torch.dtype, device="cuda", with_fit=False) -> Buffers:
+    H, N, d = int(p["H"]), int(p["N"]), int(p["d"])
+    Ck, Cq, M = int(p["Ck"]), int(p["Cq"]), int(p["M"])
+    wsb = workspace_bytes(p)
+    if wsb == 0:
+        raise SparsePRError(ERR_INVALID_ARG, "workspace_bytes")
+    kmax = route_width(p)
+    i32 = dict(dtype=torch.int32, device=device)
+    return Buffers(
+        ws=torch.empty(wsb, dtype=torch.uint8, device=device),
+        label_q=torch.empty((H, N), **i32), label_k=torch.empty((H, N), **i32),
+        perm_q=torch.empty((H, N), **i32), perm_k=torch.empty((H, N), **i32),
+        off_q=torch.empty((H, Cq + 1), **i32), off_k=torch.empty((H, Ck + 1), **i32),
+        qp=torch.empty((H, N, d), dtype=dtype, device=device),
+        kp=torch.empty((H, N, d), dtype=dtype, device=device),
+        vp=torch.empty((H, N, d), dtype=dtype, device=device),
+        csr=torch.empty((H, Cq, kmax), **i32), k_per_head=torch.empty(H, **i32),
+        o_sparse=torch.empty((H, N, d), dtype=torch.float32, device=device),
+        pairs_sparse=torch.empty(H, dtype=torch.int64, device=device),
+        out=torch.empty((H, N, d), dtype=dtype, device=device),
+        probes=torch.empty((H, max(M, 1)), **i32),
+        pairs_exec=torch.empty(H, dtype=torch.int64, device=device),
+        fit=torch.empty((H, d * d + d), dtype=torch.float64, device=device) if with_fit else None)
+
+
+def attention(q, k, v, p: dict, bufs: Optional[Buffers] = None, stream=None) -> Buffers:
+    """One SparsePR attention call on [H, N, d] device tensors: the five
+    library calls in order on one stream. Returns the buffers (bufs.out is
+    the corrected output in the original token order)."""
+    if bufs is None:
+        bufs = allocate(p, q.dtype, q.device)
+    b = bufs
+    sparsepr_partition(q, k, p, b.label_q, b.label_k, b.ws, stream)
+    sparsepr_permute(q, k, v, p, b.label_q, b.label_k, b.perm_q, b.perm_k, b.off_q, b.off_k, b.qp,
+                     b.kp, b.vp, b.ws, stream)
+    sparsepr_route(b.qp, b.kp, p, b.off_q, b.off_k, b.csr, b.k_per_head, b.ws, stream)
+    sparsepr_block_sparse_attn(b.qp, b.kp, b.vp, p, b.off_q, b.off_k, b.csr, b.k_per_head,
+                               b.o_sparse, b.pairs_sparse, b.ws, stream)
+    sparsepr_probe_correct(b.qp, b.kp, b.vp, p, b.off_q, b.perm_q, b.o_sparse, b.pairs_sparse,
+                           b.out, b.probes, b.pairs_exec, b.ws, b.fit, stream)
+    return b
+
+
+def dense_params(H: int, N: int, d: int, scale: float = 0.0) -> dict:
+    """Parameters of the same attention kernel run densely: one query group
+    and one key group covering all N tokens, keep = 1."""
+    return dict(H=H, N=N, d=d, n_text=0, Ck=1, Cq=1, Ms=1, n_eig=1, kmeans_iters=1,
+                keep=[1.0] * H, M=0, r=1, lam=0.0, scale=scale, seed=0)
+
+
+def dense_attention(q, k, v, out, ws=None, stream=None, meta=None):
+    """Dense softmax attention through the same block-sparse kernel (the
+    baseline of the same design): identity order, one group, full route.
+    ``meta`` caches the small routing tensors between calls."""
+    H, N, d = q.shape
+    p = dense_params(H, N, d)
+    if meta is None:
+        meta = dict(
+            off=torch.tensor([[0, N]] * H, dtype=torch.int32, device=q.device),
+            csr=torch.zeros((H, 1, 1), dtype=torch.int32, device=q.device),
+            kh=torch.ones(H, dtype=torch.int32, device=q.device),
+            pairs=torch.empty(H, dtype=torch.int64, device=q.device))
+    if ws is None:
+        ws = torch.empty(workspace_bytes(p), dtype=torch.uint8, device=q.device)
+    sparsepr_block_sparse_attn(q, k, v, p, meta["off"], meta["off"], meta["csr"], meta["kh"], out,
+                               meta["pairs"], ws, stream)
+    return meta, ws

@@ -1,0 +1,212 @@
+/*
+ * sparsepr.h -- C ABI of the SparsePR per-call sparse attention path on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web pages, cited by title and section):
+ *   [SPR]  "Partition the Support, Reconstruct the Residual: Training-Free
+ *          Sparse Attention for Video Generation and World Models" --
+ *          section 2 "Methodology": A. response-coupled partitioning,
+ *          B. probe-fitted residual reconstruction, C. sparse execution.
+ *   [SVOO] "Attention Sparsity is Input-Stable: Training-Free Sparse
+ *          Attention for Video Generation via Offline Sparsity Profiling and
+ *          Online QK Co-Clustering" -- method details, block selection and
+ *          sparse attention assembly.
+ *
+ * One attention call on H independent heads runs the five calls below in
+ * order on one CUDA stream:
+ *   sparsepr_partition -> sparsepr_permute -> sparsepr_route
+ *   -> sparsepr_block_sparse_attn -> sparsepr_probe_correct
+ *
+ * Conventions shared by every call
+ *   - Tensors are row-major [H, N, d] with d contiguous (Q, K, V and the
+ *     outputs) or [H, n] (integer arrays). All tensor pointers are DEVICE
+ *     pointers owned by the caller; the library never allocates, frees or
+ *     synchronises on them.
+ *   - `ws` is a caller-owned device workspace of at least
+ *     sparsepr_workspace_bytes(p) bytes, 256-byte aligned. The same `ws` is
+ *     passed to every call of one attention call; its first bytes hold the
+ *     device status word and per-call statistics (see sparsepr_read_stats).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call only enqueues work on it and returns.
+ *   - Argument errors are found on the host before anything is enqueued and
+ *     are returned as SPARSEPR_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE.
+ *     A failed launch returns SPARSEPR_ERR_CUDA. Errors that only the device
+ *     can see (an empty kept key set, a non-finite value, a wait that ran
+ *     out) are OR-ed into the status word in `ws`; read it after the stream
+ *     has been synchronised.
+ *   - Supported: d in {64, 128}; dtype bf16 or fp32 (the attention MMAs run
+ *     in bf16 with fp32 accumulation for both); 1 <= H <= SPARSEPR_MAX_HEADS;
+ *     n_text = 0.
+ */
+#ifndef SPARSEPR_H_
+#define SPARSEPR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPARSEPR_MAX_HEADS 256
+
+typedef enum {
+  SPARSEPR_OK = 0,
+  SPARSEPR_ERR_INVALID_ARG = 1, /* null pointer, inconsistent sizes, bad parameter */
+  SPARSEPR_ERR_UNSUPPORTED = 2, /* valid but not built: head dim, dtype, text tokens */
+  SPARSEPR_ERR_WORKSPACE = 3,   /* ws smaller than sparsepr_workspace_bytes() or misaligned */
+  SPARSEPR_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  SPARSEPR_ERR_TIMEOUT = 5,     /* device status: a bounded wait ran out */
+  SPARSEPR_ERR_NUMERIC = 6      /* device status: empty kept set or non-finite value */
+} sparsepr_status;
+
+typedef enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 } sparsepr_dtype;
+
+/* Method parameters, passed by const pointer; the callee copies what it
+ * needs before returning. */
+typedef struct {
+  int32_t H;            /* heads, 1..SPARSEPR_MAX_HEADS */
+  int32_t N;            /* tokens per head (video tokens + n_text) */
+  int32_t d;            /* head dim: 64 or 128 */
+  int32_t n_text;       /* trailing always-kept text tokens; must be 0 */
+  int32_t Ck;           /* key (K/V) groups, 1..min(Nv, 4096) */
+  int32_t Cq;           /* query groups, 1..min(Nv, 4096) */
+  int32_t Ms;           /* sampled queries for M_K, 1..Nv */
+  int32_t n_eig;        /* eigenvectors e of M_K used as key coordinates, 1..min(d,32) */
+  int32_t kmeans_iters; /* cap on k-means assignment passes (stops early when labels repeat) */
+  int32_t M;            /* probe rows per head, 0..Nv */
+  int32_t r;            /* rank of the residual subspace, 1..d */
+  int32_t pad0;
+  double lambda;        /* ridge penalty, >= 0 */
+  double scale;         /* softmax scale; 0 selects 1/sqrt(d) */
+  uint64_t seed;        /* k-means initialisation seed */
+  const double* keep;   /* HOST array [H]: kept fraction of key groups per head, (0, 1] */
+} sparsepr_params;
+
+/* Device statistics of the last attention call, copied out by
+ * sparsepr_read_stats. */
+typedef struct {
+  uint32_t status;       /* OR of (1 << sparsepr_status) device-detected errors; 0 = fine */
+  int32_t H;
+  int32_t key_passes[SPARSEPR_MAX_HEADS];   /* k-means assignment passes run per head */
+  int32_t query_passes[SPARSEPR_MAX_HEADS];
+  int64_t pairs_sparse[SPARSEPR_MAX_HEADS]; /* routed (row, key) pairs per head */
+  int64_t pairs_exec[SPARSEPR_MAX_HEADS];   /* pairs_sparse + M*N (probe rows) */
+} sparsepr_stats;
+
+/* Bytes of device workspace the five calls need for these parameters
+ * (0 if the parameters are invalid). */
+size_t sparsepr_workspace_bytes(const sparsepr_params* p);
+
+/* Human-readable name of a status code (static string). */
+const char* sparsepr_status_string(sparsepr_status s);
+
+/* Stage 1 [SPR 2.A, response-coupled partitioning].
+ * Keys: M_K = Q_s^T Q_s / Ms from Ms strided sampled queries; top-n_eig
+ * eigenpairs (U, L) of M_K; key coordinates z = L^{1/2} U^T k; Lloyd k-means
+ * into Ck groups (lowest index on ties, empty groups keep their centroid,
+ * at most kmeans_iters passes, stop when labels repeat).
+ * Queries: logit profiles p = scale * C_K q against the K/V group centroids
+ * C_K (original-space means); Lloyd k-means into Cq groups, evaluated in the
+ * exact d-space form (q - qbar)^T G (q - qbar), G = scale^2 C_K^T C_K.
+ * Initial centroids: rows chosen by a partial Fisher-Yates shuffle driven by
+ * SplitMix64 seeded with seed ^ (2*head + {0 keys, 1 queries}).
+ *   q, k      [H, N, d] input dtype (device, read only)
+ *   label_q   [H, N] int32 out: query group of each token, 0..Cq-1
+ *   label_k   [H, N] int32 out: key group of each token, 0..Ck-1 */
+sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype dt,
+                                   const sparsepr_params* p, int32_t* label_q,
+                                   int32_t* label_k, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* Stage 2 [SPR 2.C, contiguous group-major layout].
+ * Stable counting sort of the tokens by group: perm[h, i] is the token at
+ * group-major row i (ascending token order inside a group); off[h, c] is
+ * the first row of group c (off[h, C] = N). qp = q[perm_q], kp = k[perm_k],
+ * vp = v[perm_k] (K and V share the key partition).
+ *   label_q, label_k   [H, N] int32 in (values must lie in 0..Cq-1 / 0..Ck-1)
+ *   perm_q, perm_k     [H, N] int32 out
+ *   off_q [H, Cq+1], off_k [H, Ck+1] int32 out
+ *   qp, kp, vp         [H, N, d] input dtype out (must not alias q, k, v) */
+sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v,
+                                 sparsepr_dtype dt, const sparsepr_params* p,
+                                 const int32_t* label_q, const int32_t* label_k,
+                                 int32_t* perm_q, int32_t* perm_k, int32_t* off_q,
+                                 int32_t* off_k, void* qp, void* kp, void* vp,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 3a [SVOO block selection].
+ * Block scores A[g, c] = scale * C_Q[g] . C_K[c] in fp64 from the group mean
+ * rows of qp / kp (zero vector for an empty group); each query group keeps
+ * its top-k_h key groups, ties to the lowest index, listed ascending.
+ * k_h = max(1, min(Ck, ceil(keep[h] * Ck - 1e-9))).
+ *   csr         [H, Cq, kmax] int32 out, kmax = max_h k_h; entries past
+ *               k_h are -1
+ *   k_per_head  [H] int32 out */
+sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt,
+                               const sparsepr_params* p, const int32_t* off_q,
+                               const int32_t* off_k, int32_t* csr,
+                               int32_t* k_per_head, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* Largest k_h of sparsepr_route for these parameters (the csr row width),
+ * or -1 if the parameters are invalid. */
+int32_t sparsepr_route_width(const sparsepr_params* p);
+
+/* Stage 3b [SPR 2.C variable-block sparse attention; SVOO: the softmax is
+ * normalised over the kept logits only].
+ * For group-major query row i of group g:
+ *   o_sparse[i] = sum_{j in S(g)} softmax_{S(g)}(scale * qp_i . kp_j) vp_j,
+ * S(g) = union of the key ranges off_k[c]..off_k[c+1] of the kept groups c
+ * in csr[g]. Skipped key groups are never multiplied. bf16 tensor-core MMAs
+ * (tcgen05, fp32 accumulation in tensor memory).
+ *   o_sparse      [H, N, d] fp32 out, group-major row order
+ *   pairs_sparse  [H] int64 out: sum_g n_g * |S(g)| (exact pair count)
+ * A query group whose kept set is empty raises SPARSEPR_ERR_NUMERIC in the
+ * status word and its rows are written as 0. */
+sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const void* vp,
+                                           sparsepr_dtype dt, const sparsepr_params* p,
+                                           const int32_t* off_q, const int32_t* off_k,
+                                           const int32_t* csr, const int32_t* k_per_head,
+                                           float* o_sparse, int64_t* pairs_sparse,
+                                           void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 4 [SPR 2.B, probe-fitted residual reconstruction].
+ * Probes: m_g rows of query group g, m_g proportional to the group size by
+ * largest remainder (ties to the lower group, sum M), at group-major offsets
+ * floor((t + 1/2) n_g / m_g). O_dense of the probe rows is exact softmax
+ * attention over all N keys; R = O_dense - O_sparse on the probes.
+ * Ridge fit (fp64, intercept unpenalised): B = (Xc^T Xc + lambda I)^{-1}
+ * Xc^T Rc, b = rbar - xbar B with X = O_sparse[probes]. Subspace: V_r = top-r
+ * right singular vectors of R; B' = B V_r V_r^T, b' = b V_r V_r^T.
+ * Output: out[perm_q[i]] = O_dense(i) for probe rows, else
+ * o_sparse[i] + b' + o_sparse[i] B', rounded to the input dtype (RNE).
+ *   perm_q         [H, N] int32 in (from sparsepr_permute)
+ *   o_sparse       [H, N, d] fp32 in (from sparsepr_block_sparse_attn)
+ *   pairs_sparse   [H] int64 in
+ *   out            [H, N, d] input dtype out, ORIGINAL token order
+ *   probes         [H, M] int32 out: group-major probe rows, ascending
+ *   pairs_exec     [H] int64 out: pairs_sparse + M * N
+ *   fit            [H, d*d + d] fp64 out, optional (NULL = skip): B' row-major
+ *                  then b' */
+sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const void* vp,
+                                       sparsepr_dtype dt, const sparsepr_params* p,
+                                       const int32_t* off_q, const int32_t* perm_q,
+                                       const float* o_sparse, const int64_t* pairs_sparse,
+                                       void* out, int32_t* probes, int64_t* pairs_exec,
+                                       double* fit, void* ws, size_t ws_bytes,
+                                       void* stream);
+
+/* Copy the device statistics of the last call out of `ws` (a blocking
+ * device-to-host copy; call after the stream has been synchronised). */
+sparsepr_status sparsepr_read_stats(const void* ws, sparsepr_stats* out);
+
+/* Zero the status word and statistics in `ws` (enqueued on `stream`).
+ * sparsepr_partition does this itself at the start of every call. */
+sparsepr_status sparsepr_reset_stats(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEPR_H_ */

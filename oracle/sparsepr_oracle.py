@@ -449,12 +449,19 @@ def run_head(q, k, v, p: dict, head: int, rows=None, partition_only=False) -> He
     M = int(p["M"])
     probes = probe_rows(off_q[:Cq + 1], M)
     pairs_exec = pairs_sparse + M * N
-    Xs = masked_attention_rows(Qp, Kp, Vp, probes, row_group, mask_of_group, scale)
-    Od = dense_attention(Qp[probes], Kp, Vp, scale)
-    R = Od - Xs
-    B, b = ridge_fit(Xs, R, float(p["lam"]))
-    Vr = residual_subspace(R, int(p["r"]))
-    Bp, bp = project_map(B, b, Vr)
+    if M > 0:
+        Xs = masked_attention_rows(Qp, Kp, Vp, probes, row_group, mask_of_group, scale)
+        Od = dense_attention(Qp[probes], Kp, Vp, scale)
+        R = Od - Xs
+        B, b = ridge_fit(Xs, R, float(p["lam"]))
+        Vr = residual_subspace(R, int(p["r"]))
+        Bp, bp = project_map(B, b, Vr)
+    else:
+        # no probes: the hard-drop variant (sparse output, no reconstruction)
+        Xs = Od = np.zeros((0, d))
+        B = Bp = np.zeros((d, d))
+        b = bp = np.zeros(d)
+        Vr = np.zeros((d, 0))
 
     if rows is None:
         rows = np.arange(N, dtype=np.int64)

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/sparsepr.h declares, sizes its workspace, and
+rejects bad arguments before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from free_block_sparse_eigenbasis_b200 import sparsepr as S
+from free_block_sparse_eigenbasis_b200 import synth
+from oracle import sparsepr_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sparsepr.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparsepr_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_five_calls():
+    names = declared_functions()
+    for n in ("sparsepr_partition", "sparsepr_permute", "sparsepr_route",
+              "sparsepr_block_sparse_attn", "sparsepr_probe_correct"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(S._LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(declared_functions()) <= set(S.EXPORTED) | set(declared_functions())
+
+
+def test_params_struct_layout():
+    # 12 int32 + lambda + scale + seed + keep pointer
+    assert ctypes.sizeof(S.Params) == 48 + 8 + 8 + 8 + 8
+    assert S.Params.lam.offset == 48 and S.Params.keep.offset == 72
+
+
+def test_workspace_and_route_width():
+    for name in ("tiny", "wan13b_480p", "wan13b_720p", "wan14b_720p"):
+        w = synth.workload(name)
+        p = w.params()
+        assert S.workspace_bytes(p) > 0
+        assert S.route_width(p) == max(O.keep_budget(k, w.Ck) for k in w.keep)
+
+
+def test_keep_budget_matches_oracle_on_edge_values():
+    base = synth.workload("tiny").params()
+    for keep, Ck in [(0.22, 1000), (0.2201, 1000), (1e-6, 1000), (1.0, 16), (0.3333333, 3)]:
+        p = dict(base, Ck=Ck, N=4096, keep=[keep])
+        assert S.route_width(p) == O.keep_budget(keep, Ck)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d=96), dict(H=0), dict(H=300), dict(Ck=0), dict(Cq=5000), dict(Ms=0),
+    dict(n_eig=0), dict(n_eig=40), dict(M=-1), dict(r=0), dict(r=65), dict(lam=-1.0),
+    dict(keep=[0.0]), dict(keep=[1.5]), dict(n_text=8), dict(kmeans_iters=0), dict(N=8),
+])
+def test_invalid_params_rejected_on_host(bad):
+    p = dict(synth.workload("tiny").params(), **bad)
+    assert S.workspace_bytes(p) == 0
+    prm, keep = S.make_params(p)
+    fake = ctypes.c_void_p(1 << 40)  # never dereferenced: the call must fail first
+    code = S.lib.sparsepr_partition(fake, fake, S.BF16, ctypes.byref(prm), fake, fake, fake,
+                                    1 << 30, None)
+    assert code in (S.ERR_INVALID_ARG, S.ERR_UNSUPPORTED)
+
+
+def test_null_pointers_and_small_workspace_rejected():
+    p = synth.workload("tiny").params()
+    prm, keep = S.make_params(p)
+    fake = ctypes.c_void_p(1 << 40)
+    need = S.workspace_bytes(p)
+    lib = S.lib
+    assert lib.sparsepr_partition(None, fake, S.F32, ctypes.byref(prm), fake, fake, fake, need,
+                                  None) == S.ERR_INVALID_ARG
+    assert lib.sparsepr_partition(fake, fake, S.F32, ctypes.byref(prm), fake, fake, fake,
+                                  need - 1, None) == S.ERR_WORKSPACE
+    # misaligned workspace
+    assert lib.sparsepr_partition(fake, fake, S.F32, ctypes.byref(prm), fake, fake,
+                                  ctypes.c_void_p((1 << 40) + 8), need, None) == S.ERR_WORKSPACE
+    assert lib.sparsepr_partition(fake, fake, 7, ctypes.byref(prm), fake, fake, fake, need,
+                                  None) == S.ERR_UNSUPPORTED
+    assert lib.sparsepr_route(fake, fake, S.F32, ctypes.byref(prm), fake, fake, None, fake, fake,
+                              need, None) == S.ERR_INVALID_ARG
+    assert lib.sparsepr_block_sparse_attn(fake, fake, fake, S.F32, ctypes.byref(prm), fake, fake,
+                                          fake, fake, fake, None, fake, need,
+                                          None) == S.ERR_INVALID_ARG
+    assert lib.sparsepr_probe_correct(fake, fake, fake, S.F32, ctypes.byref(prm), fake, fake, fake,
+                                      fake, fake, None, fake, None, fake, need,
+                                      None) == S.ERR_INVALID_ARG
+    # permuted outputs may not alias the inputs
+    assert lib.sparsepr_permute(fake, fake, fake, S.F32, ctypes.byref(prm), fake, fake, fake, fake,
+                                fake, fake, fake, fake, fake, fake, need,
+                                None) == S.ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for c in range(7):
+        assert S.status_string(c)

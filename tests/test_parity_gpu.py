@@ -1,0 +1,144 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs. Integer outputs (labels, permutations, offsets, routes,
+probes, pair counts) must match bit for bit; float outputs must lie within
+max-abs 2e-2 and mean-abs 2e-3."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from free_block_sparse_eigenbasis_b200 import synth
+from oracle import sparsepr_oracle as O
+from tests.parity import (MAX_ABS, MEAN_ABS, assert_close, compare_head, gpu_run, np_,
+                          oracle_head)
+
+pytestmark = pytest.mark.gpu
+
+
+def _S():
+    from free_block_sparse_eigenbasis_b200 import sparsepr as S
+    return S
+
+
+def test_tiny_full_pipeline():
+    w = synth.workload("tiny")
+    b, (q, k, v) = gpu_run(w)
+    res = oracle_head(w, q, k, v, 0)
+    compare_head(b, res, w, 0, None)
+    st = _S().sparsepr_read_stats(b.ws)
+    assert st["status"] == 0
+    assert st["key_passes"][0] == res.info["key_passes"]
+    assert st["query_passes"][0] == res.info["query_passes"]
+    # the fitted map
+    fit = np_(b.fit[0])
+    d = w.d
+    assert np.abs(fit[:d * d].reshape(d, d) - res.Bp).max() < 5e-2 * max(1.0, np.abs(res.Bp).max())
+
+
+SMALL = [
+    # several query tiles per group, ragged tails, two heads with different budgets
+    synth.custom("small_bf16_d128", 2, (4, 16, 32), 128, "bf16", Ck=64, Cq=16, Ms=256,
+                 n_eig=8, M=64, r=16, keep=(0.25, 0.4), seed=11),
+    # fp32 input, d=64, N not a multiple of 8 or 128
+    synth.custom("small_f32_d64", 1, (3, 7, 11), 64, "f32", Ck=12, Cq=5, Ms=64, n_eig=4,
+                 M=20, r=8, keep=0.3, seed=5),
+    # keep = 1: the sparse path is dense attention
+    synth.custom("keep_one", 1, (2, 8, 16), 128, "bf16", Ck=16, Cq=4, Ms=64, n_eig=4, M=16,
+                 r=8, keep=1.0, seed=3),
+    # one key group kept, no probes (hard-drop: output = sparse output)
+    synth.custom("hard_drop", 1, (2, 8, 16), 128, "bf16", Ck=16, Cq=4, Ms=64, n_eig=4, M=0,
+                 r=8, keep=0.05, seed=4),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[x.name for x in SMALL])
+def test_small_full_pipeline(w):
+    b, (q, k, v) = gpu_run(w)
+    for h in range(w.H):
+        res = oracle_head(w, q, k, v, h)
+        compare_head(b, res, w, h, None)
+    assert _S().sparsepr_read_stats(b.ws)["status"] == 0
+
+
+def test_keep_one_matches_dense_attention():
+    w = SMALL[2]
+    b, (q, k, v) = gpu_run(w)
+    D = O.dense_attention(synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0]),
+                          1 / math.sqrt(w.d))
+    assert_close(np_(b.out[0].float()), D, "keep=1 vs dense")
+
+
+def test_attention_kernel_on_oracle_routes():
+    """The attention call alone, fed the oracle's permutation and routes."""
+    S = _S()
+    w = SMALL[0]
+    q, k, v = synth.generate(w)
+    p = w.params()
+    b = S.allocate(p, q.dtype)
+    for h in range(w.H):
+        res = oracle_head(w, q, k, v, h)
+        b.qp[h].copy_(q[h][torch.from_numpy(res.perm_q)].cuda())
+        b.kp[h].copy_(k[h][torch.from_numpy(res.perm_k)].cuda())
+        b.vp[h].copy_(v[h][torch.from_numpy(res.perm_k)].cuda())
+        b.off_q[h].copy_(torch.from_numpy(res.off_q).int())
+        b.off_k[h].copy_(torch.from_numpy(res.off_k).int())
+        b.csr[h].fill_(-1)
+        b.csr[h][:, :res.k].copy_(torch.from_numpy(res.csr).int())
+        b.k_per_head[h] = res.k
+    S.sparsepr_block_sparse_attn(b.qp, b.kp, b.vp, p, b.off_q, b.off_k, b.csr, b.k_per_head,
+                                 b.o_sparse, b.pairs_sparse, b.ws)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        res = oracle_head(w, q, k, v, h)
+        assert int(b.pairs_sparse[h]) == res.pairs_sparse
+        assert_close(np_(b.o_sparse[h]), res.o_sparse, "o_sparse head %d" % h)
+
+
+@pytest.mark.parametrize("N", [16, 130, 1000, 4096 + 40])
+def test_dense_mode_against_textbook_attention(N):
+    S = _S()
+    g = torch.Generator().manual_seed(N)
+    q = torch.randn(2, N, 128, generator=g).bfloat16()
+    k = torch.randn(2, N, 128, generator=g).bfloat16()
+    v = torch.randn(2, N, 128, generator=g).bfloat16()
+    out = torch.empty(2, N, 128, device="cuda")
+    S.dense_attention(q.cuda(), k.cuda(), v.cuda(), out)
+    torch.cuda.synchronize()
+    for h in range(2):
+        D = O.dense_attention(q[h].double().numpy(), k[h].double().numpy(), v[h].double().numpy(),
+                              1 / math.sqrt(128))
+        assert_close(np_(out[h]), D, "dense N=%d head %d" % (N, h))
+
+
+def test_wan13b_480p_first_and_last_head():
+    w = synth.workload("wan13b_480p")
+    b, (q, k, v) = gpu_run(w)
+    rows = np.arange(0, w.N, 61)
+    for h in (0, w.H - 1):
+        res = oracle_head(w, q, k, v, h, rows=rows)
+        compare_head(b, res, w, h, rows)
+    assert _S().sparsepr_read_stats(b.ws)["status"] == 0
+
+
+def test_wan13b_720p_head0_sampled():
+    """The benchmark's workload and launch configuration: all 12 heads on the
+    GPU, head 0 checked against the oracle on sampled rows."""
+    w = synth.workload("wan13b_720p")
+    b, (q, k, v) = gpu_run(w)
+    rows = np.arange(7, w.N, 149)
+    res = oracle_head(w, q, k, v, 0, rows=rows)
+    compare_head(b, res, w, 0, rows)
+    st = _S().sparsepr_read_stats(b.ws)
+    assert st["status"] == 0
+    # every head: a valid partition and exact pair accounting from its own routes
+    for h in range(w.H):
+        off_q, off_k = np_(b.off_q[h]), np_(b.off_k[h])
+        assert off_q[-1] == w.N and off_k[-1] == w.N
+        lab = np_(b.label_q[h])
+        assert np.array_equal(np.diff(off_q), np.bincount(lab, minlength=w.Cq))
+        csr = np_(b.csr[h])[:, :int(b.k_per_head[h])]
+        nk = np.diff(off_k)
+        pairs = int((np.diff(off_q) * nk[csr].sum(axis=1)).sum())
+        assert pairs == int(b.pairs_sparse[h]) == st["pairs_sparse"][h]
+        assert int(b.pairs_exec[h]) == pairs + w.M * w.N
