@@ -1,0 +1,105 @@
+// sparsepr_route_noalloc: the routing call without a caller workspace.
+//
+// Some callers cannot call cudaMalloc or hand the library a workspace: code
+// that must not synchronise the device (cudaMalloc can), processes that
+// reserve all device memory up front in their own pool, and hosts whose
+// memory plan is fixed before the first call. This entry point computes the
+// same routes as sparsepr_route, but its scratch (the fp64 group means of Q
+// and K) lives in one file-scope device array of fixed size instead of the
+// caller's workspace, and it allocates nothing.
+//
+//   * Scratch: kRouteScratchBytes (4 MiB) per GPU that loads the library,
+//     held until the process exits. Heads are processed in chunks that fit;
+//     one head needs (Cq + Ck) * d * 8 bytes, and parameters whose single
+//     head does not fit are rejected with SPARSEPR_ERR_WORKSPACE.
+//   * Set-up: the first call on each device looks up the array's device
+//     address (cudaGetSymbolAddress) with that device current. Make that
+//     first call before any stream capture.
+//   * Every call shares the one array and it keeps the last call's
+//     contents; each call overwrites all the scratch it reads, so nothing
+//     needs clearing. Calls whose work overlaps on the GPU (other streams,
+//     other host threads) race on the array: order them on one stream.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+namespace {
+
+constexpr size_t kRouteScratchBytes = 4u << 20;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array for the current device (looked up once).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace spr
+
+using namespace spr;
+
+extern "C" sparsepr_status sparsepr_route_noalloc(const void* qp, const void* kp,
+                                                  sparsepr_dtype dt, const sparsepr_params* p,
+                                                  const int32_t* off_q, const int32_t* off_k,
+                                                  int32_t* csr, int32_t* k_per_head,
+                                                  void* stream) {
+  if (sparsepr_workspace_bytes(p) == 0) {
+    if (p && p->keep && (p->d != 64 && p->d != 128)) return SPARSEPR_ERR_UNSUPPORTED;
+    return SPARSEPR_ERR_INVALID_ARG;
+  }
+  if (p->n_text != 0) return SPARSEPR_ERR_UNSUPPORTED;
+  if (dt != SPARSEPR_BF16 && dt != SPARSEPR_F32) return SPARSEPR_ERR_UNSUPPORTED;
+  if (!qp || !kp || !off_q || !off_k || !csr || !k_per_head) return SPARSEPR_ERR_INVALID_ARG;
+  const int H = p->H, N = p->N, d = p->d, Ck = p->Ck, Cq = p->Cq;
+  const size_t per_head = (static_cast<size_t>(Cq) + Ck) * d * sizeof(double);
+  if (per_head > kRouteScratchBytes) return SPARSEPR_ERR_WORKSPACE;
+  const int chunk = static_cast<int>(kRouteScratchBytes / per_head);
+  void* base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return SPARSEPR_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const double scale = p->scale > 0.0 ? p->scale : 1.0 / sqrt(static_cast<double>(d));
+  const int kind = (dt == SPARSEPR_BF16) ? kXbf16 : kXf32;
+  const size_t eb = (dt == SPARSEPR_BF16) ? 2 : 4;
+  int32_t kh[SPARSEPR_MAX_HEADS];
+  int kmax = 1;
+  for (int h = 0; h < H; ++h) {
+    kh[h] = keep_budget(p->keep[h], Ck);
+    if (kh[h] > kmax) kmax = kh[h];
+  }
+  if (launch_write_k(kh, H, k_per_head, st) != cudaSuccess) return SPARSEPR_ERR_CUDA;
+  double* cq = static_cast<double*>(base);
+  for (int h0 = 0; h0 < H; h0 += chunk) {
+    const int hc = (H - h0 < chunk) ? (H - h0) : chunk;
+    double* ckr = cq + static_cast<size_t>(hc) * Cq * d;
+    const size_t head_elems = static_cast<size_t>(N) * d;
+    const char* qh = static_cast<const char*>(qp) + h0 * head_elems * eb;
+    const char* kh0 = static_cast<const char*>(kp) + h0 * head_elems * eb;
+    if (launch_range_mean(qh, kind, hc, N, d, off_q + static_cast<size_t>(h0) * (Cq + 1), Cq, cq,
+                          st) != cudaSuccess ||
+        launch_range_mean(kh0, kind, hc, N, d, off_k + static_cast<size_t>(h0) * (Ck + 1), Ck,
+                          ckr, st) != cudaSuccess ||
+        launch_route(cq, ckr, hc, Cq, Ck, d, scale, k_per_head + h0, kmax,
+                     csr + static_cast<size_t>(h0) * Cq * kmax, st) != cudaSuccess)
+      return SPARSEPR_ERR_CUDA;
+  }
+  return SPARSEPR_OK;
+}

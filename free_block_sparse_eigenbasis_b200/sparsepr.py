@@ -71,6 +71,8 @@ def _load():
                                                V, sz, V]
     lib.sparsepr_probe_correct.argtypes = [P, P, P, st, PP, I32P, I32P, P, I64P, P, I32P, I64P, P,
                                            V, sz, V]
+    lib.sparsepr_route_noalloc.argtypes = [P, P, st, PP, I32P, I32P, I32P, I32P, V]
+    lib.sparsepr_route_noalloc.restype = st
     lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
     lib.sparsepr_reset_stats.argtypes = [V, V]
     for name in ("sparsepr_partition", "sparsepr_permute", "sparsepr_route",
@@ -160,6 +162,15 @@ def sparsepr_route(qp, kp, p, off_q, off_k, csr, k_per_head, ws, stream=None):
     _check(lib.sparsepr_route(_ptr(qp), _ptr(kp), _dtype_code(qp), ctypes.byref(prm), _ptr(off_q),
                               _ptr(off_k), _ptr(csr), _ptr(k_per_head), _ptr(ws), ws.numel(),
                               _stream(stream)), "sparsepr_route")
+
+
+def sparsepr_route_noalloc(qp, kp, p, off_q, off_k, csr, k_per_head, stream=None):
+    """sparsepr_route without a workspace (its scratch is a fixed device array
+    inside the library); for callers that cannot allocate device memory."""
+    prm, keep = make_params(p)
+    _check(lib.sparsepr_route_noalloc(_ptr(qp), _ptr(kp), _dtype_code(qp), ctypes.byref(prm),
+                                      _ptr(off_q), _ptr(off_k), _ptr(csr), _ptr(k_per_head),
+                                      _stream(stream)), "sparsepr_route_noalloc")
 
 
 def sparsepr_block_sparse_attn(qp, kp, vp, p, off_q, off_k, csr, k_per_head, o_sparse,

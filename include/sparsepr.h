@@ -153,6 +153,27 @@ sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt
  * or -1 if the parameters are invalid. */
 int32_t sparsepr_route_width(const sparsepr_params* p);
 
+/* sparsepr_route without a workspace, for callers that cannot allocate
+ * device memory or pass a workspace (code that must not trigger the implicit
+ * device synchronisation of cudaMalloc, or that works inside a memory pool
+ * reserved up front). No counterpart in the paper: it is a memory-management
+ * variant of the routing call above, with the same arguments (minus ws) and
+ * the same outputs.
+ * Its scratch is one fixed 4 MiB device array per GPU, held from the moment
+ * the library is loaded until the process exits; heads are processed in
+ * chunks that fit. A single head needs (Cq + Ck) * d * 8 bytes; larger
+ * parameters are rejected with SPARSEPR_ERR_WORKSPACE before anything is
+ * enqueued. It calls no allocating routine.
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * All calls share the array and the last call's contents stay in it (every
+ * call overwrites what it reads, nothing needs clearing). Calls that overlap
+ * on the GPU race on the array: issue them in order on one stream. */
+sparsepr_status sparsepr_route_noalloc(const void* qp, const void* kp, sparsepr_dtype dt,
+                                       const sparsepr_params* p, const int32_t* off_q,
+                                       const int32_t* off_k, int32_t* csr,
+                                       int32_t* k_per_head, void* stream);
+
 /* Stage 3b [SPR 2.C variable-block sparse attention; SVOO: the softmax is
  * normalised over the kept logits only].
  * For group-major query row i of group g:
