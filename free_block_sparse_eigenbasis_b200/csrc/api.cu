@@ -74,6 +74,30 @@ sparsepr_status cuda_status(cudaError_t e) {
 
 __global__ void set_i32_kernel(int32_t* p, int v) { *p = v; }
 
+constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+AssignTC assign_common(const Ctx& c, void* ws, int32_t* labels, int32_t* flags, int flag_base,
+                       int sms) {
+  AssignTC a = {};
+  a.H = c.p.H;
+  a.n = c.L.Nv;
+  a.labels = labels;
+  a.flags = flags;
+  a.flag_base = flag_base;
+  a.recheck = at<int32_t>(ws, c.L.recheck);
+  a.nrecheck = at<int32_t>(ws, c.L.nrecheck);
+  a.stats = c.stats;
+  a.sm_count = sms;
+  return a;
+}
+
 // Dense-mode routing metadata per head: one query group [0, M), one key
 // group [0, N) kept by it.
 __global__ void dense_meta_kernel(int32_t* meta, int H, int M, int N) {
@@ -176,8 +200,54 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
   const long long hs_z = static_cast<long long>(Nv) * e;
   SPR_TRY(launch_gather_init(z, kXf64, hs_z, e, e, init_k, Ck, H, mu, mun, st));
+  // tensor-core assignment when the centroid planes fit in shared memory
+  const int sms = sm_count();
+  // (a 128-row TMA box needs at least 128 rows in the tensor)
+  const bool tc_keys = assign_tc_smem_bytes(3, 3, L.Dpk, L.CpadK) <= kMaxDynSmem &&
+                       static_cast<size_t>(H) * Nv >= static_cast<size_t>(kTileM);
+  AssignTC ak;
+  if (tc_keys) {
+    __nv_bfloat16* zp = at<__nv_bfloat16>(ws, L.zplanes);
+    const long long zps = static_cast<long long>(H) * Nv * L.Dpk;
+    SPR_TRY(launch_split_rows(z, kXf64, hs_z, e, Nv, e, L.Dpk, 3, H, zp, zps,
+                              at<float>(ws, L.xnk), st));
+    ak = assign_common(c, ws, lab_k, flags, 0, sms);
+    ak.a_planes = zp;
+    ak.a_plane_stride = zps;
+    ak.a_rows_total = static_cast<size_t>(H) * Nv;
+    ak.a_head = Nv;
+    ak.nA = 3;
+    ak.b_planes = at<__nv_bfloat16>(ws, L.muplanes);
+    ak.b_plane_stride = static_cast<long long>(H) * L.CpadK * L.Dpk;
+    ak.nB = 3;
+    ak.Dp = L.Dpk;
+    ak.Cpad = L.CpadK;
+    ak.npairs = 6;
+    const int pk[6] = {0 * 4 + 0, 0 * 4 + 1, 1 * 4 + 0, 0 * 4 + 2, 1 * 4 + 1, 2 * 4 + 0};
+    for (int i = 0; i < 6; ++i) ak.pairs[i] = pk[i];
+    ak.cvals = at<float>(ws, L.cfk);
+    ak.xnorm = at<float>(ws, L.xnk);
+    ak.hmax = at<float>(ws, L.hmk);
+    ak.x_exact = z;
+    ak.x_kind = kXf64;
+    ak.x_hs = hs_z;
+    ak.x_ld = e;
+    ak.D = e;
+    ak.y_exact = mu;
+    ak.c_exact = mun;
+    ak.m = Ck;
+    ak.direct = 1;
+  }
   for (int t = 0; t < iters; ++t) {
-    SPR_TRY(launch_argmin(z, kXf64, hs_z, e, Nv, e, mu, mun, Ck, H, lab_k, flags, 0, st));
+    if (tc_keys) {
+      SPR_TRY(launch_prep_centroids(mu, mun, Ck, e, L.Dpk, L.CpadK, 3, H,
+                                    at<__nv_bfloat16>(ws, L.muplanes),
+                                    static_cast<long long>(H) * L.CpadK * L.Dpk,
+                                    at<float>(ws, L.cfk), at<float>(ws, L.hmk), flags, 0, st));
+      SPR_TRY(launch_argmin_tc(ak, st));
+    } else {
+      SPR_TRY(launch_argmin(z, kXf64, hs_z, e, Nv, e, mu, mun, Ck, H, lab_k, flags, 0, st));
+    }
     SPR_TRY(launch_finalize_pass(H, t, flags, 0, c.stats->key_passes, st));
     if (t + 1 < iters) {
       SPR_TRY(launch_counting_sort(lab_k, H, Nv, Ck, L.nchunk, hist, sperm, soff, flags + 1, 4,
@@ -196,9 +266,55 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
                           static_cast<long long>(d) * d, 0, st));
   // queries: Lloyd passes on logit profiles in the d-space form
   SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
+  // queries on the tensor cores for bf16 inputs (exact in one bf16 plane)
+  int nbq = 0;
+  if (c.bf16 && static_cast<size_t>(H) * N >= static_cast<size_t>(kTileM)) {
+    if (assign_tc_smem_bytes(1, 3, d, L.CpadQ) <= kMaxDynSmem)
+      nbq = 3;
+    else if (assign_tc_smem_bytes(1, 2, d, L.CpadQ) <= kMaxDynSmem)
+      nbq = 2;
+  }
+  AssignTC aq;
+  if (nbq) {
+    SPR_TRY(launch_split_rows(q, c.kind, hs_in, d, Nv, d, d, 0, H, nullptr, 0,
+                              at<float>(ws, L.xnq), st));
+    aq = assign_common(c, ws, lab_q, flags, 2, sms);
+    aq.a_planes = static_cast<const __nv_bfloat16*>(q);
+    aq.a_plane_stride = 0;
+    aq.a_rows_total = static_cast<size_t>(H) * N;
+    aq.a_head = N;
+    aq.nA = 1;
+    aq.b_planes = at<__nv_bfloat16>(ws, L.wplanes);
+    aq.b_plane_stride = static_cast<long long>(H) * L.CpadQ * d;
+    aq.nB = nbq;
+    aq.Dp = d;
+    aq.Cpad = L.CpadQ;
+    aq.npairs = nbq;
+    for (int i = 0; i < 6; ++i) aq.pairs[i] = (i < nbq) ? i : 0;
+    aq.cvals = at<float>(ws, L.cfq);
+    aq.xnorm = at<float>(ws, L.xnq);
+    aq.hmax = at<float>(ws, L.hmq);
+    aq.x_exact = q;
+    aq.x_kind = c.kind;
+    aq.x_hs = hs_in;
+    aq.x_ld = d;
+    aq.D = d;
+    aq.y_exact = wg;
+    aq.c_exact = cg;
+    aq.m = Cq;
+    aq.direct = 0;
+  }
   for (int t = 0; t < iters; ++t) {
     SPR_TRY(launch_query_metric_apply(G, qbar, Cq, H, d, wg, cg, flags + 3, 4, st));
-    SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, st));
+    if (nbq) {
+      SPR_TRY(launch_prep_centroids(wg, cg, Cq, d, d, L.CpadQ, nbq, H,
+                                    at<__nv_bfloat16>(ws, L.wplanes),
+                                    static_cast<long long>(H) * L.CpadQ * d, at<float>(ws, L.cfq),
+                                    at<float>(ws, L.hmq), flags, 2, st));
+      SPR_TRY(launch_argmin_tc(aq, st));
+    } else {
+      SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, st));
+    }
     SPR_TRY(launch_finalize_pass(H, t, flags, 2, c.stats->query_passes, st));
     if (t + 1 < iters) {
       SPR_TRY(launch_counting_sort(lab_q, H, Nv, Cq, L.nchunk, hist, sperm, soff, flags + 3, 4,
@@ -304,6 +420,8 @@ sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const
   a.nwork = at<int32_t>(ws, c.L.nwork);
   a.tiles_per_head = c.L.tiles_per_head;
   a.nslots = at<int32_t>(ws, c.L.nslots);
+  a.runs = at<int2>(ws, c.L.runs);
+  a.nruns = at<int32_t>(ws, c.L.nruns);
   a.pairs = pairs_sparse;
   a.stats = c.stats;
   SPR_TRY(launch_block_sparse_attn(a, c.st));
@@ -365,6 +483,8 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     a.nwork = at<int32_t>(ws, L.pnwork);
     a.tiles_per_head = M / kTileM + 2;
     a.nslots = meta + 6 * H;
+    a.nruns = meta + 7 * H;
+    a.runs = reinterpret_cast<int2*>(meta + 8 * H);
     a.pairs = nullptr;
     a.stats = c.stats;
     SPR_TRY(launch_block_sparse_attn(a, st));

@@ -1,0 +1,529 @@
+// Nearest-centroid assignment of the k-means passes of "Partition the Support,
+// Reconstruct the Residual" (2.A) on the 5th-generation tensor cores, with a
+// certified error bound so that the labels equal those of exact fp64
+// arithmetic.
+//
+// For rows x_i and centroid-side vectors y_j with offsets c_j, the label is
+// argmin_j d_ij, d_ij = c_j - 2 x_i . y_j (lowest j on ties):
+//   keys:    x = z (response coordinates), y = mu, c = |mu|^2
+//   queries: x = q, y = G qbar, c = qbar^T G qbar   (d-space profile form)
+// x and y are split into bf16 planes (x = x1 + x2 + x3 + r, |r| <= 2^-24 |x|);
+// the plane products x_a . y_b with a + b <= 4 (planes counted from 0) are
+// summed by tcgen05.mma in fp32. With K_t accumulated terms per dot product
+// the computed d'_ij satisfies
+//   |d'_ij - d_ij| <= E_i = (K_t 2^-22 + 2^-20) |x_i| Y + 2^-22 (C + 2 |x_i| Y),
+// Y = max_j |y_j|, C = max_j |c_j| (a generous bound: products of bf16 values
+// are exact in fp32, each accumulation step loses at most 2^-23 relative).
+// A row whose best and second-best d' differ by more than 2 E_i has a
+// certain label; every other row is appended to a list and decided again in
+// fp64 by recheck_kernel.
+//
+// One persistent CTA per (slice of row tiles, head): all centroid planes stay
+// in shared memory, row tiles of 128 stream through a 2-stage TMA ring, and
+// the 128 x (<=256) accumulator of each centroid chunk alternates between two
+// TMEM buffers so that the epilogue of one chunk overlaps the MMAs of the next.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+namespace {
+
+constexpr int kAsThreads = 160;  // warps 0-3 epilogue (thread = row), warp 4: TMA + MMA
+constexpr int kAsChunk = 256;    // centroids per accumulator chunk
+constexpr uint32_t kAsTmemCols = 512;
+
+struct AsBars {
+  uint64_t b_full;
+  uint64_t a_full[2], a_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_idle;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct AsMaps {
+  CUtensorMap a[3];  // row planes, box (inner, 128 rows)
+  CUtensorMap b[3];  // centroid planes, box (inner, 16 rows)
+};
+
+struct AsParams {
+  int n;          // rows per head
+  int a_head;     // row offset between heads in the A maps
+  int b_head;     // row offset between heads in the B maps (= Cpad)
+  int Cpad;       // centroids per head, padded to a multiple of 32
+  int nA, nB;     // planes
+  int npairs;
+  int pairs[6];   // (plane of x) * 4 + (plane of y)
+  int sw32;       // 1: 32-byte rows (D = 16), 0: 128-byte swizzle atoms (D = 64 * atoms)
+  int atoms;      // 64-column atoms (sw32: 1)
+  int Kt;         // accumulated terms per dot product
+  float res;      // bound on the plane-split residual and dropped plane products, relative
+  int tiles_per_head;
+  const float* cvals;  // [H, Cpad] fp32 offsets (+inf on padding)
+  const float* xnorm;  // [H, n] |x_i| (rounded up)
+  const float* hmax;   // [H, 2] Y, C (rounded up)
+  int32_t* labels;     // [H, n]
+  int32_t* flags;      // [H, 4]; changes counter at flag_base, done flag at flag_base + 1
+  int flag_base;
+  int32_t* recheck;    // [H, n] rows to decide in fp64
+  int32_t* nrecheck;   // [H]
+  DeviceStats* stats;
+};
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, bool sw32) {
+  // K-major canonical layouts: LBO = 16 bytes (unused), SBO = stride of 8-row groups
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>((sw32 ? 256u : 1024u) >> 4) << 32;
+  d |= 1ull << 46;
+  d |= (sw32 ? 6ull : 2ull) << 61;
+  return d;
+}
+
+__global__ void __launch_bounds__(kAsThreads, 1)
+    argmin_tc_kernel(const __grid_constant__ AsMaps maps, const AsParams p) {
+  const int h = blockIdx.y;
+  int32_t* fl = p.flags + h * 4;
+  if (fl[p.flag_base + 1]) return;  // converged head
+  const int row_bytes = p.sw32 ? 32 : 128;
+  const int slab_a = kTileM * row_bytes;                // one atom of a 128-row tile
+  const int a_stage = p.nA * p.atoms * slab_a;
+  const int slab_b = p.Cpad * row_bytes;                // one atom of all centroids
+  const int b_bytes = p.nB * p.atoms * slab_b;
+  const int nchunks = (p.Cpad + kAsChunk - 1) / kAsChunk;
+
+  extern __shared__ uint8_t as_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(as_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint8_t* Bs = sm;
+  uint8_t* As = sm + ((b_bytes + 1023) & ~1023);
+  float* cs = reinterpret_cast<float*>(As + 2 * a_stage);
+  AsBars* bars = reinterpret_cast<AsBars*>(cs + p.Cpad);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->b_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->a_full[s], 1);
+      mbar_init(&bars->a_empty[s], 1);
+      mbar_init(&bars->acc_full[s], 1);
+      mbar_init(&bars->acc_empty[s], kTileM);
+    }
+    mbar_init(&bars->mma_idle, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  for (int j = threadIdx.x; j < p.Cpad; j += blockDim.x)
+    cs[j] = p.cvals[static_cast<size_t>(h) * p.Cpad + j];
+  if (warp == 0) {
+    tmem_alloc(&bars->tmem_base, kAsTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+  // this CTA's row tiles: t = blockIdx.x + u * gridDim.x
+  const int ntile = (p.tiles_per_head - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                    static_cast<int>(gridDim.x);
+  const int inner = p.sw32 ? 16 : 64;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ----------------------------- TMA producer -----------------------------
+      mbar_arrive_expect_tx(&bars->b_full, b_bytes);
+      for (int pl = 0; pl < p.nB; ++pl)
+        for (int a = 0; a < p.atoms; ++a)
+          for (int r = 0; r < p.Cpad; r += 16)
+            tma_load_2d(Bs + (pl * p.atoms + a) * slab_b + r * row_bytes, &maps.b[pl],
+                        &bars->b_full, a * inner, h * p.b_head + r);
+      int issued = -1;
+      bool ok = true;
+      for (int u = 0; u < ntile; ++u) {
+        const int s = u & 1;
+        if (u >= 2 && !mbar_wait(&bars->a_empty[s], ((u - 2) >> 1) & 1, abort)) { ok = false; break; }
+        const int t = blockIdx.x + u * gridDim.x;
+        mbar_arrive_expect_tx(&bars->a_full[s], a_stage);
+        for (int pl = 0; pl < p.nA; ++pl)
+          for (int a = 0; a < p.atoms; ++a)
+            tma_load_2d(As + s * a_stage + (pl * p.atoms + a) * slab_a, &maps.a[pl],
+                        &bars->a_full[s], a * inner, h * p.a_head + t * kTileM);
+        issued = u;
+      }
+      volatile int never = 0;
+      if (!ok)
+        for (int u = max(0, issued - 1); u <= issued; ++u)
+          mbar_wait(&bars->a_full[u & 1], (u >> 1) & 1, &never);
+      mbar_wait(&bars->b_full, 0, &never);
+    } else if (lane == 1) {
+      // ------------------------------ MMA issuer ------------------------------
+      bool ok = mbar_wait(&bars->b_full, 0, abort);
+      const uint32_t a_addr = smem_u32(As), b_addr = smem_u32(Bs);
+      int gc = 0;
+      for (int u = 0; u < ntile && ok; ++u) {
+        const int s = u & 1;
+        if (!mbar_wait(&bars->a_full[s], (u >> 1) & 1, abort)) { ok = false; break; }
+        for (int c = 0; c < nchunks; ++c, ++gc) {
+          const int buf = gc & 1;
+          if (gc >= 2 && !mbar_wait(&bars->acc_empty[buf], ((gc - 2) >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
+          const uint32_t idesc = idesc_bf16(kTileM, N, 0);
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * kAsChunk);
+          int first = 1;
+          for (int pi = 0; pi < p.npairs; ++pi) {
+            const int pa = p.pairs[pi] >> 2, pb = p.pairs[pi] & 3;
+            const int ksteps = p.sw32 ? 1 : p.atoms * 4;
+            for (int ks = 0; ks < ksteps; ++ks) {
+              const int atom = p.sw32 ? 0 : (ks >> 2);
+              const uint32_t koff = p.sw32 ? 0u : static_cast<uint32_t>((ks & 3) * 32);
+              const uint32_t aa = a_addr + s * a_stage + (pa * p.atoms + atom) * slab_a + koff;
+              const uint32_t ba = b_addr + (pb * p.atoms + atom) * slab_b +
+                                  c * kAsChunk * row_bytes + koff;
+              mma_bf16_ss(d_tmem, smem_desc(aa, p.sw32), smem_desc(ba, p.sw32), idesc,
+                          first ? 0u : 1u);
+              first = 0;
+            }
+          }
+          mma_commit(&bars->acc_full[buf]);
+        }
+        mma_commit(&bars->a_empty[s]);
+      }
+      // all MMAs issued by this thread complete before tensor memory is freed
+      mma_commit(&bars->mma_idle);
+      volatile int never = 0;
+      mbar_wait(&bars->mma_idle, 0, &never);
+    }
+  } else {
+    // --------------------------- epilogue (thread = row) ---------------------------
+    const int r = threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>((warp * 32) << 16);
+    const float Y = p.hmax[h * 2 + 0], C = p.hmax[h * 2 + 1];
+    const float kt_term = static_cast<float>(p.Kt) * 2.384185791015625e-07f + p.res;
+    int gc = 0;
+    bool ok = true;
+    for (int u = 0; u < ntile && ok; ++u) {
+      const int t = blockIdx.x + u * gridDim.x;
+      const int row = t * kTileM + r;
+      float d1 = INFINITY, d2 = INFINITY;
+      int i1 = 0x7fffffff;
+      for (int c = 0; c < nchunks; ++c, ++gc) {
+        const int buf = gc & 1;
+        if (!mbar_wait(&bars->acc_full[buf], (gc >> 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
+        const uint32_t base = tmem + lane_base + static_cast<uint32_t>(buf * kAsChunk);
+        for (int c32 = 0; c32 < N; c32 += 32) {
+          uint32_t v[32];
+          const int w = min(32, N - c32);  // 32, or 16 for the last group
+          if (w == 32)
+            tmem_ld32(base + c32, v);
+          else
+            tmem_ld16(base + c32, *reinterpret_cast<uint32_t(*)[16]>(v));
+          tmem_wait_ld();
+          const int j0 = c * kAsChunk + c32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i >= w) break;
+            const float dd = fmaf(-2.f, __uint_as_float(v[i]), cs[j0 + i]);
+            if (dd < d1) {
+              d2 = d1;
+              d1 = dd;
+              i1 = j0 + i;
+            } else if (dd < d2) {
+              d2 = dd;
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->acc_empty[buf]);
+      }
+      if (!ok || row >= p.n) continue;
+      const float xn = p.xnorm[static_cast<size_t>(h) * p.n + row];
+      const float xy = xn * Y;
+      const float E = kt_term * xy + 2.384185791015625e-07f * (C + 2.f * xy);
+      const size_t li = static_cast<size_t>(h) * p.n + row;
+      if (d2 - d1 > 2.f * E) {
+        if (p.labels[li] != i1) atomicAdd(&fl[p.flag_base], 1);
+        p.labels[li] = i1;
+      } else {
+        const int k = atomicAdd(&p.nrecheck[h], 1);
+        p.recheck[static_cast<size_t>(h) * p.n + k] = row;
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort && threadIdx.x == 0) raise_status(p.stats, SPARSEPR_ERR_TIMEOUT);
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kAsTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fp64 decision of the flagged rows: one warp per row, lanes over centroids.
+// direct = 1: d = sum_t (x_t - y_jt)^2; else d = c_j - 2 x . y_j.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
+  if (kind == kXf64) return static_cast<const double*>(X)[i];
+  if (kind == kXbf16) return static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(X)[i]));
+  return static_cast<double>(static_cast<const float*>(X)[i]);
+}
+
+__global__ void recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
+                               const double* Y, const double* c, int m, int direct,
+                               int32_t* labels, int32_t* flags, int flag_base,
+                               const int32_t* recheck, const int32_t* nrecheck) {
+  const int h = blockIdx.y;
+  int32_t* fl = flags + h * 4;
+  if (fl[flag_base + 1]) return;
+  const int cnt = nrecheck[h];
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const double* Yh = Y + static_cast<size_t>(h) * m * D;
+  for (int w = blockIdx.x * wpb + (threadIdx.x >> 5); w < cnt; w += gridDim.x * wpb) {
+    const int row = recheck[static_cast<size_t>(h) * n + w];
+    const size_t xb = h * hsx + static_cast<size_t>(row) * ldx_;
+    double best = INFINITY;
+    int bi = 0x7fffffff;
+    for (int j = lane; j < m; j += 32) {
+      double dd;
+      if (direct) {
+        dd = 0.0;
+        for (int t = 0; t < D; ++t) {
+          const double diff = ldx(X, kind, xb + t) - Yh[static_cast<size_t>(j) * D + t];
+          dd = fma(diff, diff, dd);
+        }
+      } else {
+        double s = 0.0;
+        for (int t = 0; t < D; ++t) s = fma(ldx(X, kind, xb + t), Yh[static_cast<size_t>(j) * D + t], s);
+        dd = c[static_cast<size_t>(h) * m + j] - 2.0 * s;
+      }
+      if (dd < best) {
+        best = dd;
+        bi = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob < best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      const size_t li = static_cast<size_t>(h) * n + row;
+      if (labels[li] != bi) atomicAdd(&fl[flag_base], 1);
+      labels[li] = bi;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Operand preparation.
+// ---------------------------------------------------------------------------
+// Split rows of fp64 X (or widen bf16 / fp32 X) into P bf16 planes of Dp
+// columns (zero padded); norm[row] = |x| rounded up.
+__global__ void split_rows_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
+                                  int Dp, int P, __nv_bfloat16* planes, long long plane_stride,
+                                  float* norms) {
+  const int h = blockIdx.y;
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n) return;
+  const size_t xb = h * hsx + static_cast<size_t>(row) * ldx_;
+  const size_t ob = (static_cast<size_t>(h) * n + row) * Dp;
+  double ss = 0.0;
+  for (int t = lane; t < Dp; t += 32) {
+    double v = (t < D) ? ldx(X, kind, xb + t) : 0.0;
+    ss = fma(v, v, ss);
+    for (int pl = 0; pl < P; ++pl) {
+      const __nv_bfloat16 b = __double2bfloat16(v);
+      planes[pl * plane_stride + ob + t] = b;
+      v -= static_cast<double>(__bfloat162float(b));
+    }
+  }
+  ss = warp_sum_f64(ss);
+  if (norms && lane == 0)
+    norms[static_cast<size_t>(h) * n + row] = static_cast<float>(sqrt(ss) * (1.0 + 1e-6));
+}
+
+// Centroid side: planes of y (padded to Cpad rows with zeros), fp32 offsets
+// (+inf on padding), and the per-head maxima Y = max |y_j|, C = max |c_j|.
+__global__ void prep_centroids_kernel(const double* Yv, const double* cv, int m, int D, int Dp,
+                                      int Cpad, int P, __nv_bfloat16* planes,
+                                      long long plane_stride, float* cf, float* hmax,
+                                      const int32_t* flags, int flag_base) {
+  __shared__ double ym[32], cm[32];
+  const int h = blockIdx.x;
+  if (flags && flags[h * 4 + flag_base + 1]) return;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  double ymax = 0.0, cmax = 0.0;
+  for (int j = wid; j < Cpad; j += nw) {
+    const size_t ob = (static_cast<size_t>(h) * Cpad + j) * Dp;
+    double ss = 0.0;
+    for (int t = lane; t < Dp; t += 32) {
+      double v = (j < m && t < D) ? Yv[(static_cast<size_t>(h) * m + j) * D + t] : 0.0;
+      ss = fma(v, v, ss);
+      for (int pl = 0; pl < P; ++pl) {
+        const __nv_bfloat16 b = __double2bfloat16(v);
+        planes[pl * plane_stride + ob + t] = b;
+        v -= static_cast<double>(__bfloat162float(b));
+      }
+    }
+    ss = warp_sum_f64(ss);
+    if (lane == 0) {
+      if (j < m) {
+        const double cj = cv[static_cast<size_t>(h) * m + j];
+        cf[static_cast<size_t>(h) * Cpad + j] = static_cast<float>(cj);
+        ymax = fmax(ymax, sqrt(ss));
+        cmax = fmax(cmax, fabs(cj));
+      } else {
+        cf[static_cast<size_t>(h) * Cpad + j] = INFINITY;
+      }
+    }
+  }
+  if (lane == 0) {
+    ym[wid] = ymax;
+    cm[wid] = cmax;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < nw; ++w) {
+      ymax = fmax(ymax, ym[w]);
+      cmax = fmax(cmax, cm[w]);
+    }
+    hmax[h * 2 + 0] = static_cast<float>(ymax * (1.0 + 1e-6));
+    hmax[h * 2 + 1] = static_cast<float>(cmax * (1.0 + 1e-6));
+  }
+}
+
+__global__ void zero_counts_kernel(int32_t* p, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = 0;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool plane_map(CUtensorMap* m, const void* base, size_t rows, int Dp, bool sw32, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(Dp), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(Dp) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(sw32 ? 16 : 64),
+                       static_cast<cuuint32_t>(rows < static_cast<size_t>(box_rows) ? rows : box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             sw32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t assign_tc_smem_bytes(int nA, int nB, int Dp, int Cpad) {
+  const bool sw32 = (Dp == 16);
+  const int row_bytes = sw32 ? 32 : 128;
+  const int atoms = sw32 ? 1 : Dp / 64;
+  const size_t b = static_cast<size_t>(nB) * atoms * Cpad * row_bytes;
+  const size_t a = static_cast<size_t>(nA) * atoms * kTileM * row_bytes;
+  return 1024 + ((b + 1023) & ~static_cast<size_t>(1023)) + 2 * a + static_cast<size_t>(Cpad) * 4 +
+         sizeof(AsBars);
+}
+
+cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, int n, int D,
+                              int Dp, int P, int H, __nv_bfloat16* planes, long long plane_stride,
+                              float* norms, cudaStream_t st) {
+  dim3 grid((n + 7) / 8, H);
+  split_rows_kernel<<<grid, 256, 0, st>>>(X, kind, hsx, ldx, n, D, Dp, P, planes, plane_stride,
+                                          norms);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_centroids(const double* Y, const double* c, int m, int D, int Dp,
+                                  int Cpad, int P, int H, __nv_bfloat16* planes,
+                                  long long plane_stride, float* cf, float* hmax,
+                                  const int32_t* flags, int flag_base, cudaStream_t st) {
+  prep_centroids_kernel<<<H, 512, 0, st>>>(Y, c, m, D, Dp, Cpad, P, planes, plane_stride, cf, hmax,
+                                           flags, flag_base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
+  const bool sw32 = (a.Dp == 16);
+  AsMaps maps;
+  for (int pl = 0; pl < 3; ++pl) {
+    const int ia = pl < a.nA ? pl : 0, ib = pl < a.nB ? pl : 0;
+    if (!plane_map(&maps.a[pl], a.a_planes + ia * a.a_plane_stride, a.a_rows_total, a.Dp, sw32,
+                   kTileM) ||
+        !plane_map(&maps.b[pl], a.b_planes + ib * a.b_plane_stride,
+                   static_cast<size_t>(a.H) * a.Cpad, a.Dp, sw32, 16))
+      return cudaErrorInvalidValue;
+  }
+  AsParams p;
+  p.n = a.n;
+  p.a_head = a.a_head;
+  p.b_head = a.Cpad;
+  p.Cpad = a.Cpad;
+  p.nA = a.nA;
+  p.nB = a.nB;
+  p.npairs = a.npairs;
+  for (int i = 0; i < 6; ++i) p.pairs[i] = a.pairs[i];
+  p.sw32 = sw32 ? 1 : 0;
+  p.atoms = sw32 ? 1 : a.Dp / 64;
+  p.Kt = a.npairs * a.Dp;
+  // 3 planes: residual <= 2^-24 per side, dropped products <= 2^-23 (bound 2^-20);
+  // 2 planes of y: residual <= 2^-16 (bound 2^-14)
+  p.res = (a.nB >= 3) ? 9.5367431640625e-07f : 6.103515625e-05f;
+  p.tiles_per_head = (a.n + kTileM - 1) / kTileM;
+  p.cvals = a.cvals;
+  p.xnorm = a.xnorm;
+  p.hmax = a.hmax;
+  p.labels = a.labels;
+  p.flags = a.flags;
+  p.flag_base = a.flag_base;
+  p.recheck = a.recheck;
+  p.nrecheck = a.nrecheck;
+  p.stats = a.stats;
+  zero_counts_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.nrecheck, a.H);
+  const size_t shb = assign_tc_smem_bytes(a.nA, a.nB, a.Dp, a.Cpad);
+  cudaError_t e = cudaFuncSetAttribute(argmin_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(shb));
+  if (e != cudaSuccess) return e;
+  int ctas = (a.sm_count + a.H - 1) / a.H;
+  if (ctas > p.tiles_per_head) ctas = p.tiles_per_head;
+  if (ctas < 1) ctas = 1;
+  argmin_tc_kernel<<<dim3(ctas, a.H), kAsThreads, shb, st>>>(maps, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  recheck_kernel<<<dim3(64, a.H), 256, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
+                                                a.y_exact, a.c_exact, a.m, a.direct, a.labels,
+                                                a.flags, a.flag_base, a.recheck, a.nrecheck);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -5,19 +5,26 @@
 //
 // One CTA computes one 128-row query tile of one query group. The key side
 // is the union of the kept key groups' contiguous ranges in the group-major
-// K/V; runs of adjacent kept groups are merged and cut into 8-row slots,
-// 16 slots per 128-key tile, each slot fetched by TMA at an arbitrary row.
-// Rows of a slot past its run's end are masked to -inf, so skipped key
-// groups are never multiplied (only the tail padding of a run is).
+// K/V; runs of adjacent kept groups are merged (once per query group, by the
+// slot-count kernel) and cut into 8-row slots, 16 slots per 128-key tile,
+// each slot fetched by TMA at an arbitrary row. Rows of a slot past its
+// run's end are masked to -inf, so skipped key groups are never multiplied
+// (only the tail padding of a run is).
 //
 // Roles (192 threads): warps 0-3 own one query row per thread (TMEM lane =
-// row) and run the online softmax and the epilogue; warp 4 lane 0 issues TMA
-// loads; warp 5 lane 0 issues tcgen05.mma. S = Q K^T goes to one of two TMEM
-// buffers (S(j+1) runs while the softmax of tile j works), P is written bf16
-// to shared memory in the 128B-swizzled K-major layout, and O += P V
-// accumulates in TMEM. O is rescaled only when a row maximum grows by more
-// than 2^8; O and the row sum always share one reference maximum, so the
-// result is exact.
+// row) and run the online softmax and the epilogue; warp 4 lanes 0 and 1
+// stream Q+K and V with TMA (each contiguous piece of slots as power-of-two
+// boxes of 8..128 rows); warp 5 lane 0 issues tcgen05.mma.
+//   * S = Q K^T goes to one of two TMEM buffers, so S(j+1) runs on the
+//     tensor cores while the softmax of tile j works;
+//   * P is written bf16 to one of two shared-memory buffers (128B-swizzled,
+//     K-major), so the softmax of tile j+1 overlaps P(j) V(j);
+//   * O += P V accumulates in TMEM. O is rescaled only when a row maximum
+//     grows by more than 2^8; O and the row sum always share one reference
+//     maximum, so the result is exact.
+// Every mbarrier wait is bounded; a wait that runs out marks the status word
+// and the CTA drains its in-flight copies and MMAs, frees tensor memory and
+// returns.
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,8 +33,9 @@ namespace {
 
 constexpr int kStages = 2;
 constexpr int kSlotsPerTile = kTileN / kSlotRows;  // 16
-constexpr int kAttnThreads = 192;
-constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256, 256+d)
+constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256, 256+d), exchange [480,512)
+constexpr uint32_t kXchCol = 480;    // row-max / row-sum exchange between the two halves of a row
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -41,50 +49,47 @@ struct Smem {
   static constexpr int q_off = 0;
   static constexpr int k_off = q_off + kQBytes;
   static constexpr int v_off = k_off + kStages * kKVBytes;
-  static constexpr int p_off = v_off + kStages * kKVBytes;
-  static constexpr int bar_off = p_off + kPBytes;
+  static constexpr int p_off = v_off + kStages * kKVBytes;  // two P buffers
+  static constexpr int bar_off = p_off + 2 * kPBytes;
+  static constexpr int runs_off = bar_off + 256;
 };
-// Dynamic shared memory requested: the d=128 footprint for both head dims, so
-// that one CTA holds an SM (each CTA allocates 512 TMEM columns), plus
-// 1024 bytes of alignment slack.
-constexpr int kAttnSmemBytes = Smem<128>::bar_off + 256 + 1024;
+// Dynamic shared memory: the d=128 footprint for both head dims (one CTA per
+// SM; each CTA allocates 512 TMEM columns), the barrier block, a run list of
+// up to kSmemRuns entries, and 1024 bytes of alignment slack.
+constexpr int kSmemRuns = 96;
+constexpr int kAttnSmemBytes = Smem<128>::runs_off + kSmemRuns * 8 + 1024;
 static_assert(kAttnSmemBytes <= 232448, "shared memory");
 
 struct Bars {
   uint64_t q_full;
   uint64_t kfull[kStages], vfull[kStages], kempty[kStages], vempty[kStages];
   uint64_t s_full[2];
-  uint64_t p_full, pv_done, mma_idle;
+  uint64_t p_full[2], pv_done[2];
+  uint64_t mma_idle;
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// Walks the kept key groups of one query group in ascending order, merging
-// adjacent ranges, and hands out 8-row slots (start row, valid rows).
+// Walks the merged key runs of one query group in ascending order and hands
+// out 8-row slots (start row, valid rows).
 struct SlotIter {
-  const int32_t* csr;
-  const int32_t* offk;
-  int k, ci, pos, end;
-  __device__ void init(const int32_t* c, const int32_t* o, int kk) {
-    csr = c;
-    offk = o;
-    k = kk;
-    ci = -1;
+  const int2* runs;
+  int nruns, ri, pos, end;
+  __device__ void init(const int2* r, int n) {
+    runs = r;
+    nruns = n;
+    ri = -1;
     pos = 0;
     end = 0;
   }
   __device__ bool next(int& start, int& valid) {
     while (pos >= end) {
-      ++ci;
-      if (ci >= k) return false;
-      const int c = csr[ci];
-      pos = offk[c];
-      end = offk[c + 1];
-      while (ci + 1 < k && offk[csr[ci + 1]] == end) {
-        ++ci;
-        end = offk[csr[ci] + 1];
-      }
+      ++ri;
+      if (ri >= nruns) return false;
+      const int2 rr = runs[ri];
+      pos = rr.x;
+      end = rr.x + rr.y;
     }
     start = pos;
     valid = min(kSlotRows, end - pos);
@@ -93,21 +98,45 @@ struct SlotIter {
   }
 };
 
+// TMA maps: Q (64-column x 128-row boxes) and K / V with boxes of 8, 16, 32,
+// 64 and 128 rows (index = log2(rows / 8)).
+struct AttnMaps {
+  CUtensorMap q;
+  CUtensorMap k[5];
+  CUtensorMap v[5];
+};
+
 struct AttnParams {
-  int H, N, q_rows, Cq, Ck, kmax;
+  int H, N, q_rows, Cq, kmax;
   const int32_t* off_q;   // [H, Cq+1]
-  const int32_t* off_k;   // [H, Ck+1]
-  const int32_t* csr;     // [H, Cq, kmax]
-  const int32_t* kh;      // [H]
   const int32_t* work;    // [H, tiles_per_head]
   const int32_t* nwork;   // [H]
   const int32_t* nslots;  // [H, Cq]
+  const int2* runs;       // [H, Cq, kmax] merged key runs (start, length)
+  const int32_t* nruns;   // [H, Cq]
   int tiles_per_head;
   int q_box_rows;  // rows of one Q TMA box (128, fewer for tiny tensors)
-  float sc;  // scale * log2(e)
+  int max_lg;      // largest K/V box used: 8 << max_lg rows (<= rows of the tensor)
+  float sc;        // scale * log2(e)
   float* out;
   DeviceStats* stats;
 };
+
+// The two warps that share a lane quarter (w and w+4) swap one float per
+// row: each stores its value in tensor-memory column base + half, then reads
+// the partner's column. Buffers alternate between calls, so one barrier per
+// call suffices (a column is rewritten only after the partner passed the
+// next barrier, i.e. after it read the old value).
+__device__ __forceinline__ float exchange_pair(uint32_t col_base, int half, int quarter, float v) {
+  tmem_st1(col_base + half, __float_as_uint(v));
+  tmem_wait_st();
+  tc_fence_before();
+  named_barrier_sync(1 + quarter, 64);
+  tc_fence_after();
+  const uint32_t o = tmem_ld1(col_base + (half ^ 1));
+  tmem_wait_ld();
+  return __uint_as_float(o);
+}
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   // byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128B-swizzled slab
@@ -116,9 +145,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 
 template <int HD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
-                       const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    sparse_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using L = Smem<HD>;
   constexpr int kAtoms = HD / 64;
   const int h = blockIdx.y;
@@ -126,13 +153,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int wcode = p.work[static_cast<size_t>(h) * p.tiles_per_head + blockIdx.x];
   const int g = wcode >> 16, tq = wcode & 0xFFFF;
   const int32_t* offq = p.off_q + static_cast<size_t>(h) * (p.Cq + 1);
-  const int32_t* offk = p.off_k + static_cast<size_t>(h) * (p.Ck + 1);
   const int row0 = offq[g] + tq * kTileM;
   const int rows_valid = min(kTileM, offq[g + 1] - row0);
-  const int ns = p.nslots[static_cast<size_t>(h) * p.Cq + g];
+  const size_t gi = static_cast<size_t>(h) * p.Cq + g;
+  const int ns = p.nslots[gi];
   const int T = (ns + kSlotsPerTile - 1) / kSlotsPerTile;
-  const int kk = p.kh[h];
-  const int32_t* csr_row = p.csr + (static_cast<size_t>(h) * p.Cq + g) * p.kmax;
+  const int nr = p.nruns[gi];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (T == 0) {
@@ -152,6 +178,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* Vs = smem + L::v_off;
   uint8_t* Ps = smem + L::p_off;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::bar_off);
+  int2* runs_s = reinterpret_cast<int2*>(smem + L::runs_off);
+  // run-list capacity left in the dynamic allocation after alignment
+  const int cap = (kAttnSmemBytes - static_cast<int>(smem - smem_raw) - L::runs_off) / 8;
+  const int2* runs_g = p.runs + gi * p.kmax;
+  const bool runs_in_smem = nr <= cap;
+  const int2* runs = runs_in_smem ? runs_s : runs_g;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -161,14 +193,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars->kempty[s], 1);
       mbar_init(&bars->vempty[s], 1);
     }
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_full, kTileM);
-    mbar_init(&bars->pv_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->p_full[b], 2 * kTileM);
+      mbar_init(&bars->pv_done[b], 1);
+    }
     mbar_init(&bars->mma_idle, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
+  if (runs_in_smem)
+    for (int i = threadIdx.x; i < nr; i += blockDim.x) runs_s[i] = runs_g[i];
   if (warp == 0) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -179,56 +214,73 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
 
-  if (warp == 4) {
-    // ------------------------------ TMA producer ------------------------------
-    if (lane == 0) {
+  if (warp == 8) {
+    // --------------- TMA producers: lane 0 streams Q and K, lane 1 V ---------------
+    if (lane < 2) {
+      const bool is_k = (lane == 0);
       const int krow_base = h * p.N;
-      mbar_arrive_expect_tx(&bars->q_full, kAtoms * p.q_box_rows * 128);
-      for (int a = 0; a < kAtoms; ++a)
-        tma_load_2d(Qs + a * L::kSlab, &tmQ, &bars->q_full, a * 64, h * p.q_rows + row0);
+      if (is_k) {
+        mbar_arrive_expect_tx(&bars->q_full, kAtoms * p.q_box_rows * 128);
+        for (int a = 0; a < kAtoms; ++a)
+          tma_load_2d(Qs + a * L::kSlab, &maps.q, &bars->q_full, a * 64, h * p.q_rows + row0);
+      }
+      const CUtensorMap* bm = is_k ? maps.k : maps.v;
+      uint8_t* base = is_k ? Ks : Vs;
+      uint64_t* full = is_k ? bars->kfull : bars->vfull;
+      uint64_t* empty = is_k ? bars->kempty : bars->vempty;
       SlotIter it;
-      it.init(csr_row, offk, kk);
-      int issued_k = -1, issued_v = -1;
+      it.init(runs, nr);
+      int issued = -1;
       bool ok = true;
-      for (int j = 0; j < T && ok; ++j) {
+      for (int j = 0; j < T; ++j) {
         const int st = j % kStages;
-        const uint32_t par = ((j / kStages) + 1) & 1;  // phase of tile j - kStages
-        int starts[kSlotsPerTile];
-#pragma unroll
-        for (int s = 0; s < kSlotsPerTile; ++s) {
-          int st0 = 0, vv = 0;
-          if (!it.next(st0, vv)) st0 = 0;
-          starts[s] = st0;
+        if (j >= kStages && !mbar_wait(&empty[st], ((j / kStages) + 1) & 1, abort)) {
+          ok = false;
+          break;
         }
-        if (j >= kStages && !mbar_wait(&bars->kempty[st], par, abort)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars->kfull[st], L::kKVBytes);
-        uint8_t* kd = Ks + st * L::kKVBytes;
-        for (int s = 0; s < kSlotsPerTile; ++s)
-          for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(kd + a * L::kSlab + s * 1024, &tmK, &bars->kfull[st], a * 64,
-                        krow_base + starts[s]);
-        issued_k = j;
-        if (j >= kStages && !mbar_wait(&bars->vempty[st], par, abort)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars->vfull[st], L::kKVBytes);
-        uint8_t* vd = Vs + st * L::kKVBytes;
-        for (int s = 0; s < kSlotsPerTile; ++s)
-          for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(vd + a * L::kSlab + s * 1024, &tmV, &bars->vfull[st], a * 64,
-                        krow_base + starts[s]);
-        issued_v = j;
+        mbar_arrive_expect_tx(&full[st], L::kKVBytes);
+        uint8_t* dst = base + st * L::kKVBytes;
+        // contiguous pieces of consecutive slots, each loaded as power-of-two boxes
+        int s = 0;
+        while (s < kSlotsPerTile) {
+          int r0 = 0, vv = 0;
+          if (!it.next(r0, vv)) r0 = 0;  // past the last run: any valid rows (masked)
+          int n = 1;
+          int la = r0, lv = 0;
+          while (s + n < kSlotsPerTile) {
+            SlotIter peek = it;
+            if (!peek.next(la, lv)) la = -1;
+            if (la != r0 + kSlotRows * n) break;
+            it = peek;
+            ++n;
+          }
+          int t = s, r = r0, m = n;
+#pragma unroll 1
+          for (int lg = p.max_lg; lg >= 0; --lg) {
+            const int sz = 1 << lg;
+            while (m >= sz) {
+#pragma unroll
+              for (int a = 0; a < kAtoms; ++a)
+                tma_load_2d(dst + a * L::kSlab + t * 1024, &bm[lg], &full[st], a * 64,
+                            krow_base + r);
+              t += sz;
+              r += sz * kSlotRows;
+              m -= sz;
+            }
+          }
+          s += n;
+        }
+        issued = j;
       }
       if (!ok) {
         // let the loads already in flight land before the CTA exits
         volatile int never = 0;
-        for (int j = max(0, issued_k - kStages + 1); j <= issued_k; ++j)
-          mbar_wait(&bars->kfull[j % kStages], (j / kStages) & 1, &never);
-        for (int j = max(0, issued_v - kStages + 1); j <= issued_v; ++j)
-          mbar_wait(&bars->vfull[j % kStages], (j / kStages) & 1, &never);
-        volatile int never2 = 0;
-        mbar_wait(&bars->q_full, 0, &never2);
+        for (int j = max(0, issued - kStages + 1); j <= issued; ++j)
+          mbar_wait(&full[j % kStages], (j / kStages) & 1, &never);
+        if (is_k) mbar_wait(&bars->q_full, 0, &never);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileM, kTileN, 0);
@@ -262,20 +314,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           issue_s(j + 1);
         }
         const int st = j % kStages;
-        if (!mbar_wait(&bars->p_full, j & 1, abort)) { ok = false; break; }
+        if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort)) { ok = false; break; }
         if (!mbar_wait(&bars->vfull[st], (j / kStages) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t o_tmem = tmem + 2u * kTileN;
+        const uint32_t pb = p_addr + static_cast<uint32_t>((j & 1) * L::kPBytes);
 #pragma unroll
         for (int ks = 0; ks < kTileN / 16; ++ks) {
           const uint32_t aoff = static_cast<uint32_t>((ks >> 2) * L::kSlab + (ks & 3) * 32);
-          const uint64_t ad = smem_desc_sw128(p_addr + aoff, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(pb + aoff, 16, 1024);
           const uint64_t bd =
               smem_desc_sw128(v_addr + st * L::kKVBytes + ks * 16 * 128, L::kSlab, 1024);
           mma_bf16_ss(o_tmem, ad, bd, idO, (j > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&bars->vempty[st]);
-        mma_commit(&bars->pv_done);
+        mma_commit(&bars->pv_done[j & 1]);
       }
       // all issued MMAs complete before the CTA releases tensor memory
       mma_commit(&bars->mma_idle);
@@ -283,99 +336,112 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(&bars->mma_idle, 0, &never);
     }
   } else {
-    // --------------------- softmax (warps 0-3, one row per thread) -------------
-    const int row = threadIdx.x;  // 0..127 == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((warp * 32) << 16);
+    // ------------- softmax (warps 0-7): two threads per query row -------------
+    // warp w owns TMEM lanes 32*(w%4).. (rows) and key columns 64*(w/4)..+63;
+    // the two halves of a row agree on the row maximum through shared memory
+    constexpr int kHalf = kTileN / 2;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;  // 0..127 == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((quarter * 32) << 16);
+    const uint32_t o_tmem = tmem + lane_base + 2u * kTileN + half * (HD / 2);
+    const uint32_t xch = tmem + lane_base + kXchCol;  // columns: 2 buffers x 2 halves
     const float sc = p.sc;
     float m_ref = -INFINITY, l_sum = 0.f;
     SlotIter it;
-    it.init(csr_row, offk, kk);
+    it.init(runs, nr);
     bool ok = true;
     for (int j = 0; j < T; ++j) {
-      // which of the 128 key columns are real keys
-      uint32_t vmask[4] = {0, 0, 0, 0};
+      // which of this half's 64 key columns are real keys
+      uint32_t vmask[2] = {0, 0};
 #pragma unroll
       for (int s = 0; s < kSlotsPerTile; ++s) {
         int st0 = 0, vv = 0;
         if (!it.next(st0, vv)) vv = 0;
         const uint32_t bits = (vv >= 8) ? 0xFFu : ((1u << vv) - 1u);
-        vmask[s >> 2] |= bits << ((s & 3) * 8);
+        if ((s >> 3) == half) vmask[(s >> 2) & 1] |= bits << ((s & 3) * 8);
       }
       if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      float sv[kTileN];
-      const uint32_t s_tmem = tmem + lane_base + static_cast<uint32_t>((j & 1) * kTileN);
-#pragma unroll
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_tmem + c * 32, r);
+      float sv[kHalf];
+      {
+        uint32_t r[kHalf];
+        const uint32_t s_tmem =
+            tmem + lane_base + static_cast<uint32_t>((j & 1) * kTileN + half * kHalf);
+        tmem_ld32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
+        tmem_ld32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool valid = (vmask[c] >> i) & 1u;
-          sv[c * 32 + i] = valid ? __uint_as_float(r[i]) * sc : -INFINITY;
-        }
+        for (int i = 0; i < kHalf; ++i)
+          sv[i] = ((vmask[i >> 5] >> (i & 31)) & 1u) ? __uint_as_float(r[i]) * sc : -INFINITY;
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < kTileN; ++i) mx = fmaxf(mx, sv[i]);
-      // P_{j-1} V_{j-1} must be complete before P is overwritten or O rescaled
-      if (j > 0 && !mbar_wait(&bars->pv_done, (j - 1) & 1, abort)) { ok = false; break; }
-      tc_fence_after();
+      for (int i = 0; i < kHalf; ++i) mx = fmaxf(mx, sv[i]);
+      // row maximum over both halves (through tensor memory)
+      mx = fmaxf(mx, exchange_pair(xch + (j & 1) * 2, half, quarter, mx));
+      // reference maximum for this tile (moves only when it grows by > 2^8)
+      float alpha = 1.f;
+      bool need = false;
       if (j == 0) {
         m_ref = mx;
-      } else {
-        const bool need = mx > m_ref + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m_ref - mx) : 1.f;
-          if (need) {
-            l_sum *= alpha;
-            m_ref = mx;
-          }
-          const uint32_t o_tmem = tmem + lane_base + 2u * kTileN;
-#pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(o_tmem + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(o_tmem + c * 32, r);
-          }
-          tmem_wait_st();
-        }
+      } else if (mx > m_ref + kRescaleThreshold) {
+        need = true;
+        alpha = ex2_approx(m_ref - mx);
+        m_ref = mx;
       }
-      // P = 2^(s - m_ref) in bf16, row sum in fp32
+      // P = 2^(s - m_ref): bf16 pairs in registers, partial row sum in fp32
+      uint32_t pk[kHalf / 2];
       float rs = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < kTileN / 8; ++c8) {
-        float pv[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          pv[i] = ex2_approx(sv[c8 * 8 + i] - m_ref);
-          rs += pv[i];
-        }
-        uint4 pk;
-        pk.x = pack_bf16x2(pv[0], pv[1]);
-        pk.y = pack_bf16x2(pv[2], pv[3]);
-        pk.z = pack_bf16x2(pv[4], pv[5]);
-        pk.w = pack_bf16x2(pv[6], pv[7]);
-        const uint32_t off = static_cast<uint32_t>((c8 >> 3) * L::kSlab) + swz(row, c8 & 7);
-        *reinterpret_cast<uint4*>(Ps + off) = pk;
+      for (int i = 0; i < kHalf; i += 2) {
+        const float a = ex2_approx(sv[i] - m_ref), b = ex2_approx(sv[i + 1] - m_ref);
+        rs += a + b;
+        pk[i >> 1] = pack_bf16x2(a, b);
       }
-      l_sum += rs;
+      // P buffer (j & 1) is free once P(j-2) V(j-2) has completed
+      if (j >= 2 && !mbar_wait(&bars->pv_done[j & 1], ((j - 2) >> 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        // O must hold P(j-1) V(j-1) before it is rescaled (this half's columns)
+        if (!mbar_wait(&bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < HD / 64; ++c) {
+          uint32_t r[32];
+          tmem_ld32(o_tmem + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(o_tmem + c * 32, r);
+        }
+        tmem_wait_st();
+      }
+      l_sum = l_sum * alpha + rs;
+      uint8_t* pbuf = Ps + (j & 1) * L::kPBytes + half * L::kSlab;
+#pragma unroll
+      for (int c8 = 0; c8 < kHalf / 8; ++c8) {
+        const uint4 v4 = make_uint4(pk[c8 * 4 + 0], pk[c8 * 4 + 1], pk[c8 * 4 + 2], pk[c8 * 4 + 3]);
+        *reinterpret_cast<uint4*>(pbuf + swz(row, c8)) = v4;
+      }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive(&bars->p_full[j & 1]);
     }
     // ---------------- epilogue: O / l -> global (fp32, group-major rows) ------
-    if (ok && mbar_wait(&bars->pv_done, (T - 1) & 1, abort)) {
+    // both halves of a row combine their partial sums (buffer T & 1 is free:
+    // the partner read buffer (T-1) & 1 last)
+    l_sum += exchange_pair(xch + (T & 1) * 2, half, quarter, l_sum);
+    if (ok && mbar_wait(&bars->pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort)) {
       tc_fence_after();
       const float inv = 1.f / l_sum;
-      const uint32_t o_tmem = tmem + lane_base + 2u * kTileN;
-      float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD;
+      float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD + half * (HD / 2);
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < HD / 64; ++c) {
         uint32_t r[32];
         tmem_ld32(o_tmem + c * 32, r);
         tmem_wait_ld();
@@ -400,36 +466,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Work list: one entry per 128-row tile of each query group, (g << 16) | t.
+// One warp per head: tile counts are prefix-summed 32 groups at a time.
 // ---------------------------------------------------------------------------
 __global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_head, int32_t* work,
                                  int32_t* nwork) {
-  const int h = blockIdx.x;
+  const int h = blockIdx.x, lane = threadIdx.x;
   const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
-  __shared__ int32_t total;
-  if (threadIdx.x == 0) {
-    int32_t pos = 0;
-    for (int g = 0; g < Cq; ++g) {
-      const int n = oq[g + 1] - oq[g];
-      const int t = (n + kTileM - 1) / kTileM;
-      for (int i = 0; i < t && pos < tiles_per_head; ++i)
-        work[static_cast<size_t>(h) * tiles_per_head + pos++] = (g << 16) | i;
+  int32_t* wl = work + static_cast<size_t>(h) * tiles_per_head;
+  int32_t base = 0;
+  for (int g0 = 0; g0 < Cq; g0 += 32) {
+    const int g = g0 + lane;
+    const int n = (g < Cq) ? oq[g + 1] - oq[g] : 0;
+    const int t = n > 0 ? (n + kTileM - 1) / kTileM : 0;
+    int x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    total = pos;
-    nwork[h] = pos;
+    const int start = base + x - t;
+    for (int i = 0; i < t && start + i < tiles_per_head; ++i) wl[start + i] = (g << 16) | i;
+    base += __shfl_sync(0xffffffffu, x, 31);
   }
+  if (lane == 0) nwork[h] = min(base, tiles_per_head);
 }
 
-// KV slot counts per query group (same merge rule as the attention kernel's
-// walk) and the exact routed pair count per head.
+// Merged key runs and KV slot counts per query group (same rule the attention
+// kernel walks), and the exact routed pair count per head.
 __global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, const int32_t* csr,
                                    const int32_t* kh, int H, int N, int Cq, int Ck, int kmax,
-                                   int32_t* nslots, int64_t* pairs, DeviceStats* stats) {
+                                   int32_t* nslots, int2* runs, int32_t* nruns, int64_t* pairs,
+                                   DeviceStats* stats) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= H * Cq) return;
   const int h = i / Cq, g = i % Cq;
   const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
   const int32_t* ok = off_k + static_cast<size_t>(h) * (Ck + 1);
   const int32_t* row = csr + static_cast<size_t>(i) * kmax;
+  int2* rout = runs + static_cast<size_t>(i) * kmax;
   const int k = kh[h];
   const int64_t nq = oq[g + 1] - oq[g];
   // reject malformed routes before the attention kernel walks them
@@ -440,24 +514,30 @@ __global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, c
   }
   if (!valid) {
     nslots[i] = 0;
+    nruns[i] = 0;
     raise_status(stats, SPARSEPR_ERR_INVALID_ARG);
     return;
   }
   int64_t keys = 0;
-  int slots = 0;
+  int slots = 0, nr = 0;
   int ci = 0;
   while (ci < k) {
-    int c = row[ci];
-    int lo = ok[c], hi = ok[c + 1];
+    const int c = row[ci];
+    const int lo = ok[c];
+    int hi = ok[c + 1];
     while (ci + 1 < k && ok[row[ci + 1]] == hi) {
       ++ci;
       hi = ok[row[ci] + 1];
     }
-    keys += hi - lo;
-    slots += (hi - lo + kSlotRows - 1) / kSlotRows;
+    if (hi > lo) {
+      rout[nr++] = make_int2(lo, hi - lo);
+      keys += hi - lo;
+      slots += (hi - lo + kSlotRows - 1) / kSlotRows;
+    }
     ++ci;
   }
   nslots[i] = slots;
+  nruns[i] = nr;
   if (pairs && nq > 0) atomicAdd(reinterpret_cast<unsigned long long*>(&pairs[h]),
                                  static_cast<unsigned long long>(nq * keys));
   if (nq > 0 && keys == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
@@ -522,19 +602,28 @@ bool make_map(CUtensorMap* m, const void* base, size_t rows, int d, int box_rows
 
 template <int HD>
 cudaError_t launch_attn_hd(const AttnArgs& a, AttnParams prm, cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
+  AttnMaps maps;
   const size_t qrows_total = static_cast<size_t>(a.H) * a.q_rows;
+  const size_t krows_total = static_cast<size_t>(a.H) * a.N;
   prm.q_box_rows = qrows_total < static_cast<size_t>(kTileM) ? static_cast<int>(qrows_total) : kTileM;
-  if (!make_map(&tq, a.qp, qrows_total, HD, prm.q_box_rows) ||
-      !make_map(&tk, a.kp, static_cast<size_t>(a.H) * a.N, HD, kSlotRows) ||
-      !make_map(&tv, a.vp, static_cast<size_t>(a.H) * a.N, HD, kSlotRows))
-    return cudaErrorInvalidValue;
+  if (!make_map(&maps.q, a.qp, qrows_total, HD, prm.q_box_rows)) return cudaErrorInvalidValue;
+  prm.max_lg = 0;
+  for (int lg = 0; lg < 5; ++lg) {
+    // boxes larger than the tensor (tiny inputs) are never used
+    const int rows = kSlotRows << lg;
+    const bool fits = static_cast<size_t>(rows) <= krows_total;
+    if (fits) prm.max_lg = lg;
+    const int box = fits ? rows : kSlotRows;
+    if (!make_map(&maps.k[lg], a.kp, krows_total, HD, box) ||
+        !make_map(&maps.v[lg], a.vp, krows_total, HD, box))
+      return cudaErrorInvalidValue;
+  }
   const int shb = kAttnSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<HD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
   if (e != cudaSuccess) return e;
   dim3 grid(a.tiles_per_head, a.H);
-  sparse_attn_kernel<HD><<<grid, kAttnThreads, shb, st>>>(tq, tk, tv, prm);
+  sparse_attn_kernel<HD><<<grid, kAttnThreads, shb, st>>>(maps, prm);
   return cudaGetLastError();
 }
 
@@ -545,24 +634,23 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   if (a.pairs) zero_i64_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H);
   const int n = a.H * a.Cq;
   slots_pairs_kernel<<<(n + 127) / 128, 128, 0, st>>>(a.off_q, a.off_k, a.csr, a.kh, a.H, a.N,
-                                                     a.Cq, a.Ck, a.kmax, a.nslots, a.pairs,
-                                                     a.stats);
+                                                     a.Cq, a.Ck, a.kmax, a.nslots, a.runs,
+                                                     a.nruns, a.pairs, a.stats);
   if (a.pairs) pairs_to_stats_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H, a.stats);
   AttnParams prm;
   prm.H = a.H;
   prm.N = a.N;
   prm.q_rows = a.q_rows;
   prm.Cq = a.Cq;
-  prm.Ck = a.Ck;
   prm.kmax = a.kmax;
   prm.off_q = a.off_q;
-  prm.off_k = a.off_k;
-  prm.csr = a.csr;
-  prm.kh = a.kh;
   prm.work = a.work;
   prm.nwork = a.nwork;
   prm.nslots = a.nslots;
+  prm.runs = a.runs;
+  prm.nruns = a.nruns;
   prm.tiles_per_head = a.tiles_per_head;
+  prm.q_box_rows = kTileM;
   prm.sc = a.scale * kLog2e;
   prm.out = a.out;
   prm.stats = a.stats;

@@ -64,6 +64,52 @@ constexpr int kXf64 = 0;
 constexpr int kXbf16 = 1;
 constexpr int kXf32 = 2;
 
+// ---- assign.cu: certified tensor-core nearest-centroid assignment ----------
+struct AssignTC {
+  const __nv_bfloat16* a_planes;  // [nA][a_rows_total][Dp]
+  long long a_plane_stride;       // elements between planes
+  size_t a_rows_total;
+  int a_head;                     // rows between heads in the A planes
+  int nA;
+  const __nv_bfloat16* b_planes;  // [nB][H * Cpad][Dp]
+  long long b_plane_stride;
+  int nB;
+  int Dp;                         // 16 (32-byte rows) or a multiple of 64
+  int Cpad;                       // centroids per head padded to a multiple of 16
+  int H, n;                       // heads, rows per head
+  int npairs;
+  int pairs[6];
+  const float* cvals;             // [H, Cpad]
+  const float* xnorm;             // [H, n]
+  const float* hmax;              // [H, 2]
+  int32_t* labels;                // [H, n]
+  int32_t* flags;
+  int flag_base;
+  int32_t* recheck;               // [H, n]
+  int32_t* nrecheck;              // [H]
+  DeviceStats* stats;
+  int sm_count;
+  // exact operands for the fp64 decision of flagged rows
+  const void* x_exact;
+  int x_kind;
+  long long x_hs;
+  int x_ld;
+  int D;
+  const double* y_exact;          // [H, m, D]
+  const double* c_exact;          // [H, m] (unused when direct)
+  int m;
+  int direct;                     // 1: d = |x - y|^2, 0: d = c - 2 x.y
+};
+size_t assign_tc_smem_bytes(int nA, int nB, int Dp, int Cpad);
+cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, int n, int D,
+                              int Dp, int P, int H, __nv_bfloat16* planes, long long plane_stride,
+                              float* norms, cudaStream_t st);
+cudaError_t launch_prep_centroids(const double* Y, const double* c, int m, int D, int Dp,
+                                  int Cpad, int P, int H, __nv_bfloat16* planes,
+                                  long long plane_stride, float* cf, float* hmax,
+                                  const int32_t* flags, int flag_base, cudaStream_t st);
+cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st);
+
 // ---- linalg.cu -------------------------------------------------------------
 // Cyclic-parallel Jacobi eigensolver, one CTA per head: A [H, d, d] fp64
 // symmetric -> eval [H, d], evec [H, d, d] (eigenvectors in columns).
@@ -104,6 +150,8 @@ struct AttnArgs {
   int32_t* nwork;        // [H]
   int tiles_per_head;
   int32_t* nslots;       // [H, Cq]
+  int2* runs;            // [H, Cq, kmax] merged key runs (start, length)
+  int32_t* nruns;        // [H, Cq]
   int64_t* pairs;        // [H] (may be null)
   DeviceStats* stats;
 };

@@ -43,6 +43,18 @@ struct Layout {
   size_t qbar;     // [H, Cq, d] f64 query centroids
   size_t wg;       // [H, Cq, d] f64 G * qbar
   size_t cg;       // [H, Cq] f64 qbar^T G qbar
+  // tensor-core assignment operands
+  size_t zplanes;  // [3][H * Nv][Dpk] bf16 planes of z
+  size_t xnk;      // [H, Nv] f32 |z|
+  size_t xnq;      // [H, Nv] f32 |q|
+  size_t muplanes; // [3][H * CpadK][Dpk] bf16
+  size_t cfk;      // [H, CpadK] f32
+  size_t hmk;      // [H, 2] f32
+  size_t wplanes;  // [3][H * CpadQ][d] bf16
+  size_t cfq;      // [H, CpadQ] f32
+  size_t hmq;      // [H, 2] f32
+  size_t recheck;  // [H, Nv] int32
+  size_t nrecheck; // [H] int32
   // stage 3
   size_t cq;       // [H, Cq, d] f64 query-group means (route)
   size_t ckr;      // [H, Ck, d] f64 key-group means (route)
@@ -50,6 +62,8 @@ struct Layout {
   size_t work;     // [H, tiles_per_head] int32 attention work list
   size_t nwork;    // [H] int32
   size_t nslots;   // [H, Cq] int32 KV row-slots per query group
+  size_t runs;     // [H, Cq, kmax] int2 merged kept key runs (start, length)
+  size_t nruns;    // [H, Cq] int32
   // stage 4
   size_t probe_q;  // [H, M, d] bf16 gathered probe rows (group-major)
   size_t od;       // [H, M, d] f32 dense outputs of the probes
@@ -62,10 +76,12 @@ struct Layout {
   size_t bv32;     // [H, d] f32 projected b'
   size_t pwork;    // [H, M/128 + 1] int32 probe attention work list
   size_t pnwork;   // [H] int32
-  size_t pmeta;    // [H, 7] int32: dense-mode off_q(2), off_k(2), csr(1), k(1), nslots(1)
+  size_t pmeta;    // [H, 10] int32: dense-mode off_q(2), off_k(2), csr(1), k(1), nslots(1),
+                   // nruns(1), runs(2)
   size_t total;
 
   int Nv, e, Cmax, nchunk, tiles_per_head, kmax;
+  int Dpk, CpadK, CpadQ;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -125,12 +141,28 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->qbar = take(H * Cq * d * 8);
   L->wg = take(H * Cq * d * 8);
   L->cg = take(H * Cq * 8);
+  L->Dpk = (p.n_eig <= 16) ? 16 : 64;
+  L->CpadK = (p.Ck + 15) / 16 * 16;
+  L->CpadQ = (p.Cq + 15) / 16 * 16;
+  L->zplanes = take(3 * H * Nv * static_cast<size_t>(L->Dpk) * 2);
+  L->xnk = take(H * Nv * 4);
+  L->xnq = take(H * Nv * 4);
+  L->muplanes = take(3 * H * static_cast<size_t>(L->CpadK) * L->Dpk * 2);
+  L->cfk = take(H * static_cast<size_t>(L->CpadK) * 4);
+  L->hmk = take(H * 8);
+  L->wplanes = take(3 * H * static_cast<size_t>(L->CpadQ) * d * 2);
+  L->cfq = take(H * static_cast<size_t>(L->CpadQ) * 4);
+  L->hmq = take(H * 8);
+  L->recheck = take(H * Nv * 4);
+  L->nrecheck = take(H * 4);
   L->cq = take(H * Cq * d * 8);
   L->ckr = take(H * Ck * d * 8);
   L->bf16_qkv = take(3 * H * N * d * 2);
   L->work = take(H * static_cast<size_t>(L->tiles_per_head) * 4);
   L->nwork = take(H * 4);
   L->nslots = take(H * Cq * 4);
+  L->runs = take(H * Cq * static_cast<size_t>(kmax) * 8);
+  L->nruns = take(H * Cq * 4);
   L->probe_q = take(H * (M + kTileM) * d * 2);
   L->od = take(H * (M + 1) * d * 4);
   L->xr = take(H * 2 * (M + 1) * d * 8);
@@ -142,7 +174,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->bv32 = take(H * d * 4);
   L->pwork = take(H * (M / kTileM + 2) * 4);
   L->pnwork = take(H * 4);
-  L->pmeta = take(H * 7 * 4);
+  L->pmeta = take(H * 10 * 4);
   L->total = o;
 }
 
