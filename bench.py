@@ -327,7 +327,9 @@ def main():
             dense_same_kernel_tflops=4.0 * w.d * w.H * w.N * w.N / (dense_max * 1e-3) / 1e12,
             speedup_vs_dense=dense_max / ms_max,
             attn_only_speedup_vs_dense=dense_max / attn_max,
-            kmeans_passes=dict(key=st["key_passes"], query=st["query_passes"]),
+            kmeans_passes=dict(key=st["key_passes"], query=st["query_passes"],
+                               fp64_recheck_rows=st["recheck_rows"]),
+            eigen_sweeps=st["eig_sweeps"],
             device_status=st["status"],
             roofline=dict(bound="tensor", kernel="sparse_attn_kernel<128>",
                           achieved=attn_tflops, peak=peak, unit="TFLOP/s",

@@ -195,7 +195,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
   SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, st));
   SPR_TRY(launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st));
-  SPR_TRY(launch_jacobi(mk, H, d, evl, evc, c.stats, st));
+  SPR_TRY(launch_jacobi(mk, H, d, evl, evc, c.stats, 0, st));
   SPR_TRY(launch_top_eig_projector(evl, evc, H, d, e, wk, st));
   SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
   const long long hs_z = static_cast<long long>(Nv) * e;
@@ -507,7 +507,7 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
                             static_cast<long long>(d) * d, 0, st));
     double* evl = at<double>(ws, L.eval);
     double* evc = at<double>(ws, L.evec);
-    SPR_TRY(launch_jacobi(rtr, H, d, evl, evc, c.stats, st));
+    SPR_TRY(launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st));
     SPR_TRY(launch_project_map(bmat, bvec, evl, evc, H, d, c.p.r, bp32, bv32, fit, st));
   } else {
     SPR_TRY(cudaMemsetAsync(bp32, 0, static_cast<size_t>(H) * d * d * 4, st));

@@ -210,33 +210,46 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     for (int u = 0; u < ntile && ok; ++u) {
       const int t = blockIdx.x + u * gridDim.x;
       const int row = t * kTileM + r;
-      float d1 = INFINITY, d2 = INFINITY;
-      int i1 = 0x7fffffff;
+      float b1[8], b2[8];
+      int bi[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        b1[k] = INFINITY;
+        b2[k] = INFINITY;
+        bi[k] = 0x7fffffff;
+      }
       for (int c = 0; c < nchunks; ++c, ++gc) {
         const int buf = gc & 1;
         if (!mbar_wait(&bars->acc_full[buf], (gc >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
         const uint32_t base = tmem + lane_base + static_cast<uint32_t>(buf * kAsChunk);
-        for (int c32 = 0; c32 < N; c32 += 32) {
-          uint32_t v[32];
-          const int w = min(32, N - c32);  // 32, or 16 for the last group
-          if (w == 32)
-            tmem_ld32(base + c32, v);
-          else
-            tmem_ld16(base + c32, *reinterpret_cast<uint32_t(*)[16]>(v));
-          tmem_wait_ld();
-          const int j0 = c * kAsChunk + c32;
+        for (int cb = 0; cb < N; cb += 128) {
+          // up to 128 columns per wait; widths are multiples of 16 (warp-uniform)
+          uint32_t v[128];
+          const int w = min(128, N - cb);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i >= w) break;
-            const float dd = fmaf(-2.f, __uint_as_float(v[i]), cs[j0 + i]);
-            if (dd < d1) {
-              d2 = d1;
-              d1 = dd;
-              i1 = j0 + i;
-            } else if (dd < d2) {
-              d2 = dd;
+          for (int qd = 0; qd < 4; ++qd) {
+            const int off = qd * 32;
+            if (off + 32 <= w)
+              tmem_ld32(base + cb + off, *reinterpret_cast<uint32_t(*)[32]>(v + off));
+            else if (off + 16 <= w)
+              tmem_ld16(base + cb + off, *reinterpret_cast<uint32_t(*)[16]>(v + off));
+          }
+          tmem_wait_ld();
+          const int j0 = c * kAsChunk + cb;
+          // running best and second best in eight independent chains (column
+          // i goes to chain i % 8), branch-free; within a chain columns ascend,
+          // so equal values keep the lower index
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            if (i < w) {
+              const int k = i & 7;
+              const float dd = fmaf(-2.f, __uint_as_float(v[i]), cs[j0 + i]);
+              const bool lt = dd < b1[k];
+              b2[k] = fminf(b2[k], fmaxf(b1[k], dd));
+              bi[k] = lt ? (j0 + i) : bi[k];
+              b1[k] = fminf(b1[k], dd);
             }
           }
         }
@@ -244,6 +257,26 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         mbar_arrive(&bars->acc_empty[buf]);
       }
       if (!ok || row >= p.n) continue;
+      // merge the chains: best by (value, index), second = smallest of the
+      // chains' seconds and the other chains' bests
+      float d1 = b1[0];
+      int i1 = bi[0];
+#pragma unroll
+      for (int k = 1; k < 8; ++k)
+        if (b1[k] < d1 || (b1[k] == d1 && bi[k] < i1)) {
+          d1 = b1[k];
+          i1 = bi[k];
+        }
+      float d2 = INFINITY;
+      bool used = false;  // the winning chain's best is not a second candidate
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        d2 = fminf(d2, b2[k]);
+        if (!used && b1[k] == d1 && bi[k] == i1)
+          used = true;
+        else
+          d2 = fminf(d2, b1[k]);
+      }
       const float xn = p.xnorm[static_cast<size_t>(h) * p.n + row];
       const float xy = xn * Y;
       const float E = kt_term * xy + 2.384185791015625e-07f * (C + 2.f * xy);
@@ -254,6 +287,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       } else {
         const int k = atomicAdd(&p.nrecheck[h], 1);
         p.recheck[static_cast<size_t>(h) * p.n + k] = row;
+        atomicAdd(reinterpret_cast<unsigned long long*>(&p.stats->recheck_rows[p.flag_base >> 1]),
+                  1ull);
       }
     }
   }
@@ -267,9 +302,12 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// fp64 decision of the flagged rows: one warp per row, lanes over centroids.
+// fp64 decision of the flagged rows: blocks of 16 rows scan the centroids in
+// chunks of 16 staged in shared memory.
 // direct = 1: d = sum_t (x_t - y_jt)^2; else d = c_j - 2 x . y_j.
 // ---------------------------------------------------------------------------
+constexpr int kRcRows = 16, kRcCols = 16, kRcMaxD = 128;
+
 __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   if (kind == kXf64) return static_cast<const double*>(X)[i];
   if (kind == kXbf16) return static_cast<double>(__bfloat162float(static_cast<const __nv_bfloat16*>(X)[i]));
@@ -280,38 +318,66 @@ __global__ void recheck_kernel(const void* X, int kind, long long hsx, int ldx_,
                                const double* Y, const double* c, int m, int direct,
                                int32_t* labels, int32_t* flags, int flag_base,
                                const int32_t* recheck, const int32_t* nrecheck) {
+  // a block of up to 16 flagged rows against the centroids, 16 at a time;
+  // thread (r, s) = (row in block, centroid in chunk), 256 threads
+  __shared__ double xs[kRcRows][kRcMaxD];
+  __shared__ double ys[kRcCols][kRcMaxD + 1];
+  __shared__ double cc[kRcCols];
+  __shared__ int rows_s[kRcRows];
   const int h = blockIdx.y;
   int32_t* fl = flags + h * 4;
   if (fl[flag_base + 1]) return;
   const int cnt = nrecheck[h];
-  const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
+  const int r = threadIdx.x >> 4, s = threadIdx.x & 15;
   const double* Yh = Y + static_cast<size_t>(h) * m * D;
-  for (int w = blockIdx.x * wpb + (threadIdx.x >> 5); w < cnt; w += gridDim.x * wpb) {
-    const int row = recheck[static_cast<size_t>(h) * n + w];
-    const size_t xb = h * hsx + static_cast<size_t>(row) * ldx_;
+  for (int b0 = blockIdx.x * kRcRows; b0 < cnt; b0 += gridDim.x * kRcRows) {
+    const int nb = min(kRcRows, cnt - b0);
+    if (threadIdx.x < kRcRows)
+      rows_s[threadIdx.x] = (static_cast<int>(threadIdx.x) < nb)
+                                ? recheck[static_cast<size_t>(h) * n + b0 + threadIdx.x]
+                                : -1;
+    __syncthreads();
+    for (int t = threadIdx.x; t < kRcRows * D; t += blockDim.x) {
+      const int rr = t / D, cc_ = t % D;
+      xs[rr][cc_] = (rows_s[rr] >= 0) ? ldx(X, kind, h * hsx + static_cast<size_t>(rows_s[rr]) * ldx_ + cc_)
+                                      : 0.0;
+    }
     double best = INFINITY;
     int bi = 0x7fffffff;
-    for (int j = lane; j < m; j += 32) {
-      double dd;
-      if (direct) {
-        dd = 0.0;
-        for (int t = 0; t < D; ++t) {
-          const double diff = ldx(X, kind, xb + t) - Yh[static_cast<size_t>(j) * D + t];
-          dd = fma(diff, diff, dd);
-        }
-      } else {
-        double s = 0.0;
-        for (int t = 0; t < D; ++t) s = fma(ldx(X, kind, xb + t), Yh[static_cast<size_t>(j) * D + t], s);
-        dd = c[static_cast<size_t>(h) * m + j] - 2.0 * s;
+    for (int j0 = 0; j0 < m; j0 += kRcCols) {
+      __syncthreads();  // previous chunk consumed (and xs written, first time)
+      for (int t = threadIdx.x; t < kRcCols * D; t += blockDim.x) {
+        const int jj = t / D, cc_ = t % D;
+        ys[jj][cc_] = (j0 + jj < m) ? Yh[static_cast<size_t>(j0 + jj) * D + cc_] : 0.0;
       }
-      if (dd < best) {
-        best = dd;
-        bi = j;
+      if (!direct && threadIdx.x < kRcCols)
+        cc[threadIdx.x] = (j0 + static_cast<int>(threadIdx.x) < m)
+                              ? c[static_cast<size_t>(h) * m + j0 + threadIdx.x]
+                              : 0.0;
+      __syncthreads();
+      const int j = j0 + s;
+      if (j < m) {
+        double dd;
+        if (direct) {
+          dd = 0.0;
+          for (int t = 0; t < D; ++t) {
+            const double diff = xs[r][t] - ys[s][t];
+            dd = fma(diff, diff, dd);
+          }
+        } else {
+          double sm = 0.0;
+          for (int t = 0; t < D; ++t) sm = fma(xs[r][t], ys[s][t], sm);
+          dd = cc[s] - 2.0 * sm;
+        }
+        if (dd < best) {  // within a thread centroids ascend
+          best = dd;
+          bi = j;
+        }
       }
     }
+    // reduce over the 16 threads of each row (lowest index on ties)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int o = 8; o > 0; o >>= 1) {
       const double ob = __shfl_xor_sync(0xffffffffu, best, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ob < best || (ob == best && oi < bi)) {
@@ -319,11 +385,12 @@ __global__ void recheck_kernel(const void* X, int kind, long long hsx, int ldx_,
         bi = oi;
       }
     }
-    if (lane == 0) {
-      const size_t li = static_cast<size_t>(h) * n + row;
+    if (s == 0 && r < nb) {
+      const size_t li = static_cast<size_t>(h) * n + rows_s[r];
       if (labels[li] != bi) atomicAdd(&fl[flag_base], 1);
       labels[li] = bi;
     }
+    __syncthreads();  // rows_s / xs are rewritten by the next block
   }
 }
 

@@ -56,9 +56,10 @@ struct Smem {
 // Dynamic shared memory: the d=128 footprint for both head dims (one CTA per
 // SM; each CTA allocates 512 TMEM columns), the barrier block, a run list of
 // up to kSmemRuns entries, and 1024 bytes of alignment slack.
-constexpr int kSmemRuns = 96;
-constexpr int kAttnSmemBytes = Smem<128>::runs_off + kSmemRuns * 8 + 1024;
-static_assert(kAttnSmemBytes <= 232448, "shared memory");
+// The whole per-block maximum is requested; what the 1024-byte alignment of
+// the tile region leaves after the barriers holds the run list (>= 226 runs).
+constexpr int kAttnSmemBytes = 232448;
+static_assert(Smem<128>::runs_off + 226 * 8 + 1008 <= kAttnSmemBytes, "shared memory");
 
 struct Bars {
   uint64_t q_full;
@@ -374,9 +375,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < kHalf; ++i)
           sv[i] = ((vmask[i >> 5] >> (i & 31)) & 1u) ? __uint_as_float(r[i]) * sc : -INFINITY;
       }
-      float mx = -INFINITY;
+      // row maximum of this half: eight independent chains, then a tree
+      float m8[8];
 #pragma unroll
-      for (int i = 0; i < kHalf; ++i) mx = fmaxf(mx, sv[i]);
+      for (int k = 0; k < 8; ++k) m8[k] = sv[k];
+#pragma unroll
+      for (int i = 8; i < kHalf; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       // row maximum over both halves (through tensor memory)
       mx = fmaxf(mx, exchange_pair(xch + (j & 1) * 2, half, quarter, mx));
       // reference maximum for this tile (moves only when it grows by > 2^8)
@@ -391,13 +397,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // P = 2^(s - m_ref): bf16 pairs in registers, partial row sum in fp32
       uint32_t pk[kHalf / 2];
-      float rs = 0.f;
+      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < kHalf; i += 2) {
         const float a = ex2_approx(sv[i] - m_ref), b = ex2_approx(sv[i + 1] - m_ref);
-        rs += a + b;
+        r8[(i >> 1) & 7] += a + b;
         pk[i >> 1] = pack_bf16x2(a, b);
       }
+      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       // P buffer (j & 1) is free once P(j-2) V(j-2) has completed
       if (j >= 2 && !mbar_wait(&bars->pv_done[j & 1], ((j - 2) >> 1) & 1, abort)) {
         ok = false;

@@ -114,7 +114,7 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st);
 // Cyclic-parallel Jacobi eigensolver, one CTA per head: A [H, d, d] fp64
 // symmetric -> eval [H, d], evec [H, d, d] (eigenvectors in columns).
 cudaError_t launch_jacobi(const double* A, int H, int d, double* eval, double* evec,
-                          DeviceStats* stats, cudaStream_t st);
+                          DeviceStats* stats, int which, cudaStream_t st);
 // wk[h, a, t] = evec[h, a, j_t] * sqrt(max(eval_j_t, 0)) for the e largest
 // eigenvalues (t = rank, ties to the lower index).
 cudaError_t launch_top_eig_projector(const double* eval, const double* evec, int H, int d, int e,

@@ -8,88 +8,96 @@
 // per sweep. Rotation angles follow the symmetric 2x2 Schur decomposition
 // (Golub & Van Loan, Matrix Computations, sec. 8.5). One CTA per matrix; the
 // upper triangle of A (packed) and the full eigenvector matrix live in
-// shared memory.
+// shared memory. Blocks whose two rotations are both the identity are
+// skipped, so late sweeps cost little.
 #include "common.cuh"
 #include "internal.h"
 
 namespace spr {
 namespace {
 
-constexpr int kJacobiThreads = 512;
-constexpr int kMaxSweeps = 24;
+constexpr int kJacobiThreads = 1024;
+constexpr int kMaxSweeps = 30;
 
-__device__ __forceinline__ int tri(int i, int j, int d) {
+template <int D>
+__device__ __forceinline__ int tri(int i, int j) {
   // packed upper triangle, i <= j
-  return i * d - (i * (i - 1)) / 2 + (j - i);
+  return i * D - ((i * (i - 1)) >> 1) + (j - i);
 }
-__device__ __forceinline__ int sym(int i, int j, int d) {
-  return i <= j ? tri(i, j, d) : tri(j, i, d);
+template <int D>
+__device__ __forceinline__ int sym(int i, int j) {
+  return i <= j ? tri<D>(i, j) : tri<D>(j, i);
 }
 
-__global__ void __launch_bounds__(kJacobiThreads) jacobi_kernel(const double* A_in, int d,
-                                                                double* eval, double* evec,
-                                                                DeviceStats* stats) {
+template <int D>
+__global__ void __launch_bounds__(kJacobiThreads) jacobi_kernel(const double* A_in, double* eval,
+                                                                double* evec, DeviceStats* stats,
+                                                                int which) {
+  constexpr int P = D / 2;
+  constexpr int NT = D * (D + 1) / 2;
   extern __shared__ double jsm[];
-  const int P = d / 2;
-  const int ntri = d * (d + 1) / 2;
-  double* A = jsm;              // [ntri]
-  double* V = A + ntri;         // [d*d], V[i*d + j]
-  double* cs = V + d * d;       // [P] cos
-  double* sn = cs + P;          // [P] sin
+  double* A = jsm;           // [NT]
+  double* V = A + NT;        // [D*D], V[i*D + j]
+  double* cs = V + D * D;    // [P] cos
+  double* sn = cs + P;       // [P] sin
   int* pp = reinterpret_cast<int*>(sn + P);  // [P]
   int* qq = pp + P;                          // [P]
-  __shared__ double red[kJacobiThreads / 32];
+  __shared__ double red[kJacobiThreads / 32][2];
   __shared__ int stop;
   const int h = blockIdx.x;
-  const double* Ah = A_in + static_cast<size_t>(h) * d * d;
-  for (int t = threadIdx.x; t < d * d; t += blockDim.x) {
-    const int i = t / d, j = t % d;
-    if (i <= j) A[tri(i, j, d)] = Ah[t];
+  const double* Ah = A_in + static_cast<size_t>(h) * D * D;
+  for (int t = threadIdx.x; t < D * D; t += blockDim.x) {
+    const int i = t / D, j = t % D;
+    if (i <= j) A[tri<D>(i, j)] = Ah[t];
     V[t] = (i == j) ? 1.0 : 0.0;
   }
   __syncthreads();
-  for (int sweep = 0; sweep < kMaxSweeps; ++sweep) {
+  int sweep = 0;
+  for (; sweep < kMaxSweeps; ++sweep) {
     // convergence: off-diagonal Frobenius mass relative to the diagonal
     double off = 0.0, dia = 0.0;
-    for (int t = threadIdx.x; t < d * d; t += blockDim.x) {
-      const int i = t / d, j = t % d;
-      if (i < j) {
-        const double v = A[tri(i, j, d)];
-        off += v * v;
-      } else if (i == j) {
-        const double v = A[tri(i, i, d)];
-        dia += v * v;
+    for (int t = threadIdx.x; t < NT; t += blockDim.x) {
+      const double v = A[t];
+      // t is the packed index of (i, j); diagonal entries sit at tri(i, i)
+      int i = 0;
+      // find the row of packed index t (rows have D, D-1, ... entries)
+      int lo = 0, hi = D - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tri<D>(mid, mid) <= t) lo = mid; else hi = mid - 1;
       }
+      i = lo;
+      if (t == tri<D>(i, i))
+        dia += v * v;
+      else
+        off += v * v;
     }
     off = warp_sum_f64(off);
     dia = warp_sum_f64(dia);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = off;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double o = 0.0;
-      for (int w = 0; w < kJacobiThreads / 32; ++w) o += red[w];
-      red[0] = o;
+    if ((threadIdx.x & 31) == 0) {
+      red[threadIdx.x >> 5][0] = off;
+      red[threadIdx.x >> 5][1] = dia;
     }
     __syncthreads();
-    const double off_tot = red[0];
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dia;
-    __syncthreads();
     if (threadIdx.x == 0) {
-      double o = 0.0;
-      for (int w = 0; w < kJacobiThreads / 32; ++w) o += red[w];
-      stop = (off_tot <= 1e-28 * o) || (off_tot == 0.0);
+      double o = 0.0, g = 0.0;
+      for (int w = 0; w < kJacobiThreads / 32; ++w) {
+        o += red[w][0];
+        g += red[w][1];
+      }
+      stop = (o <= 1e-28 * g) || (o == 0.0);
     }
     __syncthreads();
     if (stop) break;
-    for (int step = 0; step < d - 1; ++step) {
+    for (int step = 0; step < D - 1; ++step) {
       // pairs of this step and their rotations
-      for (int k = threadIdx.x; k < P; k += blockDim.x) {
-        // players 0..d-1: player 0 fixed, the others rotate by `step`
-        const int a = (k == 0) ? 0 : 1 + ((k - 1 + step) % (d - 1));
-        const int b = 1 + ((d - 2 - k + step) % (d - 1));
+      if (threadIdx.x < P) {
+        const int k = threadIdx.x;
+        // players 0..D-1: player 0 fixed, the others rotate by `step`
+        const int a = (k == 0) ? 0 : 1 + ((k - 1 + step) % (D - 1));
+        const int b = 1 + ((D - 2 - k + step) % (D - 1));
         const int p0 = min(a, b), q0 = max(a, b);
-        const double app = A[tri(p0, p0, d)], aqq = A[tri(q0, q0, d)], apq = A[tri(p0, q0, d)];
+        const double app = A[tri<D>(p0, p0)], aqq = A[tri<D>(q0, q0)], apq = A[tri<D>(p0, q0)];
         double c = 1.0, s = 0.0;
         if (apq != 0.0 && fabs(apq) > 1e-300 && fabs(apq) >= 1e-18 * sqrt(fabs(app * aqq))) {
           const double tau = (aqq - app) / (2.0 * apq);
@@ -111,21 +119,21 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_kernel(const double* A_
       for (int idx = threadIdx.x; idx < P * P; idx += blockDim.x) {
         const int a = idx / P, b = idx % P;
         if (a > b) continue;
+        const double sa = sn[a], sb = sn[b];
+        if (sa == 0.0 && sb == 0.0) continue;  // both rotations are the identity
         const int pa = pp[a], qa = qq[a];
-        const double ca = cs[a], sa = sn[a];
+        const double ca = cs[a];
         if (a == b) {
-          const double app = A[tri(pa, pa, d)], aqq = A[tri(qa, qa, d)], apq = A[tri(pa, qa, d)];
-          if (sa != 0.0) {
-            const double t = sa / ca;
-            A[tri(pa, pa, d)] = app - t * apq;
-            A[tri(qa, qa, d)] = aqq + t * apq;
-            A[tri(pa, qa, d)] = 0.0;
-          }
+          const double app = A[tri<D>(pa, pa)], aqq = A[tri<D>(qa, qa)], apq = A[tri<D>(pa, qa)];
+          const double t = sa / ca;
+          A[tri<D>(pa, pa)] = app - t * apq;
+          A[tri<D>(qa, qa)] = aqq + t * apq;
+          A[tri<D>(pa, qa)] = 0.0;
         } else {
           const int pb = pp[b], qb = qq[b];
-          const double cb = cs[b], sb = sn[b];
-          const int i00 = sym(pa, pb, d), i01 = sym(pa, qb, d), i10 = sym(qa, pb, d),
-                    i11 = sym(qa, qb, d);
+          const double cb = cs[b];
+          const int i00 = sym<D>(pa, pb), i01 = sym<D>(pa, qb), i10 = sym<D>(qa, pb),
+                    i11 = sym<D>(qa, qb);
           const double x00 = A[i00], x01 = A[i01], x10 = A[i10], x11 = A[i11];
           // Y = R_a^T X, R = [[c, s], [-s, c]]
           const double y00 = ca * x00 - sa * x10, y01 = ca * x01 - sa * x11;
@@ -138,22 +146,25 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_kernel(const double* A_
         }
       }
       // V <- V J
-      for (int idx = threadIdx.x; idx < d * P; idx += blockDim.x) {
+      for (int idx = threadIdx.x; idx < D * P; idx += blockDim.x) {
         const int i = idx / P, k = idx % P;
-        const double c = cs[k], s = sn[k];
+        const double s = sn[k];
         if (s == 0.0) continue;
-        double* vr = V + static_cast<size_t>(i) * d;
-        const double vp = vr[pp[k]], vq = vr[qq[k]];
-        vr[pp[k]] = c * vp - s * vq;
-        vr[qq[k]] = s * vp + c * vq;
+        const double c = cs[k];
+        double* vr = V + i * D;
+        const int p0 = pp[k], q0 = qq[k];
+        const double vp = vr[p0], vq = vr[q0];
+        vr[p0] = c * vp - s * vq;
+        vr[q0] = s * vp + c * vq;
       }
       __syncthreads();
     }
   }
-  for (int t = threadIdx.x; t < d * d; t += blockDim.x)
-    evec[static_cast<size_t>(h) * d * d + t] = V[t];
-  for (int j = threadIdx.x; j < d; j += blockDim.x)
-    eval[static_cast<size_t>(h) * d + j] = A[tri(j, j, d)];
+  for (int t = threadIdx.x; t < D * D; t += blockDim.x)
+    evec[static_cast<size_t>(h) * D * D + t] = V[t];
+  for (int j = threadIdx.x; j < D; j += blockDim.x)
+    eval[static_cast<size_t>(h) * D + j] = A[tri<D>(j, j)];
+  if (threadIdx.x == 0 && stats) atomicMax(&stats->eig_sweeps[which], sweep);
 }
 
 // wk[h, a, t] = evec[h, a, j] * sqrt(max(lambda_j, 0)) where j has rank t in
@@ -176,18 +187,27 @@ __global__ void top_eig_projector_kernel(const double* eval, const double* evec,
     wk[(static_cast<size_t>(h) * d + a) * e + rank] = V[static_cast<size_t>(a) * d + j] * sc;
 }
 
+template <int D>
+cudaError_t launch_jacobi_d(const double* A, int H, double* eval, double* evec,
+                            DeviceStats* stats, int which, cudaStream_t st) {
+  constexpr int P = D / 2;
+  const size_t shb = (static_cast<size_t>(D) * (D + 1) / 2 + static_cast<size_t>(D) * D + 2 * P) * 8 +
+                     2 * P * 4;
+  cudaError_t e = cudaFuncSetAttribute(jacobi_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(shb));
+  if (e != cudaSuccess) return e;
+  jacobi_kernel<D><<<H, kJacobiThreads, shb, st>>>(A, eval, evec, stats, which);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_jacobi(const double* A, int H, int d, double* eval, double* evec,
-                          DeviceStats* stats, cudaStream_t st) {
-  const int P = d / 2;
-  const size_t shb = (static_cast<size_t>(d) * (d + 1) / 2 + static_cast<size_t>(d) * d + 2 * P) * 8 +
-                     2 * P * 4;
-  cudaError_t e = cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(shb));
-  if (e != cudaSuccess) return e;
-  jacobi_kernel<<<H, kJacobiThreads, shb, st>>>(A, d, eval, evec, stats);
-  return cudaGetLastError();
+                          DeviceStats* stats, int which, cudaStream_t st) {
+  if (d == 128) return launch_jacobi_d<128>(A, H, eval, evec, stats, which, st);
+  if (d == 64) return launch_jacobi_d<64>(A, H, eval, evec, stats, which, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_top_eig_projector(const double* eval, const double* evec, int H, int d, int e,

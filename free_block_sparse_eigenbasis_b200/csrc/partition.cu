@@ -313,39 +313,63 @@ __global__ void finalize_pass_kernel(int H, int pass, int32_t* flags, int flag_b
 // Group means in a fixed order: one warp per group, lanes own coordinates,
 // members summed in ascending position order of the stable sort.
 // ---------------------------------------------------------------------------
-__global__ void group_mean_kernel(const void* X, int kind, long long hsx, int ldx, int D,
-                                  const int32_t* perm, int perm_stride, const int32_t* off,
-                                  int off_stride, int C, bool keep_prev, double* out,
-                                  double* norms, const int32_t* skip, int skip_stride) {
-  const int h = blockIdx.y;
+// One CTA of 4 warps per group: warp w sums the w-th quarter of the members
+// (ascending positions, lanes own coordinates), the four partial sums are
+// added in warp order.
+constexpr int kMeanWarps = 4;
+constexpr int kMeanMaxD = 128;
+
+__global__ void __launch_bounds__(kMeanWarps * 32) group_mean_kernel(
+    const void* X, int kind, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
+    const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
+    const int32_t* skip, int skip_stride) {
+  __shared__ double part[kMeanWarps][kMeanMaxD];
+  const int h = blockIdx.y, c = blockIdx.x;
   if (skip && skip[h * skip_stride]) return;
-  const int c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (c >= C) return;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int32_t* oo = off + static_cast<size_t>(h) * off_stride;
   const int32_t* pp = perm ? perm + static_cast<size_t>(h) * perm_stride : nullptr;
-  const int lo = oo[c], hi = oo[c + 1];
-  double* dst = out + (static_cast<size_t>(h) * C + c) * D;
-  double ss = 0.0;
+  const int lo = oo[c], hi = oo[c + 1], n = hi - lo;
+  const int a = lo + static_cast<int>((static_cast<long long>(n) * w) / kMeanWarps);
+  const int b = lo + static_cast<int>((static_cast<long long>(n) * (w + 1)) / kMeanWarps);
   for (int t0 = 0; t0 < D; t0 += 32) {
     const int t = t0 + lane;
     double acc = 0.0;
     if (t < D) {
-      for (int p = lo; p < hi; ++p) {
+#pragma unroll 8
+      for (int p = a; p < b; ++p) {
         const size_t row = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
         acc += load_x(X, kind, h * hsx + row * ldx + t);
       }
-      double v;
-      if (hi > lo)
-        v = acc / static_cast<double>(hi - lo);
-      else
-        v = keep_prev ? dst[t] : 0.0;
-      dst[t] = v;
-      ss = fma(v, v, ss);
+      part[w][t] = acc;
     }
   }
-  ss = warp_sum_f64(ss);
-  if (norms && lane == 0) norms[static_cast<size_t>(h) * C + c] = ss;
+  __syncthreads();
+  double* dst = out + (static_cast<size_t>(h) * C + c) * D;
+  double ss = 0.0;
+  for (int t = threadIdx.x; t < D; t += blockDim.x) {
+    double v;
+    if (n > 0) {
+      double s = part[0][t];
+      for (int ww = 1; ww < kMeanWarps; ++ww) s += part[ww][t];
+      v = s / static_cast<double>(n);
+    } else {
+      v = keep_prev ? dst[t] : 0.0;
+    }
+    dst[t] = v;
+    ss = fma(v, v, ss);
+  }
+  if (norms) {
+    __shared__ double red[kMeanWarps];
+    ss = warp_sum_f64(ss);
+    if (lane == 0) red[w] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double s = red[0];
+      for (int ww = 1; ww < kMeanWarps; ++ww) s += red[ww];
+      norms[static_cast<size_t>(h) * C + c] = s;
+    }
+  }
 }
 
 // W_g = G qbar_g, c_g = qbar_g^T G qbar_g (fp64, fixed-order reduction).
@@ -457,8 +481,9 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx,
                               int off_stride, int C, int H, bool keep_prev, double* out,
                               double* norms, const int32_t* skip, int skip_stride,
                               cudaStream_t st) {
-  dim3 grid((C + 3) / 4, H);
-  group_mean_kernel<<<grid, 128, 0, st>>>(X, x_kind, hsx, ldx, D, perm, perm_stride, off,
+  if (D > kMeanMaxD) return cudaErrorInvalidValue;
+  dim3 grid(C, H);
+  group_mean_kernel<<<grid, kMeanWarps * 32, 0, st>>>(X, x_kind, hsx, ldx, D, perm, perm_stride, off,
                                           off_stride, C, keep_prev, out, norms, skip,
                                           skip_stride);
   return cudaGetLastError();

@@ -39,7 +39,9 @@ class Stats(ctypes.Structure):
                 ("key_passes", ctypes.c_int32 * MAX_HEADS),
                 ("query_passes", ctypes.c_int32 * MAX_HEADS),
                 ("pairs_sparse", ctypes.c_int64 * MAX_HEADS),
-                ("pairs_exec", ctypes.c_int64 * MAX_HEADS)]
+                ("pairs_exec", ctypes.c_int64 * MAX_HEADS),
+                ("recheck_rows", ctypes.c_int64 * 2),
+                ("eig_sweeps", ctypes.c_int32 * 2)]
 
 
 class SparsePRError(RuntimeError):
@@ -199,7 +201,8 @@ def sparsepr_read_stats(ws) -> dict:
     H = max(0, min(s.H, MAX_HEADS))
     return dict(status=int(s.status), H=H, key_passes=list(s.key_passes[:H]),
                 query_passes=list(s.query_passes[:H]), pairs_sparse=list(s.pairs_sparse[:H]),
-                pairs_exec=list(s.pairs_exec[:H]))
+                pairs_exec=list(s.pairs_exec[:H]), recheck_rows=list(s.recheck_rows),
+                eig_sweeps=list(s.eig_sweeps))
 
 
 # ---- buffers + the whole call ----------------------------------------------
