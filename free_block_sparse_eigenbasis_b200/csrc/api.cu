@@ -195,8 +195,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
   SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, st));
   SPR_TRY(launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st));
-  SPR_TRY(launch_jacobi(mk, H, d, evl, evc, c.stats, 0, st));
-  SPR_TRY(launch_top_eig_projector(evl, evc, H, d, e, wk, st));
+  SPR_TRY(launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st));
+  SPR_TRY(launch_scale_columns(evl, evc, H, d, e, wk, st));
   SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
   const long long hs_z = static_cast<long long>(Nv) * e;
   SPR_TRY(launch_gather_init(z, kXf64, hs_z, e, e, init_k, Ck, H, mu, mun, st));
@@ -507,8 +507,17 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
                             static_cast<long long>(d) * d, 0, st));
     double* evl = at<double>(ws, L.eval);
     double* evc = at<double>(ws, L.evec);
-    SPR_TRY(launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st));
-    SPR_TRY(launch_project_map(bmat, bvec, evl, evc, H, d, c.p.r, bp32, bv32, fit, st));
+    // leading-r right singular vectors of R = top-r eigenvectors of R^T R
+    const double* vr = evc;
+    if (c.p.r <= 32) {
+      SPR_TRY(launch_sym_eigs(rtr, H, d, c.p.r, evl, evc, at<double>(ws, L.eigscr), st));
+    } else {
+      double* sel = gram;  // free after the ridge solve: [H, d, r] selected vectors
+      SPR_TRY(launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st));
+      SPR_TRY(launch_top_eig_projector(evl, evc, H, d, c.p.r, sel, false, st));
+      vr = sel;
+    }
+    SPR_TRY(launch_project_map(bmat, bvec, vr, H, d, c.p.r, bp32, bv32, fit, st));
   } else {
     SPR_TRY(cudaMemsetAsync(bp32, 0, static_cast<size_t>(H) * d * d * 4, st));
     SPR_TRY(cudaMemsetAsync(bv32, 0, static_cast<size_t>(H) * d * 4, st));

@@ -1,0 +1,325 @@
+// Leading eigenpairs of the small symmetric PSD matrices of the path, in fp64:
+// the sampled-query metric M_K ("Partition the Support, Reconstruct the
+// Residual", 2.A: k-means on the eigenvectors of M_K) and the probe residual
+// Gram R^T R (2.B: leading singular vectors of the probe residuals).
+//
+// Textbook dense symmetric eigensolver, specialised to "top ne of d":
+//   1. Householder reduction to tridiagonal form, A = Q T Q^T with
+//      Q = H_0 H_1 ... H_{d-3}, H_k = I - tau_k v_k v_k^T (Golub & Van Loan,
+//      Matrix Computations, sec. 8.3.1), one CTA per matrix in shared memory;
+//   2. the ne largest eigenvalues of T by bisection on Sturm-sequence counts
+//      (sec. 8.4.1), one thread per eigenvalue;
+//   3. their eigenvectors by inverse iteration on T - lambda I with
+//      partial-pivoting tridiagonal LU (sec. 8.2.2 / 7.6.1), with
+//      Gram-Schmidt inside clusters of close eigenvalues after each step;
+//   4. back-transformation u = Q y, one warp per vector.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+namespace {
+
+constexpr int kTriThreads = 512;
+constexpr int kInvIters = 3;
+
+// Scratch per matrix (fp64): hv [D][D] Householder vectors (column k holds
+// v_k at rows k+1.., v_k[0] = 1), tau [D], dg [D], od [D].
+template <int D>
+__global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in, double* scratch) {
+  extern __shared__ double tsm[];
+  double* A = tsm;              // [D*D] full symmetric
+  double* v = A + D * D;        // [D]
+  double* w = v + D;            // [D]
+  __shared__ double red[kTriThreads / 32];
+  __shared__ double bc[4];
+  const int h = blockIdx.x;
+  const double* Ah = A_in + static_cast<size_t>(h) * D * D;
+  double* hv = scratch + static_cast<size_t>(h) * (D * D + 3 * D);
+  double* tau = hv + D * D;
+  double* dg = tau + D;
+  double* od = dg + D;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  for (int t = tid; t < D * D; t += blockDim.x) A[t] = Ah[t];
+  __syncthreads();
+  auto block_sum = [&](double x) -> double {
+    x = warp_sum_f64(x);
+    if (lane == 0) red[wid] = x;
+    __syncthreads();
+    if (tid == 0) {
+      double s = 0.0;
+      for (int i = 0; i < kTriThreads / 32; ++i) s += red[i];
+      bc[3] = s;
+    }
+    __syncthreads();
+    const double s = bc[3];
+    __syncthreads();
+    return s;
+  };
+  for (int k = 0; k < D - 2; ++k) {
+    const int n1 = D - k - 1;  // length of v (rows k+1 .. D-1)
+    double x2 = 0.0;
+    for (int i = k + 2 + tid; i < D; i += blockDim.x) {
+      const double a = A[i * D + k];
+      x2 += a * a;
+    }
+    x2 = block_sum(x2);
+    const double alpha = A[(k + 1) * D + k];
+    if (x2 == 0.0) {  // column already reduced: H_k = I
+      if (tid == 0) {
+        tau[k] = 0.0;
+        od[k] = alpha;
+      }
+      for (int i = tid; i < n1; i += blockDim.x) hv[(k + 1 + i) * D + k] = (i == 0) ? 1.0 : 0.0;
+      __syncthreads();
+      continue;
+    }
+    const double beta = -copysign(sqrt(alpha * alpha + x2), alpha);
+    const double tk = (beta - alpha) / beta;
+    const double scl = 1.0 / (alpha - beta);
+    for (int i = tid; i < n1; i += blockDim.x) {
+      const double vi = (i == 0) ? 1.0 : A[(k + 1 + i) * D + k] * scl;
+      v[i] = vi;
+      hv[(k + 1 + i) * D + k] = vi;
+    }
+    if (tid == 0) {
+      tau[k] = tk;
+      od[k] = beta;
+    }
+    __syncthreads();
+    // p = tau A22 v: 4 threads per row, fixed combination order
+    {
+      const int r = tid >> 2, part = tid & 3;
+      double s = 0.0;
+      if (r < n1) {
+        const double* row = A + (k + 1 + r) * D + (k + 1);
+        for (int c = part; c < n1; c += 4) s = fma(row[c], v[c], s);
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (r < n1 && part == 0) w[r] = tk * s;
+    }
+    __syncthreads();
+    double pv = 0.0;
+    for (int i = tid; i < n1; i += blockDim.x) pv += w[i] * v[i];
+    pv = block_sum(pv);
+    const double kk = -0.5 * tk * pv;
+    for (int i = tid; i < n1; i += blockDim.x) w[i] += kk * v[i];
+    __syncthreads();
+    // A22 -= v w^T + w v^T
+    for (int t = tid; t < n1 * n1; t += blockDim.x) {
+      const int r = t / n1, c = t % n1;
+      A[(k + 1 + r) * D + (k + 1 + c)] -= v[r] * w[c] + w[r] * v[c];
+    }
+    __syncthreads();
+  }
+  for (int i = tid; i < D; i += blockDim.x) dg[i] = A[i * D + i];
+  if (tid == 0) {
+    od[D - 2] = A[(D - 1) * D + (D - 2)];
+    od[D - 1] = 0.0;
+    tau[D - 2] = 0.0;
+    tau[D - 1] = 0.0;
+  }
+}
+
+// Number of eigenvalues of T below x (Sturm sequence of the LDL^T pivots).
+template <int D>
+__device__ int sturm_count(const double* dg, const double* e2, double x, double pivmin) {
+  int cnt = 0;
+  double q = dg[0] - x;
+  if (fabs(q) < pivmin) q = -pivmin;
+  cnt += (q < 0.0);
+#pragma unroll 1
+  for (int i = 1; i < D; ++i) {
+    q = dg[i] - x - e2[i - 1] / q;
+    if (fabs(q) < pivmin) q = -pivmin;
+    cnt += (q < 0.0);
+  }
+  return cnt;
+}
+
+// Solve (T - lam I) y = b in place (b <- y) with a partial-pivoting LU of
+// the tridiagonal system; a, dl, du, du2 are thread-private work arrays.
+template <int D>
+__device__ void tri_solve(const double* dg, const double* od, double lam, double tiny, double* a,
+                          double* dl, double* du, double* du2, int* pv, double* b) {
+  for (int i = 0; i < D; ++i) a[i] = dg[i] - lam;
+  for (int i = 0; i < D - 1; ++i) {
+    dl[i] = od[i];
+    du[i] = od[i];
+    du2[i] = 0.0;
+  }
+#pragma unroll 1
+  for (int i = 0; i < D - 1; ++i) {
+    if (fabs(a[i]) >= fabs(dl[i])) {
+      if (a[i] == 0.0) a[i] = tiny;
+      const double f = dl[i] / a[i];
+      dl[i] = f;
+      a[i + 1] -= f * du[i];
+      pv[i] = 0;
+    } else {
+      const double f = a[i] / dl[i];
+      a[i] = dl[i];
+      dl[i] = f;
+      const double t = du[i];
+      du[i] = a[i + 1];
+      a[i + 1] = t - f * a[i + 1];
+      if (i < D - 2) {
+        du2[i] = du[i + 1];
+        du[i + 1] = -f * du[i + 1];
+      }
+      pv[i] = 1;
+    }
+  }
+  if (a[D - 1] == 0.0) a[D - 1] = tiny;
+  // L solve
+#pragma unroll 1
+  for (int i = 0; i < D - 1; ++i) {
+    if (pv[i] == 0) {
+      b[i + 1] -= dl[i] * b[i];
+    } else {
+      const double t = b[i];
+      b[i] = b[i + 1];
+      b[i + 1] = t - dl[i] * b[i];
+    }
+  }
+  // U solve
+  b[D - 1] /= a[D - 1];
+  b[D - 2] = (b[D - 2] - du[D - 2] * b[D - 1]) / a[D - 2];
+#pragma unroll 1
+  for (int i = D - 3; i >= 0; --i) b[i] = (b[i] - du[i] * b[i + 1] - du2[i] * b[i + 2]) / a[i];
+}
+
+constexpr int kEigThreads = 256;
+
+// One CTA per matrix, ne <= 32 eigenpairs (largest first): bisection and
+// inverse iteration by thread t, clustered Gram-Schmidt by warp 0, then
+// back-transformation by warp t % 8. Writes evals [H, ne] and evecs [H, D, ne].
+template <int D>
+__global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scratch, int ne,
+                                                       double* evals, double* evecs,
+                                                       double* work) {
+  __shared__ double dg[D], od[D], e2[D];
+  __shared__ double lam[32];
+  __shared__ double Y[32][D + 1];  // padded: thread t walks row t
+  __shared__ double tnorm;
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const double* hv = scratch + static_cast<size_t>(h) * (D * D + 3 * D);
+  const double* tau = hv + D * D;
+  for (int i = tid; i < D; i += blockDim.x) {
+    dg[i] = tau[D + i];
+    od[i] = tau[2 * D + i];
+  }
+  __syncthreads();
+  for (int i = tid; i < D; i += blockDim.x) e2[i] = (i < D - 1) ? od[i] * od[i] : 0.0;
+  if (tid == 0) {
+    double m = 0.0;
+    for (int i = 0; i < D; ++i)
+      m = fmax(m, fabs(dg[i]) + (i > 0 ? fabs(od[i - 1]) : 0.0) + (i < D - 1 ? fabs(od[i]) : 0.0));
+    tnorm = m;
+  }
+  __syncthreads();
+  const double eps = 1.1102230246251565e-16;
+  double emax2 = 0.0;
+  for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
+  const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
+  // bisection: thread t finds the eigenvalue of ascending index D-1-t
+  if (tid < ne) {
+    const int m = D - 1 - tid;
+    double lo = -tnorm - 1.0, hi = tnorm + 1.0;
+    for (int it = 0; it < 200; ++it) {
+      const double mid = 0.5 * (lo + hi);
+      if (hi - lo <= 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin || mid == lo || mid == hi) break;
+      if (sturm_count<D>(dg, e2, mid, pivmin) <= m)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    lam[tid] = 0.5 * (lo + hi);
+  }
+  __syncthreads();
+  // inverse iteration from a fixed, index-dependent start vector
+  double* wk = work + (static_cast<size_t>(h) * 32 + tid) * (5 * D);
+  int* pv = reinterpret_cast<int*>(wk + 4 * D);
+  const double tiny = eps * fmax(tnorm, 1e-300);
+  if (tid < ne)
+    for (int i = 0; i < D; ++i) Y[tid][i] = 1.0 + 0.5 * sin(0.7 * (i + 1) * (tid + 1));
+  const double ortol = 1e-3 * tnorm;
+  for (int it = 0; it < kInvIters; ++it) {
+    if (tid < ne) {
+      double* b = Y[tid];
+      tri_solve<D>(dg, od, lam[tid], tiny, wk, wk + D, wk + 2 * D, wk + 3 * D, pv, b);
+      double s = 0.0;
+      for (int i = 0; i < D; ++i) s = fma(b[i], b[i], s);
+      const double inv = 1.0 / sqrt(s);
+      for (int i = 0; i < D; ++i) b[i] *= inv;
+    }
+    __syncthreads();
+    // Gram-Schmidt against earlier vectors of the same cluster, in rank order
+    if (wid == 0) {
+      for (int t = 1; t < ne; ++t) {
+        for (int s = t - 1; s >= 0; --s) {
+          if (fabs(lam[s] - lam[s + 1]) > ortol) break;  // cluster boundary
+          double dot = 0.0;
+          for (int i = lane; i < D; i += 32) dot = fma(Y[s][i], Y[t][i], dot);
+          dot = warp_sum_f64(dot);
+          for (int i = lane; i < D; i += 32) Y[t][i] -= dot * Y[s][i];
+          __syncwarp();
+        }
+        double nn = 0.0;
+        for (int i = lane; i < D; i += 32) nn = fma(Y[t][i], Y[t][i], nn);
+        nn = warp_sum_f64(nn);
+        const double inv = 1.0 / sqrt(nn);
+        for (int i = lane; i < D; i += 32) Y[t][i] *= inv;
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+  }
+  // back-transformation: u = H_0 (H_1 (... H_{D-3} y)), warp w owns vectors w, w + 8, ...
+  for (int t = wid; t < ne; t += kEigThreads / 32) {
+    double* y = Y[t];
+    for (int k = D - 3; k >= 0; --k) {
+      const double tk = tau[k];
+      if (tk == 0.0) continue;
+      double dot = 0.0;
+      for (int i = k + 1 + lane; i < D; i += 32) dot = fma(hv[i * D + k], y[i], dot);
+      dot = warp_sum_f64(dot) * tk;
+      for (int i = k + 1 + lane; i < D; i += 32) y[i] -= dot * hv[i * D + k];
+      __syncwarp();
+    }
+    for (int i = lane; i < D; i += 32)
+      evecs[(static_cast<size_t>(h) * D + i) * ne + t] = y[i];
+    if (lane == 0) evals[static_cast<size_t>(h) * ne + t] = lam[t];
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const double* A, int H, int ne, double* evals, double* evecs,
+                     double* scratch, double* work, cudaStream_t st) {
+  const size_t shb = (static_cast<size_t>(D) * D + 2 * D) * 8;
+  cudaError_t e = cudaFuncSetAttribute(tridiag_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(shb));
+  if (e != cudaSuccess) return e;
+  tridiag_kernel<D><<<H, kTriThreads, shb, st>>>(A, scratch);
+  tri_eig_kernel<D><<<H, kEigThreads, 0, st>>>(scratch, ne, evals, evecs, work);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t sym_eigs_scratch_doubles(int H, int d) {
+  return static_cast<size_t>(H) * (static_cast<size_t>(d) * d + 3 * d) +
+         static_cast<size_t>(H) * 32 * 5 * d;
+}
+
+cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals, double* evecs,
+                            double* scratch, cudaStream_t st) {
+  if (ne < 1 || ne > 32 || ne > d) return cudaErrorInvalidValue;
+  double* work = scratch + static_cast<size_t>(H) * (static_cast<size_t>(d) * d + 3 * d);
+  if (d == 128) return launch_d<128>(A, H, ne, evals, evecs, scratch, work, st);
+  if (d == 64) return launch_d<64>(A, H, ne, evals, evecs, scratch, work, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace spr

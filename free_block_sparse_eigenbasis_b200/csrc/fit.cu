@@ -174,46 +174,36 @@ __global__ void ridge_solve_kernel(const double* gram, int d, double* bmat, doub
   }
 }
 
-// P_r = sum over the r largest eigenpairs of R^T R of v v^T; B' = B P_r,
-// b' = b P_r (fp64), stored fp32 for the correction (and fp64 if asked).
-__global__ void project_map_kernel(const double* bmat, const double* bvec, const double* eval,
-                                   const double* evec, int d, int r, float* bp32, float* bv32,
-                                   double* fit_out) {
-  extern __shared__ double psm2[];
-  double* Pr = psm2;  // [d][d]
-  __shared__ int sel[128];
-  const int h = blockIdx.x;
-  const double* ev = eval + static_cast<size_t>(h) * d;
-  const double* V = evec + static_cast<size_t>(h) * d * d;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    const double lj = ev[j];
-    int rank = 0;
-    for (int i = 0; i < d; ++i) rank += (ev[i] > lj) || (ev[i] == lj && i < j);
-    sel[j] = rank < r;
-  }
+// Restriction to the residual subspace: with V_r [d, r] the leading right
+// singular vectors of R, B' = (B V_r) V_r^T and b' = (b V_r) V_r^T (fp64),
+// stored fp32 for the correction (and fp64 if asked). One CTA per row of B'
+// (row d is the intercept).
+__global__ void project_map_kernel(const double* bmat, const double* bvec, const double* vr,
+                                   int d, int r, float* bp32, float* bv32, double* fit_out) {
+  __shared__ double rw[128], T[128];
+  const int a = blockIdx.x, h = blockIdx.y;
+  const double* row = (a < d) ? bmat + (static_cast<size_t>(h) * d + a) * d
+                              : bvec + static_cast<size_t>(h) * d;
+  const double* V = vr + static_cast<size_t>(h) * d * r;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) rw[k] = row[k];
   __syncthreads();
-  for (int t = threadIdx.x; t < d * d; t += blockDim.x) {
-    const int a = t / d, b = t % d;
+  for (int t = threadIdx.x; t < r; t += blockDim.x) {
     double s = 0.0;
-    for (int j = 0; j < d; ++j)
-      if (sel[j]) s += V[static_cast<size_t>(a) * d + j] * V[static_cast<size_t>(b) * d + j];
-    Pr[t] = s;
+    for (int k = 0; k < d; ++k) s = fma(rw[k], V[static_cast<size_t>(k) * r + t], s);
+    T[t] = s;
   }
   __syncthreads();
-  const double* B = bmat + static_cast<size_t>(h) * d * d;
   const int col = threadIdx.x;
   if (col < d) {
-    for (int a = 0; a < d; ++a) {
-      double s = 0.0;
-      for (int k = 0; k < d; ++k) s += B[static_cast<size_t>(a) * d + k] * Pr[k * d + col];
+    double s = 0.0;
+    for (int t = 0; t < r; ++t) s = fma(T[t], V[static_cast<size_t>(col) * r + t], s);
+    if (a < d) {
       bp32[(static_cast<size_t>(h) * d + a) * d + col] = static_cast<float>(s);
       if (fit_out) fit_out[static_cast<size_t>(h) * (d * d + d) + a * d + col] = s;
+    } else {
+      bv32[static_cast<size_t>(h) * d + col] = static_cast<float>(s);
+      if (fit_out) fit_out[static_cast<size_t>(h) * (d * d + d) + d * d + col] = s;
     }
-    const double* b = bvec + static_cast<size_t>(h) * d;
-    double s = 0.0;
-    for (int k = 0; k < d; ++k) s += b[k] * Pr[k * d + col];
-    bv32[static_cast<size_t>(h) * d + col] = static_cast<float>(s);
-    if (fit_out) fit_out[static_cast<size_t>(h) * (d * d + d) + d * d + col] = s;
   }
 }
 
@@ -315,15 +305,10 @@ cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double*
   return cudaGetLastError();
 }
 
-cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* eval,
-                               const double* evec, int H, int d, int r, float* bp32, float* bv32,
-                               double* fit_out, cudaStream_t st) {
-  const size_t shb = static_cast<size_t>(d) * d * 8;
-  cudaError_t e = cudaFuncSetAttribute(project_map_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(shb));
-  if (e != cudaSuccess) return e;
-  project_map_kernel<<<H, 128, shb, st>>>(bmat, bvec, eval, evec, d, r, bp32, bv32, fit_out);
+cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* vr, int H,
+                               int d, int r, float* bp32, float* bv32, double* fit_out,
+                               cudaStream_t st) {
+  project_map_kernel<<<dim3(d + 1, H), 128, 0, st>>>(bmat, bvec, vr, d, r, bp32, bv32, fit_out);
   return cudaGetLastError();
 }
 

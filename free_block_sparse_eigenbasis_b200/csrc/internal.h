@@ -115,10 +115,20 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st);
 // symmetric -> eval [H, d], evec [H, d, d] (eigenvectors in columns).
 cudaError_t launch_jacobi(const double* A, int H, int d, double* eval, double* evec,
                           DeviceStats* stats, int which, cudaStream_t st);
-// wk[h, a, t] = evec[h, a, j_t] * sqrt(max(eval_j_t, 0)) for the e largest
-// eigenvalues (t = rank, ties to the lower index).
+// wk[h, a, t] = evec[h, a, j_t] (* sqrt(max(eval_j_t, 0)) if sqrt_scale) for
+// the e largest eigenvalues (t = rank, ties to the lower index).
 cudaError_t launch_top_eig_projector(const double* eval, const double* evec, int H, int d, int e,
-                                     double* wk, cudaStream_t st);
+                                     double* wk, bool sqrt_scale, cudaStream_t st);
+// wk[h, a, t] = vecs[h, a, t] * sqrt(max(vals[h, t], 0)), t < e.
+cudaError_t launch_scale_columns(const double* vals, const double* vecs, int H, int d, int e,
+                                 double* wk, cudaStream_t st);
+
+// ---- eigen.cu: top-ne eigenpairs (ne <= 32) by tridiagonal reduction,
+// bisection and inverse iteration ---------------------------------------------
+size_t sym_eigs_scratch_doubles(int H, int d);
+// evals [H, ne] descending, evecs [H, d, ne].
+cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals, double* evecs,
+                            double* scratch, cudaStream_t st);
 
 // ---- permute.cu ------------------------------------------------------------
 cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, int H, int N,
@@ -168,9 +178,10 @@ cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const
                                    cudaStream_t st);
 cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
                                const double* means, DeviceStats* stats, cudaStream_t st);
-cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* eval,
-                               const double* evec, int H, int d, int r, float* bp32, float* bv32,
-                               double* fit_out, cudaStream_t st);
+// B' = (B V_r) V_r^T, b' = (b V_r) V_r^T with vr [H, d, r].
+cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* vr, int H,
+                               int d, int r, float* bp32, float* bv32, double* fit_out,
+                               cudaStream_t st);
 cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t* probes,
                            const int32_t* perm_q, const float* bp32, const float* bv32, int H,
                            int N, int M, int d, void* out, bool out_bf16, cudaStream_t st);

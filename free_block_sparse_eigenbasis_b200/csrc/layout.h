@@ -28,6 +28,7 @@ struct Layout {
   size_t mk;       // [H, d, d] f64 (M_K, later the probe residual Gram R^T R)
   size_t evec;     // [H, d, d] f64 Jacobi eigenvectors (columns)
   size_t eval;     // [H, d] f64 Jacobi eigenvalues
+  size_t eigscr;   // tridiagonal eigensolver scratch: [H, d*d + 3d] + [H, 32, 5d] f64
   size_t wk;       // [H, d, e] f64 key projector U_e L_e^{1/2}
   size_t z;        // [H, Nv, e] f64 key coordinates
   size_t mu;       // [H, Ck, e] f64 key centroids
@@ -126,6 +127,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->mk = take(H * d * d * 8);
   L->evec = take(H * d * d * 8);
   L->eval = take(H * d * 8);
+  L->eigscr = take((H * (d * d + 3 * d) + H * 32 * 5 * d) * 8);
   L->wk = take(H * d * e * 8);
   L->z = take(H * Nv * e * 8);
   L->mu = take(H * Ck * e * 8);

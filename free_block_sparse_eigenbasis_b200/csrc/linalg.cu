@@ -167,10 +167,10 @@ __global__ void __launch_bounds__(kJacobiThreads) jacobi_kernel(const double* A_
   if (threadIdx.x == 0 && stats) atomicMax(&stats->eig_sweeps[which], sweep);
 }
 
-// wk[h, a, t] = evec[h, a, j] * sqrt(max(lambda_j, 0)) where j has rank t in
-// descending eigenvalue order (ties to the lower index), t < e.
+// wk[h, a, t] = evec[h, a, j] (* sqrt(max(lambda_j, 0))) where j has rank t
+// in descending eigenvalue order (ties to the lower index), t < e.
 __global__ void top_eig_projector_kernel(const double* eval, const double* evec, int d, int e,
-                                         double* wk) {
+                                         double* wk, int sqrt_scale) {
   const int h = blockIdx.x, j = threadIdx.x;
   if (j >= d) return;
   const double* ev = eval + static_cast<size_t>(h) * d;
@@ -181,10 +181,20 @@ __global__ void top_eig_projector_kernel(const double* eval, const double* evec,
     rank += (li > lj) || (li == lj && i < j);
   }
   if (rank >= e) return;
-  const double sc = sqrt(fmax(lj, 0.0));
+  const double sc = sqrt_scale ? sqrt(fmax(lj, 0.0)) : 1.0;
   const double* V = evec + static_cast<size_t>(h) * d * d;
   for (int a = 0; a < d; ++a)
     wk[(static_cast<size_t>(h) * d + a) * e + rank] = V[static_cast<size_t>(a) * d + j] * sc;
+}
+
+__global__ void scale_columns_kernel(const double* vals, const double* vecs, int d, int e,
+                                     double* wk) {
+  const int h = blockIdx.x;
+  for (int t = threadIdx.x; t < d * e; t += blockDim.x) {
+    const int c = t % e;
+    wk[static_cast<size_t>(h) * d * e + t] =
+        vecs[static_cast<size_t>(h) * d * e + t] * sqrt(fmax(vals[static_cast<size_t>(h) * e + c], 0.0));
+  }
 }
 
 template <int D>
@@ -211,8 +221,14 @@ cudaError_t launch_jacobi(const double* A, int H, int d, double* eval, double* e
 }
 
 cudaError_t launch_top_eig_projector(const double* eval, const double* evec, int H, int d, int e,
-                                     double* wk, cudaStream_t st) {
-  top_eig_projector_kernel<<<H, 128, 0, st>>>(eval, evec, d, e, wk);
+                                     double* wk, bool sqrt_scale, cudaStream_t st) {
+  top_eig_projector_kernel<<<H, 128, 0, st>>>(eval, evec, d, e, wk, sqrt_scale ? 1 : 0);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale_columns(const double* vals, const double* vecs, int H, int d, int e,
+                                 double* wk, cudaStream_t st) {
+  scale_columns_kernel<<<H, 256, 0, st>>>(vals, vecs, d, e, wk);
   return cudaGetLastError();
 }
 
