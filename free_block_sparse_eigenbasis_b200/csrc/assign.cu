@@ -18,22 +18,33 @@
 // certain label; every other row is appended to a list and decided again in
 // fp64 by recheck_kernel.
 //
-// One persistent CTA per (slice of row tiles, head): all centroid planes stay
-// in shared memory, row tiles of 128 stream through a 2-stage TMA ring, and
+// Persistent CTAs (at most one per SM) each take a contiguous range of the
+// row tiles of all heads, ordered head-major; the centroid planes of the
+// current head stay in shared memory and are reloaded when the range crosses
+// into the next head. Row tiles of 128 stream through a 2-stage TMA ring;
 // the 128 x (<=256) accumulator of each centroid chunk alternates between two
-// TMEM buffers so that the epilogue of one chunk overlaps the MMAs of the next.
+// TMEM buffers, so the epilogue of one chunk overlaps the MMAs of the next.
+// The epilogue is four groups of four warps: every group sees all 128 rows
+// (warp w reads TMEM lanes 32 (w % 4) ..) and a quarter of each chunk's
+// columns; the groups' partial minima meet in shared memory at the end of a
+// tile.
 #include "common.cuh"
 #include "internal.h"
 
 namespace spr {
 namespace {
 
-constexpr int kAsThreads = 160;  // warps 0-3 epilogue (thread = row), warp 4: TMA + MMA
-constexpr int kAsChunk = 256;    // centroids per accumulator chunk
+constexpr int kAsGroups = 4;                 // epilogue column groups
+constexpr int kAsEpi = kAsGroups * kTileM;   // epilogue threads (thread = row within a group)
+constexpr int kAsThreads = kAsEpi + 32;      // + one warp: lane 0 TMA, lane 1 MMA
+constexpr int kAsChunk = 256;                // centroids per accumulator chunk
 constexpr uint32_t kAsTmemCols = 512;
+constexpr size_t kAsMinSmem = 120 * 1024;    // keeps one CTA (and one TMEM owner) per SM
+// named barriers of the epilogue threads (0 is __syncthreads)
+constexpr int kBarXchFull = 1, kBarXchFree = 2, kBarHead = 3;
 
 struct AsBars {
-  uint64_t b_full;
+  uint64_t b_full, b_empty;
   uint64_t a_full[2], a_empty[2];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_idle;
@@ -50,7 +61,7 @@ struct AsParams {
   int n;          // rows per head
   int a_head;     // row offset between heads in the A maps
   int b_head;     // row offset between heads in the B maps (= Cpad)
-  int Cpad;       // centroids per head, padded to a multiple of 32
+  int Cpad;       // centroids per head, padded to a multiple of 16
   int nA, nB;     // planes
   int npairs;
   int pairs[6];   // (plane of x) * 4 + (plane of y)
@@ -59,6 +70,7 @@ struct AsParams {
   int Kt;         // accumulated terms per dot product
   float res;      // bound on the plane-split residual and dropped plane products, relative
   int tiles_per_head;
+  int H;
   const float* cvals;  // [H, Cpad] fp32 offsets (+inf on padding)
   const float* xnorm;  // [H, n] |x_i| (rounded up)
   const float* hmax;   // [H, 2] Y, C (rounded up)
@@ -81,17 +93,38 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, bool sw32) {
   return d;
 }
 
+// Walks the head segments of a CTA's tile range [g, g1): calls f(h, t0, t1)
+// for every head that has not converged, with its tiles t0..t1-1.
+template <typename F>
+__device__ __forceinline__ void for_segments(const AsParams& p, int g, int g1, F&& f) {
+  while (g < g1) {
+    const int h = g / p.tiles_per_head;
+    const int ge = min(g1, (h + 1) * p.tiles_per_head);
+    if (!p.flags[h * 4 + p.flag_base + 1]) f(h, g - h * p.tiles_per_head, ge - h * p.tiles_per_head);
+    g = ge;
+  }
+}
+
+// running best / second best of one chain; columns of a chain ascend, so
+// equal values keep the lower index
+__device__ __forceinline__ void chain_step(float dd, int j, float& b1, float& b2, int& bi) {
+  const bool lt = dd < b1;
+  b2 = fminf(b2, fmaxf(b1, dd));
+  bi = lt ? j : bi;
+  b1 = fminf(b1, dd);
+}
+
 __global__ void __launch_bounds__(kAsThreads, 1)
     argmin_tc_kernel(const __grid_constant__ AsMaps maps, const AsParams p) {
-  const int h = blockIdx.y;
-  int32_t* fl = p.flags + h * 4;
-  if (fl[p.flag_base + 1]) return;  // converged head
   const int row_bytes = p.sw32 ? 32 : 128;
   const int slab_a = kTileM * row_bytes;                // one atom of a 128-row tile
   const int a_stage = p.nA * p.atoms * slab_a;
   const int slab_b = p.Cpad * row_bytes;                // one atom of all centroids
   const int b_bytes = p.nB * p.atoms * slab_b;
   const int nchunks = (p.Cpad + kAsChunk - 1) / kAsChunk;
+  const int T = p.H * p.tiles_per_head;
+  const int g0 = static_cast<int>(static_cast<long long>(blockIdx.x) * T / gridDim.x);
+  const int g1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * T / gridDim.x);
 
   extern __shared__ uint8_t as_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(as_raw) + 1023) &
@@ -99,23 +132,25 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   uint8_t* Bs = sm;
   uint8_t* As = sm + ((b_bytes + 1023) & ~1023);
   float* cs = reinterpret_cast<float*>(As + 2 * a_stage);
-  AsBars* bars = reinterpret_cast<AsBars*>(cs + p.Cpad);
+  float* xd1 = cs + p.Cpad;                 // [kAsGroups - 1][128]
+  float* xd2 = xd1 + (kAsGroups - 1) * kTileM;
+  int* xi1 = reinterpret_cast<int*>(xd2 + (kAsGroups - 1) * kTileM);
+  AsBars* bars = reinterpret_cast<AsBars*>(xi1 + (kAsGroups - 1) * kTileM);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->b_full, 1);
+    mbar_init(&bars->b_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->a_full[s], 1);
       mbar_init(&bars->a_empty[s], 1);
       mbar_init(&bars->acc_full[s], 1);
-      mbar_init(&bars->acc_empty[s], kTileM);
+      mbar_init(&bars->acc_empty[s], kAsEpi);
     }
     mbar_init(&bars->mma_idle, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
-  for (int j = threadIdx.x; j < p.Cpad; j += blockDim.x)
-    cs[j] = p.cvals[static_cast<size_t>(h) * p.Cpad + j];
   if (warp == 0) {
     tmem_alloc(&bars->tmem_base, kAsTmemCols);
     tmem_relinquish();
@@ -125,172 +160,203 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
-  // this CTA's row tiles: t = blockIdx.x + u * gridDim.x
-  const int ntile = (p.tiles_per_head - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
-                    static_cast<int>(gridDim.x);
   const int inner = p.sw32 ? 16 : 64;
+  volatile int never = 0;
 
-  if (warp == 4) {
+  if (warp == kAsEpi / 32) {
     if (lane == 0) {
       // ----------------------------- TMA producer -----------------------------
-      mbar_arrive_expect_tx(&bars->b_full, b_bytes);
-      for (int pl = 0; pl < p.nB; ++pl)
-        for (int a = 0; a < p.atoms; ++a)
-          for (int r = 0; r < p.Cpad; r += 16)
-            tma_load_2d(Bs + (pl * p.atoms + a) * slab_b + r * row_bytes, &maps.b[pl],
-                        &bars->b_full, a * inner, h * p.b_head + r);
-      int issued = -1;
+      int u = 0, seg = 0;
       bool ok = true;
-      for (int u = 0; u < ntile; ++u) {
-        const int s = u & 1;
-        if (u >= 2 && !mbar_wait(&bars->a_empty[s], ((u - 2) >> 1) & 1, abort)) { ok = false; break; }
-        const int t = blockIdx.x + u * gridDim.x;
-        mbar_arrive_expect_tx(&bars->a_full[s], a_stage);
-        for (int pl = 0; pl < p.nA; ++pl)
+      for_segments(p, g0, g1, [&](int h, int t0, int t1) {
+        if (!ok) return;
+        if (seg > 0 && !mbar_wait(&bars->b_empty, (seg - 1) & 1, abort)) { ok = false; return; }
+        mbar_arrive_expect_tx(&bars->b_full, b_bytes);
+        for (int pl = 0; pl < p.nB; ++pl)
           for (int a = 0; a < p.atoms; ++a)
-            tma_load_2d(As + s * a_stage + (pl * p.atoms + a) * slab_a, &maps.a[pl],
-                        &bars->a_full[s], a * inner, h * p.a_head + t * kTileM);
-        issued = u;
-      }
-      volatile int never = 0;
-      if (!ok)
-        for (int u = max(0, issued - 1); u <= issued; ++u)
-          mbar_wait(&bars->a_full[u & 1], (u >> 1) & 1, &never);
-      mbar_wait(&bars->b_full, 0, &never);
+            for (int r = 0; r < p.Cpad; r += 16)
+              tma_load_2d(Bs + (pl * p.atoms + a) * slab_b + r * row_bytes, &maps.b[pl],
+                          &bars->b_full, a * inner, h * p.b_head + r);
+        ++seg;
+        for (int t = t0; t < t1; ++t) {
+          const int s = u & 1;
+          if (u >= 2 && !mbar_wait(&bars->a_empty[s], ((u - 2) >> 1) & 1, abort)) { ok = false; return; }
+          mbar_arrive_expect_tx(&bars->a_full[s], a_stage);
+          for (int pl = 0; pl < p.nA; ++pl)
+            for (int a = 0; a < p.atoms; ++a)
+              tma_load_2d(As + s * a_stage + (pl * p.atoms + a) * slab_a, &maps.a[pl],
+                          &bars->a_full[s], a * inner, h * p.a_head + t * kTileM);
+          ++u;
+        }
+      });
+      // let every load this thread issued land before the CTA exits
+      for (int x = max(0, u - 2); x < u; ++x) mbar_wait(&bars->a_full[x & 1], (x >> 1) & 1, &never);
+      if (seg > 0) mbar_wait(&bars->b_full, (seg - 1) & 1, &never);
     } else if (lane == 1) {
       // ------------------------------ MMA issuer ------------------------------
-      bool ok = mbar_wait(&bars->b_full, 0, abort);
       const uint32_t a_addr = smem_u32(As), b_addr = smem_u32(Bs);
-      int gc = 0;
-      for (int u = 0; u < ntile && ok; ++u) {
-        const int s = u & 1;
-        if (!mbar_wait(&bars->a_full[s], (u >> 1) & 1, abort)) { ok = false; break; }
-        for (int c = 0; c < nchunks; ++c, ++gc) {
-          const int buf = gc & 1;
-          if (gc >= 2 && !mbar_wait(&bars->acc_empty[buf], ((gc - 2) >> 1) & 1, abort)) {
-            ok = false;
-            break;
-          }
+      int u = 0, gc = 0, seg = 0;
+      bool ok = true;
+      for_segments(p, g0, g1, [&](int h, int t0, int t1) {
+        if (!ok) return;
+        if (!mbar_wait(&bars->b_full, seg & 1, abort)) { ok = false; return; }
+        ++seg;
+        for (int t = t0; t < t1; ++t, ++u) {
+          const int s = u & 1;
+          if (!mbar_wait(&bars->a_full[s], (u >> 1) & 1, abort)) { ok = false; return; }
           tc_fence_after();
-          const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
-          const uint32_t idesc = idesc_bf16(kTileM, N, 0);
-          const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * kAsChunk);
-          int first = 1;
-          for (int pi = 0; pi < p.npairs; ++pi) {
-            const int pa = p.pairs[pi] >> 2, pb = p.pairs[pi] & 3;
-            const int ksteps = p.sw32 ? 1 : p.atoms * 4;
-            for (int ks = 0; ks < ksteps; ++ks) {
-              const int atom = p.sw32 ? 0 : (ks >> 2);
-              const uint32_t koff = p.sw32 ? 0u : static_cast<uint32_t>((ks & 3) * 32);
-              const uint32_t aa = a_addr + s * a_stage + (pa * p.atoms + atom) * slab_a + koff;
-              const uint32_t ba = b_addr + (pb * p.atoms + atom) * slab_b +
-                                  c * kAsChunk * row_bytes + koff;
-              mma_bf16_ss(d_tmem, smem_desc(aa, p.sw32), smem_desc(ba, p.sw32), idesc,
-                          first ? 0u : 1u);
-              first = 0;
+          for (int c = 0; c < nchunks; ++c, ++gc) {
+            const int buf = gc & 1;
+            if (gc >= 2 && !mbar_wait(&bars->acc_empty[buf], ((gc - 2) >> 1) & 1, abort)) {
+              ok = false;
+              return;
             }
+            tc_fence_after();
+            const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
+            const uint32_t idesc = idesc_bf16(kTileM, N, 0);
+            const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * kAsChunk);
+            int first = 1;
+            for (int pi = 0; pi < p.npairs; ++pi) {
+              const int pa = p.pairs[pi] >> 2, pb = p.pairs[pi] & 3;
+              const int ksteps = p.sw32 ? 1 : p.atoms * 4;
+              for (int ks = 0; ks < ksteps; ++ks) {
+                const int atom = p.sw32 ? 0 : (ks >> 2);
+                const uint32_t koff = p.sw32 ? 0u : static_cast<uint32_t>((ks & 3) * 32);
+                const uint32_t aa = a_addr + s * a_stage + (pa * p.atoms + atom) * slab_a + koff;
+                const uint32_t ba = b_addr + (pb * p.atoms + atom) * slab_b +
+                                    c * kAsChunk * row_bytes + koff;
+                mma_bf16_ss(d_tmem, smem_desc(aa, p.sw32), smem_desc(ba, p.sw32), idesc,
+                            first ? 0u : 1u);
+                first = 0;
+              }
+            }
+            mma_commit(&bars->acc_full[buf]);
           }
-          mma_commit(&bars->acc_full[buf]);
+          mma_commit(&bars->a_empty[s]);
         }
-        mma_commit(&bars->a_empty[s]);
-      }
+        mma_commit(&bars->b_empty);  // the head's centroid planes may be replaced
+      });
       // all MMAs issued by this thread complete before tensor memory is freed
       mma_commit(&bars->mma_idle);
-      volatile int never = 0;
       mbar_wait(&bars->mma_idle, 0, &never);
     }
   } else {
-    // --------------------------- epilogue (thread = row) ---------------------------
-    const int r = threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>((warp * 32) << 16);
-    const float Y = p.hmax[h * 2 + 0], C = p.hmax[h * 2 + 1];
+    // ------------------- epilogue: group q, row r of the tile -------------------
+    // Every epilogue thread passes the same sequence of named barriers, also
+    // after a failed wait (it then skips the work), so none is left behind.
+    const int q = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const int et = threadIdx.x;  // 0 .. kAsEpi - 1
+    const uint32_t lane_base = static_cast<uint32_t>(((warp & 3) * 32) << 16);
     const float kt_term = static_cast<float>(p.Kt) * 2.384185791015625e-07f + p.res;
-    int gc = 0;
+    int gc = 0, nx = 0;
     bool ok = true;
-    for (int u = 0; u < ntile && ok; ++u) {
-      const int t = blockIdx.x + u * gridDim.x;
-      const int row = t * kTileM + r;
-      float b1[8], b2[8];
-      int bi[8];
+    for_segments(p, g0, g1, [&](int h, int t0, int t1) {
+      named_barrier_sync(kBarHead, kAsEpi);  // the previous head's offsets are no longer read
+      for (int j = et; j < p.Cpad; j += kAsEpi) cs[j] = p.cvals[static_cast<size_t>(h) * p.Cpad + j];
+      named_barrier_sync(kBarHead, kAsEpi);
+      const float Y = p.hmax[h * 2 + 0], C = p.hmax[h * 2 + 1];
+      int32_t* fl = p.flags + h * 4;
+      for (int t = t0; t < t1; ++t) {
+        float b1[4], b2[4];
+        int bi[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        b1[k] = INFINITY;
-        b2[k] = INFINITY;
-        bi[k] = 0x7fffffff;
-      }
-      for (int c = 0; c < nchunks; ++c, ++gc) {
-        const int buf = gc & 1;
-        if (!mbar_wait(&bars->acc_full[buf], (gc >> 1) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
-        const uint32_t base = tmem + lane_base + static_cast<uint32_t>(buf * kAsChunk);
-        for (int cb = 0; cb < N; cb += 128) {
-          // up to 128 columns per wait; widths are multiples of 16 (warp-uniform)
-          uint32_t v[128];
-          const int w = min(128, N - cb);
+        for (int k = 0; k < 4; ++k) {
+          b1[k] = INFINITY;
+          b2[k] = INFINITY;
+          bi[k] = 0x7fffffff;
+        }
+        for (int c = 0; c < nchunks; ++c, ++gc) {
+          const int buf = gc & 1;
+          ok = ok && mbar_wait(&bars->acc_full[buf], (gc >> 1) & 1, abort);
+          if (ok) {
+            tc_fence_after();
+            const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
+            const int nb = N >> 4;  // 16-column blocks of the chunk
+            const int c0 = 16 * ((q * nb) / kAsGroups), c1 = 16 * (((q + 1) * nb) / kAsGroups);
+            const uint32_t base = tmem + lane_base + static_cast<uint32_t>(buf * kAsChunk);
+            for (int col = c0; col < c1; col += 32) {
+              uint32_t v[32];
+              const bool full = (c1 - col >= 32);  // warp-uniform
+              if (full)
+                tmem_ld32(base + col, v);
+              else
+                tmem_ld16(base + col, *reinterpret_cast<uint32_t(*)[16]>(v));
+              tmem_wait_ld();
+              const int j0 = c * kAsChunk + col;
+              const float4* c4 = reinterpret_cast<const float4*>(cs + j0);
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            const int off = qd * 32;
-            if (off + 32 <= w)
-              tmem_ld32(base + cb + off, *reinterpret_cast<uint32_t(*)[32]>(v + off));
-            else if (off + 16 <= w)
-              tmem_ld16(base + cb + off, *reinterpret_cast<uint32_t(*)[16]>(v + off));
+              for (int i4 = 0; i4 < 8; ++i4) {
+                if (i4 < 4 || full) {
+                  const float4 cc = c4[i4];
+                  const int j = j0 + 4 * i4;
+                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 0]), cc.x), j + 0, b1[0], b2[0], bi[0]);
+                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 1]), cc.y), j + 1, b1[1], b2[1], bi[1]);
+                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 2]), cc.z), j + 2, b1[2], b2[2], bi[2]);
+                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 3]), cc.w), j + 3, b1[3], b2[3], bi[3]);
+                }
+              }
+            }
           }
-          tmem_wait_ld();
-          const int j0 = c * kAsChunk + cb;
-          // running best and second best in eight independent chains (column
-          // i goes to chain i % 8), branch-free; within a chain columns ascend,
-          // so equal values keep the lower index
+          tc_fence_before();
+          mbar_arrive(&bars->acc_empty[buf]);
+        }
+        // merge the chains: best by (value, index), second = smallest of the
+        // chains' seconds and the other chains' bests
+        float d1 = b1[0], d2 = b2[0];
+        int i1 = bi[0];
 #pragma unroll
-          for (int i = 0; i < 128; ++i) {
-            if (i < w) {
-              const int k = i & 7;
-              const float dd = fmaf(-2.f, __uint_as_float(v[i]), cs[j0 + i]);
-              const bool lt = dd < b1[k];
-              b2[k] = fminf(b2[k], fmaxf(b1[k], dd));
-              bi[k] = lt ? (j0 + i) : bi[k];
-              b1[k] = fminf(b1[k], dd);
+        for (int k = 1; k < 4; ++k) {
+          if (b1[k] < d1 || (b1[k] == d1 && bi[k] < i1)) {
+            d2 = fminf(d1, b2[k]);
+            d1 = b1[k];
+            i1 = bi[k];
+          } else {
+            d2 = fminf(d2, b1[k]);
+          }
+        }
+        if (q > 0) {
+          if (nx > 0) named_barrier_sync(kBarXchFree, kAsEpi);  // group 0 has read the last tile
+          xd1[(q - 1) * kTileM + r] = d1;
+          xd2[(q - 1) * kTileM + r] = d2;
+          xi1[(q - 1) * kTileM + r] = i1;
+          named_barrier_arrive(kBarXchFull, kAsEpi);
+        } else {
+          named_barrier_sync(kBarXchFull, kAsEpi);
+#pragma unroll
+          for (int g = 0; g < kAsGroups - 1; ++g) {
+            const float od1 = xd1[g * kTileM + r], od2 = xd2[g * kTileM + r];
+            const int oi1 = xi1[g * kTileM + r];
+            if (od1 < d1 || (od1 == d1 && oi1 < i1)) {
+              d2 = fminf(d1, od2);
+              d1 = od1;
+              i1 = oi1;
+            } else {
+              d2 = fminf(d2, od1);
+            }
+          }
+          named_barrier_arrive(kBarXchFree, kAsEpi);
+          const int row = t * kTileM + r;
+          if (ok && row < p.n) {
+            const size_t li = static_cast<size_t>(h) * p.n + row;
+            const float xy = p.xnorm[li] * Y;
+            const float E = kt_term * xy + 2.384185791015625e-07f * (C + 2.f * xy);
+            if (d2 - d1 > 2.f * E) {
+              if (p.labels[li] != i1) atomicAdd(&fl[p.flag_base], 1);
+              p.labels[li] = i1;
+            } else {
+              const int k = atomicAdd(&p.nrecheck[h], 1);
+              p.recheck[static_cast<size_t>(h) * p.n + k] = row;
+              atomicAdd(reinterpret_cast<unsigned long long*>(
+                            &p.stats->recheck_rows[p.flag_base >> 1]),
+                        1ull);
             }
           }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->acc_empty[buf]);
+        ++nx;
       }
-      if (!ok || row >= p.n) continue;
-      // merge the chains: best by (value, index), second = smallest of the
-      // chains' seconds and the other chains' bests
-      float d1 = b1[0];
-      int i1 = bi[0];
-#pragma unroll
-      for (int k = 1; k < 8; ++k)
-        if (b1[k] < d1 || (b1[k] == d1 && bi[k] < i1)) {
-          d1 = b1[k];
-          i1 = bi[k];
-        }
-      float d2 = INFINITY;
-      bool used = false;  // the winning chain's best is not a second candidate
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        d2 = fminf(d2, b2[k]);
-        if (!used && b1[k] == d1 && bi[k] == i1)
-          used = true;
-        else
-          d2 = fminf(d2, b1[k]);
-      }
-      const float xn = p.xnorm[static_cast<size_t>(h) * p.n + row];
-      const float xy = xn * Y;
-      const float E = kt_term * xy + 2.384185791015625e-07f * (C + 2.f * xy);
-      const size_t li = static_cast<size_t>(h) * p.n + row;
-      if (d2 - d1 > 2.f * E) {
-        if (p.labels[li] != i1) atomicAdd(&fl[p.flag_base], 1);
-        p.labels[li] = i1;
-      } else {
-        const int k = atomicAdd(&p.nrecheck[h], 1);
-        p.recheck[static_cast<size_t>(h) * p.n + k] = row;
-        atomicAdd(reinterpret_cast<unsigned long long*>(&p.stats->recheck_rows[p.flag_base >> 1]),
-                  1ull);
-      }
-    }
+    });
+    if (q > 0 && nx > 0) named_barrier_sync(kBarXchFree, kAsEpi);  // balance the last arrival
   }
   __syncthreads();
   if (*abort && threadIdx.x == 0) raise_status(p.stats, SPARSEPR_ERR_TIMEOUT);
@@ -519,7 +585,7 @@ size_t assign_tc_smem_bytes(int nA, int nB, int Dp, int Cpad) {
   const size_t b = static_cast<size_t>(nB) * atoms * Cpad * row_bytes;
   const size_t a = static_cast<size_t>(nA) * atoms * kTileM * row_bytes;
   return 1024 + ((b + 1023) & ~static_cast<size_t>(1023)) + 2 * a + static_cast<size_t>(Cpad) * 4 +
-         sizeof(AsBars);
+         static_cast<size_t>(kAsGroups - 1) * kTileM * 12 + sizeof(AsBars);
 }
 
 cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, int n, int D,
@@ -567,6 +633,7 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   // 2 planes of y: residual <= 2^-16 (bound 2^-14)
   p.res = (a.nB >= 3) ? 9.5367431640625e-07f : 6.103515625e-05f;
   p.tiles_per_head = (a.n + kTileM - 1) / kTileM;
+  p.H = a.H;
   p.cvals = a.cvals;
   p.xnorm = a.xnorm;
   p.hmax = a.hmax;
@@ -577,14 +644,16 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   p.nrecheck = a.nrecheck;
   p.stats = a.stats;
   zero_counts_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.nrecheck, a.H);
-  const size_t shb = assign_tc_smem_bytes(a.nA, a.nB, a.Dp, a.Cpad);
+  size_t shb = assign_tc_smem_bytes(a.nA, a.nB, a.Dp, a.Cpad);
+  if (shb < kAsMinSmem) shb = kAsMinSmem;
   cudaError_t e = cudaFuncSetAttribute(argmin_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(shb));
   if (e != cudaSuccess) return e;
-  int ctas = (a.sm_count + a.H - 1) / a.H;
-  if (ctas > p.tiles_per_head) ctas = p.tiles_per_head;
+  const long long tiles = static_cast<long long>(a.H) * p.tiles_per_head;
+  int ctas = a.sm_count;
+  if (ctas > tiles) ctas = static_cast<int>(tiles);
   if (ctas < 1) ctas = 1;
-  argmin_tc_kernel<<<dim3(ctas, a.H), kAsThreads, shb, st>>>(maps, p);
+  argmin_tc_kernel<<<ctas, kAsThreads, shb, st>>>(maps, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   recheck_kernel<<<dim3(64, a.H), 256, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
