@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsparsepr.so")
 SOURCES = ["api.cu", "sort.cu", "partition.cu", "linalg.cu", "permute.cu", "attn.cu", "fit.cu",
-           "noalloc.cu", "assign.cu", "eigen.cu"]
+           "noalloc.cu", "assign.cu", "eigen.cu", "correct.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

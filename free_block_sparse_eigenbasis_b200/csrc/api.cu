@@ -23,6 +23,12 @@ struct Ctx {
 
 bool finite_nonneg(double x) { return isfinite(x) && x >= 0.0; }
 
+// Tensor rows are read with 16-byte vector loads and TMA: every tensor
+// pointer must be 16-byte aligned.
+inline bool al16(const void* a) { return (reinterpret_cast<uintptr_t>(a) & 15) == 0; }
+template <typename... Ts>
+inline bool al16(const void* a, Ts... rest) { return al16(a) && al16(rest...); }
+
 sparsepr_status check_params(const sparsepr_params* p) {
   if (!p || !p->keep) return SPARSEPR_ERR_INVALID_ARG;
   if (p->H < 1 || p->H > SPARSEPR_MAX_HEADS) return SPARSEPR_ERR_INVALID_ARG;
@@ -163,6 +169,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
   if (s != SPARSEPR_OK) return s;
   if (!q || !k || !label_q || !label_k) return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(q, k)) return SPARSEPR_ERR_INVALID_ARG;
   const Layout& L = c.L;
   const int H = c.p.H, N = c.p.N, d = c.p.d, Nv = L.Nv, e = c.p.n_eig, Ck = c.p.Ck, Cq = c.p.Cq;
   const int iters = c.p.kmeans_iters;
@@ -340,6 +347,7 @@ sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v, sp
       !kp || !vp)
     return SPARSEPR_ERR_INVALID_ARG;
   if (qp == q || kp == k || vp == v) return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(q, k, v, qp, kp, vp)) return SPARSEPR_ERR_INVALID_ARG;
   const int H = c.p.H, N = c.p.N, d = c.p.d;
   const int nchunk = (N + kSortChunk - 1) / kSortChunk;
   if (static_cast<size_t>(H) * nchunk * c.L.Cmax > static_cast<size_t>(H) * c.L.nchunk * c.L.Cmax)
@@ -364,6 +372,7 @@ sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt
   sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
   if (s != SPARSEPR_OK) return s;
   if (!qp || !kp || !off_q || !off_k || !csr || !k_per_head) return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(qp, kp)) return SPARSEPR_ERR_INVALID_ARG;
   const int H = c.p.H, N = c.p.N, d = c.p.d, Ck = c.p.Ck, Cq = c.p.Cq;
   double* cq = at<double>(ws, c.L.cq);
   double* ckr = at<double>(ws, c.L.ckr);
@@ -372,7 +381,8 @@ sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt
   int32_t kh[SPARSEPR_MAX_HEADS];
   for (int h = 0; h < H; ++h) kh[h] = keep_budget(c.p.keep[h], Ck);
   SPR_TRY(launch_write_k(kh, H, k_per_head, c.st));
-  SPR_TRY(launch_route(cq, ckr, H, Cq, Ck, d, c.scale, k_per_head, c.L.kmax, csr, c.st));
+  SPR_TRY(launch_route_gemm(cq, ckr, H, Cq, Ck, d, c.scale, k_per_head, c.L.kmax,
+                            at<double>(ws, c.L.scores), c.L.scores_bytes, csr, c.st));
   return SPARSEPR_OK;
 }
 
@@ -387,6 +397,7 @@ sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const
   if (s != SPARSEPR_OK) return s;
   if (!qp || !kp || !vp || !off_q || !off_k || !csr || !k_per_head || !o_sparse || !pairs_sparse)
     return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(qp, kp, vp, o_sparse)) return SPARSEPR_ERR_INVALID_ARG;
   const int H = c.p.H, N = c.p.N, d = c.p.d;
   const size_t n = static_cast<size_t>(H) * N * d;
   const void *q16 = qp, *k16 = kp, *v16 = vp;
@@ -440,6 +451,7 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
   if (!qp || !kp || !vp || !off_q || !perm_q || !o_sparse || !pairs_sparse || !out ||
       !pairs_exec || (c.p.M > 0 && !probes))
     return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(qp, kp, vp, o_sparse, out)) return SPARSEPR_ERR_INVALID_ARG;
   const Layout& L = c.L;
   const int H = c.p.H, N = c.p.N, d = c.p.d, M = c.p.M, Cq = c.p.Cq;
   cudaStream_t st = c.st;
@@ -523,7 +535,11 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     SPR_TRY(cudaMemsetAsync(bv32, 0, static_cast<size_t>(H) * d * 4, st));
     if (fit) SPR_TRY(cudaMemsetAsync(fit, 0, static_cast<size_t>(H) * (d * d + d) * 8, st));
   }
-  SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, M, d, out, c.bf16, st));
+  if (correct_tc_supported(H, N, d))
+    SPR_TRY(launch_correct_tc(o_sparse, od, probes, perm_q, bp32, bv32, H, N, M, d, out, c.bf16,
+                              sm_count(), c.stats, st));
+  else
+    SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, M, d, out, c.bf16, st));
   SPR_TRY(launch_pairs_exec(pairs_sparse, H, static_cast<int64_t>(M) * N, pairs_exec, c.stats, st));
   return SPARSEPR_OK;
 }

@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         for (int c = 0; c < nchunks; ++c, ++gc) {
           const int buf = gc & 1;
           ok = ok && mbar_wait(&bars->acc_full[buf], (gc >> 1) & 1, abort);
+          ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
           if (ok) {
             tc_fence_after();
             const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
@@ -337,12 +338,13 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           }
           named_barrier_arrive(kBarXchFree, kAsEpi);
           const int row = t * kTileM + r;
+          bool changed = false;
           if (ok && row < p.n) {
             const size_t li = static_cast<size_t>(h) * p.n + row;
             const float xy = p.xnorm[li] * Y;
             const float E = kt_term * xy + 2.384185791015625e-07f * (C + 2.f * xy);
             if (d2 - d1 > 2.f * E) {
-              if (p.labels[li] != i1) atomicAdd(&fl[p.flag_base], 1);
+              changed = p.labels[li] != i1;
               p.labels[li] = i1;
             } else {
               const int k = atomicAdd(&p.nrecheck[h], 1);
@@ -352,6 +354,9 @@ __global__ void __launch_bounds__(kAsThreads, 1)
                         1ull);
             }
           }
+          // one atomic per warp for the label-change counter
+          const unsigned cb = __ballot_sync(0xffffffffu, changed);
+          if (lane == 0 && cb) atomicAdd(&fl[p.flag_base], __popc(cb));
         }
         ++nx;
       }
@@ -368,11 +373,12 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// fp64 decision of the flagged rows: blocks of 16 rows scan the centroids in
-// chunks of 16 staged in shared memory.
+// fp64 decision of the flagged rows: a block takes eight flagged rows (one
+// per warp) and streams the centroids through shared memory 32 at a time;
+// lane l scores centroid j0 + l against its warp's row, then a warp argmin.
 // direct = 1: d = sum_t (x_t - y_jt)^2; else d = c_j - 2 x . y_j.
 // ---------------------------------------------------------------------------
-constexpr int kRcRows = 16, kRcCols = 16, kRcMaxD = 128;
+constexpr int kRcWarps = 8, kRcMaxD = 128, kRcChunk = 32;
 
 __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   if (kind == kXf64) return static_cast<const double*>(X)[i];
@@ -380,70 +386,60 @@ __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   return static_cast<double>(static_cast<const float*>(X)[i]);
 }
 
-__global__ void recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
-                               const double* Y, const double* c, int m, int direct,
-                               int32_t* labels, int32_t* flags, int flag_base,
-                               const int32_t* recheck, const int32_t* nrecheck) {
-  // a block of up to 16 flagged rows against the centroids, 16 at a time;
-  // thread (r, s) = (row in block, centroid in chunk), 256 threads
-  __shared__ double xs[kRcRows][kRcMaxD];
-  __shared__ double ys[kRcCols][kRcMaxD + 1];
-  __shared__ double cc[kRcCols];
-  __shared__ int rows_s[kRcRows];
+__global__ void __launch_bounds__(kRcWarps * 32)
+    recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
+                   const double* Y, const double* c, int m, int direct, int32_t* labels,
+                   int32_t* flags, int flag_base, const int32_t* recheck,
+                   const int32_t* nrecheck) {
+  __shared__ double xs[kRcWarps][kRcMaxD];
+  __shared__ double ys[kRcChunk][kRcMaxD + 1];
+  __shared__ double cc[kRcChunk];
   const int h = blockIdx.y;
   int32_t* fl = flags + h * 4;
   if (fl[flag_base + 1]) return;
   const int cnt = nrecheck[h];
-  const int r = threadIdx.x >> 4, s = threadIdx.x & 15;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const double* Yh = Y + static_cast<size_t>(h) * m * D;
-  for (int b0 = blockIdx.x * kRcRows; b0 < cnt; b0 += gridDim.x * kRcRows) {
-    const int nb = min(kRcRows, cnt - b0);
-    if (threadIdx.x < kRcRows)
-      rows_s[threadIdx.x] = (static_cast<int>(threadIdx.x) < nb)
-                                ? recheck[static_cast<size_t>(h) * n + b0 + threadIdx.x]
-                                : -1;
-    __syncthreads();
-    for (int t = threadIdx.x; t < kRcRows * D; t += blockDim.x) {
-      const int rr = t / D, cc_ = t % D;
-      xs[rr][cc_] = (rows_s[rr] >= 0) ? ldx(X, kind, h * hsx + static_cast<size_t>(rows_s[rr]) * ldx_ + cc_)
-                                      : 0.0;
-    }
+  const double* ch = c + static_cast<size_t>(h) * m;
+  for (int base = blockIdx.x * kRcWarps; base < cnt; base += gridDim.x * kRcWarps) {
+    const int k = base + w;
+    const bool has = k < cnt;
+    const int row = has ? recheck[static_cast<size_t>(h) * n + k] : 0;
+    if (has)
+      for (int t = lane; t < D; t += 32) xs[w][t] = ldx(X, kind, h * hsx + static_cast<size_t>(row) * ldx_ + t);
     double best = INFINITY;
     int bi = 0x7fffffff;
-    for (int j0 = 0; j0 < m; j0 += kRcCols) {
-      __syncthreads();  // previous chunk consumed (and xs written, first time)
-      for (int t = threadIdx.x; t < kRcCols * D; t += blockDim.x) {
-        const int jj = t / D, cc_ = t % D;
-        ys[jj][cc_] = (j0 + jj < m) ? Yh[static_cast<size_t>(j0 + jj) * D + cc_] : 0.0;
+    for (int j0 = 0; j0 < m; j0 += kRcChunk) {
+      __syncthreads();  // the previous chunk is consumed (first time: xs written)
+      for (int t = threadIdx.x; t < kRcChunk * D; t += blockDim.x) {
+        const int jj = t / D, a = t % D;
+        ys[jj][a] = (j0 + jj < m) ? Yh[static_cast<size_t>(j0 + jj) * D + a] : 0.0;
       }
-      if (!direct && threadIdx.x < kRcCols)
-        cc[threadIdx.x] = (j0 + static_cast<int>(threadIdx.x) < m)
-                              ? c[static_cast<size_t>(h) * m + j0 + threadIdx.x]
-                              : 0.0;
+      if (!direct && threadIdx.x < kRcChunk)
+        cc[threadIdx.x] = (j0 + static_cast<int>(threadIdx.x) < m) ? ch[j0 + threadIdx.x] : 0.0;
       __syncthreads();
-      const int j = j0 + s;
-      if (j < m) {
+      const int j = j0 + lane;  // ascending within the lane
+      if (has && j < m) {
         double dd;
         if (direct) {
           dd = 0.0;
           for (int t = 0; t < D; ++t) {
-            const double diff = xs[r][t] - ys[s][t];
+            const double diff = xs[w][t] - ys[lane][t];
             dd = fma(diff, diff, dd);
           }
         } else {
           double sm = 0.0;
-          for (int t = 0; t < D; ++t) sm = fma(xs[r][t], ys[s][t], sm);
-          dd = cc[s] - 2.0 * sm;
+          for (int t = 0; t < D; ++t) sm = fma(xs[w][t], ys[lane][t], sm);
+          dd = cc[lane] - 2.0 * sm;
         }
-        if (dd < best) {  // within a thread centroids ascend
+        if (dd < best) {
           best = dd;
           bi = j;
         }
       }
     }
-    // reduce over the 16 threads of each row (lowest index on ties)
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) {
+    for (int o = 16; o > 0; o >>= 1) {  // lowest index on ties
       const double ob = __shfl_xor_sync(0xffffffffu, best, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ob < best || (ob == best && oi < bi)) {
@@ -451,12 +447,11 @@ __global__ void recheck_kernel(const void* X, int kind, long long hsx, int ldx_,
         bi = oi;
       }
     }
-    if (s == 0 && r < nb) {
-      const size_t li = static_cast<size_t>(h) * n + rows_s[r];
+    if (has && lane == 0) {
+      const size_t li = static_cast<size_t>(h) * n + row;
       if (labels[li] != bi) atomicAdd(&fl[flag_base], 1);
       labels[li] = bi;
     }
-    __syncthreads();  // rows_s / xs are rewritten by the next block
   }
 }
 
@@ -490,17 +485,22 @@ __global__ void split_rows_kernel(const void* X, int kind, long long hsx, int ld
 }
 
 // Centroid side: planes of y (padded to Cpad rows with zeros), fp32 offsets
-// (+inf on padding), and the per-head maxima Y = max |y_j|, C = max |c_j|.
-__global__ void prep_centroids_kernel(const double* Yv, const double* cv, int m, int D, int Dp,
-                                      int Cpad, int P, __nv_bfloat16* planes,
-                                      long long plane_stride, float* cf, float* hmax,
-                                      const int32_t* flags, int flag_base) {
-  __shared__ double ym[32], cm[32];
-  const int h = blockIdx.x;
+// (+inf on padding), and the per-head maxima Y = max |y_j|, C = max |c_j|
+// (rounded up; merged across CTAs with an integer max on the bits of the
+// non-negative floats, after hmax was zeroed). One warp per centroid row.
+constexpr int kPrepWarps = 16;
+
+__global__ void __launch_bounds__(kPrepWarps * 32)
+    prep_centroids_kernel(const double* Yv, const double* cv, int m, int D, int Dp, int Cpad,
+                          int P, __nv_bfloat16* planes, long long plane_stride, float* cf,
+                          float* hmax, const int32_t* flags, int flag_base) {
+  __shared__ float ym[kPrepWarps], cm[kPrepWarps];
+  const int h = blockIdx.y;
   if (flags && flags[h * 4 + flag_base + 1]) return;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  double ymax = 0.0, cmax = 0.0;
-  for (int j = wid; j < Cpad; j += nw) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int j = blockIdx.x * kPrepWarps + wid;
+  float yv = 0.f, cvv = 0.f;
+  if (j < Cpad) {
     const size_t ob = (static_cast<size_t>(h) * Cpad + j) * Dp;
     double ss = 0.0;
     for (int t = lane; t < Dp; t += 32) {
@@ -517,25 +517,26 @@ __global__ void prep_centroids_kernel(const double* Yv, const double* cv, int m,
       if (j < m) {
         const double cj = cv[static_cast<size_t>(h) * m + j];
         cf[static_cast<size_t>(h) * Cpad + j] = static_cast<float>(cj);
-        ymax = fmax(ymax, sqrt(ss));
-        cmax = fmax(cmax, fabs(cj));
+        yv = static_cast<float>(sqrt(ss) * (1.0 + 1e-6));
+        cvv = static_cast<float>(fabs(cj) * (1.0 + 1e-6));
       } else {
         cf[static_cast<size_t>(h) * Cpad + j] = INFINITY;
       }
     }
   }
   if (lane == 0) {
-    ym[wid] = ymax;
-    cm[wid] = cmax;
+    ym[wid] = yv;
+    cm[wid] = cvv;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < nw; ++w) {
-      ymax = fmax(ymax, ym[w]);
-      cmax = fmax(cmax, cm[w]);
+    float a = ym[0], c = cm[0];
+    for (int w = 1; w < kPrepWarps; ++w) {
+      a = fmaxf(a, ym[w]);
+      c = fmaxf(c, cm[w]);
     }
-    hmax[h * 2 + 0] = static_cast<float>(ymax * (1.0 + 1e-6));
-    hmax[h * 2 + 1] = static_cast<float>(cmax * (1.0 + 1e-6));
+    atomicMax(reinterpret_cast<int*>(&hmax[h * 2 + 0]), __float_as_int(a));
+    atomicMax(reinterpret_cast<int*>(&hmax[h * 2 + 1]), __float_as_int(c));
   }
 }
 
@@ -544,26 +545,8 @@ __global__ void zero_counts_kernel(int32_t* p, int n) {
   if (i < n) p[i] = 0;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 bool plane_map(CUtensorMap* m, const void* base, size_t rows, int Dp, bool sw32, int box_rows) {
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(Dp), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(Dp) * 2};
@@ -601,8 +584,10 @@ cudaError_t launch_prep_centroids(const double* Y, const double* c, int m, int D
                                   int Cpad, int P, int H, __nv_bfloat16* planes,
                                   long long plane_stride, float* cf, float* hmax,
                                   const int32_t* flags, int flag_base, cudaStream_t st) {
-  prep_centroids_kernel<<<H, 512, 0, st>>>(Y, c, m, D, Dp, Cpad, P, planes, plane_stride, cf, hmax,
-                                           flags, flag_base);
+  zero_counts_kernel<<<(2 * H + 127) / 128, 128, 0, st>>>(reinterpret_cast<int32_t*>(hmax), 2 * H);
+  dim3 grid((Cpad + kPrepWarps - 1) / kPrepWarps, H);
+  prep_centroids_kernel<<<grid, kPrepWarps * 32, 0, st>>>(Y, c, m, D, Dp, Cpad, P, planes,
+                                                          plane_stride, cf, hmax, flags, flag_base);
   return cudaGetLastError();
 }
 
@@ -656,7 +641,7 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   argmin_tc_kernel<<<ctas, kAsThreads, shb, st>>>(maps, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  recheck_kernel<<<dim3(64, a.H), 256, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
+  recheck_kernel<<<dim3(16, a.H), kRcWarps * 32, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
                                                 a.y_exact, a.c_exact, a.m, a.direct, a.labels,
                                                 a.flags, a.flag_base, a.recheck, a.nrecheck);
   return cudaGetLastError();

@@ -3,25 +3,28 @@
 // "Attention Sparsity is Input-Stable", block selection: the softmax is
 // normalised over the kept logits only).
 //
-// One CTA computes one 128-row query tile of one query group. The key side
-// is the union of the kept key groups' contiguous ranges in the group-major
-// K/V; runs of adjacent kept groups are merged (once per query group, by the
-// slot-count kernel) and cut into 8-row slots, 16 slots per 128-key tile,
-// each slot fetched by TMA at an arbitrary row. Rows of a slot past its
-// run's end are masked to -inf, so skipped key groups are never multiplied
-// (only the tail padding of a run is).
+// One CTA computes one unit of up to 256 query rows of one query group. The
+// key side is the union of the kept key groups' contiguous ranges in the
+// group-major K/V; runs of adjacent kept groups are merged (once per query
+// group, by the slot-count kernel) and cut into 8-row slots, 16 slots per
+// 128-key tile, each contiguous piece fetched by TMA at an arbitrary row.
+// Rows of a slot past its run's end are masked to -inf, so skipped key groups
+// are never multiplied (only the tail padding of a run is).
 //
-// Roles (192 threads): warps 0-3 own one query row per thread (TMEM lane =
-// row) and run the online softmax and the epilogue; warp 4 lanes 0 and 1
-// stream Q+K and V with TMA (each contiguous piece of slots as power-of-two
-// boxes of 8..128 rows); warp 5 lane 0 issues tcgen05.mma.
-//   * S = Q K^T goes to one of two TMEM buffers, so S(j+1) runs on the
-//     tensor cores while the softmax of tile j works;
-//   * P is written bf16 to one of two shared-memory buffers (128B-swizzled,
-//     K-major), so the softmax of tile j+1 overlaps P(j) V(j);
-//   * O += P V accumulates in TMEM. O is rescaled only when a row maximum
-//     grows by more than 2^8; O and the row sum always share one reference
-//     maximum, so the result is exact.
+// Roles (320 threads): two softmax warpgroups (warps 0-3 and 4-7, thread =
+// query row = TMEM lane) each own one TMEM slot (S_i, O_i, with P_i written
+// as packed bf16 over the first 64 columns of S_i); warp 8 lane 0 streams Q,
+// K and V with TMA; warp 9 lane 0 issues tcgen05.mma.
+//   * a unit of two 128-row query tiles gives tile i to warpgroup i: both
+//     see every key tile, and the tensor cores alternate between them
+//     (P_0 V, S_0 of the next tile, P_1 V, S_1 of the next tile), so one
+//     warpgroup's softmax overlaps the other's MMAs;
+//   * a unit of one query tile splits the key tiles instead (even ones to
+//     warpgroup 0, odd ones to warpgroup 1) with separate running maxima
+//     and accumulators, merged at the end;
+//   * P V reads P from tensor memory (no shared-memory round trip); O is
+//     rescaled only when a row maximum grows by more than 2^8, and O and the
+//     row sum always share one reference maximum, so the result is exact.
 // Every mbarrier wait is bounded; a wait that runs out marks the status word
 // and the CTA drains its in-flight copies and MMAs, frees tensor memory and
 // returns.
@@ -31,11 +34,11 @@
 namespace spr {
 namespace {
 
-constexpr int kStages = 2;
+constexpr int kStages = 2;                         // K and V ring depth
 constexpr int kSlotsPerTile = kTileN / kSlotRows;  // 16
+constexpr int kUnitRows = 2 * kTileM;              // query rows per CTA
 constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
-constexpr uint32_t kTmemCols = 512;  // S0 [0,128), S1 [128,256), O [256, 256+d), exchange [480,512)
-constexpr uint32_t kXchCol = 480;    // row-max / row-sum exchange between the two halves of a row
+constexpr uint32_t kTmemCols = 512;  // S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 after
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -43,61 +46,32 @@ template <int HD>
 struct Smem {
   static constexpr int kAtoms = HD / 64;           // 128-byte swizzle atoms along d
   static constexpr int kSlab = kTileM * 128;       // one 64-column slab of 128 rows (16 KB)
-  static constexpr int kQBytes = kAtoms * kSlab;
+  static constexpr int kQBytes = kAtoms * kSlab;   // one query tile
   static constexpr int kKVBytes = kAtoms * kSlab;  // kTileN == kTileM
-  static constexpr int kPBytes = (kTileN / 64) * kSlab;
-  static constexpr int q_off = 0;
-  static constexpr int k_off = q_off + kQBytes;
+  static constexpr int q_off = 0;                  // two query tiles
+  static constexpr int k_off = q_off + 2 * kQBytes;
   static constexpr int v_off = k_off + kStages * kKVBytes;
-  static constexpr int p_off = v_off + kStages * kKVBytes;  // two P buffers
-  static constexpr int bar_off = p_off + 2 * kPBytes;
-  static constexpr int runs_off = bar_off + 256;
+  static constexpr int bar_off = v_off + kStages * kKVBytes;
+  static constexpr int ml_off = bar_off + 256;     // [2][2][128] f32 row maxima and sums
+  static constexpr int runs_off = ml_off + 2048;
 };
 // Dynamic shared memory: the d=128 footprint for both head dims (one CTA per
-// SM; each CTA allocates 512 TMEM columns), the barrier block, a run list of
-// up to kSmemRuns entries, and 1024 bytes of alignment slack.
-// The whole per-block maximum is requested; what the 1024-byte alignment of
-// the tile region leaves after the barriers holds the run list (>= 226 runs).
+// SM; each CTA allocates 512 TMEM columns), the barrier block, the final
+// merge buffer, a run list, and 1024 bytes of alignment slack. What the
+// 1024-byte alignment of the tile region leaves holds the run list (>= 4000
+// runs); longer lists are read from global memory.
 constexpr int kAttnSmemBytes = 232448;
-static_assert(Smem<128>::runs_off + 226 * 8 + 1008 <= kAttnSmemBytes, "shared memory");
+static_assert(Smem<128>::runs_off + 4000 * 8 + 1008 <= kAttnSmemBytes, "shared memory");
 
 struct Bars {
   uint64_t q_full;
   uint64_t kfull[kStages], vfull[kStages], kempty[kStages], vempty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t mma_idle;
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
-
-// Walks the merged key runs of one query group in ascending order and hands
-// out 8-row slots (start row, valid rows).
-struct SlotIter {
-  const int2* runs;
-  int nruns, ri, pos, end;
-  __device__ void init(const int2* r, int n) {
-    runs = r;
-    nruns = n;
-    ri = -1;
-    pos = 0;
-    end = 0;
-  }
-  __device__ bool next(int& start, int& valid) {
-    while (pos >= end) {
-      ++ri;
-      if (ri >= nruns) return false;
-      const int2 rr = runs[ri];
-      pos = rr.x;
-      end = rr.x + rr.y;
-    }
-    start = pos;
-    valid = min(kSlotRows, end - pos);
-    pos += kSlotRows;
-    return true;
-  }
-};
 
 // TMA maps: Q (64-column x 128-row boxes) and K / V with boxes of 8, 16, 32,
 // 64 and 128 rows (index = log2(rows / 8)).
@@ -123,25 +97,51 @@ struct AttnParams {
   DeviceStats* stats;
 };
 
-// The two warps that share a lane quarter (w and w+4) swap one float per
-// row: each stores its value in tensor-memory column base + half, then reads
-// the partner's column. Buffers alternate between calls, so one barrier per
-// call suffices (a column is rewritten only after the partner passed the
-// next barrier, i.e. after it read the old value).
-__device__ __forceinline__ float exchange_pair(uint32_t col_base, int half, int quarter, float v) {
-  tmem_st1(col_base + half, __float_as_uint(v));
-  tmem_wait_st();
-  tc_fence_before();
-  named_barrier_sync(1 + quarter, 64);
-  tc_fence_after();
-  const uint32_t o = tmem_ld1(col_base + (half ^ 1));
-  tmem_wait_ld();
-  return __uint_as_float(o);
-}
+// Key-column validity of the key tiles of one query group, walked in
+// ascending tile order: every run contributes ceil(len / 8) slots, of which
+// only the last may be partial; slots past the last run are padding.
+struct MaskWalk {
+  const int2* runs;
+  int nr, ns, ri, rend;  // rend: slots up to and including run ri
+  __device__ void init(const int2* r, int n, int nslots) {
+    runs = r;
+    nr = n;
+    ns = nslots;
+    ri = 0;
+    rend = (n > 0) ? (r[0].y + kSlotRows - 1) / kSlotRows : 0;
+  }
+  // bit c of m[c / 32] = key column c of tile j is a real key
+  __device__ void tile(int j, uint32_t (&m)[4]) {
+    m[0] = m[1] = m[2] = m[3] = 0xFFFFFFFFu;
+    const int lo = j * kSlotsPerTile, hi = lo + kSlotsPerTile;
+    while (ri < nr && rend <= hi) {
+      const int rem = runs[ri].y & (kSlotRows - 1);
+      const int last = rend - 1;
+      if (rem && last >= lo) {
+        const int s = last - lo;
+        m[s >> 2] &= ~((0xFFu & ~((1u << rem) - 1u)) << ((s & 3) * 8));
+      }
+      ++ri;
+      if (ri < nr) rend += (runs[ri].y + kSlotRows - 1) / kSlotRows;
+    }
+    for (int s = max(ns, lo) - lo; s < kSlotsPerTile; ++s) m[s >> 2] &= ~(0xFFu << ((s & 3) * 8));
+  }
+};
 
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  // byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128B-swizzled slab
-  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+// 2^x on the FMA pipe, used for a quarter of the columns so that the
+// special-function unit (ex2.approx) is not the bottleneck of the softmax:
+// x = n + f with n = round(x) (added into the exponent field) and f in
+// [-1/2, 1/2], 2^f by a cubic whose coefficients minimise the relative
+// error on that interval (Lawson-weighted least squares on Chebyshev nodes;
+// maximum relative error 7.5e-5, below the 2^-9 rounding of the bf16 P it
+// feeds). x is clamped at -126, so a masked logit gives 2^-126 instead of 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
+  const float f = x - (t - 12582912.f);
+  const float q = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f,
+                       0.9999280572f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 template <int HD>
@@ -152,10 +152,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int h = blockIdx.y;
   if (static_cast<int>(blockIdx.x) >= p.nwork[h]) return;
   const int wcode = p.work[static_cast<size_t>(h) * p.tiles_per_head + blockIdx.x];
-  const int g = wcode >> 16, tq = wcode & 0xFFFF;
+  const int g = wcode >> 16, tu = wcode & 0xFFFF;
   const int32_t* offq = p.off_q + static_cast<size_t>(h) * (p.Cq + 1);
-  const int row0 = offq[g] + tq * kTileM;
-  const int rows_valid = min(kTileM, offq[g + 1] - row0);
+  const int row0 = offq[g] + tu * kUnitRows;
+  const int rows_unit = min(kUnitRows, offq[g + 1] - row0);
+  const int nq = rows_unit > kTileM ? 2 : 1;  // query tiles in this unit
   const size_t gi = static_cast<size_t>(h) * p.Cq + g;
   const int ns = p.nslots[gi];
   const int T = (ns + kSlotsPerTile - 1) / kSlotsPerTile;
@@ -164,12 +165,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (T == 0) {
     // empty kept set (reported by the slot-count kernel): rows are zero
-    if (static_cast<int>(threadIdx.x) < rows_valid) {
+    if (static_cast<int>(threadIdx.x) < rows_unit) {
       float* o = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x) * HD;
       for (int c = 0; c < HD; c += 4) *reinterpret_cast<float4*>(o + c) = make_float4(0, 0, 0, 0);
     }
     return;
   }
+  // tasks (query tile, key tile) of warpgroup i: two tiles -> (i, t) for every
+  // key tile t; one tile -> (0, 2t + i)
+  const bool two = (nq == 2);
+  const int ntask[2] = {two ? T : (T + 1) / 2, two ? T : T / 2};
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -177,8 +182,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* Qs = smem + L::q_off;
   uint8_t* Ks = smem + L::k_off;
   uint8_t* Vs = smem + L::v_off;
-  uint8_t* Ps = smem + L::p_off;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::bar_off);
+  float* ml = reinterpret_cast<float*>(smem + L::ml_off);
   int2* runs_s = reinterpret_cast<int2*>(smem + L::runs_off);
   // run-list capacity left in the dynamic allocation after alignment
   const int cap = (kAttnSmemBytes - static_cast<int>(smem - smem_raw) - L::runs_off) / 8;
@@ -196,8 +201,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], 2 * kTileM);
-      mbar_init(&bars->pv_done[b], 1);
+      mbar_init(&bars->p_full[b], kTileM);
+      mbar_init(&bars->o_done[b], 1);
     }
     mbar_init(&bars->mma_idle, 1);
     bars->abort = 0;
@@ -216,248 +221,298 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort = &bars->abort;
 
   if (warp == 8) {
-    // --------------- TMA producers: lane 0 streams Q and K, lane 1 V ---------------
-    if (lane < 2) {
-      const bool is_k = (lane == 0);
+    // ---------------- TMA producer: Q once, then K(j), V(j) in order ----------------
+    if (lane == 0) {
       const int krow_base = h * p.N;
-      if (is_k) {
-        mbar_arrive_expect_tx(&bars->q_full, kAtoms * p.q_box_rows * 128);
+      mbar_arrive_expect_tx(&bars->q_full, nq * kAtoms * p.q_box_rows * 128);
+      for (int qt = 0; qt < nq; ++qt)
         for (int a = 0; a < kAtoms; ++a)
-          tma_load_2d(Qs + a * L::kSlab, &maps.q, &bars->q_full, a * 64, h * p.q_rows + row0);
-      }
-      const CUtensorMap* bm = is_k ? maps.k : maps.v;
-      uint8_t* base = is_k ? Ks : Vs;
-      uint64_t* full = is_k ? bars->kfull : bars->vfull;
-      uint64_t* empty = is_k ? bars->kempty : bars->vempty;
-      SlotIter it;
-      it.init(runs, nr);
-      int issued = -1;
-      bool ok = true;
+          tma_load_2d(Qs + qt * L::kQBytes + a * L::kSlab, &maps.q, &bars->q_full, a * 64,
+                      h * p.q_rows + row0 + qt * kTileM);
+      int ri = -1, pos = 0, rend = 0;  // current run and its row range [pos, rend)
+      int k_issued = -1, v_issued = -1;
       for (int j = 0; j < T; ++j) {
-        const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(&empty[st], ((j / kStages) + 1) & 1, abort)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[st], L::kKVBytes);
-        uint8_t* dst = base + st * L::kKVBytes;
-        // contiguous pieces of consecutive slots, each loaded as power-of-two boxes
-        int s = 0;
-        while (s < kSlotsPerTile) {
-          int r0 = 0, vv = 0;
-          if (!it.next(r0, vv)) r0 = 0;  // past the last run: any valid rows (masked)
-          int n = 1;
-          int la = r0, lv = 0;
-          while (s + n < kSlotsPerTile) {
-            SlotIter peek = it;
-            if (!peek.next(la, lv)) la = -1;
-            if (la != r0 + kSlotRows * n) break;
-            it = peek;
-            ++n;
+        // box plan of key tile j: (slot, first row, log2 size) per box
+        int bslot[kSlotsPerTile], brow[kSlotsPerTile], blg[kSlotsPerTile];
+        int nb = 0;
+        int t = 0;
+        while (t < kSlotsPerTile) {
+          while (pos >= rend && ri < nr) {
+            ++ri;
+            if (ri < nr) {
+              pos = runs[ri].x;
+              rend = pos + runs[ri].y;
+            }
           }
-          int t = s, r = r0, m = n;
-#pragma unroll 1
-          for (int lg = p.max_lg; lg >= 0; --lg) {
+          int r, m;
+          if (pos < rend) {
+            r = pos;
+            m = min(kSlotsPerTile - t, (rend - pos + kSlotRows - 1) / kSlotRows);
+            pos += m * kSlotRows;
+          } else {
+            r = 0;  // past the last run: any rows of the head (masked)
+            m = kSlotsPerTile - t;
+          }
+          for (int lg = p.max_lg; lg >= 0 && m > 0; --lg) {
             const int sz = 1 << lg;
             while (m >= sz) {
-#pragma unroll
-              for (int a = 0; a < kAtoms; ++a)
-                tma_load_2d(dst + a * L::kSlab + t * 1024, &bm[lg], &full[st], a * 64,
-                            krow_base + r);
+              bslot[nb] = t;
+              brow[nb] = r;
+              blg[nb] = lg;
+              ++nb;
               t += sz;
               r += sz * kSlotRows;
               m -= sz;
             }
           }
-          s += n;
         }
-        issued = j;
+        const int st = j % kStages;
+        const uint32_t ph = ((j / kStages) + 1) & 1;
+        if (j >= kStages && !mbar_wait(&bars->kempty[st], ph, abort)) break;
+        mbar_arrive_expect_tx(&bars->kfull[st], L::kKVBytes);
+        for (int b = 0; b < nb; ++b)
+#pragma unroll
+          for (int a = 0; a < kAtoms; ++a)
+            tma_load_2d(Ks + st * L::kKVBytes + a * L::kSlab + bslot[b] * 1024, &maps.k[blg[b]],
+                        &bars->kfull[st], a * 64, krow_base + brow[b]);
+        k_issued = j;
+        if (j >= kStages && !mbar_wait(&bars->vempty[st], ph, abort)) break;
+        mbar_arrive_expect_tx(&bars->vfull[st], L::kKVBytes);
+        for (int b = 0; b < nb; ++b)
+#pragma unroll
+          for (int a = 0; a < kAtoms; ++a)
+            tma_load_2d(Vs + st * L::kKVBytes + a * L::kSlab + bslot[b] * 1024, &maps.v[blg[b]],
+                        &bars->vfull[st], a * 64, krow_base + brow[b]);
+        v_issued = j;
       }
-      if (!ok) {
-        // let the loads already in flight land before the CTA exits
-        volatile int never = 0;
-        for (int j = max(0, issued - kStages + 1); j <= issued; ++j)
-          mbar_wait(&full[j % kStages], (j / kStages) & 1, &never);
-        if (is_k) mbar_wait(&bars->q_full, 0, &never);
-      }
+      // let the loads already in flight land before the CTA exits
+      volatile int never = 0;
+      for (int j = max(0, k_issued - kStages + 1); j <= k_issued; ++j)
+        mbar_wait(&bars->kfull[j % kStages], (j / kStages) & 1, &never);
+      for (int j = max(0, v_issued - kStages + 1); j <= v_issued; ++j)
+        mbar_wait(&bars->vfull[j % kStages], (j / kStages) & 1, &never);
+      mbar_wait(&bars->q_full, 0, &never);
     }
   } else if (warp == 9) {
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileM, kTileN, 0);
       constexpr uint32_t idO = idesc_bf16(kTileM, HD, 1);
-      const uint32_t q_addr = smem_u32(Qs), k_addr = smem_u32(Ks), v_addr = smem_u32(Vs),
-                     p_addr = smem_u32(Ps);
-      auto issue_s = [&](int j) {
-        const int st = j % kStages;
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>((j & 1) * kTileN);
+      const uint32_t q_addr = smem_u32(Qs), k_addr = smem_u32(Ks), v_addr = smem_u32(Vs);
+      bool ok = mbar_wait(&bars->q_full, 0, abort);
+      auto kv_of = [&](int i, int t) { return two ? t : 2 * t + i; };
+      // S_i = Q_(tile of i) K(kv)^T
+      auto issue_s = [&](int i, int t) -> bool {
+        const int kv = kv_of(i, t), st = kv % kStages;
+        if (!mbar_wait(&bars->kfull[st], (kv / kStages) & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t qa = q_addr + (two ? i : 0) * L::kQBytes;
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(i * kTileN);
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
           const uint32_t off = static_cast<uint32_t>((ks >> 2) * L::kSlab + (ks & 3) * 32);
-          const uint64_t ad = smem_desc_sw128(q_addr + off, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(qa + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(k_addr + st * L::kKVBytes + off, 16, 1024);
           mma_bf16_ss(d_tmem, ad, bd, idS, ks > 0 ? 1u : 0u);
         }
-        mma_commit(&bars->kempty[st]);
-        mma_commit(&bars->s_full[j & 1]);
+        mma_commit(&bars->s_full[i]);
+        if (!two || i == 1) mma_commit(&bars->kempty[st]);  // last reader of K(kv)
+        return true;
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort);
-      if (ok) ok = mbar_wait(&bars->kfull[0], 0, abort);
-      if (ok) {
+      // O_i += P_i V(kv), P_i from tensor memory
+      auto issue_pv = [&](int i, int t) -> bool {
+        const int kv = kv_of(i, t), st = kv % kStages;
+        if (!mbar_wait(&bars->p_full[i], t & 1, abort)) return false;
+        if (!mbar_wait(&bars->vfull[st], (kv / kStages) & 1, abort)) return false;
         tc_fence_after();
-        issue_s(0);
-      }
-      for (int j = 0; j < T && ok; ++j) {
-        if (j + 1 < T) {
-          const int st1 = (j + 1) % kStages;
-          if (!mbar_wait(&bars->kfull[st1], ((j + 1) / kStages) & 1, abort)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(j + 1);
-        }
-        const int st = j % kStages;
-        if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort)) { ok = false; break; }
-        if (!mbar_wait(&bars->vfull[st], (j / kStages) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t o_tmem = tmem + 2u * kTileN;
-        const uint32_t pb = p_addr + static_cast<uint32_t>((j & 1) * L::kPBytes);
+        const uint32_t o_tmem = tmem + 2u * kTileN + static_cast<uint32_t>(i * HD);
+        const uint32_t p_tmem = tmem + static_cast<uint32_t>(i * kTileN);
 #pragma unroll
         for (int ks = 0; ks < kTileN / 16; ++ks) {
-          const uint32_t aoff = static_cast<uint32_t>((ks >> 2) * L::kSlab + (ks & 3) * 32);
-          const uint64_t ad = smem_desc_sw128(pb + aoff, 16, 1024);
           const uint64_t bd =
               smem_desc_sw128(v_addr + st * L::kKVBytes + ks * 16 * 128, L::kSlab, 1024);
-          mma_bf16_ss(o_tmem, ad, bd, idO, (j > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(o_tmem, p_tmem + static_cast<uint32_t>(ks * 8), bd, idO,
+                      (t > 0 || ks > 0) ? 1u : 0u);
         }
-        mma_commit(&bars->vempty[st]);
-        mma_commit(&bars->pv_done[j & 1]);
-      }
+        if (!two || i == 1) mma_commit(&bars->vempty[st]);  // last reader of V(kv)
+        if (t == ntask[i] - 1) mma_commit(&bars->o_done[i]);
+        return true;
+      };
+      for (int i = 0; i < 2 && ok; ++i)
+        if (ntask[i] > 0) ok = issue_s(i, 0);
+      const int nt = max(ntask[0], ntask[1]);
+      for (int t = 0; t < nt && ok; ++t)
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (t >= ntask[i]) continue;
+          ok = issue_pv(i, t);
+          if (ok && t + 1 < ntask[i]) ok = issue_s(i, t + 1);
+        }
       // all issued MMAs complete before the CTA releases tensor memory
       mma_commit(&bars->mma_idle);
       volatile int never = 0;
       mbar_wait(&bars->mma_idle, 0, &never);
     }
   } else {
-    // ------------- softmax (warps 0-7): two threads per query row -------------
-    // warp w owns TMEM lanes 32*(w%4).. (rows) and key columns 64*(w/4)..+63;
-    // the two halves of a row agree on the row maximum through shared memory
-    constexpr int kHalf = kTileN / 2;
-    const int quarter = warp & 3, half = warp >> 2;
-    const int row = quarter * 32 + lane;  // 0..127 == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>((quarter * 32) << 16);
-    const uint32_t o_tmem = tmem + lane_base + 2u * kTileN + half * (HD / 2);
-    const uint32_t xch = tmem + lane_base + kXchCol;  // columns: 2 buffers x 2 halves
+    // ------------- softmax: warpgroup i = warp / 4, thread = row -------------
+    const int i = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;  // 0..127 == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(((warp & 3) * 32) << 16);
+    const uint32_t s_tmem = tmem + lane_base + static_cast<uint32_t>(i * kTileN);
+    const uint32_t o_base = tmem + lane_base + 2u * kTileN;
     const float sc = p.sc;
     float m_ref = -INFINITY, l_sum = 0.f;
-    SlotIter it;
-    it.init(runs, nr);
+    MaskWalk mw;
+    mw.init(runs, nr, ns);
     bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      // which of this half's 64 key columns are real keys
-      uint32_t vmask[2] = {0, 0};
-#pragma unroll
-      for (int s = 0; s < kSlotsPerTile; ++s) {
-        int st0 = 0, vv = 0;
-        if (!it.next(st0, vv)) vv = 0;
-        const uint32_t bits = (vv >= 8) ? 0xFFu : ((1u << vv) - 1u);
-        if ((s >> 3) == half) vmask[(s >> 2) & 1] |= bits << ((s & 3) * 8);
+    for (int t = 0; t < ntask[i]; ++t) {
+      const int kv = two ? t : 2 * t + i;
+      uint32_t vm[4];
+      if (!two && i == 1) {
+        uint32_t skip[4];
+        mw.tile(kv - 1, skip);  // advance past the other warpgroup's tile
       }
-      if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort)) { ok = false; break; }
+      mw.tile(kv, vm);
+      if (!two && i == 0 && kv + 1 < T) {
+        uint32_t skip[4];
+        mw.tile(kv + 1, skip);
+      }
+      // tcgen05.ld / st below are warp-collective: the warp proceeds or stops as one
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], t & 1, abort))) { ok = false; break; }
       tc_fence_after();
-      float sv[kHalf];
-      {
-        uint32_t r[kHalf];
-        const uint32_t s_tmem =
-            tmem + lane_base + static_cast<uint32_t>((j & 1) * kTileN + half * kHalf);
-        tmem_ld32(s_tmem + 0, *reinterpret_cast<uint32_t(*)[32]>(r + 0));
-        tmem_ld32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-        tmem_wait_ld();
+      uint32_t r[kTileN];
 #pragma unroll
-        for (int i = 0; i < kHalf; ++i)
-          sv[i] = ((vmask[i >> 5] >> (i & 31)) & 1u) ? __uint_as_float(r[i]) * sc : -INFINITY;
+      for (int c = 0; c < kTileN / 32; ++c)
+        tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
+      tmem_wait_ld();
+      if ((vm[0] & vm[1] & vm[2] & vm[3]) != 0xFFFFFFFFu) {
+        // only partial or padding slots (the same for every row) are touched
+#pragma unroll
+        for (int sl = 0; sl < kSlotsPerTile; ++sl) {
+          const uint32_t b = (vm[sl >> 2] >> ((sl & 3) * 8)) & 0xFFu;
+          if (b != 0xFFu) {
+#pragma unroll
+            for (int q = 0; q < kSlotRows; ++q)
+              if (!((b >> q) & 1u)) r[sl * kSlotRows + q] = __float_as_uint(-INFINITY);
+          }
+        }
       }
-      // row maximum of this half: eight independent chains, then a tree
+      // row maximum: eight independent chains, then a tree
       float m8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = sv[k];
+      for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(r[k]);
 #pragma unroll
-      for (int i = 8; i < kHalf; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      // row maximum over both halves (through tensor memory)
-      mx = fmaxf(mx, exchange_pair(xch + (j & 1) * 2, half, quarter, mx));
-      // reference maximum for this tile (moves only when it grows by > 2^8)
+      for (int c = 8; c < kTileN; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(r[c]));
+      const float mx = sc * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                  fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      // reference maximum (moves only when it grows by more than 2^8)
       float alpha = 1.f;
       bool need = false;
-      if (j == 0) {
+      if (t == 0) {
         m_ref = mx;
       } else if (mx > m_ref + kRescaleThreshold) {
         need = true;
         alpha = ex2_approx(m_ref - mx);
         m_ref = mx;
       }
-      // P = 2^(s - m_ref): bf16 pairs in registers, partial row sum in fp32
-      uint32_t pk[kHalf / 2];
+      // P = 2^(s sc - m_ref) as bf16 pairs over the first 64 columns of S_i;
+      // row sum in fp32. S_i(t) was produced after P_i(t-1) V completed, so
+      // these columns are free.
       float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float nm = -m_ref;
 #pragma unroll
-      for (int i = 0; i < kHalf; i += 2) {
-        const float a = ex2_approx(sv[i] - m_ref), b = ex2_approx(sv[i + 1] - m_ref);
-        r8[(i >> 1) & 7] += a + b;
-        pk[i >> 1] = pack_bf16x2(a, b);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float xa = fmaf(__uint_as_float(r[hf * 64 + c]), sc, nm);
+          const float xb = fmaf(__uint_as_float(r[hf * 64 + c + 1]), sc, nm);
+          const bool poly = ((c >> 1) & 3) == 3;  // one pair in four
+          const float a = poly ? exp2_poly(xa) : ex2_approx(xa);
+          const float b = poly ? exp2_poly(xb) : ex2_approx(xb);
+          r8[(c >> 1) & 7] += a + b;
+          pk[c >> 1] = pack_bf16x2(a, b);
+        }
+        tmem_st32(s_tmem + hf * 32, pk);
       }
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      // P buffer (j & 1) is free once P(j-2) V(j-2) has completed
-      if (j >= 2 && !mbar_wait(&bars->pv_done[j & 1], ((j - 2) >> 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
       if (__any_sync(0xffffffffu, need)) {
-        // O must hold P(j-1) V(j-1) before it is rescaled (this half's columns)
-        if (!mbar_wait(&bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        // P_i(t-1) V has completed (it precedes S_i(t)); O_i is not read again
+        // before P_i(t) is published below
+        const uint32_t o_tmem = o_base + static_cast<uint32_t>(i * HD);
 #pragma unroll
-        for (int c = 0; c < HD / 64; ++c) {
-          uint32_t r[32];
-          tmem_ld32(o_tmem + c * 32, r);
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_tmem + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(o_tmem + c * 32, r);
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(o_tmem + c * 32, o);
         }
-        tmem_wait_st();
       }
       l_sum = l_sum * alpha + rs;
-      uint8_t* pbuf = Ps + (j & 1) * L::kPBytes + half * L::kSlab;
-#pragma unroll
-      for (int c8 = 0; c8 < kHalf / 8; ++c8) {
-        const uint4 v4 = make_uint4(pk[c8 * 4 + 0], pk[c8 * 4 + 1], pk[c8 * 4 + 2], pk[c8 * 4 + 3]);
-        *reinterpret_cast<uint4*>(pbuf + swz(row, c8)) = v4;
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[j & 1]);
+      mbar_arrive(&bars->p_full[i]);
     }
     // ---------------- epilogue: O / l -> global (fp32, group-major rows) ------
-    // both halves of a row combine their partial sums (buffer T & 1 is free:
-    // the partner read buffer (T-1) & 1 last)
-    l_sum += exchange_pair(xch + (T & 1) * 2, half, quarter, l_sum);
-    if (ok && mbar_wait(&bars->pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort)) {
-      tc_fence_after();
-      const float inv = 1.f / l_sum;
-      float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD + half * (HD / 2);
+    if (two) {
+      if (__all_sync(0xffffffffu, ok && mbar_wait(&bars->o_done[i], 0, abort))) {
+        tc_fence_after();
+        const float inv = 1.f / l_sum;
+        const uint32_t o_tmem = o_base + static_cast<uint32_t>(i * HD);
+        const bool valid = i * kTileM + row < rows_unit;
+        float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row) * HD;
 #pragma unroll
-      for (int c = 0; c < HD / 64; ++c) {
-        uint32_t r[32];
-        tmem_ld32(o_tmem + c * 32, r);
-        tmem_wait_ld();
-        if (row < rows_valid) {
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_tmem + c * 32, o);
+          tmem_wait_ld();
+          if (valid) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(orow + c * 32 + i) =
-                make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
-                            __uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
+            for (int k = 0; k < 32; k += 4)
+              *reinterpret_cast<float4*>(orow + c * 32 + k) =
+                  make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
+                              __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+          }
+        }
+      }
+    } else {
+      // merge the two halves of the key tiles: each warpgroup writes half of
+      // the columns of every row
+      ml[i * 2 * kTileM + row] = m_ref;
+      ml[i * 2 * kTileM + kTileM + row] = l_sum;
+      named_barrier_sync(1, 2 * kTileM);
+      const float m0 = ml[row], l0 = ml[kTileM + row];
+      const float m1 = ml[2 * kTileM + row], l1 = ml[3 * kTileM + row];
+      const bool has1 = ntask[1] > 0;
+      const float mm = has1 ? fmaxf(m0, m1) : m0;
+      const float a0 = ex2_approx(m0 - mm), a1 = has1 ? ex2_approx(m1 - mm) : 0.f;
+      const float inv = 1.f / (l0 * a0 + l1 * a1);
+      const float f0 = a0 * inv, f1 = a1 * inv;
+      ok = ok && mbar_wait(&bars->o_done[0], 0, abort);
+      if (has1) ok = ok && mbar_wait(&bars->o_done[1], 0, abort);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const bool valid = row < rows_unit;
+        float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD;
+#pragma unroll
+        for (int c = 0; c < HD / 64; ++c) {
+          const int col = i * (HD / 2) + c * 32;
+          uint32_t o0[32], o1[32];
+          tmem_ld32(o_base + col, o0);
+          if (has1) tmem_ld32(o_base + HD + col, o1);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 4) {
+              float4 v;
+              v.x = __uint_as_float(o0[k]) * f0 + (has1 ? __uint_as_float(o1[k]) * f1 : 0.f);
+              v.y = __uint_as_float(o0[k + 1]) * f0 + (has1 ? __uint_as_float(o1[k + 1]) * f1 : 0.f);
+              v.z = __uint_as_float(o0[k + 2]) * f0 + (has1 ? __uint_as_float(o1[k + 2]) * f1 : 0.f);
+              v.w = __uint_as_float(o0[k + 3]) * f0 + (has1 ? __uint_as_float(o1[k + 3]) * f1 : 0.f);
+              *reinterpret_cast<float4*>(orow + col + k) = v;
+            }
+          }
         }
       }
     }
@@ -472,7 +527,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Work list: one entry per 128-row tile of each query group, (g << 16) | t.
+// Work list: one entry per 256-row unit of each query group, (g << 16) | u.
 // One warp per head: tile counts are prefix-summed 32 groups at a time.
 // ---------------------------------------------------------------------------
 __global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_head, int32_t* work,
@@ -484,7 +539,7 @@ __global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_hea
   for (int g0 = 0; g0 < Cq; g0 += 32) {
     const int g = g0 + lane;
     const int n = (g < Cq) ? oq[g + 1] - oq[g] : 0;
-    const int t = n > 0 ? (n + kTileM - 1) / kTileM : 0;
+    const int t = n > 0 ? (n + kUnitRows - 1) / kUnitRows : 0;
     int x = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -574,28 +629,10 @@ __global__ void cast_bf16_kernel(const float* src, __nv_bfloat16* dst, size_t n)
 // ---------------------------------------------------------------------------
 // Host side: tensor maps (driver entry point fetched through the runtime).
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 // 2D bf16 map over [rows, d] with a box of 64 columns x box_rows rows,
 // 128-byte swizzle; rows past the end read as zero.
 bool make_map(CUtensorMap* m, const void* base, size_t rows, int d, int box_rows) {
-  EncodeTiledFn enc = get_encode();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};

@@ -22,8 +22,8 @@ namespace {
 constexpr int kTriThreads = 512;
 constexpr int kInvIters = 3;
 
-// Scratch per matrix (fp64): hv [D][D] Householder vectors (column k holds
-// v_k at rows k+1.., v_k[0] = 1), tau [D], dg [D], od [D].
+// Scratch per matrix (fp64): hv [D][D] Householder vectors (row k holds v_k
+// at columns k+1.., v_k[0] = 1), tau [D], dg [D], od [D].
 template <int D>
 __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in, double* scratch) {
   extern __shared__ double tsm[];
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
         tau[k] = 0.0;
         od[k] = alpha;
       }
-      for (int i = tid; i < n1; i += blockDim.x) hv[(k + 1 + i) * D + k] = (i == 0) ? 1.0 : 0.0;
+      for (int i = tid; i < n1; i += blockDim.x) hv[k * D + (k + 1 + i)] = (i == 0) ? 1.0 : 0.0;
       __syncthreads();
       continue;
     }
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
     for (int i = tid; i < n1; i += blockDim.x) {
       const double vi = (i == 0) ? 1.0 : A[(k + 1 + i) * D + k] * scl;
       v[i] = vi;
-      hv[(k + 1 + i) * D + k] = vi;
+      hv[k * D + (k + 1 + i)] = vi;
     }
     if (tid == 0) {
       tau[k] = tk;
@@ -138,55 +138,60 @@ __device__ int sturm_count(const double* dg, const double* e2, double x, double 
 }
 
 // Solve (T - lam I) y = b in place (b <- y) with a partial-pivoting LU of
-// the tridiagonal system; a, dl, du, du2 are thread-private work arrays.
-template <int D>
+// the tridiagonal system. a, dl, du, du2, pv are the calling thread's work
+// arrays in shared memory, element i at [i * S] (S threads interleaved).
+template <int D, int S>
 __device__ void tri_solve(const double* dg, const double* od, double lam, double tiny, double* a,
                           double* dl, double* du, double* du2, int* pv, double* b) {
-  for (int i = 0; i < D; ++i) a[i] = dg[i] - lam;
+  for (int i = 0; i < D; ++i) a[i * S] = dg[i] - lam;
   for (int i = 0; i < D - 1; ++i) {
-    dl[i] = od[i];
-    du[i] = od[i];
-    du2[i] = 0.0;
+    dl[i * S] = od[i];
+    du[i * S] = od[i];
+    du2[i * S] = 0.0;
   }
 #pragma unroll 1
   for (int i = 0; i < D - 1; ++i) {
-    if (fabs(a[i]) >= fabs(dl[i])) {
-      if (a[i] == 0.0) a[i] = tiny;
-      const double f = dl[i] / a[i];
-      dl[i] = f;
-      a[i + 1] -= f * du[i];
-      pv[i] = 0;
+    const double ai = a[i * S], li = dl[i * S];
+    if (fabs(ai) >= fabs(li)) {
+      const double piv = (ai == 0.0) ? tiny : ai;
+      a[i * S] = piv;
+      const double f = li / piv;
+      dl[i * S] = f;
+      a[(i + 1) * S] -= f * du[i * S];
+      pv[i * S] = 0;
     } else {
-      const double f = a[i] / dl[i];
-      a[i] = dl[i];
-      dl[i] = f;
-      const double t = du[i];
-      du[i] = a[i + 1];
-      a[i + 1] = t - f * a[i + 1];
+      const double f = ai / li;
+      a[i * S] = li;
+      dl[i * S] = f;
+      const double t = du[i * S];
+      const double an = a[(i + 1) * S];
+      du[i * S] = an;
+      a[(i + 1) * S] = t - f * an;
       if (i < D - 2) {
-        du2[i] = du[i + 1];
-        du[i + 1] = -f * du[i + 1];
+        du2[i * S] = du[(i + 1) * S];
+        du[(i + 1) * S] = -f * du[(i + 1) * S];
       }
-      pv[i] = 1;
+      pv[i * S] = 1;
     }
   }
-  if (a[D - 1] == 0.0) a[D - 1] = tiny;
+  if (a[(D - 1) * S] == 0.0) a[(D - 1) * S] = tiny;
   // L solve
 #pragma unroll 1
   for (int i = 0; i < D - 1; ++i) {
-    if (pv[i] == 0) {
-      b[i + 1] -= dl[i] * b[i];
+    if (pv[i * S] == 0) {
+      b[i + 1] -= dl[i * S] * b[i];
     } else {
       const double t = b[i];
       b[i] = b[i + 1];
-      b[i + 1] = t - dl[i] * b[i];
+      b[i + 1] = t - dl[i * S] * b[i];
     }
   }
   // U solve
-  b[D - 1] /= a[D - 1];
-  b[D - 2] = (b[D - 2] - du[D - 2] * b[D - 1]) / a[D - 2];
+  b[D - 1] /= a[(D - 1) * S];
+  b[D - 2] = (b[D - 2] - du[(D - 2) * S] * b[D - 1]) / a[(D - 2) * S];
 #pragma unroll 1
-  for (int i = D - 3; i >= 0; --i) b[i] = (b[i] - du[i] * b[i + 1] - du2[i] * b[i + 2]) / a[i];
+  for (int i = D - 3; i >= 0; --i)
+    b[i] = (b[i] - du[i * S] * b[i + 1] - du2[i * S] * b[i + 2]) / a[i * S];
 }
 
 constexpr int kEigThreads = 256;
@@ -195,9 +200,14 @@ constexpr int kEigThreads = 256;
 // inverse iteration by thread t, clustered Gram-Schmidt by warp 0, then
 // back-transformation by warp t % 8. Writes evals [H, ne] and evecs [H, D, ne].
 template <int D>
+constexpr size_t eig_work_bytes() {
+  return static_cast<size_t>(4) * D * 32 * 8 + static_cast<size_t>(D) * 32 * 4;
+}
+
+template <int D>
 __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scratch, int ne,
-                                                       double* evals, double* evecs,
-                                                       double* work) {
+                                                       double* evals, double* evecs) {
+  extern __shared__ double eig_work[];  // inverse-iteration work arrays, 32 threads interleaved
   __shared__ double dg[D], od[D], e2[D];
   __shared__ double lam[32];
   __shared__ double Y[32][D + 1];  // padded: thread t walks row t
@@ -222,24 +232,35 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   double emax2 = 0.0;
   for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
   const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
-  // bisection: thread t finds the eigenvalue of ascending index D-1-t
-  if (tid < ne) {
-    const int m = D - 1 - tid;
+  // multisection: eight threads per wanted eigenvalue (rank e_i = tid / 8,
+  // ascending index D-1-e_i) evaluate the Sturm count at eight interior
+  // points of the current interval, which shrinks nine-fold per round
+  {
+    const int e_i = tid >> 3, q = tid & 7;
+    const bool act = e_i < ne;
+    const int m = D - 1 - e_i;
     double lo = -tnorm - 1.0, hi = tnorm + 1.0;
-    for (int it = 0; it < 200; ++it) {
-      const double mid = 0.5 * (lo + hi);
-      if (hi - lo <= 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin || mid == lo || mid == hi) break;
-      if (sturm_count<D>(dg, e2, mid, pivmin) <= m)
-        lo = mid;
-      else
-        hi = mid;
+    for (int it = 0; it < 100; ++it) {
+      const double w = hi - lo;
+      const bool done = !(w > 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin);
+      if (__all_sync(0xffffffffu, done || !act)) break;
+      bool pred = false;
+      if (act && !done) pred = sturm_count<D>(dg, e2, lo + w * (q + 1) * (1.0 / 9.0), pivmin) <= m;
+      const unsigned bal = __ballot_sync(0xffffffffu, pred);
+      const int nt = __popc((bal >> ((lane >> 3) * 8)) & 0xFFu);  // points below lambda
+      if (act && !done) {
+        const double nlo = nt > 0 ? lo + w * nt * (1.0 / 9.0) : lo;
+        const double nhi = nt < 8 ? lo + w * (nt + 1) * (1.0 / 9.0) : hi;
+        lo = nlo;
+        hi = nhi;
+      }
     }
-    lam[tid] = 0.5 * (lo + hi);
+    if (act && q == 0) lam[e_i] = 0.5 * (lo + hi);
   }
   __syncthreads();
   // inverse iteration from a fixed, index-dependent start vector
-  double* wk = work + (static_cast<size_t>(h) * 32 + tid) * (5 * D);
-  int* pv = reinterpret_cast<int*>(wk + 4 * D);
+  double* wk = eig_work + (tid & 31);
+  int* pv = reinterpret_cast<int*>(eig_work + 4 * D * 32) + (tid & 31);
   const double tiny = eps * fmax(tnorm, 1e-300);
   if (tid < ne)
     for (int i = 0; i < D; ++i) Y[tid][i] = 1.0 + 0.5 * sin(0.7 * (i + 1) * (tid + 1));
@@ -247,7 +268,7 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   for (int it = 0; it < kInvIters; ++it) {
     if (tid < ne) {
       double* b = Y[tid];
-      tri_solve<D>(dg, od, lam[tid], tiny, wk, wk + D, wk + 2 * D, wk + 3 * D, pv, b);
+      tri_solve<D, 32>(dg, od, lam[tid], tiny, wk, wk + D * 32, wk + 2 * D * 32, wk + 3 * D * 32, pv, b);
       double s = 0.0;
       for (int i = 0; i < D; ++i) s = fma(b[i], b[i], s);
       const double inv = 1.0 / sqrt(s);
@@ -282,9 +303,9 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
       const double tk = tau[k];
       if (tk == 0.0) continue;
       double dot = 0.0;
-      for (int i = k + 1 + lane; i < D; i += 32) dot = fma(hv[i * D + k], y[i], dot);
+      for (int i = k + 1 + lane; i < D; i += 32) dot = fma(hv[k * D + i], y[i], dot);
       dot = warp_sum_f64(dot) * tk;
-      for (int i = k + 1 + lane; i < D; i += 32) y[i] -= dot * hv[i * D + k];
+      for (int i = k + 1 + lane; i < D; i += 32) y[i] -= dot * hv[k * D + i];
       __syncwarp();
     }
     for (int i = lane; i < D; i += 32)
@@ -295,30 +316,31 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
 
 template <int D>
 cudaError_t launch_d(const double* A, int H, int ne, double* evals, double* evecs,
-                     double* scratch, double* work, cudaStream_t st) {
+                     double* scratch, cudaStream_t st) {
   const size_t shb = (static_cast<size_t>(D) * D + 2 * D) * 8;
   cudaError_t e = cudaFuncSetAttribute(tridiag_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(shb));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tri_eig_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(eig_work_bytes<D>()));
+  if (e != cudaSuccess) return e;
   tridiag_kernel<D><<<H, kTriThreads, shb, st>>>(A, scratch);
-  tri_eig_kernel<D><<<H, kEigThreads, 0, st>>>(scratch, ne, evals, evecs, work);
+  tri_eig_kernel<D><<<H, kEigThreads, eig_work_bytes<D>(), st>>>(scratch, ne, evals, evecs);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t sym_eigs_scratch_doubles(int H, int d) {
-  return static_cast<size_t>(H) * (static_cast<size_t>(d) * d + 3 * d) +
-         static_cast<size_t>(H) * 32 * 5 * d;
+  return static_cast<size_t>(H) * (static_cast<size_t>(d) * d + 3 * d);
 }
 
 cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals, double* evecs,
                             double* scratch, cudaStream_t st) {
   if (ne < 1 || ne > 32 || ne > d) return cudaErrorInvalidValue;
-  double* work = scratch + static_cast<size_t>(H) * (static_cast<size_t>(d) * d + 3 * d);
-  if (d == 128) return launch_d<128>(A, H, ne, evals, evecs, scratch, work, st);
-  if (d == 64) return launch_d<64>(A, H, ne, evals, evecs, scratch, work, st);
+  if (d == 128) return launch_d<128>(A, H, ne, evals, evecs, scratch, st);
+  if (d == 64) return launch_d<64>(A, H, ne, evals, evecs, scratch, st);
   return cudaErrorInvalidValue;
 }
 

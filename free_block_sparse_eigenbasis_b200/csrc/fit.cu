@@ -198,7 +198,7 @@ __global__ void project_map_kernel(const double* bmat, const double* bvec, const
     double s = 0.0;
     for (int t = 0; t < r; ++t) s = fma(T[t], V[static_cast<size_t>(col) * r + t], s);
     if (a < d) {
-      bp32[(static_cast<size_t>(h) * d + a) * d + col] = static_cast<float>(s);
+      bp32[(static_cast<size_t>(h) * d + col) * d + a] = static_cast<float>(s);  // B'^T
       if (fit_out) fit_out[static_cast<size_t>(h) * (d * d + d) + a * d + col] = s;
     } else {
       bv32[static_cast<size_t>(h) * d + col] = static_cast<float>(s);
@@ -209,6 +209,7 @@ __global__ void project_map_kernel(const double* bmat, const double* bvec, const
 
 // out[perm_q[i]] = O_dense(probe) for probe rows, else x + b' + x B'
 // (x = o_sparse row, fp32); 32 group-major rows per CTA, B' in shared memory.
+// CUDA-core form for inputs too small for the tensor-core kernel.
 constexpr int kCorrRows = 32;
 
 template <bool OUT_BF16>
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(256) correct_kernel(const float* o_sparse, con
   const int h = blockIdx.y;
   const int i0 = blockIdx.x * kCorrRows;
   const float* Bh = bp32 + static_cast<size_t>(h) * d * d;
-  for (int t = threadIdx.x; t < d * d; t += blockDim.x) Bs[t] = Bh[t];
+  for (int t = threadIdx.x; t < d * d; t += blockDim.x) Bs[(t % d) * d + t / d] = Bh[t];  // B' from B'^T
   for (int t = threadIdx.x; t < kCorrRows * d; t += blockDim.x) {
     const int r = t / d, a = t % d;
     const int i = i0 + r;

@@ -10,6 +10,14 @@
 
 namespace spr {
 
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry point
+// (null if the driver does not provide it).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
 // ---- sort.cu: stable counting sort of per-head labels ----------------------
 // labels [H, n] in 0..C-1 -> perm [H, n] (group-major order, ascending token
 // index inside a group) and off [H, C+1]. Heads with skip[h] != 0 are left
@@ -136,6 +144,12 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, 
 cudaError_t launch_route(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
                          double scale, const int32_t* kh, int kmax, int32_t* csr,
                          cudaStream_t st);
+// Workspace path: score GEMM + warp top-k, heads in groups whose scores fit
+// in `scores` (route_scores_bytes(H, Cq, Ck) bytes).
+size_t route_scores_bytes(int H, int Cq, int Ck);
+cudaError_t launch_route_gemm(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
+                              double scale, const int32_t* kh, int kmax, double* scores,
+                              size_t scores_bytes, int32_t* csr, cudaStream_t st);
 cudaError_t launch_range_mean(const void* X, int x_kind, int H, int N, int d, const int32_t* off,
                               int C, double* out, cudaStream_t st);
 cudaError_t launch_write_k(const int32_t* kh_host_vals, int H, int32_t* k_per_head,
@@ -178,10 +192,18 @@ cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const
                                    cudaStream_t st);
 cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
                                const double* means, DeviceStats* stats, cudaStream_t st);
-// B' = (B V_r) V_r^T, b' = (b V_r) V_r^T with vr [H, d, r].
+// B' = (B V_r) V_r^T, b' = (b V_r) V_r^T with vr [H, d, r]; bp32 holds B'^T
+// ([H, column, row]), fit_out (optional) B' row-major and b' in fp64.
 cudaError_t launch_project_map(const double* bmat, const double* bvec, const double* vr, int H,
                                int d, int r, float* bp32, float* bv32, double* fit_out,
                                cudaStream_t st);
+// ---- correct.cu: tensor-core residual correction ---------------------------
+bool correct_tc_supported(int H, int N, int d);
+// out[perm_q[i]] = od[probe] for probe rows, else x + x B' + b' (bpT = B'^T).
+cudaError_t launch_correct_tc(const float* o_sparse, const float* od, const int32_t* probes,
+                              const int32_t* perm_q, const float* bpT, const float* bv32, int H,
+                              int N, int M, int d, void* out, bool out_bf16, int sm_count,
+                              DeviceStats* stats, cudaStream_t st);
 cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t* probes,
                            const int32_t* perm_q, const float* bp32, const float* bv32, int H,
                            int N, int M, int d, void* out, bool out_bf16, cudaStream_t st);

@@ -28,7 +28,7 @@ struct Layout {
   size_t mk;       // [H, d, d] f64 (M_K, later the probe residual Gram R^T R)
   size_t evec;     // [H, d, d] f64 Jacobi eigenvectors (columns)
   size_t eval;     // [H, d] f64 Jacobi eigenvalues
-  size_t eigscr;   // tridiagonal eigensolver scratch: [H, d*d + 3d] + [H, 32, 5d] f64
+  size_t eigscr;   // tridiagonal eigensolver scratch: [H, d*d + 3d] f64
   size_t wk;       // [H, d, e] f64 key projector U_e L_e^{1/2}
   size_t z;        // [H, Nv, e] f64 key coordinates
   size_t mu;       // [H, Ck, e] f64 key centroids
@@ -59,6 +59,7 @@ struct Layout {
   // stage 3
   size_t cq;       // [H, Cq, d] f64 query-group means (route)
   size_t ckr;      // [H, Ck, d] f64 key-group means (route)
+  size_t scores;   // [heads per pass, Cq, Ck] f64 block scores (route)
   size_t bf16_qkv; // [3, H, N, d] bf16 copies (fp32 inputs only)
   size_t work;     // [H, tiles_per_head] int32 attention work list
   size_t nwork;    // [H] int32
@@ -83,6 +84,7 @@ struct Layout {
 
   int Nv, e, Cmax, nchunk, tiles_per_head, kmax;
   int Dpk, CpadK, CpadQ;
+  size_t scores_bytes;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -127,7 +129,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->mk = take(H * d * d * 8);
   L->evec = take(H * d * d * 8);
   L->eval = take(H * d * 8);
-  L->eigscr = take((H * (d * d + 3 * d) + H * 32 * 5 * d) * 8);
+  L->eigscr = take(H * (d * d + 3 * d) * 8);
   L->wk = take(H * d * e * 8);
   L->z = take(H * Nv * e * 8);
   L->mu = take(H * Ck * e * 8);
@@ -159,6 +161,14 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->nrecheck = take(H * 4);
   L->cq = take(H * Cq * d * 8);
   L->ckr = take(H * Ck * d * 8);
+  {
+    const size_t per_head = Cq * Ck * 8;
+    size_t heads = (static_cast<size_t>(64) << 20) / per_head;
+    if (heads < 1) heads = 1;
+    if (heads > H) heads = H;
+    L->scores_bytes = heads * per_head;
+    L->scores = take(L->scores_bytes);
+  }
   L->bf16_qkv = take(3 * H * N * d * 2);
   L->work = take(H * static_cast<size_t>(L->tiles_per_head) * 4);
   L->nwork = take(H * 4);

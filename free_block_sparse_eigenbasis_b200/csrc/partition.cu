@@ -135,11 +135,36 @@ __global__ void gram_f64_kernel(const double* X, const double* Y, const double* 
 // ---------------------------------------------------------------------------
 // Key response coordinates z = W^T k, W = U_e L_e^{1/2} ([d, e] fp64).
 // ---------------------------------------------------------------------------
-constexpr int kZRows = 64;
+constexpr int kZRows = 128;
+constexpr int kZThreads = 256;
 
+// 16-byte vector of k widened to float
+__device__ __forceinline__ int zvec_elems(const __nv_bfloat16*) { return 8; }
+__device__ __forceinline__ int zvec_elems(const float*) { return 4; }
+__device__ __forceinline__ void zvec_store(const __nv_bfloat16* src, float* dst) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    dst[2 * i] = __uint_as_float(w[i] << 16);
+    dst[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void zvec_store(const float* src, float* dst) {
+  const float4 v = *reinterpret_cast<const float4*>(src);
+  dst[0] = v.x;
+  dst[1] = v.y;
+  dst[2] = v.z;
+  dst[3] = v.w;
+}
+
+// Block = 128 key rows: the rows are staged in shared memory with 16-byte
+// loads, then thread t computes 8 of the e coordinates of row t % 128 (one
+// shared load of k per 8 fma; w broadcast to the warp), summing over the d
+// columns in ascending order in fp64.
 template <typename T>
-__global__ void zproj_kernel(const T* k, int N, int Nv, int d, int e, const double* wk,
-                             double* z) {
+__global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int Nv, int d, int e,
+                                                          const double* wk, double* z) {
   extern __shared__ double zsm[];
   double* w = zsm;                  // [d][e]
   float* ks = reinterpret_cast<float*>(zsm + d * e);  // [kZRows][d+1]
@@ -148,20 +173,40 @@ __global__ void zproj_kernel(const T* k, int N, int Nv, int d, int e, const doub
   const double* W = wk + static_cast<size_t>(h) * d * e;
   for (int t = threadIdx.x; t < d * e; t += blockDim.x) w[t] = W[t];
   const T* kh = k + static_cast<size_t>(h) * N * d;
-  for (int t = threadIdx.x; t < kZRows * d; t += blockDim.x) {
-    const int r = t / d, a = t % d;
+  const int ve = zvec_elems(kh), vpr = d / ve;  // elements per vector, vectors per row
+  for (int t = threadIdx.x; t < kZRows * vpr; t += blockDim.x) {
+    const int r = t / vpr, a = (t % vpr) * ve;
     const int j = j0 + r;
-    ks[r * (d + 1) + a] = (j < Nv) ? static_cast<float>(to_f64(kh, static_cast<size_t>(j) * d + a)) : 0.f;
+    float tmp[8];
+    if (j < Nv) {
+      zvec_store(kh + static_cast<size_t>(j) * d + a, tmp);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tmp[i] = 0.f;
+    }
+    for (int i = 0; i < ve; ++i) ks[r * (d + 1) + a + i] = tmp[i];
   }
   __syncthreads();
-  // thread -> (row, output coordinate)
-  for (int t = threadIdx.x; t < kZRows * e; t += blockDim.x) {
-    const int r = t / e, c = t % e;
-    const int j = j0 + r;
-    if (j >= Nv) continue;
-    double acc = 0.0;
-    for (int a = 0; a < d; ++a) acc = fma(static_cast<double>(ks[r * (d + 1) + a]), w[a * e + c], acc);
-    z[(static_cast<size_t>(h) * Nv + j) * e + c] = acc;
+  const int r = threadIdx.x % kZRows;
+  const int j = j0 + r;
+  if (j >= Nv) return;
+  const float* kr = ks + r * (d + 1);
+  double* zr = z + (static_cast<size_t>(h) * Nv + j) * e;
+  for (int c0 = (threadIdx.x / kZRows) * 8; c0 < e; c0 += 16) {
+    const int ne = min(8, e - c0);
+    double acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.0;
+    for (int a = 0; a < d; ++a) {
+      const double kv = static_cast<double>(kr[a]);
+      const double* wa = w + a * e + c0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c < ne) acc[c] = fma(kv, wa[c], acc[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < ne) zr[c0 + c] = acc[c];
   }
 }
 
@@ -316,43 +361,73 @@ __global__ void finalize_pass_kernel(int H, int pass, int32_t* flags, int flag_b
 // One CTA of 4 warps per group: warp w sums the w-th quarter of the members
 // (ascending positions, lanes own coordinates), the four partial sums are
 // added in warp order.
-constexpr int kMeanWarps = 4;
+constexpr int kMeanThreads = 256;
 constexpr int kMeanMaxD = 128;
 
-__global__ void __launch_bounds__(kMeanWarps * 32) group_mean_kernel(
-    const void* X, int kind, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
+// One CTA per (group, head). Thread t sums column t % D over the rows
+// lo + t / D, lo + t / D + 256 / D, ... of the group (consecutive threads
+// read consecutive columns of one row), then the row lanes' partial sums
+// are added in shared memory in a fixed order.
+template <typename T>
+__device__ __forceinline__ double mean_ld(const T* X, size_t i) { return to_f64(X, i); }
+template <>
+__device__ __forceinline__ double mean_ld<double>(const double* X, size_t i) { return X[i]; }
+
+template <typename T>
+__global__ void __launch_bounds__(kMeanThreads) group_mean_kernel(
+    const T* X, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
     const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
     const int32_t* skip, int skip_stride) {
-  __shared__ double part[kMeanWarps][kMeanMaxD];
+  __shared__ double part[kMeanThreads];
+  __shared__ double red[kMeanThreads / 32];
   const int h = blockIdx.y, c = blockIdx.x;
   if (skip && skip[h * skip_stride]) return;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int32_t* oo = off + static_cast<size_t>(h) * off_stride;
   const int32_t* pp = perm ? perm + static_cast<size_t>(h) * perm_stride : nullptr;
   const int lo = oo[c], hi = oo[c + 1], n = hi - lo;
-  const int a = lo + static_cast<int>((static_cast<long long>(n) * w) / kMeanWarps);
-  const int b = lo + static_cast<int>((static_cast<long long>(n) * (w + 1)) / kMeanWarps);
-  for (int t0 = 0; t0 < D; t0 += 32) {
-    const int t = t0 + lane;
-    double acc = 0.0;
-    if (t < D) {
-#pragma unroll 8
-      for (int p = a; p < b; ++p) {
-        const size_t row = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
-        acc += load_x(X, kind, h * hsx + row * ldx + t);
+  const int RL = kMeanThreads / D;  // row lanes
+  const int col = threadIdx.x % D, rl = threadIdx.x / D;
+  const T* Xh = X + h * hsx;
+  double acc = 0.0;
+  if (rl < RL) {
+    int p = lo + rl;
+#pragma unroll 1
+    for (; p + 3 * RL < hi; p += 4 * RL) {
+      size_t r0, r1, r2, r3;
+      if (pp) {
+        r0 = pp[p];
+        r1 = pp[p + RL];
+        r2 = pp[p + 2 * RL];
+        r3 = pp[p + 3 * RL];
+      } else {
+        r0 = p;
+        r1 = p + RL;
+        r2 = p + 2 * RL;
+        r3 = p + 3 * RL;
       }
-      part[w][t] = acc;
+      const double v0 = mean_ld(Xh, r0 * ldx + col), v1 = mean_ld(Xh, r1 * ldx + col);
+      const double v2 = mean_ld(Xh, r2 * ldx + col), v3 = mean_ld(Xh, r3 * ldx + col);
+      acc += v0;
+      acc += v1;
+      acc += v2;
+      acc += v3;
+    }
+    for (; p < hi; p += RL) {
+      const size_t r = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
+      acc += mean_ld(Xh, r * ldx + col);
     }
   }
+  part[threadIdx.x] = acc;
   __syncthreads();
   double* dst = out + (static_cast<size_t>(h) * C + c) * D;
   double ss = 0.0;
   for (int t = threadIdx.x; t < D; t += blockDim.x) {
     double v;
     if (n > 0) {
-      double s = part[0][t];
-      for (int ww = 1; ww < kMeanWarps; ++ww) s += part[ww][t];
-      v = s / static_cast<double>(n);
+      double sum = part[t];
+      for (int q = 1; q < RL; ++q) sum += part[q * D + t];
+      v = sum / static_cast<double>(n);
     } else {
       v = keep_prev ? dst[t] : 0.0;
     }
@@ -360,14 +435,114 @@ __global__ void __launch_bounds__(kMeanWarps * 32) group_mean_kernel(
     ss = fma(v, v, ss);
   }
   if (norms) {
-    __shared__ double red[kMeanWarps];
     ss = warp_sum_f64(ss);
     if (lane == 0) red[w] = ss;
     __syncthreads();
     if (threadIdx.x == 0) {
-      double s = red[0];
-      for (int ww = 1; ww < kMeanWarps; ++ww) s += red[ww];
-      norms[static_cast<size_t>(h) * C + c] = s;
+      double sum = red[0];
+      for (int q = 1; q < kMeanThreads / 32; ++q) sum += red[q];
+      norms[static_cast<size_t>(h) * C + c] = sum;
+    }
+  }
+}
+
+// Vector form of the group mean for rows of D * sizeof(T) bytes that split
+// into 16-byte pieces: TPR = D * sizeof(T) / 16 threads per row, each summing
+// EPT = 16 / sizeof(T) columns over the rows lo + rl, lo + rl + RL, ...
+// (RL = 256 / TPR row lanes), then the row lanes' sums are added in a fixed
+// order.
+template <typename T>
+__device__ __forceinline__ void vload16(const T* p, double* out);
+template <>
+__device__ __forceinline__ void vload16<__nv_bfloat16>(const __nv_bfloat16* p, double* out) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = static_cast<double>(__uint_as_float(w[i] << 16));
+    out[2 * i + 1] = static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+  }
+}
+template <>
+__device__ __forceinline__ void vload16<float>(const float* p, double* out) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  out[0] = v.x;
+  out[1] = v.y;
+  out[2] = v.z;
+  out[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void vload16<double>(const double* p, double* out) {
+  const double2 v = *reinterpret_cast<const double2*>(p);
+  out[0] = v.x;
+  out[1] = v.y;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
+    const T* X, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
+    const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
+    const int32_t* skip, int skip_stride) {
+  constexpr int EPT = 16 / sizeof(T);
+  __shared__ double part[kMeanThreads * EPT];
+  __shared__ double red[kMeanThreads / 32];
+  const int h = blockIdx.y, c = blockIdx.x;
+  if (skip && skip[h * skip_stride]) return;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int32_t* oo = off + static_cast<size_t>(h) * off_stride;
+  const int32_t* pp = perm ? perm + static_cast<size_t>(h) * perm_stride : nullptr;
+  const int lo = oo[c], hi = oo[c + 1], n = hi - lo;
+  const int TPR = D / EPT, RL = kMeanThreads / TPR;
+  const int col = (threadIdx.x % TPR) * EPT, rl = threadIdx.x / TPR;
+  const T* Xh = X + h * hsx + col;
+  double acc[EPT];
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) acc[i] = 0.0;
+  int p = lo + rl;
+#pragma unroll 1
+  for (; p + RL < hi; p += 2 * RL) {
+    const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
+    const size_t r1 = pp ? static_cast<size_t>(pp[p + RL]) : static_cast<size_t>(p + RL);
+    double v0[EPT], v1[EPT];
+    vload16(Xh + r0 * ldx, v0);
+    vload16(Xh + r1 * ldx, v1);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] += v1[i];
+  }
+  if (p < hi) {
+    const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
+    double v0[EPT];
+    vload16(Xh + r0 * ldx, v0);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
+  }
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) part[rl * D + col + i] = acc[i];
+  __syncthreads();
+  double* dst = out + (static_cast<size_t>(h) * C + c) * D;
+  double ss = 0.0;
+  for (int t = threadIdx.x; t < D; t += blockDim.x) {
+    double v;
+    if (n > 0) {
+      double sum = part[t];
+      for (int q = 1; q < RL; ++q) sum += part[q * D + t];
+      v = sum / static_cast<double>(n);
+    } else {
+      v = keep_prev ? dst[t] : 0.0;
+    }
+    dst[t] = v;
+    ss = fma(v, v, ss);
+  }
+  if (norms) {
+    ss = warp_sum_f64(ss);
+    if (lane == 0) red[w] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double sum = red[0];
+      for (int q = 1; q < kMeanThreads / 32; ++q) sum += red[q];
+      norms[static_cast<size_t>(h) * C + c] = sum;
     }
   }
 }
@@ -444,11 +619,11 @@ cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, 
   if (bf16) {
     cudaFuncSetAttribute(zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(shb));
-    zproj_kernel<<<grid, 256, shb, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv, d, e, wk, z);
+    zproj_kernel<<<grid, kZThreads, shb, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv, d, e, wk, z);
   } else {
     cudaFuncSetAttribute(zproj_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(shb));
-    zproj_kernel<<<grid, 256, shb, st>>>(static_cast<const float*>(k), N, Nv, d, e, wk, z);
+    zproj_kernel<<<grid, kZThreads, shb, st>>>(static_cast<const float*>(k), N, Nv, d, e, wk, z);
   }
   return cudaGetLastError();
 }
@@ -481,11 +656,38 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx,
                               int off_stride, int C, int H, bool keep_prev, double* out,
                               double* norms, const int32_t* skip, int skip_stride,
                               cudaStream_t st) {
-  if (D > kMeanMaxD) return cudaErrorInvalidValue;
+  if (D > kMeanMaxD || D < 1) return cudaErrorInvalidValue;
   dim3 grid(C, H);
-  group_mean_kernel<<<grid, kMeanWarps * 32, 0, st>>>(X, x_kind, hsx, ldx, D, perm, perm_stride, off,
-                                          off_stride, C, keep_prev, out, norms, skip,
-                                          skip_stride);
+  const int es = (x_kind == kXf64) ? 8 : (x_kind == kXbf16 ? 2 : 4);
+  const bool vec = (D * es) % 16 == 0 && kMeanThreads % (D * es / 16) == 0 && (ldx * es) % 16 == 0 &&
+                   (hsx * es) % 16 == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+  if (vec) {
+    if (x_kind == kXf64)
+      group_mean_vec_kernel<<<grid, kMeanThreads, 0, st>>>(static_cast<const double*>(X), hsx, ldx,
+                                                           D, perm, perm_stride, off, off_stride, C,
+                                                           keep_prev, out, norms, skip, skip_stride);
+    else if (x_kind == kXbf16)
+      group_mean_vec_kernel<<<grid, kMeanThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(X), hsx, ldx, D, perm, perm_stride, off, off_stride, C,
+          keep_prev, out, norms, skip, skip_stride);
+    else
+      group_mean_vec_kernel<<<grid, kMeanThreads, 0, st>>>(static_cast<const float*>(X), hsx, ldx,
+                                                           D, perm, perm_stride, off, off_stride, C,
+                                                           keep_prev, out, norms, skip, skip_stride);
+    return cudaGetLastError();
+  }
+  if (x_kind == kXf64)
+    group_mean_kernel<<<grid, kMeanThreads, 0, st>>>(static_cast<const double*>(X), hsx, ldx, D,
+                                                     perm, perm_stride, off, off_stride, C,
+                                                     keep_prev, out, norms, skip, skip_stride);
+  else if (x_kind == kXbf16)
+    group_mean_kernel<<<grid, kMeanThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(X), hsx,
+                                                     ldx, D, perm, perm_stride, off, off_stride,
+                                                     C, keep_prev, out, norms, skip, skip_stride);
+  else
+    group_mean_kernel<<<grid, kMeanThreads, 0, st>>>(static_cast<const float*>(X), hsx, ldx, D,
+                                                     perm, perm_stride, off, off_stride, C,
+                                                     keep_prev, out, norms, skip, skip_stride);
   return cudaGetLastError();
 }
 

@@ -23,49 +23,72 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ src, uint4* __restr
 }
 
 // One CTA per (query group g, head h): fp64 scores of all key groups in
-// shared memory, top-k by rank (greater score first, lower index on ties),
-// kept ids written in ascending order.
+// shared memory (one warp per key group), a bitonic sort of (score, id)
+// pairs into the route order (greater score first, lower id on ties), and
+// the first k ids written in ascending order.
 constexpr int kRouteThreads = 256;
+
+__device__ __forceinline__ bool route_before(double sa, int ia, double sb, int ib) {
+  return sa > sb || (sa == sb && ia < ib);
+}
 
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const double* __restrict__ cq,
                                                               const double* __restrict__ ckr,
                                                               int Cq, int Ck, int d, double scale,
                                                               const int32_t* __restrict__ kh,
-                                                              int kmax, int32_t* __restrict__ csr) {
+                                                              int kmax, int P,
+                                                              int32_t* __restrict__ csr) {
   extern __shared__ double rsm[];
-  double* score = rsm;                                       // [Ck]
-  double* qv = rsm + Ck;                                     // [d]
-  int* kept = reinterpret_cast<int*>(qv + d);                // [Ck]
+  double* score = rsm;                                       // [P], P = pow2 >= Ck
+  double* qv = rsm + P;                                      // [d]
+  int* ids = reinterpret_cast<int*>(qv + d);                 // [P]
+  int* kept = ids + P;                                       // [Ck]
   __shared__ int wsum[kRouteThreads / 32];
   __shared__ int carry;
   const int g = blockIdx.x, h = blockIdx.y;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const double* qrow = cq + (static_cast<size_t>(h) * Cq + g) * d;
   for (int a = threadIdx.x; a < d; a += blockDim.x) qv[a] = qrow[a];
   __syncthreads();
   const double* ckh = ckr + static_cast<size_t>(h) * Ck * d;
-  for (int c = threadIdx.x; c < Ck; c += blockDim.x) {
+  for (int c = wid; c < Ck; c += kRouteThreads / 32) {
     const double* kr = ckh + static_cast<size_t>(c) * d;
     double acc = 0.0;
-    for (int a = 0; a < d; ++a) acc = fma(qv[a], kr[a], acc);
-    score[c] = scale * acc;
+    for (int a = lane; a < d; a += 32) acc = fma(qv[a], kr[a], acc);
+    acc = warp_sum_f64(acc);
+    if (lane == 0) score[c] = scale * acc;
+  }
+  for (int c = threadIdx.x; c < P; c += blockDim.x) {
+    ids[c] = c;
+    if (c >= Ck) score[c] = -INFINITY;  // padding sorts last
   }
   __syncthreads();
-  const int k = kh[h];
-  for (int c = threadIdx.x; c < Ck; c += blockDim.x) {
-    const double sc = score[c];
-    int rank = 0;
-    for (int o = 0; o < Ck; ++o) {
-      const double so = score[o];
-      rank += (so > sc) || (so == sc && o < c);
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < (P >> 1); t += blockDim.x) {
+        const int lo = 2 * stride * (t / stride) + (t % stride), hi = lo + stride;
+        const double sa = score[lo], sb = score[hi];
+        const int ia = ids[lo], ib = ids[hi];
+        const bool in_order = route_before(sa, ia, sb, ib);
+        if (((lo & size) == 0) != in_order) {
+          score[lo] = sb;
+          score[hi] = sa;
+          ids[lo] = ib;
+          ids[hi] = ia;
+        }
+      }
+      __syncthreads();
     }
-    kept[c] = rank < k ? 1 : 0;
   }
+  const int k = kh[h];
+  for (int c = threadIdx.x; c < Ck; c += blockDim.x) kept[c] = 0;
+  __syncthreads();
+  for (int r = threadIdx.x; r < k; r += blockDim.x) kept[ids[r]] = 1;
   __syncthreads();
   // ascending compaction of the kept ids (block-wide exclusive scan)
   int32_t* out = csr + (static_cast<size_t>(h) * Cq + g) * kmax;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int base = 0; base < Ck; base += blockDim.x) {
     const int c = base + threadIdx.x;
     const int f = (c < Ck) ? kept[c] : 0;
@@ -86,6 +109,150 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const double* __re
     __syncthreads();
   }
   for (int i = k + threadIdx.x; i < kmax; i += blockDim.x) out[i] = -1;
+}
+
+// ---------------------------------------------------------------------------
+// Routing in two kernels for the workspace path: the block-score matrix
+// S_h = scale * C_Q C_K^T of a group of heads as one fp64 GEMM (64 x 64 tiles,
+// 4 x 4 outputs per thread, dot products summed in ascending column order),
+// then one warp per query group selects the top-k key groups by a radix
+// select on the scores' order-preserving bit patterns (greater score first,
+// lower id on ties) and writes their ids in ascending order.
+// ---------------------------------------------------------------------------
+constexpr int kSgT = 64, kSgK = 16;
+
+__global__ void __launch_bounds__(256) score_gemm_kernel(const double* __restrict__ A,
+                                                         const double* __restrict__ B, int M,
+                                                         int Nn, int d, double scale,
+                                                         double* __restrict__ S) {
+  __shared__ double As[kSgK][kSgT + 1], Bs[kSgK][kSgT + 1];
+  const int h = blockIdx.z, i0 = blockIdx.y * kSgT, j0 = blockIdx.x * kSgT;
+  const double* Ah = A + static_cast<size_t>(h) * M * d;
+  const double* Bh = B + static_cast<size_t>(h) * Nn * d;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+  for (int k0 = 0; k0 < d; k0 += kSgK) {
+    for (int t = threadIdx.x; t < kSgT * kSgK; t += blockDim.x) {
+      const int row = t / kSgK, kk = t % kSgK;
+      const int k = k0 + kk;
+      As[kk][row] = (i0 + row < M && k < d) ? Ah[static_cast<size_t>(i0 + row) * d + k] : 0.0;
+      Bs[kk][row] = (j0 + row < Nn && k < d) ? Bh[static_cast<size_t>(j0 + row) * d + k] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kSgK; ++kk) {
+      double a[4], b[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) a[r] = As[kk][ty * 4 + r];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) b[c] = Bs[kk][tx * 4 + c];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fma(a[r], b[c], acc[r][c]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + ty * 4 + r;
+    if (i >= M) continue;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + tx * 4 + c;
+      if (j < Nn) S[(static_cast<size_t>(h) * M + i) * Nn + j] = scale * acc[r][c];
+    }
+  }
+}
+
+// order-preserving bit pattern of a finite double (-0 taken as +0)
+__device__ __forceinline__ uint64_t score_key(double x) {
+  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x + 0.0));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+constexpr int kTopkWarps = 8;
+
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_route_kernel(
+    const double* __restrict__ S, int H, int Cq, int Ck, const int32_t* __restrict__ kh, int h0,
+    int kmax, int32_t* __restrict__ csr) {
+  __shared__ int hist[kTopkWarps][256];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gi = blockIdx.x * kTopkWarps + w;  // (head within the chunk, query group)
+  if (gi >= H * Cq) return;
+  const int hl = gi / Cq, g = gi % Cq;
+  const double* row = S + static_cast<size_t>(gi) * Ck;
+  const int k = kh[h0 + hl];
+  int* hs = hist[w];
+  // radix select of the k-th largest key, eight bits at a time
+  uint64_t prefix = 0;
+  int want = k;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hs[b] = 0;
+    __syncwarp();
+    for (int c = lane; c < Ck; c += 32) {
+      const uint64_t u = score_key(row[c]);
+      const bool match = (shift == 56) || ((u >> (shift + 8)) == (prefix >> (shift + 8)));
+      if (match) atomicAdd(&hs[(u >> shift) & 255], 1);
+    }
+    __syncwarp();
+    // lane l owns bins 255 - 8l - 7 .. 255 - 8l (from the top); suffix counts
+    int cnt[8], tot = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      cnt[q] = hs[255 - 8 * lane - q];
+      tot += cnt[q];
+    }
+    int incl = tot;  // inclusive prefix over lanes = count of bins above this lane's last bin
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int before = incl - tot;  // keys in higher bins than this lane's
+    // the lane whose range holds the want-th key finds the bin
+    int bin = -1, above = 0;
+    if (before < want && want <= incl) {
+      int run = before;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (bin < 0 && run + cnt[q] >= want) {
+          bin = 255 - 8 * lane - q;
+          above = run;
+        }
+        run += cnt[q];
+      }
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, bin >= 0);
+    const int src = __ffs(who) - 1;
+    bin = __shfl_sync(0xffffffffu, bin, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    want -= above;
+    prefix |= static_cast<uint64_t>(bin) << shift;
+    __syncwarp();
+  }
+  // prefix = key of the k-th largest score; take every larger key and the
+  // `want` lowest ids among the equal ones, in ascending id order
+  int32_t* out = csr + static_cast<size_t>(gi) * kmax;
+  int n_out = 0, n_eq = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < Ck; c0 += 32) {
+    const int c = c0 + lane;
+    uint64_t u = 0;
+    if (c < Ck) u = score_key(row[c]);
+    const bool gt = c < Ck && u > prefix, eq = c < Ck && u == prefix;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && n_eq + __popc(beq & lt) < want);
+    const unsigned bk = __ballot_sync(0xffffffffu, take);
+    if (take) out[n_out + __popc(bk & lt)] = c;
+    n_out += __popc(bk);
+    n_eq += __popc(beq);
+  }
+  for (int i = k + lane; i < kmax; i += 32) out[i] = -1;
 }
 
 struct KhParam {
@@ -111,12 +278,42 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, 
 cudaError_t launch_route(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
                          double scale, const int32_t* kh, int kmax, int32_t* csr,
                          cudaStream_t st) {
-  const size_t shb = static_cast<size_t>(Ck) * 8 + static_cast<size_t>(d) * 8 +
-                     static_cast<size_t>(Ck) * 4;
+  int P = 2;
+  while (P < Ck) P <<= 1;
+  const size_t shb = static_cast<size_t>(P) * 8 + static_cast<size_t>(d) * 8 +
+                     static_cast<size_t>(P) * 4 + static_cast<size_t>(Ck) * 4;
   cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(shb));
   if (e != cudaSuccess) return e;
-  route_kernel<<<dim3(Cq, H), kRouteThreads, shb, st>>>(cq, ckr, Cq, Ck, d, scale, kh, kmax, csr);
+  route_kernel<<<dim3(Cq, H), kRouteThreads, shb, st>>>(cq, ckr, Cq, Ck, d, scale, kh, kmax, P,
+                                                        csr);
+  return cudaGetLastError();
+}
+
+size_t route_scores_bytes(int H, int Cq, int Ck) {
+  const size_t per_head = static_cast<size_t>(Cq) * Ck * 8;
+  size_t heads = (static_cast<size_t>(64) << 20) / per_head;
+  if (heads < 1) heads = 1;
+  if (heads > static_cast<size_t>(H)) heads = H;
+  return heads * per_head;
+}
+
+cudaError_t launch_route_gemm(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
+                              double scale, const int32_t* kh, int kmax, double* scores,
+                              size_t scores_bytes, int32_t* csr, cudaStream_t st) {
+  const size_t per_head = static_cast<size_t>(Cq) * Ck * 8;
+  const int hc = static_cast<int>(scores_bytes / per_head);
+  if (hc < 1) return cudaErrorInvalidValue;
+  for (int h0 = 0; h0 < H; h0 += hc) {
+    const int nh = min(hc, H - h0);
+    dim3 g1((Ck + kSgT - 1) / kSgT, (Cq + kSgT - 1) / kSgT, nh);
+    score_gemm_kernel<<<g1, 256, 0, st>>>(cq + static_cast<size_t>(h0) * Cq * d,
+                                          ckr + static_cast<size_t>(h0) * Ck * d, Cq, Ck, d, scale,
+                                          scores);
+    const int rows = nh * Cq;
+    topk_route_kernel<<<(rows + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(
+        scores, nh, Cq, Ck, kh, h0, kmax, csr + static_cast<size_t>(h0) * Cq * kmax);
+  }
   return cudaGetLastError();
 }
 

@@ -36,8 +36,9 @@ __global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int n, int 
   for (int c = threadIdx.x; c < C; c += blockDim.x) out[c] = sh[c];
 }
 
-// One CTA per head. hist[h][chunk][c] becomes the first output position of
-// chunk's elements of group c; off[h][c] the first position of group c.
+// One CTA per head. hist[h][chunk][c] becomes the position of chunk's first
+// element of group c relative to the start of group c; off[h][c] the first
+// position of group c.
 __global__ void sort_scan_kernel(int n, int C, int nchunk, int32_t* __restrict__ hist,
                                  int32_t* __restrict__ off, const int32_t* skip,
                                  int skip_stride) {
@@ -50,8 +51,19 @@ __global__ void sort_scan_kernel(int n, int C, int nchunk, int32_t* __restrict__
   // per-group totals, turning each column into its exclusive running prefix
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     int32_t run = 0;
-    for (int k = 0; k < nchunk; ++k) {
-      int32_t v = hh[static_cast<size_t>(k) * C + c];
+    int k = 0;
+    for (; k + 8 <= nchunk; k += 8) {  // eight independent loads in flight
+      int32_t v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = hh[static_cast<size_t>(k + q) * C + c];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        hh[static_cast<size_t>(k + q) * C + c] = run;
+        run += v[q];
+      }
+    }
+    for (; k < nchunk; ++k) {
+      const int32_t v = hh[static_cast<size_t>(k) * C + c];
       hh[static_cast<size_t>(k) * C + c] = run;
       run += v;
     }
@@ -90,21 +102,18 @@ __global__ void sort_scan_kernel(int n, int C, int nchunk, int32_t* __restrict__
     __syncthreads();
   }
   if (threadIdx.x == 0) oo[C] = n;
-  __syncthreads();
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    const int32_t b = oo[c];
-    for (int k = 0; k < nchunk; ++k) hh[static_cast<size_t>(k) * C + c] += b;
-  }
 }
 
 __global__ void sort_scatter_kernel(const int32_t* __restrict__ labels, int n, int C, int nchunk,
-                                    const int32_t* __restrict__ hist, int32_t* __restrict__ perm,
+                                    const int32_t* __restrict__ hist,
+                                    const int32_t* __restrict__ off, int32_t* __restrict__ perm,
                                     const int32_t* skip, int skip_stride) {
   extern __shared__ int32_t cnt[];
   const int h = blockIdx.y, chunk = blockIdx.x;
   if (skip && skip[h * skip_stride]) return;
   const int32_t* start = hist + (static_cast<size_t>(h) * nchunk + chunk) * C;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = start[c];
+  const int32_t* oo = off + static_cast<size_t>(h) * (C + 1);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = oo[c] + start[c];
   __syncthreads();
   const int32_t* lab = labels + static_cast<size_t>(h) * n;
   int32_t* pp = perm + static_cast<size_t>(h) * n;
@@ -141,7 +150,7 @@ cudaError_t launch_counting_sort(const int32_t* labels, int H, int n, int C, int
   sort_hist_kernel<<<g2, kSortThreads, shb, st>>>(labels, n, C, nchunk, hist, skip, skip_stride,
                                                   stats);
   sort_scan_kernel<<<H, 1024, 0, st>>>(n, C, nchunk, hist, off, skip, skip_stride);
-  sort_scatter_kernel<<<g2, kSortThreads, shb, st>>>(labels, n, C, nchunk, hist, perm, skip,
+  sort_scatter_kernel<<<g2, kSortThreads, shb, st>>>(labels, n, C, nchunk, hist, off, perm, skip,
                                                        skip_stride);
   return cudaGetLastError();
 }

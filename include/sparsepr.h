@@ -21,7 +21,9 @@
  *   - Tensors are row-major [H, N, d] with d contiguous (Q, K, V and the
  *     outputs) or [H, n] (integer arrays). All tensor pointers are DEVICE
  *     pointers owned by the caller; the library never allocates, frees or
- *     synchronises on them.
+ *     synchronises on them. Q/K/V-shaped tensors (inputs, permuted copies,
+ *     outputs) must be 16-byte aligned; a misaligned pointer is rejected
+ *     with SPARSEPR_ERR_INVALID_ARG.
  *   - `ws` is a caller-owned device workspace of at least
  *     sparsepr_workspace_bytes(p) bytes, 256-byte aligned. The same `ws` is
  *     passed to every call of one attention call; its first bytes hold the
