@@ -499,12 +499,29 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     a.runs = reinterpret_cast<int2*>(meta + 8 * H);
     a.pairs = nullptr;
     a.stats = c.stats;
+    // few units (H * ceil(M / 256)) over all N keys: split the key tiles so
+    // that about one CTA per SM runs
+    {
+      const int units = H * ((M + 255) / 256);
+      const int ktiles = (N + kTileN - 1) / kTileN;
+      int sp = sm_count() / (units > 0 ? units : 1);
+      if (sp > kMaxSplits) sp = kMaxSplits;
+      if (sp > ktiles) sp = ktiles;
+      if (sp < 1) sp = 1;
+      a.splits = sp;
+      a.units = L.punits;
+      a.opart = at<float>(ws, L.opart);
+      a.lpart = at<float>(ws, L.lpart);
+    }
     SPR_TRY(launch_block_sparse_attn(a, st));
     double* xr = at<double>(ws, L.xr);
     double* means = at<double>(ws, L.means);
     double* gram = at<double>(ws, L.gram);
     const long long hs = 2LL * M * d;
-    SPR_TRY(launch_probe_residuals(o_sparse, od, probes, H, N, M, d, xr, means, st));
+    // the block sums of the residual pass live in the Gram region until the
+    // Grams are formed
+    SPR_TRY(launch_probe_residuals(o_sparse, od, probes, H, N, M, d, xr, means, gram,
+                                   static_cast<size_t>(H) * 2 * d * d, st));
     SPR_TRY(launch_gram_f64(xr, xr, means, means, hs, hs, d, M, H, d, 1.0, c.p.lambda, gram,
                             2LL * d * d, 2LL * d, st));
     SPR_TRY(launch_gram_f64(xr, xr + static_cast<size_t>(M) * d, means, means + d, hs, hs, d, M, H,

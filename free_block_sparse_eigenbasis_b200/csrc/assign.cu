@@ -373,12 +373,14 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// fp64 decision of the flagged rows: a block takes eight flagged rows (one
-// per warp) and streams the centroids through shared memory 32 at a time;
-// lane l scores centroid j0 + l against its warp's row, then a warp argmin.
+// fp64 decision of the flagged rows: one block per flagged row (grid-stride).
+// Short rows (D <= 32): thread j scores centroids j, j + 256, ... reading
+// each centroid row contiguously; long rows: warp w scores centroids w,
+// w + 8, ... with its lanes over the columns (butterfly sum, identical in
+// every lane). Then a block argmin, lowest index on ties.
 // direct = 1: d = sum_t (x_t - y_jt)^2; else d = c_j - 2 x . y_j.
 // ---------------------------------------------------------------------------
-constexpr int kRcWarps = 8, kRcMaxD = 128, kRcChunk = 32;
+constexpr int kRcThreads = 256, kRcMaxD = 128;
 
 __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   if (kind == kXf64) return static_cast<const double*>(X)[i];
@@ -386,14 +388,21 @@ __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   return static_cast<double>(static_cast<const float*>(X)[i]);
 }
 
-__global__ void __launch_bounds__(kRcWarps * 32)
+__device__ __forceinline__ void argmin_merge(double& best, int& bi, double ob, int oi) {
+  if (ob < best || (ob == best && oi < bi)) {
+    best = ob;
+    bi = oi;
+  }
+}
+
+__global__ void __launch_bounds__(kRcThreads)
     recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
                    const double* Y, const double* c, int m, int direct, int32_t* labels,
                    int32_t* flags, int flag_base, const int32_t* recheck,
                    const int32_t* nrecheck) {
-  __shared__ double xs[kRcWarps][kRcMaxD];
-  __shared__ double ys[kRcChunk][kRcMaxD + 1];
-  __shared__ double cc[kRcChunk];
+  __shared__ double xs[kRcMaxD];
+  __shared__ double wbest[kRcThreads / 32];
+  __shared__ int wbi[kRcThreads / 32];
   const int h = blockIdx.y;
   int32_t* fl = flags + h * 4;
   if (fl[flag_base + 1]) return;
@@ -401,53 +410,66 @@ __global__ void __launch_bounds__(kRcWarps * 32)
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const double* Yh = Y + static_cast<size_t>(h) * m * D;
   const double* ch = c + static_cast<size_t>(h) * m;
-  for (int base = blockIdx.x * kRcWarps; base < cnt; base += gridDim.x * kRcWarps) {
-    const int k = base + w;
-    const bool has = k < cnt;
-    const int row = has ? recheck[static_cast<size_t>(h) * n + k] : 0;
-    if (has)
-      for (int t = lane; t < D; t += 32) xs[w][t] = ldx(X, kind, h * hsx + static_cast<size_t>(row) * ldx_ + t);
+  for (int k = blockIdx.x; k < cnt; k += gridDim.x) {
+    const int row = recheck[static_cast<size_t>(h) * n + k];
+    __syncthreads();  // xs and the warp results of the previous row are consumed
+    for (int t = threadIdx.x; t < D; t += blockDim.x)
+      xs[t] = ldx(X, kind, h * hsx + static_cast<size_t>(row) * ldx_ + t);
+    __syncthreads();
     double best = INFINITY;
     int bi = 0x7fffffff;
-    for (int j0 = 0; j0 < m; j0 += kRcChunk) {
-      __syncthreads();  // the previous chunk is consumed (first time: xs written)
-      for (int t = threadIdx.x; t < kRcChunk * D; t += blockDim.x) {
-        const int jj = t / D, a = t % D;
-        ys[jj][a] = (j0 + jj < m) ? Yh[static_cast<size_t>(j0 + jj) * D + a] : 0.0;
-      }
-      if (!direct && threadIdx.x < kRcChunk)
-        cc[threadIdx.x] = (j0 + static_cast<int>(threadIdx.x) < m) ? ch[j0 + threadIdx.x] : 0.0;
-      __syncthreads();
-      const int j = j0 + lane;  // ascending within the lane
-      if (has && j < m) {
+    if (D <= 32) {
+      for (int j = threadIdx.x; j < m; j += blockDim.x) {  // ascending within the thread
+        const double* y = Yh + static_cast<size_t>(j) * D;
         double dd;
         if (direct) {
           dd = 0.0;
           for (int t = 0; t < D; ++t) {
-            const double diff = xs[w][t] - ys[lane][t];
+            const double diff = xs[t] - y[t];
             dd = fma(diff, diff, dd);
           }
         } else {
           double sm = 0.0;
-          for (int t = 0; t < D; ++t) sm = fma(xs[w][t], ys[lane][t], sm);
-          dd = cc[lane] - 2.0 * sm;
+          for (int t = 0; t < D; ++t) sm = fma(xs[t], y[t], sm);
+          dd = ch[j] - 2.0 * sm;
         }
         if (dd < best) {
           best = dd;
           bi = j;
         }
       }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {  // lowest index on ties
-      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ob < best || (ob == best && oi < bi)) {
-        best = ob;
-        bi = oi;
+      for (int o = 16; o > 0; o >>= 1)
+        argmin_merge(best, bi, __shfl_xor_sync(0xffffffffu, best, o),
+                     __shfl_xor_sync(0xffffffffu, bi, o));
+    } else {
+      for (int j = w; j < m; j += kRcThreads / 32) {  // ascending within the warp
+        const double* y = Yh + static_cast<size_t>(j) * D;
+        double part = 0.0;
+        for (int t = lane; t < D; t += 32) {
+          if (direct) {
+            const double diff = xs[t] - y[t];
+            part = fma(diff, diff, part);
+          } else {
+            part = fma(xs[t], y[t], part);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        const double dd = direct ? part : ch[j] - 2.0 * part;
+        if (dd < best) {
+          best = dd;
+          bi = j;
+        }
       }
     }
-    if (has && lane == 0) {
+    if (lane == 0) {
+      wbest[w] = best;
+      wbi[w] = bi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int q = 1; q < kRcThreads / 32; ++q) argmin_merge(best, bi, wbest[q], wbi[q]);
       const size_t li = static_cast<size_t>(h) * n + row;
       if (labels[li] != bi) atomicAdd(&fl[flag_base], 1);
       labels[li] = bi;
@@ -641,7 +663,7 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   argmin_tc_kernel<<<ctas, kAsThreads, shb, st>>>(maps, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  recheck_kernel<<<dim3(16, a.H), kRcWarps * 32, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
+  recheck_kernel<<<dim3(64, a.H), kRcThreads, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
                                                 a.y_exact, a.c_exact, a.m, a.direct, a.labels,
                                                 a.flags, a.flag_base, a.recheck, a.nrecheck);
   return cudaGetLastError();

@@ -95,6 +95,9 @@ struct AttnParams {
   float sc;        // scale * log2(e)
   float* out;
   DeviceStats* stats;
+  int splits, units;  // split-KV (splits > 1): partial outputs per (unit, split)
+  float* opart;
+  float* lpart;
 };
 
 // Key-column validity of the key tiles of one query group, walked in
@@ -109,6 +112,13 @@ struct MaskWalk {
     ns = nslots;
     ri = 0;
     rend = (n > 0) ? (r[0].y + kSlotRows - 1) / kSlotRows : 0;
+  }
+  // consume the runs that end before tile j (start of a key-tile range)
+  __device__ void advance_to(int j) {
+    while (ri < nr && rend <= j * kSlotsPerTile) {
+      ++ri;
+      if (ri < nr) rend += (runs[ri].y + kSlotRows - 1) / kSlotRows;
+    }
   }
   // bit c of m[c / 32] = key column c of tile j is a real key
   __device__ void tile(int j, uint32_t (&m)[4]) {
@@ -128,20 +138,19 @@ struct MaskWalk {
   }
 };
 
-// 2^x on the FMA pipe, used for a quarter of the columns so that the
-// special-function unit (ex2.approx) is not the bottleneck of the softmax:
-// x = n + f with n = round(x) (added into the exponent field) and f in
-// [-1/2, 1/2], 2^f by a cubic whose coefficients minimise the relative
-// error on that interval (Lawson-weighted least squares on Chebyshev nodes;
-// maximum relative error 7.5e-5, below the 2^-9 rounding of the bf16 P it
-// feeds). x is clamped at -126, so a masked logit gives 2^-126 instead of 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
-  const float f = x - (t - 12582912.f);
-  const float q = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f,
-                       0.9999280572f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+// Packed fp32x2 fma (one instruction for two columns) and the three-input
+// maximum of sm_100, used by the softmax.
+__device__ __forceinline__ void fma2(float& x0, float& x1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(x0), "=f"(x1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 template <int HD>
@@ -150,8 +159,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using L = Smem<HD>;
   constexpr int kAtoms = HD / 64;
   const int h = blockIdx.y;
-  if (static_cast<int>(blockIdx.x) >= p.nwork[h]) return;
-  const int wcode = p.work[static_cast<size_t>(h) * p.tiles_per_head + blockIdx.x];
+  const int wi = static_cast<int>(blockIdx.x) / p.splits, split = static_cast<int>(blockIdx.x) % p.splits;
+  if (wi >= p.nwork[h]) return;
+  const int wcode = p.work[static_cast<size_t>(h) * p.tiles_per_head + wi];
   const int g = wcode >> 16, tu = wcode & 0xFFFF;
   const int32_t* offq = p.off_q + static_cast<size_t>(h) * (p.Cq + 1);
   const int row0 = offq[g] + tu * kUnitRows;
@@ -159,15 +169,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nq = rows_unit > kTileM ? 2 : 1;  // query tiles in this unit
   const size_t gi = static_cast<size_t>(h) * p.Cq + g;
   const int ns = p.nslots[gi];
-  const int T = (ns + kSlotsPerTile - 1) / kSlotsPerTile;
+  const int T_all = (ns + kSlotsPerTile - 1) / kSlotsPerTile;
+  // this CTA's key tiles [j0, j0 + T)
+  const int j0 = static_cast<int>(static_cast<long long>(T_all) * split / p.splits);
+  const int T = static_cast<int>(static_cast<long long>(T_all) * (split + 1) / p.splits) - j0;
   const int nr = p.nruns[gi];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool partial = p.splits > 1;
+  const size_t pbase = ((static_cast<size_t>(h) * p.units + wi) * p.splits + split) * kUnitRows;
 
   if (T == 0) {
-    // empty kept set (reported by the slot-count kernel): rows are zero
+    // empty kept set (reported by the slot-count kernel) or an empty split:
+    // rows are zero (partials: zero with log-sum -inf)
     if (static_cast<int>(threadIdx.x) < rows_unit) {
-      float* o = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x) * HD;
+      float* o = partial ? p.opart + (pbase + threadIdx.x) * HD
+                         : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x) * HD;
       for (int c = 0; c < HD; c += 4) *reinterpret_cast<float4*>(o + c) = make_float4(0, 0, 0, 0);
+      if (partial) p.lpart[pbase + threadIdx.x] = -INFINITY;
     }
     return;
   }
@@ -230,6 +248,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tma_load_2d(Qs + qt * L::kQBytes + a * L::kSlab, &maps.q, &bars->q_full, a * 64,
                       h * p.q_rows + row0 + qt * kTileM);
       int ri = -1, pos = 0, rend = 0;  // current run and its row range [pos, rend)
+      for (int skip = j0 * kSlotsPerTile; skip > 0 && ri + 1 < nr;) {
+        ++ri;
+        pos = runs[ri].x;
+        rend = pos + runs[ri].y;
+        const int rs = (runs[ri].y + kSlotRows - 1) / kSlotRows;
+        const int take = min(skip, rs);
+        pos += take * kSlotRows;
+        skip -= take;
+      }
       int k_issued = -1, v_issued = -1;
       for (int j = 0; j < T; ++j) {
         // box plan of key tile j: (slot, first row, log2 size) per box
@@ -363,18 +390,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_ref = -INFINITY, l_sum = 0.f;
     MaskWalk mw;
     mw.init(runs, nr, ns);
+    mw.advance_to(j0);
     bool ok = true;
     for (int t = 0; t < ntask[i]; ++t) {
-      const int kv = two ? t : 2 * t + i;
+      const int kv = two ? t : 2 * t + i;  // local key tile; global tile j0 + kv
       uint32_t vm[4];
       if (!two && i == 1) {
         uint32_t skip[4];
-        mw.tile(kv - 1, skip);  // advance past the other warpgroup's tile
+        mw.tile(j0 + kv - 1, skip);  // advance past the other warpgroup's tile
       }
-      mw.tile(kv, vm);
+      mw.tile(j0 + kv, vm);
       if (!two && i == 0 && kv + 1 < T) {
         uint32_t skip[4];
-        mw.tile(kv + 1, skip);
+        mw.tile(j0 + kv + 1, skip);
       }
       // tcgen05.ld / st below are warp-collective: the warp proceeds or stops as one
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], t & 1, abort))) { ok = false; break; }
@@ -396,14 +424,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
-      // row maximum: eight independent chains, then a tree
+      // row maximum: eight independent chains of three-input maxima, then a tree
       float m8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(r[k]);
 #pragma unroll
-      for (int c = 8; c < kTileN; ++c) m8[c & 7] = fmaxf(m8[c & 7], __uint_as_float(r[c]));
-      const float mx = sc * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                  fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      for (int c = 8; c < kTileN; c += 2)
+        m8[(c >> 1) & 7] = max3f(m8[(c >> 1) & 7], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+      const float mx = sc * fmaxf(max3f(m8[0], m8[1], m8[2]),
+                                  fmaxf(max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       // reference maximum (moves only when it grows by more than 2^8)
       float alpha = 1.f;
       bool need = false;
@@ -415,8 +444,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         m_ref = mx;
       }
       // P = 2^(s sc - m_ref) as bf16 pairs over the first 64 columns of S_i;
-      // row sum in fp32. S_i(t) was produced after P_i(t-1) V completed, so
-      // these columns are free.
+      // row sum in fp32 (eight chains). S_i(t) was produced
+      // after P_i(t-1) V completed, so these columns are free.
       float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       const float nm = -m_ref;
 #pragma unroll
@@ -424,11 +453,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const float xa = fmaf(__uint_as_float(r[hf * 64 + c]), sc, nm);
-          const float xb = fmaf(__uint_as_float(r[hf * 64 + c + 1]), sc, nm);
-          const bool poly = ((c >> 1) & 3) == 3;  // one pair in four
-          const float a = poly ? exp2_poly(xa) : ex2_approx(xa);
-          const float b = poly ? exp2_poly(xb) : ex2_approx(xb);
+          float xa, xb;
+          fma2(xa, xb, __uint_as_float(r[hf * 64 + c]), __uint_as_float(r[hf * 64 + c + 1]), sc, nm);
+          const float a = ex2_approx(xa), b = ex2_approx(xb);
           r8[(c >> 1) & 7] += a + b;
           pk[c >> 1] = pack_bf16x2(a, b);
         }
@@ -461,7 +488,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float inv = 1.f / l_sum;
         const uint32_t o_tmem = o_base + static_cast<uint32_t>(i * HD);
         const bool valid = i * kTileM + row < rows_unit;
-        float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row) * HD;
+        float* orow = partial ? p.opart + (pbase + i * kTileM + row) * HD
+                              : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row) * HD;
+        if (partial && valid) p.lpart[pbase + i * kTileM + row] = m_ref + __log2f(l_sum);
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
@@ -494,7 +523,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const bool valid = row < rows_unit;
-        float* orow = p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD;
+        float* orow = partial ? p.opart + (pbase + row) * HD
+                              : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD;
+        if (partial && valid && i == 0) p.lpart[pbase + row] = mm + __log2f(l0 * a0 + l1 * a1);
 #pragma unroll
         for (int c = 0; c < HD / 64; ++c) {
           const int col = i * (HD / 2) + c * 32;
@@ -605,6 +636,39 @@ __global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, c
   if (nq > 0 && keys == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
 }
 
+// Split-KV combine: out = sum_s 2^(l_s - L) O_s / sum_s 2^(l_s - L),
+// L = max_s l_s, over the splits' normalised partial outputs O_s and
+// log2-sum-exps l_s. One block per (unit, head), thread = column, rows in
+// turn (fixed order over the splits).
+__global__ void split_combine_kernel(const float* opart, const float* lpart, const int32_t* off_q,
+                                     const int32_t* work, const int32_t* nwork, int Cq,
+                                     int tiles_per_head, int units, int splits, int q_rows, int d,
+                                     float* out) {
+  const int h = blockIdx.y, wi = blockIdx.x;
+  if (wi >= nwork[h]) return;
+  const int wcode = work[static_cast<size_t>(h) * tiles_per_head + wi];
+  const int g = wcode >> 16, tu = wcode & 0xFFFF;
+  const int32_t* offq = off_q + static_cast<size_t>(h) * (Cq + 1);
+  const int row0 = offq[g] + tu * kUnitRows;
+  const int rows = min(kUnitRows, offq[g + 1] - row0);
+  const size_t ub = (static_cast<size_t>(h) * units + wi) * splits;
+  for (int r = 0; r < rows; ++r) {
+    float L = -INFINITY;
+    for (int s = 0; s < splits; ++s) L = fmaxf(L, lpart[(ub + s) * kUnitRows + r]);
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+      float num = 0.f, den = 0.f;
+      for (int s = 0; s < splits; ++s) {
+        const float ls = lpart[(ub + s) * kUnitRows + r];
+        if (ls == -INFINITY) continue;
+        const float wgt = exp2f(ls - L);
+        num = fmaf(wgt, opart[((ub + s) * kUnitRows + r) * d + c], num);
+        den += wgt;
+      }
+      out[(static_cast<size_t>(h) * q_rows + row0 + r) * d + c] = den > 0.f ? num / den : 0.f;
+    }
+  }
+}
+
 __global__ void zero_i64_kernel(int64_t* p, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) p[i] = 0;
@@ -666,8 +730,12 @@ cudaError_t launch_attn_hd(const AttnArgs& a, AttnParams prm, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<HD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.tiles_per_head, a.H);
+  dim3 grid(a.tiles_per_head * prm.splits, a.H);
   sparse_attn_kernel<HD><<<grid, kAttnThreads, shb, st>>>(maps, prm);
+  if (prm.splits > 1)
+    split_combine_kernel<<<dim3(a.units, a.H), 128, 0, st>>>(
+        a.opart, a.lpart, a.off_q, a.work, a.nwork, a.Cq, a.tiles_per_head, a.units, prm.splits,
+        a.q_rows, HD, a.out);
   return cudaGetLastError();
 }
 
@@ -698,6 +766,11 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   prm.sc = a.scale * kLog2e;
   prm.out = a.out;
   prm.stats = a.stats;
+  prm.splits = a.splits > 1 ? a.splits : 1;
+  prm.units = a.units;
+  prm.opart = a.opart;
+  prm.lpart = a.lpart;
+  if (prm.splits > 1 && (!a.opart || !a.lpart || a.units < 1)) return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.d == 128) return launch_attn_hd<128>(a, prm, st);

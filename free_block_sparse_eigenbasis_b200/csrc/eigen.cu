@@ -105,10 +105,11 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
     const double kk = -0.5 * tk * pv;
     for (int i = tid; i < n1; i += blockDim.x) w[i] += kk * v[i];
     __syncthreads();
-    // A22 -= v w^T + w v^T
-    for (int t = tid; t < n1 * n1; t += blockDim.x) {
-      const int r = t / n1, c = t % n1;
-      A[(k + 1 + r) * D + (k + 1 + c)] -= v[r] * w[c] + w[r] * v[c];
+    // A22 -= v w^T + w v^T (warp = row stripe, lane = column stripe)
+    for (int r = wid; r < n1; r += kTriThreads / 32) {
+      const double vr = v[r], wr = w[r];
+      double* Ar = A + (k + 1 + r) * D + (k + 1);
+      for (int c = lane; c < n1; c += 32) Ar[c] -= vr * w[c] + wr * v[c];
     }
     __syncthreads();
   }
@@ -130,7 +131,7 @@ __device__ int sturm_count(const double* dg, const double* e2, double x, double 
   cnt += (q < 0.0);
 #pragma unroll 1
   for (int i = 1; i < D; ++i) {
-    q = dg[i] - x - e2[i - 1] / q;
+    q = dg[i] - x - e2[i - 1] * __drcp_rn(q);
     if (fabs(q) < pivmin) q = -pivmin;
     cnt += (q < 0.0);
   }

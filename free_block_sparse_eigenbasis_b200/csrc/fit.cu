@@ -79,15 +79,20 @@ __global__ void gather_probe_rows_kernel(const void* qp, int bf16, const int32_t
 }
 
 // X = O_sparse[probes], R = O_dense - X (fp64), column means xbar, rbar.
+// X = O_sparse[probes], R = O_dense - X (fp64) for a block of probe rows
+// per CTA (thread = column), with the block's column sums of X and R in
+// part [H, nblk, 2, d]; probe_means_kernel adds the blocks in order.
 __global__ void probe_residuals_kernel(const float* o_sparse, const float* od,
-                                       const int32_t* probes, int N, int M, int d, double* xr,
-                                       double* means) {
-  const int h = blockIdx.x, a = threadIdx.x;
+                                       const int32_t* probes, int N, int M, int d, int rows_blk,
+                                       double* xr, double* part) {
+  const int h = blockIdx.y, blk = blockIdx.x, a = threadIdx.x;
   if (a >= d) return;
   double* X = xr + static_cast<size_t>(h) * 2 * M * d;
   double* R = X + static_cast<size_t>(M) * d;
   double sx = 0.0, sr = 0.0;
-  for (int t = 0; t < M; ++t) {
+  const int t0 = blk * rows_blk, t1 = min(M, t0 + rows_blk);
+#pragma unroll 4
+  for (int t = t0; t < t1; ++t) {
     const size_t row = static_cast<size_t>(h) * N + probes[static_cast<size_t>(h) * M + t];
     const double x = o_sparse[row * d + a];
     const double r = static_cast<double>(od[(static_cast<size_t>(h) * M + t) * d + a]) - x;
@@ -96,80 +101,105 @@ __global__ void probe_residuals_kernel(const float* o_sparse, const float* od,
     sx += x;
     sr += r;
   }
+  double* pp = part + ((static_cast<size_t>(h) * gridDim.x + blk) * 2) * d;
+  pp[a] = sx;
+  pp[d + a] = sr;
+}
+
+__global__ void probe_means_kernel(const double* part, int nblk, int M, int d, double* means) {
+  const int h = blockIdx.x, a = threadIdx.x;
+  if (a >= d) return;
+  double sx = 0.0, sr = 0.0;
+  for (int b = 0; b < nblk; ++b) {
+    const double* pp = part + ((static_cast<size_t>(h) * nblk + b) * 2) * d;
+    sx += pp[a];
+    sr += pp[d + a];
+  }
   means[(static_cast<size_t>(h) * 2 + 0) * d + a] = M > 0 ? sx / M : 0.0;
   means[(static_cast<size_t>(h) * 2 + 1) * d + a] = M > 0 ? sr / M : 0.0;
 }
 
-// Ridge solve per head: L L^T = A (Cholesky, packed lower L in shared
-// memory), B = A^{-1} C with one right-hand-side column per thread, then
-// b = rbar - xbar B.
-__global__ void ridge_solve_kernel(const double* gram, int d, double* bmat, double* bvec,
-                                   const double* means, DeviceStats* stats) {
+// Ridge solve per head: L L^T = A (right-looking Cholesky on the packed
+// lower triangle in shared memory), then L Y = C and L^T B = Y with all d
+// right-hand sides at once (row-by-row elimination, parallel over the rows
+// below and the columns), and b = rbar - xbar B.
+constexpr int kRidgeThreads = 512;
+
+__global__ void __launch_bounds__(kRidgeThreads)
+    ridge_solve_kernel(const double* gram, int d, double* bmat, double* bvec, const double* means,
+                       DeviceStats* stats) {
   extern __shared__ double rsm[];
   const int ntri = d * (d + 1) / 2;
   double* Lp = rsm;          // packed lower triangle, L[i][k] at i*(i+1)/2 + k
   double* Cm = rsm + ntri;   // [d][d] right-hand sides (row-major), solved in place
   __shared__ int bad;
-  const int h = blockIdx.x;
+  const int h = blockIdx.x, tid = threadIdx.x;
   const double* A = gram + static_cast<size_t>(h) * 2 * d * d;
   const double* C = A + static_cast<size_t>(d) * d;
-  for (int t = threadIdx.x; t < d * d; t += blockDim.x) {
+  for (int t = tid; t < d * d; t += blockDim.x) {
     const int i = t / d, k = t % d;
     if (k <= i) Lp[i * (i + 1) / 2 + k] = A[t];
     Cm[t] = C[t];
   }
-  if (threadIdx.x == 0) bad = 0;
+  if (tid == 0) bad = 0;
   __syncthreads();
+  auto L = [&](int i, int k) -> double& { return Lp[i * (i + 1) / 2 + k]; };
+  // Cholesky: column j, then the trailing triangle (4 threads per row)
   for (int j = 0; j < d; ++j) {
-    if (threadIdx.x == 0) {
-      double s = Lp[j * (j + 1) / 2 + j];
-      for (int k = 0; k < j; ++k) {
-        const double l = Lp[j * (j + 1) / 2 + k];
-        s -= l * l;
-      }
+    if (tid == 0) {
+      double s = L(j, j);
       if (!(s > 0.0)) {
         bad = 1;
         s = 1.0;
       }
-      Lp[j * (j + 1) / 2 + j] = sqrt(s);
+      L(j, j) = sqrt(s);
     }
     __syncthreads();
-    const double ljj = Lp[j * (j + 1) / 2 + j];
-    for (int i = j + 1 + threadIdx.x; i < d; i += blockDim.x) {
-      double s = Lp[i * (i + 1) / 2 + j];
-      for (int k = 0; k < j; ++k) s -= Lp[i * (i + 1) / 2 + k] * Lp[j * (j + 1) / 2 + k];
-      Lp[i * (i + 1) / 2 + j] = s / ljj;
+    const double ljj = L(j, j);
+    for (int i = j + 1 + tid; i < d; i += blockDim.x) L(i, j) /= ljj;
+    __syncthreads();
+    for (int q = tid; q < (d - j - 1) * 4; q += blockDim.x) {
+      const int i = j + 1 + (q >> 2);
+      const double lij = L(i, j);
+      for (int k = j + 1 + (q & 3); k <= i; k += 4) L(i, k) -= lij * L(k, j);
     }
     __syncthreads();
   }
-  const int col = threadIdx.x;
-  if (col < d) {
-    // forward: L Y = C
-    for (int i = 0; i < d; ++i) {
-      double s = Cm[i * d + col];
-      for (int k = 0; k < i; ++k) s -= Lp[i * (i + 1) / 2 + k] * Cm[k * d + col];
-      Cm[i * d + col] = s / Lp[i * (i + 1) / 2 + i];
+  // forward: L Y = C
+  for (int i = 0; i < d; ++i) {
+    const double lii = L(i, i);
+    for (int c = tid; c < d; c += blockDim.x) Cm[i * d + c] /= lii;
+    __syncthreads();
+    for (int t = tid; t < (d - i - 1) * d; t += blockDim.x) {
+      const int r = i + 1 + t / d, c = t % d;
+      Cm[r * d + c] -= L(r, i) * Cm[i * d + c];
     }
-    // backward: L^T B = Y
-    for (int i = d - 1; i >= 0; --i) {
-      double s = Cm[i * d + col];
-      for (int k = i + 1; k < d; ++k) s -= Lp[k * (k + 1) / 2 + i] * Cm[k * d + col];
-      Cm[i * d + col] = s / Lp[i * (i + 1) / 2 + i];
-    }
+    __syncthreads();
   }
-  __syncthreads();
+  // backward: L^T B = Y
+  for (int i = d - 1; i >= 0; --i) {
+    const double lii = L(i, i);
+    for (int c = tid; c < d; c += blockDim.x) Cm[i * d + c] /= lii;
+    __syncthreads();
+    for (int t = tid; t < i * d; t += blockDim.x) {
+      const int r = t / d, c = t % d;
+      Cm[r * d + c] -= L(i, r) * Cm[i * d + c];
+    }
+    __syncthreads();
+  }
   if (bad) {
-    for (int t = threadIdx.x; t < d * d; t += blockDim.x) Cm[t] = 0.0;
-    if (threadIdx.x == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
+    for (int t = tid; t < d * d; t += blockDim.x) Cm[t] = 0.0;
+    if (tid == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
     __syncthreads();
   }
   double* Bo = bmat + static_cast<size_t>(h) * d * d;
-  for (int t = threadIdx.x; t < d * d; t += blockDim.x) Bo[t] = Cm[t];
-  if (col < d) {
+  for (int t = tid; t < d * d; t += blockDim.x) Bo[t] = Cm[t];
+  if (tid < d) {
+    const int col = tid;
     const double* xbar = means + static_cast<size_t>(h) * 2 * d;
     const double* rbar = xbar + d;
     double s = rbar[col];
-    for (int a = 0; a < d; ++a) s -= xbar[a] * Cm[a * d + col];
+    for (int a2 = 0; a2 < d; ++a2) s -= xbar[a2] * Cm[a2 * d + col];
     bvec[static_cast<size_t>(h) * d + col] = bad ? 0.0 : s;
   }
 }
@@ -290,8 +320,18 @@ cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* p
 
 cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const int32_t* probes,
                                    int H, int N, int M, int d, double* xr, double* means,
-                                   cudaStream_t st) {
-  probe_residuals_kernel<<<H, 128, 0, st>>>(o_sparse, od, probes, N, M, d, xr, means);
+                                   double* part, size_t part_doubles, cudaStream_t st) {
+  // blocks of >= 16 rows, at most part_doubles / (2 d H) of them
+  int nblk = (M + 15) / 16;
+  const int cap = static_cast<int>(part_doubles / (2 * static_cast<size_t>(d) * H));
+  if (nblk > cap) nblk = cap;
+  if (nblk < 1) return cudaErrorInvalidValue;
+  const int rows_blk = (M + nblk - 1) / nblk;
+  nblk = (M + rows_blk - 1) / rows_blk;
+  if (nblk < 1) nblk = 1;
+  probe_residuals_kernel<<<dim3(nblk, H), d, 0, st>>>(o_sparse, od, probes, N, M, d, rows_blk, xr,
+                                                      part);
+  probe_means_kernel<<<H, d, 0, st>>>(part, nblk, M, d, means);
   return cudaGetLastError();
 }
 
@@ -302,7 +342,7 @@ cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double*
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(shb));
   if (e != cudaSuccess) return e;
-  ridge_solve_kernel<<<H, 128, shb, st>>>(gram, d, bmat, bvec, means, stats);
+  ridge_solve_kernel<<<H, kRidgeThreads, shb, st>>>(gram, d, bmat, bvec, means, stats);
   return cudaGetLastError();
 }
 

@@ -178,6 +178,15 @@ struct AttnArgs {
   int32_t* nruns;        // [H, Cq]
   int64_t* pairs;        // [H] (may be null)
   DeviceStats* stats;
+  // split of every unit's key tiles into `splits` contiguous ranges run by
+  // separate CTAs (1: off). With splits > 1 each CTA writes its normalised
+  // partial output and log2-sum-exp to opart [H, units, splits, 256, d] /
+  // lpart [H, units, splits, 256] (units = partial-buffer units per head),
+  // and a combine kernel writes `out`.
+  int splits = 1;
+  int units = 0;
+  float* opart = nullptr;
+  float* lpart = nullptr;
 };
 cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st);
@@ -187,9 +196,10 @@ cudaError_t launch_probe_select(const int32_t* off_q, int H, int Cq, int M, int3
                                 cudaStream_t st);
 cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* probes, int H,
                                      int N, int M, int d, __nv_bfloat16* dst, cudaStream_t st);
+// part: scratch of part_doubles fp64 for per-block column sums.
 cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const int32_t* probes,
                                    int H, int N, int M, int d, double* xr, double* means,
-                                   cudaStream_t st);
+                                   double* part, size_t part_doubles, cudaStream_t st);
 cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
                                const double* means, DeviceStats* stats, cudaStream_t st);
 // B' = (B V_r) V_r^T, b' = (b V_r) V_r^T with vr [H, d, r]; bp32 holds B'^T

@@ -17,6 +17,7 @@ constexpr int kTileN = 128;     // keys per attention KV tile
 constexpr int kSlotRows = 8;    // keys per TMA row-slot of a KV tile
 constexpr int kSortChunk = 1024;  // tokens per counting-sort chunk
 constexpr int kMaxGroups = 4096;
+constexpr int kMaxSplits = 8;   // split-KV ranges of the dense probe pass
 
 struct Layout {
   // statistics / status (always at offset 0)
@@ -80,11 +81,14 @@ struct Layout {
   size_t pnwork;   // [H] int32
   size_t pmeta;    // [H, 10] int32: dense-mode off_q(2), off_k(2), csr(1), k(1), nslots(1),
                    // nruns(1), runs(2)
+  size_t opart;    // [H, punits, kMaxSplits, 256, d] f32 split-KV partial outputs (probes)
+  size_t lpart;    // [H, punits, kMaxSplits, 256] f32 split-KV log2-sum-exps
   size_t total;
 
   int Nv, e, Cmax, nchunk, tiles_per_head, kmax;
   int Dpk, CpadK, CpadQ;
   size_t scores_bytes;
+  int punits;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -187,6 +191,9 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->pwork = take(H * (M / kTileM + 2) * 4);
   L->pnwork = take(H * 4);
   L->pmeta = take(H * 10 * 4);
+  L->punits = static_cast<int>(M / 256 + 1);
+  L->opart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * d * 4);
+  L->lpart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * 4);
   L->total = o;
 }
 
