@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -81,6 +83,48 @@ sparsepr_status cuda_status(cudaError_t e) {
 __global__ void set_i32_kernel(int32_t* p, int v) { *p = v; }
 
 constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
+
+// A second stream per device for small independent kernels that occupy few
+// SMs (the Fisher-Yates init beside the M_K eigen solve, the ridge solve beside
+// the residual eigen solve). It forks from and joins the caller's stream
+// through events, so a stream capture of the caller's stream follows it. The
+// stream and events are created by the first call on a device (make that call
+// before capturing); `g_side_mu` is held from fork to join so that concurrent
+// callers do not interleave the event records.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+SideStream* side_stream() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (!ss.s) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+  }
+  return &ss;
+}
+
+// fork: work enqueued on the returned stream runs beside `st` (st itself if
+// no side stream could be made); join: `st` waits for it.
+cudaStream_t fork_side(SideStream* ss, cudaStream_t st) {
+  if (!ss) return st;
+  if (cudaEventRecord(ss->fork, st) != cudaSuccess || cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess)
+    return st;
+  return ss->s;
+}
+cudaError_t join_side(SideStream* ss, cudaStream_t side, cudaStream_t st) {
+  if (!ss || side == st) return cudaSuccess;
+  cudaError_t e = cudaEventRecord(ss->join, side);
+  if (e != cudaSuccess) return e;
+  return cudaStreamWaitEvent(st, ss->join, 0);
+}
 
 int sm_count() {
   int dev = 0, n = 148;
@@ -200,11 +244,17 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   const long long hs_in = static_cast<long long>(N) * d;
 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
-  SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, st));
-  SPR_TRY(launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st));
-  SPR_TRY(launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st));
-  SPR_TRY(launch_scale_columns(evl, evc, H, d, e, wk, st));
-  SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
+  {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStream* ss = side_stream();
+    const cudaStream_t side = fork_side(ss, st);
+    SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, side));
+    SPR_TRY(launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st));
+    SPR_TRY(launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st));
+    SPR_TRY(launch_scale_columns(evl, evc, H, d, e, wk, st));
+    SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
+    SPR_TRY(join_side(ss, side, st));
+  }
   const long long hs_z = static_cast<long long>(Nv) * e;
   SPR_TRY(launch_gather_init(z, kXf64, hs_z, e, e, init_k, Ck, H, mu, mun, st));
   // tensor-core assignment when the centroid planes fit in shared memory
@@ -529,8 +579,14 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
                             st));
     double* bmat = at<double>(ws, L.bmat);
     double* bvec = at<double>(ws, L.bvec);
-    SPR_TRY(launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, st));
     double* rtr = at<double>(ws, L.mk);
+    // the ridge solve (reads the Grams) runs beside R^T R and its eigen solve
+    // (they touch other regions); with r > 32 the Gram region is reused below,
+    // so the two stay in order
+    std::unique_lock<std::mutex> lk(g_side_mu);
+    SideStream* ss = (c.p.r <= 32) ? side_stream() : nullptr;
+    const cudaStream_t side = fork_side(ss, st);
+    SPR_TRY(launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side));
     SPR_TRY(launch_gram_f64(xr + static_cast<size_t>(M) * d, xr + static_cast<size_t>(M) * d,
                             nullptr, nullptr, hs, hs, d, M, H, d, 1.0, 0.0, rtr,
                             static_cast<long long>(d) * d, 0, st));
@@ -546,6 +602,8 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
       SPR_TRY(launch_top_eig_projector(evl, evc, H, d, c.p.r, sel, false, st));
       vr = sel;
     }
+    SPR_TRY(join_side(ss, side, st));
+    lk.unlock();
     SPR_TRY(launch_project_map(bmat, bvec, vr, H, d, c.p.r, bp32, bv32, fit, st));
   } else {
     SPR_TRY(cudaMemsetAsync(bp32, 0, static_cast<size_t>(H) * d * d * 4, st));

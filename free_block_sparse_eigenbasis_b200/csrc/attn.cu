@@ -638,35 +638,42 @@ __global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, c
 
 // Split-KV combine: out = sum_s 2^(l_s - L) O_s / sum_s 2^(l_s - L),
 // L = max_s l_s, over the splits' normalised partial outputs O_s and
-// log2-sum-exps l_s. One block per (unit, head), thread = column, rows in
-// turn (fixed order over the splits).
+// log2-sum-exps l_s (fixed order over the splits). Block = 8 rows of one
+// unit, thread = (row, 4 columns).
 __global__ void split_combine_kernel(const float* opart, const float* lpart, const int32_t* off_q,
                                      const int32_t* work, const int32_t* nwork, int Cq,
                                      int tiles_per_head, int units, int splits, int q_rows, int d,
                                      float* out) {
-  const int h = blockIdx.y, wi = blockIdx.x;
+  const int h = blockIdx.z, wi = blockIdx.y;
   if (wi >= nwork[h]) return;
   const int wcode = work[static_cast<size_t>(h) * tiles_per_head + wi];
   const int g = wcode >> 16, tu = wcode & 0xFFFF;
   const int32_t* offq = off_q + static_cast<size_t>(h) * (Cq + 1);
   const int row0 = offq[g] + tu * kUnitRows;
   const int rows = min(kUnitRows, offq[g + 1] - row0);
+  const int cpr = d / 4;  // threads per row
+  const int r = blockIdx.x * (blockDim.x / cpr) + threadIdx.x / cpr;
+  const int c = (threadIdx.x % cpr) * 4;
+  if (r >= rows) return;
   const size_t ub = (static_cast<size_t>(h) * units + wi) * splits;
-  for (int r = 0; r < rows; ++r) {
-    float L = -INFINITY;
-    for (int s = 0; s < splits; ++s) L = fmaxf(L, lpart[(ub + s) * kUnitRows + r]);
-    for (int c = threadIdx.x; c < d; c += blockDim.x) {
-      float num = 0.f, den = 0.f;
-      for (int s = 0; s < splits; ++s) {
-        const float ls = lpart[(ub + s) * kUnitRows + r];
-        if (ls == -INFINITY) continue;
-        const float wgt = exp2f(ls - L);
-        num = fmaf(wgt, opart[((ub + s) * kUnitRows + r) * d + c], num);
-        den += wgt;
-      }
-      out[(static_cast<size_t>(h) * q_rows + row0 + r) * d + c] = den > 0.f ? num / den : 0.f;
-    }
+  float L = -INFINITY;
+  for (int s = 0; s < splits; ++s) L = fmaxf(L, lpart[(ub + s) * kUnitRows + r]);
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float ls = lpart[(ub + s) * kUnitRows + r];
+    if (ls == -INFINITY) continue;
+    const float wgt = exp2f(ls - L);
+    const float4 o = *reinterpret_cast<const float4*>(opart + ((ub + s) * kUnitRows + r) * d + c);
+    num.x = fmaf(wgt, o.x, num.x);
+    num.y = fmaf(wgt, o.y, num.y);
+    num.z = fmaf(wgt, o.z, num.z);
+    num.w = fmaf(wgt, o.w, num.w);
+    den += wgt;
   }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  *reinterpret_cast<float4*>(out + (static_cast<size_t>(h) * q_rows + row0 + r) * d + c) =
+      make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
 }
 
 __global__ void zero_i64_kernel(int64_t* p, int n) {
@@ -733,7 +740,7 @@ cudaError_t launch_attn_hd(const AttnArgs& a, AttnParams prm, cudaStream_t st) {
   dim3 grid(a.tiles_per_head * prm.splits, a.H);
   sparse_attn_kernel<HD><<<grid, kAttnThreads, shb, st>>>(maps, prm);
   if (prm.splits > 1)
-    split_combine_kernel<<<dim3(a.units, a.H), 128, 0, st>>>(
+    split_combine_kernel<<<dim3(kUnitRows / (256 / (HD / 4)), a.units, a.H), 256, 0, st>>>(
         a.opart, a.lpart, a.off_q, a.work, a.nwork, a.Cq, a.tiles_per_head, a.units, prm.splits,
         a.q_rows, HD, a.out);
   return cudaGetLastError();

@@ -27,11 +27,11 @@ constexpr int kInvIters = 3;
 template <int D>
 __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in, double* scratch) {
   extern __shared__ double tsm[];
-  double* A = tsm;              // [D*D] full symmetric
+  double* A = tsm;              // [D*D] full symmetric (rows are read instead of columns)
   double* v = A + D * D;        // [D]
   double* w = v + D;            // [D]
-  __shared__ double red[kTriThreads / 32];
-  __shared__ double bc[4];
+  __shared__ double red[2][kTriThreads / 32];
+  __shared__ double pw[kTriThreads / D][D];
   const int h = blockIdx.x;
   const double* Ah = A_in + static_cast<size_t>(h) * D * D;
   double* hv = scratch + static_cast<size_t>(h) * (D * D + 3 * D);
@@ -41,29 +41,27 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int t = tid; t < D * D; t += blockDim.x) A[t] = Ah[t];
   __syncthreads();
+  int nsum = 0;
+  // sum over the block with one barrier (alternating buffers; every thread
+  // adds the warp partials in the same order)
   auto block_sum = [&](double x) -> double {
     x = warp_sum_f64(x);
-    if (lane == 0) red[wid] = x;
+    double* rb = red[nsum++ & 1];
+    if (lane == 0) rb[wid] = x;
     __syncthreads();
-    if (tid == 0) {
-      double s = 0.0;
-      for (int i = 0; i < kTriThreads / 32; ++i) s += red[i];
-      bc[3] = s;
-    }
-    __syncthreads();
-    const double s = bc[3];
-    __syncthreads();
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < kTriThreads / 32; ++i) s += rb[i];
     return s;
   };
+  constexpr int kParts = kTriThreads / D;  // row parts of the matrix-vector product
   for (int k = 0; k < D - 2; ++k) {
     const int n1 = D - k - 1;  // length of v (rows k+1 .. D-1)
+    const double* Ak = A + k * D;  // row k = column k (symmetry)
     double x2 = 0.0;
-    for (int i = k + 2 + tid; i < D; i += blockDim.x) {
-      const double a = A[i * D + k];
-      x2 += a * a;
-    }
+    for (int i = k + 2 + tid; i < D; i += blockDim.x) x2 = fma(Ak[i], Ak[i], x2);
     x2 = block_sum(x2);
-    const double alpha = A[(k + 1) * D + k];
+    const double alpha = Ak[k + 1];
     if (x2 == 0.0) {  // column already reduced: H_k = I
       if (tid == 0) {
         tau[k] = 0.0;
@@ -77,7 +75,7 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
     const double tk = (beta - alpha) / beta;
     const double scl = 1.0 / (alpha - beta);
     for (int i = tid; i < n1; i += blockDim.x) {
-      const double vi = (i == 0) ? 1.0 : A[(k + 1 + i) * D + k] * scl;
+      const double vi = (i == 0) ? 1.0 : Ak[k + 1 + i] * scl;
       v[i] = vi;
       hv[k * D + (k + 1 + i)] = vi;
     }
@@ -86,24 +84,30 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
       od[k] = beta;
     }
     __syncthreads();
-    // p = tau A22 v: 4 threads per row, fixed combination order
+    // p = tau A22 v by columns (A22 symmetric): thread (column c, part) sums
+    // the rows r = part, part + kParts, ...
     {
-      const int r = tid >> 2, part = tid & 3;
-      double s = 0.0;
-      if (r < n1) {
-        const double* row = A + (k + 1 + r) * D + (k + 1);
-        for (int c = part; c < n1; c += 4) s = fma(row[c], v[c], s);
+      const int c = tid % D, part = tid / D;
+      double sacc = 0.0;
+      if (c < n1) {
+        const double* col = A + (k + 1) * D + (k + 1) + c;
+        for (int r = part; r < n1; r += kParts) sacc = fma(col[r * D], v[r], sacc);
       }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (r < n1 && part == 0) w[r] = tk * s;
+      pw[part][c] = sacc;
     }
     __syncthreads();
     double pv = 0.0;
-    for (int i = tid; i < n1; i += blockDim.x) pv += w[i] * v[i];
+    if (tid < n1) {
+      double sacc = pw[0][tid];
+#pragma unroll
+      for (int q = 1; q < kParts; ++q) sacc += pw[q][tid];
+      const double wi = tk * sacc;
+      w[tid] = wi;
+      pv = wi * v[tid];
+    }
     pv = block_sum(pv);
     const double kk = -0.5 * tk * pv;
-    for (int i = tid; i < n1; i += blockDim.x) w[i] += kk * v[i];
+    if (tid < n1) w[tid] += kk * v[tid];
     __syncthreads();
     // A22 -= v w^T + w v^T (warp = row stripe, lane = column stripe)
     for (int r = wid; r < n1; r += kTriThreads / 32) {
@@ -204,6 +208,9 @@ template <int D>
 constexpr size_t eig_work_bytes() {
   return static_cast<size_t>(4) * D * 32 * 8 + static_cast<size_t>(D) * 32 * 4;
 }
+static_assert(eig_work_bytes<128>() >= (128 * 128 + 128) * 8 &&
+                  eig_work_bytes<64>() >= (64 * 64 + 64) * 8,
+              "the back-transformation reuses the work space for the Householder vectors");
 
 template <int D>
 __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scratch, int ne,
@@ -297,16 +304,24 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
     }
     __syncthreads();
   }
-  // back-transformation: u = H_0 (H_1 (... H_{D-3} y)), warp w owns vectors w, w + 8, ...
+  // back-transformation: u = H_0 (H_1 (... H_{D-3} y)), warp w owns vectors
+  // w, w + 8, ...; the Householder vectors and tau are first staged in the
+  // (now free) inverse-iteration work space
+  double* hs = eig_work;          // [D][D]
+  double* ts = eig_work + D * D;  // [D]
+  for (int i = tid; i < D * D; i += blockDim.x) hs[i] = hv[i];
+  for (int i = tid; i < D; i += blockDim.x) ts[i] = tau[i];
+  __syncthreads();
   for (int t = wid; t < ne; t += kEigThreads / 32) {
     double* y = Y[t];
     for (int k = D - 3; k >= 0; --k) {
-      const double tk = tau[k];
+      const double tk = ts[k];
       if (tk == 0.0) continue;
+      const double* hk = hs + k * D;
       double dot = 0.0;
-      for (int i = k + 1 + lane; i < D; i += 32) dot = fma(hv[k * D + i], y[i], dot);
+      for (int i = k + 1 + lane; i < D; i += 32) dot = fma(hk[i], y[i], dot);
       dot = warp_sum_f64(dot) * tk;
-      for (int i = k + 1 + lane; i < D; i += 32) y[i] -= dot * hv[k * D + i];
+      for (int i = k + 1 + lane; i < D; i += 32) y[i] -= dot * hk[i];
       __syncwarp();
     }
     for (int i = lane; i < D; i += 32)

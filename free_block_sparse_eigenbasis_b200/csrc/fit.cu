@@ -125,8 +125,9 @@ __global__ void probe_means_kernel(const double* part, int nblk, int M, int d, d
 // below and the columns), and b = rbar - xbar B.
 constexpr int kRidgeThreads = 512;
 
+template <int d>
 __global__ void __launch_bounds__(kRidgeThreads)
-    ridge_solve_kernel(const double* gram, int d, double* bmat, double* bvec, const double* means,
+    ridge_solve_kernel(const double* gram, double* bmat, double* bvec, const double* means,
                        DeviceStats* stats) {
   extern __shared__ double rsm[];
   const int ntri = d * (d + 1) / 2;
@@ -338,11 +339,11 @@ cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const
 cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
                                const double* means, DeviceStats* stats, cudaStream_t st) {
   const size_t shb = (static_cast<size_t>(d) * (d + 1) / 2 + static_cast<size_t>(d) * d) * 8;
-  cudaError_t e = cudaFuncSetAttribute(ridge_solve_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(shb));
+  if (d != 64 && d != 128) return cudaErrorInvalidValue;
+  auto kern = (d == 128) ? ridge_solve_kernel<128> : ridge_solve_kernel<64>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shb));
   if (e != cudaSuccess) return e;
-  ridge_solve_kernel<<<H, kRidgeThreads, shb, st>>>(gram, d, bmat, bvec, means, stats);
+  kern<<<H, kRidgeThreads, shb, st>>>(gram, bmat, bvec, means, stats);
   return cudaGetLastError();
 }
 

@@ -135,8 +135,8 @@ __global__ void gram_f64_kernel(const double* X, const double* Y, const double* 
 // ---------------------------------------------------------------------------
 // Key response coordinates z = W^T k, W = U_e L_e^{1/2} ([d, e] fp64).
 // ---------------------------------------------------------------------------
-constexpr int kZRows = 128;
-constexpr int kZThreads = 256;
+constexpr int kZRows = 64;
+constexpr int kZThreads = 128;
 
 // 16-byte vector of k widened to float
 __device__ __forceinline__ int zvec_elems(const __nv_bfloat16*) { return 8; }
@@ -158,16 +158,16 @@ __device__ __forceinline__ void zvec_store(const float* src, float* dst) {
   dst[3] = v.w;
 }
 
-// Block = 128 key rows: the rows are staged in shared memory with 16-byte
-// loads, then thread t computes 8 of the e coordinates of row t % 128 (one
-// shared load of k per 8 fma; w broadcast to the warp), summing over the d
-// columns in ascending order in fp64.
+// Block = 128 key rows: the rows are staged in shared memory (as fp64) with
+// 16-byte loads; thread t computes 4 of the e coordinates of 2 rows (register
+// blocking: per column of k two shared loads of k and two 16-byte loads of
+// w serve 8 fma), summing over the d columns in ascending order in fp64.
 template <typename T>
 __global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int Nv, int d, int e,
                                                           const double* wk, double* z) {
   extern __shared__ double zsm[];
-  double* w = zsm;                  // [d][e]
-  float* ks = reinterpret_cast<float*>(zsm + d * e);  // [kZRows][d+1]
+  double* w = zsm;                   // [d][e]
+  double* ks = zsm + d * e;          // [kZRows][d+1]
   const int h = blockIdx.y;
   const int j0 = blockIdx.x * kZRows;
   const double* W = wk + static_cast<size_t>(h) * d * e;
@@ -184,29 +184,49 @@ __global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int
 #pragma unroll
       for (int i = 0; i < 8; ++i) tmp[i] = 0.f;
     }
-    for (int i = 0; i < ve; ++i) ks[r * (d + 1) + a + i] = tmp[i];
+    for (int i = 0; i < ve; ++i) ks[r * (d + 1) + a + i] = static_cast<double>(tmp[i]);
   }
   __syncthreads();
-  const int r = threadIdx.x % kZRows;
-  const int j = j0 + r;
-  if (j >= Nv) return;
-  const float* kr = ks + r * (d + 1);
-  double* zr = z + (static_cast<size_t>(h) * Nv + j) * e;
-  for (int c0 = (threadIdx.x / kZRows) * 8; c0 < e; c0 += 16) {
-    const int ne = min(8, e - c0);
-    double acc[8];
+  const int nq = (e + 3) / 4;                       // column quads
+  const int pairs = (kZRows / 2) * nq;              // (row pair, quad) items
+  for (int item = threadIdx.x; item < pairs; item += blockDim.x) {
+    const int rp = item % (kZRows / 2), qd = item / (kZRows / 2);
+    const int r0 = 2 * rp, c0 = 4 * qd;
+    const int nc = min(4, e - c0);
+    double acc0[4] = {0.0, 0.0, 0.0, 0.0}, acc1[4] = {0.0, 0.0, 0.0, 0.0};
+    const double* k0 = ks + r0 * (d + 1);
+    const double* k1 = k0 + (d + 1);
+    if (nc == 4 && (e % 2) == 0) {
+      for (int a = 0; a < d; ++a) {
+        const double x0 = k0[a], x1 = k1[a];
+        const double2 wa = *reinterpret_cast<const double2*>(w + a * e + c0);
+        const double2 wb = *reinterpret_cast<const double2*>(w + a * e + c0 + 2);
+        acc0[0] = fma(x0, wa.x, acc0[0]);
+        acc0[1] = fma(x0, wa.y, acc0[1]);
+        acc0[2] = fma(x0, wb.x, acc0[2]);
+        acc0[3] = fma(x0, wb.y, acc0[3]);
+        acc1[0] = fma(x1, wa.x, acc1[0]);
+        acc1[1] = fma(x1, wa.y, acc1[1]);
+        acc1[2] = fma(x1, wb.x, acc1[2]);
+        acc1[3] = fma(x1, wb.y, acc1[3]);
+      }
+    } else {
+      for (int a = 0; a < d; ++a) {
+        const double x0 = k0[a], x1 = k1[a];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.0;
-    for (int a = 0; a < d; ++a) {
-      const double kv = static_cast<double>(kr[a]);
-      const double* wa = w + a * e + c0;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c < ne) acc[c] = fma(kv, wa[c], acc[c]);
+        for (int c = 0; c < 4; ++c)
+          if (c < nc) {
+            acc0[c] = fma(x0, w[a * e + c0 + c], acc0[c]);
+            acc1[c] = fma(x1, w[a * e + c0 + c], acc1[c]);
+          }
+      }
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      if (c < ne) zr[c0 + c] = acc[c];
+    for (int c = 0; c < 4; ++c) {
+      if (c >= nc) continue;
+      if (j0 + r0 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r0) * e + c0 + c] = acc0[c];
+      if (j0 + r0 + 1 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r0 + 1) * e + c0 + c] = acc1[c];
+    }
   }
 }
 
@@ -614,7 +634,7 @@ cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
 
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
                          const double* wk, double* z, cudaStream_t st) {
-  const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;
+  const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 8;
   dim3 grid((Nv + kZRows - 1) / kZRows, H);
   if (bf16) {
     cudaFuncSetAttribute(zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
