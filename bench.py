@@ -98,17 +98,45 @@ class ClockSampler:
                     reasons=sorted(reasons), samples=len(sm))
 
 
+def count_launches(call) -> int:
+    """Kernels of this library launched by one call, counted from the CUDA
+    activity records of torch's profiler on an untimed call (torch's own
+    kernels excluded). Returns -1 if the profiler is unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            call()
+            torch.cuda.synchronize()
+        n = 0
+        for ev in prof.events():
+            dev_type = getattr(ev, "device_type", None)
+            if dev_type is None or "CUDA" not in str(dev_type):
+                continue
+            name = ev.name or ""
+            if name.startswith("void at::") or "at::native" in name or name.startswith("Memcpy") \
+                    or name.startswith("Memset"):
+                continue
+            n += 1
+        return n
+    except Exception:
+        return -1
+
+
 def gpu_launches_per_call(w) -> int:
-    """Kernels the library launches for one call of this workload (mirrors the
-    launch sequences of the C ABI; checked against the profiler's launch list)."""
+    """Kernels the library launches for one call of this workload when every
+    k-means runs all its passes (mirrors the launch sequences of the C ABI;
+    the fallback when the profiler count is unavailable)."""
     it = w.kmeans_iters
-    partition = (7 + 2 * it + 4 * (it - 1)      # setup, metric, eigen, coordinates; key passes
-                 + 3 + 1 + 1 + 1                 # final key sort, C_K, G, query init
-                 + 3 * it + 4 * (it - 1) + 2)    # query passes, labels out
-    permute = 3 + 3 + 3
-    route = 4
-    attn = 5 if True else 0
-    probe = (3 + 5 + 1 + 2 + 1 + 1 + 1 + 1 + 1 + 1) if w.M > 0 else 2
+    partition = (11                    # reset, Fisher-Yates, M_K, eigen (2), scaling, z, inits, planes
+                 + 6 * it + 4 * (it - 1)  # key passes (2 zero, centroid planes, argmin, recheck,
+                                          # finalize) and centroid updates (sort + mean)
+                 + 5                      # final key sort, C_K, G
+                 + 7 * it + 4 * (it - 1)  # query passes (+ metric apply) and updates
+                 + 2)                     # labels out
+    permute = 2 * 3 + 3
+    route = 5
+    attn = 5
+    probe = 18 if w.M > 0 else 5
     return partition + permute + route + attn + probe
 
 
@@ -295,6 +323,12 @@ def main():
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
+    # kernels per call, counted on one extra (untimed) call
+    launches = count_launches(lambda: call(qd, kd, vd))
+    launches_src = "profiler count of one call"
+    if launches <= 0:
+        launches, launches_src = gpu_launches_per_call(w), "launch-sequence formula"
+
     # max over ranks
     vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms], device=dev,
                         dtype=torch.float64)
@@ -341,7 +375,9 @@ def main():
             e2e=dict(value=4.0 * w.d * P_exec_all / (e2e_max * 1e-3) / 1e12, unit="TFLOPS",
                      ms=e2e_max, h2d_bytes_per_step=3 * qd.numel() * qd.element_size(),
                      d2h_bytes_per_step=b.out.numel() * b.out.element_size()),
-            gpu_launches=gpu_launches_per_call(w) * args.steps,
+            gpu_launches=launches * args.steps,
+            gpu_launches_per_call=launches,
+            gpu_launches_source=launches_src,
         )
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline_sample(w)

@@ -36,7 +36,6 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->H < 1 || p->H > SPARSEPR_MAX_HEADS) return SPARSEPR_ERR_INVALID_ARG;
   if (p->n_text < 0 || p->N < 16) return SPARSEPR_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SPARSEPR_ERR_UNSUPPORTED;
-  if (p->n_text != 0) return SPARSEPR_ERR_UNSUPPORTED;
   const long long Nv = static_cast<long long>(p->N) - p->n_text;
   if (Nv < 1) return SPARSEPR_ERR_INVALID_ARG;
   if (static_cast<long long>(p->H) * p->N >= (1LL << 31)) return SPARSEPR_ERR_UNSUPPORTED;
@@ -399,13 +398,12 @@ sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v, sp
   if (qp == q || kp == k || vp == v) return SPARSEPR_ERR_INVALID_ARG;
   if (!al16(q, k, v, qp, kp, vp)) return SPARSEPR_ERR_INVALID_ARG;
   const int H = c.p.H, N = c.p.N, d = c.p.d;
-  const int nchunk = (N + kSortChunk - 1) / kSortChunk;
-  if (static_cast<size_t>(H) * nchunk * c.L.Cmax > static_cast<size_t>(H) * c.L.nchunk * c.L.Cmax)
-    return SPARSEPR_ERR_UNSUPPORTED;  // only while n_text == 0 (N == Nv)
+  const int nchunk = c.L.nchunk;  // chunks of all N tokens
   int32_t* hist = at<int32_t>(ws, c.L.hist);
-  SPR_TRY(launch_counting_sort(label_q, H, N, c.p.Cq, nchunk, hist, perm_q, off_q, nullptr, 0,
+  // with text tokens the last group of each side is the text group
+  SPR_TRY(launch_counting_sort(label_q, H, N, c.L.Cqt, nchunk, hist, perm_q, off_q, nullptr, 0,
                                c.stats, c.st));
-  SPR_TRY(launch_counting_sort(label_k, H, N, c.p.Ck, nchunk, hist, perm_k, off_k, nullptr, 0,
+  SPR_TRY(launch_counting_sort(label_k, H, N, c.L.Ckt, nchunk, hist, perm_k, off_k, nullptr, 0,
                                c.stats, c.st));
   const int eb = c.bf16 ? 2 : 4;
   SPR_TRY(launch_gather_rows(q, qp, perm_q, H, N, d, eb, c.st));
@@ -426,8 +424,9 @@ sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt
   const int H = c.p.H, N = c.p.N, d = c.p.d, Ck = c.p.Ck, Cq = c.p.Cq;
   double* cq = at<double>(ws, c.L.cq);
   double* ckr = at<double>(ws, c.L.ckr);
-  SPR_TRY(launch_range_mean(qp, c.kind, H, N, d, off_q, Cq, cq, c.st));
-  SPR_TRY(launch_range_mean(kp, c.kind, H, N, d, off_k, Ck, ckr, c.st));
+  // block scores of the video groups (the text groups are kept outside the budget)
+  SPR_TRY(launch_range_mean(qp, c.kind, H, N, d, off_q, Cq, c.L.Cqt + 1, cq, c.st));
+  SPR_TRY(launch_range_mean(kp, c.kind, H, N, d, off_k, Ck, c.L.Ckt + 1, ckr, c.st));
   int32_t kh[SPARSEPR_MAX_HEADS];
   for (int h = 0; h < H; ++h) kh[h] = keep_budget(c.p.keep[h], Ck);
   SPR_TRY(launch_write_k(kh, H, k_per_head, c.st));
@@ -468,8 +467,9 @@ sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const
   a.N = N;
   a.d = d;
   a.q_rows = N;
-  a.Cq = c.p.Cq;
-  a.Ck = c.p.Ck;
+  a.Cq = c.L.Cqt;
+  a.Ck = c.L.Ckt;
+  a.text = c.p.n_text > 0 ? 1 : 0;
   a.off_q = off_q;
   a.off_k = off_k;
   a.csr = csr;
@@ -509,7 +509,7 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
   float* bv32 = at<float>(ws, L.bv32);
   float* od = at<float>(ws, L.od);
   if (M > 0) {
-    SPR_TRY(launch_probe_select(off_q, H, Cq, M, probes, st));
+    SPR_TRY(launch_probe_select(off_q, L.Cqt + 1, H, Cq, M, probes, st));  // video groups only
     __nv_bfloat16* pq = at<__nv_bfloat16>(ws, L.probe_q);
     SPR_TRY(launch_gather_probe_rows(qp, c.bf16, probes, H, N, M, d, pq, st));
     const void *k16 = kp, *v16 = vp;
@@ -611,10 +611,11 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     if (fit) SPR_TRY(cudaMemsetAsync(fit, 0, static_cast<size_t>(H) * (d * d + d) * 8, st));
   }
   if (correct_tc_supported(H, N, d))
-    SPR_TRY(launch_correct_tc(o_sparse, od, probes, perm_q, bp32, bv32, H, N, M, d, out, c.bf16,
+    SPR_TRY(launch_correct_tc(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out, c.bf16,
                               sm_count(), c.stats, st));
   else
-    SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, M, d, out, c.bf16, st));
+    SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out, c.bf16,
+                           st));
   SPR_TRY(launch_pairs_exec(pairs_sparse, H, static_cast<int64_t>(M) * N, pairs_exec, c.stats, st));
   return SPARSEPR_OK;
 }

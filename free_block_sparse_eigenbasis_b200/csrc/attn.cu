@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   int2* runs_s = reinterpret_cast<int2*>(smem + L::runs_off);
   // run-list capacity left in the dynamic allocation after alignment
   const int cap = (kAttnSmemBytes - static_cast<int>(smem - smem_raw) - L::runs_off) / 8;
-  const int2* runs_g = p.runs + gi * p.kmax;
+  const int2* runs_g = p.runs + gi * (p.kmax + 1);
   const bool runs_in_smem = nr <= cap;
   const int2* runs = runs_in_smem ? runs_s : runs_g;
 
@@ -239,80 +239,83 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort = &bars->abort;
 
   if (warp == 8) {
-    // ---------------- TMA producer: Q once, then K(j), V(j) in order ----------------
+    // ------- TMA producer warp: Q once, then K(j) and V(j) in order. Lane s
+    // (and s + 16) finds the first row of slot s of the tile; a tile whose
+    // slots are all contiguous is fetched as one 128-row box, any other
+    // tile slot by slot (8-row boxes, lanes 0-15 in parallel). -------
+    const int krow_base = h * p.N;
     if (lane == 0) {
-      const int krow_base = h * p.N;
       mbar_arrive_expect_tx(&bars->q_full, nq * kAtoms * p.q_box_rows * 128);
       for (int qt = 0; qt < nq; ++qt)
         for (int a = 0; a < kAtoms; ++a)
           tma_load_2d(Qs + qt * L::kQBytes + a * L::kSlab, &maps.q, &bars->q_full, a * 64,
                       h * p.q_rows + row0 + qt * kTileM);
-      int ri = -1, pos = 0, rend = 0;  // current run and its row range [pos, rend)
-      for (int skip = j0 * kSlotsPerTile; skip > 0 && ri + 1 < nr;) {
-        ++ri;
-        pos = runs[ri].x;
-        rend = pos + runs[ri].y;
-        const int rs = (runs[ri].y + kSlotRows - 1) / kSlotRows;
-        const int take = min(skip, rs);
-        pos += take * kSlotRows;
-        skip -= take;
+    }
+    const int sl = lane & (kSlotsPerTile - 1);
+    auto run_slots = [&](int r) { return (runs[r].y + kSlotRows - 1) / kSlotRows; };
+    // run holding the first slot of this CTA's key range, and that run's first slot
+    int rb = 0, cb = 0;
+    {
+      const int t0 = j0 * kSlotsPerTile;
+      while (rb < nr && t0 >= cb + run_slots(rb)) {
+        cb += run_slots(rb);
+        ++rb;
       }
-      int k_issued = -1, v_issued = -1;
-      for (int j = 0; j < T; ++j) {
-        // box plan of key tile j: (slot, first row, log2 size) per box
-        int bslot[kSlotsPerTile], brow[kSlotsPerTile], blg[kSlotsPerTile];
-        int nb = 0;
-        int t = 0;
-        while (t < kSlotsPerTile) {
-          while (pos >= rend && ri < nr) {
-            ++ri;
-            if (ri < nr) {
-              pos = runs[ri].x;
-              rend = pos + runs[ri].y;
-            }
-          }
-          int r, m;
-          if (pos < rend) {
-            r = pos;
-            m = min(kSlotsPerTile - t, (rend - pos + kSlotRows - 1) / kSlotRows);
-            pos += m * kSlotRows;
-          } else {
-            r = 0;  // past the last run: any rows of the head (masked)
-            m = kSlotsPerTile - t;
-          }
-          for (int lg = p.max_lg; lg >= 0 && m > 0; --lg) {
-            const int sz = 1 << lg;
-            while (m >= sz) {
-              bslot[nb] = t;
-              brow[nb] = r;
-              blg[nb] = lg;
-              ++nb;
-              t += sz;
-              r += sz * kSlotRows;
-              m -= sz;
-            }
-          }
-        }
-        const int st = j % kStages;
-        const uint32_t ph = ((j / kStages) + 1) & 1;
-        if (j >= kStages && !mbar_wait(&bars->kempty[st], ph, abort)) break;
-        mbar_arrive_expect_tx(&bars->kfull[st], L::kKVBytes);
-        for (int b = 0; b < nb; ++b)
-#pragma unroll
-          for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(Ks + st * L::kKVBytes + a * L::kSlab + bslot[b] * 1024, &maps.k[blg[b]],
-                        &bars->kfull[st], a * 64, krow_base + brow[b]);
-        k_issued = j;
-        if (j >= kStages && !mbar_wait(&bars->vempty[st], ph, abort)) break;
-        mbar_arrive_expect_tx(&bars->vfull[st], L::kKVBytes);
-        for (int b = 0; b < nb; ++b)
-#pragma unroll
-          for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(Vs + st * L::kKVBytes + a * L::kSlab + bslot[b] * 1024, &maps.v[blg[b]],
-                        &bars->vfull[st], a * 64, krow_base + brow[b]);
-        v_issued = j;
+    }
+    int k_issued = -1, v_issued = -1;
+    const bool big_box = p.max_lg == 4;  // the tensor holds at least one 128-row box
+    for (int j = 0; j < T; ++j) {
+      const int t = (j0 + j) * kSlotsPerTile + sl;
+      int r = rb, c = cb;
+      while (r < nr && t >= c + run_slots(r)) {
+        c += run_slots(r);
+        ++r;
       }
-      // let the loads already in flight land before the CTA exits
+      // past the last run: any rows of the head (masked)
+      const int row = (r < nr) ? runs[r].x + (t - c) * kSlotRows : 0;
+      rb = __shfl_sync(0xffffffffu, r, kSlotsPerTile - 1);  // runs ascend: the next tile starts here
+      cb = __shfl_sync(0xffffffffu, c, kSlotsPerTile - 1);
+      const int prev = __shfl_up_sync(0xffffffffu, row, 1);
+      const bool follows = lane == 0 || lane >= kSlotsPerTile || row == prev + kSlotRows;
+      const bool whole = big_box && __all_sync(0xffffffffu, follows);
+      const int row_first = __shfl_sync(0xffffffffu, row, 0);
+      const int st = j % kStages;
+      const uint32_t ph = ((j / kStages) + 1) & 1;
+      bool w = true;
+      if (lane == 0 && j >= kStages) w = mbar_wait(&bars->kempty[st], ph, abort);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&bars->kfull[st], L::kKVBytes);
+      __syncwarp();
+      if (whole) {
+        if (lane == 0)
+          for (int a = 0; a < kAtoms; ++a)
+            tma_load_2d(Ks + st * L::kKVBytes + a * L::kSlab, &maps.k[4], &bars->kfull[st], a * 64,
+                        krow_base + row_first);
+      } else if (lane < kSlotsPerTile) {
+        for (int a = 0; a < kAtoms; ++a)
+          tma_load_2d(Ks + st * L::kKVBytes + a * L::kSlab + sl * 1024, &maps.k[0],
+                      &bars->kfull[st], a * 64, krow_base + row);
+      }
+      k_issued = j;
+      w = true;
+      if (lane == 0 && j >= kStages) w = mbar_wait(&bars->vempty[st], ph, abort);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&bars->vfull[st], L::kKVBytes);
+      __syncwarp();
+      if (whole) {
+        if (lane == 0)
+          for (int a = 0; a < kAtoms; ++a)
+            tma_load_2d(Vs + st * L::kKVBytes + a * L::kSlab, &maps.v[4], &bars->vfull[st], a * 64,
+                        krow_base + row_first);
+      } else if (lane < kSlotsPerTile) {
+        for (int a = 0; a < kAtoms; ++a)
+          tma_load_2d(Vs + st * L::kKVBytes + a * L::kSlab + sl * 1024, &maps.v[0],
+                      &bars->vfull[st], a * 64, krow_base + row);
+      }
+      v_issued = j;
+    }
+    // let the loads already in flight land before the CTA exits
+    if (lane == 0) {
       volatile int never = 0;
       for (int j = max(0, k_issued - kStages + 1); j <= k_issued; ++j)
         mbar_wait(&bars->kfull[j % kStages], (j / kStages) & 1, &never);
@@ -585,49 +588,70 @@ __global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_hea
 }
 
 // Merged key runs and KV slot counts per query group (same rule the attention
-// kernel walks), and the exact routed pair count per head.
+// kernel walks), and the exact routed pair count per head. With text tokens
+// (text = 1) the last query group keeps every key and every other group
+// also keeps the last key group (the text tokens), outside its budget.
 __global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, const int32_t* csr,
                                    const int32_t* kh, int H, int N, int Cq, int Ck, int kmax,
-                                   int32_t* nslots, int2* runs, int32_t* nruns, int64_t* pairs,
-                                   DeviceStats* stats) {
+                                   int text, int32_t* nslots, int2* runs, int32_t* nruns,
+                                   int64_t* pairs, DeviceStats* stats) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= H * Cq) return;
   const int h = i / Cq, g = i % Cq;
+  const int Cqv = Cq - text, Ckv = Ck - text;  // routed (video) groups
   const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
   const int32_t* ok = off_k + static_cast<size_t>(h) * (Ck + 1);
-  const int32_t* row = csr + static_cast<size_t>(i) * kmax;
-  int2* rout = runs + static_cast<size_t>(i) * kmax;
-  const int k = kh[h];
+  int2* rout = runs + static_cast<size_t>(i) * (kmax + 1);
   const int64_t nq = oq[g + 1] - oq[g];
-  // reject malformed routes before the attention kernel walks them
-  bool valid = (k >= 0 && k <= kmax && ok[0] >= 0 && ok[Ck] <= N && nq >= 0);
-  for (int ci = 0; valid && ci < k; ++ci) {
-    const int c = row[ci];
-    valid = (c >= 0 && c < Ck && ok[c] >= 0 && ok[c] <= ok[c + 1]);
+  bool valid = (ok[0] >= 0 && ok[Ck] <= N && nq >= 0);
+  int64_t keys = 0;
+  int slots = 0, nr = 0;
+  auto add_run = [&](int lo, int hi) {
+    if (hi <= lo) return;
+    if (nr > 0 && rout[nr - 1].x + rout[nr - 1].y == lo) {
+      // adjacent to the previous run: extend it (slots are re-cut)
+      const int plen = rout[nr - 1].y;
+      slots -= (plen + kSlotRows - 1) / kSlotRows;
+      rout[nr - 1].y = plen + (hi - lo);
+      slots += (rout[nr - 1].y + kSlotRows - 1) / kSlotRows;
+    } else {
+      rout[nr++] = make_int2(lo, hi - lo);
+      slots += (hi - lo + kSlotRows - 1) / kSlotRows;
+    }
+    keys += hi - lo;
+  };
+  if (text && g == Cqv) {
+    if (valid) add_run(0, N);  // the text query group: every key
+  } else {
+    const int32_t* row = csr + (static_cast<size_t>(h) * Cqv + g) * kmax;
+    const int k = kh[h];
+    valid = valid && k >= 0 && k <= kmax;
+    // reject malformed routes before the attention kernel walks them
+    for (int ci = 0; valid && ci < k; ++ci) {
+      const int c = row[ci];
+      valid = (c >= 0 && c < Ckv && ok[c] >= 0 && ok[c] <= ok[c + 1]);
+    }
+    if (valid) {
+      int ci = 0;
+      while (ci < k) {
+        const int c = row[ci];
+        const int lo = ok[c];
+        int hi = ok[c + 1];
+        while (ci + 1 < k && ok[row[ci + 1]] == hi) {
+          ++ci;
+          hi = ok[row[ci] + 1];
+        }
+        add_run(lo, hi);
+        ++ci;
+      }
+      if (text) add_run(ok[Ckv], ok[Ckv + 1]);  // the text key group
+    }
   }
   if (!valid) {
     nslots[i] = 0;
     nruns[i] = 0;
     raise_status(stats, SPARSEPR_ERR_INVALID_ARG);
     return;
-  }
-  int64_t keys = 0;
-  int slots = 0, nr = 0;
-  int ci = 0;
-  while (ci < k) {
-    const int c = row[ci];
-    const int lo = ok[c];
-    int hi = ok[c + 1];
-    while (ci + 1 < k && ok[row[ci + 1]] == hi) {
-      ++ci;
-      hi = ok[row[ci] + 1];
-    }
-    if (hi > lo) {
-      rout[nr++] = make_int2(lo, hi - lo);
-      keys += hi - lo;
-      slots += (hi - lo + kSlotRows - 1) / kSlotRows;
-    }
-    ++ci;
   }
   nslots[i] = slots;
   nruns[i] = nr;
@@ -753,7 +777,7 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   if (a.pairs) zero_i64_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H);
   const int n = a.H * a.Cq;
   slots_pairs_kernel<<<(n + 127) / 128, 128, 0, st>>>(a.off_q, a.off_k, a.csr, a.kh, a.H, a.N,
-                                                     a.Cq, a.Ck, a.kmax, a.nslots, a.runs,
+                                                     a.Cq, a.Ck, a.kmax, a.text, a.nslots, a.runs,
                                                      a.nruns, a.pairs, a.stats);
   if (a.pairs) pairs_to_stats_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H, a.stats);
   AttnParams prm;

@@ -53,6 +53,7 @@ struct CtMaps {
 
 struct CtParams {
   int H, N, M, tiles_per_head;
+  int n_corr;             // rows >= n_corr (text tokens) are copied, not corrected
   const float* od;        // [H, M, d] dense outputs of the probes
   const int32_t* probes;  // [H, M] ascending group-major positions
   const int32_t* perm_q;  // [H, N] group-major position -> token
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kCtThreads, 1)
             if (pr[mid] < i) lo = mid + 1; else hi = mid;
           }
           const bool is_probe = valid && lo < p.M && pr[lo] == i;
+          const bool plain = i >= p.n_corr;  // text row: x itself
           const size_t dst =
               valid ? (static_cast<size_t>(h) * p.N + p.perm_q[static_cast<size_t>(h) * p.N + i]) * D : 0;
           const float* odr = p.od + (static_cast<size_t>(h) * p.M + lo) * D;
@@ -225,10 +227,17 @@ __global__ void __launch_bounds__(kCtThreads, 1)
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 xv = *reinterpret_cast<const float4*>(xrow + ((q ^ (r & 7)) << 4));
-              y[4 * q + 0] = xv.x + __uint_as_float(acc[4 * q + 0]) + bvs[col0 + 4 * q + 0];
-              y[4 * q + 1] = xv.y + __uint_as_float(acc[4 * q + 1]) + bvs[col0 + 4 * q + 1];
-              y[4 * q + 2] = xv.z + __uint_as_float(acc[4 * q + 2]) + bvs[col0 + 4 * q + 2];
-              y[4 * q + 3] = xv.w + __uint_as_float(acc[4 * q + 3]) + bvs[col0 + 4 * q + 3];
+              if (plain) {
+                y[4 * q + 0] = xv.x;
+                y[4 * q + 1] = xv.y;
+                y[4 * q + 2] = xv.z;
+                y[4 * q + 3] = xv.w;
+              } else {
+                y[4 * q + 0] = xv.x + __uint_as_float(acc[4 * q + 0]) + bvs[col0 + 4 * q + 0];
+                y[4 * q + 1] = xv.y + __uint_as_float(acc[4 * q + 1]) + bvs[col0 + 4 * q + 1];
+                y[4 * q + 2] = xv.z + __uint_as_float(acc[4 * q + 2]) + bvs[col0 + 4 * q + 2];
+                y[4 * q + 3] = xv.w + __uint_as_float(acc[4 * q + 3]) + bvs[col0 + 4 * q + 3];
+              }
             }
             if (is_probe) {
 #pragma unroll
@@ -306,8 +315,8 @@ bool correct_tc_supported(int H, int N, int d) {
 
 cudaError_t launch_correct_tc(const float* o_sparse, const float* od, const int32_t* probes,
                               const int32_t* perm_q, const float* bpT, const float* bv32, int H,
-                              int N, int M, int d, void* out, bool out_bf16, int sm_count,
-                              DeviceStats* stats, cudaStream_t st) {
+                              int N, int n_corr, int M, int d, void* out, bool out_bf16,
+                              int sm_count, DeviceStats* stats, cudaStream_t st) {
   CtMaps maps;
   if (!map_f32(&maps.a, o_sparse, static_cast<size_t>(H) * N, d, kTileM) ||
       !map_f32(&maps.b, bpT, static_cast<size_t>(H) * d, d, d))
@@ -316,6 +325,7 @@ cudaError_t launch_correct_tc(const float* o_sparse, const float* od, const int3
   p.H = H;
   p.N = N;
   p.M = M;
+  p.n_corr = n_corr;
   p.tiles_per_head = (N + kTileM - 1) / kTileM;
   p.od = od;
   p.probes = probes;

@@ -11,14 +11,15 @@ namespace {
 
 // Probes per query group by largest remainder (ties to the lower group),
 // rows at offsets floor((t + 1/2) n_g / m_g) inside each group.
-__global__ void probe_select_kernel(const int32_t* off_q, int Cq, int M, int32_t* probes) {
+__global__ void probe_select_kernel(const int32_t* off_q, int off_stride, int Cq, int M,
+                                    int32_t* probes) {
   extern __shared__ int64_t psm[];
   int64_t* rem = psm;                                  // [Cq]
   int32_t* m = reinterpret_cast<int32_t*>(rem + Cq);   // [Cq]
   int32_t* start = m + Cq;                             // [Cq]
   __shared__ int32_t left;
   const int h = blockIdx.x;
-  const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
+  const int32_t* oq = off_q + static_cast<size_t>(h) * off_stride;
   const int64_t Nt = oq[Cq] - oq[0];
   for (int g = threadIdx.x; g < Cq; g += blockDim.x) {
     const int64_t n = oq[g + 1] - oq[g];
@@ -247,8 +248,8 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(256) correct_kernel(const float* o_sparse, const float* od,
                                                       const int32_t* probes,
                                                       const int32_t* perm_q, const float* bp32,
-                                                      const float* bv32, int N, int M, int d,
-                                                      void* out) {
+                                                      const float* bv32, int N, int n_corr, int M,
+                                                      int d, void* out) {
   extern __shared__ float csm[];
   float* Bs = csm;                 // [d][d]
   float* xs = Bs + d * d;          // [kCorrRows][d]
@@ -279,7 +280,9 @@ __global__ void __launch_bounds__(256) correct_kernel(const float* o_sparse, con
     const int i = i0 + r;
     if (i >= N) continue;
     float y;
-    if (prow[r] >= 0) {
+    if (i >= n_corr) {
+      y = xs[r * d + col];  // text rows: exact already, not corrected
+    } else if (prow[r] >= 0) {
       y = od[(static_cast<size_t>(h) * M + prow[r]) * d + col];
     } else {
       const float* xr = xs + r * d;
@@ -306,10 +309,10 @@ __global__ void pairs_exec_kernel(const int64_t* ps, int H, int64_t add, int64_t
 
 }  // namespace
 
-cudaError_t launch_probe_select(const int32_t* off_q, int H, int Cq, int M, int32_t* probes,
-                                cudaStream_t st) {
+cudaError_t launch_probe_select(const int32_t* off_q, int off_stride, int H, int Cq, int M,
+                                int32_t* probes, cudaStream_t st) {
   const size_t shb = static_cast<size_t>(Cq) * 16;
-  probe_select_kernel<<<H, 256, shb, st>>>(off_q, Cq, M, probes);
+  probe_select_kernel<<<H, 256, shb, st>>>(off_q, off_stride, Cq, M, probes);
   return cudaGetLastError();
 }
 
@@ -356,7 +359,8 @@ cudaError_t launch_project_map(const double* bmat, const double* bvec, const dou
 
 cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t* probes,
                            const int32_t* perm_q, const float* bp32, const float* bv32, int H,
-                           int N, int M, int d, void* out, bool out_bf16, cudaStream_t st) {
+                           int N, int n_corr, int M, int d, void* out, bool out_bf16,
+                           cudaStream_t st) {
   const size_t shb = (static_cast<size_t>(d) * d + static_cast<size_t>(kCorrRows) * d) * 4;
   dim3 grid((N + kCorrRows - 1) / kCorrRows, H);
   cudaError_t e;
@@ -364,14 +368,14 @@ cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t
     e = cudaFuncSetAttribute(correct_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(shb));
     if (e != cudaSuccess) return e;
-    correct_kernel<true><<<grid, 256, shb, st>>>(o_sparse, od, probes, perm_q, bp32, bv32, N, M,
-                                                 d, out);
+    correct_kernel<true><<<grid, 256, shb, st>>>(o_sparse, od, probes, perm_q, bp32, bv32, N,
+                                                 n_corr, M, d, out);
   } else {
     e = cudaFuncSetAttribute(correct_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(shb));
     if (e != cudaSuccess) return e;
-    correct_kernel<false><<<grid, 256, shb, st>>>(o_sparse, od, probes, perm_q, bp32, bv32, N, M,
-                                                  d, out);
+    correct_kernel<false><<<grid, 256, shb, st>>>(o_sparse, od, probes, perm_q, bp32, bv32, N,
+                                                  n_corr, M, d, out);
   }
   return cudaGetLastError();
 }

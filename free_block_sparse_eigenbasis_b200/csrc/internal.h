@@ -150,8 +150,9 @@ size_t route_scores_bytes(int H, int Cq, int Ck);
 cudaError_t launch_route_gemm(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
                               double scale, const int32_t* kh, int kmax, double* scores,
                               size_t scores_bytes, int32_t* csr, cudaStream_t st);
+// out[h, c] = mean of rows off[h, c]..off[h, c+1] (c < C; off rows of off_stride entries)
 cudaError_t launch_range_mean(const void* X, int x_kind, int H, int N, int d, const int32_t* off,
-                              int C, double* out, cudaStream_t st);
+                              int C, int off_stride, double* out, cudaStream_t st);
 cudaError_t launch_write_k(const int32_t* kh_host_vals, int H, int32_t* k_per_head,
                            cudaStream_t st);
 
@@ -162,10 +163,12 @@ struct AttnArgs {
   const void* vp;   // bf16 [H*N, d]
   int H, N, d;
   int q_rows;       // rows per head of the query tensor
-  int Cq, Ck;       // query groups per head (work list), key groups
+  int Cq, Ck;       // query groups per head (work list), key groups (with the text group)
+  int text = 0;     // 1: the last query group (Cq - 1) is the text group and keeps every
+                    // key; every other group also keeps the last key group (Ck - 1)
   const int32_t* off_q;  // [H, Cq+1]
   const int32_t* off_k;  // [H, Ck+1]
-  const int32_t* csr;    // [H, Cq, kmax]
+  const int32_t* csr;    // [H, Cq - text, kmax] routes of the (video) query groups
   const int32_t* kh;     // [H]
   int kmax;
   float scale;
@@ -174,7 +177,7 @@ struct AttnArgs {
   int32_t* nwork;        // [H]
   int tiles_per_head;
   int32_t* nslots;       // [H, Cq]
-  int2* runs;            // [H, Cq, kmax] merged key runs (start, length)
+  int2* runs;            // [H, Cq, kmax + 1] merged key runs (start, length)
   int32_t* nruns;        // [H, Cq]
   int64_t* pairs;        // [H] (may be null)
   DeviceStats* stats;
@@ -192,8 +195,8 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st);
 
 // ---- fit.cu ----------------------------------------------------------------
-cudaError_t launch_probe_select(const int32_t* off_q, int H, int Cq, int M, int32_t* probes,
-                                cudaStream_t st);
+cudaError_t launch_probe_select(const int32_t* off_q, int off_stride, int H, int Cq, int M,
+                                int32_t* probes, cudaStream_t st);
 cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* probes, int H,
                                      int N, int M, int d, __nv_bfloat16* dst, cudaStream_t st);
 // part: scratch of part_doubles fp64 for per-block column sums.
@@ -210,13 +213,15 @@ cudaError_t launch_project_map(const double* bmat, const double* bvec, const dou
 // ---- correct.cu: tensor-core residual correction ---------------------------
 bool correct_tc_supported(int H, int N, int d);
 // out[perm_q[i]] = od[probe] for probe rows, else x + x B' + b' (bpT = B'^T).
+// Rows >= n_corr (text tokens) are copied uncorrected.
 cudaError_t launch_correct_tc(const float* o_sparse, const float* od, const int32_t* probes,
                               const int32_t* perm_q, const float* bpT, const float* bv32, int H,
-                              int N, int M, int d, void* out, bool out_bf16, int sm_count,
-                              DeviceStats* stats, cudaStream_t st);
+                              int N, int n_corr, int M, int d, void* out, bool out_bf16,
+                              int sm_count, DeviceStats* stats, cudaStream_t st);
 cudaError_t launch_correct(const float* o_sparse, const float* od, const int32_t* probes,
                            const int32_t* perm_q, const float* bp32, const float* bv32, int H,
-                           int N, int M, int d, void* out, bool out_bf16, cudaStream_t st);
+                           int N, int n_corr, int M, int d, void* out, bool out_bf16,
+                           cudaStream_t st);
 cudaError_t launch_pairs_exec(const int64_t* pairs_sparse, int H, int64_t add, int64_t* pairs_exec,
                               DeviceStats* stats, cudaStream_t st);
 

@@ -64,9 +64,9 @@ struct Layout {
   size_t bf16_qkv; // [3, H, N, d] bf16 copies (fp32 inputs only)
   size_t work;     // [H, tiles_per_head] int32 attention work list
   size_t nwork;    // [H] int32
-  size_t nslots;   // [H, Cq] int32 KV row-slots per query group
-  size_t runs;     // [H, Cq, kmax] int2 merged kept key runs (start, length)
-  size_t nruns;    // [H, Cq] int32
+  size_t nslots;   // [H, Cqt] int32 KV row-slots per query group
+  size_t runs;     // [H, Cqt, kmax + 1] int2 merged kept key runs (start, length)
+  size_t nruns;    // [H, Cqt] int32
   // stage 4
   size_t probe_q;  // [H, M, d] bf16 gathered probe rows (group-major)
   size_t od;       // [H, M, d] f32 dense outputs of the probes
@@ -79,13 +79,14 @@ struct Layout {
   size_t bv32;     // [H, d] f32 projected b'
   size_t pwork;    // [H, M/128 + 1] int32 probe attention work list
   size_t pnwork;   // [H] int32
-  size_t pmeta;    // [H, 10] int32: dense-mode off_q(2), off_k(2), csr(1), k(1), nslots(1),
-                   // nruns(1), runs(2)
+  size_t pmeta;    // [H, 12] int32: dense-mode off_q(2), off_k(2), csr(1), k(1), nslots(1),
+                   // nruns(1), runs(2 int2: run-list stride kmax + 1 = 2)
   size_t opart;    // [H, punits, kMaxSplits, 256, d] f32 split-KV partial outputs (probes)
   size_t lpart;    // [H, punits, kMaxSplits, 256] f32 split-KV log2-sum-exps
   size_t total;
 
   int Nv, e, Cmax, nchunk, tiles_per_head, kmax;
+  int Ckt, Cqt;    // groups including the text group (n_text > 0: Ck + 1, Cq + 1)
   int Dpk, CpadK, CpadQ;
   size_t scores_bytes;
   int punits;
@@ -110,9 +111,12 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   const size_t e = p.n_eig, Ck = p.Ck, Cq = p.Cq, M = p.M;
   L->Nv = Nv;
   L->e = p.n_eig;
-  L->Cmax = (p.Ck > p.Cq ? p.Ck : p.Cq);
-  L->nchunk = (Nv + kSortChunk - 1) / kSortChunk;
-  L->tiles_per_head = (p.N + kTileM - 1) / kTileM + p.Cq;
+  const int text = p.n_text > 0 ? 1 : 0;
+  L->Ckt = p.Ck + text;
+  L->Cqt = p.Cq + text;
+  L->Cmax = (L->Ckt > L->Cqt ? L->Ckt : L->Cqt);
+  L->nchunk = (p.N + kSortChunk - 1) / kSortChunk;
+  L->tiles_per_head = (p.N + kTileM - 1) / kTileM + L->Cqt;
   int kmax = 1;
   if (p.keep)
     for (int h = 0; h < p.H; ++h) {
@@ -176,9 +180,9 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->bf16_qkv = take(3 * H * N * d * 2);
   L->work = take(H * static_cast<size_t>(L->tiles_per_head) * 4);
   L->nwork = take(H * 4);
-  L->nslots = take(H * Cq * 4);
-  L->runs = take(H * Cq * static_cast<size_t>(kmax) * 8);
-  L->nruns = take(H * Cq * 4);
+  L->nslots = take(H * static_cast<size_t>(L->Cqt) * 4);
+  L->runs = take(H * static_cast<size_t>(L->Cqt) * (kmax + 1) * 8);
+  L->nruns = take(H * static_cast<size_t>(L->Cqt) * 4);
   L->probe_q = take(H * (M + kTileM) * d * 2);
   L->od = take(H * (M + 1) * d * 4);
   L->xr = take(H * 2 * (M + 1) * d * 8);
@@ -190,7 +194,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->bv32 = take(H * d * 4);
   L->pwork = take(H * (M / kTileM + 2) * 4);
   L->pnwork = take(H * 4);
-  L->pmeta = take(H * 10 * 4);
+  L->pmeta = take(H * 12 * 4);
   L->punits = static_cast<int>(M / 256 + 1);
   L->opart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * d * 4);
   L->lpart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * 4);

@@ -93,9 +93,9 @@ extern "C" sparsepr_status sparsepr_route_noalloc(const void* qp, const void* kp
     const size_t head_elems = static_cast<size_t>(N) * d;
     const char* qh = static_cast<const char*>(qp) + h0 * head_elems * eb;
     const char* kh0 = static_cast<const char*>(kp) + h0 * head_elems * eb;
-    if (launch_range_mean(qh, kind, hc, N, d, off_q + static_cast<size_t>(h0) * (Cq + 1), Cq, cq,
+    if (launch_range_mean(qh, kind, hc, N, d, off_q + static_cast<size_t>(h0) * (Cq + 1), Cq, Cq + 1, cq,
                           st) != cudaSuccess ||
-        launch_range_mean(kh0, kind, hc, N, d, off_k + static_cast<size_t>(h0) * (Ck + 1), Ck,
+        launch_range_mean(kh0, kind, hc, N, d, off_k + static_cast<size_t>(h0) * (Ck + 1), Ck, Ck + 1,
                           ckr, st) != cudaSuccess ||
         launch_route(cq, ckr, hc, Cq, Ck, d, scale, k_per_head + h0, kmax,
                      csr + static_cast<size_t>(h0) * Cq * kmax, st) != cudaSuccess)

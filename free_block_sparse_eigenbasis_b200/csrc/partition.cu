@@ -190,12 +190,14 @@ __global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int
   const int nq = (e + 3) / 4;                       // column quads
   const int pairs = (kZRows / 2) * nq;              // (row pair, quad) items
   for (int item = threadIdx.x; item < pairs; item += blockDim.x) {
+    // rows rp and rp + kZRows / 2: consecutive threads read consecutive
+    // (padded) rows, so the shared loads of k do not conflict
     const int rp = item % (kZRows / 2), qd = item / (kZRows / 2);
-    const int r0 = 2 * rp, c0 = 4 * qd;
+    const int r0 = rp, r1 = rp + kZRows / 2, c0 = 4 * qd;
     const int nc = min(4, e - c0);
     double acc0[4] = {0.0, 0.0, 0.0, 0.0}, acc1[4] = {0.0, 0.0, 0.0, 0.0};
     const double* k0 = ks + r0 * (d + 1);
-    const double* k1 = k0 + (d + 1);
+    const double* k1 = ks + r1 * (d + 1);
     if (nc == 4 && (e % 2) == 0) {
       for (int a = 0; a < d; ++a) {
         const double x0 = k0[a], x1 = k1[a];
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int
     for (int c = 0; c < 4; ++c) {
       if (c >= nc) continue;
       if (j0 + r0 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r0) * e + c0 + c] = acc0[c];
-      if (j0 + r0 + 1 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r0 + 1) * e + c0 + c] = acc1[c];
+      if (j0 + r1 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r1) * e + c0 + c] = acc1[c];
     }
   }
 }

@@ -318,9 +318,9 @@ cudaError_t launch_route_gemm(const double* cq, const double* ckr, int H, int Cq
 }
 
 cudaError_t launch_range_mean(const void* X, int x_kind, int H, int N, int d, const int32_t* off,
-                              int C, double* out, cudaStream_t st) {
-  return launch_group_mean(X, x_kind, static_cast<long long>(N) * d, d, d, nullptr, 0, off, C + 1,
-                           C, H, false, out, nullptr, nullptr, 0, st);
+                              int C, int off_stride, double* out, cudaStream_t st) {
+  return launch_group_mean(X, x_kind, static_cast<long long>(N) * d, d, d, nullptr, 0, off,
+                           off_stride, C, H, false, out, nullptr, nullptr, 0, st);
 }
 
 cudaError_t launch_write_k(const int32_t* kh_host_vals, int H, int32_t* k_per_head,

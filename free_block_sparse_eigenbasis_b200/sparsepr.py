@@ -233,6 +233,7 @@ class Buffers:
 def allocate(p: dict, dtype: torch.dtype, device="cuda", with_fit=False) -> Buffers:
     H, N, d = int(p["H"]), int(p["N"]), int(p["d"])
     Ck, Cq, M = int(p["Ck"]), int(p["Cq"]), int(p["M"])
+    text = 1 if int(p.get("n_text", 0)) > 0 else 0  # text tokens form one extra group per side
     wsb = workspace_bytes(p)
     if wsb == 0:
         raise SparsePRError(ERR_INVALID_ARG, "workspace_bytes")
@@ -242,7 +243,7 @@ def allocate(p: dict, dtype: torch.dtype, device="cuda", with_fit=False) -> Buff
         ws=torch.empty(wsb, dtype=torch.uint8, device=device),
         label_q=torch.empty((H, N), **i32), label_k=torch.empty((H, N), **i32),
         perm_q=torch.empty((H, N), **i32), perm_k=torch.empty((H, N), **i32),
-        off_q=torch.empty((H, Cq + 1), **i32), off_k=torch.empty((H, Ck + 1), **i32),
+        off_q=torch.empty((H, Cq + text + 1), **i32), off_k=torch.empty((H, Ck + text + 1), **i32),
         qp=torch.empty((H, N, d), dtype=dtype, device=device),
         kp=torch.empty((H, N, d), dtype=dtype, device=device),
         vp=torch.empty((H, N, d), dtype=dtype, device=device),

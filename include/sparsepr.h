@@ -37,8 +37,14 @@
  *     out) are OR-ed into the status word in `ws`; read it after the stream
  *     has been synchronised.
  *   - Supported: d in {64, 128}; dtype bf16 or fp32 (the attention MMAs run
- *     in bf16 with fp32 accumulation for both); 1 <= H <= SPARSEPR_MAX_HEADS;
- *     n_text = 0.
+ *     in bf16 with fp32 accumulation for both); 1 <= H <= SPARSEPR_MAX_HEADS.
+ *   - Text tokens (n_text > 0, the trailing tokens of every head; the
+ *     HunyuanVideo-shaped joint attention): they take part in neither
+ *     k-means nor the sampled queries; they form one extra key group (index
+ *     Ck) that every query group keeps outside its budget, and one extra
+ *     query group (index Cq) that keeps every key; text rows are never probes
+ *     and are not corrected. With text tokens the group counts below are
+ *     Ckt = Ck + 1 and Cqt = Cq + 1, otherwise Ckt = Ck and Cqt = Cq.
  */
 #ifndef SPARSEPR_H_
 #define SPARSEPR_H_
@@ -70,7 +76,7 @@ typedef struct {
   int32_t H;            /* heads, 1..SPARSEPR_MAX_HEADS */
   int32_t N;            /* tokens per head (video tokens + n_text) */
   int32_t d;            /* head dim: 64 or 128 */
-  int32_t n_text;       /* trailing always-kept text tokens; must be 0 */
+  int32_t n_text;       /* trailing text tokens (0 <= n_text < N) */
   int32_t Ck;           /* key (K/V) groups, 1..min(Nv, 4096) */
   int32_t Cq;           /* query groups, 1..min(Nv, 4096) */
   int32_t Ms;           /* sampled queries for M_K, 1..Nv */
@@ -116,8 +122,9 @@ const char* sparsepr_status_string(sparsepr_status s);
  * Initial centroids: rows chosen by a partial Fisher-Yates shuffle driven by
  * SplitMix64 seeded with seed ^ (2*head + {0 keys, 1 queries}).
  *   q, k      [H, N, d] input dtype (device, read only)
- *   label_q   [H, N] int32 out: query group of each token, 0..Cq-1
- *   label_k   [H, N] int32 out: key group of each token, 0..Ck-1 */
+ *   label_q   [H, N] int32 out: query group of each token, 0..Cqt-1
+ *   label_k   [H, N] int32 out: key group of each token, 0..Ckt-1
+ *             (text tokens: Cq and Ck) */
 sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype dt,
                                    const sparsepr_params* p, int32_t* label_q,
                                    int32_t* label_k, void* ws, size_t ws_bytes,
@@ -128,9 +135,9 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
  * group-major row i (ascending token order inside a group); off[h, c] is
  * the first row of group c (off[h, C] = N). qp = q[perm_q], kp = k[perm_k],
  * vp = v[perm_k] (K and V share the key partition).
- *   label_q, label_k   [H, N] int32 in (values must lie in 0..Cq-1 / 0..Ck-1)
+ *   label_q, label_k   [H, N] int32 in (values must lie in 0..Cqt-1 / 0..Ckt-1)
  *   perm_q, perm_k     [H, N] int32 out
- *   off_q [H, Cq+1], off_k [H, Ck+1] int32 out
+ *   off_q [H, Cqt+1], off_k [H, Ckt+1] int32 out
  *   qp, kp, vp         [H, N, d] input dtype out (must not alias q, k, v) */
 sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v,
                                  sparsepr_dtype dt, const sparsepr_params* p,
@@ -142,7 +149,9 @@ sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v,
 /* Stage 3a [SVOO block selection].
  * Block scores A[g, c] = scale * C_Q[g] . C_K[c] in fp64 from the group mean
  * rows of qp / kp (zero vector for an empty group); each query group keeps
- * its top-k_h key groups, ties to the lowest index, listed ascending.
+ * its top-k_h key groups, ties to the lowest index, listed ascending. Only
+ * the Cq x Ck video groups are routed (off_q, off_k as from sparsepr_permute,
+ * Cqt + 1 / Ckt + 1 entries per head).
  * k_h = max(1, min(Ck, ceil(keep[h] * Ck - 1e-9))).
  *   csr         [H, Cq, kmax] int32 out, kmax = max_h k_h; entries past
  *               k_h are -1
@@ -172,7 +181,8 @@ int32_t sparsepr_route_width(const sparsepr_params* p);
  * that device current; make that first call before any stream capture.
  * All calls share the array and the last call's contents stay in it (every
  * call overwrites what it reads, nothing needs clearing). Calls that overlap
- * on the GPU race on the array: issue them in order on one stream. */
+ * on the GPU race on the array: issue them in order on one stream.
+ * Parameters with text tokens (n_text > 0) return SPARSEPR_ERR_UNSUPPORTED. */
 sparsepr_status sparsepr_route_noalloc(const void* qp, const void* kp, sparsepr_dtype dt,
                                        const sparsepr_params* p, const int32_t* off_q,
                                        const int32_t* off_k, int32_t* csr,
@@ -183,8 +193,9 @@ sparsepr_status sparsepr_route_noalloc(const void* qp, const void* kp, sparsepr_
  * For group-major query row i of group g:
  *   o_sparse[i] = sum_{j in S(g)} softmax_{S(g)}(scale * qp_i . kp_j) vp_j,
  * S(g) = union of the key ranges off_k[c]..off_k[c+1] of the kept groups c
- * in csr[g]. Skipped key groups are never multiplied. bf16 tensor-core MMAs
- * (tcgen05, fp32 accumulation in tensor memory).
+ * in csr[g] (plus the text key group when n_text > 0; the text query group
+ * keeps every key). Skipped key groups are never multiplied. bf16
+ * tensor-core MMAs (tcgen05, fp32 accumulation in tensor memory).
  *   o_sparse      [H, N, d] fp32 out, group-major row order
  *   pairs_sparse  [H] int64 out: sum_g n_g * |S(g)| (exact pair count)
  * A query group whose kept set is empty raises SPARSEPR_ERR_NUMERIC in the
@@ -204,8 +215,9 @@ sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const
  * Ridge fit (fp64, intercept unpenalised): B = (Xc^T Xc + lambda I)^{-1}
  * Xc^T Rc, b = rbar - xbar B with X = O_sparse[probes]. Subspace: V_r = top-r
  * right singular vectors of R; B' = B V_r V_r^T, b' = b V_r V_r^T.
- * Output: out[perm_q[i]] = O_dense(i) for probe rows, else
- * o_sparse[i] + b' + o_sparse[i] B', rounded to the input dtype (RNE).
+ * Output: out[perm_q[i]] = O_dense(i) for probe rows, o_sparse[i] for text
+ * rows, else o_sparse[i] + b' + o_sparse[i] B', rounded to the input dtype
+ * (RNE). Probes are drawn from the Cq video query groups only.
  *   perm_q         [H, N] int32 in (from sparsepr_permute)
  *   o_sparse       [H, N, d] fp32 in (from sparsepr_block_sparse_attn)
  *   pairs_sparse   [H] int64 in

@@ -58,7 +58,8 @@ def test_keep_budget_matches_oracle_on_edge_values():
 @pytest.mark.parametrize("bad", [
     dict(d=96), dict(H=0), dict(H=300), dict(Ck=0), dict(Cq=5000), dict(Ms=0),
     dict(n_eig=0), dict(n_eig=40), dict(M=-1), dict(r=0), dict(r=65), dict(lam=-1.0),
-    dict(keep=[0.0]), dict(keep=[1.5]), dict(n_text=8), dict(kmeans_iters=0), dict(N=8),
+    dict(keep=[0.0]), dict(keep=[1.5]), dict(n_text=-1), dict(n_text=256), dict(kmeans_iters=0),
+    dict(N=8),
 ])
 def test_invalid_params_rejected_on_host(bad):
     p = dict(synth.workload("tiny").params(), **bad)
@@ -68,6 +69,13 @@ def test_invalid_params_rejected_on_host(bad):
     code = S.lib.sparsepr_partition(fake, fake, S.BF16, ctypes.byref(prm), fake, fake, fake,
                                     1 << 30, None)
     assert code in (S.ERR_INVALID_ARG, S.ERR_UNSUPPORTED)
+
+
+def test_text_tokens_accepted_and_sized():
+    # trailing text tokens add one key group and one query group per head
+    p = dict(synth.workload("tiny").params(), n_text=8)
+    assert S.workspace_bytes(p) > 0
+    assert S.route_width(p) == S.route_width(dict(p, n_text=0))  # routes cover video groups
 
 
 def test_null_pointers_and_small_workspace_rejected():

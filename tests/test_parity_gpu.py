@@ -49,6 +49,12 @@ SMALL = [
     # one key group kept, no probes (hard-drop: output = sparse output)
     synth.custom("hard_drop", 1, (2, 8, 16), 128, "bf16", Ck=16, Cq=4, Ms=64, n_eig=4, M=0,
                  r=8, keep=0.05, seed=4),
+    # trailing text tokens: an always-kept key group and a dense query group,
+    # never probed or corrected (HunyuanVideo-shaped joint attention)
+    synth.custom("text_bf16_d128", 2, (3, 8, 16), 128, "bf16", n_text=40, Ck=24, Cq=6, Ms=128,
+                 n_eig=8, M=32, r=8, keep=(0.2, 0.3), seed=21),
+    synth.custom("text_f32_d64_hard_drop", 1, (2, 5, 13), 64, "f32", n_text=9, Ck=10, Cq=4,
+                 Ms=64, n_eig=4, M=0, r=4, keep=0.25, seed=22),
 ]
 
 
