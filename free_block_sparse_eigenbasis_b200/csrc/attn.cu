@@ -11,7 +11,7 @@
 // Rows of a slot past its run's end are masked to -inf, so skipped key groups
 // are never multiplied (only the tail padding of a run is).
 //
-// Roles (320 threads): two softmax warpgroups (warps 0-3 and 4-7, thread =
+// Roles (352 threads): two softmax warpgroups (warps 0-3 and 4-7, thread =
 // query row = TMEM lane) each own one TMEM slot (S_i, O_i, with P_i written
 // as packed bf16 over the first 64 columns of S_i); warp 8 lane 0 streams Q,
 // K and V with TMA; warp 9 lane 0 issues tcgen05.mma.
@@ -37,7 +37,7 @@ namespace {
 constexpr int kStages = 2;                         // K and V ring depth
 constexpr int kSlotsPerTile = kTileN / kSlotRows;  // 16
 constexpr int kUnitRows = 2 * kTileM;              // query rows per CTA
-constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr int kAttnThreads = 352;  // 8 softmax warps, K TMA warp (8), MMA warp (9), V TMA warp (10)
 constexpr uint32_t kTmemCols = 512;  // S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 after
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -238,13 +238,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
 
-  if (warp == 8) {
-    // ------- TMA producer warp: Q once, then K(j) and V(j) in order. Lane s
-    // (and s + 16) finds the first row of slot s of the tile; a tile whose
-    // slots are all contiguous is fetched as one 128-row box, any other
-    // tile slot by slot (8-row boxes, lanes 0-15 in parallel). -------
+  if (warp == 8 || warp == 10) {
+    // ------- TMA producers: warp 8 streams Q once and the K tiles, warp 10
+    // the V tiles, each through its own ring. Lane s (and s + 16) finds the
+    // first row of slot s of a tile; a tile whose slots are all contiguous is
+    // fetched as one 128-row box, any other tile slot by slot (8-row boxes,
+    // lanes 0-15 in parallel). -------
+    const bool is_k = (warp == 8);
     const int krow_base = h * p.N;
-    if (lane == 0) {
+    if (is_k && lane == 0) {
       mbar_arrive_expect_tx(&bars->q_full, nq * kAtoms * p.q_box_rows * 128);
       for (int qt = 0; qt < nq; ++qt)
         for (int a = 0; a < kAtoms; ++a)
@@ -262,7 +264,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ++rb;
       }
     }
-    int k_issued = -1, v_issued = -1;
+    uint8_t* ring = is_k ? Ks : Vs;
+    uint64_t* full = is_k ? bars->kfull : bars->vfull;
+    uint64_t* empty = is_k ? bars->kempty : bars->vempty;
+    const CUtensorMap* map_slot = is_k ? &maps.k[0] : &maps.v[0];
+    const CUtensorMap* map_tile = is_k ? &maps.k[4] : &maps.v[4];
+    int issued = -1;
     const bool big_box = p.max_lg == 4;  // the tensor holds at least one 128-row box
     for (int j = 0; j < T; ++j) {
       const int t = (j0 + j) * kSlotsPerTile + sl;
@@ -280,48 +287,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool whole = big_box && __all_sync(0xffffffffu, follows);
       const int row_first = __shfl_sync(0xffffffffu, row, 0);
       const int st = j % kStages;
-      const uint32_t ph = ((j / kStages) + 1) & 1;
       bool w = true;
-      if (lane == 0 && j >= kStages) w = mbar_wait(&bars->kempty[st], ph, abort);
+      if (lane == 0 && j >= kStages) w = mbar_wait(&empty[st], ((j / kStages) + 1) & 1, abort);
       if (!__shfl_sync(0xffffffffu, w, 0)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&bars->kfull[st], L::kKVBytes);
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], L::kKVBytes);
       __syncwarp();
       if (whole) {
         if (lane == 0)
           for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(Ks + st * L::kKVBytes + a * L::kSlab, &maps.k[4], &bars->kfull[st], a * 64,
+            tma_load_2d(ring + st * L::kKVBytes + a * L::kSlab, map_tile, &full[st], a * 64,
                         krow_base + row_first);
       } else if (lane < kSlotsPerTile) {
         for (int a = 0; a < kAtoms; ++a)
-          tma_load_2d(Ks + st * L::kKVBytes + a * L::kSlab + sl * 1024, &maps.k[0],
-                      &bars->kfull[st], a * 64, krow_base + row);
+          tma_load_2d(ring + st * L::kKVBytes + a * L::kSlab + sl * 1024, map_slot, &full[st],
+                      a * 64, krow_base + row);
       }
-      k_issued = j;
-      w = true;
-      if (lane == 0 && j >= kStages) w = mbar_wait(&bars->vempty[st], ph, abort);
-      if (!__shfl_sync(0xffffffffu, w, 0)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&bars->vfull[st], L::kKVBytes);
-      __syncwarp();
-      if (whole) {
-        if (lane == 0)
-          for (int a = 0; a < kAtoms; ++a)
-            tma_load_2d(Vs + st * L::kKVBytes + a * L::kSlab, &maps.v[4], &bars->vfull[st], a * 64,
-                        krow_base + row_first);
-      } else if (lane < kSlotsPerTile) {
-        for (int a = 0; a < kAtoms; ++a)
-          tma_load_2d(Vs + st * L::kKVBytes + a * L::kSlab + sl * 1024, &maps.v[0],
-                      &bars->vfull[st], a * 64, krow_base + row);
-      }
-      v_issued = j;
+      issued = j;
     }
     // let the loads already in flight land before the CTA exits
     if (lane == 0) {
       volatile int never = 0;
-      for (int j = max(0, k_issued - kStages + 1); j <= k_issued; ++j)
-        mbar_wait(&bars->kfull[j % kStages], (j / kStages) & 1, &never);
-      for (int j = max(0, v_issued - kStages + 1); j <= v_issued; ++j)
-        mbar_wait(&bars->vfull[j % kStages], (j / kStages) & 1, &never);
-      mbar_wait(&bars->q_full, 0, &never);
+      for (int j = max(0, issued - kStages + 1); j <= issued; ++j)
+        mbar_wait(&full[j % kStages], (j / kStages) & 1, &never);
+      if (is_k) mbar_wait(&bars->q_full, 0, &never);
     }
   } else if (warp == 9) {
     // ------------------------------ MMA issuer --------------------------------
