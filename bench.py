@@ -47,6 +47,25 @@ def workload_desc(w):
                statistics.mean(w.keep), w.M, w.r, w.lam, w.kmeans_iters))
 
 
+# DRAM traffic of the routed attention launch on the 720p workload from one ncu
+# capture (profiles/sparse_attn_kernel_wan13b_720p_traffic.md), valid for the
+# attention source it was taken on.
+ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=722669312 + 448694016,
+                    source_sha256_prefix="0de883bc14ce4ada")
+
+
+def attn_traffic(w):
+    import hashlib
+    src = os.path.join(ROOT, "free_block_sparse_eigenbasis_b200", "csrc", "attn.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if w.name != ATTN_TRAFFIC["workload"] or h != ATTN_TRAFFIC["source_sha256_prefix"]:
+        return None
+    return ATTN_TRAFFIC["bytes"]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -128,12 +147,12 @@ def gpu_launches_per_call(w) -> int:
     the fallback when the profiler count is unavailable)."""
     it = w.kmeans_iters
     partition = (11                    # reset, Fisher-Yates, M_K, eigen (2), scaling, z, inits, planes
-                 + 6 * it + 4 * (it - 1)  # key passes (2 zero, centroid planes, argmin, recheck,
-                                          # finalize) and centroid updates (sort + mean)
-                 + 5                      # final key sort, C_K, G
-                 + 7 * it + 4 * (it - 1)  # query passes (+ metric apply) and updates
+                 + 6 * it + 5 * (it - 1)  # key passes (2 zero, centroid planes, argmin, recheck,
+                                          # finalize) and centroid updates (4-kernel sort + mean)
+                 + 6                      # final key sort, C_K, G
+                 + 7 * it + 5 * (it - 1)  # query passes (+ metric apply) and updates
                  + 2)                     # labels out
-    permute = 2 * 3 + 3
+    permute = 2 * 4 + 3
     route = 5
     attn = 5
     probe = 18 if w.M > 0 else 5
@@ -368,7 +387,8 @@ def main():
             roofline=dict(bound="tensor", kernel="sparse_attn_kernel<128>",
                           achieved=attn_tflops, peak=peak, unit="TFLOP/s",
                           frac=attn_tflops / peak, peak_source="bf16_tflops (burst) of " + src,
-                          traffic=None,
+                          traffic=attn_traffic(w),
+                          traffic_unit="bytes per launch (dram read + write, ncu)",
                           note="achieved = 4 d P_sparse / duration of the block-sparse "
                                "attention call (CUDA events on its stream)"),
             clocks=clocks,

@@ -289,7 +289,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     ak.x_hs = hs_z;
     ak.x_ld = e;
     ak.D = e;
-    ak.y_exact = mu;
+    ak.y_tr = at<double>(ws, L.ytr);
     ak.c_exact = mun;
     ak.m = Ck;
     ak.direct = 1;
@@ -299,7 +299,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
       SPR_TRY(launch_prep_centroids(mu, mun, Ck, e, L.Dpk, L.CpadK, 3, H,
                                     at<__nv_bfloat16>(ws, L.muplanes),
                                     static_cast<long long>(H) * L.CpadK * L.Dpk,
-                                    at<float>(ws, L.cfk), at<float>(ws, L.hmk), flags, 0, st));
+                                    at<float>(ws, L.cfk), at<float>(ws, L.hmk),
+                                    at<double>(ws, L.ytr), flags, 0, st));
       SPR_TRY(launch_argmin_tc(ak, st));
     } else {
       SPR_TRY(launch_argmin(z, kXf64, hs_z, e, Nv, e, mu, mun, Ck, H, lab_k, flags, 0, st));
@@ -355,7 +356,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     aq.x_hs = hs_in;
     aq.x_ld = d;
     aq.D = d;
-    aq.y_exact = wg;
+    aq.y_tr = at<double>(ws, L.ytr);
     aq.c_exact = cg;
     aq.m = Cq;
     aq.direct = 0;
@@ -366,7 +367,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
       SPR_TRY(launch_prep_centroids(wg, cg, Cq, d, d, L.CpadQ, nbq, H,
                                     at<__nv_bfloat16>(ws, L.wplanes),
                                     static_cast<long long>(H) * L.CpadQ * d, at<float>(ws, L.cfq),
-                                    at<float>(ws, L.hmq), flags, 2, st));
+                                    at<float>(ws, L.hmq), at<double>(ws, L.ytr), flags, 2, st));
       SPR_TRY(launch_argmin_tc(aq, st));
     } else {
       SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, st));

@@ -14,9 +14,12 @@
 //   |d'_ij - d_ij| <= E_i = (K_t 2^-22 + 2^-20) |x_i| Y + 2^-22 (C + 2 |x_i| Y),
 // Y = max_j |y_j|, C = max_j |c_j| (a generous bound: products of bf16 values
 // are exact in fp32, each accumulation step loses at most 2^-23 relative).
-// A row whose best and second-best d' differ by more than 2 E_i has a
-// certain label; every other row is appended to a list and decided again in
-// fp64 by recheck_kernel.
+// The epilogue reduces values whose three low mantissa bits are replaced by
+// the column's position within its piece (at most 7 ulp, < 2^-20 |d'|), so
+// the bound it uses adds 2^-20 (C + 2 |x_i| Y). A row whose best and
+// second-best packed d' differ by more than 2 E_i has a certain label; every
+// other row is appended to a list and decided again in fp64 by
+// recheck_kernel.
 //
 // Persistent CTAs (at most one per SM) each take a contiguous range of the
 // row tiles of all heads, ordered head-major; the centroid planes of the
@@ -26,8 +29,10 @@
 // TMEM buffers, so the epilogue of one chunk overlaps the MMAs of the next.
 // The epilogue is four groups of four warps: every group sees all 128 rows
 // (warp w reads TMEM lanes 32 (w % 4) ..) and a quarter of each chunk's
-// columns; the groups' partial minima meet in shared memory at the end of a
-// tile.
+// columns; each thread keeps four chains (columns k mod 4) of best, second
+// best and the piece of the best, takes two columns of a chain per step
+// (min / max of the pair, then a three-input min for the second best), and
+// the groups' partial results meet in shared memory at the end of a tile.
 #include "common.cuh"
 #include "internal.h"
 
@@ -105,13 +110,25 @@ __device__ __forceinline__ void for_segments(const AsParams& p, int g, int g1, F
   }
 }
 
-// running best / second best of one chain; columns of a chain ascend, so
-// equal values keep the lower index
-__device__ __forceinline__ void chain_step(float dd, int j, float& b1, float& b2, int& bi) {
-  const bool lt = dd < b1;
-  b2 = fminf(b2, fmaxf(b1, dd));
-  bi = lt ? j : bi;
-  b1 = fminf(b1, dd);
+// value with its position (0..7) within a chain piece in the low three
+// mantissa bits: changes the value by at most 7 ulp, and the minimum of
+// packed values carries the position of its column
+__device__ __forceinline__ float pack_pos(float v, int pos) {
+  return __uint_as_float((__float_as_uint(v) & ~7u) | static_cast<uint32_t>(pos));
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// orders later reads of the registers after the preceding tcgen05.wait::ld
+__device__ __forceinline__ void reg_fence32(uint32_t (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 8)
+    asm volatile("" : "+r"(v[i]), "+r"(v[i + 1]), "+r"(v[i + 2]), "+r"(v[i + 3]), "+r"(v[i + 4]),
+                 "+r"(v[i + 5]), "+r"(v[i + 6]), "+r"(v[i + 7]));
 }
 
 __global__ void __launch_bounds__(kAsThreads, 1)
@@ -244,74 +261,96 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     // ------------------- epilogue: group q, row r of the tile -------------------
     // Every epilogue thread passes the same sequence of named barriers, also
     // after a failed wait (it then skips the work), so none is left behind.
-    const int q = warp >> 2;
+    // Group q reads its columns of a chunk in pieces of at most 32.
+    const int q = warp / 4;
     const int r = (warp & 3) * 32 + lane;
     const int et = threadIdx.x;  // 0 .. kAsEpi - 1
     const uint32_t lane_base = static_cast<uint32_t>(((warp & 3) * 32) << 16);
+    // E bound: MMA terms, fp32 offsets and rounding, and the index bits
+    // packed into the low three mantissa bits of each value (<= 7 ulp)
     const float kt_term = static_cast<float>(p.Kt) * 2.384185791015625e-07f + p.res;
     int gc = 0, nx = 0;
     bool ok = true;
+    uint32_t va[32];
     for_segments(p, g0, g1, [&](int h, int t0, int t1) {
       named_barrier_sync(kBarHead, kAsEpi);  // the previous head's offsets are no longer read
       for (int j = et; j < p.Cpad; j += kAsEpi) cs[j] = p.cvals[static_cast<size_t>(h) * p.Cpad + j];
       named_barrier_sync(kBarHead, kAsEpi);
       const float Y = p.hmax[h * 2 + 0], C = p.hmax[h * 2 + 1];
       int32_t* fl = p.flags + h * 4;
-      for (int t = t0; t < t1; ++t) {
-        float b1[4], b2[4];
-        int bi[4];
+      float b1[4], b2[4];
+      int blk[4];
+      // reduce one piece of w (16 or 32) columns starting at column jb:
+      // values packed with their position within the chain, then a pair at
+      // a time into the chain's best and second best
+      auto reduce = [&](const uint32_t (&v)[32], int w, int jb) {
+        const float4* c4 = reinterpret_cast<const float4*>(cs + jb);
+        const float ob[4] = {b1[0], b1[1], b1[2], b1[3]};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          b1[k] = INFINITY;
-          b2[k] = INFINITY;
-          bi[k] = 0x7fffffff;
-        }
-        for (int c = 0; c < nchunks; ++c, ++gc) {
-          const int buf = gc & 1;
-          ok = ok && mbar_wait(&bars->acc_full[buf], (gc >> 1) & 1, abort);
-          ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
-          if (ok) {
-            tc_fence_after();
-            const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
-            const int nb = N >> 4;  // 16-column blocks of the chunk
-            const int c0 = 16 * ((q * nb) / kAsGroups), c1 = 16 * (((q + 1) * nb) / kAsGroups);
-            const uint32_t base = tmem + lane_base + static_cast<uint32_t>(buf * kAsChunk);
-            for (int col = c0; col < c1; col += 32) {
-              uint32_t v[32];
-              const bool full = (c1 - col >= 32);  // warp-uniform
-              if (full)
-                tmem_ld32(base + col, v);
-              else
-                tmem_ld16(base + col, *reinterpret_cast<uint32_t(*)[16]>(v));
-              tmem_wait_ld();
-              const int j0 = c * kAsChunk + col;
-              const float4* c4 = reinterpret_cast<const float4*>(cs + j0);
+        for (int pr = 0; pr < 4; ++pr) {
+          if (pr < 2 || w >= 32) {
+            const float4 ca = c4[2 * pr], cb = c4[2 * pr + 1];
+            const float ea[4] = {ca.x, ca.y, ca.z, ca.w}, eb[4] = {cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
-                if (i4 < 4 || full) {
-                  const float4 cc = c4[i4];
-                  const int j = j0 + 4 * i4;
-                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 0]), cc.x), j + 0, b1[0], b2[0], bi[0]);
-                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 1]), cc.y), j + 1, b1[1], b2[1], bi[1]);
-                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 2]), cc.z), j + 2, b1[2], b2[2], bi[2]);
-                  chain_step(fmaf(-2.f, __uint_as_float(v[4 * i4 + 3]), cc.w), j + 3, b1[3], b2[3], bi[3]);
-                }
-              }
+            for (int k = 0; k < 4; ++k) {
+              const float x = pack_pos(fmaf(-2.f, __uint_as_float(v[8 * pr + k]), ea[k]), 2 * pr);
+              const float y = pack_pos(fmaf(-2.f, __uint_as_float(v[8 * pr + 4 + k]), eb[k]), 2 * pr + 1);
+              const float m = fminf(x, y), M = fmaxf(x, y);
+              b2[k] = min3f(b2[k], fmaxf(b1[k], m), M);
+              b1[k] = fminf(b1[k], m);
             }
           }
-          tc_fence_before();
-          mbar_arrive(&bars->acc_empty[buf]);
         }
-        // merge the chains: best by (value, index), second = smallest of the
-        // chains' seconds and the other chains' bests
+#pragma unroll
+        for (int k = 0; k < 4; ++k) blk[k] = (b1[k] < ob[k]) ? jb : blk[k];
+      };
+      const int U = (t1 - t0) * nchunks;  // (tile, chunk) steps of this head
+      for (int u = 0; u < U; ++u) {
+        const int c = u % nchunks;
+        const int t = t0 + u / nchunks;
+        if (c == 0) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            b1[k] = INFINITY;
+            b2[k] = INFINITY;
+            blk[k] = 0;
+          }
+        }
+        ok = ok && mbar_wait(&bars->acc_full[gc & 1], (gc >> 1) & 1, abort);
+        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+        tc_fence_after();
+        // this group's columns [a0, a1) of chunk c
+        const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
+        const int nb = N >> 4;
+        const int a0 = 16 * ((q * nb) / kAsGroups), a1 = 16 * (((q + 1) * nb) / kAsGroups);
+        const uint32_t base = tmem + lane_base + static_cast<uint32_t>((gc & 1) * kAsChunk);
+        for (int col = a0; col < a1; col += 32) {
+          const int w = min(32, a1 - col);  // warp-uniform
+          if (ok) {
+            if (w >= 32)
+              tmem_ld32(base + col, va);
+            else
+              tmem_ld16(base + col, *reinterpret_cast<uint32_t(*)[16]>(va));
+          }
+          tmem_wait_ld();
+          reg_fence32(va);
+          if (ok) reduce(va, w, c * kAsChunk + col);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->acc_empty[gc & 1]);
+        ++gc;
+        if (c + 1 < nchunks) continue;
+        // ---- end of tile t: merge the chains, then the groups ----
+        // a chain's best sits at column blk + 4 * (packed position) + k
         float d1 = b1[0], d2 = b2[0];
-        int i1 = bi[0];
+        int i1 = blk[0] + 4 * static_cast<int>(__float_as_uint(b1[0]) & 7u);
 #pragma unroll
         for (int k = 1; k < 4; ++k) {
-          if (b1[k] < d1 || (b1[k] == d1 && bi[k] < i1)) {
+          const int ik = blk[k] + 4 * static_cast<int>(__float_as_uint(b1[k]) & 7u) + k;
+          if (b1[k] < d1 || (b1[k] == d1 && ik < i1)) {
             d2 = fminf(d1, b2[k]);
             d1 = b1[k];
-            i1 = bi[k];
+            i1 = ik;
           } else {
             d2 = fminf(d2, b1[k]);
           }
@@ -342,7 +381,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           if (ok && row < p.n) {
             const size_t li = static_cast<size_t>(h) * p.n + row;
             const float xy = p.xnorm[li] * Y;
-            const float E = kt_term * xy + 2.384185791015625e-07f * (C + 2.f * xy);
+            const float E = kt_term * xy + 1.25e-06f * (C + 2.f * xy);
             if (d2 - d1 > 2.f * E) {
               changed = p.labels[li] != i1;
               p.labels[li] = i1;
@@ -373,14 +412,14 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// fp64 decision of the flagged rows: one block per flagged row (grid-stride).
-// Short rows (D <= 32): thread j scores centroids j, j + 256, ... reading
-// each centroid row contiguously; long rows: warp w scores centroids w,
-// w + 8, ... with its lanes over the columns (butterfly sum, identical in
-// every lane). Then a block argmin, lowest index on ties.
+// fp64 decision of the flagged rows: one block per flagged row (grid-stride
+// over the head's list). Thread j scores centroids j, j + 256, ... in
+// ascending order from the transposed centroid side yT [D, m], so the loads
+// of a warp are contiguous; four partial sums per dot product keep the fp64
+// pipes busy. Then a block argmin, lowest index on ties.
 // direct = 1: d = sum_t (x_t - y_jt)^2; else d = c_j - 2 x . y_j.
 // ---------------------------------------------------------------------------
-constexpr int kRcThreads = 256, kRcMaxD = 128;
+constexpr int kRcThreads = 256, kRcMaxD = 128, kRcBlocksPerHead = 128;
 
 __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   if (kind == kXf64) return static_cast<const double*>(X)[i];
@@ -395,11 +434,49 @@ __device__ __forceinline__ void argmin_merge(double& best, int& bi, double ob, i
   }
 }
 
+// score of centroid j: DT > 0 fixes the length at compile time
+template <int DT, bool DIRECT>
+__device__ __forceinline__ double rc_score(const double* xs, const double* yT, int m, int j, int Drt,
+                                           const double* ch) {
+  const int D = DT > 0 ? DT : Drt;
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  int t = 0;
+  constexpr int kTUnroll = (DT > 0 && DT <= 32) ? (DT / 4 > 0 ? DT / 4 : 1) : 4;  // 16 loads in flight
+#pragma unroll kTUnroll
+  for (; t + 4 <= D; t += 4) {
+    const double y0 = yT[static_cast<size_t>(t) * m + j], y1 = yT[static_cast<size_t>(t + 1) * m + j];
+    const double y2 = yT[static_cast<size_t>(t + 2) * m + j], y3 = yT[static_cast<size_t>(t + 3) * m + j];
+    if (DIRECT) {
+      const double e0 = xs[t] - y0, e1 = xs[t + 1] - y1, e2 = xs[t + 2] - y2, e3 = xs[t + 3] - y3;
+      a0 = fma(e0, e0, a0);
+      a1 = fma(e1, e1, a1);
+      a2 = fma(e2, e2, a2);
+      a3 = fma(e3, e3, a3);
+    } else {
+      a0 = fma(xs[t], y0, a0);
+      a1 = fma(xs[t + 1], y1, a1);
+      a2 = fma(xs[t + 2], y2, a2);
+      a3 = fma(xs[t + 3], y3, a3);
+    }
+  }
+  for (; t < D; ++t) {
+    const double y = yT[static_cast<size_t>(t) * m + j];
+    if (DIRECT) {
+      const double e0 = xs[t] - y;
+      a0 = fma(e0, e0, a0);
+    } else {
+      a0 = fma(xs[t], y, a0);
+    }
+  }
+  const double sm = (a0 + a1) + (a2 + a3);
+  return DIRECT ? sm : ch[j] - 2.0 * sm;
+}
+
+template <int DT, bool DIRECT>
 __global__ void __launch_bounds__(kRcThreads)
     recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
-                   const double* Y, const double* c, int m, int direct, int32_t* labels,
-                   int32_t* flags, int flag_base, const int32_t* recheck,
-                   const int32_t* nrecheck) {
+                   const double* yT, const double* c, int m, int32_t* labels, int32_t* flags,
+                   int flag_base, const int32_t* recheck, const int32_t* nrecheck) {
   __shared__ double xs[kRcMaxD];
   __shared__ double wbest[kRcThreads / 32];
   __shared__ int wbi[kRcThreads / 32];
@@ -408,8 +485,8 @@ __global__ void __launch_bounds__(kRcThreads)
   if (fl[flag_base + 1]) return;
   const int cnt = nrecheck[h];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const double* Yh = Y + static_cast<size_t>(h) * m * D;
-  const double* ch = c + static_cast<size_t>(h) * m;
+  const double* Yh = yT + static_cast<size_t>(h) * D * m;
+  const double* ch = DIRECT ? nullptr : c + static_cast<size_t>(h) * m;
   for (int k = blockIdx.x; k < cnt; k += gridDim.x) {
     const int row = recheck[static_cast<size_t>(h) * n + k];
     __syncthreads();  // xs and the warp results of the previous row are consumed
@@ -418,51 +495,18 @@ __global__ void __launch_bounds__(kRcThreads)
     __syncthreads();
     double best = INFINITY;
     int bi = 0x7fffffff;
-    if (D <= 32) {
-      for (int j = threadIdx.x; j < m; j += blockDim.x) {  // ascending within the thread
-        const double* y = Yh + static_cast<size_t>(j) * D;
-        double dd;
-        if (direct) {
-          dd = 0.0;
-          for (int t = 0; t < D; ++t) {
-            const double diff = xs[t] - y[t];
-            dd = fma(diff, diff, dd);
-          }
-        } else {
-          double sm = 0.0;
-          for (int t = 0; t < D; ++t) sm = fma(xs[t], y[t], sm);
-          dd = ch[j] - 2.0 * sm;
-        }
-        if (dd < best) {
-          best = dd;
-          bi = j;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-        argmin_merge(best, bi, __shfl_xor_sync(0xffffffffu, best, o),
-                     __shfl_xor_sync(0xffffffffu, bi, o));
-    } else {
-      for (int j = w; j < m; j += kRcThreads / 32) {  // ascending within the warp
-        const double* y = Yh + static_cast<size_t>(j) * D;
-        double part = 0.0;
-        for (int t = lane; t < D; t += 32) {
-          if (direct) {
-            const double diff = xs[t] - y[t];
-            part = fma(diff, diff, part);
-          } else {
-            part = fma(xs[t], y[t], part);
-          }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        const double dd = direct ? part : ch[j] - 2.0 * part;
-        if (dd < best) {
-          best = dd;
-          bi = j;
-        }
+    constexpr int kJUnroll = (DT > 0 && DT <= 16) ? 2 : 1;  // short rows: two centroids in flight
+#pragma unroll kJUnroll
+    for (int j = threadIdx.x; j < m; j += kRcThreads) {  // ascending within the thread
+      const double dd = rc_score<DT, DIRECT>(xs, Yh, m, j, D, ch);
+      if (dd < best) {
+        best = dd;
+        bi = j;
       }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+      argmin_merge(best, bi, __shfl_xor_sync(0xffffffffu, best, o), __shfl_xor_sync(0xffffffffu, bi, o));
     if (lane == 0) {
       wbest[w] = best;
       wbi[w] = bi;
@@ -475,6 +519,24 @@ __global__ void __launch_bounds__(kRcThreads)
       labels[li] = bi;
     }
   }
+}
+
+template <bool DIRECT>
+void launch_recheck_d(const AssignTC& a, cudaStream_t st) {
+  const dim3 grid(kRcBlocksPerHead, a.H);
+#define SPR_RC(DT)                                                                          \
+  recheck_kernel<DT, DIRECT><<<grid, kRcThreads, 0, st>>>(                                 \
+      a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D, a.y_tr, a.c_exact, a.m, a.labels, a.flags, \
+      a.flag_base, a.recheck, a.nrecheck)
+  if (a.D == 16)
+    SPR_RC(16);
+  else if (a.D == 64)
+    SPR_RC(64);
+  else if (a.D == 128)
+    SPR_RC(128);
+  else
+    SPR_RC(0);
+#undef SPR_RC
 }
 
 // ---------------------------------------------------------------------------
@@ -506,16 +568,59 @@ __global__ void split_rows_kernel(const void* X, int kind, long long hsx, int ld
     norms[static_cast<size_t>(h) * n + row] = static_cast<float>(sqrt(ss) * (1.0 + 1e-6));
 }
 
+// The same for rows that split into 16-byte pieces (D = Dp, TPR = D / EPT
+// threads per row dividing 32, 16-byte aligned rows): each thread widens one
+// piece, writes its plane values, and the row's lanes sum the squares.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    split_rows_vec_kernel(const T* X, long long hsx, int ldx_, int n, int D, int P,
+                          __nv_bfloat16* planes, long long plane_stride, float* norms) {
+  constexpr int EPT = 16 / sizeof(T);
+  const int TPR = D / EPT;
+  const int h = blockIdx.y;
+  const int row = blockIdx.x * (256 / TPR) + static_cast<int>(threadIdx.x) / TPR;
+  const int col = (static_cast<int>(threadIdx.x) % TPR) * EPT;
+  double ss = 0.0;
+  if (row < n) {
+    double v[EPT];
+    vload16(X + h * hsx + static_cast<size_t>(row) * ldx_ + col, v);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) ss = fma(v[i], v[i], ss);
+    const size_t ob = (static_cast<size_t>(h) * n + row) * D + col;
+    for (int pl = 0; pl < P; ++pl) {
+      __align__(16) __nv_bfloat16 b[EPT];
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) {
+        b[i] = __double2bfloat16(v[i]);
+        v[i] -= static_cast<double>(__bfloat162float(b[i]));
+      }
+      if (EPT == 8)
+        *reinterpret_cast<uint4*>(planes + pl * plane_stride + ob) = *reinterpret_cast<const uint4*>(b);
+      else if (EPT == 4)
+        *reinterpret_cast<uint2*>(planes + pl * plane_stride + ob) = *reinterpret_cast<const uint2*>(b);
+      else
+        *reinterpret_cast<uint32_t*>(planes + pl * plane_stride + ob) = *reinterpret_cast<const uint32_t*>(b);
+    }
+  }
+  for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (norms && row < n && col == 0)
+    norms[static_cast<size_t>(h) * n + row] = static_cast<float>(sqrt(ss) * (1.0 + 1e-6));
+}
+
 // Centroid side: planes of y (padded to Cpad rows with zeros), fp32 offsets
-// (+inf on padding), and the per-head maxima Y = max |y_j|, C = max |c_j|
-// (rounded up; merged across CTAs with an integer max on the bits of the
-// non-negative floats, after hmax was zeroed). One warp per centroid row.
+// (a large finite value on padding, so that values with index bits packed
+// into their low mantissa bits stay ordered numbers), the per-head maxima
+// Y = max |y_j|, C = max |c_j| (rounded up; merged across CTAs with an
+// integer max on the bits of the non-negative floats, after hmax was zeroed)
+// and the transposed fp64 copy yT [D, m] read by the fp64 decisions. One warp
+// per centroid row.
 constexpr int kPrepWarps = 16;
+constexpr float kPadOffset = 1.0e38f;
 
 __global__ void __launch_bounds__(kPrepWarps * 32)
     prep_centroids_kernel(const double* Yv, const double* cv, int m, int D, int Dp, int Cpad,
                           int P, __nv_bfloat16* planes, long long plane_stride, float* cf,
-                          float* hmax, const int32_t* flags, int flag_base) {
+                          float* hmax, double* ytr, const int32_t* flags, int flag_base) {
   __shared__ float ym[kPrepWarps], cm[kPrepWarps];
   const int h = blockIdx.y;
   if (flags && flags[h * 4 + flag_base + 1]) return;
@@ -527,6 +632,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
     double ss = 0.0;
     for (int t = lane; t < Dp; t += 32) {
       double v = (j < m && t < D) ? Yv[(static_cast<size_t>(h) * m + j) * D + t] : 0.0;
+      if (j < m && t < D) ytr[(static_cast<size_t>(h) * D + t) * m + j] = v;
       ss = fma(v, v, ss);
       for (int pl = 0; pl < P; ++pl) {
         const __nv_bfloat16 b = __double2bfloat16(v);
@@ -542,7 +648,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32)
         yv = static_cast<float>(sqrt(ss) * (1.0 + 1e-6));
         cvv = static_cast<float>(fabs(cj) * (1.0 + 1e-6));
       } else {
-        cf[static_cast<size_t>(h) * Cpad + j] = INFINITY;
+        cf[static_cast<size_t>(h) * Cpad + j] = kPadOffset;
       }
     }
   }
@@ -596,6 +702,25 @@ size_t assign_tc_smem_bytes(int nA, int nB, int Dp, int Cpad) {
 cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, int n, int D,
                               int Dp, int P, int H, __nv_bfloat16* planes, long long plane_stride,
                               float* norms, cudaStream_t st) {
+  const int es = kind == kXf64 ? 8 : (kind == kXbf16 ? 2 : 4);
+  const int ept = 16 / es;
+  const int tpr = D / ept;
+  const bool vec = D == Dp && D % ept == 0 && tpr >= 1 && tpr <= 32 && (tpr & (tpr - 1)) == 0 &&
+                   reinterpret_cast<uintptr_t>(X) % 16 == 0 && (static_cast<long long>(ldx) * es) % 16 == 0 &&
+                   (hsx * es) % 16 == 0;
+  if (vec) {
+    dim3 grid((n + 256 / tpr - 1) / (256 / tpr), H);
+    if (kind == kXf64)
+      split_rows_vec_kernel<<<grid, 256, 0, st>>>(static_cast<const double*>(X), hsx, ldx, n, D, P,
+                                                  planes, plane_stride, norms);
+    else if (kind == kXbf16)
+      split_rows_vec_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), hsx, ldx, n,
+                                                  D, P, planes, plane_stride, norms);
+    else
+      split_rows_vec_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(X), hsx, ldx, n, D, P,
+                                                  planes, plane_stride, norms);
+    return cudaGetLastError();
+  }
   dim3 grid((n + 7) / 8, H);
   split_rows_kernel<<<grid, 256, 0, st>>>(X, kind, hsx, ldx, n, D, Dp, P, planes, plane_stride,
                                           norms);
@@ -604,12 +729,13 @@ cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, i
 
 cudaError_t launch_prep_centroids(const double* Y, const double* c, int m, int D, int Dp,
                                   int Cpad, int P, int H, __nv_bfloat16* planes,
-                                  long long plane_stride, float* cf, float* hmax,
+                                  long long plane_stride, float* cf, float* hmax, double* ytr,
                                   const int32_t* flags, int flag_base, cudaStream_t st) {
   zero_counts_kernel<<<(2 * H + 127) / 128, 128, 0, st>>>(reinterpret_cast<int32_t*>(hmax), 2 * H);
   dim3 grid((Cpad + kPrepWarps - 1) / kPrepWarps, H);
   prep_centroids_kernel<<<grid, kPrepWarps * 32, 0, st>>>(Y, c, m, D, Dp, Cpad, P, planes,
-                                                          plane_stride, cf, hmax, flags, flag_base);
+                                                          plane_stride, cf, hmax, ytr, flags,
+                                                          flag_base);
   return cudaGetLastError();
 }
 
@@ -663,9 +789,10 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   argmin_tc_kernel<<<ctas, kAsThreads, shb, st>>>(maps, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  recheck_kernel<<<dim3(64, a.H), kRcThreads, 0, st>>>(a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D,
-                                                a.y_exact, a.c_exact, a.m, a.direct, a.labels,
-                                                a.flags, a.flag_base, a.recheck, a.nrecheck);
+  if (a.direct)
+    launch_recheck_d<true>(a, st);
+  else
+    launch_recheck_d<false>(a, st);
   return cudaGetLastError();
 }
 

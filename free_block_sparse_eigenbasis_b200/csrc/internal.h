@@ -103,7 +103,7 @@ struct AssignTC {
   long long x_hs;
   int x_ld;
   int D;
-  const double* y_exact;          // [H, m, D]
+  const double* y_tr;             // [H, D, m] centroid side transposed (prep_centroids)
   const double* c_exact;          // [H, m] (unused when direct)
   int m;
   int direct;                     // 1: d = |x - y|^2, 0: d = c - 2 x.y
@@ -114,7 +114,7 @@ cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, i
                               float* norms, cudaStream_t st);
 cudaError_t launch_prep_centroids(const double* Y, const double* c, int m, int D, int Dp,
                                   int Cpad, int P, int H, __nv_bfloat16* planes,
-                                  long long plane_stride, float* cf, float* hmax,
+                                  long long plane_stride, float* cf, float* hmax, double* ytr,
                                   const int32_t* flags, int flag_base, cudaStream_t st);
 cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st);
 

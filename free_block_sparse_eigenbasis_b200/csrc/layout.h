@@ -57,6 +57,8 @@ struct Layout {
   size_t hmq;      // [H, 2] f32
   size_t recheck;  // [H, Nv] int32
   size_t nrecheck; // [H] int32
+  size_t ytr;      // [H, D, m] f64 centroid side, transposed, for the fp64 decisions
+                   // (keys: D = e, m = Ck; queries: D = d, m = Cq)
   // stage 3
   size_t cq;       // [H, Cq, d] f64 query-group means (route)
   size_t ckr;      // [H, Ck, d] f64 key-group means (route)
@@ -167,6 +169,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->hmq = take(H * 8);
   L->recheck = take(H * Nv * 4);
   L->nrecheck = take(H * 4);
+  L->ytr = take(H * (Ck * e > Cq * d ? Ck * e : Cq * d) * 8);
   L->cq = take(H * Cq * d * 8);
   L->ckr = take(H * Ck * d * 8);
   {

@@ -135,8 +135,8 @@ __global__ void gram_f64_kernel(const double* X, const double* Y, const double* 
 // ---------------------------------------------------------------------------
 // Key response coordinates z = W^T k, W = U_e L_e^{1/2} ([d, e] fp64).
 // ---------------------------------------------------------------------------
-constexpr int kZRows = 64;
-constexpr int kZThreads = 128;
+constexpr int kZRows = 128;
+constexpr int kZThreads = 256;
 
 // 16-byte vector of k widened to float
 __device__ __forceinline__ int zvec_elems(const __nv_bfloat16*) { return 8; }
@@ -158,16 +158,17 @@ __device__ __forceinline__ void zvec_store(const float* src, float* dst) {
   dst[3] = v.w;
 }
 
-// Block = 128 key rows: the rows are staged in shared memory (as fp64) with
-// 16-byte loads; thread t computes 4 of the e coordinates of 2 rows (register
-// blocking: per column of k two shared loads of k and two 16-byte loads of
-// w serve 8 fma), summing over the d columns in ascending order in fp64.
+// Block = 128 key rows: the rows are staged in shared memory (as fp32, exact
+// for bf16 / fp32 inputs) with 16-byte loads; thread t computes 8 of the e
+// coordinates of row t % 128 (per column of k: one shared load of k and four
+// 16-byte broadcast loads of w serve 8 fma), summing over the d columns in
+// ascending order in fp64.
 template <typename T>
 __global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int Nv, int d, int e,
                                                           const double* wk, double* z) {
   extern __shared__ double zsm[];
-  double* w = zsm;                   // [d][e]
-  double* ks = zsm + d * e;          // [kZRows][d+1]
+  double* w = zsm;                                    // [d][e]
+  float* ks = reinterpret_cast<float*>(zsm + d * e);  // [kZRows][d+1]
   const int h = blockIdx.y;
   const int j0 = blockIdx.x * kZRows;
   const double* W = wk + static_cast<size_t>(h) * d * e;
@@ -184,51 +185,42 @@ __global__ void __launch_bounds__(kZThreads) zproj_kernel(const T* k, int N, int
 #pragma unroll
       for (int i = 0; i < 8; ++i) tmp[i] = 0.f;
     }
-    for (int i = 0; i < ve; ++i) ks[r * (d + 1) + a + i] = static_cast<double>(tmp[i]);
+    for (int i = 0; i < ve; ++i) ks[r * (d + 1) + a + i] = tmp[i];
   }
   __syncthreads();
-  const int nq = (e + 3) / 4;                       // column quads
-  const int pairs = (kZRows / 2) * nq;              // (row pair, quad) items
-  for (int item = threadIdx.x; item < pairs; item += blockDim.x) {
-    // rows rp and rp + kZRows / 2: consecutive threads read consecutive
-    // (padded) rows, so the shared loads of k do not conflict
-    const int rp = item % (kZRows / 2), qd = item / (kZRows / 2);
-    const int r0 = rp, r1 = rp + kZRows / 2, c0 = 4 * qd;
-    const int nc = min(4, e - c0);
-    double acc0[4] = {0.0, 0.0, 0.0, 0.0}, acc1[4] = {0.0, 0.0, 0.0, 0.0};
-    const double* k0 = ks + r0 * (d + 1);
-    const double* k1 = ks + r1 * (d + 1);
-    if (nc == 4 && (e % 2) == 0) {
+  const int r = threadIdx.x % kZRows;
+  const int j = j0 + r;
+  if (j >= Nv) return;
+  const float* kr = ks + r * (d + 1);
+  double* zr = z + (static_cast<size_t>(h) * Nv + j) * e;
+  for (int c0 = (threadIdx.x / kZRows) * 8; c0 < e; c0 += (kZThreads / kZRows) * 8) {
+    const int ne = min(8, e - c0);
+    double acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.0;
+    if (ne == 8 && (e % 2) == 0) {
       for (int a = 0; a < d; ++a) {
-        const double x0 = k0[a], x1 = k1[a];
-        const double2 wa = *reinterpret_cast<const double2*>(w + a * e + c0);
-        const double2 wb = *reinterpret_cast<const double2*>(w + a * e + c0 + 2);
-        acc0[0] = fma(x0, wa.x, acc0[0]);
-        acc0[1] = fma(x0, wa.y, acc0[1]);
-        acc0[2] = fma(x0, wb.x, acc0[2]);
-        acc0[3] = fma(x0, wb.y, acc0[3]);
-        acc1[0] = fma(x1, wa.x, acc1[0]);
-        acc1[1] = fma(x1, wa.y, acc1[1]);
-        acc1[2] = fma(x1, wb.x, acc1[2]);
-        acc1[3] = fma(x1, wb.y, acc1[3]);
+        const double kv = static_cast<double>(kr[a]);
+        const double2* wa = reinterpret_cast<const double2*>(w + a * e + c0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const double2 wv = wa[c];
+          acc[2 * c] = fma(kv, wv.x, acc[2 * c]);
+          acc[2 * c + 1] = fma(kv, wv.y, acc[2 * c + 1]);
+        }
       }
     } else {
       for (int a = 0; a < d; ++a) {
-        const double x0 = k0[a], x1 = k1[a];
+        const double kv = static_cast<double>(kr[a]);
+        const double* wa = w + a * e + c0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < nc) {
-            acc0[c] = fma(x0, w[a * e + c0 + c], acc0[c]);
-            acc1[c] = fma(x1, w[a * e + c0 + c], acc1[c]);
-          }
+        for (int c = 0; c < 8; ++c)
+          if (c < ne) acc[c] = fma(kv, wa[c], acc[c]);
       }
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (c >= nc) continue;
-      if (j0 + r0 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r0) * e + c0 + c] = acc0[c];
-      if (j0 + r1 < Nv) z[(static_cast<size_t>(h) * Nv + j0 + r1) * e + c0 + c] = acc1[c];
-    }
+    for (int c = 0; c < 8; ++c)
+      if (c < ne) zr[c0 + c] = acc[c];
   }
 }
 
@@ -474,33 +466,6 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_kernel(
 // (RL = 256 / TPR row lanes), then the row lanes' sums are added in a fixed
 // order.
 template <typename T>
-__device__ __forceinline__ void vload16(const T* p, double* out);
-template <>
-__device__ __forceinline__ void vload16<__nv_bfloat16>(const __nv_bfloat16* p, double* out) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    out[2 * i] = static_cast<double>(__uint_as_float(w[i] << 16));
-    out[2 * i + 1] = static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
-  }
-}
-template <>
-__device__ __forceinline__ void vload16<float>(const float* p, double* out) {
-  const float4 v = *reinterpret_cast<const float4*>(p);
-  out[0] = v.x;
-  out[1] = v.y;
-  out[2] = v.z;
-  out[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void vload16<double>(const double* p, double* out) {
-  const double2 v = *reinterpret_cast<const double2*>(p);
-  out[0] = v.x;
-  out[1] = v.y;
-}
-
-template <typename T>
 __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
     const T* X, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
     const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
@@ -570,30 +535,44 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
 }
 
 // W_g = G qbar_g, c_g = qbar_g^T G qbar_g (fp64, fixed-order reduction).
-__global__ void query_metric_apply_kernel(const double* G, const double* qbar, int Cq, int d,
-                                          double* wg, double* cg, const int32_t* skip,
-                                          int skip_stride) {
-  __shared__ double qs[128];
-  __shared__ double part[128];
-  const int h = blockIdx.y, g = blockIdx.x;
+// One CTA per (8 query centroids, head); thread a owns column a of W for the
+// CTA's centroids, so every element of G is read once per CTA.
+constexpr int kQmaG = 8;
+
+__global__ void __launch_bounds__(128)
+    query_metric_apply_kernel(const double* G, const double* qbar, int Cq, int d, double* wg,
+                              double* cg, const int32_t* skip, int skip_stride) {
+  __shared__ double qs[kQmaG][128];
+  __shared__ double red[kQmaG][4];
+  const int h = blockIdx.y, g0 = blockIdx.x * kQmaG;
   if (skip && skip[h * skip_stride]) return;
+  const int ng = min(kQmaG, Cq - g0);
   const double* Gh = G + static_cast<size_t>(h) * d * d;
-  const double* qb = qbar + (static_cast<size_t>(h) * Cq + g) * d;
-  const int a = threadIdx.x;
-  if (a < d) qs[a] = qb[a];
+  const int a = threadIdx.x, lane = a & 31, wp = a >> 5;
+  for (int i = a; i < kQmaG * 128; i += 128) {
+    const int g = i >> 7, b = i & 127;
+    qs[g][b] = (g < ng && b < d) ? qbar[(static_cast<size_t>(h) * Cq + g0 + g) * d + b] : 0.0;
+  }
   __syncthreads();
-  double w = 0.0;
+  double w[kQmaG];
+#pragma unroll
+  for (int g = 0; g < kQmaG; ++g) w[g] = 0.0;
   if (a < d) {
-    for (int b = 0; b < d; ++b) w = fma(Gh[static_cast<size_t>(b) * d + a], qs[b], w);
-    wg[(static_cast<size_t>(h) * Cq + g) * d + a] = w;
+#pragma unroll 4
+    for (int b = 0; b < d; ++b) {
+      const double gb = Gh[static_cast<size_t>(b) * d + a];
+#pragma unroll
+      for (int g = 0; g < kQmaG; ++g) w[g] = fma(gb, qs[g][b], w[g]);
+    }
   }
-  part[a] = (a < d) ? qs[a] * w : 0.0;
+#pragma unroll
+  for (int g = 0; g < kQmaG; ++g) {
+    if (a < d && g < ng) wg[(static_cast<size_t>(h) * Cq + g0 + g) * d + a] = w[g];
+    const double v = warp_sum_f64((a < d) ? qs[g][a] * w[g] : 0.0);
+    if (lane == 0) red[g][wp] = v;
+  }
   __syncthreads();
-  for (int s = 64; s > 0; s >>= 1) {
-    if (a < s) part[a] += part[a + s];
-    __syncthreads();
-  }
-  if (a == 0) cg[static_cast<size_t>(h) * Cq + g] = part[0];
+  if (a < ng) cg[static_cast<size_t>(h) * Cq + g0 + a] = (red[a][0] + red[a][1]) + (red[a][2] + red[a][3]);
 }
 
 __global__ void write_labels_kernel(const int32_t* lab, int H, int N, int Nv, int C_text,
@@ -636,7 +615,7 @@ cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
 
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
                          const double* wk, double* z, cudaStream_t st) {
-  const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 8;
+  const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;
   dim3 grid((Nv + kZRows - 1) / kZRows, H);
   if (bf16) {
     cudaFuncSetAttribute(zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -716,8 +695,8 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx,
 cudaError_t launch_query_metric_apply(const double* G, const double* qbar, int Cq, int H, int d,
                                       double* wg, double* cg, const int32_t* skip,
                                       int skip_stride, cudaStream_t st) {
-  query_metric_apply_kernel<<<dim3(Cq, H), 128, 0, st>>>(G, qbar, Cq, d, wg, cg, skip,
-                                                         skip_stride);
+  query_metric_apply_kernel<<<dim3((Cq + kQmaG - 1) / kQmaG, H), 128, 0, st>>>(
+      G, qbar, Cq, d, wg, cg, skip, skip_stride);
   return cudaGetLastError();
 }
 

@@ -3,9 +3,9 @@
 // group-major layouts), also used to form the k-means group sums in a fixed
 // (ascending token) order.
 //
-// Three passes per head: per-chunk histograms, an exclusive scan in
-// (group, chunk) order, and a stable scatter in which the warps of a chunk
-// claim positions one after another.
+// Per head: per-chunk histograms, an exclusive scan in (group, chunk) order
+// (down the chunks of every group, then over the group totals), and a stable
+// scatter in which the warps of a chunk claim positions one after another.
 #include "common.cuh"
 #include "internal.h"
 
@@ -36,41 +36,47 @@ __global__ void sort_hist_kernel(const int32_t* __restrict__ labels, int n, int 
   for (int c = threadIdx.x; c < C; c += blockDim.x) out[c] = sh[c];
 }
 
-// One CTA per head. hist[h][chunk][c] becomes the position of chunk's first
-// element of group c relative to the start of group c; off[h][c] the first
-// position of group c.
-__global__ void sort_scan_kernel(int n, int C, int nchunk, int32_t* __restrict__ hist,
-                                 int32_t* __restrict__ off, const int32_t* skip,
-                                 int skip_stride) {
+// hist[h][chunk][c] becomes the position of chunk's first element of group c
+// relative to the start of group c, and off[h][c] the size of group c: one
+// thread per (group, head) walks the chunks with 16 loads in flight.
+constexpr int kColThreads = 128;
+
+__global__ void __launch_bounds__(kColThreads)
+    sort_colscan_kernel(int C, int nchunk, int32_t* __restrict__ hist, int32_t* __restrict__ off,
+                        const int32_t* skip, int skip_stride) {
+  const int h = blockIdx.y, c = blockIdx.x * kColThreads + threadIdx.x;
+  if (skip && skip[h * skip_stride]) return;
+  if (c >= C) return;
+  int32_t* col = hist + static_cast<size_t>(h) * nchunk * C + c;
+  int32_t run = 0;
+  int k = 0;
+  for (; k + 16 <= nchunk; k += 16) {
+    int32_t v[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v[q] = col[static_cast<size_t>(k + q) * C];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      col[static_cast<size_t>(k + q) * C] = run;
+      run += v[q];
+    }
+  }
+  for (; k < nchunk; ++k) {
+    const int32_t v = col[static_cast<size_t>(k) * C];
+    col[static_cast<size_t>(k) * C] = run;
+    run += v;
+  }
+  off[static_cast<size_t>(h) * (C + 1) + c] = run;  // total for now
+}
+
+// One CTA per head: the group sizes in off[h] become the groups' first
+// positions (exclusive scan), off[h][C] = n.
+__global__ void __launch_bounds__(1024) sort_scan_kernel(int n, int C, int32_t* __restrict__ off,
+                                                         const int32_t* skip, int skip_stride) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
   const int h = blockIdx.x;
   if (skip && skip[h * skip_stride]) return;
-  int32_t* hh = hist + static_cast<size_t>(h) * nchunk * C;
   int32_t* oo = off + static_cast<size_t>(h) * (C + 1);
-  // per-group totals, turning each column into its exclusive running prefix
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    int32_t run = 0;
-    int k = 0;
-    for (; k + 8 <= nchunk; k += 8) {  // eight independent loads in flight
-      int32_t v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = hh[static_cast<size_t>(k + q) * C + c];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        hh[static_cast<size_t>(k + q) * C + c] = run;
-        run += v[q];
-      }
-    }
-    for (; k < nchunk; ++k) {
-      const int32_t v = hh[static_cast<size_t>(k) * C + c];
-      hh[static_cast<size_t>(k) * C + c] = run;
-      run += v;
-    }
-    oo[c] = run;  // total for now
-  }
-  __syncthreads();
-  // exclusive scan of the totals over c, blockDim.x elements at a time
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -149,7 +155,9 @@ cudaError_t launch_counting_sort(const int32_t* labels, int H, int n, int C, int
   dim3 g2(nchunk, H);
   sort_hist_kernel<<<g2, kSortThreads, shb, st>>>(labels, n, C, nchunk, hist, skip, skip_stride,
                                                   stats);
-  sort_scan_kernel<<<H, 1024, 0, st>>>(n, C, nchunk, hist, off, skip, skip_stride);
+  sort_colscan_kernel<<<dim3((C + kColThreads - 1) / kColThreads, H), kColThreads, 0, st>>>(
+      C, nchunk, hist, off, skip, skip_stride);
+  sort_scan_kernel<<<H, 1024, 0, st>>>(n, C, off, skip, skip_stride);
   sort_scatter_kernel<<<g2, kSortThreads, shb, st>>>(labels, n, C, nchunk, hist, off, perm, skip,
                                                        skip_stride);
   return cudaGetLastError();
