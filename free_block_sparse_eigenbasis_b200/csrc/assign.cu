@@ -278,8 +278,9 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       named_barrier_sync(kBarHead, kAsEpi);
       const float Y = p.hmax[h * 2 + 0], C = p.hmax[h * 2 + 1];
       int32_t* fl = p.flags + h * 4;
-      float b1[4], b2[4];
-      int blk[4];
+      float b1[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+      float b2[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+      int blk[4] = {0, 0, 0, 0};
       // reduce one piece of w (16 or 32) columns starting at column jb:
       // values packed with their position within the chain, then a pair at
       // a time into the chain's best and second best
@@ -305,6 +306,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         for (int k = 0; k < 4; ++k) blk[k] = (b1[k] < ob[k]) ? jb : blk[k];
       };
       const int U = (t1 - t0) * nchunks;  // (tile, chunk) steps of this head
+      float xn_pf = 0.f;  // |x| and the current label of group 0's row, loaded at
+      int lab_pf = -1;    // the start of the tile so the latency overlaps its chunks
       for (int u = 0; u < U; ++u) {
         const int c = u % nchunks;
         const int t = t0 + u / nchunks;
@@ -314,6 +317,12 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             b1[k] = INFINITY;
             b2[k] = INFINITY;
             blk[k] = 0;
+          }
+          const int row = t * kTileM + r;
+          if (q == 0 && row < p.n) {
+            const size_t li = static_cast<size_t>(h) * p.n + row;
+            xn_pf = p.xnorm[li];
+            lab_pf = p.labels[li];
           }
         }
         ok = ok && mbar_wait(&bars->acc_full[gc & 1], (gc >> 1) & 1, abort);
@@ -377,21 +386,29 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           }
           named_barrier_arrive(kBarXchFree, kAsEpi);
           const int row = t * kTileM + r;
-          bool changed = false;
+          bool changed = false, flag = false;
           if (ok && row < p.n) {
             const size_t li = static_cast<size_t>(h) * p.n + row;
-            const float xy = p.xnorm[li] * Y;
+            const float xy = xn_pf * Y;
             const float E = kt_term * xy + 1.25e-06f * (C + 2.f * xy);
             if (d2 - d1 > 2.f * E) {
-              changed = p.labels[li] != i1;
-              p.labels[li] = i1;
+              changed = lab_pf != i1;
+              if (changed) p.labels[li] = i1;
             } else {
-              const int k = atomicAdd(&p.nrecheck[h], 1);
-              p.recheck[static_cast<size_t>(h) * p.n + k] = row;
-              atomicAdd(reinterpret_cast<unsigned long long*>(
-                            &p.stats->recheck_rows[p.flag_base >> 1]),
-                        1ull);
+              flag = true;
             }
+          }
+          // rows to decide in fp64: one list append per warp
+          const unsigned fb = __ballot_sync(0xffffffffu, flag);
+          if (fb) {
+            int base = 0;
+            if (lane == 0) {
+              base = atomicAdd(&p.nrecheck[h], __popc(fb));
+              atomicAdd(reinterpret_cast<unsigned long long*>(&p.stats->recheck_rows[p.flag_base >> 1]),
+                        static_cast<unsigned long long>(__popc(fb)));
+            }
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (flag) p.recheck[static_cast<size_t>(h) * p.n + base + __popc(fb & ((1u << lane) - 1u))] = row;
           }
           // one atomic per warp for the label-change counter
           const unsigned cb = __ballot_sync(0xffffffffu, changed);

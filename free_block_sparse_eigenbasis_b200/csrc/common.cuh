@@ -273,12 +273,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------------------
 // Warp / block reductions (fixed order -> deterministic).
 // ---------------------------------------------------------------------------
-// 16 bytes of T at p (16-byte aligned) widened to fp64
+// 16 bytes of T (16-byte aligned), widened to fp64
 template <typename T>
-__device__ __forceinline__ void vload16(const T* p, double* out);
+__device__ __forceinline__ void vwiden16(const uint4 u, double* out);
 template <>
-__device__ __forceinline__ void vload16<__nv_bfloat16>(const __nv_bfloat16* p, double* out) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void vwiden16<__nv_bfloat16>(const uint4 u, double* out) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -287,18 +286,20 @@ __device__ __forceinline__ void vload16<__nv_bfloat16>(const __nv_bfloat16* p, d
   }
 }
 template <>
-__device__ __forceinline__ void vload16<float>(const float* p, double* out) {
-  const float4 v = *reinterpret_cast<const float4*>(p);
-  out[0] = v.x;
-  out[1] = v.y;
-  out[2] = v.z;
-  out[3] = v.w;
+__device__ __forceinline__ void vwiden16<float>(const uint4 u, double* out) {
+  out[0] = __uint_as_float(u.x);
+  out[1] = __uint_as_float(u.y);
+  out[2] = __uint_as_float(u.z);
+  out[3] = __uint_as_float(u.w);
 }
 template <>
-__device__ __forceinline__ void vload16<double>(const double* p, double* out) {
-  const double2 v = *reinterpret_cast<const double2*>(p);
-  out[0] = v.x;
-  out[1] = v.y;
+__device__ __forceinline__ void vwiden16<double>(const uint4 u, double* out) {
+  out[0] = __hiloint2double(static_cast<int>(u.y), static_cast<int>(u.x));
+  out[1] = __hiloint2double(static_cast<int>(u.w), static_cast<int>(u.z));
+}
+template <typename T>
+__device__ __forceinline__ void vload16(const T* p, double* out) {
+  vwiden16<T>(*reinterpret_cast<const uint4*>(p), out);
 }
 
 __device__ __forceinline__ double warp_sum_f64(double v) {

@@ -7,12 +7,14 @@
 //   1. Householder reduction to tridiagonal form, A = Q T Q^T with
 //      Q = H_0 H_1 ... H_{d-3}, H_k = I - tau_k v_k v_k^T (Golub & Van Loan,
 //      Matrix Computations, sec. 8.3.1), one CTA per matrix in shared memory;
-//   2. the ne largest eigenvalues of T by bisection on Sturm-sequence counts
-//      (sec. 8.4.1), one thread per eigenvalue;
-//   3. their eigenvectors by inverse iteration on T - lambda I with
-//      partial-pivoting tridiagonal LU (sec. 8.2.2 / 7.6.1), with
-//      Gram-Schmidt inside clusters of close eigenvalues after each step;
-//   4. back-transformation u = Q y, one warp per vector.
+//   2. the ne largest eigenvalues of T by multisection on Sturm-sequence
+//      counts (sec. 8.4.1): 16 or 32 threads per eigenvalue, one point each;
+//   3. their eigenvectors by inverse iteration on T - lambda I with one
+//      partial-pivoting tridiagonal LU per eigenvalue reused by every step
+//      (sec. 8.2.2 / 7.6.1), and classical Gram-Schmidt applied twice inside
+//      clusters of close eigenvalues after each step;
+//   4. back-transformation u = Q y, each warp applying every reflection to
+//      its (up to two) vectors at once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -55,19 +57,35 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
     return s;
   };
   constexpr int kParts = kTriThreads / D;  // row parts of the matrix-vector product
+  __shared__ double x2s;  // squared norm of the next column below its subdiagonal
+  {
+    double x2 = 0.0;
+    for (int i = 2 + tid; i < D; i += blockDim.x) x2 = fma(A[i], A[i], x2);
+    x2 = block_sum(x2);
+    if (tid == 0) x2s = x2;
+    __syncthreads();
+  }
+  // Three barriers per column: after the matrix-vector product, after its
+  // dot with v, after the rank-2 update (which also yields the next x2).
   for (int k = 0; k < D - 2; ++k) {
     const int n1 = D - k - 1;  // length of v (rows k+1 .. D-1)
     const double* Ak = A + k * D;  // row k = column k (symmetry)
-    double x2 = 0.0;
-    for (int i = k + 2 + tid; i < D; i += blockDim.x) x2 = fma(Ak[i], Ak[i], x2);
-    x2 = block_sum(x2);
+    const double x2 = x2s;
     const double alpha = Ak[k + 1];
     if (x2 == 0.0) {  // column already reduced: H_k = I
+      __syncthreads();  // every thread has read x2s
       if (tid == 0) {
         tau[k] = 0.0;
         od[k] = alpha;
       }
       for (int i = tid; i < n1; i += blockDim.x) hv[k * D + (k + 1 + i)] = (i == 0) ? 1.0 : 0.0;
+      if (wid == 0) {  // next column's norm (A is unchanged)
+        double y2 = 0.0;
+        for (int i = k + 3 + lane; i < D; i += 32) y2 = fma(A[(k + 1) * D + i], A[(k + 1) * D + i], y2);
+        y2 = warp_sum_f64(y2);
+        __syncwarp();
+        if (lane == 0) x2s = y2;
+      }
       __syncthreads();
       continue;
     }
@@ -83,15 +101,18 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
       tau[k] = tk;
       od[k] = beta;
     }
-    __syncthreads();
     // p = tau A22 v by columns (A22 symmetric): thread (column c, part) sums
-    // the rows r = part, part + kParts, ...
+    // the rows r = part, part + kParts, ...; v_r is formed from row k of A,
+    // which this column does not change
     {
       const int c = tid % D, part = tid / D;
       double sacc = 0.0;
       if (c < n1) {
         const double* col = A + (k + 1) * D + (k + 1) + c;
-        for (int r = part; r < n1; r += kParts) sacc = fma(col[r * D], v[r], sacc);
+        for (int r = part; r < n1; r += kParts) {
+          const double vr = (r == 0) ? 1.0 : Ak[k + 1 + r] * scl;
+          sacc = fma(col[r * D], vr, sacc);
+        }
       }
       pw[part][c] = sacc;
     }
@@ -106,14 +127,23 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
       pv = wi * v[tid];
     }
     pv = block_sum(pv);
-    const double kk = -0.5 * tk * pv;
-    if (tid < n1) w[tid] += kk * v[tid];
-    __syncthreads();
-    // A22 -= v w^T + w v^T (warp = row stripe, lane = column stripe)
+    const double kk2 = -tk * pv;  // A22 -= v w'^T + w' v^T with w' = w + (kk2 / 2) v
+    // (warp = row stripe, lane = column stripe); warp 0 owns row k+1 and
+    // forms the next column's squared norm below its subdiagonal
     for (int r = wid; r < n1; r += kTriThreads / 32) {
       const double vr = v[r], wr = w[r];
+      const double a_r = fma(kk2, vr, wr);
       double* Ar = A + (k + 1 + r) * D + (k + 1);
-      for (int c = lane; c < n1; c += 32) Ar[c] -= vr * w[c] + wr * v[c];
+      double y2 = 0.0;
+      for (int c = lane; c < n1; c += 32) {
+        const double nv = Ar[c] - (vr * w[c] + a_r * v[c]);
+        Ar[c] = nv;
+        if (c >= 2) y2 = fma(nv, nv, y2);
+      }
+      if (r == 0) {
+        y2 = warp_sum_f64(y2);
+        if (lane == 0) x2s = y2;
+      }
     }
     __syncthreads();
   }
@@ -126,29 +156,41 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
   }
 }
 
-// Number of eigenvalues of T below x (Sturm sequence of the LDL^T pivots).
-template <int D>
-__device__ int sturm_count(const double* dg, const double* e2, double x, double pivmin) {
-  int cnt = 0;
-  double q = dg[0] - x;
-  if (fabs(q) < pivmin) q = -pivmin;
-  cnt += (q < 0.0);
+// Number of eigenvalues of T below each of P points x (Sturm sequences of
+// the LDL^T pivots), the P recurrences interleaved.
+template <int D, int P>
+__device__ void sturm_counts(const double* dg, const double* e2, const double (&x)[P],
+                             double pivmin, int (&cnt)[P]) {
+  double q[P];
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    q[p] = dg[0] - x[p];
+    if (fabs(q[p]) < pivmin) q[p] = -pivmin;
+    cnt[p] = (q[p] < 0.0);
+  }
 #pragma unroll 1
   for (int i = 1; i < D; ++i) {
-    q = dg[i] - x - e2[i - 1] * __drcp_rn(q);
-    if (fabs(q) < pivmin) q = -pivmin;
-    cnt += (q < 0.0);
+    const double d = dg[i], e = e2[i - 1];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      q[p] = d - x[p] - e * __drcp_rn(q[p]);
+      if (fabs(q[p]) < pivmin) q[p] = -pivmin;
+      cnt[p] += (q[p] < 0.0);
+    }
   }
-  return cnt;
 }
 
-// Solve (T - lam I) y = b in place (b <- y) with a partial-pivoting LU of
-// the tridiagonal system. a, dl, du, du2, pv are the calling thread's work
-// arrays in shared memory, element i at [i * S] (S threads interleaved).
+// Partial-pivoting LU of the tridiagonal T - lam I (LAPACK dgttrf layout):
+// multipliers dl, pivots pv, U's diagonal (stored as its reciprocal in a),
+// first and second superdiagonals du, du2. The arrays are the calling
+// thread's work arrays in shared memory, element i at [i * S] (S threads
+// interleaved).
 template <int D, int S>
-__device__ void tri_solve(const double* dg, const double* od, double lam, double tiny, double* a,
-                          double* dl, double* du, double* du2, int* pv, double* b) {
+__device__ void tri_factor(const double* dg, const double* od, double lam, double tiny, double* a,
+                           double* dl, double* du, double* du2, int* pv) {
+#pragma unroll 4
   for (int i = 0; i < D; ++i) a[i * S] = dg[i] - lam;
+#pragma unroll 4
   for (int i = 0; i < D - 1; ++i) {
     dl[i * S] = od[i];
     du[i * S] = od[i];
@@ -180,7 +222,14 @@ __device__ void tri_solve(const double* dg, const double* od, double lam, double
     }
   }
   if (a[(D - 1) * S] == 0.0) a[(D - 1) * S] = tiny;
-  // L solve
+#pragma unroll 1
+  for (int i = 0; i < D; ++i) a[i * S] = 1.0 / a[i * S];
+}
+
+// b <- (T - lam I)^-1 b with the factors of tri_factor.
+template <int D, int S>
+__device__ void tri_apply(const double* ra, const double* dl, const double* du, const double* du2,
+                          const int* pv, double* b) {
 #pragma unroll 1
   for (int i = 0; i < D - 1; ++i) {
     if (pv[i * S] == 0) {
@@ -191,15 +240,15 @@ __device__ void tri_solve(const double* dg, const double* od, double lam, double
       b[i + 1] = t - dl[i * S] * b[i];
     }
   }
-  // U solve
-  b[D - 1] /= a[(D - 1) * S];
-  b[D - 2] = (b[D - 2] - du[(D - 2) * S] * b[D - 1]) / a[(D - 2) * S];
+  b[D - 1] *= ra[(D - 1) * S];
+  b[D - 2] = (b[D - 2] - du[(D - 2) * S] * b[D - 1]) * ra[(D - 2) * S];
 #pragma unroll 1
   for (int i = D - 3; i >= 0; --i)
-    b[i] = (b[i] - du[i * S] * b[i + 1] - du2[i * S] * b[i + 2]) / a[i * S];
+    b[i] = (b[i] - du[i * S] * b[i + 1] - du2[i * S] * b[i + 2]) * ra[i * S];
 }
 
-constexpr int kEigThreads = 256;
+constexpr int kEigThreads = 512;
+constexpr int kEigWarps = kEigThreads / 32;
 
 // One CTA per matrix, ne <= 32 eigenpairs (largest first): bisection and
 // inverse iteration by thread t, clustered Gram-Schmidt by warp 0, then
@@ -220,6 +269,7 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   __shared__ double lam[32];
   __shared__ double Y[32][D + 1];  // padded: thread t walks row t
   __shared__ double tnorm;
+  __shared__ double gdot[32], gred[kEigThreads / 32];
   const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const double* hv = scratch + static_cast<size_t>(h) * (D * D + 3 * D);
   const double* tau = hv + D * D;
@@ -240,25 +290,30 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   double emax2 = 0.0;
   for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
   const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
-  // multisection: eight threads per wanted eigenvalue (rank e_i = tid / 8,
-  // ascending index D-1-e_i) evaluate the Sturm count at eight interior
-  // points of the current interval, which shrinks nine-fold per round
+  // multisection: tpe threads per wanted eigenvalue (rank e_i = tid / tpe,
+  // ascending index D-1-e_i; tpe = 32 for ne <= 16, 16 for ne <= 32) each
+  // evaluate the Sturm count at one interior point of the current interval,
+  // which shrinks (tpe + 1)-fold per round
   {
-    const int e_i = tid >> 3, q = tid & 7;
+    const int tpe = ne <= kEigThreads / 32 ? 32 : 16;
+    const int e_i = tid / tpe, q = tid % tpe;
     const bool act = e_i < ne;
     const int m = D - 1 - e_i;
+    const double inv_parts = 1.0 / (tpe + 1);
+    const unsigned gmask = tpe == 32 ? 0xFFFFFFFFu : 0xFFFFu;
     double lo = -tnorm - 1.0, hi = tnorm + 1.0;
     for (int it = 0; it < 100; ++it) {
       const double w = hi - lo;
       const bool done = !(w > 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin);
       if (__all_sync(0xffffffffu, done || !act)) break;
-      bool pred = false;
-      if (act && !done) pred = sturm_count<D>(dg, e2, lo + w * (q + 1) * (1.0 / 9.0), pivmin) <= m;
-      const unsigned bal = __ballot_sync(0xffffffffu, pred);
-      const int nt = __popc((bal >> ((lane >> 3) * 8)) & 0xFFu);  // points below lambda
+      double x[1] = {lo + w * (q + 1) * inv_parts};
+      int cnt[1] = {D};
+      if (act && !done) sturm_counts<D, 1>(dg, e2, x, pivmin, cnt);
+      const unsigned bal = __ballot_sync(0xffffffffu, act && !done && cnt[0] <= m);
+      const int nt = __popc((bal >> ((lane / tpe) * tpe)) & gmask);  // points below lambda
       if (act && !done) {
-        const double nlo = nt > 0 ? lo + w * nt * (1.0 / 9.0) : lo;
-        const double nhi = nt < 8 ? lo + w * (nt + 1) * (1.0 / 9.0) : hi;
+        const double nlo = nt > 0 ? lo + w * nt * inv_parts : lo;
+        const double nhi = nt < tpe ? lo + w * (nt + 1) * inv_parts : hi;
         lo = nlo;
         hi = nhi;
       }
@@ -271,38 +326,57 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   int* pv = reinterpret_cast<int*>(eig_work + 4 * D * 32) + (tid & 31);
   const double tiny = eps * fmax(tnorm, 1e-300);
   if (tid < ne)
+#pragma unroll 1
     for (int i = 0; i < D; ++i) Y[tid][i] = 1.0 + 0.5 * sin(0.7 * (i + 1) * (tid + 1));
   const double ortol = 1e-3 * tnorm;
+  double* wa = wk;
+  double* wdl = wk + D * 32;
+  double* wdu = wk + 2 * D * 32;
+  double* wdu2 = wk + 3 * D * 32;
+  if (tid < ne) tri_factor<D, 32>(dg, od, lam[tid], tiny, wa, wdl, wdu, wdu2, pv);
   for (int it = 0; it < kInvIters; ++it) {
     if (tid < ne) {
       double* b = Y[tid];
-      tri_solve<D, 32>(dg, od, lam[tid], tiny, wk, wk + D * 32, wk + 2 * D * 32, wk + 3 * D * 32, pv, b);
+      tri_apply<D, 32>(wa, wdl, wdu, wdu2, pv, b);
       double s = 0.0;
+#pragma unroll 4
       for (int i = 0; i < D; ++i) s = fma(b[i], b[i], s);
       const double inv = 1.0 / sqrt(s);
+#pragma unroll 4
       for (int i = 0; i < D; ++i) b[i] *= inv;
     }
     __syncthreads();
-    // Gram-Schmidt against earlier vectors of the same cluster, in rank order
-    if (wid == 0) {
-      for (int t = 1; t < ne; ++t) {
-        for (int s = t - 1; s >= 0; --s) {
-          if (fabs(lam[s] - lam[s + 1]) > ortol) break;  // cluster boundary
+    // Gram-Schmidt against the earlier vectors of the same cluster (rank
+    // order; classical Gram-Schmidt applied twice), all warps
+    for (int t = 1; t < ne; ++t) {
+      int s0 = t;
+      while (s0 > 0 && fabs(lam[s0 - 1] - lam[s0]) <= ortol) --s0;
+      if (s0 == t) continue;  // the same for every thread
+      for (int pass = 0; pass < 2; ++pass) {
+        for (int s = s0 + wid; s < t; s += kEigThreads / 32) {
           double dot = 0.0;
           for (int i = lane; i < D; i += 32) dot = fma(Y[s][i], Y[t][i], dot);
           dot = warp_sum_f64(dot);
-          for (int i = lane; i < D; i += 32) Y[t][i] -= dot * Y[s][i];
-          __syncwarp();
+          if (lane == 0) gdot[s] = dot;
         }
-        double nn = 0.0;
-        for (int i = lane; i < D; i += 32) nn = fma(Y[t][i], Y[t][i], nn);
-        nn = warp_sum_f64(nn);
-        const double inv = 1.0 / sqrt(nn);
-        for (int i = lane; i < D; i += 32) Y[t][i] *= inv;
-        __syncwarp();
+        __syncthreads();
+        if (tid < D) {
+          double y = Y[t][tid];
+          for (int s = s0; s < t; ++s) y -= gdot[s] * Y[s][tid];
+          Y[t][tid] = y;
+        }
+        __syncthreads();
       }
+      double nn = (tid < D) ? Y[t][tid] * Y[t][tid] : 0.0;
+      nn = warp_sum_f64(nn);
+      if (lane == 0) gred[wid] = nn;
+      __syncthreads();
+      double tot = 0.0;
+#pragma unroll
+      for (int w = 0; w < kEigThreads / 32; ++w) tot += gred[w];
+      if (tid < D) Y[t][tid] *= 1.0 / sqrt(tot);
+      __syncthreads();
     }
-    __syncthreads();
   }
   // back-transformation: u = H_0 (H_1 (... H_{D-3} y)), warp w owns vectors
   // w, w + 8, ...; the Householder vectors and tau are first staged in the
@@ -312,20 +386,35 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   for (int i = tid; i < D * D; i += blockDim.x) hs[i] = hv[i];
   for (int i = tid; i < D; i += blockDim.x) ts[i] = tau[i];
   __syncthreads();
-  for (int t = wid; t < ne; t += kEigThreads / 32) {
-    double* y = Y[t];
-    for (int k = D - 3; k >= 0; --k) {
-      const double tk = ts[k];
-      if (tk == 0.0) continue;
-      const double* hk = hs + k * D;
-      double dot = 0.0;
-      for (int i = k + 1 + lane; i < D; i += 32) dot = fma(hk[i], y[i], dot);
-      dot = warp_sum_f64(dot) * tk;
-      for (int i = k + 1 + lane; i < D; i += 32) y[i] -= dot * hk[i];
-      __syncwarp();
+  // warp w owns vectors w and w + 16 (ne <= 32) and applies each reflection
+  // to both at once
+  const int nv = ne > wid ? (ne - wid + kEigWarps - 1) / kEigWarps : 0;
+  for (int k = D - 3; k >= 0; --k) {
+    const double tk = ts[k];
+    if (tk == 0.0) continue;
+    const double* hk = hs + k * D;
+    double dot[2] = {0.0, 0.0};
+    for (int i = k + 1 + lane; i < D; i += 32) {
+      const double hi = hk[i];
+#pragma unroll
+      for (int v = 0; v < 2; ++v)
+        if (v < nv) dot[v] = fma(hi, Y[wid + kEigWarps * v][i], dot[v]);
     }
-    for (int i = lane; i < D; i += 32)
-      evecs[(static_cast<size_t>(h) * D + i) * ne + t] = y[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int v = 0; v < 2; ++v) dot[v] += __shfl_xor_sync(0xffffffffu, dot[v], o);
+    for (int i = k + 1 + lane; i < D; i += 32) {
+      const double hi = hk[i];
+#pragma unroll
+      for (int v = 0; v < 2; ++v)
+        if (v < nv) Y[wid + kEigWarps * v][i] -= (dot[v] * tk) * hi;
+    }
+    __syncwarp();
+  }
+  for (int v = 0; v < nv; ++v) {
+    const int t = wid + kEigWarps * v;
+    for (int i = lane; i < D; i += 32) evecs[(static_cast<size_t>(h) * D + i) * ne + t] = Y[t][i];
     if (lane == 0) evals[static_cast<size_t>(h) * ne + t] = lam[t];
   }
 }

@@ -485,20 +485,27 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
   double acc[EPT];
 #pragma unroll
   for (int i = 0; i < EPT; ++i) acc[i] = 0.0;
+  // rows p, p + RL, p + 2 RL, p + 3 RL of this row lane in flight together,
+  // summed in ascending position order
   int p = lo + rl;
 #pragma unroll 1
-  for (; p + RL < hi; p += 2 * RL) {
-    const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
-    const size_t r1 = pp ? static_cast<size_t>(pp[p + RL]) : static_cast<size_t>(p + RL);
-    double v0[EPT], v1[EPT];
-    vload16(Xh + r0 * ldx, v0);
-    vload16(Xh + r1 * ldx, v1);
+  for (; p + 3 * RL < hi; p += 4 * RL) {
+    size_t r[4];
 #pragma unroll
-    for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
+    for (int j = 0; j < 4; ++j) r[j] = pp ? static_cast<size_t>(pp[p + j * RL]) : static_cast<size_t>(p + j * RL);
+    uint4 u[4];
 #pragma unroll
-    for (int i = 0; i < EPT; ++i) acc[i] += v1[i];
+    for (int j = 0; j < 4; ++j) u[j] = *reinterpret_cast<const uint4*>(Xh + r[j] * ldx);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double v[EPT];
+      vwiden16<T>(u[j], v);
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) acc[i] += v[i];
+    }
   }
-  if (p < hi) {
+#pragma unroll 1
+  for (; p < hi; p += RL) {
     const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
     double v0[EPT];
     vload16(Xh + r0 * ldx, v0);
