@@ -81,7 +81,6 @@ sparsepr_status cuda_status(cudaError_t e) {
 
 __global__ void set_i32_kernel(int32_t* p, int v) { *p = v; }
 
-constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
 
 // A second stream per device for small independent kernels that occupy few
 // SMs (the Fisher-Yates init beside the M_K eigen solve, the ridge solve beside

@@ -24,7 +24,9 @@
 // Persistent CTAs (at most one per SM) each take a contiguous range of the
 // row tiles of all heads, ordered head-major; the centroid planes of the
 // current head stay in shared memory and are reloaded when the range crosses
-// into the next head. Row tiles of 128 stream through a 2-stage TMA ring;
+// into the next head. One warp issues the TMA loads and another the MMAs
+// (each on its own, so neither waits behind the other's barrier polls).
+// Row tiles of 128 stream through a 2-stage TMA ring;
 // the 128 x (<=256) accumulator of each centroid chunk alternates between two
 // TMEM buffers, so the epilogue of one chunk overlaps the MMAs of the next.
 // The epilogue is four groups of four warps: every group sees all 128 rows
@@ -41,16 +43,17 @@ namespace {
 
 constexpr int kAsGroups = 4;                 // epilogue column groups
 constexpr int kAsEpi = kAsGroups * kTileM;   // epilogue threads (thread = row within a group)
-constexpr int kAsThreads = kAsEpi + 32;      // + one warp: lane 0 TMA, lane 1 MMA
+constexpr int kAsThreads = kAsEpi + 64;      // + a TMA producer warp and an MMA warp
 constexpr int kAsChunk = 256;                // centroids per accumulator chunk
 constexpr uint32_t kAsTmemCols = 512;
 constexpr size_t kAsMinSmem = 120 * 1024;    // keeps one CTA (and one TMEM owner) per SM
+constexpr int kAsMaxStages = 4;              // row-tile ring depth (as shared memory allows)
 // named barriers of the epilogue threads (0 is __syncthreads)
 constexpr int kBarXchFull = 1, kBarXchFree = 2, kBarHead = 3;
 
 struct AsBars {
   uint64_t b_full, b_empty;
-  uint64_t a_full[2], a_empty[2];
+  uint64_t a_full[kAsMaxStages], a_empty[kAsMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_idle;
   uint32_t tmem_base;
@@ -76,6 +79,7 @@ struct AsParams {
   float res;      // bound on the plane-split residual and dropped plane products, relative
   int tiles_per_head;
   int H;
+  int stages;          // row-tile ring depth, 2 .. kAsMaxStages
   const float* cvals;  // [H, Cpad] fp32 offsets (+inf on padding)
   const float* xnorm;  // [H, n] |x_i| (rounded up)
   const float* hmax;   // [H, 2] Y, C (rounded up)
@@ -148,7 +152,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* Bs = sm;
   uint8_t* As = sm + ((b_bytes + 1023) & ~1023);
-  float* cs = reinterpret_cast<float*>(As + 2 * a_stage);
+  float* cs = reinterpret_cast<float*>(As + p.stages * a_stage);
   float* xd1 = cs + p.Cpad;                 // [kAsGroups - 1][128]
   float* xd2 = xd1 + (kAsGroups - 1) * kTileM;
   int* xi1 = reinterpret_cast<int*>(xd2 + (kAsGroups - 1) * kTileM);
@@ -158,9 +162,11 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->b_full, 1);
     mbar_init(&bars->b_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kAsMaxStages; ++s) {
       mbar_init(&bars->a_full[s], 1);
       mbar_init(&bars->a_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->acc_full[s], 1);
       mbar_init(&bars->acc_empty[s], kAsEpi);
     }
@@ -196,8 +202,11 @@ __global__ void __launch_bounds__(kAsThreads, 1)
                           &bars->b_full, a * inner, h * p.b_head + r);
         ++seg;
         for (int t = t0; t < t1; ++t) {
-          const int s = u & 1;
-          if (u >= 2 && !mbar_wait(&bars->a_empty[s], ((u - 2) >> 1) & 1, abort)) { ok = false; return; }
+          const int s = u % p.stages;
+          if (u >= p.stages && !mbar_wait(&bars->a_empty[s], ((u - p.stages) / p.stages) & 1, abort)) {
+            ok = false;
+            return;
+          }
           mbar_arrive_expect_tx(&bars->a_full[s], a_stage);
           for (int pl = 0; pl < p.nA; ++pl)
             for (int a = 0; a < p.atoms; ++a)
@@ -207,9 +216,12 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         }
       });
       // let every load this thread issued land before the CTA exits
-      for (int x = max(0, u - 2); x < u; ++x) mbar_wait(&bars->a_full[x & 1], (x >> 1) & 1, &never);
+      for (int x = max(0, u - p.stages); x < u; ++x)
+        mbar_wait(&bars->a_full[x % p.stages], (x / p.stages) & 1, &never);
       if (seg > 0) mbar_wait(&bars->b_full, (seg - 1) & 1, &never);
-    } else if (lane == 1) {
+    }
+  } else if (warp == kAsEpi / 32 + 1) {
+    if (lane == 0) {
       // ------------------------------ MMA issuer ------------------------------
       const uint32_t a_addr = smem_u32(As), b_addr = smem_u32(Bs);
       int u = 0, gc = 0, seg = 0;
@@ -219,8 +231,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         if (!mbar_wait(&bars->b_full, seg & 1, abort)) { ok = false; return; }
         ++seg;
         for (int t = t0; t < t1; ++t, ++u) {
-          const int s = u & 1;
-          if (!mbar_wait(&bars->a_full[s], (u >> 1) & 1, abort)) { ok = false; return; }
+          const int s = u % p.stages;
+          if (!mbar_wait(&bars->a_full[s], (u / p.stages) & 1, abort)) { ok = false; return; }
           tc_fence_after();
           for (int c = 0; c < nchunks; ++c, ++gc) {
             const int buf = gc & 1;
@@ -458,24 +470,32 @@ __device__ __forceinline__ double rc_score(const double* xs, const double* yT, i
   const int D = DT > 0 ? DT : Drt;
   double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
   int t = 0;
-  constexpr int kTUnroll = (DT > 0 && DT <= 32) ? (DT / 4 > 0 ? DT / 4 : 1) : 4;  // 16 loads in flight
-#pragma unroll kTUnroll
-  for (; t + 4 <= D; t += 4) {
-    const double y0 = yT[static_cast<size_t>(t) * m + j], y1 = yT[static_cast<size_t>(t + 1) * m + j];
-    const double y2 = yT[static_cast<size_t>(t + 2) * m + j], y3 = yT[static_cast<size_t>(t + 3) * m + j];
+  auto step4 = [&](int t4, double y0, double y1, double y2, double y3) {
     if (DIRECT) {
-      const double e0 = xs[t] - y0, e1 = xs[t + 1] - y1, e2 = xs[t + 2] - y2, e3 = xs[t + 3] - y3;
+      const double e0 = xs[t4] - y0, e1 = xs[t4 + 1] - y1, e2 = xs[t4 + 2] - y2, e3 = xs[t4 + 3] - y3;
       a0 = fma(e0, e0, a0);
       a1 = fma(e1, e1, a1);
       a2 = fma(e2, e2, a2);
       a3 = fma(e3, e3, a3);
     } else {
-      a0 = fma(xs[t], y0, a0);
-      a1 = fma(xs[t + 1], y1, a1);
-      a2 = fma(xs[t + 2], y2, a2);
-      a3 = fma(xs[t + 3], y3, a3);
+      a0 = fma(xs[t4], y0, a0);
+      a1 = fma(xs[t4 + 1], y1, a1);
+      a2 = fma(xs[t4 + 2], y2, a2);
+      a3 = fma(xs[t4 + 3], y3, a3);
     }
+  };
+  // 16 loads in flight, then their products (column t goes to sum t % 4)
+#pragma unroll 1
+  for (; t + 16 <= D; t += 16) {
+    double y[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) y[q] = yT[static_cast<size_t>(t + q) * m + j];
+#pragma unroll
+    for (int q = 0; q < 16; q += 4) step4(t + q, y[q], y[q + 1], y[q + 2], y[q + 3]);
   }
+  for (; t + 4 <= D; t += 4)
+    step4(t, yT[static_cast<size_t>(t) * m + j], yT[static_cast<size_t>(t + 1) * m + j],
+          yT[static_cast<size_t>(t + 2) * m + j], yT[static_cast<size_t>(t + 3) * m + j]);
   for (; t < D; ++t) {
     const double y = yT[static_cast<size_t>(t) * m + j];
     if (DIRECT) {
@@ -794,7 +814,15 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   p.nrecheck = a.nrecheck;
   p.stats = a.stats;
   zero_counts_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.nrecheck, a.H);
+  // as many row-tile stages as shared memory holds (at least the two that
+  // assign_tc_smem_bytes counts)
   size_t shb = assign_tc_smem_bytes(a.nA, a.nB, a.Dp, a.Cpad);
+  const size_t a_stage = static_cast<size_t>(a.nA) * p.atoms * kTileM * (sw32 ? 32 : 128);
+  p.stages = 2;
+  while (p.stages < kAsMaxStages && shb + a_stage <= static_cast<size_t>(kMaxDynSmem)) {
+    shb += a_stage;
+    ++p.stages;
+  }
   if (shb < kAsMinSmem) shb = kAsMinSmem;
   cudaError_t e = cudaFuncSetAttribute(argmin_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(shb));

@@ -579,12 +579,20 @@ __global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_hea
 // kernel walks), and the exact routed pair count per head. With text tokens
 // (text = 1) the last query group keeps every key and every other group
 // also keeps the last key group (the text tokens), outside its budget.
-__global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, const int32_t* csr,
-                                   const int32_t* kh, int H, int N, int Cq, int Ck, int kmax,
-                                   int text, int32_t* nslots, int2* runs, int32_t* nruns,
-                                   int64_t* pairs, DeviceStats* stats) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= H * Cq) return;
+// One warp per (head, query group), lanes over the kept key groups: a kept
+// group starts a run unless its keys begin where the previous kept group's
+// end, and ends it unless the next one begins where it ends; runs of no
+// keys are then dropped in order.
+constexpr int kSpWarps = 8;
+
+__global__ void __launch_bounds__(kSpWarps * 32)
+    slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, const int32_t* csr,
+                       const int32_t* kh, int H, int N, int Cq, int Ck, int kmax, int text,
+                       int32_t* nslots, int2* runs, int32_t* nruns, int64_t* pairs,
+                       DeviceStats* stats) {
+  const int i = blockIdx.x * kSpWarps + static_cast<int>(threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= H * Cq) return;  // the whole warp
   const int h = i / Cq, g = i % Cq;
   const int Cqv = Cq - text, Ckv = Ck - text;  // routed (video) groups
   const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
@@ -592,49 +600,88 @@ __global__ void slots_pairs_kernel(const int32_t* off_q, const int32_t* off_k, c
   int2* rout = runs + static_cast<size_t>(i) * (kmax + 1);
   const int64_t nq = oq[g + 1] - oq[g];
   bool valid = (ok[0] >= 0 && ok[Ck] <= N && nq >= 0);
-  int64_t keys = 0;
+  long long keys = 0;
   int slots = 0, nr = 0;
-  auto add_run = [&](int lo, int hi) {
-    if (hi <= lo) return;
-    if (nr > 0 && rout[nr - 1].x + rout[nr - 1].y == lo) {
-      // adjacent to the previous run: extend it (slots are re-cut)
-      const int plen = rout[nr - 1].y;
-      slots -= (plen + kSlotRows - 1) / kSlotRows;
-      rout[nr - 1].y = plen + (hi - lo);
-      slots += (rout[nr - 1].y + kSlotRows - 1) / kSlotRows;
-    } else {
-      rout[nr++] = make_int2(lo, hi - lo);
-      slots += (hi - lo + kSlotRows - 1) / kSlotRows;
-    }
-    keys += hi - lo;
-  };
   if (text && g == Cqv) {
-    if (valid) add_run(0, N);  // the text query group: every key
+    if (valid && N > 0) {  // the text query group: every key
+      if (lane == 0) rout[0] = make_int2(0, N);
+      nr = 1;
+      slots = (N + kSlotRows - 1) / kSlotRows;
+      keys = N;
+    }
   } else {
     const int32_t* row = csr + (static_cast<size_t>(h) * Cqv + g) * kmax;
     const int k = kh[h];
     valid = valid && k >= 0 && k <= kmax;
     // reject malformed routes before the attention kernel walks them
-    for (int ci = 0; valid && ci < k; ++ci) {
-      const int c = row[ci];
-      valid = (c >= 0 && c < Ckv && ok[c] >= 0 && ok[c] <= ok[c + 1]);
-    }
-    if (valid) {
-      int ci = 0;
-      while (ci < k) {
+    if (valid)
+      for (int ci = lane; ci < k; ci += 32) {
         const int c = row[ci];
-        const int lo = ok[c];
-        int hi = ok[c + 1];
-        while (ci + 1 < k && ok[row[ci + 1]] == hi) {
-          ++ci;
-          hi = ok[row[ci] + 1];
-        }
-        add_run(lo, hi);
-        ++ci;
+        valid = valid && (c >= 0 && c < Ckv && ok[c] >= 0 && ok[c] <= ok[c + 1]);
       }
-      if (text) add_run(ok[Ckv], ok[Ckv + 1]);  // the text key group
+    valid = __all_sync(0xffffffffu, valid);
+    if (valid) {
+      for (int b0 = 0; b0 < k; b0 += 32) {
+        const int ci = b0 + lane;
+        bool start = false, last = false;
+        int lo = 0, hi = 0;
+        if (ci < k) {
+          const int c = row[ci];
+          lo = ok[c];
+          hi = ok[c + 1];
+          start = ci == 0 || ok[row[ci - 1] + 1] != lo;
+          last = ci == k - 1 || ok[row[ci + 1]] != hi;
+          keys += hi - lo;
+        }
+        const unsigned sb = __ballot_sync(0xffffffffu, start);
+        const int r = nr + __popc(sb & ((2u << lane) - 1u)) - 1;  // this group's run
+        if (start) rout[r].x = lo;
+        if (last) rout[r].y = hi;  // the run's end, for now
+        nr += __popc(sb);
+      }
+      __syncwarp();
+      int kept = 0;  // lengths; runs without keys dropped in order
+      for (int b0 = 0; b0 < nr; b0 += 32) {
+        const int r = b0 + lane;
+        int2 v = make_int2(0, 0);
+        if (r < nr) {
+          v = rout[r];
+          v.y -= v.x;
+        }
+        const bool keep = r < nr && v.y > 0;
+        const unsigned kb = __ballot_sync(0xffffffffu, keep);
+        __syncwarp();  // the chunk is read before any of it is rewritten
+        if (keep) {
+          rout[kept + __popc(kb & ((1u << lane) - 1u))] = v;
+          slots += (v.y + kSlotRows - 1) / kSlotRows;
+        }
+        kept += __popc(kb);
+      }
+      nr = kept;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        slots += __shfl_xor_sync(0xffffffffu, slots, o);
+        keys += __shfl_xor_sync(0xffffffffu, keys, o);
+      }
+      __syncwarp();
+      if (text && lane == 0) {  // the text key group, merged into the last run when adjacent
+        const int lo = ok[Ckv], hi = ok[Ckv + 1];
+        if (hi > lo) {
+          if (nr > 0 && rout[nr - 1].x + rout[nr - 1].y == lo) {
+            const int plen = rout[nr - 1].y;
+            slots -= (plen + kSlotRows - 1) / kSlotRows;
+            rout[nr - 1].y = plen + (hi - lo);
+            slots += (rout[nr - 1].y + kSlotRows - 1) / kSlotRows;
+          } else {
+            rout[nr++] = make_int2(lo, hi - lo);
+            slots += (hi - lo + kSlotRows - 1) / kSlotRows;
+          }
+          keys += hi - lo;
+        }
+      }
     }
   }
+  if (lane != 0) return;
   if (!valid) {
     nslots[i] = 0;
     nruns[i] = 0;
@@ -764,9 +811,9 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   work_list_kernel<<<a.H, 32, 0, st>>>(a.off_q, a.Cq, a.tiles_per_head, a.work, a.nwork);
   if (a.pairs) zero_i64_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H);
   const int n = a.H * a.Cq;
-  slots_pairs_kernel<<<(n + 127) / 128, 128, 0, st>>>(a.off_q, a.off_k, a.csr, a.kh, a.H, a.N,
-                                                     a.Cq, a.Ck, a.kmax, a.text, a.nslots, a.runs,
-                                                     a.nruns, a.pairs, a.stats);
+  slots_pairs_kernel<<<(n + kSpWarps - 1) / kSpWarps, kSpWarps * 32, 0, st>>>(
+      a.off_q, a.off_k, a.csr, a.kh, a.H, a.N, a.Cq, a.Ck, a.kmax, a.text, a.nslots, a.runs,
+      a.nruns, a.pairs, a.stats);
   if (a.pairs) pairs_to_stats_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H, a.stats);
   AttnParams prm;
   prm.H = a.H;

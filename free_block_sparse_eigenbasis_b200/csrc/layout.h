@@ -18,6 +18,7 @@ constexpr int kSlotRows = 8;    // keys per TMA row-slot of a KV tile
 constexpr int kSortChunk = 1024;  // tokens per counting-sort chunk
 constexpr int kMaxGroups = 4096;
 constexpr int kMaxSplits = 8;   // split-KV ranges of the dense probe pass
+constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
 
 struct Layout {
   // statistics / status (always at offset 0)

@@ -565,8 +565,18 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int g = 0; g < kQmaG; ++g) w[g] = 0.0;
   if (a < d) {
-#pragma unroll 4
-    for (int b = 0; b < d; ++b) {
+    int b = 0;
+#pragma unroll 1
+    for (; b + 16 <= d; b += 16) {  // 16 loads of G in flight
+      double gb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) gb[i] = Gh[static_cast<size_t>(b + i) * d + a];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int g = 0; g < kQmaG; ++g) w[g] = fma(gb[i], qs[g][b + i], w[g]);
+    }
+    for (; b < d; ++b) {
       const double gb = Gh[static_cast<size_t>(b) * d + a];
 #pragma unroll
       for (int g = 0; g < kQmaG; ++g) w[g] = fma(gb, qs[g][b], w[g]);
