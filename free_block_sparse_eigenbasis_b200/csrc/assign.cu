@@ -80,6 +80,7 @@ struct AsParams {
   int tiles_per_head;
   int H;
   int stages;          // row-tile ring depth, 2 .. kAsMaxStages
+  uint32_t pos_clear;  // ~7: clears the three low mantissa bits that carry a column position
   const float* cvals;  // [H, Cpad] fp32 offsets (+inf on padding)
   const float* xnorm;  // [H, n] |x_i| (rounded up)
   const float* hmax;   // [H, 2] Y, C (rounded up)
@@ -117,8 +118,10 @@ __device__ __forceinline__ void for_segments(const AsParams& p, int g, int g1, F
 // value with its position (0..7) within a chain piece in the low three
 // mantissa bits: changes the value by at most 7 ulp, and the minimum of
 // packed values carries the position of its column
-__device__ __forceinline__ float pack_pos(float v, int pos) {
-  return __uint_as_float((__float_as_uint(v) & ~7u) | static_cast<uint32_t>(pos));
+// (clear = ~7 comes in as a runtime value so that the compiler emits one
+// three-input logic op with the position as its immediate)
+__device__ __forceinline__ float pack_pos(float v, int pos, uint32_t clear) {
+  return __uint_as_float((__float_as_uint(v) & clear) | static_cast<uint32_t>(pos));
 }
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
@@ -223,7 +226,23 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   } else if (warp == kAsEpi / 32 + 1) {
     if (lane == 0) {
       // ------------------------------ MMA issuer ------------------------------
-      const uint32_t a_addr = smem_u32(As), b_addr = smem_u32(Bs);
+      // Descriptors are the base descriptors of the A ring and the B planes
+      // plus 16-byte offsets (the start-address field; shared memory < 256 KB),
+      // precomputed per plane pair and per K step.
+      const uint64_t da0 = smem_desc(smem_u32(As), p.sw32), db0 = smem_desc(smem_u32(Bs), p.sw32);
+      const int ksteps = p.sw32 ? 1 : p.atoms * 4;  // 16-column K steps
+      uint32_t pa_off[6], pb_off[6], ka_off[8], kb_off[8];
+#pragma unroll
+      for (int pi = 0; pi < 6; ++pi) {
+        pa_off[pi] = static_cast<uint32_t>(((p.pairs[pi] >> 2) * p.atoms * slab_a) >> 4);
+        pb_off[pi] = static_cast<uint32_t>(((p.pairs[pi] & 3) * p.atoms * slab_b) >> 4);
+      }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int atom = p.sw32 ? 0 : (ks >> 2), koff = p.sw32 ? 0 : (ks & 3) * 32;
+        ka_off[ks] = static_cast<uint32_t>((atom * slab_a + koff) >> 4);
+        kb_off[ks] = static_cast<uint32_t>((atom * slab_b + koff) >> 4);
+      }
       int u = 0, gc = 0, seg = 0;
       bool ok = true;
       for_segments(p, g0, g1, [&](int h, int t0, int t1) {
@@ -234,6 +253,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           const int s = u % p.stages;
           if (!mbar_wait(&bars->a_full[s], (u / p.stages) & 1, abort)) { ok = false; return; }
           tc_fence_after();
+          const uint64_t abase = da0 + static_cast<uint64_t>((s * a_stage) >> 4);
           for (int c = 0; c < nchunks; ++c, ++gc) {
             const int buf = gc & 1;
             if (gc >= 2 && !mbar_wait(&bars->acc_empty[buf], ((gc - 2) >> 1) & 1, abort)) {
@@ -244,19 +264,16 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             const int N = min(kAsChunk, p.Cpad - c * kAsChunk);
             const uint32_t idesc = idesc_bf16(kTileM, N, 0);
             const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * kAsChunk);
-            int first = 1;
-            for (int pi = 0; pi < p.npairs; ++pi) {
-              const int pa = p.pairs[pi] >> 2, pb = p.pairs[pi] & 3;
-              const int ksteps = p.sw32 ? 1 : p.atoms * 4;
-              for (int ks = 0; ks < ksteps; ++ks) {
-                const int atom = p.sw32 ? 0 : (ks >> 2);
-                const uint32_t koff = p.sw32 ? 0u : static_cast<uint32_t>((ks & 3) * 32);
-                const uint32_t aa = a_addr + s * a_stage + (pa * p.atoms + atom) * slab_a + koff;
-                const uint32_t ba = b_addr + (pb * p.atoms + atom) * slab_b +
-                                    c * kAsChunk * row_bytes + koff;
-                mma_bf16_ss(d_tmem, smem_desc(aa, p.sw32), smem_desc(ba, p.sw32), idesc,
-                            first ? 0u : 1u);
-                first = 0;
+            const uint64_t bbase = db0 + static_cast<uint64_t>((c * kAsChunk * row_bytes) >> 4);
+#pragma unroll
+            for (int pi = 0; pi < 6; ++pi) {
+              if (pi < p.npairs) {
+                const uint64_t ap = abase + pa_off[pi], bp = bbase + pb_off[pi];
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                  if (ks < ksteps)
+                    mma_bf16_ss(d_tmem, ap + ka_off[ks], bp + kb_off[ks], idesc,
+                                (pi > 0 || ks > 0) ? 1u : 0u);
               }
             }
             mma_commit(&bars->acc_full[buf]);
@@ -281,6 +298,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     // E bound: MMA terms, fp32 offsets and rounding, and the index bits
     // packed into the low three mantissa bits of each value (<= 7 ulp)
     const float kt_term = static_cast<float>(p.Kt) * 2.384185791015625e-07f + p.res;
+    const uint32_t clear = p.pos_clear;
     int gc = 0, nx = 0;
     bool ok = true;
     uint32_t va[32];
@@ -306,8 +324,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             const float ea[4] = {ca.x, ca.y, ca.z, ca.w}, eb[4] = {cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const float x = pack_pos(fmaf(-2.f, __uint_as_float(v[8 * pr + k]), ea[k]), 2 * pr);
-              const float y = pack_pos(fmaf(-2.f, __uint_as_float(v[8 * pr + 4 + k]), eb[k]), 2 * pr + 1);
+              const float x = pack_pos(fmaf(-2.f, __uint_as_float(v[8 * pr + k]), ea[k]), 2 * pr, clear);
+              const float y = pack_pos(fmaf(-2.f, __uint_as_float(v[8 * pr + 4 + k]), eb[k]), 2 * pr + 1, clear);
               const float m = fminf(x, y), M = fmaxf(x, y);
               b2[k] = min3f(b2[k], fmaxf(b1[k], m), M);
               b1[k] = fminf(b1[k], m);
@@ -803,6 +821,7 @@ cudaError_t launch_argmin_tc(const AssignTC& a, cudaStream_t st) {
   // 2 planes of y: residual <= 2^-16 (bound 2^-14)
   p.res = (a.nB >= 3) ? 9.5367431640625e-07f : 6.103515625e-05f;
   p.tiles_per_head = (a.n + kTileM - 1) / kTileM;
+  p.pos_clear = ~7u;
   p.H = a.H;
   p.cvals = a.cvals;
   p.xnorm = a.xnorm;
