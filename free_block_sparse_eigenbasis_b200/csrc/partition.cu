@@ -57,6 +57,47 @@ __global__ void fy_init_kernel(int Nv, int Ck, int Cq, uint64_t seed, int32_t* i
   }
 }
 
+// e = 16 (the workloads' eigenbasis size): thread = key row with all 16
+// coordinates in registers; the row of k is streamed with 16-byte loads and
+// W [d][16] is read from shared memory as 16-byte broadcasts, so every
+// widened element of k serves 16 fma. Same ascending-column sums as above.
+constexpr int kZRowThreads = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(kZRowThreads)
+    zproj_row16_kernel(const T* k, int N, int Nv, int d, const double* wk, double* z) {
+  constexpr int E = 16, EPT = 16 / sizeof(T);
+  extern __shared__ double w16[];  // [d][16]
+  const int h = blockIdx.y;
+  const int j = blockIdx.x * kZRowThreads + threadIdx.x;
+  const double* W = wk + static_cast<size_t>(h) * d * E;
+  for (int t = threadIdx.x; t < d * E; t += kZRowThreads) w16[t] = W[t];
+  __syncthreads();
+  if (j >= Nv) return;
+  const T* kr = k + (static_cast<size_t>(h) * N + j) * d;
+  double acc[E];
+#pragma unroll
+  for (int c = 0; c < E; ++c) acc[c] = 0.0;
+#pragma unroll 1
+  for (int a0 = 0; a0 < d; a0 += EPT) {
+    double kv[EPT];
+    vload16(kr + a0, kv);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const double2* wa = reinterpret_cast<const double2*>(w16 + (a0 + i) * E);
+#pragma unroll
+      for (int c2 = 0; c2 < E / 2; ++c2) {
+        const double2 wv = wa[c2];
+        acc[2 * c2] = fma(kv[i], wv.x, acc[2 * c2]);
+        acc[2 * c2 + 1] = fma(kv[i], wv.y, acc[2 * c2 + 1]);
+      }
+    }
+  }
+  double2* zr = reinterpret_cast<double2*>(z + (static_cast<size_t>(h) * Nv + j) * E);
+#pragma unroll
+  for (int c2 = 0; c2 < E / 2; ++c2) zr[c2] = make_double2(acc[2 * c2], acc[2 * c2 + 1]);
+}
+
 // ---------------------------------------------------------------------------
 // Gram kernels: out = factor * sum_s x_s y_s^T (+ diag I), 32x32 output tile
 // per CTA, rows s summed in ascending order.
@@ -512,8 +553,19 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
 #pragma unroll
     for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
   }
+  // the row lanes of a warp that share columns (lanes TPR apart) first, by
+  // shuffles; then the warps' partial rows in shared memory, in warp order
+  int prow = rl, npart = RL;
+  if (TPR <= 32) {
+    for (int o = TPR; o < 32; o <<= 1)
 #pragma unroll
-  for (int i = 0; i < EPT; ++i) part[rl * D + col + i] = acc[i];
+      for (int i = 0; i < EPT; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    prow = w;
+    npart = kMeanThreads / 32;
+  }
+  if (TPR > 32 || lane < TPR)
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) part[prow * D + col + i] = acc[i];
   __syncthreads();
   double* dst = out + (static_cast<size_t>(h) * C + c) * D;
   double ss = 0.0;
@@ -521,7 +573,7 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
     double v;
     if (n > 0) {
       double sum = part[t];
-      for (int q = 1; q < RL; ++q) sum += part[q * D + t];
+      for (int q = 1; q < npart; ++q) sum += part[q * D + t];
       v = sum / static_cast<double>(n);
     } else {
       v = keep_prev ? dst[t] : 0.0;
@@ -632,6 +684,17 @@ cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
 
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
                          const double* wk, double* z, cudaStream_t st) {
+  if (e == 16 && d % 8 == 0 && reinterpret_cast<uintptr_t>(k) % 16 == 0) {
+    const size_t shb16 = static_cast<size_t>(d) * 16 * 8;
+    dim3 g16((Nv + kZRowThreads - 1) / kZRowThreads, H);
+    if (bf16)
+      zproj_row16_kernel<<<g16, kZRowThreads, shb16, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv,
+                                                           d, wk, z);
+    else
+      zproj_row16_kernel<<<g16, kZRowThreads, shb16, st>>>(static_cast<const float*>(k), N, Nv, d,
+                                                           wk, z);
+    return cudaGetLastError();
+  }
   const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;
   dim3 grid((Nv + kZRows - 1) / kZRows, H);
   if (bf16) {
