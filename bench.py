@@ -50,8 +50,8 @@ def workload_desc(w):
 # DRAM traffic of the routed attention launch on the 720p workload from one ncu
 # capture (profiles/sparse_attn_kernel_wan13b_720p_traffic.md), valid for the
 # attention source it was taken on.
-ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=722669312 + 448694016,
-                    source_sha256_prefix="0de883bc14ce4ada")
+ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=724185600 + 449008640,
+                    source_sha256_prefix="8673188ba6275a7e")
 
 
 def attn_traffic(w):
