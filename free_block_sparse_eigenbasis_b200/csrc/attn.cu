@@ -13,8 +13,9 @@
 //
 // Roles (352 threads): two softmax warpgroups (warps 0-3 and 4-7, thread =
 // query row = TMEM lane) each own one TMEM slot (S_i, O_i, with P_i written
-// as packed bf16 over the first 64 columns of S_i); warp 8 lane 0 streams Q,
-// K and V with TMA; warp 9 lane 0 issues tcgen05.mma.
+// as packed bf16 over the first 64 columns of S_i); warp 8 streams Q and the
+// K tiles and warp 10 the V tiles with TMA, each through its own ring; warp 9
+// lane 0 issues tcgen05.mma.
 //   * a unit of two 128-row query tiles gives tile i to warpgroup i: both
 //     see every key tile, and the tensor cores alternate between them
 //     (P_0 V, S_0 of the next tile, P_1 V, S_1 of the next tile), so one
