@@ -51,7 +51,7 @@ def workload_desc(w):
 # capture (profiles/sparse_attn_kernel_wan13b_720p_traffic.md), valid for the
 # attention source it was taken on.
 ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=724185600 + 449008640,
-                    source_sha256_prefix="8673188ba6275a7e")
+                    source_sha256_prefix="d4a872a215d524c3")
 
 
 def attn_traffic(w):
