@@ -108,15 +108,18 @@ template <typename Loader>
 __device__ void gram_tile(Loader ld, int S, int d, double factor, double diag, double* out) {
   __shared__ double xs[kGT][kGT + 1];
   __shared__ double ys[kGT][kGT + 1];
+  __shared__ long long rows[kGT];  // source rows of the chunk's samples
   const int a0 = blockIdx.x * kGT, b0 = blockIdx.y * kGT;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 256 threads: ty 0..7
   double acc[4] = {0, 0, 0, 0};
   for (int s0 = 0; s0 < S; s0 += kGT) {
+    if (threadIdx.x < kGT) rows[threadIdx.x] = ld.row(s0 + threadIdx.x);
+    __syncthreads();
     for (int t = threadIdx.x; t < kGT * kGT; t += blockDim.x) {
       const int ss = t / kGT, cc = t % kGT;
       const int s = s0 + ss;
-      xs[ss][cc] = (s < S && a0 + cc < d) ? ld.x(s, a0 + cc) : 0.0;
-      ys[ss][cc] = (s < S && b0 + cc < d) ? ld.y(s, b0 + cc) : 0.0;
+      xs[ss][cc] = (s < S && a0 + cc < d) ? ld.x(rows[ss], a0 + cc) : 0.0;
+      ys[ss][cc] = (s < S && b0 + cc < d) ? ld.y(rows[ss], b0 + cc) : 0.0;
     }
     __syncthreads();
 #pragma unroll 4
@@ -134,15 +137,15 @@ __device__ void gram_tile(Loader ld, int S, int d, double factor, double diag, d
   }
 }
 
+// x(row, a) / y(row, b): element a (b) of source row `row`; row(s): the
+// source row of sample s (computed once per chunk of samples)
 template <typename T>
 struct SampledQueryLoader {
   const T* q;
   int Nv, Ms, d;
-  __device__ double x(int s, int a) const {
-    const long long row = ((2LL * s + 1) * Nv) / (2LL * Ms);
-    return to_f64(q, static_cast<size_t>(row) * d + a);
-  }
-  __device__ double y(int s, int b) const { return x(s, b); }
+  __device__ long long row(int s) const { return ((2LL * s + 1) * Nv) / (2LL * Ms); }
+  __device__ double x(long long row, int a) const { return to_f64(q, static_cast<size_t>(row) * d + a); }
+  __device__ double y(long long row, int b) const { return x(row, b); }
 };
 
 template <typename T>
@@ -155,10 +158,11 @@ __global__ void metric_mk_kernel(const T* q, int N, int Nv, int d, int Ms, doubl
 struct F64Loader {
   const double *X, *Y, *xm, *ym;
   int ld;
-  __device__ double x(int s, int a) const {
+  __device__ long long row(int s) const { return s; }
+  __device__ double x(long long s, int a) const {
     return X[static_cast<size_t>(s) * ld + a] - (xm ? xm[a] : 0.0);
   }
-  __device__ double y(int s, int b) const {
+  __device__ double y(long long s, int b) const {
     return Y[static_cast<size_t>(s) * ld + b] - (ym ? ym[b] : 0.0);
   }
 };
