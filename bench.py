@@ -262,22 +262,45 @@ def main():
     b = S.allocate(p, qd.dtype, dev)
     stream = torch.cuda.current_stream(dev)
 
-    def call(qx, kx, vx, ev=None):
-        if ev: ev[0].record(stream)
-        S.sparsepr_partition(qx, kx, p, b.label_q, b.label_k, b.ws, stream)
-        if ev: ev[1].record(stream)
+    def call(qx, kx, vx, ev=None, strm=None):
+        sx = stream if strm is None else strm
+        if ev: ev[0].record(sx)
+        S.sparsepr_partition(qx, kx, p, b.label_q, b.label_k, b.ws, sx)
+        if ev: ev[1].record(sx)
         S.sparsepr_permute(qx, kx, vx, p, b.label_q, b.label_k, b.perm_q, b.perm_k, b.off_q,
-                           b.off_k, b.qp, b.kp, b.vp, b.ws, stream)
-        if ev: ev[2].record(stream)
-        S.sparsepr_route(b.qp, b.kp, p, b.off_q, b.off_k, b.csr, b.k_per_head, b.ws, stream)
-        if ev: ev[3].record(stream)
+                           b.off_k, b.qp, b.kp, b.vp, b.ws, sx)
+        if ev: ev[2].record(sx)
+        S.sparsepr_route(b.qp, b.kp, p, b.off_q, b.off_k, b.csr, b.k_per_head, b.ws, sx)
+        if ev: ev[3].record(sx)
         S.sparsepr_block_sparse_attn(b.qp, b.kp, b.vp, p, b.off_q, b.off_k, b.csr, b.k_per_head,
-                                     b.o_sparse, b.pairs_sparse, b.ws, stream)
-        if ev: ev[4].record(stream)
+                                     b.o_sparse, b.pairs_sparse, b.ws, sx)
+        if ev: ev[4].record(sx)
         S.sparsepr_probe_correct(b.qp, b.kp, b.vp, p, b.off_q, b.perm_q, b.o_sparse,
                                  b.pairs_sparse, b.out, b.probes, b.pairs_exec, b.ws, None,
-                                 stream)
-        if ev: ev[5].record(stream)
+                                 sx)
+        if ev: ev[5].record(sx)
+
+    def capture_graph():
+        """The five calls captured once into a CUDA graph (the same kernels on the same
+        buffers; the library never synchronises or allocates inside a call). Used for the
+        timed steps only if its replay reproduces the direct call's output bit for bit."""
+        try:
+            ref_out, ref_lab = b.out.clone(), b.label_q.clone()
+            g = torch.cuda.CUDAGraph()
+            cs = torch.cuda.Stream(dev)
+            cs.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cs, capture_error_mode="relaxed"):
+                call(qd, kd, vd, strm=torch.cuda.current_stream(dev))
+            torch.cuda.synchronize(dev)
+            b.out.zero_()
+            g.replay()
+            torch.cuda.synchronize(dev)
+            if torch.equal(b.out, ref_out) and torch.equal(b.label_q, ref_lab):
+                return g
+        except Exception:
+            pass
+        torch.cuda.synchronize(dev)
+        return None
 
     def barrier():
         if world > 1:
@@ -290,6 +313,10 @@ def main():
     pairs_sparse = int(b.pairs_sparse.sum())
     pairs_exec = int(b.pairs_exec.sum())
 
+    graph = capture_graph()
+    if graph is not None:
+        for _ in range(2):
+            graph.replay()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     barrier()
@@ -299,16 +326,31 @@ def main():
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for s in range(args.steps):
-        call(qd, kd, vd, evs[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            call(qd, kd, vd, evs[s])
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop()
     total_ms = t0.elapsed_time(t1)
+    ms = total_ms / args.steps
+    # per-stage times (and the whole call) from direct calls with events between the stages
+    direct_ms = ms
+    barrier()  # (the same collective steps on every rank, graph or not)
+    torch.cuda.synchronize(dev)
+    if graph is not None:
+        t0.record(stream)
+        for s in range(args.steps):
+            call(qd, kd, vd, evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        direct_ms = t0.elapsed_time(t1) / args.steps
+    barrier()
     stage_names = ["partition", "permute", "route", "block_sparse_attn", "probe_correct"]
     stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
                 for i, n in enumerate(stage_names)}
-    ms = total_ms / args.steps
 
     # dense baseline of the same kernel design on the same inputs
     dense_out = torch.empty((w.H, w.N, w.d), dtype=torch.float32, device=dev)
@@ -349,13 +391,13 @@ def main():
         launches, launches_src = gpu_launches_per_call(w), "launch-sequence formula"
 
     # max over ranks
-    vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms], device=dev,
-                        dtype=torch.float64)
+    vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms, direct_ms],
+                        device=dev, dtype=torch.float64)
     tot_pairs = torch.tensor([pairs_exec, pairs_sparse], device=dev, dtype=torch.float64)
     if world > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
         dist.all_reduce(tot_pairs, op=dist.ReduceOp.SUM)
-    ms_max, e2e_max, attn_max, dense_max = vals.tolist()
+    ms_max, e2e_max, attn_max, dense_max, direct_max = vals.tolist()
     P_exec_all, P_sparse_all = tot_pairs.tolist()
 
     if rank == 0:
@@ -369,10 +411,14 @@ def main():
             vs_baseline=None, dtype="bf16", data="synthetic",
             config=dict(workload=workload_desc(w), heads_per_rank=w.H,
                         l2="inputs (697 MB of Q/K/V per call) are larger than the 126 MB L2",
-                        parallelism="replicas: each rank runs its own call (dp%d)" % world),
+                        parallelism="replicas: each rank runs its own call (dp%d)" % world,
+                        launch=("one CUDA graph of the five calls, replayed per step (its output "
+                                "checked bit-identical to a direct call)") if graph is not None
+                        else "the five calls launched directly"),
             attn_call_ms=ms_max,
+            direct_call_ms=direct_max,
             stage_ms=stage_ms,
-            stage_share={n: stage_ms[n] / ms for n in stage_ms},
+            stage_share={n: stage_ms[n] / direct_ms for n in stage_ms},
             rho_exec=pairs_exec / (w.H * w.N * w.N),
             rho_sparse=pairs_sparse / (w.H * w.N * w.N),
             attn_kernel_tflops=attn_tflops,
