@@ -148,3 +148,51 @@ def test_wan13b_720p_head0_sampled():
         pairs = int((np.diff(off_q) * nk[csr].sum(axis=1)).sum())
         assert pairs == int(b.pairs_sparse[h]) == st["pairs_sparse"][h]
         assert int(b.pairs_exec[h]) == pairs + w.M * w.N
+
+
+def _check_partition_and_pairs(b, w, st, heads):
+    """A valid partition per head and, for video-only layers, exact pair
+    accounting from the head's own routes."""
+    for h in heads:
+        off_q, off_k = np_(b.off_q[h]), np_(b.off_k[h])
+        assert off_q[-1] == w.N and off_k[-1] == w.N
+        lab = np_(b.label_q[h])
+        assert np.array_equal(np.diff(off_q), np.bincount(lab, minlength=len(off_q) - 1))
+        if w.n_text == 0:
+            csr = np_(b.csr[h])[:, :int(b.k_per_head[h])]
+            nk = np.diff(off_k)
+            pairs = int((np.diff(off_q) * nk[csr].sum(axis=1)).sum())
+            assert pairs == int(b.pairs_sparse[h]) == st["pairs_sparse"][h]
+            assert int(b.pairs_exec[h]) == pairs + w.M * w.N
+
+
+def test_wan14b_720p_extreme_budgets_sampled():
+    """Wan2.1-14B-shaped layer (its first 8 of 40 heads, with their per-head
+    keep fractions drawn from [0.15, 0.35]) in one call; the heads with the
+    smallest and the largest budget checked against the oracle on sampled
+    rows."""
+    w = synth.workload("wan14b_720p", heads=8)
+    b, (q, k, v) = gpu_run(w)
+    st = _S().sparsepr_read_stats(b.ws)
+    assert st["status"] == 0
+    rows = np.arange(11, w.N, 397)
+    keep = np.asarray(w.keep)
+    for h in sorted({int(keep.argmin()), int(keep.argmax())}):
+        res = oracle_head(w, q, k, v, h, rows=rows)
+        compare_head(b, res, w, h, rows)
+    _check_partition_and_pairs(b, w, st, range(w.H))
+
+
+def test_hunyuan13b_720p_text_sampled():
+    """HunyuanVideo-shaped joint attention (its first 4 of 24 heads): 118,800
+    video tokens and 256 always-kept text tokens, 1500 key and 300 query
+    groups; head 0 checked against the oracle on sampled video rows and text
+    rows (the text query group is last in group-major order)."""
+    w = synth.workload("hunyuan13b_720p", heads=4)
+    b, (q, k, v) = gpu_run(w)
+    st = _S().sparsepr_read_stats(b.ws)
+    assert st["status"] == 0
+    rows = np.concatenate([np.arange(5, w.Nv, 601), np.arange(w.N - w.n_text, w.N, 17)])
+    res = oracle_head(w, q, k, v, 0, rows=rows)
+    compare_head(b, res, w, 0, rows)
+    _check_partition_and_pairs(b, w, st, range(w.H))
