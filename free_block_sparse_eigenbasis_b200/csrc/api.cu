@@ -163,6 +163,21 @@ __global__ void dense_meta_kernel(int32_t* meta, int H, int M, int N) {
   kh[h] = 1;
 }
 
+// One thread waits, through the same bounded mbarrier wait as every kernel
+// of the library, on a barrier that nothing completes; when the limit runs
+// out the wait gives up and the status word gets SPARSEPR_ERR_TIMEOUT.
+__global__ void wait_limit_kernel(DeviceStats* stats) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort)) raise_status(stats, SPARSEPR_ERR_TIMEOUT);
+}
+
 }  // namespace
 
 extern "C" {
@@ -192,6 +207,13 @@ int32_t sparsepr_route_width(const sparsepr_params* p) {
   Layout L;
   compute_layout(*p, &L);
   return L.kmax;
+}
+
+sparsepr_status sparsepr_check_wait_limit(void* ws, void* stream) {
+  if (!ws) return SPARSEPR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return SPARSEPR_ERR_INVALID_ARG;
+  wait_limit_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<DeviceStats*>(ws));
+  return cuda_status(cudaGetLastError());
 }
 
 sparsepr_status sparsepr_reset_stats(void* ws, void* stream) {

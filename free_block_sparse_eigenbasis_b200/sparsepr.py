@@ -22,7 +22,7 @@ BF16, F32 = 0, 1
 EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_partition",
             "sparsepr_permute", "sparsepr_route", "sparsepr_route_width",
             "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
-            "sparsepr_reset_stats")
+            "sparsepr_reset_stats", "sparsepr_check_wait_limit")
 
 
 class Params(ctypes.Structure):
@@ -77,9 +77,10 @@ def _load():
     lib.sparsepr_route_noalloc.restype = st
     lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
     lib.sparsepr_reset_stats.argtypes = [V, V]
+    lib.sparsepr_check_wait_limit.argtypes = [V, V]
     for name in ("sparsepr_partition", "sparsepr_permute", "sparsepr_route",
                  "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
-                 "sparsepr_reset_stats"):
+                 "sparsepr_reset_stats", "sparsepr_check_wait_limit"):
         getattr(lib, name).restype = st
     return lib
 
@@ -193,6 +194,14 @@ def sparsepr_probe_correct(qp, kp, vp, p, off_q, perm_q, o_sparse, pairs_sparse,
                                       _ptr(o_sparse), _ptr(pairs_sparse), _ptr(out),
                                       _ptr(probes), _ptr(pairs_exec), _ptr(fit), _ptr(ws),
                                       ws.numel(), _stream(stream)), "sparsepr_probe_correct")
+
+
+def sparsepr_reset_stats(ws, stream=None):
+    _check(lib.sparsepr_reset_stats(_ptr(ws), _stream(stream)), "sparsepr_reset_stats")
+
+
+def sparsepr_check_wait_limit(ws, stream=None):
+    _check(lib.sparsepr_check_wait_limit(_ptr(ws), _stream(stream)), "sparsepr_check_wait_limit")
 
 
 def sparsepr_read_stats(ws) -> dict:

@@ -242,6 +242,16 @@ sparsepr_status sparsepr_read_stats(const void* ws, sparsepr_stats* out);
  * sparsepr_partition does this itself at the start of every call. */
 sparsepr_status sparsepr_reset_stats(void* ws, void* stream);
 
+/* Check of the device-side failure path, for tests and health checks: one
+ * kernel whose thread waits, through the same bounded mbarrier wait as every
+ * kernel of the library, on a barrier that nothing completes. After the wait
+ * limit (2 s) the wait gives up, SPARSEPR_ERR_TIMEOUT is OR-ed into the status
+ * word of `ws` and the kernel returns; the device and the CUDA context stay
+ * usable. Enqueued on `stream`; read the result with sparsepr_read_stats after
+ * synchronising. Errors: INVALID_ARG for a NULL or not 256-byte-aligned `ws`,
+ * CUDA for a failed launch. */
+sparsepr_status sparsepr_check_wait_limit(void* ws, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -196,3 +196,21 @@ def test_hunyuan13b_720p_text_sampled():
     res = oracle_head(w, q, k, v, 0, rows=rows)
     compare_head(b, res, w, 0, rows)
     _check_partition_and_pairs(b, w, st, range(w.H))
+
+
+def test_bounded_wait_reports_timeout_and_context_stays_usable():
+    """A wait on a barrier that nothing completes gives up after the limit and
+    sets the TIMEOUT bit; the next call on the same context runs normally."""
+    S = _S()
+    w = SMALL[0]
+    p = w.params()
+    ws = torch.zeros(S.workspace_bytes(p), dtype=torch.uint8, device="cuda")
+    S.sparsepr_reset_stats(ws)
+    S.sparsepr_check_wait_limit(ws)
+    torch.cuda.synchronize()
+    st = S.sparsepr_read_stats(ws)
+    assert st["status"] & (1 << S.ERR_TIMEOUT)
+    b, (q, k, v) = gpu_run(w)  # partition resets the status word at the start of its call
+    assert S.sparsepr_read_stats(b.ws)["status"] == 0
+    res = oracle_head(w, q, k, v, 0)
+    compare_head(b, res, w, 0, None)
