@@ -159,6 +159,21 @@ def gpu_launches_per_call(w) -> int:
     return partition + permute + route + attn + probe
 
 
+def reduce_over_ranks(dist, times, pairs):
+    """Job aggregation across ranks, in place: every timing is the slowest rank's (MAX),
+    every pair count the sum over ranks (SUM). dist None: one rank, nothing to do. The
+    same two collectives run on every rank."""
+    if dist is None:
+        return
+    dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    dist.all_reduce(pairs, op=dist.ReduceOp.SUM)
+
+
+def job_tflops(d, pairs_exec_all, ms):
+    """Whole-job executed-pair throughput: 4 d flop per pair (QK^T and PV)."""
+    return 4.0 * d * pairs_exec_all / (ms * 1e-3) / 1e12
+
+
 def run_reference(args, w, rank):
     """The oracle as it stands, on the host cores, on a bounded sample of the
     same workload per step (head 0: full partition, routing and probe fit;
@@ -394,16 +409,14 @@ def main():
     vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms, direct_ms],
                         device=dev, dtype=torch.float64)
     tot_pairs = torch.tensor([pairs_exec, pairs_sparse], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tot_pairs, op=dist.ReduceOp.SUM)
+    reduce_over_ranks(dist if world > 1 else None, vals, tot_pairs)
     ms_max, e2e_max, attn_max, dense_max, direct_max = vals.tolist()
     P_exec_all, P_sparse_all = tot_pairs.tolist()
 
     if rank == 0:
         peaks, src = load_peaks()
         peak = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
-        value = 4.0 * w.d * P_exec_all / (ms_max * 1e-3) / 1e12
+        value = job_tflops(w.d, P_exec_all, ms_max)
         attn_tflops = 4.0 * w.d * pairs_sparse / (stage_ms["block_sparse_attn"] * 1e-3) / 1e12
         line = dict(
             metric=METRIC, value=value, unit="TFLOPS", n_gpus=world, steps=args.steps,
