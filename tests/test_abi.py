@@ -110,3 +110,38 @@ def test_null_pointers_and_small_workspace_rejected():
 def test_status_strings():
     for c in range(7):
         assert S.status_string(c)
+
+
+def test_header_is_plain_c_and_a_c_program_links_and_runs(tmp_path):
+    """The boundary is a C ABI: the header compiles as pedantic C99, and a C
+    program links against the library and gets the same host-side answers
+    as the Python binding (no GPU needed for these calls)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "sparsepr.h"\n'
+        "int main(void) {\n"
+        "  double keep[2] = {0.25, 0.4};\n"
+        "  sparsepr_params p = {0};\n"
+        "  p.H = 2; p.N = 2048; p.d = 128; p.n_text = 0; p.Ck = 64; p.Cq = 16; p.Ms = 256;\n"
+        "  p.n_eig = 8; p.kmeans_iters = 10; p.M = 64; p.r = 16; p.lambda = 1e-2; p.scale = 0.0;\n"
+        "  p.seed = 11; p.keep = keep;\n"
+        '  printf("%zu %d %s\\n", sparsepr_workspace_bytes(&p), (int)sparsepr_route_width(&p),\n'
+        "         sparsepr_status_string(SPARSEPR_ERR_TIMEOUT));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "abi"
+    pkg = os.path.join(root, "free_block_sparse_eigenbasis_b200")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(root, "include"), str(src), "-L", pkg, "-lsparsepr",
+                    "-Wl,-rpath," + pkg, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    p = dict(H=2, N=2048, d=128, n_text=0, Ck=64, Cq=16, Ms=256, n_eig=8, kmeans_iters=10,
+             keep=[0.25, 0.4], M=64, r=16, lam=1e-2, scale=0.0, seed=11)
+    assert int(out[0]) == S.workspace_bytes(p)
+    assert int(out[1]) == S.route_width(p)
+    assert " ".join(out[2:]) == S.status_string(S.ERR_TIMEOUT)
