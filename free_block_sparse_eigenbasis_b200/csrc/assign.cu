@@ -26,9 +26,10 @@
 // current head stay in shared memory and are reloaded when the range crosses
 // into the next head. One warp issues the TMA loads and another the MMAs
 // (each on its own, so neither waits behind the other's barrier polls).
-// Row tiles of 128 stream through a 2-stage TMA ring;
-// the 128 x (<=256) accumulator of each centroid chunk alternates between two
-// TMEM buffers, so the epilogue of one chunk overlaps the MMAs of the next.
+// Row tiles of 128 stream through a TMA ring of 2 to 4 stages (as many as
+// shared memory holds beside the centroid planes); the 128 x (<=256)
+// accumulator of each centroid chunk alternates between two TMEM buffers, so
+// the epilogue of one chunk overlaps the MMAs of the next.
 // The epilogue is four groups of four warps: every group sees all 128 rows
 // (warp w reads TMEM lanes 32 (w % 4) ..) and a quarter of each chunk's
 // columns; each thread keeps four chains (columns k mod 4) of best, second
