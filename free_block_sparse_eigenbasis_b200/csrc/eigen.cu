@@ -250,9 +250,10 @@ __device__ void tri_apply(const double* ra, const double* dl, const double* du, 
 constexpr int kEigThreads = 512;
 constexpr int kEigWarps = kEigThreads / 32;
 
-// One CTA per matrix, ne <= 32 eigenpairs (largest first): bisection and
-// inverse iteration by thread t, clustered Gram-Schmidt by warp 0, then
-// back-transformation by warp t % 8. Writes evals [H, ne] and evecs [H, D, ne].
+// One CTA of 512 threads per matrix, ne <= 32 eigenpairs (largest first):
+// multisection by 16-32 threads per eigenvalue, inverse iteration by thread t
+// (one LU, three solves), Gram-Schmidt inside clusters by all warps, then the
+// back-transformation by warp t % 16. Writes evals [H, ne] and evecs [H, D, ne].
 template <int D>
 constexpr size_t eig_work_bytes() {
   return static_cast<size_t>(4) * D * 32 * 8 + static_cast<size_t>(D) * 32 * 4;
