@@ -414,12 +414,9 @@ __global__ void finalize_pass_kernel(int H, int pass, int32_t* flags, int flag_b
 }
 
 // ---------------------------------------------------------------------------
-// Group means in a fixed order: one warp per group, lanes own coordinates,
-// members summed in ascending position order of the stable sort.
+// Group means in a fixed order over the members in the stable sort's order
+// (so repeated calls give the same bits).
 // ---------------------------------------------------------------------------
-// One CTA of 4 warps per group: warp w sums the w-th quarter of the members
-// (ascending positions, lanes own coordinates), the four partial sums are
-// added in warp order.
 constexpr int kMeanThreads = 256;
 constexpr int kMeanMaxD = 128;
 
@@ -508,8 +505,9 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_kernel(
 // Vector form of the group mean for rows of D * sizeof(T) bytes that split
 // into 16-byte pieces: TPR = D * sizeof(T) / 16 threads per row, each summing
 // EPT = 16 / sizeof(T) columns over the rows lo + rl, lo + rl + RL, ...
-// (RL = 256 / TPR row lanes), then the row lanes' sums are added in a fixed
-// order.
+// (RL = 256 / TPR row lanes, four rows in flight), then the row lanes' sums
+// are combined in a fixed order (within a warp by shuffles, across warps in
+// shared memory).
 template <typename T>
 __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
     const T* X, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
