@@ -55,6 +55,9 @@ SMALL = [
                  n_eig=8, M=32, r=8, keep=(0.2, 0.3), seed=21),
     synth.custom("text_f32_d64_hard_drop", 1, (2, 5, 13), 64, "f32", n_text=9, Ck=10, Cq=4,
                  Ms=64, n_eig=4, M=0, r=4, keep=0.25, seed=22),
+    # bf16 d=64 with e=24: 64-column operand rows on both tensor-core assignment passes
+    synth.custom("bf16_d64_e24", 1, (3, 8, 16), 64, "bf16", Ck=40, Cq=10, Ms=128, n_eig=24,
+                 M=24, r=8, keep=0.3, seed=31),
 ]
 
 
