@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_route_kernel(
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gi = blockIdx.x * kTopkWarps + w;  // (head within the chunk, query group)
   if (gi >= H * Cq) return;
-  const int hl = gi / Cq, g = gi % Cq;
+  const int hl = gi / Cq;  // (the query group is gi % Cq)
   const double* row = S + static_cast<size_t>(gi) * Ck;
   const int k = kh[h0 + hl];
   int* hs = hist[w];
