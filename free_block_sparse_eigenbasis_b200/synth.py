@@ -11,6 +11,7 @@ because trained weights and prompts are not available):
     tiny              1 head,  d=64,  fp32, N=256 on a 4x8x8 grid
     wan13b_480p      12 heads, d=128, bf16, N=32,760 on 21x30x52
     wan13b_720p      12 heads, d=128, bf16, N=75,600 on 21x45x80
+    wan13b_720p_rho25  the same layer with keep 0.244 (executed-pair density about 0.25)
     wan14b_720p      40 heads, d=128, bf16, N=75,600, per-head keep in [0.15,0.35]
     hunyuan13b_720p  24 heads, d=128, bf16, N=118,800 video + 256 text tokens
 
@@ -106,6 +107,13 @@ def workload(name: str, heads: Optional[int] = None) -> Workload:
         w = Workload(name, 12, (21, 45, 80), 128, "bf16", 128, 0.5, 0.1, 0,
                      Ck=1000, Cq=200, Ms=1024, n_eig=16, kmeans_iters=10,
                      keep=(0.22,) * 12, M=512, r=32, lam=1e-2, scale=0.0,
+                     seed=2)
+    elif name == "wan13b_720p_rho25":
+        # the 720p layer with the keep fraction raised so that the realised
+        # executed-pair density (routed pairs + probe rows) is about 0.25
+        w = Workload(name, 12, (21, 45, 80), 128, "bf16", 128, 0.5, 0.1, 0,
+                     Ck=1000, Cq=200, Ms=1024, n_eig=16, kmeans_iters=10,
+                     keep=(0.244,) * 12, M=512, r=32, lam=1e-2, scale=0.0,
                      seed=2)
     elif name == "wan14b_720p":
         w = Workload(name, 40, (21, 45, 80), 128, "bf16", 128, 0.5, 0.1, 0,
