@@ -4,9 +4,13 @@ d = 128, bf16, 1000 key groups, 200 query groups, keep 0.22, M = 512 probes,
 r = 32, lambda = 1e-2. Inputs are seeded synthetic Q/K/V of that shape.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--no-cpu-baseline]
 
 One step = one whole call (partition, permute, route, block-sparse attention,
-probe-fitted correction) over the 12 heads, inputs resident in HBM. Under
+probe-fitted correction) over the 12 heads, inputs resident in HBM. The timed
+steps replay one CUDA graph of the five calls when its replay reproduces a
+direct call bit for bit (else the calls are launched directly); the per-stage
+times come from direct calls with events between the stages. Under
 torchrun every rank runs its own call on its own GPU (heads are independent;
 no collective on the data path) and the job value is the sum of the ranks'
 executed pairs over the slowest rank's time.
