@@ -315,11 +315,12 @@ def main():
             g.replay()
             torch.cuda.synchronize(dev)
             if torch.equal(b.out, ref_out) and torch.equal(b.label_q, ref_lab):
-                return g
-        except Exception:
-            pass
+                return g, None
+            reason = "graph replay differed from the direct call"
+        except Exception as exc:  # capture refused: fall back to direct launches, say why
+            reason = "graph capture failed: %s" % str(exc).splitlines()[0][:120]
         torch.cuda.synchronize(dev)
-        return None
+        return None, reason
 
     def barrier():
         if world > 1:
@@ -332,7 +333,7 @@ def main():
     pairs_sparse = int(b.pairs_sparse.sum())
     pairs_exec = int(b.pairs_exec.sum())
 
-    graph = capture_graph()
+    graph, graph_note = capture_graph()
     if graph is not None:
         for _ in range(2):
             graph.replay()
@@ -431,7 +432,7 @@ def main():
                         parallelism="replicas: each rank runs its own call (dp%d)" % world,
                         launch=("one CUDA graph of the five calls, replayed per step (its output "
                                 "checked bit-identical to a direct call)") if graph is not None
-                        else "the five calls launched directly"),
+                        else "the five calls launched directly (%s)" % graph_note),
             attn_call_ms=ms_max,
             direct_call_ms=direct_max,
             stage_ms=stage_ms,
