@@ -101,7 +101,7 @@ typedef struct {
   int64_t pairs_sparse[SPARSEPR_MAX_HEADS]; /* routed (row, key) pairs per head */
   int64_t pairs_exec[SPARSEPR_MAX_HEADS];   /* pairs_sparse + M*N (probe rows) */
   int64_t recheck_rows[2]; /* k-means rows decided again in fp64 (keys, queries), all passes */
-  int32_t eig_sweeps[2];   /* reserved, 0 (the eigensolver runs no sweeps) */
+  int32_t eig_sweeps[2];   /* Jacobi sweeps, max over heads: [1] = probe residual Gram when r > 32 (the tridiagonal solver serves r <= 32 and M_K, and leaves 0) */
 } sparsepr_stats;
 
 /* Bytes of device workspace the five calls need for these parameters
