@@ -371,3 +371,64 @@ def test_text_tokens_reading():
     D = O.dense_attention(q[res.perm_q], k[res.perm_k], v[res.perm_k], 1 / math.sqrt(w.d))
     trows = np.arange(res.off_q[w.Cq], w.N)
     assert np.abs(res.out[trows] - D[trows]).max() < 1e-12
+
+
+def test_partition_wiring_is_a_two_stage_lloyd_fixed_point():
+    """End-to-end wiring of the partition stage [SPR 2.A]: with e = d the
+    key labels must be a Lloyd fixed point of the response-profile metric
+    M_K = Q_s^T Q_s / M_s in the ORIGINAL key space (no eigen solver needed:
+    |Lambda^1/2 U^T (k - m)|^2 = (k - m)^T M_K (k - m)), and the query labels
+    a Lloyd fixed point of the logit profiles against the original-space
+    means of the FINAL key groups. Everything here is recomputed with plain
+    loops from the labels alone; a query stage fed other key groups (initial
+    ones, z-space means, unfinished Lloyd) breaks the second check."""
+    w = synth.custom("wire", 1, (2, 4, 8), 16, "f32", n_comp=6, sigma=0.4,
+                     noise_var=0.05, Ck=6, Cq=4, Ms=32, n_eig=16,
+                     kmeans_iters=200, M=8, r=4, seed=3, keep=0.5)
+    q, k, v = synth.generate(w)
+    q, k = synth.as_f64(q[0]), synth.as_f64(k[0])
+    res = O.run_head(q, k, synth.as_f64(v[0]), w.params(), 0, partition_only=True)
+    N, d = q.shape
+    assert res.info["key_passes"] < w.kmeans_iters
+    assert res.info["query_passes"] < w.kmeans_iters
+    lk, lq = res.label_k, res.label_q
+    assert len(set(lk.tolist())) == w.Ck and len(set(lq.tolist())) == w.Cq
+
+    def mean_rows(X, lab, c):
+        acc = [0.0] * X.shape[1]
+        cnt = 0
+        for i in range(X.shape[0]):
+            if lab[i] == c:
+                cnt += 1
+                for a in range(X.shape[1]):
+                    acc[a] += X[i, a]
+        return [x / cnt for x in acc]
+
+    def check_fixed_point(dist_rows, lab):
+        # the chosen group is a nearest one (up to rounding of the sums)
+        for i, row in enumerate(dist_rows):
+            lo = min(row)
+            assert row[lab[i]] <= lo + 1e-9 * max(1.0, abs(lo)), (i, lab[i], row)
+
+    # key stage: sampled rows by integer arithmetic, M_K by explicit sums
+    Ms = w.Ms
+    srows = [((2 * s + 1) * N) // (2 * Ms) for s in range(Ms)]
+    MK = [[sum(q[r, a] * q[r, b] for r in srows) / Ms for b in range(d)] for a in range(d)]
+    mk = [mean_rows(k, lk, c) for c in range(w.Ck)]
+    dk = []
+    for i in range(N):
+        row = []
+        for c in range(w.Ck):
+            t = [k[i, a] - mk[c][a] for a in range(d)]
+            row.append(sum(t[a] * MK[a][b] * t[b] for a in range(d) for b in range(d)))
+        dk.append(row)
+    check_fixed_point(dk, lk)
+
+    # query stage: logit profiles against the final key groups' means
+    scale = 1.0 / math.sqrt(d)
+    P = np.array([[scale * sum(mk[c][a] * q[i, a] for a in range(d)) for c in range(w.Ck)]
+                  for i in range(N)])
+    pq = [mean_rows(P, lq, g) for g in range(w.Cq)]
+    dq = [[sum((P[i, c] - pq[g][c]) ** 2 for c in range(w.Ck)) for g in range(w.Cq)]
+          for i in range(N)]
+    check_fixed_point(dq, lq)
