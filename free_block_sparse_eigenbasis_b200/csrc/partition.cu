@@ -659,7 +659,9 @@ __global__ void write_labels_kernel(const int32_t* lab, int H, int N, int Nv, in
 cudaError_t launch_fy_init(int H, int Nv, int Ck, int Cq, uint64_t seed, int32_t* init_k,
                            int32_t* init_q, cudaStream_t st) {
   const int shb = 2 * kFyTable * 4;
-  cudaFuncSetAttribute(fy_init_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
+  const cudaError_t e =
+      cudaFuncSetAttribute(fy_init_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
+  if (e != cudaSuccess) return e;
   fy_init_kernel<<<dim3(H, 2), 256, shb, st>>>(Nv, Ck, Cq, seed, init_k, init_q);
   return cudaGetLastError();
 }
@@ -700,12 +702,14 @@ cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, 
   const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;
   dim3 grid((Nv + kZRows - 1) / kZRows, H);
   if (bf16) {
-    cudaFuncSetAttribute(zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(shb));
+    const cudaError_t e = cudaFuncSetAttribute(
+        zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shb));
+    if (e != cudaSuccess) return e;
     zproj_kernel<<<grid, kZThreads, shb, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv, d, e, wk, z);
   } else {
-    cudaFuncSetAttribute(zproj_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(shb));
+    const cudaError_t e = cudaFuncSetAttribute(
+        zproj_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shb));
+    if (e != cudaSuccess) return e;
     zproj_kernel<<<grid, kZThreads, shb, st>>>(static_cast<const float*>(k), N, Nv, d, e, wk, z);
   }
   return cudaGetLastError();
