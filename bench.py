@@ -178,72 +178,88 @@ def job_tflops(d, pairs_exec_all, ms):
     return 4.0 * d * pairs_exec_all / (ms * 1e-3) / 1e12
 
 
+ORACLE_GROUP_STRIDE = 16
+
+
+def oracle_cores():
+    cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return cores
+
+
+def oracle_call_time(O, w, qf, kf, vf):
+    """The oracle as it stands on one bounded sample of the workload. Head 0
+    runs in full except for the per-row stage (partition, routing, probes
+    and their dense rows, fit: run_head with no output rows); the per-row
+    stage (masked attention + correction) is then timed on every row of every
+    ORACLE_GROUP_STRIDE-th query group (whole groups, so the rows are batched
+    per group as in a full run) and scaled to all N rows. Call time = H x the
+    head time. Returns (call seconds, executed flops of the call)."""
+    t0 = time.perf_counter()
+    res = O.run_head(qf, kf, vf, w.params(), 0, rows=np.zeros(0, dtype=np.int64))
+    t_fixed = time.perf_counter() - t0
+    Qp, Kp, Vp = qf[res.perm_q], kf[res.perm_k], vf[res.perm_k]
+    nt = w.n_text
+    text = (w.Ck,) if nt else ()
+    groups = list(range(0, w.Cq, ORACLE_GROUP_STRIDE)) + ([w.Cq] if nt else [])
+    masks = {g: (np.ones(w.N, dtype=bool) if g == w.Cq else
+                 O.kept_key_mask(res.csr[g], res.off_k, w.N, text)) for g in groups}
+    rows = np.concatenate([np.arange(res.off_q[g], res.off_q[g + 1]) for g in groups])
+    t0 = time.perf_counter()
+    Os = O.masked_attention_rows(Qp, Kp, Vp, rows,
+                                 lambda i: int(np.searchsorted(res.off_q, i, side="right") - 1),
+                                 masks.__getitem__, O.resolve_scale(w.scale, w.d))
+    _ = Os + res.bp[None, :] + Os @ res.Bp
+    t_rows = time.perf_counter() - t0
+    t_head = t_fixed + t_rows * w.N / max(rows.size, 1)
+    return w.H * t_head, 4.0 * w.d * res.pairs_exec * w.H
+
+
+def oracle_sample_desc(w, t_call):
+    return ("head 0 of %d in full except the per-row stage (masked attention + correction), which "
+            "is timed on the rows of every %dth query group and scaled to all %d rows; call time "
+            "= %d x head time = %.3g s" % (w.H, ORACLE_GROUP_STRIDE, w.N, w.H, t_call))
+
+
 def run_reference(args, w, rank):
-    """The oracle as it stands, on the host cores, on a bounded sample of the
-    same workload per step (head 0: full partition, routing and probe fit;
-    sparse attention + correction on every 64th group-major row)."""
+    """The oracle as it stands, on the host cores, one bounded sample of the
+    same workload per step (oracle_call_time)."""
     from oracle import sparsepr_oracle as O
     if rank != 0:
         return
     q, k, v = synth.generate(w, heads=[0])
     qf, kf, vf = synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0])
-    stride = 64
-    rows = np.arange(0, w.N, stride)
     times = []
-    res = None
+    flops = 0.0
     for s in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        res = O.run_head(qf, kf, vf, w.params(), 0, rows=rows)
-        t1 = time.perf_counter()
+        t_call, flops = oracle_call_time(O, w, qf, kf, vf)
         if s >= args.warmup:
-            times.append(t1 - t0)
-    t_head = statistics.median(times)
-    # extrapolate: the per-row part scales by the stride, the rest is per head
-    t_rows = t_head * 0.0
-    t_call = w.H * t_head  # conservative: fixed part dominates the sample
-    flops = 4.0 * w.d * res.pairs_exec * w.H
+            times.append(t_call)
+    t_call = statistics.median(times)
     value = flops / t_call / 1e12
-    cores = os.cpu_count()
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        pass
-    sample = ("head 0 of %d: full partition/route/probe fit, sparse attention + correction on "
-              "every %dth group-major row; call time = %d x head time (rows not extrapolated)"
-              % (w.H, stride, w.H))
     line = dict(metric=METRIC, value=value, unit="TFLOPS", n_gpus=args.gpus, steps=args.steps,
                 warmup=args.warmup, ms_per_step=t_call * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
                 impl="reference",
                 config=dict(workload=workload_desc(w)),
-                cpu_baseline=dict(value=value, unit="TFLOPS", cores=cores, kind="oracle",
-                                  sample=sample),
+                cpu_baseline=dict(value=value, unit="TFLOPS", cores=oracle_cores(), kind="oracle",
+                                  sample=oracle_sample_desc(w, t_call)),
                 e2e=dict(value=value, unit="TFLOPS", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
 
 
 def cpu_baseline_sample(w):
-    """Oracle (as it stands) on a bounded sample: head 0, every 64th row."""
+    """The oracle (as it stands) on one bounded sample (oracle_call_time)."""
     from oracle import sparsepr_oracle as O
     q, k, v = synth.generate(w, heads=[0])
-    rows = np.arange(0, w.N, 64)
-    t0 = time.perf_counter()
-    res = O.run_head(synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0]), w.params(), 0,
-                     rows=rows)
-    t_head = time.perf_counter() - t0
-    t_call = w.H * t_head
-    cores = os.cpu_count()
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        pass
-    return dict(value=4.0 * w.d * res.pairs_exec * w.H / t_call / 1e12, unit="TFLOPS",
-                cores=cores, kind="oracle",
-                sample="head 0 of %d (full partition/route/probe fit, sparse attention + "
-                       "correction on every 64th row), call time = %d x %.1f s"
-                       % (w.H, w.H, t_head))
+    t_call, flops = oracle_call_time(O, w, synth.as_f64(q[0]), synth.as_f64(k[0]),
+                                     synth.as_f64(v[0]))
+    return dict(value=flops / t_call / 1e12, unit="TFLOPS", cores=oracle_cores(), kind="oracle",
+                sample=oracle_sample_desc(w, t_call))
 
 
 def main():
