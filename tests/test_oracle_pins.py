@@ -176,6 +176,25 @@ def test_keep_budget_cases():
         assert O.keep_budget(keep, Ck) == k, (keep, Ck)
 
 
+def test_range_means_hand_example_and_label_form():
+    """Block-score centroids are the mean rows of the group-major ranges
+    [SVOO block selection]: a hand example with an empty range, and on random
+    labels the same means taken in the original token order by label."""
+    Xp = np.array([[1.0, 2.0], [3.0, 4.0], [5.0, 6.0]])
+    assert O.range_means(Xp, np.array([0, 2, 2, 3])).tolist() == [[2.0, 3.0], [0.0, 0.0],
+                                                                  [5.0, 6.0]]
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((200, 3))
+    lab = rng.integers(0, 9, size=200)
+    lab[lab == 4] = 5  # group 4 empty
+    perm, _, off = O.group_major(lab, 9)
+    got = O.range_means(X[perm], off)
+    for c in range(9):
+        members = [i for i in range(200) if lab[i] == c]
+        want = np.zeros(3) if not members else sum(X[i] for i in members) / len(members)
+        assert np.allclose(got[c], want, rtol=0, atol=1e-13)
+
+
 def test_route_hand_example():
     ge = GOLD["route_example"]
     for k, want in ge["k_to_csr"]:
