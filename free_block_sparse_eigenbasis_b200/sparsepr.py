@@ -109,8 +109,45 @@ def make_params(p: dict):
     return prm, arr
 
 
-def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+_DEVICE_TYPE = "cuda"  # tensors handed to the library live on this device type
+
+
+def _arg(t, name: str, shape=None, dtype=None):
+    """Device pointer of a tensor argument after the checks the C ABI cannot
+    make from a bare pointer: shape, dtype, dense row-major layout and a CUDA
+    device. Raises ValueError / TypeError before anything is enqueued."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous (row-major)" % name)
+    if t.device.type != _DEVICE_TYPE:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ws(ws, name: str = "ws"):
+    """(pointer, bytes) of the workspace: a contiguous CUDA byte buffer."""
+    return _arg(ws, name, (ws.numel(),) if isinstance(ws, torch.Tensor) else None,
+                torch.uint8), ws.numel()
+
+
+def _dims(p: dict):
+    """H, N, d and the group-offset widths (text tokens add one group per side)."""
+    H, N, d = int(p["H"]), int(p["N"]), int(p["d"])
+    text = 1 if int(p.get("n_text", 0)) > 0 else 0
+    return H, N, d, int(p["Cq"]) + text + 1, int(p["Ck"]) + text + 1
+
+
+def _qkv(p: dict, names_tensors):
+    """Checks the [H, N, d] inputs of one dtype (bf16 or fp32, set by the first)."""
+    H, N, d = int(p["H"]), int(p["N"]), int(p["d"])
+    dt = names_tensors[0][1].dtype if isinstance(names_tensors[0][1], torch.Tensor) else None
+    ptrs = [_arg(t, n, (H, N, d), dt) for n, t in names_tensors]
+    return ptrs, _dtype_code(names_tensors[0][1])
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -144,26 +181,50 @@ def route_width(p: dict) -> int:
 
 # ---- the five calls, same names as the C ABI --------------------------------
 
+I32, I64 = torch.int32, torch.int64
+
+
 def sparsepr_partition(q, k, p, label_q, label_k, ws, stream=None):
     prm, keep = make_params(p)
-    _check(lib.sparsepr_partition(_ptr(q), _ptr(k), _dtype_code(q), ctypes.byref(prm),
-                                  _ptr(label_q), _ptr(label_k), _ptr(ws), ws.numel(),
+    H, N, d, _, _ = _dims(p)
+    (pq, pk), dt = _qkv(p, [("q", q), ("k", k)])
+    wp, wb = _ws(ws)
+    _check(lib.sparsepr_partition(pq, pk, dt, ctypes.byref(prm),
+                                  _arg(label_q, "label_q", (H, N), I32),
+                                  _arg(label_k, "label_k", (H, N), I32), wp, wb,
                                   _stream(stream)), "sparsepr_partition")
 
 
 def sparsepr_permute(q, k, v, p, label_q, label_k, perm_q, perm_k, off_q, off_k, qp, kp, vp, ws,
                      stream=None):
     prm, keep = make_params(p)
-    _check(lib.sparsepr_permute(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), ctypes.byref(prm),
-                                _ptr(label_q), _ptr(label_k), _ptr(perm_q), _ptr(perm_k),
-                                _ptr(off_q), _ptr(off_k), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(ws),
-                                ws.numel(), _stream(stream)), "sparsepr_permute")
+    H, N, d, wq, wk = _dims(p)
+    (pq, pk, pv, pqp, pkp, pvp), dt = _qkv(p, [("q", q), ("k", k), ("v", v), ("qp", qp),
+                                              ("kp", kp), ("vp", vp)])
+    wp, wb = _ws(ws)
+    _check(lib.sparsepr_permute(pq, pk, pv, dt, ctypes.byref(prm),
+                                _arg(label_q, "label_q", (H, N), I32),
+                                _arg(label_k, "label_k", (H, N), I32),
+                                _arg(perm_q, "perm_q", (H, N), I32),
+                                _arg(perm_k, "perm_k", (H, N), I32),
+                                _arg(off_q, "off_q", (H, wq), I32),
+                                _arg(off_k, "off_k", (H, wk), I32), pqp, pkp, pvp, wp, wb,
+                                _stream(stream)), "sparsepr_permute")
+
+
+def _route_args(qp, kp, p, off_q, off_k, csr, k_per_head):
+    H, N, d, wq, wk = _dims(p)
+    (pq, pk), dt = _qkv(p, [("qp", qp), ("kp", kp)])
+    return (pq, pk, dt, _arg(off_q, "off_q", (H, wq), I32), _arg(off_k, "off_k", (H, wk), I32),
+            _arg(csr, "csr", (H, int(p["Cq"]), route_width(p)), I32),
+            _arg(k_per_head, "k_per_head", (H,), I32))
 
 
 def sparsepr_route(qp, kp, p, off_q, off_k, csr, k_per_head, ws, stream=None):
     prm, keep = make_params(p)
-    _check(lib.sparsepr_route(_ptr(qp), _ptr(kp), _dtype_code(qp), ctypes.byref(prm), _ptr(off_q),
-                              _ptr(off_k), _ptr(csr), _ptr(k_per_head), _ptr(ws), ws.numel(),
+    pq, pk, dt, poq, pok, pcsr, pkh = _route_args(qp, kp, p, off_q, off_k, csr, k_per_head)
+    wp, wb = _ws(ws)
+    _check(lib.sparsepr_route(pq, pk, dt, ctypes.byref(prm), poq, pok, pcsr, pkh, wp, wb,
                               _stream(stream)), "sparsepr_route")
 
 
@@ -171,42 +232,56 @@ def sparsepr_route_noalloc(qp, kp, p, off_q, off_k, csr, k_per_head, stream=None
     """sparsepr_route without a workspace (its scratch is a fixed device array
     inside the library); for callers that cannot allocate device memory."""
     prm, keep = make_params(p)
-    _check(lib.sparsepr_route_noalloc(_ptr(qp), _ptr(kp), _dtype_code(qp), ctypes.byref(prm),
-                                      _ptr(off_q), _ptr(off_k), _ptr(csr), _ptr(k_per_head),
+    pq, pk, dt, poq, pok, pcsr, pkh = _route_args(qp, kp, p, off_q, off_k, csr, k_per_head)
+    _check(lib.sparsepr_route_noalloc(pq, pk, dt, ctypes.byref(prm), poq, pok, pcsr, pkh,
                                       _stream(stream)), "sparsepr_route_noalloc")
 
 
 def sparsepr_block_sparse_attn(qp, kp, vp, p, off_q, off_k, csr, k_per_head, o_sparse,
                                pairs_sparse, ws, stream=None):
     prm, keep = make_params(p)
-    _check(lib.sparsepr_block_sparse_attn(_ptr(qp), _ptr(kp), _ptr(vp), _dtype_code(qp),
-                                          ctypes.byref(prm), _ptr(off_q), _ptr(off_k), _ptr(csr),
-                                          _ptr(k_per_head), _ptr(o_sparse), _ptr(pairs_sparse),
-                                          _ptr(ws), ws.numel(), _stream(stream)),
-           "sparsepr_block_sparse_attn")
+    H, N, d, _, _ = _dims(p)
+    pq, pk, dt, poq, pok, pcsr, pkh = _route_args(qp, kp, p, off_q, off_k, csr, k_per_head)
+    (pv,), _ = _qkv(p, [("vp", vp)])
+    if vp.dtype != qp.dtype:
+        raise TypeError("vp has dtype %s, expected %s" % (vp.dtype, qp.dtype))
+    wp, wb = _ws(ws)
+    _check(lib.sparsepr_block_sparse_attn(pq, pk, pv, dt, ctypes.byref(prm), poq, pok, pcsr, pkh,
+                                          _arg(o_sparse, "o_sparse", (H, N, d), torch.float32),
+                                          _arg(pairs_sparse, "pairs_sparse", (H,), I64), wp, wb,
+                                          _stream(stream)), "sparsepr_block_sparse_attn")
 
 
 def sparsepr_probe_correct(qp, kp, vp, p, off_q, perm_q, o_sparse, pairs_sparse, out, probes,
                            pairs_exec, ws, fit=None, stream=None):
     prm, keep = make_params(p)
-    _check(lib.sparsepr_probe_correct(_ptr(qp), _ptr(kp), _ptr(vp), _dtype_code(qp),
-                                      ctypes.byref(prm), _ptr(off_q), _ptr(perm_q),
-                                      _ptr(o_sparse), _ptr(pairs_sparse), _ptr(out),
-                                      _ptr(probes), _ptr(pairs_exec), _ptr(fit), _ptr(ws),
-                                      ws.numel(), _stream(stream)), "sparsepr_probe_correct")
+    H, N, d, wq, _ = _dims(p)
+    M = int(p["M"])
+    (pq, pk, pv, pout), dt = _qkv(p, [("qp", qp), ("kp", kp), ("vp", vp), ("out", out)])
+    wp, wb = _ws(ws)
+    _check(lib.sparsepr_probe_correct(pq, pk, pv, dt, ctypes.byref(prm),
+                                      _arg(off_q, "off_q", (H, wq), I32),
+                                      _arg(perm_q, "perm_q", (H, N), I32),
+                                      _arg(o_sparse, "o_sparse", (H, N, d), torch.float32),
+                                      _arg(pairs_sparse, "pairs_sparse", (H,), I64), pout,
+                                      _arg(probes, "probes", (H, M) if M > 0 else None, I32),
+                                      _arg(pairs_exec, "pairs_exec", (H,), I64),
+                                      None if fit is None else
+                                      _arg(fit, "fit", (H, d * d + d), torch.float64),
+                                      wp, wb, _stream(stream)), "sparsepr_probe_correct")
 
 
 def sparsepr_reset_stats(ws, stream=None):
-    _check(lib.sparsepr_reset_stats(_ptr(ws), _stream(stream)), "sparsepr_reset_stats")
+    _check(lib.sparsepr_reset_stats(_ws(ws)[0], _stream(stream)), "sparsepr_reset_stats")
 
 
 def sparsepr_check_wait_limit(ws, stream=None):
-    _check(lib.sparsepr_check_wait_limit(_ptr(ws), _stream(stream)), "sparsepr_check_wait_limit")
+    _check(lib.sparsepr_check_wait_limit(_ws(ws)[0], _stream(stream)), "sparsepr_check_wait_limit")
 
 
 def sparsepr_read_stats(ws) -> dict:
     s = Stats()
-    _check(lib.sparsepr_read_stats(_ptr(ws), ctypes.byref(s)), "sparsepr_read_stats")
+    _check(lib.sparsepr_read_stats(_ws(ws)[0], ctypes.byref(s)), "sparsepr_read_stats")
     H = max(0, min(s.H, MAX_HEADS))
     return dict(status=int(s.status), H=H, key_passes=list(s.key_passes[:H]),
                 query_passes=list(s.query_passes[:H]), pairs_sparse=list(s.pairs_sparse[:H]),
