@@ -33,7 +33,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_take_slowest_time_and_summed_pairs():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     want = [21.0, 39.0, 9.8, 32.5, 22.7, 2 * 1.7e10 + 1, 2 * 1.5e10 + 2]
     for r in range(world):
