@@ -187,6 +187,21 @@ def query_partition(q_video, CK, Cq, iters, seed, head, scale):
     return labels, dict(passes=passes)
 
 
+def semantic_partition(q_video, k_video, Ck, Cq, iters, seed, head):
+    """The comparison partition of the ablations [SPR 2.A results; SPR 4,
+    ablations]: keys and queries clustered separately by plain Euclidean
+    k-means on their own rows, no response coupling. Reading: same
+    initialisation draws and pass cap as the response-coupled partition.
+    Returns (key labels, query labels, key info, query info)."""
+    init_k = init_indices(k_video.shape[0], Ck, seed, head, 0)
+    lab_k, _, kp = lloyd(k_video, init_k, iters)
+    init_q = init_indices(q_video.shape[0], Cq, seed, head, 1)
+    lab_q, _, qp = lloyd(q_video, init_q, iters)
+    nan = np.full((q_video.shape[1], q_video.shape[1]), np.nan)
+    return lab_k, lab_q, dict(passes=kp, MK=nan, lam=np.zeros(0), U=np.zeros((0, 0))), \
+        dict(passes=qp)
+
+
 # ---------------------------------------------------------------------------
 # Stage 2: group-major layout  [SPR 2.C]
 # ---------------------------------------------------------------------------
@@ -377,7 +392,9 @@ def run_head(q, k, v, p: dict, head: int, rows=None, partition_only=False) -> He
     """The whole per-call path on one head (q, k, v: [N, d] float64).
 
     ``p`` holds the method parameters (Ck, Cq, Ms, n_eig, kmeans_iters, keep
-    [per head], M, r, lam, scale, seed, n_text). ``rows`` restricts the
+    [per head], M, r, lam, scale, seed, n_text; optionally partition =
+    "response" (default) or "semantic", the ablations' uncoupled k-means on
+    raw Q and K rows). ``rows`` restricts the
     sparse-attention and corrected outputs to those group-major rows
     (default: all rows); partition, routing, probes and the fit are always
     computed in full.
@@ -398,10 +415,13 @@ def run_head(q, k, v, p: dict, head: int, rows=None, partition_only=False) -> He
     qv, kv = q[:Nv], k[:Nv]
 
     # Stage 1 [SPR 2.A]
-    lab_k_v, kinfo = key_partition(kv, qv, Ck, int(p["Ms"]), int(p["n_eig"]),
-                                   iters, seed, head)
-    CK_part = group_means(kv, lab_k_v, Ck)  # original-space K/V group centroids
-    lab_q_v, qinfo = query_partition(qv, CK_part, Cq, iters, seed, head, scale)
+    if p.get("partition", "response") == "semantic":
+        lab_k_v, lab_q_v, kinfo, qinfo = semantic_partition(qv, kv, Ck, Cq, iters, seed, head)
+    else:
+        lab_k_v, kinfo = key_partition(kv, qv, Ck, int(p["Ms"]), int(p["n_eig"]),
+                                       iters, seed, head)
+        CK_part = group_means(kv, lab_k_v, Ck)  # original-space K/V group centroids
+        lab_q_v, qinfo = query_partition(qv, CK_part, Cq, iters, seed, head, scale)
     label_k = np.concatenate([lab_k_v, np.full(nt, Ck, dtype=np.int64)])
     label_q = np.concatenate([lab_q_v, np.full(nt, Cq, dtype=np.int64)])
     Ckt, Cqt = Ck + (1 if nt else 0), Cq + (1 if nt else 0)

@@ -130,3 +130,26 @@ def test_residual_energy_closed_forms():
     Rb = X @ B1
     e = D.residual_energy(_fit_result(X, Rb, 0.0, 2))
     assert e["explainable"] > 1 - 1e-12 and e["orthogonal_projected"] < 1e-20
+
+
+def test_semantic_partition_is_plain_lloyd_on_raw_rows_and_expands_support():
+    """The ablations' semantic partition: keys and queries each a Lloyd fixed
+    point of plain Euclidean distance on their own rows (checked with loops
+    from the labels alone); the rest of the call is unchanged, so its
+    invariants still hold."""
+    w = synth.custom("sem", 1, (2, 4, 8), 16, "f32", n_comp=6, sigma=0.4, noise_var=0.05, Ck=6,
+                     Cq=4, Ms=32, n_eig=16, kmeans_iters=200, M=8, r=4, seed=3, keep=0.5)
+    q, k, v = synth.generate(w)
+    q, k, v = synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0])
+    p = dict(w.params(), partition="semantic")
+    res = O.run_head(q, k, v, p, 0)
+    assert res.info["key_passes"] < w.kmeans_iters and res.info["query_passes"] < w.kmeans_iters
+    for X, lab, C in ((k, res.label_k, w.Ck), (q, res.label_q, w.Cq)):
+        assert len(set(lab.tolist())) == C
+        means = [[sum(X[i, a] for i in range(w.N) if lab[i] == c) / int((lab == c).sum())
+                  for a in range(w.d)] for c in range(C)]
+        for i in range(w.N):
+            dist = [sum((X[i, a] - means[c][a]) ** 2 for a in range(w.d)) for c in range(C)]
+            assert dist[lab[i]] <= min(dist) + 1e-9 * max(1.0, min(dist))
+    assert np.all(np.isfinite(res.out)) and res.pairs_exec == res.pairs_sparse + w.M * w.N
+    assert np.array_equal(np.sort(res.perm_q), np.arange(w.N))
