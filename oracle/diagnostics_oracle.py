@@ -127,3 +127,43 @@ def residual_energy(res: O.HeadResult) -> dict:
     return dict(total=tot, explainable=float((RP * RP).sum()) / tot,
                 orthogonal_fit=float((F * F).sum()) / tot,
                 orthogonal_projected=float((Fp * Fp).sum()) / tot)
+
+
+# ---------------------------------------------------------------------------
+# Per-head density profile  ["Attention Sparsity is Input-Stable: Training-Free
+# Sparse Attention for Video Generation via Offline Sparsity Profiling and
+# Online QK Co-Clustering" (papernotes.org note), "key designs", offline
+# layer-wise sparsity profiling]
+#
+# Readings: a row's density is the smallest fraction of its N attention
+# weights whose sum reaches tau (weights taken largest first); a head's
+# density on one input is the mean of its rows' densities over the rows
+# examined; the Gaussian over the calibration inputs is the maximum-
+# likelihood fit (population standard deviation); its upper alpha quantile is
+# the conservative density, clipped to [0, 1], and the sparsity is 1 minus it.
+# ---------------------------------------------------------------------------
+
+def row_density(weights: np.ndarray, tau: float) -> float:
+    """Smallest fraction of the row's weights (largest first) whose sum
+    reaches tau."""
+    w = np.sort(np.asarray(weights, dtype=np.float64))[::-1]
+    run = np.cumsum(w)
+    n = int(np.searchsorted(run, tau - 1e-15, side="left")) + 1
+    return min(n, w.size) / w.size
+
+
+def head_density(Q: np.ndarray, K: np.ndarray, rows: np.ndarray, scale: float,
+                 tau: float) -> float:
+    """Mean row density of the listed query rows' full softmax over K."""
+    W = dense_weights(Q, K, np.asarray(rows, dtype=np.int64), scale)
+    return float(np.mean([row_density(W[t], tau) for t in range(W.shape[0])]))
+
+
+def conservative_density(samples, alpha: float) -> dict:
+    """Gaussian fit of one head's densities over calibration inputs and its
+    upper alpha quantile mu + z_alpha sigma; sparsity = 1 - that density."""
+    from scipy.stats import norm
+    x = np.asarray(samples, dtype=np.float64)
+    mu, sigma = float(x.mean()), float(x.std())
+    d_hat = min(1.0, max(0.0, mu + float(norm.ppf(alpha)) * sigma))
+    return dict(mu=mu, sigma=sigma, density=d_hat, sparsity=1.0 - d_hat)

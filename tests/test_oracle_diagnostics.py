@@ -153,3 +153,50 @@ def test_semantic_partition_is_plain_lloyd_on_raw_rows_and_expands_support():
             assert dist[lab[i]] <= min(dist) + 1e-9 * max(1.0, min(dist))
     assert np.all(np.isfinite(res.out)) and res.pairs_exec == res.pairs_sparse + w.M * w.N
     assert np.array_equal(np.sort(res.perm_q), np.arange(w.N))
+
+
+def test_row_density_closed_forms_and_brute_force():
+    N = 40
+    # equal weights: ceil(tau N) of N are needed
+    for tau in (0.95, 0.5, 0.025, 1.0):
+        assert D.row_density(np.full(N, 1.0 / N), tau) == math.ceil(tau * N - 1e-9) / N
+    one_hot = np.zeros(N)
+    one_hot[17] = 1.0
+    assert D.row_density(one_hot, 0.95) == 1.0 / N
+    rng = np.random.default_rng(9)
+    for _ in range(30):
+        w = rng.dirichlet(np.full(9, 0.3))
+        tau = float(rng.uniform(0.3, 0.99))
+        best = min(s for s in range(1, 10)
+                   if any(w[list(c)].sum() >= tau - 1e-12
+                          for c in itertools.combinations(range(9), s)))
+        assert D.row_density(w, tau) == best / 9
+
+
+def test_head_density_two_levels_of_logits():
+    """Keys in two blocks of logits a (n1 keys) and 0 (n2 keys): the row's
+    weights are e^a/Z and 1/Z, so the covering count has a closed form."""
+    n1, n2, a = 5, 35, 3.0
+    K = np.zeros((n1 + n2, 2))
+    K[:n1, 0] = a
+    Q = np.array([[1.0, 0.0]])
+    Z = n1 * math.exp(a) + n2
+    hi = math.exp(a) / Z
+    for tau in (0.3, 0.8, 0.95):
+        if tau <= n1 * hi:
+            n = math.ceil(tau / hi - 1e-12)
+        else:
+            n = n1 + math.ceil((tau - n1 * hi) * Z - 1e-9)
+        assert D.head_density(Q, K, [0], 1.0, tau) == n / (n1 + n2)
+
+
+def test_conservative_density_quantile():
+    # z at 0.95 is 1.6448536...; at alpha = 0.5 the quantile is the mean
+    s = [0.2, 0.3, 0.25, 0.35]
+    mu = sum(s) / 4
+    sd = math.sqrt(sum((x - mu) ** 2 for x in s) / 4)
+    r = D.conservative_density(s, 0.95)
+    assert abs(r["density"] - (mu + 1.6448536269514722 * sd)) < 1e-12
+    assert abs(r["sparsity"] - (1 - r["density"])) < 1e-15
+    assert abs(D.conservative_density(s, 0.5)["density"] - mu) < 1e-15
+    assert D.conservative_density([0.99, 0.5], 0.999)["density"] == 1.0  # clipped
