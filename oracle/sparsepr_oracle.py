@@ -202,6 +202,44 @@ def semantic_partition(q_video, k_video, Ck, Cq, iters, seed, head):
         dict(passes=qp)
 
 
+def coclustering_partition(q_video, k_video, Ck, Cq, iters, seed, head, scale):
+    """Bidirectional QK co-clustering ["Attention Sparsity is Input-Stable"
+    (papernotes.org note), "key designs", online bidirectional
+    co-clustering], offered as an alternative partition. Each round: (A) each
+    key's affinity vector to the current query centres, P_k = scale * K C_q^T,
+    is assigned to the nearest key-block centre in that space (the mean
+    affinity vector of the block's current members), then the key centres
+    C_k are the blocks' mean K rows; (B) symmetrically for the queries with
+    P_q = scale * Q C_k^T against the just-updated C_k. Readings: C_q starts
+    at the query rows of the Fisher-Yates draws (which = 1) and the first key
+    blocks are the singletons of the key draws (which = 0), the first query
+    blocks those of the query draws; an empty block keeps its previous centre;
+    at most ``iters`` rounds, stopping after a round that changes no label.
+    Returns (key labels, query labels, rounds)."""
+    seeds_k = init_indices(k_video.shape[0], Ck, seed, head, 0)
+    seeds_q = init_indices(q_video.shape[0], Cq, seed, head, 1)
+    Cq_c = q_video[seeds_q].copy()
+    lab_k = lab_q = None
+    Pk_bar = Pq_bar = None
+    rounds = 0
+    for _ in range(iters):
+        rounds += 1
+        Pk = scale * (k_video @ Cq_c.T)
+        Pk_bar = Pk[seeds_k] if lab_k is None else group_means(Pk, lab_k, Ck, prev=Pk_bar)
+        new_k = nearest(Pk, Pk_bar)
+        Ck_c = group_means(k_video, new_k, Ck)
+        Pq = scale * (q_video @ Ck_c.T)
+        Pq_bar = Pq[seeds_q] if lab_q is None else group_means(Pq, lab_q, Cq, prev=Pq_bar)
+        new_q = nearest(Pq, Pq_bar)
+        done = (lab_k is not None and np.array_equal(new_k, lab_k)
+                and np.array_equal(new_q, lab_q))
+        lab_k, lab_q = new_k, new_q
+        Cq_c = group_means(q_video, lab_q, Cq, prev=Cq_c)
+        if done:
+            break
+    return lab_k, lab_q, rounds
+
+
 # ---------------------------------------------------------------------------
 # Stage 2: group-major layout  [SPR 2.C]
 # ---------------------------------------------------------------------------
@@ -393,8 +431,9 @@ def run_head(q, k, v, p: dict, head: int, rows=None, partition_only=False) -> He
 
     ``p`` holds the method parameters (Ck, Cq, Ms, n_eig, kmeans_iters, keep
     [per head], M, r, lam, scale, seed, n_text; optionally partition =
-    "response" (default) or "semantic", the ablations' uncoupled k-means on
-    raw Q and K rows). ``rows`` restricts the
+    "response" (default), "semantic" (the ablations' uncoupled k-means on
+    raw Q and K rows) or "coclustering" (the co-clustering page's
+    alternating QK partition)). ``rows`` restricts the
     sparse-attention and corrected outputs to those group-major rows
     (default: all rows); partition, routing, probes and the fit are always
     computed in full.
@@ -415,8 +454,14 @@ def run_head(q, k, v, p: dict, head: int, rows=None, partition_only=False) -> He
     qv, kv = q[:Nv], k[:Nv]
 
     # Stage 1 [SPR 2.A]
-    if p.get("partition", "response") == "semantic":
+    mode = p.get("partition", "response")
+    if mode == "semantic":
         lab_k_v, lab_q_v, kinfo, qinfo = semantic_partition(qv, kv, Ck, Cq, iters, seed, head)
+    elif mode == "coclustering":
+        lab_k_v, lab_q_v, rounds = coclustering_partition(qv, kv, Ck, Cq, iters, seed, head, scale)
+        kinfo = dict(passes=rounds, MK=np.full((d, d), np.nan), lam=np.zeros(0),
+                     U=np.zeros((0, 0)))
+        qinfo = dict(passes=rounds)
     else:
         lab_k_v, kinfo = key_partition(kv, qv, Ck, int(p["Ms"]), int(p["n_eig"]),
                                        iters, seed, head)

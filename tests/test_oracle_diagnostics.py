@@ -200,3 +200,37 @@ def test_conservative_density_quantile():
     assert abs(r["sparsity"] - (1 - r["density"])) < 1e-15
     assert abs(D.conservative_density(s, 0.5)["density"] - mu) < 1e-15
     assert D.conservative_density([0.99, 0.5], 0.999)["density"] == 1.0  # clipped
+
+
+def test_coclustering_partition_is_a_joint_fixed_point():
+    """The co-clustering partition at convergence: key labels are the nearest
+    key-block centres in the space of affinities to the query blocks' mean
+    rows, and query labels the nearest query-block centres in the space of
+    affinities to the key blocks' mean rows; recomputed with loops from the
+    labels alone."""
+    w = synth.custom("cocl", 1, (2, 4, 8), 16, "f32", n_comp=6, sigma=0.4, noise_var=0.05, Ck=6,
+                     Cq=4, Ms=32, n_eig=16, kmeans_iters=200, M=8, r=4, seed=3, keep=0.5)
+    q, k, v = synth.generate(w)
+    q, k, v = synth.as_f64(q[0]), synth.as_f64(k[0]), synth.as_f64(v[0])
+    p = dict(w.params(), partition="coclustering")
+    res = O.run_head(q, k, v, p, 0)
+    assert res.info["key_passes"] < w.kmeans_iters
+    lk, lq = res.label_k, res.label_q
+    assert len(set(lk.tolist())) == w.Ck and len(set(lq.tolist())) == w.Cq
+    s = 1.0 / math.sqrt(w.d)
+
+    def means(X, lab, C):
+        return [[sum(X[i][a] for i in range(len(X)) if lab[i] == c) / int((lab == c).sum())
+                 for a in range(len(X[0]))] for c in range(C)]
+
+    def check(X, lab, C, anchors):
+        P = [[s * sum(X[i, a] * anchors[c][a] for a in range(w.d)) for c in range(len(anchors))]
+             for i in range(w.N)]
+        Pb = means(P, lab, C)
+        for i in range(w.N):
+            dist = [sum((P[i][j] - Pb[c][j]) ** 2 for j in range(len(anchors))) for c in range(C)]
+            assert dist[lab[i]] <= min(dist) + 1e-9 * max(1.0, min(dist)), i
+
+    check(k, lk, w.Ck, means(q, lq, w.Cq))
+    check(q, lq, w.Cq, means(k, lk, w.Ck))
+    assert np.all(np.isfinite(res.out))
