@@ -245,7 +245,8 @@ def run_reference(args, w, rank):
                 warmup=args.warmup, ms_per_step=t_call * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
                 impl="reference",
-                config=dict(workload=workload_desc(w)),
+                config=dict(workload=workload_desc(w), heads_per_rank=w.H,
+                            parallelism="one host process on rank 0 (the oracle's numpy threads)"),
                 cpu_baseline=dict(value=value, unit="TFLOPS", cores=oracle_cores(), kind="oracle",
                                   sample=oracle_sample_desc(w, t_call)),
                 e2e=dict(value=value, unit="TFLOPS", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
