@@ -90,13 +90,21 @@ class ClockSampler:
         self.proc = None
 
     def start(self):
+        """Starts sampling every 100 ms and returns once the first sample is
+        in (it is dropped), so the samples that stop() reads were taken while
+        the caller's timed region ran."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        import select
+        ready, _, _ = select.select([self.proc.stdout], [], [], 5.0)
+        if ready:
+            self.proc.stdout.readline()
 
     def stop(self):
         if self.proc is None:
@@ -356,9 +364,9 @@ def main():
             graph.replay()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
+    sampler.start()  # returns after its first sample, before the ranks line up
     barrier()
     torch.cuda.synchronize(dev)
-    sampler.start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
