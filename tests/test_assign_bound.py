@@ -87,3 +87,38 @@ def test_certified_rows_have_the_exact_label():
             certified += 1
             assert order[0] == int(np.argmin(d))
     assert certified > 150  # the bound certifies almost every row
+
+
+def emulate_query(x, Y, c, nB, rng):
+    """The query pass: x is a bf16 row (one exact plane), the centroid side
+    G qbar is split into nB bf16 planes, products (0, b) for b < nB summed in
+    fp32, then the same fp32 fma with the offset and position packing."""
+    yp = [planes(Y[:, t], nB) for t in range(Y.shape[1])]
+    v = np.zeros(Y.shape[0], dtype=np.float32)
+    for b in range(nB):
+        for t in range(x.shape[0]):
+            v = (v + (x[t] * yp[t][b]).astype(np.float32)).astype(np.float32)
+    dd = (np.float64(-2.0) * v.astype(np.float64) + c.astype(np.float32).astype(np.float64))
+    bits = dd.astype(np.float32).view(np.uint32)
+    pos = rng.integers(0, 8, size=bits.shape).astype(np.uint32)
+    return ((bits & np.uint32(~7 & 0xFFFFFFFF)) | pos).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("nB,res", [(3, 9.5367431640625e-07), (2, 6.103515625e-05)])
+def test_query_pass_distances_within_bound(nB, res):
+    """d = 128, as in the query pass: the bound with Kt = nB * d and the
+    residual term of nB centroid planes covers every emulated distance."""
+    rng = np.random.default_rng(40 + nB)
+    D, m = 128, 24
+    Y = rng.standard_normal((m, D)) * rng.uniform(0.1, 4.0, size=(m, 1))  # G qbar rows
+    c = np.abs(rng.standard_normal(m)) * 50.0  # qbar^T G qbar >= 0
+    Ymax = float(np.sqrt((Y * Y).sum(1)).max() * (1 + 1e-6))
+    C = float(np.abs(c).max() * (1 + 1e-6))
+    kt_term = nB * D * 2.0 ** -22 + res
+    for _ in range(30):
+        x = bf16(rng.standard_normal(D) * rng.uniform(0.2, 3.0))
+        d = c - 2.0 * (Y @ x)
+        dp = emulate_query(x, Y, c, nB, rng)
+        xy = float(np.sqrt((x * x).sum()) * (1 + 1e-6)) * Ymax
+        E = kt_term * xy + 1.25e-06 * (C + 2.0 * xy)
+        assert np.all(np.abs(dp - d) <= E), (np.abs(dp - d).max(), E)
