@@ -22,8 +22,11 @@ LIB = os.path.join(PKG, "libsparsepr.so")
 SOURCES = ["api.cu", "sort.cu", "partition.cu", "linalg.cu", "permute.cu", "attn.cu", "fit.cu",
            "noalloc.cu", "assign.cu", "eigen.cu", "correct.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
-         "-I", os.path.join(ROOT, "include")]
+# -Werror=shadow: a launcher's local that shadows one of its parameters (say a
+# cudaError_t named like a size argument) silently changes the launch.
+FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC,-Werror=shadow",
+         "--expt-relaxed-constexpr"]
+INCLUDE = ["-I", os.path.join(ROOT, "include")]
 
 
 def nvcc() -> str:
@@ -44,7 +47,7 @@ def _compile(src: str, extra=()) -> str:
     newest = max(os.path.getmtime(p) for p in [src] + _headers())
     if os.path.exists(obj) and os.path.getmtime(obj) >= newest and not extra:
         return obj
-    cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
+    cmd = [nvcc(), *ARCH, *FLAGS, *INCLUDE, *extra, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, " ".join(cmd), r.stderr))
@@ -54,6 +57,11 @@ def _compile(src: str, extra=()) -> str:
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
+    # objects built with other flags or another nvcc are rebuilt
+    stamp = os.path.join(BUILD, "flags.txt")
+    want = " ".join([nvcc(), *ARCH, *FLAGS])
+    if not os.path.exists(stamp) or open(stamp).read() != want:
+        force = True
     if force:
         for s in srcs:
             o = os.path.join(BUILD, os.path.basename(s) + ".o")
@@ -68,6 +76,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("link failed:\n%s" % r.stderr)
+    with open(stamp, "w") as f:
+        f.write(want)
     return LIB
 
 

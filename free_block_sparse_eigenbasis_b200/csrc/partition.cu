@@ -702,14 +702,14 @@ cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, 
   const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;
   dim3 grid((Nv + kZRows - 1) / kZRows, H);
   if (bf16) {
-    const cudaError_t e = cudaFuncSetAttribute(
+    const cudaError_t err = cudaFuncSetAttribute(
         zproj_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shb));
-    if (e != cudaSuccess) return e;
+    if (err != cudaSuccess) return err;
     zproj_kernel<<<grid, kZThreads, shb, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv, d, e, wk, z);
   } else {
-    const cudaError_t e = cudaFuncSetAttribute(
+    const cudaError_t err = cudaFuncSetAttribute(
         zproj_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shb));
-    if (e != cudaSuccess) return e;
+    if (err != cudaSuccess) return err;
     zproj_kernel<<<grid, kZThreads, shb, st>>>(static_cast<const float*>(k), N, Nv, d, e, wk, z);
   }
   return cudaGetLastError();

@@ -13,14 +13,21 @@ MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 
 
-def gpu_run(w, q=None, k=None, v=None, with_fit=True):
-    """Full path on the GPU; returns (buffers, q, k, v) with q/k/v on CPU."""
+def gpu_run(w, q=None, k=None, v=None, with_fit=True, fill=None):
+    """Full path on the GPU; returns (buffers, q, k, v) with q/k/v on CPU.
+    fill: a byte written over every buffer of the call (workspace and
+    outputs) before it, so that a read of memory the call did not write
+    shows up as a mismatch."""
     from free_block_sparse_eigenbasis_b200 import sparsepr as S
     if q is None:
         q, k, v = synth.generate(w)
     p = w.params()
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     b = S.allocate(p, qd.dtype, with_fit=with_fit)
+    if fill is not None:
+        for t in vars(b).values():
+            if isinstance(t, torch.Tensor):
+                t.view(torch.uint8).fill_(fill)
     S.attention(qd, kd, vd, p, b)
     torch.cuda.synchronize()
     return b, (q, k, v)

@@ -36,6 +36,18 @@ def test_tiny_full_pipeline():
     assert np.abs(fit[:d * d].reshape(d, d) - res.Bp).max() < 5e-2 * max(1.0, np.abs(res.Bp).max())
 
 
+@pytest.mark.parametrize("fill", [0x00, 0xFF, 0x5A])
+def test_tiny_result_independent_of_prior_memory(fill):
+    """The whole call on buffers pre-filled with one byte pattern (0xFF makes
+    every double a NaN, 0x5A a huge finite value): integer outputs and
+    outputs must equal the oracle's whatever the memory held before."""
+    w = synth.workload("tiny")
+    b, (q, k, v) = gpu_run(w, fill=fill)
+    res = oracle_head(w, q, k, v, 0)
+    compare_head(b, res, w, 0, None)
+    assert _S().sparsepr_read_stats(b.ws)["status"] == 0
+
+
 SMALL = [
     # several query tiles per group, ragged tails, two heads with different budgets
     synth.custom("small_bf16_d128", 2, (4, 16, 32), 128, "bf16", Ck=64, Cq=16, Ms=256,
@@ -63,7 +75,7 @@ SMALL = [
 
 @pytest.mark.parametrize("w", SMALL, ids=[x.name for x in SMALL])
 def test_small_full_pipeline(w):
-    b, (q, k, v) = gpu_run(w)
+    b, (q, k, v) = gpu_run(w, fill=0xFF)
     for h in range(w.H):
         res = oracle_head(w, q, k, v, h)
         compare_head(b, res, w, h, None)
