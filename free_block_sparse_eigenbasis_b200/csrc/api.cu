@@ -209,6 +209,16 @@ int32_t sparsepr_route_width(const sparsepr_params* p) {
   return L.kmax;
 }
 
+sparsepr_status sparsepr_workspace_region(const sparsepr_params* p, const char* name,
+                                          size_t* offset, size_t* bytes) {
+  if (!name || !offset || !bytes) return SPARSEPR_ERR_INVALID_ARG;
+  const sparsepr_status s = check_params(p);
+  if (s != SPARSEPR_OK) return s;
+  Layout L;
+  compute_layout(*p, &L);
+  return named_region(*p, L, name, offset, bytes) ? SPARSEPR_OK : SPARSEPR_ERR_INVALID_ARG;
+}
+
 sparsepr_status sparsepr_check_wait_limit(void* ws, void* stream) {
   if (!ws) return SPARSEPR_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return SPARSEPR_ERR_INVALID_ARG;
@@ -265,15 +275,20 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
   {
+    // the side stream is joined on every path, also after a failed launch,
+    // so that a stream capture in progress stays valid
     std::lock_guard<std::mutex> lk(g_side_mu);
     SideStream* ss = side_stream();
     const cudaStream_t side = fork_side(ss, st);
-    SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, side));
-    SPR_TRY(launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st));
-    SPR_TRY(launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st));
-    SPR_TRY(launch_scale_columns(evl, evc, H, d, e, wk, st));
-    SPR_TRY(launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st));
-    SPR_TRY(join_side(ss, side, st));
+    cudaError_t err = launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, side);
+    if (err == cudaSuccess) err = launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st);
+    if (err == cudaSuccess)
+      err = launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st);
+    if (err == cudaSuccess) err = launch_scale_columns(evl, evc, H, d, e, wk, st);
+    if (err == cudaSuccess) err = launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st);
+    const cudaError_t ej = join_side(ss, side, st);
+    SPR_TRY(err);
+    SPR_TRY(ej);
   }
   const long long hs_z = static_cast<long long>(Nv) * e;
   SPR_TRY(launch_gather_init(z, kXf64, hs_z, e, e, init_k, Ck, H, mu, mun, st));
@@ -314,6 +329,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     ak.c_exact = mun;
     ak.m = Ck;
     ak.direct = 1;
+    ak.metric = nullptr;
   }
   for (int t = 0; t < iters; ++t) {
     if (tc_keys) {
@@ -324,7 +340,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
                                     at<double>(ws, L.ytr), flags, 0, st));
       SPR_TRY(launch_argmin_tc(ak, st));
     } else {
-      SPR_TRY(launch_argmin(z, kXf64, hs_z, e, Nv, e, mu, mun, Ck, H, lab_k, flags, 0, st));
+      SPR_TRY(launch_argmin(z, kXf64, hs_z, e, Nv, e, mu, mun, Ck, H, lab_k, flags, 0, nullptr,
+                            c.stats, st));
     }
     SPR_TRY(launch_finalize_pass(H, t, flags, 0, c.stats->key_passes, st));
     if (t + 1 < iters) {
@@ -381,6 +398,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     aq.c_exact = cg;
     aq.m = Cq;
     aq.direct = 0;
+    aq.metric = G;
   }
   for (int t = 0; t < iters; ++t) {
     SPR_TRY(launch_query_metric_apply(G, qbar, Cq, H, d, wg, cg, flags + 3, 4, st));
@@ -391,7 +409,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
                                     at<float>(ws, L.hmq), at<double>(ws, L.ytr), flags, 2, st));
       SPR_TRY(launch_argmin_tc(aq, st));
     } else {
-      SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, st));
+      SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, G, c.stats,
+                            st));
     }
     SPR_TRY(launch_finalize_pass(H, t, flags, 2, c.stats->query_passes, st));
     if (t + 1 < iters) {
@@ -605,27 +624,33 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     // the ridge solve (reads the Grams) runs beside R^T R and its eigen solve
     // (they touch other regions); with r > 32 the Gram region is reused below,
     // so the two stay in order
+    // (joined on every path, also after a failed launch)
     std::unique_lock<std::mutex> lk(g_side_mu);
     SideStream* ss = (c.p.r <= 32) ? side_stream() : nullptr;
     const cudaStream_t side = fork_side(ss, st);
-    SPR_TRY(launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side));
-    SPR_TRY(launch_gram_f64(xr + static_cast<size_t>(M) * d, xr + static_cast<size_t>(M) * d,
+    cudaError_t err = launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side);
+    if (err == cudaSuccess)
+      err = launch_gram_f64(xr + static_cast<size_t>(M) * d, xr + static_cast<size_t>(M) * d,
                             nullptr, nullptr, hs, hs, d, M, H, d, 1.0, 0.0, rtr,
-                            static_cast<long long>(d) * d, 0, st));
+                            static_cast<long long>(d) * d, 0, st);
     double* evl = at<double>(ws, L.eval);
     double* evc = at<double>(ws, L.evec);
     // leading-r right singular vectors of R = top-r eigenvectors of R^T R
     const double* vr = evc;
     if (c.p.r <= 32) {
-      SPR_TRY(launch_sym_eigs(rtr, H, d, c.p.r, evl, evc, at<double>(ws, L.eigscr), st));
+      if (err == cudaSuccess)
+        err = launch_sym_eigs(rtr, H, d, c.p.r, evl, evc, at<double>(ws, L.eigscr), st);
     } else {
       double* sel = gram;  // free after the ridge solve: [H, d, r] selected vectors
-      SPR_TRY(launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st));
-      SPR_TRY(launch_top_eig_projector(evl, evc, H, d, c.p.r, sel, false, st));
+      if (err == cudaSuccess) err = launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st);
+      if (err == cudaSuccess)
+        err = launch_top_eig_projector(evl, evc, H, d, c.p.r, sel, false, st);
       vr = sel;
     }
-    SPR_TRY(join_side(ss, side, st));
+    const cudaError_t ej = join_side(ss, side, st);
     lk.unlock();
+    SPR_TRY(err);
+    SPR_TRY(ej);
     SPR_TRY(launch_project_map(bmat, bvec, vr, H, d, c.p.r, bp32, bv32, fit, st));
   } else {
     SPR_TRY(cudaMemsetAsync(bp32, 0, static_cast<size_t>(H) * d * d * 4, st));

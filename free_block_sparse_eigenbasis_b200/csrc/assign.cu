@@ -532,10 +532,14 @@ template <int DT, bool DIRECT>
 __global__ void __launch_bounds__(kRcThreads)
     recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
                    const double* yT, const double* c, int m, int32_t* labels, int32_t* flags,
-                   int flag_base, const int32_t* recheck, const int32_t* nrecheck) {
+                   int flag_base, const int32_t* recheck, const int32_t* nrecheck,
+                   const double* G, DeviceStats* stats) {
   __shared__ double xs[kRcMaxD];
-  __shared__ double wbest[kRcThreads / 32];
+  __shared__ double wb1[kRcThreads / 32], wb2[kRcThreads / 32];
   __shared__ int wbi[kRcThreads / 32];
+  __shared__ double gtr;
+  __shared__ double xpart[kRcThreads / 32];
+  __shared__ int cand;
   const int h = blockIdx.y;
   int32_t* fl = flags + h * 4;
   if (fl[flag_base + 1]) return;
@@ -543,38 +547,83 @@ __global__ void __launch_bounds__(kRcThreads)
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const double* Yh = yT + static_cast<size_t>(h) * D * m;
   const double* ch = DIRECT ? nullptr : c + static_cast<size_t>(h) * m;
+  const double* Gh = (!DIRECT && G) ? G + static_cast<size_t>(h) * D * D : nullptr;
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    if (Gh)
+      for (int a = 0; a < D; ++a) t += Gh[static_cast<size_t>(a) * D + a];
+    gtr = t;
+  }
+  int ties = 0;
   for (int k = blockIdx.x; k < cnt; k += gridDim.x) {
     const int row = recheck[static_cast<size_t>(h) * n + k];
     __syncthreads();  // xs and the warp results of the previous row are consumed
     for (int t = threadIdx.x; t < D; t += blockDim.x)
       xs[t] = ldx(X, kind, h * hsx + static_cast<size_t>(row) * ldx_ + t);
     __syncthreads();
-    double best = INFINITY;
-    int bi = 0x7fffffff;
+    Top2 t2 = top2_empty();
     constexpr int kJUnroll = (DT > 0 && DT <= 16) ? 2 : 1;  // short rows: two centroids in flight
 #pragma unroll kJUnroll
-    for (int j = threadIdx.x; j < m; j += kRcThreads) {  // ascending within the thread
-      const double dd = rc_score<DT, DIRECT>(xs, Yh, m, j, D, ch);
-      if (dd < best) {
-        best = dd;
-        bi = j;
-      }
-    }
+    for (int j = threadIdx.x; j < m; j += kRcThreads)  // ascending within the thread
+      top2_push(t2, rc_score<DT, DIRECT>(xs, Yh, m, j, D, ch), j);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-      argmin_merge(best, bi, __shfl_xor_sync(0xffffffffu, best, o), __shfl_xor_sync(0xffffffffu, bi, o));
+    for (int o = 16; o > 0; o >>= 1) {
+      const double o1 = __shfl_xor_sync(0xffffffffu, t2.b1, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, t2.i1, o);
+      const double o2 = __shfl_xor_sync(0xffffffffu, t2.b2, o);
+      top2_merge(t2, o1, oi, o2);
+    }
     if (lane == 0) {
-      wbest[w] = best;
-      wbi[w] = bi;
+      wb1[w] = t2.b1;
+      wb2[w] = t2.b2;
+      wbi[w] = t2.i1;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-      for (int q = 1; q < kRcThreads / 32; ++q) argmin_merge(best, bi, wbest[q], wbi[q]);
+      for (int q = 1; q < kRcThreads / 32; ++q) top2_merge(t2, wb1[q], wbi[q], wb2[q]);
       const size_t li = static_cast<size_t>(h) * n + row;
-      if (labels[li] != bi) atomicAdd(&fl[flag_base], 1);
-      labels[li] = bi;
+      if (labels[li] != t2.i1) atomicAdd(&fl[flag_base], 1);
+      labels[li] = t2.i1;
+      // near tie: DIRECT values are squared distances; otherwise they lack
+      // x^T G x, formed below (by the whole block) for candidate rows only
+      const double gap = t2.b2 - t2.b1;
+      int cd = 0;
+      if (m > 1) {
+        if (DIRECT) {
+          ties += (gap <= kNearTieRel * t2.b2);
+        } else if (Gh) {
+          double xx = 0.0;
+          for (int a = 0; a < D; ++a) xx = fma(xs[a], xs[a], xx);
+          cd = gap <= 1e-11 * (fabs(t2.b2) + gtr * xx);
+        }
+      }
+      cand = cd;
+      wb1[0] = gap;
+      wb2[0] = t2.b2;
+    }
+    if (!DIRECT) {
+      __syncthreads();  // cand, wb1[0] = gap and wb2[0] = second value are visible
+      if (cand) {       // block-uniform
+        double part = 0.0;
+        for (int b = threadIdx.x; b < D; b += blockDim.x) {
+          double gb = 0.0;
+          for (int a = 0; a < D; ++a) gb = fma(xs[a], Gh[static_cast<size_t>(a) * D + b], gb);
+          part = fma(gb, xs[b], part);
+        }
+        part = warp_sum_f64(part);
+        if (lane == 0) xpart[w] = part;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          double xgx = 0.0;
+          for (int q = 0; q < kRcThreads / 32; ++q) xgx += xpart[q];
+          ties += (wb1[0] <= kNearTieRel * (wb2[0] + xgx));
+        }
+      }
     }
   }
+  if (threadIdx.x == 0 && ties)
+    atomicAdd(reinterpret_cast<unsigned long long*>(&stats->near_ties[flag_base >> 1]),
+              static_cast<unsigned long long>(ties));
 }
 
 template <bool DIRECT>
@@ -583,7 +632,7 @@ void launch_recheck_d(const AssignTC& a, cudaStream_t st) {
 #define SPR_RC(DT)                                                                          \
   recheck_kernel<DT, DIRECT><<<grid, kRcThreads, 0, st>>>(                                 \
       a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D, a.y_tr, a.c_exact, a.m, a.labels, a.flags, \
-      a.flag_base, a.recheck, a.nrecheck)
+      a.flag_base, a.recheck, a.nrecheck, a.metric, a.stats)
   if (a.D == 16)
     SPR_RC(16);
   else if (a.D == 64)

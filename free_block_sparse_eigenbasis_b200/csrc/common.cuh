@@ -302,6 +302,38 @@ __device__ __forceinline__ void vload16(const T* p, double* out) {
   vwiden16<T>(*reinterpret_cast<const uint4*>(p), out);
 }
 
+// Nearest and second-nearest value of a row over a set of centroids: b1 at
+// index i1, b2 the next value (on an exact tie the lower index is the
+// nearest and the tied value becomes b2).
+struct Top2 {
+  double b1, b2;
+  int i1;
+};
+__device__ __forceinline__ Top2 top2_empty() { return Top2{INFINITY, INFINITY, 0x7fffffff}; }
+// add value v of centroid j; j ascending across calls on one Top2
+__device__ __forceinline__ void top2_push(Top2& t, double v, int j) {
+  if (v < t.b1) {
+    t.b2 = t.b1;
+    t.b1 = v;
+    t.i1 = j;
+  } else if (v < t.b2) {
+    t.b2 = v;
+  }
+}
+// merge the Top2 of a disjoint set of centroids
+__device__ __forceinline__ void top2_merge(Top2& t, double o1, int oi, double o2) {
+  if (o1 < t.b1 || (o1 == t.b1 && oi < t.i1)) {
+    t.b2 = fmin(t.b1, o2);
+    t.b1 = o1;
+    t.i1 = oi;
+  } else {
+    t.b2 = fmin(t.b2, o1);
+  }
+}
+// A row is a near tie when its two smallest squared distances d1 <= d2
+// satisfy d2 - d1 <= 1e-12 d2 (gap and d2 of the true squared distance).
+constexpr double kNearTieRel = 1e-12;
+
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -50,7 +50,8 @@ cudaError_t launch_gather_init(const void* src, int src_kind, long long head_str
 // changes[h] += number of labels that differ from the previous value.
 cudaError_t launch_argmin(const void* X, int x_kind, long long head_stride_x, int ldx, int n,
                           int D, const double* Y, const double* c, int m, int H,
-                          int32_t* labels, int32_t* flags, int flag_base, cudaStream_t st);
+                          int32_t* labels, int32_t* flags, int flag_base, const double* G,
+                          DeviceStats* stats, cudaStream_t st);
 cudaError_t launch_finalize_pass(int H, int pass, int32_t* flags, int flag_base,
                                  int32_t* passes_out, cudaStream_t st);
 // out[h, c, :] = mean of the rows perm[off[c]..off[c+1]) of X (fp64 sums in
@@ -107,6 +108,7 @@ struct AssignTC {
   const double* c_exact;          // [H, m] (unused when direct)
   int m;
   int direct;                     // 1: d = |x - y|^2, 0: d = c - 2 x.y
+  const double* metric;           // [H, D, D] G of d = c - 2 x.y + x^T G x (near-tie count; direct: unused)
 };
 size_t assign_tc_smem_bytes(int nA, int nB, int Dp, int Cpad);
 cudaError_t launch_split_rows(const void* X, int kind, long long hsx, int ldx, int n, int D,

@@ -205,6 +205,39 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->total = o;
 }
 
+// Offset and size of a named region that holds a stage's intermediate
+// results (the read-out of sparsepr_workspace_region); false for an unknown
+// name.
+inline bool named_region(const sparsepr_params& p, const Layout& L, const char* name, size_t* off,
+                         size_t* bytes) {
+  const size_t H = p.H, d = p.d, e = p.n_eig, Ck = p.Ck, Cq = p.Cq, Nv = L.Nv;
+  struct R {
+    const char* n;
+    size_t o, b;
+  } const tab[] = {
+      {"init_k", L.init_k, H * Ck * 4}, {"init_q", L.init_q, H * Cq * 4},
+      {"mk", L.mk, H * d * d * 8},      {"eval", L.eval, H * e * 8},
+      {"evec", L.evec, H * d * e * 8},  {"wk", L.wk, H * d * e * 8},
+      {"z", L.z, H * Nv * e * 8},       {"ck", L.ck, H * Ck * d * 8},
+      {"g", L.g, H * d * d * 8},        {"bmat", L.bmat, H * d * d * 8},
+      {"bvec", L.bvec, H * d * 8},
+  };
+  for (const R& r : tab) {
+    const char* a = r.n;
+    const char* b = name;
+    while (*a && *a == *b) {
+      ++a;
+      ++b;
+    }
+    if (*a == 0 && *b == 0) {
+      *off = r.o;
+      *bytes = r.b;
+      return true;
+    }
+  }
+  return false;
+}
+
 template <typename T>
 inline T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);

@@ -299,15 +299,34 @@ __global__ void gather_init_kernel(const void* src, int kind, long long hs, int 
 // Nearest centroid: labels[i] = argmin_j (c_j - 2 x_i . y_j), lowest j on
 // ties, fp64. 64 rows x 64 centroids per tile step, 16x16 threads, 4x4
 // register block per thread, D in chunks of 32.
+// The value c_j - 2 x.y_j is the squared distance minus x^T G x, with G = I
+// (keys: y = mu, c = |mu|^2) or the query metric G (queries: y = G qbar,
+// c = qbar^T G qbar); near ties (see kNearTieRel) are counted from the two
+// smallest values plus x^T G x. For G != I the quadratic form is only
+// formed for candidate rows, whose gap lies within 1e-11 of
+// |second value| + trace(G) |x|^2 (an upper bound of the second distance,
+// G being positive semidefinite).
 // ---------------------------------------------------------------------------
 constexpr int kAR = 64, kAC = 64, kAK = 32;
+
+__device__ double quad_form_row(const void* X, int kind, size_t xb, int D, const double* G) {
+  double acc = 0.0;
+  for (int a = 0; a < D; ++a) {
+    double ga = 0.0;
+    for (int b = 0; b < D; ++b) ga = fma(G[static_cast<size_t>(a) * D + b], load_x(X, kind, xb + b), ga);
+    acc = fma(load_x(X, kind, xb + a), ga, acc);
+  }
+  return acc;
+}
 
 __global__ void __launch_bounds__(256) argmin_kernel(const void* X, int kind, long long hsx,
                                                      int ldx, int n, int D, const double* Y,
                                                      const double* c, int m, int32_t* labels,
-                                                     int32_t* flags, int flag_base) {
+                                                     int32_t* flags, int flag_base,
+                                                     const double* G, DeviceStats* stats) {
   __shared__ double xs[kAK][kAR + 2];
   __shared__ double ys[kAK][kAC + 2];
+  __shared__ double gtr;
   const int h = blockIdx.y;
   int32_t* fl = flags + h * 4;
   if (fl[flag_base + 1]) return;  // this head's k-means already converged
@@ -315,13 +334,17 @@ __global__ void __launch_bounds__(256) argmin_kernel(const void* X, int kind, lo
   const int r0 = blockIdx.x * kAR;
   const double* Yh = Y + static_cast<size_t>(h) * m * D;
   const double* ch = c + static_cast<size_t>(h) * m;
-  double best[4];
-  int bidx[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    best[i] = INFINITY;
-    bidx[i] = 0x7fffffff;
+  const double* Gh = G ? G + static_cast<size_t>(h) * D * D : nullptr;
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    if (Gh)
+      for (int a = 0; a < D; ++a) t += Gh[static_cast<size_t>(a) * D + a];
+    gtr = t;
   }
+  Top2 best[4];
+  double xx[4] = {0.0, 0.0, 0.0, 0.0};  // |x|^2 of this thread's rows
+#pragma unroll
+  for (int i = 0; i < 4; ++i) best[i] = top2_empty();
   for (int c0 = 0; c0 < m; c0 += kAC) {
     double acc[4][4];
 #pragma unroll
@@ -350,53 +373,57 @@ __global__ void __launch_bounds__(256) argmin_kernel(const void* X, int kind, lo
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv[i], yv[j], acc[i][j]);
+        if (c0 == 0)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xx[i] = fma(xv[i], xv[i], xx[i]);
       }
       __syncthreads();
     }
-    // epilogue: candidate distances of this centroid chunk
+    // epilogue: nearest and second nearest of this centroid chunk
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      double bd = INFINITY;
-      int bi = 0x7fffffff;
+      Top2 t = top2_empty();
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int cc = c0 + tx * 4 + j;
-        if (cc < m) {
-          const double dist = ch[cc] - 2.0 * acc[i][j];
-          if (dist < bd) {
-            bd = dist;
-            bi = cc;
-          }
-        }
+        if (cc < m) top2_push(t, ch[cc] - 2.0 * acc[i][j], cc);
       }
       // reduce over the 16 lanes sharing these rows (lowest index on ties)
 #pragma unroll
       for (int o = 1; o < 16; o <<= 1) {
-        const double od = __shfl_xor_sync(0xffffffffu, bd, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (od < bd || (od == bd && oi < bi)) {
-          bd = od;
-          bi = oi;
-        }
+        const double o1 = __shfl_xor_sync(0xffffffffu, t.b1, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, t.i1, o);
+        const double o2 = __shfl_xor_sync(0xffffffffu, t.b2, o);
+        top2_merge(t, o1, oi, o2);
       }
-      if (bd < best[i] || (bd == best[i] && bi < bidx[i])) {
-        best[i] = bd;
-        bidx[i] = bi;
-      }
+      top2_merge(best[i], t.b1, t.i1, t.b2);
     }
   }
   if (tx == 0) {
-    int changed = 0;
+    int changed = 0, ties = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int row = r0 + ty * 4 + i;
       if (row < n) {
         int32_t* lp = labels + static_cast<size_t>(h) * n + row;
-        if (*lp != bidx[i]) changed++;
-        *lp = bidx[i];
+        if (*lp != best[i].i1) changed++;
+        *lp = best[i].i1;
+        const double gap = best[i].b2 - best[i].b1;
+        if (m > 1) {
+          if (!Gh) {
+            ties += (gap <= kNearTieRel * (best[i].b2 + xx[i]));
+          } else if (gap <= 1e-11 * (fabs(best[i].b2) + gtr * xx[i])) {
+            const double xgx =
+                quad_form_row(X, kind, h * hsx + static_cast<size_t>(row) * ldx, D, Gh);
+            ties += (gap <= kNearTieRel * (best[i].b2 + xgx));
+          }
+        }
       }
     }
     if (changed) atomicAdd(&fl[flag_base + 0], changed);
+    if (ties)
+      atomicAdd(reinterpret_cast<unsigned long long*>(&stats->near_ties[flag_base >> 1]),
+                static_cast<unsigned long long>(ties));
   }
 }
 
@@ -725,10 +752,11 @@ cudaError_t launch_gather_init(const void* src, int src_kind, long long head_str
 
 cudaError_t launch_argmin(const void* X, int x_kind, long long hsx, int ldx, int n, int D,
                           const double* Y, const double* c, int m, int H, int32_t* labels,
-                          int32_t* flags, int flag_base, cudaStream_t st) {
+                          int32_t* flags, int flag_base, const double* G, DeviceStats* stats,
+                          cudaStream_t st) {
   dim3 grid((n + kAR - 1) / kAR, H);
   argmin_kernel<<<grid, 256, 0, st>>>(X, x_kind, hsx, ldx, n, D, Y, c, m, labels, flags,
-                                      flag_base);
+                                      flag_base, G, stats);
   return cudaGetLastError();
 }
 

@@ -22,7 +22,8 @@ BF16, F32 = 0, 1
 EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_partition",
             "sparsepr_permute", "sparsepr_route", "sparsepr_route_width",
             "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
-            "sparsepr_reset_stats", "sparsepr_check_wait_limit")
+            "sparsepr_reset_stats", "sparsepr_check_wait_limit", "sparsepr_route_noalloc",
+            "sparsepr_workspace_region")
 
 
 class Params(ctypes.Structure):
@@ -41,7 +42,7 @@ class Stats(ctypes.Structure):
                 ("pairs_sparse", ctypes.c_int64 * MAX_HEADS),
                 ("pairs_exec", ctypes.c_int64 * MAX_HEADS),
                 ("recheck_rows", ctypes.c_int64 * 2),
-                ("eig_sweeps", ctypes.c_int32 * 2)]
+                ("eig_sweeps", ctypes.c_int32 * 2), ("near_ties", ctypes.c_int64 * 2)]
 
 
 class SparsePRError(RuntimeError):
@@ -75,6 +76,9 @@ def _load():
                                            V, sz, V]
     lib.sparsepr_route_noalloc.argtypes = [P, P, st, PP, I32P, I32P, I32P, I32P, V]
     lib.sparsepr_route_noalloc.restype = st
+    lib.sparsepr_workspace_region.argtypes = [PP, ctypes.c_char_p, ctypes.POINTER(sz),
+                                              ctypes.POINTER(sz)]
+    lib.sparsepr_workspace_region.restype = st
     lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
     lib.sparsepr_reset_stats.argtypes = [V, V]
     lib.sparsepr_check_wait_limit.argtypes = [V, V]
@@ -279,6 +283,26 @@ def sparsepr_check_wait_limit(ws, stream=None):
     _check(lib.sparsepr_check_wait_limit(_ws(ws)[0], _stream(stream)), "sparsepr_check_wait_limit")
 
 
+_REGION_DTYPES = dict(init_k=torch.int32, init_q=torch.int32)
+
+
+def sparsepr_workspace_region(p: dict, name: str):
+    """(byte offset, bytes) of a named intermediate-result region of the
+    workspace for these parameters."""
+    prm, keep = make_params(p)
+    off, nb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib.sparsepr_workspace_region(ctypes.byref(prm), name.encode(), ctypes.byref(off),
+                                         ctypes.byref(nb)), "sparsepr_workspace_region")
+    return int(off.value), int(nb.value)
+
+
+def workspace_view(ws, p: dict, name: str) -> torch.Tensor:
+    """The named region of `ws` as a flat tensor of its element type (fp64,
+    or int32 for the initial centroid rows); a view, no copy."""
+    off, nb = sparsepr_workspace_region(p, name)
+    return ws[off:off + nb].view(_REGION_DTYPES.get(name, torch.float64))
+
+
 def sparsepr_read_stats(ws) -> dict:
     s = Stats()
     _check(lib.sparsepr_read_stats(_ws(ws)[0], ctypes.byref(s)), "sparsepr_read_stats")
@@ -286,7 +310,7 @@ def sparsepr_read_stats(ws) -> dict:
     return dict(status=int(s.status), H=H, key_passes=list(s.key_passes[:H]),
                 query_passes=list(s.query_passes[:H]), pairs_sparse=list(s.pairs_sparse[:H]),
                 pairs_exec=list(s.pairs_exec[:H]), recheck_rows=list(s.recheck_rows),
-                eig_sweeps=list(s.eig_sweeps))
+                eig_sweeps=list(s.eig_sweeps), near_ties=list(s.near_ties))
 
 
 # ---- buffers + the whole call ----------------------------------------------

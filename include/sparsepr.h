@@ -102,6 +102,11 @@ typedef struct {
   int64_t pairs_exec[SPARSEPR_MAX_HEADS];   /* pairs_sparse + M*N (probe rows) */
   int64_t recheck_rows[2]; /* k-means rows decided again in fp64 (keys, queries), all passes */
   int32_t eig_sweeps[2];   /* Jacobi sweeps, max over heads: [1] = probe residual Gram when r > 32 (the tridiagonal solver serves r <= 32 and M_K, and leaves 0) */
+  int64_t near_ties[2];    /* k-means rows (keys, queries), summed over heads and passes, whose
+                              two smallest fp64 squared distances d1 <= d2 satisfy
+                              d2 - d1 <= 1e-12 d2: their label is decided by the lowest-index
+                              rule or by rounding, not by the data (expected 0 on generic data;
+                              exact ties such as two identical centroids count) */
 } sparsepr_stats;
 
 /* Bytes of device workspace the five calls need for these parameters
@@ -233,6 +238,32 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
                                        void* out, int32_t* probes, int64_t* pairs_exec,
                                        double* fit, void* ws, size_t ws_bytes,
                                        void* stream);
+
+/* Where a stage's intermediate results sit inside `ws`, for stage-level
+ * tests and debugging (the workspace layout depends only on the
+ * parameters): the byte offset and size of the named region. Contents
+ * (row-major) after the call that writes them, until a later call reuses the
+ * region:
+ *   written by sparsepr_partition [SPR 2.A]:
+ *     "init_k" [H, Ck] int32, "init_q" [H, Cq] int32: initial centroid rows
+ *             (partial Fisher-Yates draws, token indices of the video tokens)
+ *     "mk"     [H, d, d] fp64: M_K = Q_s^T Q_s / M_s
+ *     "eval"   [H, n_eig] fp64: the leading eigenvalues of M_K, descending
+ *     "evec"   [H, d, n_eig] fp64: their unit eigenvectors as columns (the
+ *             sign of each column is arbitrary)
+ *     "wk"     [H, d, n_eig] fp64: key projector U_e Lambda_e^{1/2}
+ *     "z"      [H, Nv, n_eig] fp64: key response coordinates z_j = W_K^T k_j
+ *     "ck"     [H, Ck, d] fp64: K group means in the original space over the
+ *             final key labels (the zero vector for an empty group)
+ *     "g"      [H, d, d] fp64: query metric G = scale^2 C_K^T C_K
+ *   written by sparsepr_probe_correct [SPR 2.B] (M > 0; it also reuses
+ *   "mk", "eval" and "evec" for R^T R and its eigenpairs):
+ *     "bmat"   [H, d, d] fp64, "bvec" [H, d] fp64: the ridge solution B, b
+ *             before the subspace projection
+ * Errors: INVALID_ARG for invalid parameters, a NULL pointer or an unknown
+ * name; UNSUPPORTED as sparsepr_workspace_bytes. Host only, enqueues nothing. */
+sparsepr_status sparsepr_workspace_region(const sparsepr_params* p, const char* name,
+                                          size_t* offset, size_t* bytes);
 
 /* Copy the device statistics of the last call out of `ws` (a blocking
  * device-to-host copy; call after the stream has been synchronised). */

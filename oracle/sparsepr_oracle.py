@@ -129,20 +129,43 @@ def group_means(X: np.ndarray, labels: np.ndarray, C: int, prev: Optional[np.nda
     return out
 
 
-def nearest(X: np.ndarray, C: np.ndarray, chunk: int = 8192) -> np.ndarray:
+NEAR_TIE_REL = 1e-12
+
+
+def count_near_ties(D: np.ndarray) -> int:
+    """Rows of a distance matrix whose two smallest squared distances
+    d1 <= d2 satisfy d2 - d1 <= 1e-12 d2: rows whose nearest centroid is
+    decided by rounding rather than by the data (reading: the survey's
+    "several correct results" point; exact ties, e.g. two identical
+    centroids, count, and the lowest index wins them)."""
+    if D.shape[1] < 2:
+        return 0
+    two = np.partition(D, 1, axis=1)[:, :2]
+    return int(np.count_nonzero(two[:, 1] - two[:, 0] <= NEAR_TIE_REL * two[:, 1]))
+
+
+def nearest(X: np.ndarray, C: np.ndarray, chunk: int = 8192, ties: Optional[list] = None):
     """Index of the nearest centroid of every row (lowest index on ties).
-    Rows are independent; they are evaluated in chunks to bound memory."""
+    Rows are independent; they are evaluated in chunks to bound memory.
+    ``ties``: if a list, the count of near-tie rows is appended to it."""
     out = np.empty(X.shape[0], dtype=np.int64)
+    nt = 0
     for s in range(0, X.shape[0], chunk):
-        out[s:s + chunk] = np.argmin(sqdist(X[s:s + chunk], C), axis=1)
+        D = sqdist(X[s:s + chunk], C)
+        out[s:s + chunk] = np.argmin(D, axis=1)
+        if ties is not None:
+            nt += count_near_ties(D)
+    if ties is not None:
+        ties.append(nt)
     return out
 
 
-def lloyd(X: np.ndarray, init: np.ndarray, iters: int):
+def lloyd(X: np.ndarray, init: np.ndarray, iters: int, ties: Optional[list] = None):
     """Lloyd k-means: assign every row to its nearest centroid (lowest index
     on ties), stop when no label changes, else move each centroid to its
     group mean (an empty group keeps its centroid). At most ``iters``
-    assignment passes. Returns (labels, centroids, passes).
+    assignment passes. Returns (labels, centroids, passes); ``ties``, if a
+    list, receives the near-tie count of every pass.
 
     Reading: the pages fix neither init, stopping nor empty groups; SVOO's
     note says single-digit iteration counts suffice."""
@@ -150,7 +173,7 @@ def lloyd(X: np.ndarray, init: np.ndarray, iters: int):
     labels = None
     passes = 0
     for _ in range(iters):
-        new = nearest(X, mu)  # first minimum = lowest index
+        new = nearest(X, mu, ties=ties)  # first minimum = lowest index
         passes += 1
         if labels is not None and np.array_equal(new, labels):
             break
@@ -166,8 +189,9 @@ def key_partition(k_video, q_video, Ck, Ms, e, iters, seed, head):
     lam_e, U_e = eigenbasis(MK, e)
     Z = key_coordinates(k_video, lam_e, U_e)
     init = init_indices(k_video.shape[0], Ck, seed, head, 0)
-    labels, _, passes = lloyd(Z, init, iters)
-    return labels, dict(MK=MK, lam=lam_e, U=U_e, Z=Z, passes=passes)
+    ties = []
+    labels, _, passes = lloyd(Z, init, iters, ties)
+    return labels, dict(MK=MK, lam=lam_e, U=U_e, Z=Z, passes=passes, near_ties=sum(ties))
 
 
 def query_profiles(q_video: np.ndarray, CK: np.ndarray, scale: float) -> np.ndarray:
@@ -183,8 +207,9 @@ def query_partition(q_video, CK, Cq, iters, seed, head, scale):
     queries, no alternation."""
     P = query_profiles(q_video, CK, scale)
     init = init_indices(q_video.shape[0], Cq, seed, head, 1)
-    labels, _, passes = lloyd(P, init, iters)
-    return labels, dict(passes=passes)
+    ties = []
+    labels, _, passes = lloyd(P, init, iters, ties)
+    return labels, dict(passes=passes, near_ties=sum(ties))
 
 
 def semantic_partition(q_video, k_video, Ck, Cq, iters, seed, head):
@@ -475,7 +500,8 @@ def run_head(q, k, v, p: dict, head: int, rows=None, partition_only=False) -> He
     perm_q, inv_q, off_q = group_major(label_q, Cqt)
     perm_k, inv_k, off_k = group_major(label_k, Ckt)
     info = dict(key_passes=kinfo["passes"], query_passes=qinfo["passes"],
-                MK=kinfo["MK"], eig_lam=kinfo["lam"], eig_U=kinfo["U"])
+                MK=kinfo["MK"], eig_lam=kinfo["lam"], eig_U=kinfo["U"],
+                key_near_ties=kinfo.get("near_ties"), query_near_ties=qinfo.get("near_ties"))
     kk = keep_budget(float(p["keep"][head] if isinstance(p["keep"], (list, tuple)) else p["keep"]), Ck)
     if partition_only:
         return HeadResult(label_q, label_k, perm_q, perm_k, off_q, off_k, kk,

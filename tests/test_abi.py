@@ -31,7 +31,30 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(S._LIB_PATH)
     for n in declared_functions():
         assert hasattr(lib, n), n
-    assert set(declared_functions()) <= set(S.EXPORTED) | set(declared_functions())
+    assert set(declared_functions()) == set(S.EXPORTED)
+
+
+def test_workspace_regions_lie_inside_the_workspace_and_do_not_overlap():
+    w = synth.workload("wan13b_480p")
+    p = w.params()
+    total = S.workspace_bytes(p)
+    d, e, H = w.d, w.n_eig, w.H
+    want = dict(init_k=H * w.Ck * 4, init_q=H * w.Cq * 4, mk=H * d * d * 8, eval=H * e * 8,
+                evec=H * d * e * 8, wk=H * d * e * 8, z=H * w.Nv * e * 8, ck=H * w.Ck * d * 8,
+                g=H * d * d * 8, bmat=H * d * d * 8, bvec=H * d * 8)
+    spans = []
+    for name, nb in want.items():
+        off, got = S.sparsepr_workspace_region(p, name)
+        assert got == nb, name
+        assert off % 256 == 0 and off + nb <= total, name
+        spans.append((off, off + nb, name))
+    spans.sort()
+    for (a0, a1, n0), (b0, b1, n1) in zip(spans, spans[1:]):
+        assert a1 <= b0, (n0, n1)
+    for bad in ("", "Z", "mk ", "nope"):
+        with pytest.raises(S.SparsePRError) as ei:
+            S.sparsepr_workspace_region(p, bad)
+        assert ei.value.code == S.ERR_INVALID_ARG
 
 
 def test_params_struct_layout():

@@ -109,6 +109,26 @@ def test_nearest_brute_force_and_ties():
     assert O.nearest(np.array([[0.0, 0.0], [2.0, 0.0]]), C2).tolist() == [0, 0]
 
 
+def test_near_tie_count_hand_example_and_identical_centroids():
+    D = np.array([[1.0, 1.0, 3.0],                # exact tie
+                  [0.0, 2.0, 5.0],                # clear gap
+                  [5.0, 5.0 * (1 + 1e-13), 9.0],  # gap 5e-13 <= 1e-12 * d2
+                  [5.0, 5.0 * (1 + 1e-11), 1.0],  # the two smallest are 1 and 5
+                  [2.0, 2.0 * (1 + 5e-12), 7.0]])  # gap above 1e-12 * d2
+    assert O.count_near_ties(D) == 2
+    assert O.count_near_ties(np.ones((3, 1))) == 0  # one centroid: no second distance
+    # two identical centroids: every row nearest to them is a tie (brute force)
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((200, 4))
+    C = rng.standard_normal((5, 4))
+    C[3] = C[1]
+    ties = []
+    lab = O.nearest(X, C, ties=ties)
+    brute = sum(1 for x in X
+                if min(range(5), key=lambda j: (float(((x - C[j]) ** 2).sum()), j)) == 1)
+    assert ties == [brute] and brute > 0 and not np.any(lab == 3)
+
+
 def test_lloyd_fixed_point_and_planted_recovery():
     rng = np.random.default_rng(4)
     centers = rng.standard_normal((5, 4)) * 20
@@ -352,6 +372,29 @@ def test_keep_one_is_dense_with_zero_residual():
     assert np.abs(res.o_dense_probe - res.o_sparse_probe).max() < 1e-12
     assert np.abs(res.B).max() < 1e-9 and np.abs(res.b).max() < 1e-9
     assert res.pairs_exec == w.N * w.N + w.M * w.N  # rho = 1 + M/N
+
+
+def test_hard_drop_is_the_sparse_output_of_every_row():
+    """M = 0, the hard-drop variant of the ablations ([SPR] 4): no probes, no
+    fitted map, every row's output is its masked (kept-logit) attention, and
+    the executed pairs are the routed pairs alone. The sparse rows are
+    recomputed here with explicit loops from the routes and key ranges."""
+    w, q, k, v = _tiny_head()
+    p = dict(w.params(), M=0)
+    res = O.run_head(q, k, v, p, 0)
+    assert res.probes.size == 0 and res.pairs_exec == res.pairs_sparse
+    assert np.all(res.Bp == 0) and np.all(res.bp == 0)
+    assert np.array_equal(res.out, res.o_sparse)
+    Qp, Kp, Vp = q[res.perm_q], k[res.perm_k], v[res.perm_k]
+    s = 1 / math.sqrt(w.d)
+    for i in range(0, w.N, 7):
+        g = int(np.searchsorted(res.off_q, i, side="right") - 1)
+        keys = [j for c in res.csr[g] for j in range(res.off_k[c], res.off_k[c + 1])]
+        logits = [s * float(Qp[i] @ Kp[j]) for j in keys]
+        m = max(logits)
+        wts = [math.exp(x - m) for x in logits]
+        o = sum(wv * Vp[j] for wv, j in zip(wts, keys)) / sum(wts)
+        assert np.abs(res.out[i] - o).max() < 1e-12
 
 
 def test_tiny_head_invariants():

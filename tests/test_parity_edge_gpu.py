@@ -22,4 +22,7 @@ def test_repeated_rows_and_tied_initial_centroids():
     b, _ = gpu_run(w, q, k, v)
     res = oracle_head(w, q, k, v, 0)
     compare_head(b, res, w, 0, None)
-    assert S.sparsepr_read_stats(b.ws)["status"] == 0
+    st = S.sparsepr_read_stats(b.ws)
+    assert st["status"] == 0
+    # the tied rows are counted alike on both sides
+    assert st["near_ties"] == [res.info["key_near_ties"], res.info["query_near_ties"]]

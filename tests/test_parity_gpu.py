@@ -30,6 +30,7 @@ def test_tiny_full_pipeline():
     assert st["status"] == 0
     assert st["key_passes"][0] == res.info["key_passes"]
     assert st["query_passes"][0] == res.info["query_passes"]
+    assert st["near_ties"] == [res.info["key_near_ties"], res.info["query_near_ties"]]
     # the fitted map
     fit = np_(b.fit[0])
     d = w.d
@@ -76,10 +77,15 @@ SMALL = [
 @pytest.mark.parametrize("w", SMALL, ids=[x.name for x in SMALL])
 def test_small_full_pipeline(w):
     b, (q, k, v) = gpu_run(w, fill=0xFF)
+    ties = [0, 0]
     for h in range(w.H):
         res = oracle_head(w, q, k, v, h)
         compare_head(b, res, w, h, None)
-    assert _S().sparsepr_read_stats(b.ws)["status"] == 0
+        ties[0] += res.info["key_near_ties"]
+        ties[1] += res.info["query_near_ties"]
+    st = _S().sparsepr_read_stats(b.ws)
+    assert st["status"] == 0
+    assert st["near_ties"] == ties
 
 
 def test_keep_one_matches_dense_attention():
