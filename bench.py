@@ -52,8 +52,8 @@ def workload_desc(w):
 
 
 # DRAM traffic of the routed attention launch on the 720p workload from one ncu
-# capture (profiles/sparse_attn_kernel_wan13b_720p_traffic.md), valid for the
-# attention source it was taken on.
+# capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
+# attention source it was taken on (hash of attn.cu below).
 ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=724185600 + 449008640,
                     source_sha256_prefix="d4a872a215d524c3")
 
@@ -80,7 +80,7 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")

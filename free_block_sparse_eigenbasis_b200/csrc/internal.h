@@ -143,11 +143,8 @@ cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals
 // ---- permute.cu ------------------------------------------------------------
 cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, int H, int N,
                                int d, int elem_bytes, cudaStream_t st);
-cudaError_t launch_route(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
-                         double scale, const int32_t* kh, int kmax, int32_t* csr,
-                         cudaStream_t st);
-// Workspace path: score GEMM + warp top-k, heads in groups whose scores fit
-// in `scores` (route_scores_bytes(H, Cq, Ck) bytes).
+// Score GEMM + warp top-k, heads in groups whose scores fit in `scores`
+// (route_scores_bytes(H, Cq, Ck) bytes in the workspace).
 size_t route_scores_bytes(int H, int Cq, int Ck);
 cudaError_t launch_route_gemm(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
                               double scale, const int32_t* kh, int kmax, double* scores,

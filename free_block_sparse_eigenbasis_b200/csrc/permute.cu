@@ -22,97 +22,8 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ src, uint4* __restr
   dst[t] = __ldg(src + srow * vec_per_row + v);
 }
 
-// One CTA per (query group g, head h): fp64 scores of all key groups in
-// shared memory (one warp per key group), a bitonic sort of (score, id)
-// pairs into the route order (greater score first, lower id on ties), and
-// the first k ids written in ascending order.
-constexpr int kRouteThreads = 256;
-
-__device__ __forceinline__ bool route_before(double sa, int ia, double sb, int ib) {
-  return sa > sb || (sa == sb && ia < ib);
-}
-
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(const double* __restrict__ cq,
-                                                              const double* __restrict__ ckr,
-                                                              int Cq, int Ck, int d, double scale,
-                                                              const int32_t* __restrict__ kh,
-                                                              int kmax, int P,
-                                                              int32_t* __restrict__ csr) {
-  extern __shared__ double rsm[];
-  double* score = rsm;                                       // [P], P = pow2 >= Ck
-  double* qv = rsm + P;                                      // [d]
-  int* ids = reinterpret_cast<int*>(qv + d);                 // [P]
-  int* kept = ids + P;                                       // [Ck]
-  __shared__ int wsum[kRouteThreads / 32];
-  __shared__ int carry;
-  const int g = blockIdx.x, h = blockIdx.y;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const double* qrow = cq + (static_cast<size_t>(h) * Cq + g) * d;
-  for (int a = threadIdx.x; a < d; a += blockDim.x) qv[a] = qrow[a];
-  __syncthreads();
-  const double* ckh = ckr + static_cast<size_t>(h) * Ck * d;
-  for (int c = wid; c < Ck; c += kRouteThreads / 32) {
-    const double* kr = ckh + static_cast<size_t>(c) * d;
-    double acc = 0.0;
-    for (int a = lane; a < d; a += 32) acc = fma(qv[a], kr[a], acc);
-    acc = warp_sum_f64(acc);
-    if (lane == 0) score[c] = scale * acc;
-  }
-  for (int c = threadIdx.x; c < P; c += blockDim.x) {
-    ids[c] = c;
-    if (c >= Ck) score[c] = -INFINITY;  // padding sorts last
-  }
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < (P >> 1); t += blockDim.x) {
-        const int lo = 2 * stride * (t / stride) + (t % stride), hi = lo + stride;
-        const double sa = score[lo], sb = score[hi];
-        const int ia = ids[lo], ib = ids[hi];
-        const bool in_order = route_before(sa, ia, sb, ib);
-        if (((lo & size) == 0) != in_order) {
-          score[lo] = sb;
-          score[hi] = sa;
-          ids[lo] = ib;
-          ids[hi] = ia;
-        }
-      }
-      __syncthreads();
-    }
-  }
-  const int k = kh[h];
-  for (int c = threadIdx.x; c < Ck; c += blockDim.x) kept[c] = 0;
-  __syncthreads();
-  for (int r = threadIdx.x; r < k; r += blockDim.x) kept[ids[r]] = 1;
-  __syncthreads();
-  // ascending compaction of the kept ids (block-wide exclusive scan)
-  int32_t* out = csr + (static_cast<size_t>(h) * Cq + g) * kmax;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int base = 0; base < Ck; base += blockDim.x) {
-    const int c = base + threadIdx.x;
-    const int f = (c < Ck) ? kept[c] : 0;
-    int x = f;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) wsum[wid] = x;
-    __syncthreads();
-    int before = carry;
-    for (int w = 0; w < wid; ++w) before += wsum[w];
-    before += x - f;
-    if (f) out[before] = c;
-    __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry = before + f;
-    __syncthreads();
-  }
-  for (int i = k + threadIdx.x; i < kmax; i += blockDim.x) out[i] = -1;
-}
-
 // ---------------------------------------------------------------------------
-// Routing in two kernels for the workspace path: the block-score matrix
+// Routing in two kernels: the block-score matrix
 // S_h = scale * C_Q C_K^T of a group of heads as one fp64 GEMM (64 x 64 tiles,
 // 4 x 4 outputs per thread, dot products summed in ascending column order),
 // then one warp per query group selects the top-k key groups by a radix
@@ -272,21 +183,6 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, 
   const size_t total = static_cast<size_t>(H) * N * vec;
   gather_rows_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
       static_cast<const uint4*>(src), static_cast<uint4*>(dst), perm, N, vec, total);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_route(const double* cq, const double* ckr, int H, int Cq, int Ck, int d,
-                         double scale, const int32_t* kh, int kmax, int32_t* csr,
-                         cudaStream_t st) {
-  int P = 2;
-  while (P < Ck) P <<= 1;
-  const size_t shb = static_cast<size_t>(P) * 8 + static_cast<size_t>(d) * 8 +
-                     static_cast<size_t>(P) * 4 + static_cast<size_t>(Ck) * 4;
-  cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(shb));
-  if (e != cudaSuccess) return e;
-  route_kernel<<<dim3(Cq, H), kRouteThreads, shb, st>>>(cq, ckr, Cq, Ck, d, scale, kh, kmax, P,
-                                                        csr);
   return cudaGetLastError();
 }
 

@@ -175,11 +175,14 @@ int32_t sparsepr_route_width(const sparsepr_params* p);
  * device memory or pass a workspace (code that must not trigger the implicit
  * device synchronisation of cudaMalloc, or that works inside a memory pool
  * reserved up front). No counterpart in the paper: it is a memory-management
- * variant of the routing call above, with the same arguments (minus ws) and
- * the same outputs.
- * Its scratch is one fixed 4 MiB device array per GPU, held from the moment
- * the library is loaded until the process exits; heads are processed in
- * chunks that fit. A single head needs (Cq + Ck) * d * 8 bytes; larger
+ * variant of the routing call above, with the same arguments (minus ws), the
+ * same kernels and therefore the same routes, bit for bit.
+ * Its scratch is one fixed 8 MiB device array per GPU, held until the
+ * process exits. Under CUDA's default lazy module loading the array is
+ * committed by the first call on each device (that call may allocate and
+ * synchronise); with eager loading (CUDA_MODULE_LOADING=EAGER) it is
+ * committed when the library is loaded. Heads are processed in chunks that
+ * fit: a single head needs ((Cq + Ck) * d + Cq * Ck) * 8 bytes, and larger
  * parameters are rejected with SPARSEPR_ERR_WORKSPACE before anything is
  * enqueued. It calls no allocating routine.
  * The first call on each device looks up the array's device address with
@@ -187,7 +190,7 @@ int32_t sparsepr_route_width(const sparsepr_params* p);
  * All calls share the array and the last call's contents stay in it (every
  * call overwrites what it reads, nothing needs clearing). Calls that overlap
  * on the GPU race on the array: issue them in order on one stream.
- * Parameters with text tokens (n_text > 0) return SPARSEPR_ERR_UNSUPPORTED. */
+ * qp and kp must be 16-byte aligned (SPARSEPR_ERR_INVALID_ARG otherwise). */
 sparsepr_status sparsepr_route_noalloc(const void* qp, const void* kp, sparsepr_dtype dt,
                                        const sparsepr_params* p, const int32_t* off_q,
                                        const int32_t* off_k, int32_t* csr,

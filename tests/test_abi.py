@@ -168,3 +168,20 @@ def test_header_is_plain_c_and_a_c_program_links_and_runs(tmp_path):
     assert int(out[0]) == S.workspace_bytes(p)
     assert int(out[1]) == S.route_width(p)
     assert " ".join(out[2:]) == S.status_string(S.ERR_TIMEOUT)
+
+
+def test_route_noalloc_rejects_misaligned_and_oversized_before_any_launch():
+    w = synth.custom("noalloc_cpu", 1, (4, 16, 32), 128, "bf16", Ck=64, Cq=16, Ms=256, n_eig=8,
+                     M=64, r=16, keep=0.25, seed=11)
+    prm, keep = S.make_params(w.params())
+    fake = ctypes.c_void_p(1 << 40)  # never touched: every case fails on the host
+    odd = ctypes.c_void_p((1 << 40) + 4)
+    f = S.lib.sparsepr_route_noalloc
+    assert f(odd, fake, S.BF16, ctypes.byref(prm), fake, fake, fake, fake, None) == S.ERR_INVALID_ARG
+    assert f(fake, odd, S.BF16, ctypes.byref(prm), fake, fake, fake, fake, None) == S.ERR_INVALID_ARG
+    assert f(fake, fake, 7, ctypes.byref(prm), fake, fake, fake, fake, None) == S.ERR_UNSUPPORTED
+    assert f(fake, fake, S.BF16, ctypes.byref(prm), None, fake, fake, fake, None) == S.ERR_INVALID_ARG
+    big = synth.custom("noalloc_big", 1, (4, 32, 64), 128, "bf16", Ck=1100, Cq=900, Ms=64,
+                       n_eig=4, M=16, r=8, keep=0.1, seed=1)  # (2000*128 + 990000)*8 > 8 MiB
+    prm2, keep2 = S.make_params(big.params())
+    assert f(fake, fake, S.BF16, ctypes.byref(prm2), fake, fake, fake, fake, None) == S.ERR_WORKSPACE
