@@ -23,9 +23,13 @@
 //   * a unit of one query tile splits the key tiles instead (even ones to
 //     warpgroup 0, odd ones to warpgroup 1) with separate running maxima
 //     and accumulators, merged at the end;
-//   * P V reads P from tensor memory (no shared-memory round trip); O is
-//     rescaled only when a row maximum grows by more than 2^8, and O and the
-//     row sum always share one reference maximum, so the result is exact.
+//   * P V reads P from tensor memory (no shared-memory round trip). The
+//     softmax streams each row in two halves of 64 columns against a
+//     reference maximum taken from the first key tile, with no maximum pass
+//     afterwards; a half whose sum exceeds 2^32 is formed again against a
+//     reference raised by a whole number of log2 units, and O, the row sum
+//     and the stored half are scaled by that power of two. O and the row
+//     sum always share one reference, so the result is exact.
 // Every mbarrier wait is bounded; a wait that runs out marks the status word
 // and the CTA drains its in-flight copies and MMAs, frees tensor memory and
 // returns.
@@ -41,7 +45,7 @@ constexpr int kUnitRows = 2 * kTileM;              // query rows per CTA
 constexpr int kAttnThreads = 352;  // 8 softmax warps, K TMA warp (8), MMA warp (9), V TMA warp (10)
 constexpr uint32_t kTmemCols = 512;  // S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 after
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kOverflowSum = 4294967296.0f;  // 2^32: a larger half sum moves the reference
 
 template <int HD>
 struct Smem {
@@ -147,6 +151,14 @@ __device__ __forceinline__ void fma2(float& x0, float& x1, float a0, float a1, f
       "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(x0), "=f"(x1)
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+// packed fp32x2 add: (x.x, x.y) += (a, b)
+__device__ __forceinline__ void add2(float2& x, float a, float b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(x.x), "=f"(x.y)
+      : "f"(x.x), "f"(x.y), "f"(a), "f"(b));
 }
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -399,66 +411,106 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // tcgen05.ld / st below are warp-collective: the warp proceeds or stops as one
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], t & 1, abort))) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[kTileN];
+      // The row is processed in two halves of 64 key columns: S half hf is
+      // loaded, exponentiated and packed, and its P stored over columns
+      // [32 hf, 32 hf + 32) of S_i, columns that hold S values already read.
+      uint32_t r[kTileN / 2];
+      auto load_half = [&](int hf) {
+        tmem_ld32(s_tmem + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
+        tmem_ld32(s_tmem + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_wait_ld();
+        if ((vm[2 * hf] & vm[2 * hf + 1]) != 0xFFFFFFFFu) {
+          // only partial or padding slots (the same for every row) are touched
 #pragma unroll
-      for (int c = 0; c < kTileN / 32; ++c)
-        tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
-      tmem_wait_ld();
-      if ((vm[0] & vm[1] & vm[2] & vm[3]) != 0xFFFFFFFFu) {
-        // only partial or padding slots (the same for every row) are touched
+          for (int sl = 0; sl < kSlotsPerTile / 2; ++sl) {
+            const uint32_t b = (vm[2 * hf + (sl >> 2)] >> ((sl & 3) * 8)) & 0xFFu;
+            if (b != 0xFFu) {
 #pragma unroll
-        for (int sl = 0; sl < kSlotsPerTile; ++sl) {
-          const uint32_t b = (vm[sl >> 2] >> ((sl & 3) * 8)) & 0xFFu;
-          if (b != 0xFFu) {
-#pragma unroll
-            for (int q = 0; q < kSlotRows; ++q)
-              if (!((b >> q) & 1u)) r[sl * kSlotRows + q] = __float_as_uint(-INFINITY);
+              for (int q = 0; q < kSlotRows; ++q)
+                if (!((b >> q) & 1u)) r[sl * kSlotRows + q] = __float_as_uint(-INFINITY);
+            }
           }
         }
-      }
-      // row maximum: eight independent chains of three-input maxima, then a tree
-      float m8[8];
+      };
+      // scaled maximum of the loaded half: eight chains of three-input maxima
+      auto half_max = [&]() -> float {
+        float m8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(r[k]);
+        for (int k = 0; k < 8; ++k) m8[k] = __uint_as_float(r[k]);
 #pragma unroll
-      for (int c = 8; c < kTileN; c += 2)
-        m8[(c >> 1) & 7] = max3f(m8[(c >> 1) & 7], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
-      const float mx = sc * fmaxf(max3f(m8[0], m8[1], m8[2]),
-                                  fmaxf(max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      // reference maximum (moves only when it grows by more than 2^8)
-      float alpha = 1.f;
-      bool need = false;
-      if (t == 0) {
-        m_ref = mx;
-      } else if (mx > m_ref + kRescaleThreshold) {
-        need = true;
-        alpha = ex2_approx(m_ref - mx);
-        m_ref = mx;
-      }
-      // P = 2^(s sc - m_ref) as bf16 pairs over the first 64 columns of S_i;
-      // row sum in fp32 (eight chains). S_i(t) was produced
-      // after P_i(t-1) V completed, so these columns are free.
-      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const float nm = -m_ref;
+        for (int c = 8; c < kTileN / 2; c += 2)
+          m8[(c >> 1) & 7] = max3f(m8[(c >> 1) & 7], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        return sc * fmaxf(max3f(m8[0], m8[1], m8[2]),
+                          fmaxf(max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      };
+      // P = 2^(s sc - m_ref) of the loaded half as bf16 pairs; returns its sum
+      uint32_t pk[32];
+      auto exp_half = [&](float mref) -> float {
+        float2 r4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        const float nm = -mref;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
+        for (int c = 0; c < kTileN / 2; c += 2) {
           float xa, xb;
-          fma2(xa, xb, __uint_as_float(r[hf * 64 + c]), __uint_as_float(r[hf * 64 + c + 1]), sc, nm);
+          fma2(xa, xb, __uint_as_float(r[c]), __uint_as_float(r[c + 1]), sc, nm);
           const float a = ex2_approx(xa), b = ex2_approx(xb);
-          r8[(c >> 1) & 7] += a + b;
+          add2(r4[(c >> 1) & 3], a, b);
           pk[c >> 1] = pack_bf16x2(a, b);
         }
-        tmem_st32(s_tmem + hf * 32, pk);
+        return (r4[0].x + r4[0].y + r4[1].x + r4[1].y) + (r4[2].x + r4[2].y + r4[3].x + r4[3].y);
+      };
+      // Reference maximum m_ref: the first tile's row maximum; later tiles
+      // are exponentiated against it with no maximum pass. A half whose sum
+      // exceeds 2^32 (some value may exceed 2^32, or overflowed) moves the
+      // reference up by the whole number k of log2 units that brings its
+      // largest value to at most 1: its S is reloaded (P not yet stored over
+      // it) and its values formed again, and the P half already stored, the
+      // row sum and O are scaled by 2^-k, exactly. O and the row sum always
+      // share one reference, so the result is exact.
+      if (t == 0) {
+        load_half(0);
+        const float m0 = half_max();
+        load_half(1);
+        m_ref = fmaxf(m0, half_max());
       }
-      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      float alpha = 1.f, rs = 0.f;
+      bool need = false;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        load_half(hf);
+        float rh = exp_half(m_ref);
+        if (__any_sync(0xffffffffu, !(rh <= kOverflowSum))) {
+          const bool over = !(rh <= kOverflowSum);
+          load_half(hf);
+          float sh = 1.f;  // 2^-k, formed from its bits (0 when k >= 127)
+          if (over) {
+            const float k = ceilf(half_max() - m_ref);
+            sh = (k < 127.f) ? __int_as_float((127 - static_cast<int>(k)) << 23) : 0.f;
+            m_ref += k;
+            need = true;
+          }
+          alpha *= sh;
+          rs *= sh;
+          if (hf == 1 && __any_sync(0xffffffffu, sh != 1.f)) {
+            // the stored P half 0 follows the new reference (exact: a power of two)
+            uint32_t q[32];
+            tmem_ld32(s_tmem, q);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              q[c] = pack_bf16x2(__uint_as_float(q[c] << 16) * sh, __uint_as_float(q[c] & 0xFFFF0000u) * sh);
+            tmem_st32(s_tmem, q);
+          }
+          rh = exp_half(m_ref);
+        }
+        tmem_st32(s_tmem + hf * 32, pk);
+        rs += rh;
+      }
       if (__any_sync(0xffffffffu, need)) {
         // P_i(t-1) V has completed (it precedes S_i(t)); O_i is not read again
         // before P_i(t) is published below
         const uint32_t o_tmem = o_base + static_cast<uint32_t>(i * HD);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(o_tmem + c * 32, o);

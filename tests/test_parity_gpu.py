@@ -138,6 +138,35 @@ def test_dense_mode_against_textbook_attention(N):
         assert_close(np_(out[h]), D, "dense N=%d head %d" % (N, h))
 
 
+@pytest.mark.parametrize("N", [1024, 1124])
+def test_dense_mode_logit_jumps_move_the_reference(N):
+    """Keys whose logits exceed those of the first key tile by far more than
+    2^32 in probability (in the first and in the second half of later tiles,
+    and again further on): the online softmax moves its reference maximum
+    and rescales the stored values, O and the row sum; the result must still
+    be the textbook softmax attention. N = 1124 ends with a unit of one query
+    tile, whose two warpgroups split the key tiles and merge at the end."""
+    S = _S()
+    d = 128
+    g = torch.Generator().manual_seed(7)
+    q = torch.randn(2, N, d, generator=g)
+    k = torch.randn(2, N, d, generator=g)
+    v = torch.randn(2, N, d, generator=g)
+    q[:, :, 0] += 6.0
+    k[:, 128 + 70, 0] += 120.0  # tile 1, second half of its columns
+    k[:, 256 + 10, 0] += 120.0  # tile 2, first half
+    k[:, 640 + 100, 0] += 240.0  # tile 5: a further jump
+    k[1, 900, 0] -= 200.0  # a logit far below the reference
+    q, k, v = q.bfloat16(), k.bfloat16(), v.bfloat16()
+    out = torch.empty(2, N, d, device="cuda")
+    S.dense_attention(q.cuda(), k.cuda(), v.cuda(), out)
+    torch.cuda.synchronize()
+    for h in range(2):
+        D = O.dense_attention(q[h].double().numpy(), k[h].double().numpy(), v[h].double().numpy(),
+                              1 / math.sqrt(d))
+        assert_close(np_(out[h]), D, "logit jumps head %d" % h)
+
+
 def test_wan13b_480p_first_and_last_head():
     w = synth.workload("wan13b_480p")
     b, (q, k, v) = gpu_run(w)
