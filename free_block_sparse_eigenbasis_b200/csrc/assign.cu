@@ -460,14 +460,18 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// fp64 decision of the flagged rows: one block per flagged row (grid-stride
-// over the head's list). Thread j scores centroids j, j + 256, ... in
-// ascending order from the transposed centroid side yT [D, m], so the loads
-// of a warp are contiguous; four partial sums per dot product keep the fp64
-// pipes busy. Then a block argmin, lowest index on ties.
+// fp64 decision of the flagged rows, R rows per block at a time (grid stride
+// over the head's list): thread j scores centroids j, j + 256, ... in
+// ascending order from the transposed centroid side yT [D, m], each load of
+// yT (contiguous across the warp) serving the R rows of the batch, so the
+// centroid table streams from L2 once per batch instead of once per row
+// (R = 8 for rows of 64 or more columns; R = 1 for the short key rows, whose
+// few flagged rows are best spread over all blocks). Then per row the nearest
+// and second-nearest value (lowest index on ties) over the block.
 // direct = 1: d = sum_t (x_t - y_jt)^2; else d = c_j - 2 x . y_j.
 // ---------------------------------------------------------------------------
-constexpr int kRcThreads = 256, kRcMaxD = 128, kRcBlocksPerHead = 128;
+constexpr int kRcThreads = 256, kRcMaxD = 128, kRcRows = 8;
+constexpr int kRcWarps = kRcThreads / 32;
 
 __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   if (kind == kXf64) return static_cast<const double*>(X)[i];
@@ -475,71 +479,19 @@ __device__ __forceinline__ double ldx(const void* X, int kind, size_t i) {
   return static_cast<double>(static_cast<const float*>(X)[i]);
 }
 
-__device__ __forceinline__ void argmin_merge(double& best, int& bi, double ob, int oi) {
-  if (ob < best || (ob == best && oi < bi)) {
-    best = ob;
-    bi = oi;
-  }
-}
-
-// score of centroid j: DT > 0 fixes the length at compile time
-template <int DT, bool DIRECT>
-__device__ __forceinline__ double rc_score(const double* xs, const double* yT, int m, int j, int Drt,
-                                           const double* ch) {
-  const int D = DT > 0 ? DT : Drt;
-  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-  int t = 0;
-  auto step4 = [&](int t4, double y0, double y1, double y2, double y3) {
-    if (DIRECT) {
-      const double e0 = xs[t4] - y0, e1 = xs[t4 + 1] - y1, e2 = xs[t4 + 2] - y2, e3 = xs[t4 + 3] - y3;
-      a0 = fma(e0, e0, a0);
-      a1 = fma(e1, e1, a1);
-      a2 = fma(e2, e2, a2);
-      a3 = fma(e3, e3, a3);
-    } else {
-      a0 = fma(xs[t4], y0, a0);
-      a1 = fma(xs[t4 + 1], y1, a1);
-      a2 = fma(xs[t4 + 2], y2, a2);
-      a3 = fma(xs[t4 + 3], y3, a3);
-    }
-  };
-  // 16 loads in flight, then their products (column t goes to sum t % 4)
-#pragma unroll 1
-  for (; t + 16 <= D; t += 16) {
-    double y[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) y[q] = yT[static_cast<size_t>(t + q) * m + j];
-#pragma unroll
-    for (int q = 0; q < 16; q += 4) step4(t + q, y[q], y[q + 1], y[q + 2], y[q + 3]);
-  }
-  for (; t + 4 <= D; t += 4)
-    step4(t, yT[static_cast<size_t>(t) * m + j], yT[static_cast<size_t>(t + 1) * m + j],
-          yT[static_cast<size_t>(t + 2) * m + j], yT[static_cast<size_t>(t + 3) * m + j]);
-  for (; t < D; ++t) {
-    const double y = yT[static_cast<size_t>(t) * m + j];
-    if (DIRECT) {
-      const double e0 = xs[t] - y;
-      a0 = fma(e0, e0, a0);
-    } else {
-      a0 = fma(xs[t], y, a0);
-    }
-  }
-  const double sm = (a0 + a1) + (a2 + a3);
-  return DIRECT ? sm : ch[j] - 2.0 * sm;
-}
-
-template <int DT, bool DIRECT>
+template <int DT, bool DIRECT, int R>
 __global__ void __launch_bounds__(kRcThreads)
-    recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int D,
+    recheck_kernel(const void* X, int kind, long long hsx, int ldx_, int n, int Drt,
                    const double* yT, const double* c, int m, int32_t* labels, int32_t* flags,
                    int flag_base, const int32_t* recheck, const int32_t* nrecheck,
                    const double* G, DeviceStats* stats) {
-  __shared__ double xs[kRcMaxD];
-  __shared__ double wb1[kRcThreads / 32], wb2[kRcThreads / 32];
-  __shared__ int wbi[kRcThreads / 32];
+  __shared__ double xs[R][kRcMaxD];
+  __shared__ double wb1[R][kRcWarps], wb2[R][kRcWarps];
+  __shared__ int wbi[R][kRcWarps];
+  __shared__ int rows_s[R], cand_s[R];
+  __shared__ double gap_s[R], sec_s[R], xpart[kRcWarps];
   __shared__ double gtr;
-  __shared__ double xpart[kRcThreads / 32];
-  __shared__ int cand;
+  const int D = DT > 0 ? DT : Drt;
   const int h = blockIdx.y;
   int32_t* fl = flags + h * 4;
   if (fl[flag_base + 1]) return;
@@ -555,92 +507,163 @@ __global__ void __launch_bounds__(kRcThreads)
     gtr = t;
   }
   int ties = 0;
-  for (int k = blockIdx.x; k < cnt; k += gridDim.x) {
-    const int row = recheck[static_cast<size_t>(h) * n + k];
-    __syncthreads();  // xs and the warp results of the previous row are consumed
-    for (int t = threadIdx.x; t < D; t += blockDim.x)
-      xs[t] = ldx(X, kind, h * hsx + static_cast<size_t>(row) * ldx_ + t);
+  for (int k0 = blockIdx.x * R; k0 < cnt; k0 += gridDim.x * R) {
+    const int nb = min(R, cnt - k0);
+    __syncthreads();  // the previous batch's rows and results are consumed
+    if (threadIdx.x < R)
+      rows_s[threadIdx.x] = threadIdx.x < nb ? recheck[static_cast<size_t>(h) * n + k0 + threadIdx.x] : 0;
     __syncthreads();
-    Top2 t2 = top2_empty();
-    constexpr int kJUnroll = (DT > 0 && DT <= 16) ? 2 : 1;  // short rows: two centroids in flight
-#pragma unroll kJUnroll
-    for (int j = threadIdx.x; j < m; j += kRcThreads)  // ascending within the thread
-      top2_push(t2, rc_score<DT, DIRECT>(xs, Yh, m, j, D, ch), j);
+    for (int i = threadIdx.x; i < R * D; i += kRcThreads) {
+      const int r = i / D, t = i % D;
+      xs[r][t] = (r < nb) ? ldx(X, kind, h * hsx + static_cast<size_t>(rows_s[r]) * ldx_ + t) : 0.0;
+    }
+    __syncthreads();
+    Top2 t2[R];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double o1 = __shfl_xor_sync(0xffffffffu, t2.b1, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, t2.i1, o);
-      const double o2 = __shfl_xor_sync(0xffffffffu, t2.b2, o);
-      top2_merge(t2, o1, oi, o2);
+    for (int r = 0; r < R; ++r) t2[r] = top2_empty();
+    // scores of centroid j for the batch's rows: with the row length fixed at
+    // compile time the column loop is unrolled, so loads run ahead of the FMAs
+    auto score = [&](int j, double (&acc)[R]) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) acc[r] = 0.0;
+      auto step = [&](int t, double y) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (DIRECT) {
+            const double e = xs[r][t] - y;
+            acc[r] = fma(e, e, acc[r]);
+          } else {
+            acc[r] = fma(xs[r][t], y, acc[r]);
+          }
+        }
+      };
+      if (DT > 0 && DT <= 16) {
+#pragma unroll
+        for (int t = 0; t < DT; ++t) step(t, Yh[static_cast<size_t>(t) * m + j]);
+      } else if (DT > 0) {
+        // chunks of 8 columns, the next chunk's loads issued before this
+        // chunk's FMAs
+        double ya[8], yb[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ya[q] = Yh[static_cast<size_t>(q) * m + j];
+#pragma unroll 1
+        for (int t = 0; t < DT; t += 16) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) yb[q] = Yh[static_cast<size_t>(t + 8 + q) * m + j];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) step(t + q, ya[q]);
+          if (t + 16 < DT)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ya[q] = Yh[static_cast<size_t>(t + 16 + q) * m + j];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) step(t + 8 + q, yb[q]);
+        }
+      } else {
+        int t = 0;
+#pragma unroll 1
+        for (; t + 8 <= D; t += 8) {
+          double y[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) y[q] = Yh[static_cast<size_t>(t + q) * m + j];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) step(t + q, y[q]);
+        }
+        for (; t < D; ++t) step(t, Yh[static_cast<size_t>(t) * m + j]);
+      }
+    };
+    constexpr int kJU = (R == 1) ? 2 : 1;  // short rows: two centroids in flight
+#pragma unroll kJU
+    for (int j = threadIdx.x; j < m; j += kRcThreads) {  // ascending within the thread
+      double acc[R];
+      score(j, acc);
+#pragma unroll
+      for (int r = 0; r < R; ++r) top2_push(t2[r], DIRECT ? acc[r] : ch[j] - 2.0 * acc[r], j);
     }
-    if (lane == 0) {
-      wb1[w] = t2.b1;
-      wb2[w] = t2.b2;
-      wbi[w] = t2.i1;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double o1 = __shfl_xor_sync(0xffffffffu, t2[r].b1, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, t2[r].i1, o);
+        const double o2 = __shfl_xor_sync(0xffffffffu, t2[r].b2, o);
+        top2_merge(t2[r], o1, oi, o2);
+      }
+      if (lane == 0) {
+        wb1[r][w] = t2[r].b1;
+        wb2[r][w] = t2[r].b2;
+        wbi[r][w] = t2[r].i1;
+      }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      for (int q = 1; q < kRcThreads / 32; ++q) top2_merge(t2, wb1[q], wbi[q], wb2[q]);
-      const size_t li = static_cast<size_t>(h) * n + row;
-      if (labels[li] != t2.i1) atomicAdd(&fl[flag_base], 1);
-      labels[li] = t2.i1;
+    if (threadIdx.x < nb) {
+      const int r = threadIdx.x;
+      Top2 b = Top2{wb1[r][0], wb2[r][0], wbi[r][0]};
+      for (int q = 1; q < kRcWarps; ++q) top2_merge(b, wb1[r][q], wbi[r][q], wb2[r][q]);
+      const size_t li = static_cast<size_t>(h) * n + rows_s[r];
+      if (labels[li] != b.i1) atomicAdd(&fl[flag_base], 1);
+      labels[li] = b.i1;
       // near tie: DIRECT values are squared distances; otherwise they lack
       // x^T G x, formed below (by the whole block) for candidate rows only
-      const double gap = t2.b2 - t2.b1;
+      const double gap = b.b2 - b.b1;
       int cd = 0;
       if (m > 1) {
         if (DIRECT) {
-          ties += (gap <= kNearTieRel * t2.b2);
+          ties += (gap <= kNearTieRel * b.b2);
         } else if (Gh) {
           double xx = 0.0;
-          for (int a = 0; a < D; ++a) xx = fma(xs[a], xs[a], xx);
-          cd = gap <= 1e-11 * (fabs(t2.b2) + gtr * xx);
+          for (int a = 0; a < D; ++a) xx = fma(xs[r][a], xs[r][a], xx);
+          cd = gap <= 1e-11 * (fabs(b.b2) + gtr * xx);
         }
       }
-      cand = cd;
-      wb1[0] = gap;
-      wb2[0] = t2.b2;
+      cand_s[r] = cd;
+      gap_s[r] = gap;
+      sec_s[r] = b.b2;
     }
     if (!DIRECT) {
-      __syncthreads();  // cand, wb1[0] = gap and wb2[0] = second value are visible
-      if (cand) {       // block-uniform
+      __syncthreads();  // cand_s, gap_s, sec_s are visible
+      for (int r = 0; r < nb; ++r) {
+        if (!cand_s[r]) continue;  // block-uniform
         double part = 0.0;
-        for (int b = threadIdx.x; b < D; b += blockDim.x) {
+        for (int bcol = threadIdx.x; bcol < D; bcol += kRcThreads) {
           double gb = 0.0;
-          for (int a = 0; a < D; ++a) gb = fma(xs[a], Gh[static_cast<size_t>(a) * D + b], gb);
-          part = fma(gb, xs[b], part);
+          for (int a = 0; a < D; ++a) gb = fma(xs[r][a], Gh[static_cast<size_t>(a) * D + bcol], gb);
+          part = fma(gb, xs[r][bcol], part);
         }
         part = warp_sum_f64(part);
         if (lane == 0) xpart[w] = part;
         __syncthreads();
         if (threadIdx.x == 0) {
           double xgx = 0.0;
-          for (int q = 0; q < kRcThreads / 32; ++q) xgx += xpart[q];
-          ties += (wb1[0] <= kNearTieRel * (wb2[0] + xgx));
+          for (int q = 0; q < kRcWarps; ++q) xgx += xpart[q];
+          ties += (gap_s[r] <= kNearTieRel * (sec_s[r] + xgx));
         }
+        __syncthreads();  // xpart is free again
       }
     }
   }
-  if (threadIdx.x == 0 && ties)
+  if (ties)
     atomicAdd(reinterpret_cast<unsigned long long*>(&stats->near_ties[flag_base >> 1]),
               static_cast<unsigned long long>(ties));
 }
 
 template <bool DIRECT>
 void launch_recheck_d(const AssignTC& a, cudaStream_t st) {
-  const dim3 grid(kRcBlocksPerHead, a.H);
-#define SPR_RC(DT)                                                                          \
-  recheck_kernel<DT, DIRECT><<<grid, kRcThreads, 0, st>>>(                                 \
+  // short rows (D <= 16): one row per block over 128 blocks per head;
+  // longer rows: batches of kRcRows over 64 blocks per head
+#define SPR_RC(DT, R, NB)                                                                       \
+  recheck_kernel<DT, DIRECT, R><<<dim3(NB, a.H), kRcThreads, 0, st>>>(                        \
       a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D, a.y_tr, a.c_exact, a.m, a.labels, a.flags, \
       a.flag_base, a.recheck, a.nrecheck, a.metric, a.stats)
   if (a.D == 16)
-    SPR_RC(16);
+    SPR_RC(16, 1, 128);
   else if (a.D == 64)
-    SPR_RC(64);
+    SPR_RC(64, kRcRows, 64);
   else if (a.D == 128)
-    SPR_RC(128);
+    SPR_RC(128, kRcRows, 64);
+  else if (a.D < 16)
+    SPR_RC(0, 1, 128);
   else
-    SPR_RC(0);
+    SPR_RC(0, kRcRows, 64);
 #undef SPR_RC
 }
 

@@ -622,6 +622,77 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
   }
 }
 
+// Warp form of the group mean for short rows (D * sizeof(T) <= 128 bytes,
+// TPR = D * sizeof(T) / 16 <= 8 threads per row): one warp per group, eight
+// groups per CTA; lane l sums the 16-byte piece l % TPR of the rows
+// lo + l / TPR, lo + l / TPR + 32 / TPR, ... (four rows per lane in flight),
+// then the lanes that share a piece are added by shuffles in a fixed order.
+constexpr int kMeanWarpGroups = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kMeanWarpGroups * 32) group_mean_warp_kernel(
+    const T* X, long long hsx, int ldx, int D, const int32_t* perm, int perm_stride,
+    const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
+    const int32_t* skip, int skip_stride) {
+  constexpr int EPT = 16 / sizeof(T);
+  const int h = blockIdx.y;
+  const int c = blockIdx.x * kMeanWarpGroups + static_cast<int>(threadIdx.x >> 5);
+  if (c >= C) return;  // the whole warp
+  if (skip && skip[h * skip_stride]) return;
+  const int lane = threadIdx.x & 31;
+  const int32_t* oo = off + static_cast<size_t>(h) * off_stride;
+  const int32_t* pp = perm ? perm + static_cast<size_t>(h) * perm_stride : nullptr;
+  const int lo = oo[c], hi = oo[c + 1], n = hi - lo;
+  const int TPR = D / EPT, RL = 32 / TPR;  // row lanes
+  const int col = (lane % TPR) * EPT, rl = lane / TPR;
+  const T* Xh = X + h * hsx + col;
+  double acc[EPT];
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) acc[i] = 0.0;
+  int p = lo + rl;
+#pragma unroll 1
+  for (; p + 3 * RL < hi; p += 4 * RL) {
+    size_t r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r[j] = pp ? static_cast<size_t>(pp[p + j * RL]) : static_cast<size_t>(p + j * RL);
+    uint4 u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[j] = *reinterpret_cast<const uint4*>(Xh + r[j] * ldx);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      double v[EPT];
+      vwiden16<T>(u[j], v);
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) acc[i] += v[i];
+    }
+  }
+#pragma unroll 1
+  for (; p < hi; p += RL) {
+    const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
+    double v0[EPT];
+    vload16(Xh + r0 * ldx, v0);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
+  }
+  for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  double* dst = out + (static_cast<size_t>(h) * C + c) * D;
+  double ss = 0.0;
+  if (lane < TPR) {
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) {
+      const double v = (n > 0) ? acc[i] / static_cast<double>(n) : (keep_prev ? dst[col + i] : 0.0);
+      dst[col + i] = v;
+      ss = fma(v, v, ss);
+    }
+  }
+  if (norms) {
+    ss = warp_sum_f64(ss);
+    if (lane == 0) norms[static_cast<size_t>(h) * C + c] = ss;
+  }
+}
+
 // W_g = G qbar_g, c_g = qbar_g^T G qbar_g (fp64, fixed-order reduction).
 // One CTA per (8 query centroids, head); thread a owns column a of W for the
 // CTA's centroids, so every element of G is read once per CTA.
@@ -776,6 +847,22 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx,
   const int es = (x_kind == kXf64) ? 8 : (x_kind == kXbf16 ? 2 : 4);
   const bool vec = (D * es) % 16 == 0 && kMeanThreads % (D * es / 16) == 0 && (ldx * es) % 16 == 0 &&
                    (hsx * es) % 16 == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+  if (vec && D * es <= 128) {
+    const dim3 wgrid((C + kMeanWarpGroups - 1) / kMeanWarpGroups, H);
+    if (x_kind == kXf64)
+      group_mean_warp_kernel<<<wgrid, kMeanWarpGroups * 32, 0, st>>>(
+          static_cast<const double*>(X), hsx, ldx, D, perm, perm_stride, off, off_stride, C,
+          keep_prev, out, norms, skip, skip_stride);
+    else if (x_kind == kXbf16)
+      group_mean_warp_kernel<<<wgrid, kMeanWarpGroups * 32, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(X), hsx, ldx, D, perm, perm_stride, off, off_stride, C,
+          keep_prev, out, norms, skip, skip_stride);
+    else
+      group_mean_warp_kernel<<<wgrid, kMeanWarpGroups * 32, 0, st>>>(
+          static_cast<const float*>(X), hsx, ldx, D, perm, perm_stride, off, off_stride, C,
+          keep_prev, out, norms, skip, skip_stride);
+    return cudaGetLastError();
+  }
   if (vec) {
     if (x_kind == kXf64)
       group_mean_vec_kernel<<<grid, kMeanThreads, 0, st>>>(static_cast<const double*>(X), hsx, ldx,
