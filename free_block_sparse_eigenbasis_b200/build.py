@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsparsepr.so")
 SOURCES = ["api.cu", "sort.cu", "partition.cu", "linalg.cu", "permute.cu", "attn.cu", "fit.cu",
-           "noalloc.cu", "assign.cu", "eigen.cu", "correct.cu"]
+           "noalloc.cu", "assign.cu", "eigen.cu", "correct.cu", "diag.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # -Werror=shadow: a launcher's local that shadows one of its parameters (say a
 # cudaError_t named like a size argument) silently changes the launch.

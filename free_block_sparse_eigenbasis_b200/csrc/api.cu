@@ -526,6 +526,7 @@ sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const
   a.nruns = at<int32_t>(ws, c.L.nruns);
   a.pairs = pairs_sparse;
   a.stats = c.stats;
+  a.lse = at<float>(ws, c.L.lse_s);
   SPR_TRY(launch_block_sparse_attn(a, c.st));
   return SPARSEPR_OK;
 }
@@ -590,6 +591,7 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     a.runs = reinterpret_cast<int2*>(meta + 8 * H);
     a.pairs = nullptr;
     a.stats = c.stats;
+    a.lse = at<float>(ws, L.lse_d);
     // few units (H * ceil(M / 256)) over all N keys: split the key tiles so
     // that about one CTA per SM runs
     {
@@ -664,6 +666,68 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out, c.bf16,
                            st));
   SPR_TRY(launch_pairs_exec(pairs_sparse, H, static_cast<int64_t>(M) * N, pairs_exec, c.stats, st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_probe_diagnostics(const sparsepr_params* p, const int32_t* probes,
+                                           double* mass, double* error, double* energy,
+                                           void* ws, size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, SPARSEPR_BF16, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!probes || !mass || !error || !energy || c.p.M < 1) return SPARSEPR_ERR_INVALID_ARG;
+  if (c.p.r > 64) return SPARSEPR_ERR_UNSUPPORTED;
+  const Layout& L = c.L;
+  // the leading right singular vectors of R as sparsepr_probe_correct left
+  // them: the eigen solver's output for r <= 32, the projector's selection in
+  // the Gram region otherwise
+  const double* vr = at<double>(ws, c.p.r <= 32 ? L.evec : L.gram);
+  SPR_TRY(launch_probe_diagnostics(probes, at<float>(ws, L.lse_s), at<float>(ws, L.lse_d),
+                                   at<double>(ws, L.xr), at<double>(ws, L.bmat),
+                                   at<double>(ws, L.bvec), vr, c.p.H, c.p.N, c.p.M, c.p.d, c.p.r,
+                                   mass, error, at<double>(ws, L.diag), energy, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_support_expansion(const void* qp, const void* kp, sparsepr_dtype dt,
+                                           const sparsepr_params* p, const int32_t* off_q,
+                                           const int32_t* off_k, double tau, int32_t group_stride,
+                                           double* individual, double* aggregate, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!qp || !kp || !off_q || !off_k || !individual || !aggregate || group_stride < 1 ||
+      !(tau > 0.0 && tau <= 1.0))
+    return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(qp, kp)) return SPARSEPR_ERR_INVALID_ARG;
+  int R = 0, P = 0;
+  if (support_smem_bytes(c.L.Ckt, c.p.d, &R, &P) == 0) return SPARSEPR_ERR_UNSUPPORTED;
+  const int H = c.p.H, Cq = c.p.Cq;
+  const size_t words = (static_cast<size_t>(c.L.Ckt) + 31) / 32;
+  uint32_t* bits = at<uint32_t>(ws, c.L.dscr);
+  auto* sums = at<unsigned long long>(ws, c.L.dscr + align256(static_cast<size_t>(H) * Cq * words * 4));
+  SPR_TRY(launch_support_expansion(qp, kp, c.bf16, off_q, c.L.Cqt + 1, off_k, c.L.Ckt, H, c.p.N,
+                                   c.p.d, Cq, group_stride, c.scale, tau, bits, sums, individual,
+                                   aggregate, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_density_profile(const void* q, const void* k, sparsepr_dtype dt,
+                                         const sparsepr_params* p, double tau, int32_t row_stride,
+                                         double* density, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  Ctx c;
+  sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!q || !k || !density || row_stride < 1 || !(tau > 0.0 && tau <= 1.0))
+    return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(q, k)) return SPARSEPR_ERR_INVALID_ARG;
+  const int H = c.p.H, N = c.p.N;
+  double* scr = at<double>(ws, c.L.dscr);
+  auto* cnt = at<unsigned long long>(ws, c.L.dscr + align256(static_cast<size_t>(kDiagRows) * N * 8));
+  SPR_TRY(launch_density(q, k, c.bf16, H, N, c.L.Nv, c.p.d, row_stride, c.scale, tau, scr, cnt,
+                         density, c.st));
   return SPARSEPR_OK;
 }
 

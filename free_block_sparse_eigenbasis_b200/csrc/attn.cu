@@ -103,6 +103,7 @@ struct AttnParams {
   int splits, units;  // split-KV (splits > 1): partial outputs per (unit, split)
   float* opart;
   float* lpart;
+  float* lse;  // [H, q_rows] log2-sum-exp of each row's scaled logits (may be null)
 };
 
 // Key-column validity of the key tiles of one query group, walked in
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x) * HD;
       for (int c = 0; c < HD; c += 4) *reinterpret_cast<float4*>(o + c) = make_float4(0, 0, 0, 0);
       if (partial) p.lpart[pbase + threadIdx.x] = -INFINITY;
+      else if (p.lse) p.lse[static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x] = -INFINITY;
     }
     return;
   }
@@ -535,6 +537,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float* orow = partial ? p.opart + (pbase + i * kTileM + row) * HD
                               : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row) * HD;
         if (partial && valid) p.lpart[pbase + i * kTileM + row] = m_ref + __log2f(l_sum);
+        if (!partial && valid && p.lse)
+          p.lse[static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row] = m_ref + __log2f(l_sum);
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
@@ -570,6 +574,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float* orow = partial ? p.opart + (pbase + row) * HD
                               : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + row) * HD;
         if (partial && valid && i == 0) p.lpart[pbase + row] = mm + __log2f(l0 * a0 + l1 * a1);
+        if (!partial && valid && i == 0 && p.lse)
+          p.lse[static_cast<size_t>(h) * p.q_rows + row0 + row] = mm + __log2f(l0 * a0 + l1 * a1);
 #pragma unroll
         for (int c = 0; c < HD / 64; ++c) {
           const int col = i * (HD / 2) + c * 32;
@@ -755,7 +761,7 @@ __global__ void __launch_bounds__(kSpWarps * 32)
 __global__ void split_combine_kernel(const float* opart, const float* lpart, const int32_t* off_q,
                                      const int32_t* work, const int32_t* nwork, int Cq,
                                      int tiles_per_head, int units, int splits, int q_rows, int d,
-                                     float* out) {
+                                     float* out, float* lse) {
   const int h = blockIdx.z, wi = blockIdx.y;
   if (wi >= nwork[h]) return;
   const int wcode = work[static_cast<size_t>(h) * tiles_per_head + wi];
@@ -786,6 +792,8 @@ __global__ void split_combine_kernel(const float* opart, const float* lpart, con
   const float inv = den > 0.f ? 1.f / den : 0.f;
   *reinterpret_cast<float4*>(out + (static_cast<size_t>(h) * q_rows + row0 + r) * d + c) =
       make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+  if (lse && c == 0)
+    lse[static_cast<size_t>(h) * q_rows + row0 + r] = den > 0.f ? L + __log2f(den) : -INFINITY;
 }
 
 __global__ void zero_i64_kernel(int64_t* p, int n) {
@@ -854,7 +862,7 @@ cudaError_t launch_attn_hd(const AttnArgs& a, AttnParams prm, cudaStream_t st) {
   if (prm.splits > 1)
     split_combine_kernel<<<dim3(kUnitRows / (256 / (HD / 4)), a.units, a.H), 256, 0, st>>>(
         a.opart, a.lpart, a.off_q, a.work, a.nwork, a.Cq, a.tiles_per_head, a.units, prm.splits,
-        a.q_rows, HD, a.out);
+        a.q_rows, HD, a.out, a.lse);
   return cudaGetLastError();
 }
 
@@ -889,6 +897,7 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   prm.units = a.units;
   prm.opart = a.opart;
   prm.lpart = a.lpart;
+  prm.lse = a.lse;
   if (prm.splits > 1 && (!a.opart || !a.lpart || a.units < 1)) return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

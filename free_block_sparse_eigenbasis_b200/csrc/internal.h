@@ -189,9 +189,30 @@ struct AttnArgs {
   int units = 0;
   float* opart = nullptr;
   float* lpart = nullptr;
+  // log2-sum-exp of every row's scaled logits over its kept keys (log2
+  // units: m + log2 l), [H, q_rows]; may be null
+  float* lse = nullptr;
 };
 cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st);
+
+// ---- diag.cu ---------------------------------------------------------------
+cudaError_t launch_probe_diagnostics(const int32_t* probes, const float* lse_s, const float* lse_d,
+                                     const double* xr, const double* bmat, const double* bvec,
+                                     const double* vr, int H, int N, int M, int d, int r,
+                                     double* mass, double* err, double* energy_rows,
+                                     double* energy, cudaStream_t st);
+
+cudaError_t launch_support_expansion(const void* qp, const void* kp, bool bf16,
+                                     const int32_t* off_q, int oq_stride, const int32_t* off_k,
+                                     int Ckt, int H, int N, int d, int Cqv, int stride,
+                                     double scale, double tau, uint32_t* union_bits,
+                                     unsigned long long* size_sum, double* indiv,
+                                     double* aggregate, cudaStream_t st);
+size_t support_smem_bytes(int Ckt, int d, int* R, int* P);
+cudaError_t launch_density(const void* q, const void* k, bool bf16, int H, int N, int Nv, int d,
+                           int row_stride, double scale, double tau, double* scratch,
+                           unsigned long long* count_sum, double* density, cudaStream_t st);
 
 // ---- fit.cu ----------------------------------------------------------------
 cudaError_t launch_probe_select(const int32_t* off_q, int off_stride, int H, int Cq, int M,

@@ -19,6 +19,7 @@ constexpr int kSortChunk = 1024;  // tokens per counting-sort chunk
 constexpr int kMaxGroups = 4096;
 constexpr int kMaxSplits = 8;   // split-KV ranges of the dense probe pass
 constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
+constexpr int kDiagRows = 64;   // density-profile rows processed at once (one CTA each)
 
 struct Layout {
   // statistics / status (always at offset 0)
@@ -86,6 +87,11 @@ struct Layout {
                    // nruns(1), runs(2 int2: run-list stride kmax + 1 = 2)
   size_t opart;    // [H, punits, kMaxSplits, 256, d] f32 split-KV partial outputs (probes)
   size_t lpart;    // [H, punits, kMaxSplits, 256] f32 split-KV log2-sum-exps
+  size_t lse_s;    // [H, N] f32 log2-sum-exp of each row's kept logits (sparse pass, group-major)
+  size_t lse_d;    // [H, M + 1] f32 log2-sum-exp of each probe row over all keys (dense pass)
+  size_t diag;     // [H, M + 1, 4] f64 per-probe-row residual energies (diagnostics)
+  size_t dscr;     // diagnostics scratch: support union bits [H, Cq, ceil(Ckt/32)] u32 and
+                   // size sums [H, Cq] u64; or density weights [kDiagRows, N] f64 and counts [H]
   size_t total;
 
   int Nv, e, Cmax, nchunk, tiles_per_head, kmax;
@@ -202,6 +208,15 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->punits = static_cast<int>(M / 256 + 1);
   L->opart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * d * 4);
   L->lpart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * 4);
+  L->lse_s = take(H * N * 4);
+  L->lse_d = take(H * (M + 1) * 4);
+  L->diag = take(H * (M + 1) * 4 * 8);
+  {
+    const size_t words = (static_cast<size_t>(L->Ckt) + 31) / 32;
+    const size_t se = align256(H * Cq * words * 4) + H * Cq * 8;
+    const size_t dn = align256(static_cast<size_t>(kDiagRows) * N * 8) + H * 8;
+    L->dscr = take(se > dn ? se : dn);
+  }
   L->total = o;
 }
 
@@ -210,7 +225,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
 // name.
 inline bool named_region(const sparsepr_params& p, const Layout& L, const char* name, size_t* off,
                          size_t* bytes) {
-  const size_t H = p.H, d = p.d, e = p.n_eig, Ck = p.Ck, Cq = p.Cq, Nv = L.Nv;
+  const size_t H = p.H, d = p.d, e = p.n_eig, Ck = p.Ck, Cq = p.Cq, Nv = L.Nv, M = p.M;
   struct R {
     const char* n;
     size_t o, b;
@@ -220,7 +235,8 @@ inline bool named_region(const sparsepr_params& p, const Layout& L, const char* 
       {"evec", L.evec, H * d * e * 8},  {"wk", L.wk, H * d * e * 8},
       {"z", L.z, H * Nv * e * 8},       {"ck", L.ck, H * Ck * d * 8},
       {"g", L.g, H * d * d * 8},        {"bmat", L.bmat, H * d * d * 8},
-      {"bvec", L.bvec, H * d * 8},
+      {"bvec", L.bvec, H * d * 8},      {"xr", L.xr, H * 2 * M * d * 8},
+      {"vr", p.r <= 32 ? L.evec : L.gram, H * d * static_cast<size_t>(p.r) * 8},
   };
   for (const R& r : tab) {
     const char* a = r.n;

@@ -23,7 +23,8 @@ EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_part
             "sparsepr_permute", "sparsepr_route", "sparsepr_route_width",
             "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
             "sparsepr_reset_stats", "sparsepr_check_wait_limit", "sparsepr_route_noalloc",
-            "sparsepr_workspace_region")
+            "sparsepr_workspace_region", "sparsepr_probe_diagnostics",
+            "sparsepr_support_expansion", "sparsepr_density_profile")
 
 
 class Params(ctypes.Structure):
@@ -79,6 +80,14 @@ def _load():
     lib.sparsepr_workspace_region.argtypes = [PP, ctypes.c_char_p, ctypes.POINTER(sz),
                                               ctypes.POINTER(sz)]
     lib.sparsepr_workspace_region.restype = st
+    lib.sparsepr_probe_diagnostics.argtypes = [PP, I32P, P, P, P, V, sz, V]
+    lib.sparsepr_probe_diagnostics.restype = st
+    lib.sparsepr_support_expansion.argtypes = [P, P, st, PP, I32P, I32P, ctypes.c_double,
+                                               ctypes.c_int32, P, P, V, sz, V]
+    lib.sparsepr_support_expansion.restype = st
+    lib.sparsepr_density_profile.argtypes = [P, P, st, PP, ctypes.c_double, ctypes.c_int32, P, V,
+                                             sz, V]
+    lib.sparsepr_density_profile.restype = st
     lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
     lib.sparsepr_reset_stats.argtypes = [V, V]
     lib.sparsepr_check_wait_limit.argtypes = [V, V]
@@ -273,6 +282,47 @@ def sparsepr_probe_correct(qp, kp, vp, p, off_q, perm_q, o_sparse, pairs_sparse,
                                       None if fit is None else
                                       _arg(fit, "fit", (H, d * d + d), torch.float64),
                                       wp, wb, _stream(stream)), "sparsepr_probe_correct")
+
+
+def sparsepr_probe_diagnostics(p, probes, mass, error, energy, ws, stream=None):
+    """Retained mass and error of every probe row, and the residual energy
+    split per head (see include/sparsepr.h)."""
+    prm, keep = make_params(p)
+    H, M = int(p["H"]), int(p["M"])
+    f64 = torch.float64
+    _check(lib.sparsepr_probe_diagnostics(ctypes.byref(prm), _arg(probes, "probes", (H, M), I32),
+                                          _arg(mass, "mass", (H, M), f64),
+                                          _arg(error, "error", (H, M), f64),
+                                          _arg(energy, "energy", (H, 4), f64), *_ws(ws),
+                                          _stream(stream)), "sparsepr_probe_diagnostics")
+
+
+def sparsepr_support_expansion(qp, kp, p, off_q, off_k, tau, group_stride, individual,
+                               aggregate, ws, stream=None):
+    """Mean individual and aggregate (union) support size, in key groups, of
+    every group_stride-th video query group (see include/sparsepr.h)."""
+    prm, keep = make_params(p)
+    H, N, d, wq, wk = _dims(p)
+    Cq = int(p["Cq"])
+    (pq, pk), dt = _qkv(p, [("qp", qp), ("kp", kp)])
+    f64 = torch.float64
+    _check(lib.sparsepr_support_expansion(pq, pk, dt, ctypes.byref(prm),
+                                          _arg(off_q, "off_q", (H, wq), I32),
+                                          _arg(off_k, "off_k", (H, wk), I32), float(tau),
+                                          int(group_stride),
+                                          _arg(individual, "individual", (H, Cq), f64),
+                                          _arg(aggregate, "aggregate", (H, Cq), f64), *_ws(ws),
+                                          _stream(stream)), "sparsepr_support_expansion")
+
+
+def sparsepr_density_profile(q, k, p, tau, row_stride, density, ws, stream=None):
+    """Mean tau-mass density of every row_stride-th video row, per head."""
+    prm, keep = make_params(p)
+    H = int(p["H"])
+    (pq, pk), dt = _qkv(p, [("q", q), ("k", k)])
+    _check(lib.sparsepr_density_profile(pq, pk, dt, ctypes.byref(prm), float(tau), int(row_stride),
+                                        _arg(density, "density", (H,), torch.float64), *_ws(ws),
+                                        _stream(stream)), "sparsepr_density_profile")
 
 
 def sparsepr_reset_stats(ws, stream=None):

@@ -263,10 +263,69 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
  *   "mk", "eval" and "evec" for R^T R and its eigenpairs):
  *     "bmat"   [H, d, d] fp64, "bvec" [H, d] fp64: the ridge solution B, b
  *             before the subspace projection
+ *     "xr"     [H, 2, M, d] fp64: X = O_sparse of the probe rows, then
+ *             R = O_dense - X
+ *     "vr"     [H, d, r] fp64: the leading r right singular vectors of R (columns)
  * Errors: INVALID_ARG for invalid parameters, a NULL pointer or an unknown
  * name; UNSUPPORTED as sparsepr_workspace_bytes. Host only, enqueues nothing. */
 sparsepr_status sparsepr_workspace_region(const sparsepr_params* p, const char* name,
                                           size_t* offset, size_t* bytes);
+
+/* Structural diagnostics of the probe rows [SPR 3, structural analysis:
+ * retained attention mass does not bound the post-softmax error, and the
+ * partition's geometry decides how much of the residual is affine-
+ * explainable; SPR 4, ablations: orthogonal residual energy]. Call after
+ * sparsepr_probe_correct with the same parameters and `ws` (M > 0), before
+ * the workspace is reused; `probes` as written by that call.
+ *   mass    [H, M] fp64 out: dense softmax mass of probe row t on the keys its
+ *           query group keeps, sum over kept keys of softmax(scale q.k) over
+ *           all N keys (from the log-sum-exps of the sparse and dense passes)
+ *   error   [H, M] fp64 out: ||O_dense - O_sparse||_2 of probe row t
+ *   energy  [H, 4] fp64 out, over the probe rows with R = O_dense - O_sparse,
+ *           X = O_sparse, the fitted map F = b + X B and P_r = V_r V_r^T:
+ *           { ||R||_F^2, ||R P_r||^2 / ||R||^2 (explainable share),
+ *             ||R - F||^2 / ||R||^2, ||R - F P_r||^2 / ||R||^2 } (a zero R gives
+ *           {0, 1, 0, 0})
+ * Errors: INVALID_ARG for M = 0 or a NULL pointer; UNSUPPORTED for r > 64. */
+sparsepr_status sparsepr_probe_diagnostics(const sparsepr_params* p, const int32_t* probes,
+                                           double* mass, double* error, double* energy,
+                                           void* ws, size_t ws_bytes, void* stream);
+
+/* Support expansion of a shared route [SPR 3, structural analysis: the
+ * support that the rows of a query group need together is several times the
+ * support each needs alone]. For every group_stride-th video query group g
+ * of a permuted call (qp, kp, off_q, off_k as from sparsepr_permute): a row's
+ * individual support at mass tau is the smallest set of key groups (the text
+ * key group, when present, counts as one) whose dense softmax mass reaches
+ * tau (within 1e-15), taken by decreasing mass with ties to the lower index,
+ * from the row's scaled logits over all N keys in fp64; the group's
+ * aggregate support is the union of its rows' supports.
+ *   individual [H, Cq] fp64 out: mean individual support size of the group's
+ *              rows (0 for an empty group; NaN for a group not sampled)
+ *   aggregate  [H, Cq] fp64 out: size of the union (NaN when not sampled)
+ * Cost: 2 N d fp64 FMA per sampled row. Uses the diagnostics scratch of `ws`;
+ * call it after the attention call. Errors: INVALID_ARG for tau outside
+ * (0, 1], group_stride < 1, NULL or misaligned pointers; UNSUPPORTED when
+ * the key-group count does not fit one CTA's shared memory. */
+sparsepr_status sparsepr_support_expansion(const void* qp, const void* kp, sparsepr_dtype dt,
+                                           const sparsepr_params* p, const int32_t* off_q,
+                                           const int32_t* off_k, double tau, int32_t group_stride,
+                                           double* individual, double* aggregate, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/* Per-head attention density ["Attention Sparsity is Input-Stable", offline
+ * layer-wise sparsity profiling: the share of attention weights a head needs
+ * for a mass tau]. For every row_stride-th video row i of q (original token
+ * order): n_i = the smallest number of row i's N softmax weights over k,
+ * largest first, whose sum reaches tau (within 1e-15), from fp64 logits;
+ *   density [H] fp64 out: mean over the sampled rows of n_i / N
+ * (1 - density is the head's sparsity at tau; fitting it over calibration
+ * inputs is the caller's). Cost: N d fp64 FMA per sampled row. Uses the
+ * diagnostics scratch of `ws`. Errors as sparsepr_support_expansion. */
+sparsepr_status sparsepr_density_profile(const void* q, const void* k, sparsepr_dtype dt,
+                                         const sparsepr_params* p, double tau, int32_t row_stride,
+                                         double* density, void* ws, size_t ws_bytes,
+                                         void* stream);
 
 /* Copy the device statistics of the last call out of `ws` (a blocking
  * device-to-host copy; call after the stream has been synchronised). */
