@@ -46,6 +46,8 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->kmeans_iters < 1 || p->kmeans_iters > 1000) return SPARSEPR_ERR_INVALID_ARG;
   if (p->M < 0 || p->M > Nv) return SPARSEPR_ERR_INVALID_ARG;
   if (p->r < 1 || p->r > p->d) return SPARSEPR_ERR_INVALID_ARG;
+  if (p->partition < SPARSEPR_PARTITION_RESPONSE || p->partition > SPARSEPR_PARTITION_COCLUSTER)
+    return SPARSEPR_ERR_INVALID_ARG;
   if (!finite_nonneg(p->lambda) || !finite_nonneg(p->scale)) return SPARSEPR_ERR_INVALID_ARG;
   for (int h = 0; h < p->H; ++h)
     if (!(p->keep[h] > 0.0 && p->keep[h] <= 1.0)) return SPARSEPR_ERR_INVALID_ARG;
@@ -144,6 +146,183 @@ AssignTC assign_common(const Ctx& c, void* ws, int32_t* labels, int32_t* flags, 
   a.stats = c.stats;
   a.sm_count = sms;
   return a;
+}
+
+// Nearest-centroid pass in the d-space form argmin_j (cy_j - 2 x . y_j) of
+// the video rows x of X [H, N, d] (bf16 or fp32, exact) against the centroid
+// side y [H, m, d], cy [H, m] (fp64): on the tensor cores (one exact bf16
+// plane of x, two or three planes of y, certified, fp64 recheck) when the
+// centroid planes fit in shared memory, else in fp64 on the CUDA cores.
+// G: the metric of the true distance x^T G x + cy_j - 2 x . y_j, used only to
+// count near ties; the alternative partitions pass null and count none.
+struct DPass {
+  int nb = 0;  // centroid planes on the tensor cores; 0: fp64 path
+  AssignTC a = {};
+  const void* X = nullptr;
+  int m = 0, Cpad = 0, flag_base = 0;
+  int32_t* labels = nullptr;
+  const double* G = nullptr;
+};
+
+cudaError_t dpass_setup(const Ctx& c, void* ws, const void* X, int m, int Cpad, int32_t* labels,
+                        int flag_base, float* xnorm, const double* cy, const double* G, int sms,
+                        DPass* P) {
+  const int H = c.p.H, N = c.p.N, d = c.p.d, Nv = c.L.Nv;
+  const long long hs_in = static_cast<long long>(N) * d;
+  P->X = X;
+  P->m = m;
+  P->Cpad = Cpad;
+  P->flag_base = flag_base;
+  P->labels = labels;
+  P->G = G;
+  P->nb = 0;
+  // (a 128-row TMA box needs at least 128 rows in the tensor)
+  if (c.bf16 && static_cast<size_t>(H) * N >= static_cast<size_t>(kTileM)) {
+    if (assign_tc_smem_bytes(1, 3, d, Cpad) <= kMaxDynSmem)
+      P->nb = 3;
+    else if (assign_tc_smem_bytes(1, 2, d, Cpad) <= kMaxDynSmem)
+      P->nb = 2;
+  }
+  if (!P->nb) return cudaSuccess;
+  const cudaError_t e = launch_split_rows(X, c.kind, hs_in, d, Nv, d, d, 0, H, nullptr, 0, xnorm,
+                                          c.st);
+  if (e != cudaSuccess) return e;
+  AssignTC& a = P->a;
+  a = assign_common(c, ws, labels, at<int32_t>(ws, c.L.flags), flag_base, sms);
+  a.a_planes = static_cast<const __nv_bfloat16*>(X);
+  a.a_plane_stride = 0;
+  a.a_rows_total = static_cast<size_t>(H) * N;
+  a.a_head = N;
+  a.nA = 1;
+  a.b_planes = at<__nv_bfloat16>(ws, c.L.wplanes);
+  a.b_plane_stride = static_cast<long long>(H) * Cpad * d;
+  a.nB = P->nb;
+  a.Dp = d;
+  a.Cpad = Cpad;
+  a.npairs = P->nb;
+  for (int i = 0; i < 6; ++i) a.pairs[i] = (i < P->nb) ? i : 0;
+  a.cvals = at<float>(ws, c.L.cfq);
+  a.xnorm = xnorm;
+  a.hmax = at<float>(ws, c.L.hmq);
+  a.x_exact = X;
+  a.x_kind = c.kind;
+  a.x_hs = hs_in;
+  a.x_ld = d;
+  a.D = d;
+  a.y_tr = at<double>(ws, c.L.ytr);
+  a.c_exact = cy;
+  a.m = m;
+  a.direct = 0;
+  a.metric = G;
+  return cudaSuccess;
+}
+
+cudaError_t dpass_run(const Ctx& c, void* ws, const DPass& P, const double* y, const double* cy) {
+  const int H = c.p.H, N = c.p.N, d = c.p.d, Nv = c.L.Nv;
+  int32_t* flags = at<int32_t>(ws, c.L.flags);
+  if (P.nb) {
+    const cudaError_t e = launch_prep_centroids(
+        y, cy, P.m, d, d, P.Cpad, P.nb, H, at<__nv_bfloat16>(ws, c.L.wplanes),
+        static_cast<long long>(H) * P.Cpad * d, at<float>(ws, c.L.cfq), at<float>(ws, c.L.hmq),
+        at<double>(ws, c.L.ytr), flags, P.flag_base, c.st);
+    if (e != cudaSuccess) return e;
+    return launch_argmin_tc(P.a, c.st);
+  }
+  return launch_argmin(P.X, c.kind, static_cast<long long>(N) * d, d, Nv, d, y, cy, P.m, H,
+                       P.labels, flags, P.flag_base, P.G, P.G ? c.stats : nullptr, c.st);
+}
+
+// The alternative partitions ([SPR 4] ablations' semantic k-means; the
+// co-clustering page's bidirectional rounds), both on the d-space pass.
+// Initial rows, pass cap, ties and empty groups as in the method's partition.
+sparsepr_status partition_alternative(const Ctx& c, const void* q, const void* k,
+                                      int32_t* label_q, int32_t* label_k, void* ws) {
+  const Layout& L = c.L;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, Nv = L.Nv, Ck = c.p.Ck, Cq = c.p.Cq;
+  const int iters = c.p.kmeans_iters;
+  const long long hs_in = static_cast<long long>(N) * d;
+  cudaStream_t st = c.st;
+  int32_t* flags = at<int32_t>(ws, L.flags);
+  int32_t* init_k = at<int32_t>(ws, L.init_k);
+  int32_t* init_q = at<int32_t>(ws, L.init_q);
+  int32_t* lab_k = at<int32_t>(ws, L.lab_k);
+  int32_t* lab_q = at<int32_t>(ws, L.lab_q);
+  int32_t* hist = at<int32_t>(ws, L.hist);
+  int32_t* sperm = at<int32_t>(ws, L.sortperm);
+  int32_t* soff = at<int32_t>(ws, L.sortoff);
+  int32_t* cnt_k = at<int32_t>(ws, L.cnt);
+  int32_t* cnt_q = cnt_k + static_cast<size_t>(H) * Ck;
+  double* ck = at<double>(ws, L.ck);    // key centres [H, Ck, d]
+  double* qbar = at<double>(ws, L.qbar);  // query centres [H, Cq, d]
+  double* G = at<double>(ws, L.g);
+  double* wg = at<double>(ws, L.wg);    // centroid side y [H, max(Ck, Cq), d]
+  double* cg = at<double>(ws, L.cg);    // offsets cy [H, max(Ck, Cq)]
+  const int sms = sm_count();
+  SPR_TRY(launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, st));
+  SPR_TRY(launch_gather_init(k, c.kind, hs_in, d, d, init_k, Ck, H, ck, nullptr, st));
+  SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
+  DPass pk, pq;
+  SPR_TRY(dpass_setup(c, ws, k, Ck, L.CpadK, lab_k, 0, at<float>(ws, L.xnk), cg, nullptr, sms, &pk));
+  SPR_TRY(dpass_setup(c, ws, q, Cq, L.CpadQ, lab_q, 2, at<float>(ws, L.xnq), cg, nullptr, sms, &pq));
+  if (c.p.partition == SPARSEPR_PARTITION_SEMANTIC) {
+    // plain Euclidean Lloyd on each side: the d-space form with G = I
+    // (y = centre, cy = |centre|^2)
+    SPR_TRY(launch_identity(G, H, d, st));
+    for (int side = 0; side < 2; ++side) {
+      const void* X = side ? q : k;
+      double* cen = side ? qbar : ck;
+      const int m = side ? Cq : Ck;
+      const int fb = side ? 2 : 0;
+      int32_t* lab = side ? lab_q : lab_k;
+      const DPass& P = side ? pq : pk;
+      for (int t = 0; t < iters; ++t) {
+        SPR_TRY(launch_query_metric_apply(G, cen, m, H, d, wg, cg, flags + fb + 1, 4, st));
+        SPR_TRY(dpass_run(c, ws, P, wg, cg));
+        SPR_TRY(launch_finalize_pass(H, t, flags, fb,
+                                     side ? c.stats->query_passes : c.stats->key_passes, st));
+        if (t + 1 < iters) {
+          SPR_TRY(launch_counting_sort(lab, H, Nv, m, L.nchunk, hist, sperm, soff, flags + fb + 1,
+                                       4, nullptr, st));
+          SPR_TRY(launch_group_mean(X, c.kind, hs_in, d, d, sperm, Nv, soff, m + 1, m, H, true,
+                                    cen, nullptr, flags + fb + 1, 4, st));
+        }
+      }
+    }
+  } else {
+    // co-clustering rounds: keys against the query centres' affinity space,
+    // then queries against the new key centres'
+    if (static_cast<size_t>(8) * (Ck > Cq ? Ck : Cq) * 8 > kMaxDynSmem) return SPARSEPR_ERR_UNSUPPORTED;
+    double* pkbar = at<double>(ws, L.pkbar);
+    double* pqbar = at<double>(ws, L.pqbar);
+    for (int t = 0; t < iters; ++t) {
+      // key blocks: mean affinity vectors (from the seed keys in the first
+      // round, then from the blocks' mean keys; an empty block keeps its
+      // vector), their d-space form, the assignment
+      SPR_TRY(launch_affinity_centres(ck, qbar, Ck, Cq, d, H, c.scale, cnt_k, t == 0, pkbar, st));
+      SPR_TRY(launch_dspace_centres(pkbar, qbar, Ck, Cq, d, H, c.scale, wg, cg, st));
+      SPR_TRY(dpass_run(c, ws, pk, wg, cg));
+      // key centres: the blocks' mean keys (zero for an empty block)
+      SPR_TRY(launch_counting_sort(lab_k, H, Nv, Ck, L.nchunk, hist, sperm, soff, flags + 1, 4,
+                                   nullptr, st));
+      SPR_TRY(launch_group_mean(k, c.kind, hs_in, d, d, sperm, Nv, soff, Ck + 1, Ck, H, false, ck,
+                                nullptr, flags + 1, 4, st));
+      SPR_TRY(launch_group_counts(soff, Ck + 1, Ck, H, cnt_k, st));
+      // query blocks against the new key centres
+      SPR_TRY(launch_affinity_centres(qbar, ck, Cq, Ck, d, H, c.scale, cnt_q, t == 0, pqbar, st));
+      SPR_TRY(launch_dspace_centres(pqbar, ck, Cq, Ck, d, H, c.scale, wg, cg, st));
+      SPR_TRY(dpass_run(c, ws, pq, wg, cg));
+      // query centres: the blocks' mean queries (an empty block keeps its centre)
+      SPR_TRY(launch_counting_sort(lab_q, H, Nv, Cq, L.nchunk, hist, sperm, soff, flags + 3, 4,
+                                   nullptr, st));
+      SPR_TRY(launch_group_mean(q, c.kind, hs_in, d, d, sperm, Nv, soff, Cq + 1, Cq, H, true, qbar,
+                                nullptr, flags + 3, 4, st));
+      SPR_TRY(launch_group_counts(soff, Cq + 1, Cq, H, cnt_q, st));
+      SPR_TRY(launch_finalize_round(H, t, flags, c.stats->key_passes, c.stats->query_passes, st));
+    }
+  }
+  SPR_TRY(launch_write_labels(lab_q, H, N, Nv, Cq, label_q, st));
+  SPR_TRY(launch_write_labels(lab_k, H, N, Nv, Ck, label_k, st));
+  return SPARSEPR_OK;
 }
 
 // Dense-mode routing metadata per head: one query group [0, M), one key
@@ -272,6 +451,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   double* wg = at<double>(ws, L.wg);
   double* cg = at<double>(ws, L.cg);
   const long long hs_in = static_cast<long long>(N) * d;
+  if (c.p.partition != SPARSEPR_PARTITION_RESPONSE)
+    return partition_alternative(c, q, k, label_q, label_k, ws);
 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
   {
@@ -362,56 +543,11 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   // queries: Lloyd passes on logit profiles in the d-space form
   SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
   // queries on the tensor cores for bf16 inputs (exact in one bf16 plane)
-  int nbq = 0;
-  if (c.bf16 && static_cast<size_t>(H) * N >= static_cast<size_t>(kTileM)) {
-    if (assign_tc_smem_bytes(1, 3, d, L.CpadQ) <= kMaxDynSmem)
-      nbq = 3;
-    else if (assign_tc_smem_bytes(1, 2, d, L.CpadQ) <= kMaxDynSmem)
-      nbq = 2;
-  }
-  AssignTC aq;
-  if (nbq) {
-    SPR_TRY(launch_split_rows(q, c.kind, hs_in, d, Nv, d, d, 0, H, nullptr, 0,
-                              at<float>(ws, L.xnq), st));
-    aq = assign_common(c, ws, lab_q, flags, 2, sms);
-    aq.a_planes = static_cast<const __nv_bfloat16*>(q);
-    aq.a_plane_stride = 0;
-    aq.a_rows_total = static_cast<size_t>(H) * N;
-    aq.a_head = N;
-    aq.nA = 1;
-    aq.b_planes = at<__nv_bfloat16>(ws, L.wplanes);
-    aq.b_plane_stride = static_cast<long long>(H) * L.CpadQ * d;
-    aq.nB = nbq;
-    aq.Dp = d;
-    aq.Cpad = L.CpadQ;
-    aq.npairs = nbq;
-    for (int i = 0; i < 6; ++i) aq.pairs[i] = (i < nbq) ? i : 0;
-    aq.cvals = at<float>(ws, L.cfq);
-    aq.xnorm = at<float>(ws, L.xnq);
-    aq.hmax = at<float>(ws, L.hmq);
-    aq.x_exact = q;
-    aq.x_kind = c.kind;
-    aq.x_hs = hs_in;
-    aq.x_ld = d;
-    aq.D = d;
-    aq.y_tr = at<double>(ws, L.ytr);
-    aq.c_exact = cg;
-    aq.m = Cq;
-    aq.direct = 0;
-    aq.metric = G;
-  }
+  DPass pq;
+  SPR_TRY(dpass_setup(c, ws, q, Cq, L.CpadQ, lab_q, 2, at<float>(ws, L.xnq), cg, G, sms, &pq));
   for (int t = 0; t < iters; ++t) {
     SPR_TRY(launch_query_metric_apply(G, qbar, Cq, H, d, wg, cg, flags + 3, 4, st));
-    if (nbq) {
-      SPR_TRY(launch_prep_centroids(wg, cg, Cq, d, d, L.CpadQ, nbq, H,
-                                    at<__nv_bfloat16>(ws, L.wplanes),
-                                    static_cast<long long>(H) * L.CpadQ * d, at<float>(ws, L.cfq),
-                                    at<float>(ws, L.hmq), at<double>(ws, L.ytr), flags, 2, st));
-      SPR_TRY(launch_argmin_tc(aq, st));
-    } else {
-      SPR_TRY(launch_argmin(q, c.kind, hs_in, d, Nv, d, wg, cg, Cq, H, lab_q, flags, 2, G, c.stats,
-                            st));
-    }
+    SPR_TRY(dpass_run(c, ws, pq, wg, cg));
     SPR_TRY(launch_finalize_pass(H, t, flags, 2, c.stats->query_passes, st));
     if (t + 1 < iters) {
       SPR_TRY(launch_counting_sort(lab_q, H, Nv, Cq, L.nchunk, hist, sperm, soff, flags + 3, 4,

@@ -65,6 +65,16 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long head_stride_x
 cudaError_t launch_query_metric_apply(const double* G, const double* qbar, int Cq, int H, int d,
                                       double* wg, double* cg, const int32_t* skip,
                                       int skip_stride, cudaStream_t st);
+cudaError_t launch_identity(double* G, int H, int d, cudaStream_t st);
+cudaError_t launch_group_counts(const int32_t* off, int off_stride, int C, int H, int32_t* cnt,
+                                cudaStream_t st);
+cudaError_t launch_affinity_centres(const double* xbar, const double* C, int m1, int m2, int d,
+                                    int H, double scale, const int32_t* cnt, bool first,
+                                    double* pbar, cudaStream_t st);
+cudaError_t launch_dspace_centres(const double* pbar, const double* C, int m1, int m2, int d,
+                                  int H, double scale, double* y, double* c, cudaStream_t st);
+cudaError_t launch_finalize_round(int H, int round, int32_t* flags, int32_t* passes_k,
+                                  int32_t* passes_q, cudaStream_t st);
 cudaError_t launch_write_labels(const int32_t* lab, int H, int N, int Nv, int C_text,
                                 int32_t* out, cudaStream_t st);
 

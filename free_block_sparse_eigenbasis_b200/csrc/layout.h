@@ -90,6 +90,9 @@ struct Layout {
   size_t lse_s;    // [H, N] f32 log2-sum-exp of each row's kept logits (sparse pass, group-major)
   size_t lse_d;    // [H, M + 1] f32 log2-sum-exp of each probe row over all keys (dense pass)
   size_t diag;     // [H, M + 1, 4] f64 per-probe-row residual energies (diagnostics)
+  size_t pkbar;    // co-clustering: [H, Ck, Cq] f64 mean affinity vector of each key block
+  size_t pqbar;    // co-clustering: [H, Cq, Ck] f64 mean affinity vector of each query block
+  size_t cnt;      // [H, Ck + Cq] int32 members per key / query block (alternative partitions)
   size_t dscr;     // diagnostics scratch: support union bits [H, Cq, ceil(Ckt/32)] u32 and
                    // size sums [H, Cq] u64; or density weights [kDiagRows, N] f64 and counts [H]
   size_t total;
@@ -160,23 +163,32 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->ck = take(H * Ck * d * 8);
   L->g = take(H * d * d * 8);
   L->qbar = take(H * Cq * d * 8);
-  L->wg = take(H * Cq * d * 8);
-  L->cg = take(H * Cq * 8);
   L->Dpk = (p.n_eig <= 16) ? 16 : 64;
   L->CpadK = (p.Ck + 15) / 16 * 16;
   L->CpadQ = (p.Cq + 15) / 16 * 16;
+  // the alternative partitions run the d-space assignment on both sides:
+  // its centroid-side regions hold max(Ck, Cq) rows
+  const bool alt = p.partition != 0;
+  const size_t Cm = alt ? (Ck > Cq ? Ck : Cq) : Cq;
+  const size_t Cpm = alt ? (L->CpadK > L->CpadQ ? L->CpadK : L->CpadQ) : L->CpadQ;
+  L->wg = take(H * Cm * d * 8);
+  L->cg = take(H * Cm * 8);
   L->zplanes = take(3 * H * Nv * static_cast<size_t>(L->Dpk) * 2);
   L->xnk = take(H * Nv * 4);
   L->xnq = take(H * Nv * 4);
   L->muplanes = take(3 * H * static_cast<size_t>(L->CpadK) * L->Dpk * 2);
   L->cfk = take(H * static_cast<size_t>(L->CpadK) * 4);
   L->hmk = take(H * 8);
-  L->wplanes = take(3 * H * static_cast<size_t>(L->CpadQ) * d * 2);
-  L->cfq = take(H * static_cast<size_t>(L->CpadQ) * 4);
+  L->wplanes = take(3 * H * Cpm * d * 2);
+  L->cfq = take(H * Cpm * 4);
   L->hmq = take(H * 8);
   L->recheck = take(H * Nv * 4);
   L->nrecheck = take(H * 4);
-  L->ytr = take(H * (Ck * e > Cq * d ? Ck * e : Cq * d) * 8);
+  {
+    size_t yt = Ck * e > Cq * d ? Ck * e : Cq * d;
+    if (alt && Cm * d > yt) yt = Cm * d;
+    L->ytr = take(H * yt * 8);
+  }
   L->cq = take(H * Cq * d * 8);
   L->ckr = take(H * Ck * d * 8);
   {
@@ -211,6 +223,10 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->lse_s = take(H * N * 4);
   L->lse_d = take(H * (M + 1) * 4);
   L->diag = take(H * (M + 1) * 4 * 8);
+  const bool cocl = p.partition == 2;
+  L->pkbar = take(cocl ? H * Ck * Cq * 8 : 0);
+  L->pqbar = take(cocl ? H * Cq * Ck * 8 : 0);
+  L->cnt = take(alt ? H * (Ck + Cq) * 4 : 0);
   {
     const size_t words = (static_cast<size_t>(L->Ckt) + 31) / 32;
     const size_t se = align256(H * Cq * words * 4) + H * Cq * 8;

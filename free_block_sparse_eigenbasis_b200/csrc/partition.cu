@@ -302,7 +302,8 @@ __global__ void gather_init_kernel(const void* src, int kind, long long hs, int 
 // The value c_j - 2 x.y_j is the squared distance minus x^T G x, with G = I
 // (keys: y = mu, c = |mu|^2) or the query metric G (queries: y = G qbar,
 // c = qbar^T G qbar); near ties (see kNearTieRel) are counted from the two
-// smallest values plus x^T G x. For G != I the quadratic form is only
+// smallest values plus x^T G x (a null stats pointer counts none). For
+// G != I the quadratic form is only
 // formed for candidate rows, whose gap lies within 1e-11 of
 // |second value| + trace(G) |x|^2 (an upper bound of the second distance,
 // G being positive semidefinite).
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(256) argmin_kernel(const void* X, int kind, lo
       }
     }
     if (changed) atomicAdd(&fl[flag_base + 0], changed);
-    if (ties)
+    if (ties && stats)
       atomicAdd(reinterpret_cast<unsigned long long*>(&stats->near_ties[flag_base >> 1]),
                 static_cast<unsigned long long>(ties));
   }
@@ -744,6 +745,128 @@ __global__ void __launch_bounds__(128)
   if (a < ng) cg[static_cast<size_t>(h) * Cq + g0 + a] = (red[a][0] + red[a][1]) + (red[a][2] + red[a][3]);
 }
 
+// ---------------------------------------------------------------------------
+// Alternative partitions (the ablations' semantic k-means, the co-clustering
+// page's bidirectional rounds): helpers around the d-space assignment.
+// ---------------------------------------------------------------------------
+// G = I (semantic k-means is the d-space form with the identity metric)
+__global__ void identity_kernel(double* G, int d) {
+  const int h = blockIdx.y;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < d * d; t += gridDim.x * blockDim.x)
+    G[static_cast<size_t>(h) * d * d + t] = (t / d == t % d) ? 1.0 : 0.0;
+}
+
+// members per group from the counting sort's offsets
+__global__ void group_counts_kernel(const int32_t* off, int off_stride, int C, int H,
+                                    int32_t* cnt) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= H * C) return;
+  const int h = i / C, c = i % C;
+  cnt[i] = off[static_cast<size_t>(h) * off_stride + c + 1] - off[static_cast<size_t>(h) * off_stride + c];
+}
+
+// Mean affinity vectors of the blocks: pbar[j] = scale * C xbar_j (C: [m2, d]
+// centres of the other side), for blocks j whose mean xbar_j is current:
+// every block in the first round, afterwards the blocks with members (an
+// empty block keeps its vector). One warp per (8 blocks, centre g): lanes
+// over d, then shuffles.
+constexpr int kAcRows = 8;
+
+__global__ void __launch_bounds__(256)
+    affinity_centres_kernel(const double* xbar, const double* C, int m1, int m2, int d,
+                            double scale, const int32_t* cnt, int first, double* pbar) {
+  __shared__ double xs[kAcRows][128];
+  const int h = blockIdx.y, j0 = blockIdx.x * kAcRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kAcRows * 128; i += blockDim.x) {
+    const int r = i >> 7, a = i & 127;
+    xs[r][a] = (j0 + r < m1 && a < d) ? xbar[(static_cast<size_t>(h) * m1 + j0 + r) * d + a] : 0.0;
+  }
+  __syncthreads();
+  bool upd[kAcRows];
+#pragma unroll
+  for (int r = 0; r < kAcRows; ++r)
+    upd[r] = j0 + r < m1 && (first || cnt[static_cast<size_t>(h) * m1 + j0 + r] > 0);
+  const double* Ch = C + static_cast<size_t>(h) * m2 * d;
+  for (int g = warp; g < m2; g += blockDim.x / 32) {
+    double acc[kAcRows];
+#pragma unroll
+    for (int r = 0; r < kAcRows; ++r) acc[r] = 0.0;
+    for (int a = lane; a < d; a += 32) {
+      const double cv = Ch[static_cast<size_t>(g) * d + a];
+#pragma unroll
+      for (int r = 0; r < kAcRows; ++r) acc[r] = fma(xs[r][a], cv, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < kAcRows; ++r) {
+      const double v = warp_sum_f64(acc[r]);
+      if (lane == 0 && upd[r]) pbar[(static_cast<size_t>(h) * m1 + j0 + r) * m2 + g] = scale * v;
+    }
+  }
+}
+
+// The d-space form of the affinity distance: for pbar_j (in the space of the
+// other side's m2 centres C), |scale C x - pbar_j|^2 = x^T G x + c_j - 2 x . y_j
+// with y_j = scale C^T pbar_j and c_j = |pbar_j|^2 (G = scale^2 C^T C is the
+// same for every j, so it does not change the nearest block). Thread a
+// forms y_j[a]; eight blocks per CTA.
+__global__ void __launch_bounds__(128)
+    dspace_centres_kernel(const double* pbar, const double* C, int m1, int m2, int d,
+                          double scale, double* y, double* c) {
+  extern __shared__ double ps[];  // [kAcRows][m2]
+  __shared__ double red[kAcRows][4];
+  const int h = blockIdx.y, j0 = blockIdx.x * kAcRows, a = threadIdx.x;
+  const int lane = a & 31, wp = a >> 5;
+  for (int i = a; i < kAcRows * m2; i += blockDim.x) {
+    const int r = i / m2, g = i % m2;
+    ps[i] = (j0 + r < m1) ? pbar[(static_cast<size_t>(h) * m1 + j0 + r) * m2 + g] : 0.0;
+  }
+  __syncthreads();
+  const double* Ch = C + static_cast<size_t>(h) * m2 * d;
+  double acc[kAcRows];
+#pragma unroll
+  for (int r = 0; r < kAcRows; ++r) acc[r] = 0.0;
+  if (a < d)
+    for (int g = 0; g < m2; ++g) {
+      const double cv = Ch[static_cast<size_t>(g) * d + a];
+#pragma unroll
+      for (int r = 0; r < kAcRows; ++r) acc[r] = fma(ps[r * m2 + g], cv, acc[r]);
+    }
+#pragma unroll
+  for (int r = 0; r < kAcRows; ++r)
+    if (a < d && j0 + r < m1) y[(static_cast<size_t>(h) * m1 + j0 + r) * d + a] = scale * acc[r];
+  // c_j = |pbar_j|^2, fixed order: thread a sums g = a, a + 128, ...; then warps
+#pragma unroll
+  for (int r = 0; r < kAcRows; ++r) {
+    double v = 0.0;
+    for (int g = a; g < m2; g += blockDim.x) v = fma(ps[r * m2 + g], ps[r * m2 + g], v);
+    v = warp_sum_f64(v);
+    if (lane == 0) red[r][wp] = v;
+  }
+  __syncthreads();
+  if (a < kAcRows && j0 + a < m1)
+    c[static_cast<size_t>(h) * m1 + j0 + a] = (red[a][0] + red[a][1]) + (red[a][2] + red[a][3]);
+}
+
+// One co-clustering round ends when both sides' passes are counted: a round
+// after the first in which neither keys nor queries changed label ends the
+// head's rounds (both sides' done flags).
+__global__ void finalize_round_kernel(int H, int round, int32_t* flags, int32_t* passes_k,
+                                      int32_t* passes_q) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  int32_t* fl = flags + h * 4;
+  if (fl[1]) return;
+  passes_k[h] = round + 1;
+  passes_q[h] = round + 1;
+  if (round > 0 && fl[0] == 0 && fl[2] == 0) {
+    fl[1] = 1;
+    fl[3] = 1;
+  }
+  fl[0] = 0;
+  fl[2] = 0;
+}
+
 __global__ void write_labels_kernel(const int32_t* lab, int H, int N, int Nv, int C_text,
                                     int32_t* out) {
   const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -898,6 +1021,45 @@ cudaError_t launch_query_metric_apply(const double* G, const double* qbar, int C
                                       int skip_stride, cudaStream_t st) {
   query_metric_apply_kernel<<<dim3((Cq + kQmaG - 1) / kQmaG, H), 128, 0, st>>>(
       G, qbar, Cq, d, wg, cg, skip, skip_stride);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_identity(double* G, int H, int d, cudaStream_t st) {
+  identity_kernel<<<dim3((d * d + 255) / 256, H), 256, 0, st>>>(G, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_counts(const int32_t* off, int off_stride, int C, int H, int32_t* cnt,
+                                cudaStream_t st) {
+  group_counts_kernel<<<(H * C + 255) / 256, 256, 0, st>>>(off, off_stride, C, H, cnt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_affinity_centres(const double* xbar, const double* C, int m1, int m2, int d,
+                                    int H, double scale, const int32_t* cnt, bool first,
+                                    double* pbar, cudaStream_t st) {
+  if (d > 128) return cudaErrorInvalidValue;
+  affinity_centres_kernel<<<dim3((m1 + kAcRows - 1) / kAcRows, H), 256, 0, st>>>(
+      xbar, C, m1, m2, d, scale, cnt, first ? 1 : 0, pbar);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dspace_centres(const double* pbar, const double* C, int m1, int m2, int d,
+                                  int H, double scale, double* y, double* c, cudaStream_t st) {
+  const size_t shb = static_cast<size_t>(kAcRows) * m2 * 8;
+  if (d > 128 || shb > kMaxDynSmem) return cudaErrorInvalidValue;
+  const cudaError_t e = cudaFuncSetAttribute(dspace_centres_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(shb));
+  if (e != cudaSuccess) return e;
+  dspace_centres_kernel<<<dim3((m1 + kAcRows - 1) / kAcRows, H), 128, shb, st>>>(pbar, C, m1, m2,
+                                                                                  d, scale, y, c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_round(int H, int round, int32_t* flags, int32_t* passes_k,
+                                  int32_t* passes_q, cudaStream_t st) {
+  finalize_round_kernel<<<(H + 127) / 128, 128, 0, st>>>(H, round, flags, passes_k, passes_q);
   return cudaGetLastError();
 }
 

@@ -18,6 +18,8 @@ MAX_HEADS = 256
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_NUMERIC = range(7)
 BF16, F32 = 0, 1
+# sparsepr_params.partition; the parameter dicts name the mode as the oracle does
+PARTITION_MODES = dict(response=0, semantic=1, coclustering=2)
 
 EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_partition",
             "sparsepr_permute", "sparsepr_route", "sparsepr_route_width",
@@ -32,7 +34,7 @@ class Params(ctypes.Structure):
                 ("n_text", ctypes.c_int32), ("Ck", ctypes.c_int32), ("Cq", ctypes.c_int32),
                 ("Ms", ctypes.c_int32), ("n_eig", ctypes.c_int32),
                 ("kmeans_iters", ctypes.c_int32), ("M", ctypes.c_int32), ("r", ctypes.c_int32),
-                ("pad0", ctypes.c_int32), ("lam", ctypes.c_double), ("scale", ctypes.c_double),
+                ("partition", ctypes.c_int32), ("lam", ctypes.c_double), ("scale", ctypes.c_double),
                 ("seed", ctypes.c_uint64), ("keep", ctypes.POINTER(ctypes.c_double))]
 
 
@@ -115,7 +117,8 @@ def make_params(p: dict):
     arr = (ctypes.c_double * max(1, H))(*[float(x) for x in keep[:H]])
     prm = Params(H=H, N=int(p["N"]), d=int(p["d"]), n_text=int(p.get("n_text", 0)),
                  Ck=int(p["Ck"]), Cq=int(p["Cq"]), Ms=int(p["Ms"]), n_eig=int(p["n_eig"]),
-                 kmeans_iters=int(p["kmeans_iters"]), M=int(p["M"]), r=int(p["r"]), pad0=0,
+                 kmeans_iters=int(p["kmeans_iters"]), M=int(p["M"]), r=int(p["r"]),
+                 partition=PARTITION_MODES[p.get("partition", "response")],
                  lam=float(p["lam"]), scale=float(p.get("scale", 0.0)),
                  seed=int(p["seed"]) & ((1 << 64) - 1),
                  keep=ctypes.cast(arr, ctypes.POINTER(ctypes.c_double)))

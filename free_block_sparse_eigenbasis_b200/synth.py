@@ -60,6 +60,7 @@ class Workload:
     lam: float
     scale: float  # 0 -> 1/sqrt(d)
     seed: int
+    partition: str = "response"  # "response" | "semantic" | "coclustering"
 
     @property
     def Nv(self) -> int:
@@ -76,7 +77,12 @@ class Workload:
                     Ck=self.Ck, Cq=self.Cq, Ms=self.Ms, n_eig=self.n_eig,
                     kmeans_iters=self.kmeans_iters, keep=list(self.keep),
                     M=self.M, r=self.r, lam=self.lam, scale=self.scale,
-                    seed=self.seed)
+                    seed=self.seed, partition=self.partition)
+
+    def with_params(self, **kw) -> "Workload":
+        """A copy with some fields replaced (same inputs unless a generator
+        field changes)."""
+        return dataclasses.replace(self, **kw)
 
 
 def _keep_uniform(seed: int, H: int, lo: float, hi: float) -> tuple:

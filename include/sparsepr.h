@@ -70,6 +70,26 @@ typedef enum {
 
 typedef enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 } sparsepr_dtype;
 
+/* Partition computed by sparsepr_partition (sparsepr_params.partition).
+ *   RESPONSE  [SPR 2.A]: keys by k-means on their response coordinates in
+ *             the eigenbasis of M_K, then queries by k-means on their logit
+ *             profiles against the K/V group means (the method).
+ *   SEMANTIC  [SPR 4, ablations: the comparison partition]: keys and queries
+ *             each by plain Euclidean k-means on their own rows, no coupling.
+ *   COCLUSTER ["Attention Sparsity is Input-Stable", online bidirectional
+ *             QK co-clustering]: rounds that assign each key to the key block
+ *             whose mean affinity vector (scale * k . query centres) is
+ *             nearest, update the key centres, then do the same for the
+ *             queries against the new key centres.
+ * All three use the same initial rows (partial Fisher-Yates draws), pass cap
+ * (kmeans_iters), lowest-index ties and empty-group rule (the group keeps its
+ * centre). */
+typedef enum {
+  SPARSEPR_PARTITION_RESPONSE = 0,
+  SPARSEPR_PARTITION_SEMANTIC = 1,
+  SPARSEPR_PARTITION_COCLUSTER = 2
+} sparsepr_partition_mode;
+
 /* Method parameters, passed by const pointer; the callee copies what it
  * needs before returning. */
 typedef struct {
@@ -84,7 +104,8 @@ typedef struct {
   int32_t kmeans_iters; /* cap on k-means assignment passes (stops early when labels repeat) */
   int32_t M;            /* probe rows per head, 0..Nv */
   int32_t r;            /* rank of the residual subspace, 1..d */
-  int32_t pad0;
+  int32_t partition;    /* SPARSEPR_PARTITION_*: 0 (the default) is the method's
+                           response-coupled partition */
   double lambda;        /* ridge penalty, >= 0 */
   double scale;         /* softmax scale; 0 selects 1/sqrt(d) */
   uint64_t seed;        /* k-means initialisation seed */
