@@ -16,7 +16,13 @@ no collective on the data path) and the job value is the sum of the ranks'
 executed pairs over the slowest rank's time.
 
 Prints one JSON line. `value` is executed-pair TFLOPS of the whole call,
-4 d P_exec / t_call (P_exec = routed pairs + M N probe pairs).
+4 d P_exec / t_call (P_exec = routed pairs + M N probe pairs). Further fields
+(skipped with --no-extras): `configs` (the same call on the layer at
+executed-pair density 0.25, the 480p layer, the 40-head 14B-shaped layer in
+one call and the HunyuanVideo-shaped layer with text tokens), `diagnostics`
+(retained mass, residual energy split, support expansion, density profile)
+and `ablations` (semantic and co-clustering partitions, hard drop, M, r and
+lambda, each with its output error against dense attention).
 """
 from __future__ import annotations
 
@@ -271,6 +277,186 @@ def cpu_baseline_sample(w):
                 sample=oracle_sample_desc(w, t_call))
 
 
+# ---------------------------------------------------------------------------
+# Further workloads, diagnostics and ablations (fields of the same JSON line)
+# ---------------------------------------------------------------------------
+
+def time_calls(S, p, b, qd, kd, vd, stream, steps):
+    """Direct launches of the five calls with events between the stages:
+    (mean whole-call ms, per-stage ms)."""
+    names = ["partition", "permute", "route", "block_sparse_attn", "probe_correct"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for e in evs:
+        e[0].record(stream)
+        S.sparsepr_partition(qd, kd, p, b.label_q, b.label_k, b.ws, stream)
+        e[1].record(stream)
+        S.sparsepr_permute(qd, kd, vd, p, b.label_q, b.label_k, b.perm_q, b.perm_k, b.off_q,
+                           b.off_k, b.qp, b.kp, b.vp, b.ws, stream)
+        e[2].record(stream)
+        S.sparsepr_route(b.qp, b.kp, p, b.off_q, b.off_k, b.csr, b.k_per_head, b.ws, stream)
+        e[3].record(stream)
+        S.sparsepr_block_sparse_attn(b.qp, b.kp, b.vp, p, b.off_q, b.off_k, b.csr, b.k_per_head,
+                                     b.o_sparse, b.pairs_sparse, b.ws, stream)
+        e[4].record(stream)
+        S.sparsepr_probe_correct(b.qp, b.kp, b.vp, p, b.off_q, b.perm_q, b.o_sparse,
+                                 b.pairs_sparse, b.out, b.probes, b.pairs_exec, b.ws, None,
+                                 stream)
+        e[5].record(stream)
+    torch.cuda.synchronize()
+    stage = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+             for i, n in enumerate(names)}
+    return statistics.mean(e[0].elapsed_time(e[5]) for e in evs), stage
+
+
+def time_dense(S, qd, kd, vd, stream, steps=2):
+    out = torch.empty(qd.shape, dtype=torch.float32, device=qd.device)
+    meta, dws = S.dense_attention(qd, kd, vd, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        S.dense_attention(qd, kd, vd, out, ws=dws, meta=meta)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, out
+
+
+def measure_workload(S, w, dev, stream, peak, steps=3, warmup=2, qkv=None, with_dense=True):
+    """One workload's call on this GPU (direct launches): whole-call and
+    per-stage ms, executed-pair density, the attention kernel's TFLOP/s and
+    roofline fraction, the dense run of the same kernel, workspace bytes."""
+    p = w.params()
+    if qkv is None:
+        q, k, v = synth.generate(w)
+        qkv = (q.to(dev), k.to(dev), v.to(dev))
+    qd, kd, vd = qkv
+    b = S.allocate(p, qd.dtype, dev)
+    for _ in range(warmup):
+        S.attention(qd, kd, vd, p, b, stream)
+    torch.cuda.synchronize()
+    st = S.sparsepr_read_stats(b.ws)
+    ms, stage = time_calls(S, p, b, qd, kd, vd, stream, steps)
+    pairs_sparse = int(b.pairs_sparse.sum())
+    pairs_exec = int(b.pairs_exec.sum())
+    attn = 4.0 * w.d * pairs_sparse / (stage["block_sparse_attn"] * 1e-3) / 1e12
+    r = dict(workload=workload_desc(w), heads_in_one_call=w.H, call_ms=ms, stage_ms=stage,
+             stage_share={n: stage[n] / ms for n in stage},
+             partition_probe_share=(stage["partition"] + stage["probe_correct"]) / ms,
+             rho_exec=pairs_exec / (w.H * w.N * w.N), value_tflops=4.0 * w.d * pairs_exec / (ms * 1e-3) / 1e12,
+             attn_kernel_tflops=attn, attn_roofline_frac=attn / peak,
+             kmeans_passes=dict(key=st["key_passes"][:w.H], query=st["query_passes"][:w.H]),
+             fp64_recheck_rows=st["recheck_rows"], near_ties=st["near_ties"],
+             device_status=st["status"], workspace_bytes=b.ws.numel())
+    if with_dense:
+        dms, _ = time_dense(S, qd, kd, vd, stream)
+        r.update(dense_same_kernel_ms=dms, speedup_vs_dense=dms / ms,
+                 dense_same_kernel_tflops=4.0 * w.d * w.H * w.N * w.N / (dms * 1e-3) / 1e12)
+    return r
+
+
+def output_error(b, dense_out, w):
+    """Mean and max |out - dense attention| over every row (original order)."""
+    err = (b.out.float() - dense_out).abs()
+    return float(err.mean()), float(err.max())
+
+
+def ablations(S, dev, stream, steps=2):
+    """The pages' ablation axes on the 480p layer: partition (response-coupled,
+    semantic k-means, co-clustering), reconstruction on / off (M = 0, hard
+    drop), and the probe count M, rank r and ridge lambda; each with its call
+    time and its output error against dense attention."""
+    w0 = synth.workload("wan13b_480p")
+    q, k, v = synth.generate(w0)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    dms, dense_out = time_dense(S, qd, kd, vd, stream)
+    out = dict(workload=workload_desc(w0), dense_ms=dms,
+               error_note="mean / max |out - dense| over all rows and channels (dense = the same "
+                          "attention kernel over every key)")
+    variants = [("response", {}), ("semantic", dict(partition="semantic")),
+                ("coclustering", dict(partition="coclustering")), ("hard_drop", dict(M=0))]
+    variants += [("M%d" % m, dict(M=m)) for m in (64, 128, 512)]
+    variants += [("r%d" % r, dict(r=r)) for r in (8, 16, 64)]
+    variants += [("lambda%g" % lam, dict(lam=lam)) for lam in (1e-3, 1e-1, 1.0)]
+    for name, kw in variants:
+        w = w0.with_params(**kw)
+        p = w.params()
+        b = S.allocate(p, qd.dtype, dev)
+        S.attention(qd, kd, vd, p, b, stream)
+        torch.cuda.synchronize()
+        ms, stage = time_calls(S, p, b, qd, kd, vd, stream, steps)
+        e_mean, e_max = output_error(b, dense_out, w)
+        st = S.sparsepr_read_stats(b.ws)
+        out[name] = dict(params=kw, call_ms=ms, partition_ms=stage["partition"],
+                         probe_correct_ms=stage["probe_correct"], err_mean=e_mean, err_max=e_max,
+                         rho_exec=int(b.pairs_exec.sum()) / (w.H * w.N * w.N),
+                         passes=dict(key=max(st["key_passes"][:w.H]),
+                                     query=max(st["query_passes"][:w.H])),
+                         device_status=st["status"])
+        del b
+    return out
+
+
+def diagnostics(S, dev, stream, b_main, w_main, qd, kd):
+    """The structural diagnostics: probe rows of the main call (retained mass,
+    error, residual energy split), support expansion on the 480p layer (one
+    query group in 25), density profile of the main layer (one row in 2000)."""
+    p = w_main.params()
+    H, M = w_main.H, w_main.M
+    out = {}
+    mass = torch.empty(H, M, dtype=torch.float64, device=dev)
+    err = torch.empty_like(mass)
+    energy = torch.empty(H, 4, dtype=torch.float64, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    S.sparsepr_probe_diagnostics(p, b_main.probes, mass, err, energy, b_main.ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    en = energy.cpu().numpy()
+    m = mass.cpu().numpy()
+    out["probe_rows"] = dict(
+        ms=e0.elapsed_time(e1), retained_mass_mean=float(m.mean()),
+        retained_mass_min=float(m.min()), error_mean=float(err.mean()),
+        corr_mass_error=float(np.corrcoef(m.ravel(), err.cpu().numpy().ravel())[0, 1]),
+        explainable_share_mean=float(en[:, 1].mean()),
+        unexplained_by_fit_mean=float(en[:, 2].mean()),
+        unexplained_by_projected_fit_mean=float(en[:, 3].mean()))
+    # support expansion (480p, its own call)
+    w = synth.workload("wan13b_480p")
+    pw = w.params()
+    q, k, v = synth.generate(w)
+    q4, k4, v4 = q.to(dev), k.to(dev), v.to(dev)
+    b = S.allocate(pw, q4.dtype, dev)
+    S.attention(q4, k4, v4, pw, b, stream)
+    indiv = torch.empty(w.H, w.Cq, dtype=torch.float64, device=dev)
+    agg = torch.empty_like(indiv)
+    stride = 25
+    e0.record(stream)
+    S.sparsepr_support_expansion(b.qp, b.kp, pw, b.off_q, b.off_k, 0.9, stride, indiv, agg, b.ws,
+                                 stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    iv, ag = indiv.cpu().numpy(), agg.cpu().numpy()
+    sel = ~np.isnan(ag)
+    out["support_expansion"] = dict(
+        workload="wan13b_480p", tau=0.9, groups_sampled=int(sel.sum()),
+        group_stride=stride, ms=e0.elapsed_time(e1),
+        individual_mean=float(iv[sel].mean()), aggregate_mean=float(ag[sel].mean()),
+        expansion_mean=float((ag[sel] / iv[sel]).mean()))
+    del b
+    # density profile of the main layer
+    dens = torch.empty(w_main.H, dtype=torch.float64, device=dev)
+    row_stride = 2000
+    e0.record(stream)
+    S.sparsepr_density_profile(qd, kd, p, 0.95, row_stride, dens, b_main.ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dn = dens.cpu().numpy()
+    out["density"] = dict(workload=w_main.name, tau=0.95, row_stride=row_stride,
+                          ms=e0.elapsed_time(e1), per_head=[float(x) for x in dn],
+                          mean=float(dn.mean()))
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -279,6 +465,8 @@ def main():
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the further workloads, diagnostics and ablations")
     args = ap.parse_args()
     w = synth.workload(args.workload)
 
@@ -488,6 +676,21 @@ def main():
             gpu_launches_per_call=launches,
             gpu_launches_source=launches_src,
         )
+        line["workspace_bytes"] = b.ws.numel()
+        if not args.no_extras and world == 1:
+            # diagnostics first: they read the main call's workspace
+            S.attention(qd, kd, vd, p, b, stream)
+            torch.cuda.synchronize(dev)
+            line["diagnostics"] = diagnostics(S, dev, stream, b, w, qd, kd)
+            line["configs"] = {"wan13b_720p_rho25": measure_workload(
+                S, synth.workload("wan13b_720p_rho25"), dev, stream, peak, qkv=(qd, kd, vd))}
+            del b, qx, kx, vx, dense_out
+            torch.cuda.empty_cache()
+            for name in ("wan13b_480p", "wan14b_720p", "hunyuan13b_720p"):
+                line["configs"][name] = measure_workload(S, synth.workload(name), dev, stream, peak)
+                torch.cuda.empty_cache()
+            line["ablations"] = ablations(S, dev, stream)
+        line["peak_memory_bytes"] = torch.cuda.max_memory_allocated(dev)
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline_sample(w)
         print(json.dumps(line), flush=True)

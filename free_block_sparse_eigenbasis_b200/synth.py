@@ -30,7 +30,9 @@ Value recipe per head (all draws from numpy PCG64 seeded with (seed, head)):
 from __future__ import annotations
 
 import dataclasses
+import concurrent.futures
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -192,19 +194,30 @@ def torch_dtype(w: Workload):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
 
-def generate(w: Workload, heads=None):
+def generate(w: Workload, heads=None, workers=None):
     """Q, K, V as CPU torch tensors [H', N, d] in the workload's dtype, for the
     heads listed in ``heads`` (default: all). Values are generated in fp64 and
-    rounded by torch's conversion to the workload dtype."""
-    hs = range(w.H) if heads is None else list(heads)
+    rounded by torch's conversion to the workload dtype. Heads are generated
+    on ``workers`` threads (default: the CPU count); each head has its own
+    seeded generator, so the values do not depend on the thread count."""
+    hs = list(range(w.H)) if heads is None else list(heads)
     dt = torch_dtype(w)
     out = []
     for x_idx in range(3):
         out.append(torch.empty((len(hs), w.N, w.d), dtype=dt))
-    for i, h in enumerate(hs):
-        vals = _head_values(w, h)
+
+    def fill(i):
+        vals = _head_values(w, hs[i])
         for x_idx in range(3):
             out[x_idx][i].copy_(torch.from_numpy(vals[x_idx]).to(dt))
+
+    n = max(1, min(workers or os.cpu_count() or 1, len(hs)))
+    if n == 1:
+        for i in range(len(hs)):
+            fill(i)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(n) as ex:
+            list(ex.map(fill, range(len(hs))))
     return tuple(out)
 
 
