@@ -760,11 +760,11 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     double* bvec = at<double>(ws, L.bvec);
     double* rtr = at<double>(ws, L.mk);
     // the ridge solve (reads the Grams) runs beside R^T R and its eigen solve
-    // (they touch other regions); with r > 32 the Gram region is reused below,
+    // (they touch other regions); with r > kTriEigMax the Gram region is reused below,
     // so the two stay in order
     // (joined on every path, also after a failed launch)
     std::unique_lock<std::mutex> lk(g_side_mu);
-    SideStream* ss = (c.p.r <= 32) ? side_stream() : nullptr;
+    SideStream* ss = (c.p.r <= kTriEigMax) ? side_stream() : nullptr;
     const cudaStream_t side = fork_side(ss, st);
     cudaError_t err = launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side);
     if (err == cudaSuccess)
@@ -775,7 +775,7 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     double* evc = at<double>(ws, L.evec);
     // leading-r right singular vectors of R = top-r eigenvectors of R^T R
     const double* vr = evc;
-    if (c.p.r <= 32) {
+    if (c.p.r <= kTriEigMax) {
       if (err == cudaSuccess)
         err = launch_sym_eigs(rtr, H, d, c.p.r, evl, evc, at<double>(ws, L.eigscr), st);
     } else {
@@ -815,9 +815,9 @@ sparsepr_status sparsepr_probe_diagnostics(const sparsepr_params* p, const int32
   if (c.p.r > 64) return SPARSEPR_ERR_UNSUPPORTED;
   const Layout& L = c.L;
   // the leading right singular vectors of R as sparsepr_probe_correct left
-  // them: the eigen solver's output for r <= 32, the projector's selection in
+  // them: the eigen solver's output for r <= kTriEigMax, the projector's selection in
   // the Gram region otherwise
-  const double* vr = at<double>(ws, c.p.r <= 32 ? L.evec : L.gram);
+  const double* vr = at<double>(ws, c.p.r <= kTriEigMax ? L.evec : L.gram);
   SPR_TRY(launch_probe_diagnostics(probes, at<float>(ws, L.lse_s), at<float>(ws, L.lse_d),
                                    at<double>(ws, L.xr), at<double>(ws, L.bmat),
                                    at<double>(ws, L.bvec), vr, c.p.H, c.p.N, c.p.M, c.p.d, c.p.r,

@@ -1,4 +1,4 @@
-// Leading eigenpairs of the small symmetric PSD matrices of the path, in fp64:
+// Leading eigenpairs (up to 64) of the small symmetric PSD matrices of the path, in fp64:
 // the sampled-query metric M_K ("Partition the Support, Reconstruct the
 // Residual", 2.A: k-means on the eigenvectors of M_K) and the probe residual
 // Gram R^T R (2.B: leading singular vectors of the probe residuals).
@@ -249,28 +249,39 @@ __device__ void tri_apply(const double* ra, const double* dl, const double* du, 
 
 constexpr int kEigThreads = 512;
 constexpr int kEigWarps = kEigThreads / 32;
+constexpr int kEigMax = kTriEigMax;  // eigenpairs per matrix
+constexpr int kInvBatch = 32;  // eigenvalues in inverse iteration at a time
 
-// One CTA of 512 threads per matrix, ne <= 32 eigenpairs (largest first):
-// multisection by 16-32 threads per eigenvalue, inverse iteration by thread t
-// (one LU, three solves), Gram-Schmidt inside clusters by all warps, then the
-// back-transformation by warp t % 16. Writes evals [H, ne] and evecs [H, D, ne].
+// One CTA of 512 threads per matrix, ne <= 64 eigenpairs (largest first):
+// multisection by 8-32 threads per eigenvalue, inverse iteration by thread t
+// (one LU, three solves) for batches of 32 eigenvalues, Gram-Schmidt inside
+// clusters by all warps, then the back-transformation with warp w owning
+// vectors w, w + 16, ... Writes evals [H, ne] and evecs [H, D, ne].
+// Dynamic shared memory: the inverse-iteration work arrays of one batch (32
+// threads interleaved; later the staged Householder vectors), then the
+// vectors Y [kEigMax][D + 1].
 template <int D>
 constexpr size_t eig_work_bytes() {
-  return static_cast<size_t>(4) * D * 32 * 8 + static_cast<size_t>(D) * 32 * 4;
+  return static_cast<size_t>(4) * D * kInvBatch * 8 + static_cast<size_t>(D) * kInvBatch * 4;
+}
+template <int D>
+constexpr size_t eig_smem_bytes() {
+  return eig_work_bytes<D>() + static_cast<size_t>(kEigMax) * (D + 1) * 8;
 }
 static_assert(eig_work_bytes<128>() >= (128 * 128 + 128) * 8 &&
                   eig_work_bytes<64>() >= (64 * 64 + 64) * 8,
               "the back-transformation reuses the work space for the Householder vectors");
+static_assert(eig_smem_bytes<128>() <= 232448 - 4096, "shared memory");
 
 template <int D>
 __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scratch, int ne,
                                                        double* evals, double* evecs) {
-  extern __shared__ double eig_work[];  // inverse-iteration work arrays, 32 threads interleaved
+  extern __shared__ double eig_work[];  // inverse-iteration work arrays, then Y
+  double (*Y)[D + 1] = reinterpret_cast<double (*)[D + 1]>(eig_work + eig_work_bytes<D>() / 8);
   __shared__ double dg[D], od[D], e2[D];
-  __shared__ double lam[32];
-  __shared__ double Y[32][D + 1];  // padded: thread t walks row t
+  __shared__ double lam[kEigMax];
   __shared__ double tnorm;
-  __shared__ double gdot[32], gred[kEigThreads / 32];
+  __shared__ double gdot[kEigMax], gred[kEigWarps];
   const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const double* hv = scratch + static_cast<size_t>(h) * (D * D + 3 * D);
   const double* tau = hv + D * D;
@@ -292,18 +303,18 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
   const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
   // multisection: tpe threads per wanted eigenvalue (rank e_i = tid / tpe,
-  // ascending index D-1-e_i; tpe = 32 for ne <= 16, 16 for ne <= 32) each
+  // ascending index D-1-e_i; tpe = 32, 16 or 8 for ne <= 16, 32 or 64) each
   // evaluate the Sturm count at one interior point of the current interval,
   // which shrinks (tpe + 1)-fold per round
   {
-    const int tpe = ne <= kEigThreads / 32 ? 32 : 16;
+    const int tpe = ne <= kEigThreads / 32 ? 32 : (ne <= kEigThreads / 16 ? 16 : 8);
     const int e_i = tid / tpe, q = tid % tpe;
     const bool act = e_i < ne;
     const int m = D - 1 - e_i;
     const double inv_parts = 1.0 / (tpe + 1);
-    const unsigned gmask = tpe == 32 ? 0xFFFFFFFFu : 0xFFFFu;
+    const unsigned gmask = tpe == 32 ? 0xFFFFFFFFu : ((1u << tpe) - 1u);
     double lo = -tnorm - 1.0, hi = tnorm + 1.0;
-    for (int it = 0; it < 100; ++it) {
+    for (int it = 0; it < 200; ++it) {
       const double w = hi - lo;
       const bool done = !(w > 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin);
       if (__all_sync(0xffffffffu, done || !act)) break;
@@ -322,93 +333,101 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
     if (act && q == 0) lam[e_i] = 0.5 * (lo + hi);
   }
   __syncthreads();
-  // inverse iteration from a fixed, index-dependent start vector
+  // inverse iteration from a fixed, index-dependent start vector, 32
+  // eigenvalues at a time; Gram-Schmidt against the earlier vectors of the
+  // same cluster (rank order; classical Gram-Schmidt applied twice), all warps
   double* wk = eig_work + (tid & 31);
-  int* pv = reinterpret_cast<int*>(eig_work + 4 * D * 32) + (tid & 31);
+  int* pv = reinterpret_cast<int*>(eig_work + 4 * D * kInvBatch) + (tid & 31);
   const double tiny = eps * fmax(tnorm, 1e-300);
-  if (tid < ne)
-#pragma unroll 1
-    for (int i = 0; i < D; ++i) Y[tid][i] = 1.0 + 0.5 * sin(0.7 * (i + 1) * (tid + 1));
   const double ortol = 1e-3 * tnorm;
   double* wa = wk;
-  double* wdl = wk + D * 32;
-  double* wdu = wk + 2 * D * 32;
-  double* wdu2 = wk + 3 * D * 32;
-  if (tid < ne) tri_factor<D, 32>(dg, od, lam[tid], tiny, wa, wdl, wdu, wdu2, pv);
-  for (int it = 0; it < kInvIters; ++it) {
-    if (tid < ne) {
-      double* b = Y[tid];
-      tri_apply<D, 32>(wa, wdl, wdu, wdu2, pv, b);
-      double s = 0.0;
-#pragma unroll 4
-      for (int i = 0; i < D; ++i) s = fma(b[i], b[i], s);
-      const double inv = 1.0 / sqrt(s);
-#pragma unroll 4
-      for (int i = 0; i < D; ++i) b[i] *= inv;
+  double* wdl = wk + D * kInvBatch;
+  double* wdu = wk + 2 * D * kInvBatch;
+  double* wdu2 = wk + 3 * D * kInvBatch;
+  for (int b0 = 0; b0 < ne; b0 += kInvBatch) {
+    const int nb = min(kInvBatch, ne - b0);
+    const int vi = b0 + tid;  // this thread's eigenvalue (tid < nb)
+    if (tid < nb) {
+#pragma unroll 1
+      for (int i = 0; i < D; ++i) Y[vi][i] = 1.0 + 0.5 * sin(0.7 * (i + 1) * (vi + 1));
+      tri_factor<D, kInvBatch>(dg, od, lam[vi], tiny, wa, wdl, wdu, wdu2, pv);
     }
-    __syncthreads();
-    // Gram-Schmidt against the earlier vectors of the same cluster (rank
-    // order; classical Gram-Schmidt applied twice), all warps
-    for (int t = 1; t < ne; ++t) {
-      int s0 = t;
-      while (s0 > 0 && fabs(lam[s0 - 1] - lam[s0]) <= ortol) --s0;
-      if (s0 == t) continue;  // the same for every thread
-      for (int pass = 0; pass < 2; ++pass) {
-        for (int s = s0 + wid; s < t; s += kEigThreads / 32) {
-          double dot = 0.0;
-          for (int i = lane; i < D; i += 32) dot = fma(Y[s][i], Y[t][i], dot);
-          dot = warp_sum_f64(dot);
-          if (lane == 0) gdot[s] = dot;
+    for (int it = 0; it < kInvIters; ++it) {
+      if (tid < nb) {
+        double* bvec = Y[vi];
+        tri_apply<D, kInvBatch>(wa, wdl, wdu, wdu2, pv, bvec);
+        double sacc = 0.0;
+#pragma unroll 4
+        for (int i = 0; i < D; ++i) sacc = fma(bvec[i], bvec[i], sacc);
+        const double inv = 1.0 / sqrt(sacc);
+#pragma unroll 4
+        for (int i = 0; i < D; ++i) bvec[i] *= inv;
+      }
+      __syncthreads();
+      for (int t = (b0 > 0 ? b0 : 1); t < b0 + nb; ++t) {
+        int s0 = t;
+        while (s0 > 0 && fabs(lam[s0 - 1] - lam[s0]) <= ortol) --s0;
+        if (s0 == t) continue;  // the same for every thread
+        for (int pass = 0; pass < 2; ++pass) {
+          for (int sv = s0 + wid; sv < t; sv += kEigWarps) {
+            double dot = 0.0;
+            for (int i = lane; i < D; i += 32) dot = fma(Y[sv][i], Y[t][i], dot);
+            dot = warp_sum_f64(dot);
+            if (lane == 0) gdot[sv] = dot;
+          }
+          __syncthreads();
+          if (tid < D) {
+            double yv = Y[t][tid];
+            for (int sv = s0; sv < t; ++sv) yv -= gdot[sv] * Y[sv][tid];
+            Y[t][tid] = yv;
+          }
+          __syncthreads();
         }
+        double nn = (tid < D) ? Y[t][tid] * Y[t][tid] : 0.0;
+        nn = warp_sum_f64(nn);
+        if (lane == 0) gred[wid] = nn;
         __syncthreads();
-        if (tid < D) {
-          double y = Y[t][tid];
-          for (int s = s0; s < t; ++s) y -= gdot[s] * Y[s][tid];
-          Y[t][tid] = y;
-        }
+        double tot = 0.0;
+#pragma unroll
+        for (int w = 0; w < kEigWarps; ++w) tot += gred[w];
+        if (tid < D) Y[t][tid] *= 1.0 / sqrt(tot);
         __syncthreads();
       }
-      double nn = (tid < D) ? Y[t][tid] * Y[t][tid] : 0.0;
-      nn = warp_sum_f64(nn);
-      if (lane == 0) gred[wid] = nn;
-      __syncthreads();
-      double tot = 0.0;
-#pragma unroll
-      for (int w = 0; w < kEigThreads / 32; ++w) tot += gred[w];
-      if (tid < D) Y[t][tid] *= 1.0 / sqrt(tot);
-      __syncthreads();
     }
+    __syncthreads();  // the work arrays are reused by the next batch
   }
-  // back-transformation: u = H_0 (H_1 (... H_{D-3} y)), warp w owns vectors
-  // w, w + 8, ...; the Householder vectors and tau are first staged in the
-  // (now free) inverse-iteration work space
+  // back-transformation: u = H_0 (H_1 (... H_{D-3} y)); the Householder
+  // vectors and tau are first staged in the (now free) work space
   double* hs = eig_work;          // [D][D]
   double* ts = eig_work + D * D;  // [D]
   for (int i = tid; i < D * D; i += blockDim.x) hs[i] = hv[i];
   for (int i = tid; i < D; i += blockDim.x) ts[i] = tau[i];
   __syncthreads();
-  // warp w owns vectors w and w + 16 (ne <= 32) and applies each reflection
-  // to both at once
+  // warp w owns vectors w, w + 16, w + 32, w + 48 and applies each
+  // reflection to all of them at once
+  constexpr int kVpw = kEigMax / kEigWarps;
   const int nv = ne > wid ? (ne - wid + kEigWarps - 1) / kEigWarps : 0;
   for (int k = D - 3; k >= 0; --k) {
     const double tk = ts[k];
     if (tk == 0.0) continue;
     const double* hk = hs + k * D;
-    double dot[2] = {0.0, 0.0};
+    double dot[kVpw];
+#pragma unroll
+    for (int v = 0; v < kVpw; ++v) dot[v] = 0.0;
     for (int i = k + 1 + lane; i < D; i += 32) {
       const double hi = hk[i];
 #pragma unroll
-      for (int v = 0; v < 2; ++v)
+      for (int v = 0; v < kVpw; ++v)
         if (v < nv) dot[v] = fma(hi, Y[wid + kEigWarps * v][i], dot[v]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int v = 0; v < 2; ++v) dot[v] += __shfl_xor_sync(0xffffffffu, dot[v], o);
+      for (int v = 0; v < kVpw; ++v) dot[v] += __shfl_xor_sync(0xffffffffu, dot[v], o);
     for (int i = k + 1 + lane; i < D; i += 32) {
       const double hi = hk[i];
 #pragma unroll
-      for (int v = 0; v < 2; ++v)
+      for (int v = 0; v < kVpw; ++v)
         if (v < nv) Y[wid + kEigWarps * v][i] -= (dot[v] * tk) * hi;
     }
     __syncwarp();
@@ -429,10 +448,10 @@ cudaError_t launch_d(const double* A, int H, int ne, double* evals, double* evec
                                        static_cast<int>(shb));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tri_eig_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(eig_work_bytes<D>()));
+                           static_cast<int>(eig_smem_bytes<D>()));
   if (e != cudaSuccess) return e;
   tridiag_kernel<D><<<H, kTriThreads, shb, st>>>(A, scratch);
-  tri_eig_kernel<D><<<H, kEigThreads, eig_work_bytes<D>(), st>>>(scratch, ne, evals, evecs);
+  tri_eig_kernel<D><<<H, kEigThreads, eig_smem_bytes<D>(), st>>>(scratch, ne, evals, evecs);
   return cudaGetLastError();
 }
 
@@ -444,7 +463,7 @@ size_t sym_eigs_scratch_doubles(int H, int d) {
 
 cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals, double* evecs,
                             double* scratch, cudaStream_t st) {
-  if (ne < 1 || ne > 32 || ne > d) return cudaErrorInvalidValue;
+  if (ne < 1 || ne > kEigMax || ne > d) return cudaErrorInvalidValue;
   if (d == 128) return launch_d<128>(A, H, ne, evals, evecs, scratch, st);
   if (d == 64) return launch_d<64>(A, H, ne, evals, evecs, scratch, st);
   return cudaErrorInvalidValue;

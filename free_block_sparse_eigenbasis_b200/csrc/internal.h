@@ -143,7 +143,7 @@ cudaError_t launch_top_eig_projector(const double* eval, const double* evec, int
 cudaError_t launch_scale_columns(const double* vals, const double* vecs, int H, int d, int e,
                                  double* wk, cudaStream_t st);
 
-// ---- eigen.cu: top-ne eigenpairs (ne <= 32) by tridiagonal reduction,
+// ---- eigen.cu: top-ne eigenpairs (ne <= 64) by tridiagonal reduction,
 // bisection and inverse iteration ---------------------------------------------
 size_t sym_eigs_scratch_doubles(int H, int d);
 // evals [H, ne] descending, evecs [H, d, ne].

@@ -19,7 +19,8 @@ constexpr int kSortChunk = 1024;  // tokens per counting-sort chunk
 constexpr int kMaxGroups = 4096;
 constexpr int kMaxSplits = 8;   // split-KV ranges of the dense probe pass
 constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
-constexpr int kDiagRows = 64;   // density-profile rows processed at once (one CTA each)
+constexpr int kDiagRows = 64;
+constexpr int kTriEigMax = 64;  // eigenpairs of the tridiagonal solver (more: cyclic Jacobi)   // density-profile rows processed at once (one CTA each)
 
 struct Layout {
   // statistics / status (always at offset 0)
@@ -252,7 +253,7 @@ inline bool named_region(const sparsepr_params& p, const Layout& L, const char* 
       {"z", L.z, H * Nv * e * 8},       {"ck", L.ck, H * Ck * d * 8},
       {"g", L.g, H * d * d * 8},        {"bmat", L.bmat, H * d * d * 8},
       {"bvec", L.bvec, H * d * 8},      {"xr", L.xr, H * 2 * M * d * 8},
-      {"vr", p.r <= 32 ? L.evec : L.gram, H * d * static_cast<size_t>(p.r) * 8},
+      {"vr", p.r <= kTriEigMax ? L.evec : L.gram, H * d * static_cast<size_t>(p.r) * 8},
   };
   for (const R& r : tab) {
     const char* a = r.n;

@@ -695,21 +695,27 @@ __global__ void __launch_bounds__(kMeanWarpGroups * 32) group_mean_warp_kernel(
 }
 
 // W_g = G qbar_g, c_g = qbar_g^T G qbar_g (fp64, fixed-order reduction).
-// One CTA per (8 query centroids, head); thread a owns column a of W for the
-// CTA's centroids, so every element of G is read once per CTA.
+// One CTA per (8 query centroids, head), 512 threads: thread (a, part) sums
+// the quarter `part` of the columns b of row a of W for the CTA's centroids
+// (G is symmetric, so column a is read, coalesced across a); the four
+// quarters are then added in part order. Every element of G is read once per
+// CTA; four times the warps of a thread-per-column form, each with a quarter
+// of the dependent loads.
 constexpr int kQmaG = 8;
+constexpr int kQmaParts = 4;
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128 * kQmaParts)
     query_metric_apply_kernel(const double* G, const double* qbar, int Cq, int d, double* wg,
                               double* cg, const int32_t* skip, int skip_stride) {
   __shared__ double qs[kQmaG][128];
+  __shared__ double part_w[kQmaParts - 1][kQmaG][128];
   __shared__ double red[kQmaG][4];
   const int h = blockIdx.y, g0 = blockIdx.x * kQmaG;
   if (skip && skip[h * skip_stride]) return;
   const int ng = min(kQmaG, Cq - g0);
   const double* Gh = G + static_cast<size_t>(h) * d * d;
-  const int a = threadIdx.x, lane = a & 31, wp = a >> 5;
-  for (int i = a; i < kQmaG * 128; i += 128) {
+  const int a = threadIdx.x & 127, part = threadIdx.x >> 7;
+  for (int i = threadIdx.x; i < kQmaG * 128; i += blockDim.x) {
     const int g = i >> 7, b = i & 127;
     qs[g][b] = (g < ng && b < d) ? qbar[(static_cast<size_t>(h) * Cq + g0 + g) * d + b] : 0.0;
   }
@@ -717,10 +723,10 @@ __global__ void __launch_bounds__(128)
   double w[kQmaG];
 #pragma unroll
   for (int g = 0; g < kQmaG; ++g) w[g] = 0.0;
+  const int span = d / kQmaParts, b0 = part * span;
   if (a < d) {
-    int b = 0;
 #pragma unroll 1
-    for (; b + 16 <= d; b += 16) {  // 16 loads of G in flight
+    for (int b = b0; b < b0 + span; b += 16) {  // 16 loads of G in flight
       double gb[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) gb[i] = Gh[static_cast<size_t>(b + i) * d + a];
@@ -729,20 +735,27 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
         for (int g = 0; g < kQmaG; ++g) w[g] = fma(gb[i], qs[g][b + i], w[g]);
     }
-    for (; b < d; ++b) {
-      const double gb = Gh[static_cast<size_t>(b) * d + a];
+  }
+  if (part > 0)
 #pragma unroll
-      for (int g = 0; g < kQmaG; ++g) w[g] = fma(gb, qs[g][b], w[g]);
+    for (int g = 0; g < kQmaG; ++g) part_w[part - 1][g][a] = w[g];
+  __syncthreads();
+  if (part == 0) {
+    const int lane = a & 31, wp = a >> 5;
+#pragma unroll
+    for (int g = 0; g < kQmaG; ++g) {
+      double v = w[g];
+#pragma unroll
+      for (int pp = 0; pp < kQmaParts - 1; ++pp) v += part_w[pp][g][a];
+      if (a < d && g < ng) wg[(static_cast<size_t>(h) * Cq + g0 + g) * d + a] = v;
+      const double cv = warp_sum_f64((a < d) ? qs[g][a] * v : 0.0);
+      if (lane == 0) red[g][wp] = cv;
     }
   }
-#pragma unroll
-  for (int g = 0; g < kQmaG; ++g) {
-    if (a < d && g < ng) wg[(static_cast<size_t>(h) * Cq + g0 + g) * d + a] = w[g];
-    const double v = warp_sum_f64((a < d) ? qs[g][a] * w[g] : 0.0);
-    if (lane == 0) red[g][wp] = v;
-  }
   __syncthreads();
-  if (a < ng) cg[static_cast<size_t>(h) * Cq + g0 + a] = (red[a][0] + red[a][1]) + (red[a][2] + red[a][3]);
+  if (threadIdx.x < ng)
+    cg[static_cast<size_t>(h) * Cq + g0 + threadIdx.x] =
+        (red[threadIdx.x][0] + red[threadIdx.x][1]) + (red[threadIdx.x][2] + red[threadIdx.x][3]);
 }
 
 // ---------------------------------------------------------------------------
@@ -1019,7 +1032,8 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx,
 cudaError_t launch_query_metric_apply(const double* G, const double* qbar, int Cq, int H, int d,
                                       double* wg, double* cg, const int32_t* skip,
                                       int skip_stride, cudaStream_t st) {
-  query_metric_apply_kernel<<<dim3((Cq + kQmaG - 1) / kQmaG, H), 128, 0, st>>>(
+  if (d % (16 * kQmaParts) != 0 || d > 128) return cudaErrorInvalidValue;
+  query_metric_apply_kernel<<<dim3((Cq + kQmaG - 1) / kQmaG, H), 128 * kQmaParts, 0, st>>>(
       G, qbar, Cq, d, wg, cg, skip, skip_stride);
   return cudaGetLastError();
 }

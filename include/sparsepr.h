@@ -122,7 +122,7 @@ typedef struct {
   int64_t pairs_sparse[SPARSEPR_MAX_HEADS]; /* routed (row, key) pairs per head */
   int64_t pairs_exec[SPARSEPR_MAX_HEADS];   /* pairs_sparse + M*N (probe rows) */
   int64_t recheck_rows[2]; /* k-means rows decided again in fp64 (keys, queries), all passes */
-  int32_t eig_sweeps[2];   /* Jacobi sweeps, max over heads: [1] = probe residual Gram when r > 32 (the tridiagonal solver serves r <= 32 and M_K, and leaves 0) */
+  int32_t eig_sweeps[2];   /* Jacobi sweeps, max over heads: [1] = probe residual Gram when r > 64 (the tridiagonal solver serves r <= 64 and M_K, and leaves 0) */
   int64_t near_ties[2];    /* k-means rows (keys, queries), summed over heads and passes, whose
                               two smallest fp64 squared distances d1 <= d2 satisfy
                               d2 - d1 <= 1e-12 d2: their label is decided by the lowest-index

@@ -71,6 +71,12 @@ SMALL = [
     # bf16 d=64 with e=24: 64-column operand rows on both tensor-core assignment passes
     synth.custom("bf16_d64_e24", 1, (3, 8, 16), 64, "bf16", Ck=40, Cq=10, Ms=128, n_eig=24,
                  M=24, r=8, keep=0.3, seed=31),
+    # residual subspace ranks past one inverse-iteration batch (r = 48) and past
+    # the tridiagonal solver (r = 96: cyclic Jacobi)
+    synth.custom("rank48", 1, (4, 8, 16), 128, "bf16", Ck=32, Cq=8, Ms=128, n_eig=8, M=128,
+                 r=48, keep=0.3, seed=41),
+    synth.custom("rank96", 1, (4, 8, 16), 128, "bf16", Ck=32, Cq=8, Ms=128, n_eig=8, M=128,
+                 r=96, keep=0.3, seed=42),
 ]
 
 
