@@ -222,18 +222,20 @@ def _check_partition_and_pairs(b, w, st, heads):
             assert int(b.pairs_exec[h]) == pairs + w.M * w.N
 
 
-def test_wan14b_720p_extreme_budgets_sampled():
-    """Wan2.1-14B-shaped layer (its first 8 of 40 heads, with their per-head
-    keep fractions drawn from [0.15, 0.35]) in one call; the heads with the
-    smallest and the largest budget checked against the oracle on sampled
-    rows."""
-    w = synth.workload("wan14b_720p", heads=8)
+def test_wan14b_720p_all_heads_in_one_call():
+    """Wan2.1-14B-shaped layer: all 40 heads in one call, with their per-head
+    keep fractions drawn from [0.15, 0.35]; the first and last heads and the
+    heads with the smallest and the largest budget checked against the
+    oracle on sampled rows, every head for a valid partition and exact pair
+    accounting."""
+    w = synth.workload("wan14b_720p")
+    assert w.H == 40
     b, (q, k, v) = gpu_run(w)
     st = _S().sparsepr_read_stats(b.ws)
     assert st["status"] == 0
-    rows = np.arange(11, w.N, 397)
+    rows = np.arange(11, w.N, 997)
     keep = np.asarray(w.keep)
-    for h in sorted({int(keep.argmin()), int(keep.argmax())}):
+    for h in sorted({0, w.H - 1, int(keep.argmin()), int(keep.argmax())}):
         res = oracle_head(w, q, k, v, h, rows=rows)
         compare_head(b, res, w, h, rows)
     _check_partition_and_pairs(b, w, st, range(w.H))
