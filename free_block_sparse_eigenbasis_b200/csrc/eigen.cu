@@ -6,7 +6,8 @@
 // Textbook dense symmetric eigensolver, specialised to "top ne of d":
 //   1. Householder reduction to tridiagonal form, A = Q T Q^T with
 //      Q = H_0 H_1 ... H_{d-3}, H_k = I - tau_k v_k v_k^T (Golub & Van Loan,
-//      Matrix Computations, sec. 8.3.1), one CTA per matrix in shared memory;
+//      Matrix Computations, sec. 8.3.1), one CTA per matrix held in its
+//      threads' registers;
 //   2. the ne largest eigenvalues of T by multisection on Sturm-sequence
 //      counts (sec. 8.4.1): 16 or 32 threads per eigenvalue, one point each;
 //   3. their eigenvectors by inverse iteration on T - lambda I with one
@@ -26,14 +27,34 @@ constexpr int kInvIters = 3;
 
 // Scratch per matrix (fp64): hv [D][D] Householder vectors (row k holds v_k
 // at columns k+1.., v_k[0] = 1), tau [D], dg [D], od [D].
+//
+// The matrix lives in registers: warp w holds rows w, w + 16, .. (kRpw of
+// them) and lane l columns l, l + 32, .. (kCpl), so row k (= column k by
+// symmetry) sits in one warp, which forms v_k, tau_k and beta_k from it
+// alone. Per column k:
+//   1. the warp holding row k publishes v_k and tau_k (alternating buffers,
+//      so that it can run ahead while other warps still read the last v);
+//   2. every warp forms its rows of p = tau A v: per-lane partial dots, then
+//      a transposed butterfly over the lanes that leaves each row's sum in a
+//      group of lanes; the block sums v^T p from per-warp partials (one
+//      fixed order, identical in every thread);
+//   3. every thread updates its entries, A -= v w^T + w v^T with
+//      w = p - (tau / 2)(v^T p) v (Golub & Van Loan, sec. 8.3.1).
+// Rows and 32-column slots at or above k hold only zeros of v and w and are
+// skipped. Two barriers per column.
+constexpr int kTriWarps = kTriThreads / 32;
+
 template <int D>
-__global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in, double* scratch) {
-  extern __shared__ double tsm[];
-  double* A = tsm;              // [D*D] full symmetric (rows are read instead of columns)
-  double* v = A + D * D;        // [D]
-  double* w = v + D;            // [D]
-  __shared__ double red[2][kTriThreads / 32];
-  __shared__ double pw[kTriThreads / D][D];
+__global__ void __launch_bounds__(kTriThreads, 1)
+    tridiag_kernel(const double* A_in, double* scratch) {
+  constexpr int kRpw = D / kTriWarps;  // rows per warp
+  constexpr int kCpl = D / 32;         // columns per lane
+  constexpr int kLgR = kRpw == 8 ? 3 : (kRpw == 4 ? 2 : (kRpw == 2 ? 1 : 0));
+  static_assert((1 << kLgR) == kRpw, "rows per warp must be a power of two up to 8");
+  constexpr int kGroup = 32 >> kLgR;  // lanes that share one row's sum
+  __shared__ double vb[2][D + 1];     // v (and tau at [D]), two buffers
+  __shared__ double pb[D];            // p = tau A v (zero at rows <= k)
+  __shared__ double part[kTriWarps];  // per-warp partials of v^T p
   const int h = blockIdx.x;
   const double* Ah = A_in + static_cast<size_t>(h) * D * D;
   double* hv = scratch + static_cast<size_t>(h) * (D * D + 3 * D);
@@ -41,115 +62,122 @@ __global__ void __launch_bounds__(kTriThreads) tridiag_kernel(const double* A_in
   double* dg = tau + D;
   double* od = dg + D;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  for (int t = tid; t < D * D; t += blockDim.x) A[t] = Ah[t];
-  __syncthreads();
-  int nsum = 0;
-  // sum over the block with one barrier (alternating buffers; every thread
-  // adds the warp partials in the same order)
-  auto block_sum = [&](double x) -> double {
-    x = warp_sum_f64(x);
-    double* rb = red[nsum++ & 1];
-    if (lane == 0) rb[wid] = x;
-    __syncthreads();
-    double s = 0.0;
+  double a[kRpw][kCpl];
 #pragma unroll
-    for (int i = 0; i < kTriThreads / 32; ++i) s += rb[i];
-    return s;
-  };
-  constexpr int kParts = kTriThreads / D;  // row parts of the matrix-vector product
-  __shared__ double x2s;  // squared norm of the next column below its subdiagonal
-  {
-    double x2 = 0.0;
-    for (int i = 2 + tid; i < D; i += blockDim.x) x2 = fma(A[i], A[i], x2);
-    x2 = block_sum(x2);
-    if (tid == 0) x2s = x2;
-    __syncthreads();
-  }
-  // Three barriers per column: after the matrix-vector product, after its
-  // dot with v, after the rank-2 update (which also yields the next x2).
+  for (int r = 0; r < kRpw; ++r)
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) a[r][c] = Ah[(wid + kTriWarps * r) * D + lane + 32 * c];
+  const int rho = lane >> (5 - kLgR);  // the row slot whose sum this lane ends with
   for (int k = 0; k < D - 2; ++k) {
-    const int n1 = D - k - 1;  // length of v (rows k+1 .. D-1)
-    const double* Ak = A + k * D;  // row k = column k (symmetry)
-    const double x2 = x2s;
-    const double alpha = Ak[k + 1];
-    if (x2 == 0.0) {  // column already reduced: H_k = I
-      __syncthreads();  // every thread has read x2s
-      if (tid == 0) {
-        tau[k] = 0.0;
-        od[k] = alpha;
+    double* vv = vb[k & 1];
+    if (wid == (k % kTriWarps)) {
+      const int rk = k / kTriWarps;
+      double x[kCpl];
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        x[c] = 0.0;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) x[c] = (r == rk) ? a[r][c] : x[c];
       }
-      for (int i = tid; i < n1; i += blockDim.x) hv[k * D + (k + 1 + i)] = (i == 0) ? 1.0 : 0.0;
-      if (wid == 0) {  // next column's norm (A is unchanged)
-        double y2 = 0.0;
-        for (int i = k + 3 + lane; i < D; i += 32) y2 = fma(A[(k + 1) * D + i], A[(k + 1) * D + i], y2);
-        y2 = warp_sum_f64(y2);
-        __syncwarp();
-        if (lane == 0) x2s = y2;
+      double x2 = 0.0, al = 0.0;
+      const int ca = (k + 1) >> 5;
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        const int j = lane + 32 * c;
+        if (j > k + 1) x2 = fma(x[c], x[c], x2);
+        al = (c == ca) ? x[c] : al;
       }
-      __syncthreads();
-      continue;
+      x2 = warp_sum_f64(x2);
+      const double alpha = __shfl_sync(0xffffffffu, al, (k + 1) & 31);
+      double tk = 0.0, beta = alpha, scl = 0.0;
+      if (x2 != 0.0) {  // else the column is already reduced: H_k = I
+        beta = -copysign(sqrt(alpha * alpha + x2), alpha);
+        tk = (beta - alpha) / beta;
+        scl = 1.0 / (alpha - beta);
+      }
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        const int j = lane + 32 * c;
+        const double vj = (j == k + 1) ? 1.0 : (j > k + 1 ? x[c] * scl : 0.0);
+        vv[j] = vj;
+        hv[k * D + j] = vj;
+      }
+      if (lane == 0) {
+        vv[D] = tk;
+        tau[k] = tk;
+        od[k] = beta;
+      }
     }
-    const double beta = -copysign(sqrt(alpha * alpha + x2), alpha);
-    const double tk = (beta - alpha) / beta;
-    const double scl = 1.0 / (alpha - beta);
-    for (int i = tid; i < n1; i += blockDim.x) {
-      const double vi = (i == 0) ? 1.0 : Ak[k + 1 + i] * scl;
-      v[i] = vi;
-      hv[k * D + (k + 1 + i)] = vi;
-    }
-    if (tid == 0) {
-      tau[k] = tk;
-      od[k] = beta;
-    }
-    // p = tau A22 v by columns (A22 symmetric): thread (column c, part) sums
-    // the rows r = part, part + kParts, ...; v_r is formed from row k of A,
-    // which this column does not change
+    __syncthreads();
+    const double tk = vv[D];
+    double vc[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) vc[c] = vv[lane + 32 * c];
     {
-      const int c = tid % D, part = tid / D;
-      double sacc = 0.0;
-      if (c < n1) {
-        const double* col = A + (k + 1) * D + (k + 1) + c;
-        for (int r = part; r < n1; r += kParts) {
-          const double vr = (r == 0) ? 1.0 : Ak[k + 1 + r] * scl;
-          sacc = fma(col[r * D], vr, sacc);
+      double t[kRpw];
+#pragma unroll
+      for (int r = 0; r < kRpw; ++r) {
+        t[r] = 0.0;
+        if (wid + kTriWarps * r > k) {
+#pragma unroll
+          for (int c = 0; c < kCpl; ++c)
+            if (32 * c + 31 > k) t[r] = fma(a[r][c], vc[c], t[r]);
         }
       }
-      pw[part][c] = sacc;
+      // transposed butterfly: halve the rows held per lane at each step
+#pragma unroll
+      for (int st = 0; st < kLgR; ++st) {
+        const int half = kRpw >> (st + 1);
+        const int m = 16 >> st;
+        const bool hi = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const double send = hi ? t[i] : t[i + half];
+          const double keep = hi ? t[i + half] : t[i];
+          t[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+#pragma unroll
+      for (int o = kGroup >> 1; o > 0; o >>= 1) t[0] += __shfl_xor_sync(0xffffffffu, t[0], o);
+      const int row = wid + kTriWarps * rho;
+      const double pr = (row > k) ? tk * t[0] : 0.0;
+      const bool leader = (lane & (kGroup - 1)) == 0;
+      if (leader) pb[row] = pr;
+      const double pv = warp_sum_f64(leader ? pr * vv[row] : 0.0);
+      if (lane == 0) part[wid] = pv;
     }
     __syncthreads();
     double pv = 0.0;
-    if (tid < n1) {
-      double sacc = pw[0][tid];
 #pragma unroll
-      for (int q = 1; q < kParts; ++q) sacc += pw[q][tid];
-      const double wi = tk * sacc;
-      w[tid] = wi;
-      pv = wi * v[tid];
+    for (int i = 0; i < kTriWarps; ++i) pv += part[i];
+    const double hc = 0.5 * tk * pv;
+    double wc[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) {
+      const int j = lane + 32 * c;
+      wc[c] = (j > k) ? fma(-hc, vc[c], pb[j]) : 0.0;
     }
-    pv = block_sum(pv);
-    const double kk2 = -tk * pv;  // A22 -= v w'^T + w' v^T with w' = w + (kk2 / 2) v
-    // (warp = row stripe, lane = column stripe); warp 0 owns row k+1 and
-    // forms the next column's squared norm below its subdiagonal
-    for (int r = wid; r < n1; r += kTriThreads / 32) {
-      const double vr = v[r], wr = w[r];
-      const double a_r = fma(kk2, vr, wr);
-      double* Ar = A + (k + 1 + r) * D + (k + 1);
-      double y2 = 0.0;
-      for (int c = lane; c < n1; c += 32) {
-        const double nv = Ar[c] - (vr * w[c] + a_r * v[c]);
-        Ar[c] = nv;
-        if (c >= 2) y2 = fma(nv, nv, y2);
-      }
-      if (r == 0) {
-        y2 = warp_sum_f64(y2);
-        if (lane == 0) x2s = y2;
+#pragma unroll
+    for (int r = 0; r < kRpw; ++r) {
+      const int i = wid + kTriWarps * r;
+      if (i > k) {
+        const double vr = vv[i];
+        const double wr = fma(-hc, vr, pb[i]);
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c)
+          if (32 * c + 31 > k) a[r][c] -= fma(vr, wc[c], wr * vc[c]);
       }
     }
-    __syncthreads();
   }
-  for (int i = tid; i < D; i += blockDim.x) dg[i] = A[i * D + i];
+#pragma unroll
+  for (int r = 0; r < kRpw; ++r)
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) {
+      const int i = wid + kTriWarps * r, j = lane + 32 * c;
+      if (i == j) dg[i] = a[r][c];
+      if (i == D - 1 && j == D - 2) od[D - 2] = a[r][c];
+    }
   if (tid == 0) {
-    od[D - 2] = A[(D - 1) * D + (D - 2)];
     od[D - 1] = 0.0;
     tau[D - 2] = 0.0;
     tau[D - 1] = 0.0;
@@ -442,15 +470,11 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
 template <int D>
 cudaError_t launch_d(const double* A, int H, int ne, double* evals, double* evecs,
                      double* scratch, cudaStream_t st) {
-  const size_t shb = (static_cast<size_t>(D) * D + 2 * D) * 8;
-  cudaError_t e = cudaFuncSetAttribute(tridiag_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(tri_eig_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(shb));
+                                       static_cast<int>(eig_smem_bytes<D>()));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(tri_eig_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(eig_smem_bytes<D>()));
-  if (e != cudaSuccess) return e;
-  tridiag_kernel<D><<<H, kTriThreads, shb, st>>>(A, scratch);
+  tridiag_kernel<D><<<H, kTriThreads, 0, st>>>(A, scratch);
   tri_eig_kernel<D><<<H, kEigThreads, eig_smem_bytes<D>(), st>>>(scratch, ne, evals, evecs);
   return cudaGetLastError();
 }

@@ -120,90 +120,189 @@ __global__ void probe_means_kernel(const double* part, int nblk, int M, int d, d
   means[(static_cast<size_t>(h) * 2 + 1) * d + a] = M > 0 ? sr / M : 0.0;
 }
 
-// Ridge solve per head: L L^T = A (right-looking Cholesky on the packed
-// lower triangle in shared memory), then L Y = C and L^T B = Y with all d
-// right-hand sides at once (row-by-row elimination, parallel over the rows
-// below and the columns), and b = rbar - xbar B.
+// Ridge solve per head, A B = C with A = X^T X + lambda I (SPD) and C = X^T R,
+// then b = rbar - xbar B. One CTA per head; the d x d matrices live in the
+// threads' registers: warp w holds rows w, w + 16, .. and lane l columns l,
+// l + 32, .. (Golub & Van Loan, sec. 4.2, right-looking outer-product
+// Cholesky, then substitution by rows):
+//   1. Cholesky, column j: the warp holding row j of the (symmetric) trailing
+//      matrix forms l_jj = sqrt(a_jj) and l_kj = a_jk / l_jj (k > j) and
+//      publishes them as row j of Lt = L^T in shared memory; every thread
+//      then updates a_ik -= l_ij l_kj on its entries with i, k > j;
+//   2. L Y = C: the warp holding row j of C forms y_j = c_j / l_jj and
+//      publishes it; every thread updates c_i -= l_ij y_j for its rows i > j;
+//   3. L^T B = Y the same way from the last row up (y_i -= l_ji b_j, i < j).
+// One barrier per step; the published rows of Y and B alternate between two
+// buffers so that the next row's warp can run ahead. A pivot that is not
+// positive (A not SPD) is replaced by 1 for the rest of the solve and the
+// head gets B = 0, b = 0 and SPARSEPR_ERR_NUMERIC.
 constexpr int kRidgeThreads = 512;
+constexpr int kRidgeWarps = kRidgeThreads / 32;
 
 template <int d>
-__global__ void __launch_bounds__(kRidgeThreads)
+constexpr size_t ridge_smem_bytes() {
+  return (static_cast<size_t>(d) * (d + 1) + 2 * d + static_cast<size_t>(kRidgeWarps) * d) * 8;
+}
+
+template <int d>
+__global__ void __launch_bounds__(kRidgeThreads, 1)
     ridge_solve_kernel(const double* gram, double* bmat, double* bvec, const double* means,
                        DeviceStats* stats) {
+  constexpr int kRpw = d / kRidgeWarps, kCpl = d / 32;
   extern __shared__ double rsm[];
-  const int ntri = d * (d + 1) / 2;
-  double* Lp = rsm;          // packed lower triangle, L[i][k] at i*(i+1)/2 + k
-  double* Cm = rsm + ntri;   // [d][d] right-hand sides (row-major), solved in place
+  double* Lt = rsm;                                 // [d][d + 1]: row j = column j of L
+  double* rowb = Lt + static_cast<size_t>(d) * (d + 1);  // [2][d] published rows
+  double* part = rowb + 2 * d;                      // [warps][d] partial sums of xbar B
   __shared__ int bad;
-  const int h = blockIdx.x, tid = threadIdx.x;
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const double* A = gram + static_cast<size_t>(h) * 2 * d * d;
   const double* C = A + static_cast<size_t>(d) * d;
-  for (int t = tid; t < d * d; t += blockDim.x) {
-    const int i = t / d, k = t % d;
-    if (k <= i) Lp[i * (i + 1) / 2 + k] = A[t];
-    Cm[t] = C[t];
-  }
   if (tid == 0) bad = 0;
+  double m[kRpw][kCpl];
+#pragma unroll
+  for (int r = 0; r < kRpw; ++r)
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) m[r][c] = A[(wid + kRidgeWarps * r) * d + lane + 32 * c];
   __syncthreads();
-  auto L = [&](int i, int k) -> double& { return Lp[i * (i + 1) / 2 + k]; };
-  // Cholesky: column j, then the trailing triangle (4 threads per row)
+  // 1. Cholesky
   for (int j = 0; j < d; ++j) {
-    if (tid == 0) {
-      double s = L(j, j);
-      if (!(s > 0.0)) {
-        bad = 1;
-        s = 1.0;
+    double* lrow = Lt + static_cast<size_t>(j) * (d + 1);
+    if (wid == j % kRidgeWarps) {
+      const int rj = j / kRidgeWarps;
+      double x[kCpl];
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        x[c] = 0.0;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) x[c] = (r == rj) ? m[r][c] : x[c];
       }
-      L(j, j) = sqrt(s);
+      // a_jj (a select here would become an indexed local-memory load; a
+      // non-finite row makes a_jj non-finite and fails the pivot test)
+      double ajj = 0.0;
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) ajj = fma((c == (j >> 5)) ? 1.0 : 0.0, x[c], ajj);
+      ajj = __shfl_sync(0xffffffffu, ajj, j & 31);
+      if (!(ajj > 0.0)) {
+        if (lane == 0) bad = 1;
+        ajj = 1.0;
+      }
+      const double ljj = sqrt(ajj);
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        const int k = lane + 32 * c;
+        lrow[k] = (k > j) ? x[c] / ljj : (k == j ? ljj : 0.0);
+      }
     }
     __syncthreads();
-    const double ljj = L(j, j);
-    for (int i = j + 1 + tid; i < d; i += blockDim.x) L(i, j) /= ljj;
-    __syncthreads();
-    for (int q = tid; q < (d - j - 1) * 4; q += blockDim.x) {
-      const int i = j + 1 + (q >> 2);
-      const double lij = L(i, j);
-      for (int k = j + 1 + (q & 3); k <= i; k += 4) L(i, k) -= lij * L(k, j);
+    double lc[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) lc[c] = lrow[lane + 32 * c];
+#pragma unroll
+    for (int r = 0; r < kRpw; ++r) {
+      const int i = wid + kRidgeWarps * r;
+      if (i > j) {
+        const double li = lrow[i];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c)
+          if (32 * c + 31 > j) m[r][c] = fma(-li, lc[c], m[r][c]);
+      }
+    }
+  }
+  // 2. L Y = C (the registers now hold C)
+#pragma unroll
+  for (int r = 0; r < kRpw; ++r)
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) m[r][c] = C[(wid + kRidgeWarps * r) * d + lane + 32 * c];
+  for (int j = 0; j < d; ++j) {
+    double* yrow = rowb + (j & 1) * d;
+    if (wid == j % kRidgeWarps) {
+      const double ljj = Lt[static_cast<size_t>(j) * (d + 1) + j];
+      const int rj = j / kRidgeWarps;
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        double x = 0.0;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) x = (r == rj) ? m[r][c] : x;
+        yrow[lane + 32 * c] = x / ljj;
+      }
     }
     __syncthreads();
+    double yc[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) yc[c] = yrow[lane + 32 * c];
+    const double* lrow = Lt + static_cast<size_t>(j) * (d + 1);
+#pragma unroll
+    for (int r = 0; r < kRpw; ++r) {
+      const int i = wid + kRidgeWarps * r;
+      if (i > j) {
+        const double li = lrow[i];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) m[r][c] = fma(-li, yc[c], m[r][c]);
+      } else if (i == j) {
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) m[r][c] = yc[c];
+      }
+    }
   }
-  // forward: L Y = C
-  for (int i = 0; i < d; ++i) {
-    const double lii = L(i, i);
-    for (int c = tid; c < d; c += blockDim.x) Cm[i * d + c] /= lii;
-    __syncthreads();
-    for (int t = tid; t < (d - i - 1) * d; t += blockDim.x) {
-      const int r = i + 1 + t / d, c = t % d;
-      Cm[r * d + c] -= L(r, i) * Cm[i * d + c];
+  // 3. L^T B = Y
+  for (int j = d - 1; j >= 0; --j) {
+    double* brow = rowb + (j & 1) * d;
+    if (wid == j % kRidgeWarps) {
+      const double ljj = Lt[static_cast<size_t>(j) * (d + 1) + j];
+      const int rj = j / kRidgeWarps;
+#pragma unroll
+      for (int c = 0; c < kCpl; ++c) {
+        double x = 0.0;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) x = (r == rj) ? m[r][c] : x;
+        brow[lane + 32 * c] = x / ljj;
+      }
     }
     __syncthreads();
-  }
-  // backward: L^T B = Y
-  for (int i = d - 1; i >= 0; --i) {
-    const double lii = L(i, i);
-    for (int c = tid; c < d; c += blockDim.x) Cm[i * d + c] /= lii;
-    __syncthreads();
-    for (int t = tid; t < i * d; t += blockDim.x) {
-      const int r = t / d, c = t % d;
-      Cm[r * d + c] -= L(i, r) * Cm[i * d + c];
+    double bc[kCpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) bc[c] = brow[lane + 32 * c];
+#pragma unroll
+    for (int r = 0; r < kRpw; ++r) {
+      const int i = wid + kRidgeWarps * r;
+      if (i < j) {
+        const double lji = Lt[static_cast<size_t>(i) * (d + 1) + j];
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) m[r][c] = fma(-lji, bc[c], m[r][c]);
+      } else if (i == j) {
+#pragma unroll
+        for (int c = 0; c < kCpl; ++c) m[r][c] = bc[c];
+      }
     }
-    __syncthreads();
   }
-  if (bad) {
-    for (int t = tid; t < d * d; t += blockDim.x) Cm[t] = 0.0;
-    if (tid == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
-    __syncthreads();
-  }
+  const bool failed = bad != 0;  // set before the first barrier after the Cholesky
   double* Bo = bmat + static_cast<size_t>(h) * d * d;
-  for (int t = tid; t < d * d; t += blockDim.x) Bo[t] = Cm[t];
-  if (tid < d) {
-    const int col = tid;
-    const double* xbar = means + static_cast<size_t>(h) * 2 * d;
-    const double* rbar = xbar + d;
-    double s = rbar[col];
-    for (int a2 = 0; a2 < d; ++a2) s -= xbar[a2] * Cm[a2 * d + col];
-    bvec[static_cast<size_t>(h) * d + col] = bad ? 0.0 : s;
+  const double* xbar = means + static_cast<size_t>(h) * 2 * d;
+  const double* rbar = xbar + d;
+  double pc[kCpl];
+#pragma unroll
+  for (int c = 0; c < kCpl; ++c) pc[c] = 0.0;
+#pragma unroll
+  for (int r = 0; r < kRpw; ++r) {
+    const int i = wid + kRidgeWarps * r;
+    const double xi = xbar[i];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) {
+      const double v = failed ? 0.0 : m[r][c];
+      Bo[static_cast<size_t>(i) * d + lane + 32 * c] = v;
+      pc[c] = fma(xi, v, pc[c]);
+    }
   }
+#pragma unroll
+  for (int c = 0; c < kCpl; ++c) part[wid * d + lane + 32 * c] = pc[c];
+  __syncthreads();
+  if (tid < d) {
+    double sx = 0.0;
+#pragma unroll
+    for (int w = 0; w < kRidgeWarps; ++w) sx += part[w * d + tid];
+    bvec[static_cast<size_t>(h) * d + tid] = failed ? 0.0 : rbar[tid] - sx;
+  }
+  if (failed && tid == 0) raise_status(stats, SPARSEPR_ERR_NUMERIC);
 }
 
 // Restriction to the residual subspace: with V_r [d, r] the leading right
@@ -341,8 +440,8 @@ cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const
 
 cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
                                const double* means, DeviceStats* stats, cudaStream_t st) {
-  const size_t shb = (static_cast<size_t>(d) * (d + 1) / 2 + static_cast<size_t>(d) * d) * 8;
   if (d != 64 && d != 128) return cudaErrorInvalidValue;
+  const size_t shb = (d == 128) ? ridge_smem_bytes<128>() : ridge_smem_bytes<64>();
   auto kern = (d == 128) ? ridge_solve_kernel<128> : ridge_solve_kernel<64>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shb));
   if (e != cudaSuccess) return e;

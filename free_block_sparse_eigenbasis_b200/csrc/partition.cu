@@ -14,8 +14,12 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Initial centroids: partial Fisher-Yates shuffle driven by SplitMix64
-// (Steele, Lea & Flood 2014). The virtual array a[i] = i is kept as a small
-// open-addressing map of the positions that moved.
+// (Steele, Lea & Flood 2014). Draw i uses the generator's (i + 1)-th state,
+// so every swap target j_i = i + z_i mod (Nv - i) is formed in parallel
+// first; the swaps then run in order on one thread. The virtual array
+// a[i] = i is kept as a small open-addressing map of the positions that
+// moved; position i is never read after step i (later targets are > i), so
+// only the swap target j_i is written back.
 // ---------------------------------------------------------------------------
 constexpr int kFyTable = 16384;  // >= 2 * kMaxGroups, power of two
 
@@ -30,38 +34,40 @@ __global__ void fy_init_kernel(int Nv, int Ck, int Cq, uint64_t seed, int32_t* i
   extern __shared__ int32_t tab[];
   int32_t* keys = tab;
   int32_t* vals = tab + kFyTable;
+  int32_t* tgt = vals + kFyTable;  // [C] swap targets
   const int h = blockIdx.x, which = blockIdx.y;
   const int C = which ? Cq : Ck;
   int32_t* out = which ? init_q + static_cast<size_t>(h) * Cq : init_k + static_cast<size_t>(h) * Ck;
   for (int i = threadIdx.x; i < kFyTable; i += blockDim.x) keys[i] = -1;
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  uint64_t state = seed ^ static_cast<uint64_t>(2 * h + which);
-  for (int i = 0; i < C; ++i) {
-    state += 0x9E3779B97F4A7C15ull;
-    uint64_t z = state;
+  const uint64_t base = seed ^ static_cast<uint64_t>(2 * h + which);
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    uint64_t z = base + static_cast<uint64_t>(i + 1) * 0x9E3779B97F4A7C15ull;
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
     z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
     z ^= z >> 31;
-    const int j = i + static_cast<int>(z % static_cast<uint64_t>(Nv - i));
+    tgt[i] = i + static_cast<int>(z % static_cast<uint64_t>(Nv - i));
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  for (int i = 0; i < C; ++i) {
+    const int j = tgt[i];
     const int si = fy_find(keys, i);
     const int32_t vi = (keys[si] == i) ? vals[si] : i;
     const int sj = fy_find(keys, j);
     const int32_t vj = (keys[sj] == j) ? vals[sj] : j;
-    keys[si] = i;
-    vals[si] = vj;
-    const int sj2 = fy_find(keys, j);  // slot may have shifted if si took it
-    keys[sj2] = j;
-    vals[sj2] = vi;
+    keys[sj] = j;  // a match or the empty slot that ends j's probe
+    vals[sj] = vi;
     out[i] = vj;
   }
 }
 
-// e = 16 (the workloads' eigenbasis size): thread = key row with all 16
-// coordinates in registers; the row of k is streamed with 16-byte loads and
-// W [d][16] is read from shared memory as 16-byte broadcasts, so every
-// widened element of k serves 16 fma. Same ascending-column sums as above.
+// e = 16 (the workloads' eigenbasis size): thread = two key rows with all 16
+// coordinates of each in registers; the rows of k are streamed with 16-byte
+// loads and W [d][16] is read from shared memory as 16-byte broadcasts, so
+// every value of W read serves two rows. Same ascending-column sums as
+// above.
 constexpr int kZRowThreads = 128;
+constexpr int kZ16Rows = 2;  // rows per thread
 
 template <typename T>
 __global__ void __launch_bounds__(kZRowThreads)
@@ -69,33 +75,46 @@ __global__ void __launch_bounds__(kZRowThreads)
   constexpr int E = 16, EPT = 16 / sizeof(T);
   extern __shared__ double w16[];  // [d][16]
   const int h = blockIdx.y;
-  const int j = blockIdx.x * kZRowThreads + threadIdx.x;
+  const int j0 = blockIdx.x * kZRowThreads * kZ16Rows + threadIdx.x;
   const double* W = wk + static_cast<size_t>(h) * d * E;
   for (int t = threadIdx.x; t < d * E; t += kZRowThreads) w16[t] = W[t];
   __syncthreads();
-  if (j >= Nv) return;
-  const T* kr = k + (static_cast<size_t>(h) * N + j) * d;
-  double acc[E];
+  if (j0 >= Nv) return;
+  const bool two = j0 + kZRowThreads < Nv;
+  const T* kr0 = k + (static_cast<size_t>(h) * N + j0) * d;
+  const T* kr1 = two ? kr0 + static_cast<size_t>(kZRowThreads) * d : kr0;
+  double acc[kZ16Rows][E];
 #pragma unroll
-  for (int c = 0; c < E; ++c) acc[c] = 0.0;
+  for (int r = 0; r < kZ16Rows; ++r)
+#pragma unroll
+    for (int c = 0; c < E; ++c) acc[r][c] = 0.0;
 #pragma unroll 1
   for (int a0 = 0; a0 < d; a0 += EPT) {
-    double kv[EPT];
-    vload16(kr + a0, kv);
+    double kv[kZ16Rows][EPT];
+    vload16(kr0 + a0, kv[0]);
+    vload16(kr1 + a0, kv[1]);
 #pragma unroll
     for (int i = 0; i < EPT; ++i) {
       const double2* wa = reinterpret_cast<const double2*>(w16 + (a0 + i) * E);
 #pragma unroll
       for (int c2 = 0; c2 < E / 2; ++c2) {
         const double2 wv = wa[c2];
-        acc[2 * c2] = fma(kv[i], wv.x, acc[2 * c2]);
-        acc[2 * c2 + 1] = fma(kv[i], wv.y, acc[2 * c2 + 1]);
+#pragma unroll
+        for (int r = 0; r < kZ16Rows; ++r) {
+          acc[r][2 * c2] = fma(kv[r][i], wv.x, acc[r][2 * c2]);
+          acc[r][2 * c2 + 1] = fma(kv[r][i], wv.y, acc[r][2 * c2 + 1]);
+        }
       }
     }
   }
-  double2* zr = reinterpret_cast<double2*>(z + (static_cast<size_t>(h) * Nv + j) * E);
 #pragma unroll
-  for (int c2 = 0; c2 < E / 2; ++c2) zr[c2] = make_double2(acc[2 * c2], acc[2 * c2 + 1]);
+  for (int r = 0; r < kZ16Rows; ++r) {
+    if (r == 1 && !two) break;
+    double2* zr = reinterpret_cast<double2*>(
+        z + (static_cast<size_t>(h) * Nv + j0 + r * kZRowThreads) * E);
+#pragma unroll
+    for (int c2 = 0; c2 < E / 2; ++c2) zr[c2] = make_double2(acc[r][2 * c2], acc[r][2 * c2 + 1]);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -892,7 +911,8 @@ __global__ void write_labels_kernel(const int32_t* lab, int H, int N, int Nv, in
 
 cudaError_t launch_fy_init(int H, int Nv, int Ck, int Cq, uint64_t seed, int32_t* init_k,
                            int32_t* init_q, cudaStream_t st) {
-  const int shb = 2 * kFyTable * 4;
+  if (Ck > kMaxGroups || Cq > kMaxGroups) return cudaErrorInvalidValue;
+  const int shb = (2 * kFyTable + kMaxGroups) * 4;
   const cudaError_t e =
       cudaFuncSetAttribute(fy_init_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
   if (e != cudaSuccess) return e;
@@ -924,7 +944,7 @@ cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, 
                          const double* wk, double* z, cudaStream_t st) {
   if (e == 16 && d % 8 == 0 && reinterpret_cast<uintptr_t>(k) % 16 == 0) {
     const size_t shb16 = static_cast<size_t>(d) * 16 * 8;
-    dim3 g16((Nv + kZRowThreads - 1) / kZRowThreads, H);
+    dim3 g16((Nv + kZRowThreads * kZ16Rows - 1) / (kZRowThreads * kZ16Rows), H);
     if (bf16)
       zproj_row16_kernel<<<g16, kZRowThreads, shb16, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv,
                                                            d, wk, z);
