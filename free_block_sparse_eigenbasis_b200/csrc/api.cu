@@ -462,7 +462,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     SideStream* ss = side_stream();
     const cudaStream_t side = fork_side(ss, st);
     cudaError_t err = launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, side);
-    if (err == cudaSuccess) err = launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, st);
+    if (err == cudaSuccess)
+      err = launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, at<double>(ws, L.gpart), st);
     if (err == cudaSuccess)
       err = launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st);
     if (err == cudaSuccess) err = launch_scale_columns(evl, evc, H, d, e, wk, st);
@@ -539,7 +540,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
                             nullptr, nullptr, 0, st));
   SPR_TRY(launch_gram_f64(ck, ck, nullptr, nullptr, static_cast<long long>(Ck) * d,
                           static_cast<long long>(Ck) * d, d, Ck, H, d, c.scale * c.scale, 0.0, G,
-                          static_cast<long long>(d) * d, 0, st));
+                          static_cast<long long>(d) * d, 0, at<double>(ws, L.gpart), st));
   // queries: Lloyd passes on logit profiles in the d-space form
   SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
   // queries on the tensor cores for bf16 inputs (exact in one bf16 plane)
@@ -751,26 +752,35 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
     // Grams are formed
     SPR_TRY(launch_probe_residuals(o_sparse, od, probes, H, N, M, d, xr, means, gram,
                                    static_cast<size_t>(H) * 2 * d * d, st));
-    SPR_TRY(launch_gram_f64(xr, xr, means, means, hs, hs, d, M, H, d, 1.0, c.p.lambda, gram,
-                            2LL * d * d, 2LL * d, st));
-    SPR_TRY(launch_gram_f64(xr, xr + static_cast<size_t>(M) * d, means, means + d, hs, hs, d, M, H,
-                            d, 1.0, 0.0, gram + static_cast<size_t>(d) * d, 2LL * d * d, 2LL * d,
-                            st));
     double* bmat = at<double>(ws, L.bmat);
     double* bvec = at<double>(ws, L.bvec);
     double* rtr = at<double>(ws, L.mk);
-    // the ridge solve (reads the Grams) runs beside R^T R and its eigen solve
-    // (they touch other regions); with r > kTriEigMax the Gram region is reused below,
-    // so the two stay in order
+    {
+      // one launch for the three Grams over the probe rows: the centred
+      // X^T X + lambda I and X^T R of the ridge system, and the uncentred R^T R
+      const double* R = xr + static_cast<size_t>(M) * d;
+      GramJobs g = {};
+      g.part = at<double>(ws, L.gpart);
+      g.job[0] = GramJob{xr, xr, means, means, hs, hs, 2LL * d, gram, 2LL * d * d, 1.0, c.p.lambda};
+      g.job[1] = GramJob{xr, R, means, means + d, hs, hs, 2LL * d, gram + static_cast<size_t>(d) * d,
+                         2LL * d * d, 1.0, 0.0};
+      g.job[2] = GramJob{R, R, nullptr, nullptr, hs, hs, 0, rtr, static_cast<long long>(d) * d, 1.0,
+                         0.0};
+      g.njobs = 3;
+      g.ld = d;
+      g.S = M;
+      g.d = d;
+      g.H = H;
+      SPR_TRY(launch_gram_f64(g, st));
+    }
+    // the ridge solve (reads the Grams) runs beside the eigen solve of R^T R
+    // (they touch other regions); with r > kTriEigMax the Gram region is
+    // reused below, so the two stay in order
     // (joined on every path, also after a failed launch)
     std::unique_lock<std::mutex> lk(g_side_mu);
     SideStream* ss = (c.p.r <= kTriEigMax) ? side_stream() : nullptr;
     const cudaStream_t side = fork_side(ss, st);
     cudaError_t err = launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side);
-    if (err == cudaSuccess)
-      err = launch_gram_f64(xr + static_cast<size_t>(M) * d, xr + static_cast<size_t>(M) * d,
-                            nullptr, nullptr, hs, hs, d, M, H, d, 1.0, 0.0, rtr,
-                            static_cast<long long>(d) * d, 0, st);
     double* evl = at<double>(ws, L.eval);
     double* evc = at<double>(ws, L.evec);
     // leading-r right singular vectors of R = top-r eigenvectors of R^T R

@@ -9,7 +9,7 @@
 //      Matrix Computations, sec. 8.3.1), one CTA per matrix held in its
 //      threads' registers;
 //   2. the ne largest eigenvalues of T by multisection on Sturm-sequence
-//      counts (sec. 8.4.1): 16 or 32 threads per eigenvalue, one point each;
+//      counts (sec. 8.4.1): 8 to 32 threads per eigenvalue, one point each;
 //   3. their eigenvectors by inverse iteration on T - lambda I with one
 //      partial-pivoting tridiagonal LU per eigenvalue reused by every step
 //      (sec. 8.2.2 / 7.6.1), and classical Gram-Schmidt applied twice inside
@@ -250,8 +250,8 @@ __device__ void tri_factor(const double* dg, const double* od, double lam, doubl
     }
   }
   if (a[(D - 1) * S] == 0.0) a[(D - 1) * S] = tiny;
-#pragma unroll 1
-  for (int i = 0; i < D; ++i) a[i * S] = 1.0 / a[i * S];
+#pragma unroll 8
+  for (int i = 0; i < D; ++i) a[i * S] = 1.0 / a[i * S];  // independent: unrolled to overlap
 }
 
 // b <- (T - lam I)^-1 b with the factors of tri_factor.
@@ -275,16 +275,29 @@ __device__ void tri_apply(const double* ra, const double* dl, const double* du, 
     b[i] = (b[i] - du[i * S] * b[i + 1] - du2[i * S] * b[i + 2]) * ra[i * S];
 }
 
+// Fixed start vector of inverse iteration: components in [0.5, 1.5) from an
+// integer hash of (index, eigenvalue rank), so that no start vector is
+// orthogonal to an eigenvector by construction and none costs a
+// transcendental per component.
+__device__ __forceinline__ double start_component(int i, int v) {
+  uint32_t x = static_cast<uint32_t>(i) * 0x9E3779B1u ^ (static_cast<uint32_t>(v) + 0x7F4A7C15u) * 0x85EBCA77u;
+  x ^= x >> 15;
+  x *= 0x2C1B3C6Du;
+  x ^= x >> 12;
+  return 0.5 + static_cast<double>(x) * (1.0 / 4294967296.0);
+}
+
 constexpr int kEigThreads = 512;
 constexpr int kEigWarps = kEigThreads / 32;
 constexpr int kEigMax = kTriEigMax;  // eigenpairs per matrix
 constexpr int kInvBatch = 32;  // eigenvalues in inverse iteration at a time
 
 // One CTA of 512 threads per matrix, ne <= 64 eigenpairs (largest first):
-// multisection by 8-32 threads per eigenvalue, inverse iteration by thread t
-// (one LU, three solves) for batches of 32 eigenvalues, Gram-Schmidt inside
-// clusters by all warps, then the back-transformation with warp w owning
-// vectors w, w + 16, ... Writes evals [H, ne] and evecs [H, D, ne].
+// multisection by 8-32 threads per eigenvalue (one point each), inverse
+// iteration by thread t (one LU, three solves) for batches of 32 eigenvalues,
+// Gram-Schmidt inside clusters by all warps, then the back-transformation
+// with warp w owning vectors w, w + 16, ... Writes evals [H, ne] and evecs
+// [H, D, ne].
 // Dynamic shared memory: the inverse-iteration work arrays of one batch (32
 // threads interleaved; later the staged Householder vectors), then the
 // vectors Y [kEigMax][D + 1].
@@ -302,7 +315,7 @@ static_assert(eig_work_bytes<128>() >= (128 * 128 + 128) * 8 &&
 static_assert(eig_smem_bytes<128>() <= 232448 - 4096, "shared memory");
 
 template <int D>
-__global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scratch, int ne,
+__global__ void __launch_bounds__(kEigThreads, 1) tri_eig_kernel(const double* scratch, int ne,
                                                        double* evals, double* evecs) {
   extern __shared__ double eig_work[];  // inverse-iteration work arrays, then Y
   double (*Y)[D + 1] = reinterpret_cast<double (*)[D + 1]>(eig_work + eig_work_bytes<D>() / 8);
@@ -333,7 +346,8 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
   // multisection: tpe threads per wanted eigenvalue (rank e_i = tid / tpe,
   // ascending index D-1-e_i; tpe = 32, 16 or 8 for ne <= 16, 32 or 64) each
   // evaluate the Sturm count at one interior point of the current interval,
-  // which shrinks (tpe + 1)-fold per round
+  // which shrinks (tpe + 1)-fold per round (the recurrences are bound by the
+  // fp64 pipe, so more points per thread only add work)
   {
     const int tpe = ne <= kEigThreads / 32 ? 32 : (ne <= kEigThreads / 16 ? 16 : 8);
     const int e_i = tid / tpe, q = tid % tpe;
@@ -376,8 +390,8 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
     const int nb = min(kInvBatch, ne - b0);
     const int vi = b0 + tid;  // this thread's eigenvalue (tid < nb)
     if (tid < nb) {
-#pragma unroll 1
-      for (int i = 0; i < D; ++i) Y[vi][i] = 1.0 + 0.5 * sin(0.7 * (i + 1) * (vi + 1));
+#pragma unroll 4
+      for (int i = 0; i < D; ++i) Y[vi][i] = start_component(i, vi);
       tri_factor<D, kInvBatch>(dg, od, lam[vi], tiny, wa, wdl, wdu, wdu2, pv);
     }
     for (int it = 0; it < kInvIters; ++it) {
@@ -425,44 +439,58 @@ __global__ void __launch_bounds__(kEigThreads) tri_eig_kernel(const double* scra
     __syncthreads();  // the work arrays are reused by the next batch
   }
   // back-transformation: u = H_0 (H_1 (... H_{D-3} y)); the Householder
-  // vectors and tau are first staged in the (now free) work space
+  // vectors (row k holds v_k, zero at columns <= k) and tau are first staged
+  // in the (now free) work space
   double* hs = eig_work;          // [D][D]
   double* ts = eig_work + D * D;  // [D]
   for (int i = tid; i < D * D; i += blockDim.x) hs[i] = hv[i];
   for (int i = tid; i < D; i += blockDim.x) ts[i] = tau[i];
   __syncthreads();
-  // warp w owns vectors w, w + 16, w + 32, w + 48 and applies each
-  // reflection to all of them at once
+  // warp w owns vectors w, w + 16, w + 32, w + 48, held in registers (lane l:
+  // components l, l + 32, ..), and applies each reflection to all of them at
+  // once; the warps run independently
   constexpr int kVpw = kEigMax / kEigWarps;
+  constexpr int kCpl = D / 32;
   const int nv = ne > wid ? (ne - wid + kEigWarps - 1) / kEigWarps : 0;
+  double y[kVpw][kCpl];
+#pragma unroll
+  for (int v = 0; v < kVpw; ++v)
+#pragma unroll
+    for (int j = 0; j < kCpl; ++j) y[v][j] = (v < nv) ? Y[wid + kEigWarps * v][lane + 32 * j] : 0.0;
   for (int k = D - 3; k >= 0; --k) {
     const double tk = ts[k];
     if (tk == 0.0) continue;
     const double* hk = hs + k * D;
+    double hj[kCpl];
+#pragma unroll
+    for (int j = 0; j < kCpl; ++j) hj[j] = hk[lane + 32 * j];
     double dot[kVpw];
 #pragma unroll
-    for (int v = 0; v < kVpw; ++v) dot[v] = 0.0;
-    for (int i = k + 1 + lane; i < D; i += 32) {
-      const double hi = hk[i];
+    for (int v = 0; v < kVpw; ++v) {
+      dot[v] = 0.0;
 #pragma unroll
-      for (int v = 0; v < kVpw; ++v)
-        if (v < nv) dot[v] = fma(hi, Y[wid + kEigWarps * v][i], dot[v]);
+      for (int j = 0; j < kCpl; ++j) dot[v] = fma(hj[j], y[v][j], dot[v]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
       for (int v = 0; v < kVpw; ++v) dot[v] += __shfl_xor_sync(0xffffffffu, dot[v], o);
-    for (int i = k + 1 + lane; i < D; i += 32) {
-      const double hi = hk[i];
 #pragma unroll
-      for (int v = 0; v < kVpw; ++v)
-        if (v < nv) Y[wid + kEigWarps * v][i] -= (dot[v] * tk) * hi;
+    for (int v = 0; v < kVpw; ++v) {
+      const double f = dot[v] * tk;
+#pragma unroll
+      for (int j = 0; j < kCpl; ++j) y[v][j] = fma(-f, hj[j], y[v][j]);
     }
-    __syncwarp();
   }
   for (int v = 0; v < nv; ++v) {
     const int t = wid + kEigWarps * v;
-    for (int i = lane; i < D; i += 32) evecs[(static_cast<size_t>(h) * D + i) * ne + t] = Y[t][i];
+#pragma unroll
+    for (int j = 0; j < kCpl; ++j) {
+      double yv = 0.0;
+#pragma unroll
+      for (int u = 0; u < kVpw; ++u) yv = (u == v) ? y[u][j] : yv;
+      evecs[(static_cast<size_t>(h) * D + lane + 32 * j) * ne + t] = yv;
+    }
     if (lane == 0) evals[static_cast<size_t>(h) * ne + t] = lam[t];
   }
 }

@@ -30,16 +30,35 @@ cudaError_t launch_counting_sort(const int32_t* labels, int H, int n, int C, int
 // ---- partition.cu ----------------------------------------------------------
 cudaError_t launch_fy_init(int H, int Nv, int Ck, int Cq, uint64_t seed, int32_t* init_k,
                            int32_t* init_q, cudaStream_t st);
-// out[h] = factor * sum_s x_s x_s^T over the Ms strided sampled query rows.
+// Gram matrices in fp64. A Gram over S rows is split into up to kGramSplits
+// ranges of rows (CTAs of their own); their partial sums go to `part`
+// ([kGramJobs, H, kGramSplits, d, d] fp64 scratch) and a second kernel adds
+// them in range order, so results do not depend on scheduling.
+// out[h] = (1 / Ms) * sum_s x_s x_s^T over the Ms strided sampled query rows.
 cudaError_t launch_metric_mk(const void* q, bool bf16, int H, int N, int Nv, int d, int Ms,
-                             double* out, cudaStream_t st);
+                             double* out, double* part, cudaStream_t st);
 // out[h] = factor * sum_s (x_s - xm)(y_s - ym)^T + diag * I over S fp64 rows;
 // xm / ym (may be null) advance by mean_stride per head.
+struct GramJob {
+  const double *X, *Y, *xm, *ym;
+  long long hsx, hsy, ms;  // per-head strides of X, Y and the means
+  double* out;
+  long long os;            // per-head stride of out
+  double factor, diag;
+};
+// Up to kGramJobs Grams over the same S rows (row stride ld) in one launch.
+struct GramJobs {
+  GramJob job[kGramJobs];
+  int njobs, ld, S, d, H;
+  double* part;  // partial sums (set by the caller)
+  int splits;    // set by the launcher
+};
+cudaError_t launch_gram_f64(GramJobs g, cudaStream_t st);
 cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
                             const double* ym, long long head_stride_x, long long head_stride_y,
                             int ld, int S, int H, int d, double factor, double diag,
                             double* out, long long out_stride, long long mean_stride,
-                            cudaStream_t st);
+                            double* part, cudaStream_t st);
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
                          const double* wk, double* z, cudaStream_t st);
 // dst[h, c, :] = src[h, idx[h, c], :] (as fp64) and norms[h, c] = |dst|^2 (norms may be null)

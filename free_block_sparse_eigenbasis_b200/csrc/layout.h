@@ -19,8 +19,10 @@ constexpr int kSortChunk = 1024;  // tokens per counting-sort chunk
 constexpr int kMaxGroups = 4096;
 constexpr int kMaxSplits = 8;   // split-KV ranges of the dense probe pass
 constexpr size_t kMaxDynSmem = 232448;  // dynamic shared memory per block on sm_100
-constexpr int kDiagRows = 64;
-constexpr int kTriEigMax = 64;  // eigenpairs of the tridiagonal solver (more: cyclic Jacobi)   // density-profile rows processed at once (one CTA each)
+constexpr int kDiagRows = 64;   // density-profile rows processed at once (one CTA each)
+constexpr int kTriEigMax = 64;  // eigenpairs of the tridiagonal solver (more: cyclic Jacobi)
+constexpr int kGramJobs = 3;    // Grams of one launch (the probe fit forms three)
+constexpr int kGramSplits = 4;  // sample ranges of a Gram, summed in order afterwards
 
 struct Layout {
   // statistics / status (always at offset 0)
@@ -78,6 +80,7 @@ struct Layout {
   size_t xr;       // [H, 2, M, d] f64: X = O_sparse[probes], R = O_dense - X
   size_t means;    // [H, 2, d] f64: xbar, rbar
   size_t gram;     // [H, 2, d, d] f64: Xc^T Xc + lam I, Xc^T Rc
+  size_t gpart;    // [kGramJobs, H, kGramSplits, d, d] f64: partial Gram sums
   size_t bmat;     // [H, d, d] f64 ridge solution B
   size_t bvec;     // [H, d] f64 intercept b
   size_t bp32;     // [H, d, d] f32 projected B'
@@ -211,6 +214,7 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->xr = take(H * 2 * (M + 1) * d * 8);
   L->means = take(H * 2 * d * 8);
   L->gram = take(H * 2 * d * d * 8);
+  L->gpart = take(static_cast<size_t>(kGramJobs) * kGramSplits * H * d * d * 8);
   L->bmat = take(H * d * d * 8);
   L->bvec = take(H * d * 8);
   L->bp32 = take(H * d * d * 4);

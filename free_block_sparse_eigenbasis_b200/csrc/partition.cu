@@ -118,42 +118,97 @@ __global__ void __launch_bounds__(kZRowThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Gram kernels: out = factor * sum_s x_s y_s^T (+ diag I), 32x32 output tile
-// per CTA, rows s summed in ascending order.
+// Gram kernels: out = factor * sum_s x_s y_s^T (+ diag I), on the fp64 tensor
+// cores (mma.sync m8n8k4, fp64 products and sums). A CTA of 4 warps forms a
+// 32x32 output tile over one range of the rows s (ascending), each warp a
+// 16x16 quarter (2x2 accumulators of 8x8); the rows stream through shared
+// memory 32 at a time, the next chunk's loads issued before the current
+// chunk's MMAs. With several ranges per Gram (more CTAs, so more loads in
+// flight) each range writes its partial sums and gram_reduce_kernel adds the
+// ranges in order.
 // ---------------------------------------------------------------------------
-constexpr int kGT = 32;
+constexpr int kGT = 32;   // output tile edge
+constexpr int kGS = 32;   // samples per chunk
+constexpr int kGPad = 40; // shared row stride (doubles): fragment loads take two wavefronts
+constexpr int kGThreads = 128;
+constexpr int kGLoads = kGS * kGT / kGThreads;  // elements of x (and of y) per thread per chunk
+
+__device__ __forceinline__ void mma_f64_8x8x4(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
 
 template <typename Loader>
-__device__ void gram_tile(Loader ld, int S, int d, double factor, double diag, double* out) {
-  __shared__ double xs[kGT][kGT + 1];
-  __shared__ double ys[kGT][kGT + 1];
-  __shared__ long long rows[kGT];  // source rows of the chunk's samples
+__device__ void gram_tile(Loader ld, int s_beg, int S, int d, double factor, double diag,
+                          double* out) {
+  __shared__ double xs[kGS][kGPad];
+  __shared__ double ys[kGS][kGPad];
+  __shared__ long long rows[2][kGS];  // source rows of a chunk's samples, two chunks
   const int a0 = blockIdx.x * kGT, b0 = blockIdx.y * kGT;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 256 threads: ty 0..7
-  double acc[4] = {0, 0, 0, 0};
-  for (int s0 = 0; s0 < S; s0 += kGT) {
-    if (threadIdx.x < kGT) rows[threadIdx.x] = ld.row(s0 + threadIdx.x);
-    __syncthreads();
-    for (int t = threadIdx.x; t < kGT * kGT; t += blockDim.x) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wa = (warp >> 1) * 16, wb = (warp & 1) * 16;  // this warp's quarter
+  // fragments: A (8x4, row) a[r = lane / 4][k = lane % 4] = x_{s+k}[row r];
+  // B (4x8, col) b[k = lane % 4][n = lane / 4] = y_{s+k}[col n];
+  // C (8x8) c[r = lane / 4][n = 2 (lane % 4) + {0, 1}]
+  const int fr = lane >> 2, fk = lane & 3;
+  double acc[2][2][2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+  // element e of this thread's share of a chunk: sample ss = t / kGT, column cc = t % kGT
+  double px[kGLoads], py[kGLoads];
+  auto fetch = [&](int s0, const long long* rw) {
+#pragma unroll
+    for (int e = 0; e < kGLoads; ++e) {
+      const int t = threadIdx.x + e * kGThreads;
       const int ss = t / kGT, cc = t % kGT;
-      const int s = s0 + ss;
-      xs[ss][cc] = (s < S && a0 + cc < d) ? ld.x(rows[ss], a0 + cc) : 0.0;
-      ys[ss][cc] = (s < S && b0 + cc < d) ? ld.y(rows[ss], b0 + cc) : 0.0;
+      const bool in = s0 + ss < S;
+      px[e] = (in && a0 + cc < d) ? ld.x(rw[ss], a0 + cc) : 0.0;
+      py[e] = (in && b0 + cc < d) ? ld.y(rw[ss], b0 + cc) : 0.0;
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int ss = 0; ss < kGT; ++ss) {
-      const double yv = ys[ss][tx];
+  };
+  if (threadIdx.x < kGS && s_beg + static_cast<int>(threadIdx.x) < S)
+    rows[0][threadIdx.x] = ld.row(s_beg + threadIdx.x);
+  __syncthreads();
+  fetch(s_beg, rows[0]);
+  for (int c = 0, s0 = s_beg; s0 < S; ++c, s0 += kGS) {
+    __syncthreads();  // the previous chunk has been read
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fma(xs[ss][ty + 8 * i], yv, acc[i]);
+    for (int e = 0; e < kGLoads; ++e) {
+      const int t = threadIdx.x + e * kGThreads;
+      xs[t / kGT][t % kGT] = px[e];
+      ys[t / kGT][t % kGT] = py[e];
     }
+    const int s1 = s0 + kGS;
+    if (threadIdx.x < kGS && s1 + static_cast<int>(threadIdx.x) < S)
+      rows[(c + 1) & 1][threadIdx.x] = ld.row(s1 + threadIdx.x);
     __syncthreads();
+    if (s1 < S) fetch(s1, rows[(c + 1) & 1]);
+#pragma unroll
+    for (int k0 = 0; k0 < kGS; k0 += 4) {
+      double fa[2], fb[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) fa[i] = xs[k0 + fk][wa + 8 * i + fr];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) fb[j] = ys[k0 + fk][wb + 8 * j + fr];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) mma_f64_8x8x4(acc[i][j], fa[i], fb[j]);
+    }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int a = a0 + ty + 8 * i, b = b0 + tx;
-    if (a < d && b < d) out[static_cast<size_t>(a) * d + b] = factor * acc[i] + (a == b ? diag : 0.0);
-  }
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int a = a0 + wa + 8 * i + fr, b = b0 + wb + 8 * j + 2 * fk + t;
+        if (a < d && b < d)
+          out[static_cast<size_t>(a) * d + b] = factor * acc[i][j][t] + (a == b ? diag : 0.0);
+      }
 }
 
 // x(row, a) / y(row, b): element a (b) of source row `row`; row(s): the
@@ -167,11 +222,24 @@ struct SampledQueryLoader {
   __device__ double y(long long row, int b) const { return x(row, b); }
 };
 
+// range sp of `splits` equal ranges of S rows
+__device__ __forceinline__ void gram_range(int S, int splits, int sp, int* beg, int* end) {
+  *beg = static_cast<int>((static_cast<long long>(S) * sp) / splits);
+  *end = static_cast<int>((static_cast<long long>(S) * (sp + 1)) / splits);
+}
+
 template <typename T>
-__global__ void metric_mk_kernel(const T* q, int N, int Nv, int d, int Ms, double* out) {
-  const int h = blockIdx.z;
+__global__ void __launch_bounds__(kGThreads)
+    metric_mk_kernel(const T* q, int N, int Nv, int d, int Ms, int splits, double* out,
+                     double* part) {
+  const int h = blockIdx.z / splits, sp = blockIdx.z % splits;
   SampledQueryLoader<T> ld{q + static_cast<size_t>(h) * N * d, Nv, Ms, d};
-  gram_tile(ld, Ms, d, 1.0 / Ms, 0.0, out + static_cast<size_t>(h) * d * d);
+  int b, e;
+  gram_range(Ms, splits, sp, &b, &e);
+  if (splits == 1)
+    gram_tile(ld, b, e, d, 1.0 / Ms, 0.0, out + static_cast<size_t>(h) * d * d);
+  else
+    gram_tile(ld, b, e, d, 1.0, 0.0, part + (static_cast<size_t>(h) * splits + sp) * d * d);
 }
 
 struct F64Loader {
@@ -186,14 +254,40 @@ struct F64Loader {
   }
 };
 
-__global__ void gram_f64_kernel(const double* X, const double* Y, const double* xm,
-                                const double* ym, long long hsx, long long hsy, int ld, int S,
-                                int d, double factor, double diag, double* out, long long os,
-                                long long ms) {
-  const int h = blockIdx.z;
-  F64Loader l{X + h * hsx, Y + h * hsy, xm ? xm + h * ms : nullptr, ym ? ym + h * ms : nullptr,
-              ld};
-  gram_tile(l, S, d, factor, diag, out + h * os);
+__global__ void __launch_bounds__(kGThreads) gram_f64_kernel(const __grid_constant__ GramJobs g) {
+  const int jh = blockIdx.z / g.splits, sp = blockIdx.z % g.splits;  // jh = job * H + head
+  const int job = jh / g.H, h = jh % g.H;
+  const GramJob& J = g.job[job];
+  F64Loader l{J.X + h * J.hsx, J.Y + h * J.hsy, J.xm ? J.xm + h * J.ms : nullptr,
+              J.ym ? J.ym + h * J.ms : nullptr, g.ld};
+  int b, e;
+  gram_range(g.S, g.splits, sp, &b, &e);
+  if (g.splits == 1)
+    gram_tile(l, b, e, g.d, J.factor, J.diag, J.out + h * J.os);
+  else
+    gram_tile(l, b, e, g.d, 1.0, 0.0,
+              g.part + (static_cast<size_t>(jh) * g.splits + sp) * g.d * g.d);
+}
+
+// out = factor * (sum of the ranges' partial sums, in range order) + diag I
+__global__ void gram_reduce_kernel(const __grid_constant__ GramJobs g) {
+  const int jh = blockIdx.y, job = jh / g.H, h = jh % g.H;
+  const GramJob& J = g.job[job];
+  const int dd = g.d * g.d;
+  const double* P = g.part + static_cast<size_t>(jh) * g.splits * dd;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < dd; i += gridDim.x * blockDim.x) {
+    double sum = P[i];
+    for (int sp = 1; sp < g.splits; ++sp) sum += P[static_cast<size_t>(sp) * dd + i];
+    const int a = i / g.d, b = i % g.d;
+    J.out[h * J.os + i] = J.factor * sum + (a == b ? J.diag : 0.0);
+  }
+}
+
+// ranges per Gram: about 256 rows each, at most kGramSplits
+int gram_splits(int S) {
+  int sp = S / 256;
+  if (sp > kGramSplits) sp = kGramSplits;
+  return sp < 1 ? 1 : sp;
 }
 
 // ---------------------------------------------------------------------------
@@ -921,23 +1015,52 @@ cudaError_t launch_fy_init(int H, int Nv, int Ck, int Cq, uint64_t seed, int32_t
 }
 
 cudaError_t launch_metric_mk(const void* q, bool bf16, int H, int N, int Nv, int d, int Ms,
-                             double* out, cudaStream_t st) {
-  dim3 grid((d + kGT - 1) / kGT, (d + kGT - 1) / kGT, H);
+                             double* out, double* part, cudaStream_t st) {
+  const int splits = gram_splits(Ms);
+  dim3 grid((d + kGT - 1) / kGT, (d + kGT - 1) / kGT, H * splits);
   if (bf16)
-    metric_mk_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q), N, Nv, d, Ms, out);
+    metric_mk_kernel<<<grid, kGThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(q), N, Nv, d,
+                                                 Ms, splits, out, part);
   else
-    metric_mk_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(q), N, Nv, d, Ms, out);
+    metric_mk_kernel<<<grid, kGThreads, 0, st>>>(static_cast<const float*>(q), N, Nv, d, Ms,
+                                                 splits, out, part);
+  if (splits > 1) {
+    GramJobs g = {};
+    g.job[0] = GramJob{nullptr, nullptr, nullptr, nullptr, 0, 0, 0, out,
+                       static_cast<long long>(d) * d, 1.0 / Ms, 0.0};
+    g.njobs = 1;
+    g.d = d;
+    g.H = H;
+    g.part = part;
+    g.splits = splits;
+    gram_reduce_kernel<<<dim3((d * d + 255) / 256, H), 256, 0, st>>>(g);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gram_f64(GramJobs g, cudaStream_t st) {
+  if (g.njobs < 1 || g.njobs > kGramJobs) return cudaErrorInvalidValue;
+  g.splits = gram_splits(g.S);
+  dim3 grid((g.d + kGT - 1) / kGT, (g.d + kGT - 1) / kGT, g.H * g.njobs * g.splits);
+  gram_f64_kernel<<<grid, kGThreads, 0, st>>>(g);
+  if (g.splits > 1)
+    gram_reduce_kernel<<<dim3((g.d * g.d + 255) / 256, g.H * g.njobs), 256, 0, st>>>(g);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
                             const double* ym, long long hsx, long long hsy, int ld, int S, int H,
                             int d, double factor, double diag, double* out, long long os,
-                            long long ms, cudaStream_t st) {
-  dim3 grid((d + kGT - 1) / kGT, (d + kGT - 1) / kGT, H);
-  gram_f64_kernel<<<grid, 256, 0, st>>>(X, Y, xm, ym, hsx, hsy, ld, S, d, factor, diag, out, os,
-                                        ms);
-  return cudaGetLastError();
+                            long long ms, double* part, cudaStream_t st) {
+  GramJobs g = {};
+  g.job[0] = GramJob{X, Y, xm, ym, hsx, hsy, ms, out, os, factor, diag};
+  g.njobs = 1;
+  g.ld = ld;
+  g.S = S;
+  g.d = d;
+  g.H = H;
+  g.part = part;
+  return launch_gram_f64(g, st);
 }
 
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
