@@ -40,8 +40,9 @@ constexpr int kInvIters = 3;
 //      fixed order, identical in every thread);
 //   3. every thread updates its entries, A -= v w^T + w v^T with
 //      w = p - (tau / 2)(v^T p) v (Golub & Van Loan, sec. 8.3.1).
-// Rows and 32-column slots at or above k hold only zeros of v and w and are
-// skipped. Two barriers per column.
+// Every thread updates all its entries without branches (v and w are zero
+// at indices <= k, which leaves those entries unchanged): a skip test per
+// entry costs more than the two FMAs it saves. Two barriers per column.
 constexpr int kTriWarps = kTriThreads / 32;
 
 template <int D>
@@ -114,16 +115,15 @@ __global__ void __launch_bounds__(kTriThreads, 1)
 #pragma unroll
     for (int c = 0; c < kCpl; ++c) vc[c] = vv[lane + 32 * c];
     {
+      // every entry, without branches: v is zero at indices <= k, and the
+      // rows <= k are masked below
       double t[kRpw];
 #pragma unroll
-      for (int r = 0; r < kRpw; ++r) {
-        t[r] = 0.0;
-        if (wid + kTriWarps * r > k) {
+      for (int r = 0; r < kRpw; ++r) t[r] = 0.0;
 #pragma unroll
-          for (int c = 0; c < kCpl; ++c)
-            if (32 * c + 31 > k) t[r] = fma(a[r][c], vc[c], t[r]);
-        }
-      }
+      for (int c = 0; c < kCpl; ++c)
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) t[r] = fma(a[r][c], vc[c], t[r]);
       // transposed butterfly: halve the rows held per lane at each step
 #pragma unroll
       for (int st = 0; st < kLgR; ++st) {
@@ -157,16 +157,15 @@ __global__ void __launch_bounds__(kTriThreads, 1)
       const int j = lane + 32 * c;
       wc[c] = (j > k) ? fma(-hc, vc[c], pb[j]) : 0.0;
     }
+    // every entry, without branches: v and w are zero at indices <= k, so
+    // those entries are left unchanged
 #pragma unroll
     for (int r = 0; r < kRpw; ++r) {
       const int i = wid + kTriWarps * r;
-      if (i > k) {
-        const double vr = vv[i];
-        const double wr = fma(-hc, vr, pb[i]);
+      const double vr = vv[i];
+      const double wr = (i > k) ? fma(-hc, vr, pb[i]) : 0.0;
 #pragma unroll
-        for (int c = 0; c < kCpl; ++c)
-          if (32 * c + 31 > k) a[r][c] -= fma(vr, wc[c], wr * vc[c]);
-      }
+      for (int c = 0; c < kCpl; ++c) a[r][c] = fma(-wr, vc[c], fma(-vr, wc[c], a[r][c]));
     }
   }
 #pragma unroll

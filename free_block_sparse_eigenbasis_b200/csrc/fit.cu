@@ -197,15 +197,13 @@ __global__ void __launch_bounds__(kRidgeThreads, 1)
     double lc[kCpl];
 #pragma unroll
     for (int c = 0; c < kCpl; ++c) lc[c] = lrow[lane + 32 * c];
+    // every entry, without branches: l_ij is zero for i < j and l_kj for
+    // k < j; row j and column j are not read again by the factorisation
 #pragma unroll
     for (int r = 0; r < kRpw; ++r) {
-      const int i = wid + kRidgeWarps * r;
-      if (i > j) {
-        const double li = lrow[i];
+      const double li = lrow[wid + kRidgeWarps * r];
 #pragma unroll
-        for (int c = 0; c < kCpl; ++c)
-          if (32 * c + 31 > j) m[r][c] = fma(-li, lc[c], m[r][c]);
-      }
+      for (int c = 0; c < kCpl; ++c) m[r][c] = fma(-li, lc[c], m[r][c]);
     }
   }
   // 2. L Y = C (the registers now hold C)
