@@ -7,10 +7,12 @@ r = 32, lambda = 1e-2. Inputs are seeded synthetic Q/K/V of that shape.
                     [--workload NAME] [--no-cpu-baseline]
 
 One step = one whole call (partition, permute, route, block-sparse attention,
-probe-fitted correction) over the 12 heads, inputs resident in HBM. The timed
-steps replay one CUDA graph of the five calls when its replay reproduces a
-direct call bit for bit (else the calls are launched directly); the per-stage
-times come from direct calls with events between the stages. Under
+probe-fitted correction) over the 12 heads, inputs resident in HBM, through
+the library's whole-call entry point sparsepr_attention (the probe fit runs on
+a side stream beside the attention of all rows). The timed steps replay one
+CUDA graph of that call when its replay reproduces a direct call bit for bit
+(else the call is launched directly); the per-stage times come from direct
+launches of the five stage calls with events between them. Under
 torchrun every rank runs its own call on its own GPU (heads are independent;
 no collective on the data path) and the job value is the sum of the ranks'
 executed pairs over the slowest rank's time.
@@ -322,9 +324,10 @@ def time_dense(S, qd, kd, vd, stream, steps=2):
 
 
 def measure_workload(S, w, dev, stream, peak, steps=3, warmup=2, qkv=None, with_dense=True):
-    """One workload's call on this GPU (direct launches): whole-call and
-    per-stage ms, executed-pair density, the attention kernel's TFLOP/s and
-    roofline fraction, the dense run of the same kernel, workspace bytes."""
+    """One workload's call on this GPU (direct launches): whole-call ms
+    (sparsepr_attention), the five stage calls' ms and per-stage ms,
+    executed-pair density, the attention kernel's TFLOP/s and roofline
+    fraction, the dense run of the same kernel, workspace bytes."""
     p = w.params()
     if qkv is None:
         q, k, v = synth.generate(w)
@@ -333,15 +336,23 @@ def measure_workload(S, w, dev, stream, peak, steps=3, warmup=2, qkv=None, with_
     b = S.allocate(p, qd.dtype, dev)
     for _ in range(warmup):
         S.attention(qd, kd, vd, p, b, stream)
+        S.sparsepr_attention(qd, kd, vd, p, b, stream)
     torch.cuda.synchronize()
     st = S.sparsepr_read_stats(b.ws)
-    ms, stage = time_calls(S, p, b, qd, kd, vd, stream, steps)
+    five_ms, stage = time_calls(S, p, b, qd, kd, vd, stream, steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        S.sparsepr_attention(qd, kd, vd, p, b, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
     pairs_sparse = int(b.pairs_sparse.sum())
     pairs_exec = int(b.pairs_exec.sum())
     attn = 4.0 * w.d * pairs_sparse / (stage["block_sparse_attn"] * 1e-3) / 1e12
-    r = dict(workload=workload_desc(w), heads_in_one_call=w.H, call_ms=ms, stage_ms=stage,
-             stage_share={n: stage[n] / ms for n in stage},
-             partition_probe_share=(stage["partition"] + stage["probe_correct"]) / ms,
+    r = dict(workload=workload_desc(w), heads_in_one_call=w.H, call_ms=ms, five_calls_ms=five_ms,
+             stage_ms=stage, stage_share={n: stage[n] / five_ms for n in stage},
+             partition_probe_share=(stage["partition"] + stage["probe_correct"]) / five_ms,
              rho_exec=pairs_exec / (w.H * w.N * w.N), value_tflops=4.0 * w.d * pairs_exec / (ms * 1e-3) / 1e12,
              attn_kernel_tflops=attn, attn_roofline_frac=attn / peak,
              kmeans_passes=dict(key=st["key_passes"][:w.H], query=st["query_passes"][:w.H]),
@@ -514,17 +525,23 @@ def main():
                                  sx)
         if ev: ev[5].record(sx)
 
+    def fused(qx, kx, vx, strm=None):
+        S.sparsepr_attention(qx, kx, vx, p, b, stream if strm is None else strm)
+
     def capture_graph():
-        """The five calls captured once into a CUDA graph (the same kernels on the same
-        buffers; the library never synchronises or allocates inside a call). Used for the
-        timed steps only if its replay reproduces the direct call's output bit for bit."""
+        """The whole call captured once into a CUDA graph (the same kernels on the same
+        buffers; the library never synchronises or allocates inside a call, and its side
+        streams fork from and join the captured stream). Used for the timed steps only if
+        its replay reproduces the direct call's output bit for bit."""
         try:
+            fused(qd, kd, vd)
+            torch.cuda.synchronize(dev)
             ref_out, ref_lab = b.out.clone(), b.label_q.clone()
             g = torch.cuda.CUDAGraph()
             cs = torch.cuda.Stream(dev)
             cs.wait_stream(stream)
             with torch.cuda.graph(g, stream=cs, capture_error_mode="relaxed"):
-                call(qd, kd, vd, strm=torch.cuda.current_stream(dev))
+                fused(qd, kd, vd, strm=torch.cuda.current_stream(dev))
             torch.cuda.synchronize(dev)
             b.out.zero_()
             g.replay()
@@ -543,6 +560,7 @@ def main():
 
     for _ in range(args.warmup):
         call(qd, kd, vd)
+        fused(qd, kd, vd)
     torch.cuda.synchronize(dev)
     st = S.sparsepr_read_stats(b.ws)
     pairs_sparse = int(b.pairs_sparse.sum())
@@ -564,24 +582,29 @@ def main():
         if graph is not None:
             graph.replay()
         else:
-            call(qd, kd, vd, evs[s])
+            fused(qd, kd, vd)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop()
     total_ms = t0.elapsed_time(t1)
     ms = total_ms / args.steps
-    # per-stage times (and the whole call) from direct calls with events between the stages
-    direct_ms = ms
+    # the whole call launched directly, then the five stage calls with events
+    # between the stages (per-stage times)
     barrier()  # (the same collective steps on every rank, graph or not)
     torch.cuda.synchronize(dev)
-    if graph is not None:
-        t0.record(stream)
-        for s in range(args.steps):
-            call(qd, kd, vd, evs[s])
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
-        direct_ms = t0.elapsed_time(t1) / args.steps
+    t0.record(stream)
+    for s in range(args.steps):
+        fused(qd, kd, vd)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    direct_ms = t0.elapsed_time(t1) / args.steps
+    t0.record(stream)
+    for s in range(args.steps):
+        call(qd, kd, vd, evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    five_ms = t0.elapsed_time(t1) / args.steps
     barrier()
     stage_names = ["partition", "permute", "route", "block_sparse_attn", "probe_correct"]
     stage_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
@@ -612,7 +635,7 @@ def main():
         qx.copy_(qh, non_blocking=True)
         kx.copy_(kh, non_blocking=True)
         vx.copy_(vh, non_blocking=True)
-        call(qx, kx, vx)
+        fused(qx, kx, vx)
         out_h.copy_(b.out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -620,17 +643,17 @@ def main():
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     # kernels per call, counted on one extra (untimed) call
-    launches = count_launches(lambda: call(qd, kd, vd))
+    launches = count_launches(lambda: fused(qd, kd, vd))
     launches_src = "profiler count of one call"
     if launches <= 0:
         launches, launches_src = gpu_launches_per_call(w), "launch-sequence formula"
 
     # max over ranks
-    vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms, direct_ms],
+    vals = torch.tensor([ms, e2e_ms, stage_ms["block_sparse_attn"], dense_ms, direct_ms, five_ms],
                         device=dev, dtype=torch.float64)
     tot_pairs = torch.tensor([pairs_exec, pairs_sparse], device=dev, dtype=torch.float64)
     reduce_over_ranks(dist if world > 1 else None, vals, tot_pairs)
-    ms_max, e2e_max, attn_max, dense_max, direct_max = vals.tolist()
+    ms_max, e2e_max, attn_max, dense_max, direct_max, five_max = vals.tolist()
     P_exec_all, P_sparse_all = tot_pairs.tolist()
 
     if rank == 0:
@@ -645,13 +668,16 @@ def main():
             config=dict(workload=workload_desc(w), heads_per_rank=w.H,
                         l2="inputs (697 MB of Q/K/V per call) are larger than the 126 MB L2",
                         parallelism="replicas: each rank runs its own call (dp%d)" % world,
-                        launch=("one CUDA graph of the five calls, replayed per step (its output "
-                                "checked bit-identical to a direct call)") if graph is not None
-                        else "the five calls launched directly (%s)" % graph_note),
+                        launch=("one CUDA graph of sparsepr_attention (the whole call), replayed "
+                                "per step (its output checked bit-identical to a direct call)")
+                        if graph is not None
+                        else "sparsepr_attention launched directly (%s)" % graph_note),
             attn_call_ms=ms_max,
             direct_call_ms=direct_max,
+            five_calls_direct_ms=five_max,
             stage_ms=stage_ms,
-            stage_share={n: stage_ms[n] / direct_ms for n in stage_ms},
+            stage_ms_source="the five stage calls launched directly, events between the stages",
+            stage_share={n: stage_ms[n] / five_ms for n in stage_ms},
             rho_exec=pairs_exec / (w.H * w.N * w.N),
             rho_sparse=pairs_sparse / (w.H * w.N * w.N),
             attn_kernel_tflops=attn_tflops,

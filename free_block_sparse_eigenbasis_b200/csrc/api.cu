@@ -84,26 +84,36 @@ sparsepr_status cuda_status(cudaError_t e) {
 __global__ void set_i32_kernel(int32_t* p, int v) { *p = v; }
 
 
-// A second stream per device for small independent kernels that occupy few
-// SMs (the Fisher-Yates init beside the M_K eigen solve, the ridge solve beside
-// the residual eigen solve). It forks from and joins the caller's stream
-// through events, so a stream capture of the caller's stream follows it. The
-// stream and events are created by the first call on a device (make that call
-// before capturing); `g_side_mu` is held from fork to join so that concurrent
+// Side streams per device for independent work beside the caller's stream:
+// stream 0 for small kernels that occupy few SMs (the Fisher-Yates init
+// beside the M_K eigen solve, the ridge solve beside the residual eigen
+// solve) and, in sparsepr_attention, for the probe rows and the fit beside
+// the attention of all rows; stream 1 for the ridge solve inside that probe
+// branch. They are created with the highest priority, so that their
+// latency-bound kernels take SMs as soon as blocks of the caller's kernels
+// retire. Each forks from and joins its parent stream through events, so a
+// stream capture of the caller's stream follows it. The streams and events
+// are created by the first call on a device (make that call before
+// capturing); `g_side_mu` is held from fork to join so that concurrent
 // callers do not interleave the event records.
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
 };
 std::mutex g_side_mu;
-SideStream g_side[64];
+SideStream g_side[64][2];
 
-SideStream* side_stream() {
+SideStream* side_stream(int which = 0) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  SideStream& ss = g_side[dev];
+  SideStream& ss = g_side[dev][which];
   if (!ss.s) {
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
+    if (cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking, greatest) != cudaSuccess) {
+      ss.s = nullptr;
+      return nullptr;
+    }
     if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
@@ -340,6 +350,241 @@ __global__ void dense_meta_kernel(int32_t* meta, int H, int M, int N) {
   offk[2 * h + 1] = N;
   csr[h] = 0;
   kh[h] = 1;
+}
+
+// bf16 copies of the permuted Q, K, V for the attention kernels (fp32 inputs
+// are rounded into the workspace; bf16 inputs are used in place).
+struct Bf16Qkv {
+  const void *q = nullptr, *k = nullptr, *v = nullptr;
+};
+
+cudaError_t bf16_inputs(const Ctx& c, void* ws, const void* qp, const void* kp, const void* vp,
+                        bool cast_q, Bf16Qkv* t) {
+  t->q = qp;
+  t->k = kp;
+  t->v = vp;
+  if (c.bf16) return cudaSuccess;
+  const size_t n = static_cast<size_t>(c.p.H) * c.p.N * c.p.d;
+  __nv_bfloat16* b = at<__nv_bfloat16>(ws, c.L.bf16_qkv);
+  cudaError_t e = cudaSuccess;
+  if (cast_q) {
+    e = launch_cast_bf16(static_cast<const float*>(qp), b, n, c.st);
+    t->q = b;
+  }
+  if (e == cudaSuccess) e = launch_cast_bf16(static_cast<const float*>(kp), b + n, n, c.st);
+  if (e == cudaSuccess) e = launch_cast_bf16(static_cast<const float*>(vp), b + 2 * n, n, c.st);
+  t->k = b + n;
+  t->v = b + 2 * n;
+  return e;
+}
+
+// The routed attention of every row ([SPR 2.C]).
+AttnArgs main_attn_args(const Ctx& c, void* ws, const Bf16Qkv& t, const int32_t* off_q,
+                        const int32_t* off_k, const int32_t* csr, const int32_t* k_per_head,
+                        float* o_sparse, int64_t* pairs_sparse) {
+  AttnArgs a;
+  a.qp = t.q;
+  a.kp = t.k;
+  a.vp = t.v;
+  a.H = c.p.H;
+  a.N = c.p.N;
+  a.d = c.p.d;
+  a.q_rows = c.p.N;
+  a.Cq = c.L.Cqt;
+  a.Ck = c.L.Ckt;
+  a.text = c.p.n_text > 0 ? 1 : 0;
+  a.off_q = off_q;
+  a.off_k = off_k;
+  a.csr = csr;
+  a.kh = k_per_head;
+  a.kmax = c.L.kmax;
+  a.scale = static_cast<float>(c.scale);
+  a.out = o_sparse;
+  a.work = at<int32_t>(ws, c.L.work);
+  a.nwork = at<int32_t>(ws, c.L.nwork);
+  a.tiles_per_head = c.L.tiles_per_head;
+  a.nslots = at<int32_t>(ws, c.L.nslots);
+  a.runs = at<int2>(ws, c.L.runs);
+  a.nruns = at<int32_t>(ws, c.L.nruns);
+  a.pairs = pairs_sparse;
+  a.stats = c.stats;
+  a.lse = at<float>(ws, c.L.lse_s);
+  return a;
+}
+
+cudaError_t zero_fit(const Ctx& c, void* ws, double* fit, cudaStream_t st) {
+  const size_t H = c.p.H, d = c.p.d;
+  cudaError_t e = cudaMemsetAsync(at<float>(ws, c.L.bp32), 0, H * d * d * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(at<float>(ws, c.L.bv32), 0, H * d * 4, st);
+  if (e == cudaSuccess && fit) e = cudaMemsetAsync(fit, 0, H * (d * d + d) * 8, st);
+  return e;
+}
+
+// The probe rows of [SPR 2.B] (M > 0) on stream st: stratified probe rows and
+// their exact dense outputs over all keys.
+//   o_sparse given: the dense pass covers the probe rows alone (X is read
+//     later from o_sparse at the probe rows);
+//   o_sparse null (dual): one pass also forms X = their sparse outputs (each
+//     row's keys limited to its query group's kept runs, from the routed
+//     pass's metadata), so the fit does not wait for the attention of all rows.
+// qsrc: the permuted queries the probe rows are gathered from (bf16 or, with
+// fp32 inputs, fp32).
+sparsepr_status probe_pass(const Ctx& c, void* ws, const Bf16Qkv& t, const void* qsrc,
+                           const int32_t* off_q, int32_t* probes, bool dual, cudaStream_t st) {
+  const Layout& L = c.L;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, M = c.p.M, Cq = c.p.Cq;
+  float* od = at<float>(ws, L.od);
+  int32_t* pgrp = dual ? at<int32_t>(ws, L.pgrp) : nullptr;
+  SPR_TRY(launch_probe_select(off_q, L.Cqt + 1, H, Cq, M, probes, pgrp, st));  // video groups only
+  __nv_bfloat16* pq = at<__nv_bfloat16>(ws, L.probe_q);
+  SPR_TRY(launch_gather_probe_rows(qsrc, c.bf16, probes, H, N, M, d, pq, st));
+  int32_t* meta = at<int32_t>(ws, L.pmeta);
+  dense_meta_kernel<<<(H + 127) / 128, 128, 0, st>>>(meta, H, M, N);
+  SPR_TRY(cudaGetLastError());
+  {
+    AttnArgs a;
+    a.qp = pq;
+    a.kp = t.k;
+    a.vp = t.v;
+    a.H = H;
+    a.N = N;
+    a.d = d;
+    a.q_rows = M;
+    a.Cq = 1;
+    a.Ck = 1;
+    a.off_q = meta;
+    a.off_k = meta + 2 * H;
+    a.csr = meta + 4 * H;
+    a.kh = meta + 5 * H;
+    a.kmax = 1;
+    a.scale = static_cast<float>(c.scale);
+    a.out = od;
+    a.work = at<int32_t>(ws, L.pwork);
+    a.nwork = at<int32_t>(ws, L.pnwork);
+    a.tiles_per_head = M / kTileM + 2;
+    a.nslots = meta + 6 * H;
+    a.nruns = meta + 7 * H;
+    a.runs = reinterpret_cast<int2*>(meta + 8 * H);
+    a.pairs = nullptr;
+    a.stats = c.stats;
+    a.lse = at<float>(ws, L.lse_d);
+    // few units over all N keys: split the key tiles so that about one CTA
+    // per SM runs
+    const int urows = dual ? kTileM : 256;
+    const int units = (M + urows - 1) / urows;
+    const int ktiles = (N + kTileN - 1) / kTileN;
+    int sp = sm_count() / (H * units > 0 ? H * units : 1);
+    if (sp > kMaxSplits) sp = kMaxSplits;
+    if (sp > ktiles) sp = ktiles;
+    if (sp < 1) sp = 1;
+    a.splits = sp;
+    a.units = dual ? M / kTileM + 1 : L.punits;
+    a.opart = at<float>(ws, L.opart);
+    a.lpart = at<float>(ws, L.lpart);
+    if (dual) {
+      a.dual = 1;
+      a.out2 = at<float>(ws, L.xp);
+      a.opart2 = at<float>(ws, L.opart2);
+      a.lpart2 = at<float>(ws, L.lpart2);
+      a.pgrp = pgrp;
+      a.gruns = at<int2>(ws, L.runs);
+      a.gnruns = at<int32_t>(ws, L.nruns);
+      a.gCq = L.Cqt;
+      a.gkmax = L.kmax;
+    }
+    SPR_TRY(launch_block_sparse_attn(a, st));
+  }
+  return SPARSEPR_OK;
+}
+
+// The fit of [SPR 2.B] on stream st after probe_pass: R = O_dense - X (X from
+// o_sparse at the probe rows, or from the dual pass when o_sparse is null),
+// the ridge solution (B, b) and the leading-r subspace of R; writes the
+// projected map (bp32, bv32; `fit` when not null). ridge_ss: the side stream
+// the ridge solve runs on beside the subspace solve (null: in order on st);
+// the caller holds g_side_mu. The side stream is joined on every path.
+sparsepr_status probe_solve(const Ctx& c, void* ws, const int32_t* probes, const float* o_sparse,
+                            double* fit, cudaStream_t st, SideStream* ridge_ss) {
+  const Layout& L = c.L;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, M = c.p.M;
+  const bool dual = (o_sparse == nullptr);
+  const float* od = at<float>(ws, L.od);
+  double* xr = at<double>(ws, L.xr);
+  double* means = at<double>(ws, L.means);
+  double* gram = at<double>(ws, L.gram);
+  const long long hs = 2LL * M * d;
+  // the block sums of the residual pass live in the Gram region until the
+  // Grams are formed
+  SPR_TRY(launch_probe_residuals(o_sparse, dual ? at<float>(ws, L.xp) : nullptr, od, probes, H, N,
+                                 M, d, xr, means, gram, static_cast<size_t>(H) * 2 * d * d, st));
+  double* bmat = at<double>(ws, L.bmat);
+  double* bvec = at<double>(ws, L.bvec);
+  double* rtr = at<double>(ws, L.mk);
+  {
+    // one launch for the three Grams over the probe rows: the centred
+    // X^T X + lambda I and X^T R of the ridge system, and the uncentred R^T R
+    const double* R = xr + static_cast<size_t>(M) * d;
+    GramJobs g = {};
+    g.part = at<double>(ws, L.gpart);
+    g.job[0] = GramJob{xr, xr, means, means, hs, hs, 2LL * d, gram, 2LL * d * d, 1.0, c.p.lambda};
+    g.job[1] = GramJob{xr, R, means, means + d, hs, hs, 2LL * d, gram + static_cast<size_t>(d) * d,
+                       2LL * d * d, 1.0, 0.0};
+    g.job[2] = GramJob{R, R, nullptr, nullptr, hs, hs, 0, rtr, static_cast<long long>(d) * d, 1.0,
+                       0.0};
+    g.njobs = 3;
+    g.ld = d;
+    g.S = M;
+    g.d = d;
+    g.H = H;
+    SPR_TRY(launch_gram_f64(g, st));
+  }
+  // the ridge solve (reads the Grams) runs beside the eigen solve of R^T R
+  // (they touch other regions); with r > kTriEigMax the Gram region is
+  // reused below, so the two stay in order
+  SideStream* ss = (c.p.r <= kTriEigMax) ? ridge_ss : nullptr;
+  const cudaStream_t side = fork_side(ss, st);
+  cudaError_t err = launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side);
+  double* evl = at<double>(ws, L.eval);
+  double* evc = at<double>(ws, L.evec);
+  // leading-r right singular vectors of R = top-r eigenvectors of R^T R
+  const double* vr = evc;
+  if (c.p.r <= kTriEigMax) {
+    if (err == cudaSuccess)
+      err = launch_sym_eigs(rtr, H, d, c.p.r, evl, evc, at<double>(ws, L.eigscr), st);
+  } else {
+    double* sel = gram;  // free after the ridge solve: [H, d, r] selected vectors
+    if (err == cudaSuccess) err = launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st);
+    if (err == cudaSuccess)
+      err = launch_top_eig_projector(evl, evc, H, d, c.p.r, sel, false, st);
+    vr = sel;
+  }
+  const cudaError_t ej = join_side(ss, side, st);
+  SPR_TRY(err);
+  SPR_TRY(ej);
+  SPR_TRY(launch_project_map(bmat, bvec, vr, H, d, c.p.r, at<float>(ws, L.bp32),
+                             at<float>(ws, L.bv32), fit, st));
+  return SPARSEPR_OK;
+}
+
+// The correction of the unprobed rows and the unpermute [SPR 2.B]; the
+// executed-pair counts.
+cudaError_t probe_apply(const Ctx& c, void* ws, const float* o_sparse, const int32_t* probes,
+                        const int32_t* perm_q, const int64_t* pairs_sparse, void* out,
+                        int64_t* pairs_exec, cudaStream_t st) {
+  const Layout& L = c.L;
+  const int H = c.p.H, N = c.p.N, d = c.p.d, M = c.p.M;
+  const float* bp32 = at<float>(ws, L.bp32);
+  const float* bv32 = at<float>(ws, L.bv32);
+  const float* od = at<float>(ws, L.od);
+  cudaError_t e;
+  if (correct_tc_supported(H, N, d))
+    e = launch_correct_tc(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out,
+                          c.bf16, sm_count(), c.stats, st);
+  else
+    e = launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out, c.bf16,
+                       st);
+  if (e != cudaSuccess) return e;
+  return launch_pairs_exec(pairs_sparse, H, static_cast<int64_t>(M) * N, pairs_exec, c.stats, st);
 }
 
 // One thread waits, through the same bounded mbarrier wait as every kernel
@@ -625,46 +870,10 @@ sparsepr_status sparsepr_block_sparse_attn(const void* qp, const void* kp, const
   if (!qp || !kp || !vp || !off_q || !off_k || !csr || !k_per_head || !o_sparse || !pairs_sparse)
     return SPARSEPR_ERR_INVALID_ARG;
   if (!al16(qp, kp, vp, o_sparse)) return SPARSEPR_ERR_INVALID_ARG;
-  const int H = c.p.H, N = c.p.N, d = c.p.d;
-  const size_t n = static_cast<size_t>(H) * N * d;
-  const void *q16 = qp, *k16 = kp, *v16 = vp;
-  if (!c.bf16) {
-    __nv_bfloat16* b = at<__nv_bfloat16>(ws, c.L.bf16_qkv);
-    SPR_TRY(launch_cast_bf16(static_cast<const float*>(qp), b, n, c.st));
-    SPR_TRY(launch_cast_bf16(static_cast<const float*>(kp), b + n, n, c.st));
-    SPR_TRY(launch_cast_bf16(static_cast<const float*>(vp), b + 2 * n, n, c.st));
-    q16 = b;
-    k16 = b + n;
-    v16 = b + 2 * n;
-  }
-  AttnArgs a;
-  a.qp = q16;
-  a.kp = k16;
-  a.vp = v16;
-  a.H = H;
-  a.N = N;
-  a.d = d;
-  a.q_rows = N;
-  a.Cq = c.L.Cqt;
-  a.Ck = c.L.Ckt;
-  a.text = c.p.n_text > 0 ? 1 : 0;
-  a.off_q = off_q;
-  a.off_k = off_k;
-  a.csr = csr;
-  a.kh = k_per_head;
-  a.kmax = c.L.kmax;
-  a.scale = static_cast<float>(c.scale);
-  a.out = o_sparse;
-  a.work = at<int32_t>(ws, c.L.work);
-  a.nwork = at<int32_t>(ws, c.L.nwork);
-  a.tiles_per_head = c.L.tiles_per_head;
-  a.nslots = at<int32_t>(ws, c.L.nslots);
-  a.runs = at<int2>(ws, c.L.runs);
-  a.nruns = at<int32_t>(ws, c.L.nruns);
-  a.pairs = pairs_sparse;
-  a.stats = c.stats;
-  a.lse = at<float>(ws, c.L.lse_s);
-  SPR_TRY(launch_block_sparse_attn(a, c.st));
+  Bf16Qkv t;
+  SPR_TRY(bf16_inputs(c, ws, qp, kp, vp, true, &t));
+  SPR_TRY(launch_block_sparse_attn(
+      main_attn_args(c, ws, t, off_q, off_k, csr, k_per_head, o_sparse, pairs_sparse), c.st));
   return SPARSEPR_OK;
 }
 
@@ -681,137 +890,66 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
       !pairs_exec || (c.p.M > 0 && !probes))
     return SPARSEPR_ERR_INVALID_ARG;
   if (!al16(qp, kp, vp, o_sparse, out)) return SPARSEPR_ERR_INVALID_ARG;
-  const Layout& L = c.L;
-  const int H = c.p.H, N = c.p.N, d = c.p.d, M = c.p.M, Cq = c.p.Cq;
-  cudaStream_t st = c.st;
-  float* bp32 = at<float>(ws, L.bp32);
-  float* bv32 = at<float>(ws, L.bv32);
-  float* od = at<float>(ws, L.od);
-  if (M > 0) {
-    SPR_TRY(launch_probe_select(off_q, L.Cqt + 1, H, Cq, M, probes, st));  // video groups only
-    __nv_bfloat16* pq = at<__nv_bfloat16>(ws, L.probe_q);
-    SPR_TRY(launch_gather_probe_rows(qp, c.bf16, probes, H, N, M, d, pq, st));
-    const void *k16 = kp, *v16 = vp;
-    if (!c.bf16) {
-      const size_t n = static_cast<size_t>(H) * N * d;
-      __nv_bfloat16* b = at<__nv_bfloat16>(ws, L.bf16_qkv);
-      SPR_TRY(launch_cast_bf16(static_cast<const float*>(kp), b + n, n, st));
-      SPR_TRY(launch_cast_bf16(static_cast<const float*>(vp), b + 2 * n, n, st));
-      k16 = b + n;
-      v16 = b + 2 * n;
-    }
-    int32_t* meta = at<int32_t>(ws, L.pmeta);
-    dense_meta_kernel<<<(H + 127) / 128, 128, 0, st>>>(meta, H, M, N);
-    SPR_TRY(cudaGetLastError());
-    AttnArgs a;
-    a.qp = pq;
-    a.kp = k16;
-    a.vp = v16;
-    a.H = H;
-    a.N = N;
-    a.d = d;
-    a.q_rows = M;
-    a.Cq = 1;
-    a.Ck = 1;
-    a.off_q = meta;
-    a.off_k = meta + 2 * H;
-    a.csr = meta + 4 * H;
-    a.kh = meta + 5 * H;
-    a.kmax = 1;
-    a.scale = static_cast<float>(c.scale);
-    a.out = od;
-    a.work = at<int32_t>(ws, L.pwork);
-    a.nwork = at<int32_t>(ws, L.pnwork);
-    a.tiles_per_head = M / kTileM + 2;
-    a.nslots = meta + 6 * H;
-    a.nruns = meta + 7 * H;
-    a.runs = reinterpret_cast<int2*>(meta + 8 * H);
-    a.pairs = nullptr;
-    a.stats = c.stats;
-    a.lse = at<float>(ws, L.lse_d);
-    // few units (H * ceil(M / 256)) over all N keys: split the key tiles so
-    // that about one CTA per SM runs
-    {
-      const int units = H * ((M + 255) / 256);
-      const int ktiles = (N + kTileN - 1) / kTileN;
-      int sp = sm_count() / (units > 0 ? units : 1);
-      if (sp > kMaxSplits) sp = kMaxSplits;
-      if (sp > ktiles) sp = ktiles;
-      if (sp < 1) sp = 1;
-      a.splits = sp;
-      a.units = L.punits;
-      a.opart = at<float>(ws, L.opart);
-      a.lpart = at<float>(ws, L.lpart);
-    }
-    SPR_TRY(launch_block_sparse_attn(a, st));
-    double* xr = at<double>(ws, L.xr);
-    double* means = at<double>(ws, L.means);
-    double* gram = at<double>(ws, L.gram);
-    const long long hs = 2LL * M * d;
-    // the block sums of the residual pass live in the Gram region until the
-    // Grams are formed
-    SPR_TRY(launch_probe_residuals(o_sparse, od, probes, H, N, M, d, xr, means, gram,
-                                   static_cast<size_t>(H) * 2 * d * d, st));
-    double* bmat = at<double>(ws, L.bmat);
-    double* bvec = at<double>(ws, L.bvec);
-    double* rtr = at<double>(ws, L.mk);
-    {
-      // one launch for the three Grams over the probe rows: the centred
-      // X^T X + lambda I and X^T R of the ridge system, and the uncentred R^T R
-      const double* R = xr + static_cast<size_t>(M) * d;
-      GramJobs g = {};
-      g.part = at<double>(ws, L.gpart);
-      g.job[0] = GramJob{xr, xr, means, means, hs, hs, 2LL * d, gram, 2LL * d * d, 1.0, c.p.lambda};
-      g.job[1] = GramJob{xr, R, means, means + d, hs, hs, 2LL * d, gram + static_cast<size_t>(d) * d,
-                         2LL * d * d, 1.0, 0.0};
-      g.job[2] = GramJob{R, R, nullptr, nullptr, hs, hs, 0, rtr, static_cast<long long>(d) * d, 1.0,
-                         0.0};
-      g.njobs = 3;
-      g.ld = d;
-      g.S = M;
-      g.d = d;
-      g.H = H;
-      SPR_TRY(launch_gram_f64(g, st));
-    }
-    // the ridge solve (reads the Grams) runs beside the eigen solve of R^T R
-    // (they touch other regions); with r > kTriEigMax the Gram region is
-    // reused below, so the two stay in order
-    // (joined on every path, also after a failed launch)
-    std::unique_lock<std::mutex> lk(g_side_mu);
-    SideStream* ss = (c.p.r <= kTriEigMax) ? side_stream() : nullptr;
-    const cudaStream_t side = fork_side(ss, st);
-    cudaError_t err = launch_ridge_solve(gram, H, d, bmat, bvec, means, c.stats, side);
-    double* evl = at<double>(ws, L.eval);
-    double* evc = at<double>(ws, L.evec);
-    // leading-r right singular vectors of R = top-r eigenvectors of R^T R
-    const double* vr = evc;
-    if (c.p.r <= kTriEigMax) {
-      if (err == cudaSuccess)
-        err = launch_sym_eigs(rtr, H, d, c.p.r, evl, evc, at<double>(ws, L.eigscr), st);
-    } else {
-      double* sel = gram;  // free after the ridge solve: [H, d, r] selected vectors
-      if (err == cudaSuccess) err = launch_jacobi(rtr, H, d, evl, evc, c.stats, 1, st);
-      if (err == cudaSuccess)
-        err = launch_top_eig_projector(evl, evc, H, d, c.p.r, sel, false, st);
-      vr = sel;
-    }
-    const cudaError_t ej = join_side(ss, side, st);
-    lk.unlock();
-    SPR_TRY(err);
-    SPR_TRY(ej);
-    SPR_TRY(launch_project_map(bmat, bvec, vr, H, d, c.p.r, bp32, bv32, fit, st));
+  if (c.p.M > 0) {
+    Bf16Qkv t;
+    SPR_TRY(bf16_inputs(c, ws, qp, kp, vp, false, &t));
+    sparsepr_status fs = probe_pass(c, ws, t, qp, off_q, probes, false, c.st);
+    if (fs != SPARSEPR_OK) return fs;
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    fs = probe_solve(c, ws, probes, o_sparse, fit, c.st, side_stream(0));
+    if (fs != SPARSEPR_OK) return fs;
   } else {
-    SPR_TRY(cudaMemsetAsync(bp32, 0, static_cast<size_t>(H) * d * d * 4, st));
-    SPR_TRY(cudaMemsetAsync(bv32, 0, static_cast<size_t>(H) * d * 4, st));
-    if (fit) SPR_TRY(cudaMemsetAsync(fit, 0, static_cast<size_t>(H) * (d * d + d) * 8, st));
+    SPR_TRY(zero_fit(c, ws, fit, c.st));
   }
-  if (correct_tc_supported(H, N, d))
-    SPR_TRY(launch_correct_tc(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out, c.bf16,
-                              sm_count(), c.stats, st));
-  else
-    SPR_TRY(launch_correct(o_sparse, od, probes, perm_q, bp32, bv32, H, N, L.Nv, M, d, out, c.bf16,
-                           st));
-  SPR_TRY(launch_pairs_exec(pairs_sparse, H, static_cast<int64_t>(M) * N, pairs_exec, c.stats, st));
+  SPR_TRY(probe_apply(c, ws, o_sparse, probes, perm_q, pairs_sparse, out, pairs_exec, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_attention(const void* q, const void* k, const void* v, sparsepr_dtype dt,
+                                   const sparsepr_params* p, const sparsepr_call_buffers* b,
+                                   void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!b || !out) return SPARSEPR_ERR_INVALID_ARG;
+  sparsepr_status s = sparsepr_partition(q, k, dt, p, b->label_q, b->label_k, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  s = sparsepr_permute(q, k, v, dt, p, b->label_q, b->label_k, b->perm_q, b->perm_k, b->off_q,
+                       b->off_k, b->qp, b->kp, b->vp, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  s = sparsepr_route(b->qp, b->kp, dt, p, b->off_q, b->off_k, b->csr, b->k_per_head, ws, ws_bytes,
+                     stream);
+  if (s != SPARSEPR_OK) return s;
+  Ctx c;
+  s = setup(&c, p, dt, ws, ws_bytes, stream);
+  if (s != SPARSEPR_OK) return s;
+  if (!b->o_sparse || !b->pairs_sparse || !b->pairs_exec || (c.p.M > 0 && !b->probes))
+    return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(b->o_sparse, out)) return SPARSEPR_ERR_INVALID_ARG;
+  Bf16Qkv t;
+  SPR_TRY(bf16_inputs(c, ws, b->qp, b->kp, b->vp, true, &t));
+  const AttnArgs a = main_attn_args(c, ws, t, b->off_q, b->off_k, b->csr, b->k_per_head,
+                                    b->o_sparse, b->pairs_sparse);
+  SPR_TRY(launch_attn_meta(a, c.st));  // the runs the dual probe pass reads
+  if (c.p.M > 0) {
+    // the probe rows' dense and sparse outputs in one pass (work for every
+    // SM, so in order before the attention), then the fit, latency-bound on
+    // few SMs, on a side stream beside the attention of all rows; joined on
+    // every path
+    sparsepr_status fs = probe_pass(c, ws, t, b->qp, b->off_q, b->probes, true, c.st);
+    if (fs != SPARSEPR_OK) return fs;
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStream* ss = side_stream(0);
+    const cudaStream_t side = fork_side(ss, c.st);
+    fs = probe_solve(c, ws, b->probes, nullptr, b->fit, side, side_stream(1));
+    const cudaError_t ea = launch_attn_kernel(a, c.st);
+    const cudaError_t ej = join_side(ss, side, c.st);
+    if (fs != SPARSEPR_OK) return fs;
+    SPR_TRY(ea);
+    SPR_TRY(ej);
+  } else {
+    SPR_TRY(launch_attn_kernel(a, c.st));
+    SPR_TRY(zero_fit(c, ws, b->fit, c.st));
+  }
+  SPR_TRY(probe_apply(c, ws, b->o_sparse, b->probes, b->perm_q, b->pairs_sparse, out,
+                      b->pairs_exec, c.st));
   return SPARSEPR_OK;
 }
 

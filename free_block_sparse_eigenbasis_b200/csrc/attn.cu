@@ -104,6 +104,17 @@ struct AttnParams {
   float* opart;
   float* lpart;
   float* lse;  // [H, q_rows] log2-sum-exp of each row's scaled logits (may be null)
+  int unit_rows;  // query rows per unit: 256 (two tiles), 128 in the dual probe pass
+  // dual probe pass: the second warpgroup takes the same rows and key tiles
+  // with each row's keys limited to the kept runs of its query group
+  float* out2;            // [H, q_rows, d] its outputs (splits == 1)
+  float* opart2;          // its split-KV partial outputs / log2-sum-exps
+  float* lpart2;
+  float* lse2;            // [H, q_rows] (may be null)
+  const int32_t* pgrp;    // [H, q_rows] query group of each row
+  const int2* gruns;      // [H, gCq, gkmax + 1] kept runs of the query groups (ascending)
+  const int32_t* gnruns;  // [H, gCq]
+  int gCq, gkmax;
 };
 
 // Key-column validity of the key tiles of one query group, walked in
@@ -167,7 +178,8 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-template <int HD>
+// DUAL: the dual probe pass (units of one 128-row tile, see AttnParams).
+template <int HD, bool DUAL>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using L = Smem<HD>;
@@ -178,9 +190,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int wcode = p.work[static_cast<size_t>(h) * p.tiles_per_head + wi];
   const int g = wcode >> 16, tu = wcode & 0xFFFF;
   const int32_t* offq = p.off_q + static_cast<size_t>(h) * (p.Cq + 1);
-  const int row0 = offq[g] + tu * kUnitRows;
-  const int rows_unit = min(kUnitRows, offq[g + 1] - row0);
-  const int nq = rows_unit > kTileM ? 2 : 1;  // query tiles in this unit
+  const int row0 = offq[g] + tu * p.unit_rows;
+  const int rows_unit = min(p.unit_rows, offq[g + 1] - row0);
+  const int nq = (!DUAL && rows_unit > kTileM) ? 2 : 1;  // query tiles in this unit
   const size_t gi = static_cast<size_t>(h) * p.Cq + g;
   const int ns = p.nslots[gi];
   const int T_all = (ns + kSlotsPerTile - 1) / kSlotsPerTile;
@@ -190,23 +202,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nr = p.nruns[gi];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool partial = p.splits > 1;
-  const size_t pbase = ((static_cast<size_t>(h) * p.units + wi) * p.splits + split) * kUnitRows;
+  const size_t pbase = ((static_cast<size_t>(h) * p.units + wi) * p.splits + split) * p.unit_rows;
 
   if (T == 0) {
     // empty kept set (reported by the slot-count kernel) or an empty split:
     // rows are zero (partials: zero with log-sum -inf)
     if (static_cast<int>(threadIdx.x) < rows_unit) {
-      float* o = partial ? p.opart + (pbase + threadIdx.x) * HD
-                         : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x) * HD;
-      for (int c = 0; c < HD; c += 4) *reinterpret_cast<float4*>(o + c) = make_float4(0, 0, 0, 0);
-      if (partial) p.lpart[pbase + threadIdx.x] = -INFINITY;
-      else if (p.lse) p.lse[static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x] = -INFINITY;
+      for (int o2 = 0; o2 < (DUAL ? 2 : 1); ++o2) {
+        float* op = o2 ? p.opart2 : p.opart;
+        float* lp = o2 ? p.lpart2 : p.lpart;
+        float* ls = o2 ? p.lse2 : p.lse;
+        float* o = partial ? op + (pbase + threadIdx.x) * HD
+                           : (o2 ? p.out2 : p.out) + (static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x) * HD;
+        for (int c = 0; c < HD; c += 4) *reinterpret_cast<float4*>(o + c) = make_float4(0, 0, 0, 0);
+        if (partial) lp[pbase + threadIdx.x] = -INFINITY;
+        else if (ls) ls[static_cast<size_t>(h) * p.q_rows + row0 + threadIdx.x] = -INFINITY;
+      }
     }
     return;
   }
   // tasks (query tile, key tile) of warpgroup i: two tiles -> (i, t) for every
   // key tile t; one tile -> (0, 2t + i)
-  const bool two = (nq == 2);
+  const bool two = DUAL || (nq == 2);  // both warpgroups take every key tile
   const int ntask[2] = {two ? T : (T + 1) / 2, two ? T : T / 2};
 
   extern __shared__ uint8_t smem_raw[];
@@ -339,7 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int kv = kv_of(i, t), st = kv % kStages;
         if (!mbar_wait(&bars->kfull[st], (kv / kStages) & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t qa = q_addr + (two ? i : 0) * L::kQBytes;
+        const uint32_t qa = q_addr + ((two && !DUAL) ? i : 0) * L::kQBytes;  // dual: one Q tile
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(i * kTileN);
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
@@ -397,6 +414,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     MaskWalk mw;
     mw.init(runs, nr, ns);
     mw.advance_to(j0);
+    // dual pass, warpgroup 1: this row's keys are its query group's kept runs
+    // (key tile j covers keys [128 j, 128 j + 128) in the dense pass)
+    const bool kmask = DUAL && i == 1;
+    const int2* gr = nullptr;
+    int gnr = 0, gri = 0;
+    if (kmask && row < rows_unit) {
+      const size_t gg = static_cast<size_t>(h) * p.gCq + p.pgrp[static_cast<size_t>(h) * p.q_rows + row0 + row];
+      gr = p.gruns + gg * (p.gkmax + 1);
+      gnr = p.gnruns[gg];
+    }
     bool ok = true;
     for (int t = 0; t < ntask[i]; ++t) {
       const int kv = two ? t : 2 * t + i;  // local key tile; global tile j0 + kv
@@ -410,6 +437,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t skip[4];
         mw.tile(j0 + kv + 1, skip);
       }
+      uint32_t km[4] = {0u, 0u, 0u, 0u};  // dual: bit c = key column c is kept for this row
+      if (kmask) {
+        const int k0 = (j0 + kv) * kTileN, k1 = k0 + kTileN;
+        while (gri < gnr && gr[gri].x + gr[gri].y <= k0) ++gri;
+        for (int r2 = gri; r2 < gnr && gr[r2].x < k1; ++r2) {
+          const int a = max(gr[r2].x, k0) - k0, b = min(gr[r2].x + gr[r2].y, k1) - k0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int lo = max(a, 32 * w) - 32 * w, hi = min(b, 32 * w + 32) - 32 * w;
+            if (lo < hi) km[w] |= (hi == 32 ? 0xFFFFFFFFu : ((1u << hi) - 1u)) & ~((1u << lo) - 1u);
+          }
+        }
+      }
       // tcgen05.ld / st below are warp-collective: the warp proceeds or stops as one
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[i], t & 1, abort))) { ok = false; break; }
       tc_fence_after();
@@ -421,6 +461,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32(s_tmem + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
         tmem_ld32(s_tmem + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
         tmem_wait_ld();
+        if (kmask) {
+#pragma unroll
+          for (int c = 0; c < kTileN / 2; ++c)
+            if (!((km[2 * hf + (c >> 5)] >> (c & 31)) & 1u)) r[c] = __float_as_uint(-INFINITY);
+        }
         if ((vm[2 * hf] & vm[2 * hf + 1]) != 0xFFFFFFFFu) {
           // only partial or padding slots (the same for every row) are touched
 #pragma unroll
@@ -450,7 +495,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       auto exp_half = [&](float mref) -> float {
         float2 r4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                         make_float2(0.f, 0.f)};
-        const float nm = -mref;
+        const float nm = (mref == -INFINITY) ? 0.f : -mref;  // no kept key yet: P = 0
 #pragma unroll
         for (int c = 0; c < kTileN / 2; c += 2) {
           float xa, xb;
@@ -469,11 +514,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // it) and its values formed again, and the P half already stored, the
       // row sum and O are scaled by 2^-k, exactly. O and the row sum always
       // share one reference, so the result is exact.
-      if (t == 0) {
+      // (dual, masked rows: the first tile that holds one of the row's keys;
+      // nothing has been accumulated before it)
+      if (t == 0 || (kmask && __any_sync(0xffffffffu, m_ref == -INFINITY))) {
         load_half(0);
         const float m0 = half_max();
         load_half(1);
-        m_ref = fmaxf(m0, half_max());
+        const float mt = fmaxf(m0, half_max());
+        if (m_ref == -INFINITY) m_ref = mt;
       }
       float alpha = 1.f, rs = 0.f;
       bool need = false;
@@ -531,14 +579,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (two) {
       if (__all_sync(0xffffffffu, ok && mbar_wait(&bars->o_done[i], 0, abort))) {
         tc_fence_after();
-        const float inv = 1.f / l_sum;
+        // a row with no kept key in this range (dual pass) gets 0 and -inf
+        const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+        const float lsev = l_sum > 0.f ? m_ref + __log2f(l_sum) : -INFINITY;
         const uint32_t o_tmem = o_base + static_cast<uint32_t>(i * HD);
-        const bool valid = i * kTileM + row < rows_unit;
-        float* orow = partial ? p.opart + (pbase + i * kTileM + row) * HD
-                              : p.out + (static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row) * HD;
-        if (partial && valid) p.lpart[pbase + i * kTileM + row] = m_ref + __log2f(l_sum);
-        if (!partial && valid && p.lse)
-          p.lse[static_cast<size_t>(h) * p.q_rows + row0 + i * kTileM + row] = m_ref + __log2f(l_sum);
+        const int ur = DUAL ? row : i * kTileM + row;  // row within the unit
+        const bool valid = ur < rows_unit;
+        const bool second = DUAL && i == 1;
+        float* orow = partial ? (second ? p.opart2 : p.opart) + (pbase + ur) * HD
+                              : (second ? p.out2 : p.out) + (static_cast<size_t>(h) * p.q_rows + row0 + ur) * HD;
+        if (partial && valid) (second ? p.lpart2 : p.lpart)[pbase + ur] = lsev;
+        float* lsep = second ? p.lse2 : p.lse;
+        if (!partial && valid && lsep) lsep[static_cast<size_t>(h) * p.q_rows + row0 + ur] = lsev;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
@@ -608,11 +660,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Work list: one entry per 256-row unit of each query group, (g << 16) | u.
+// Work list: one entry per unit (256 rows; 128 in the dual probe pass) of
+// each query group, (g << 16) | u.
 // One warp per head: tile counts are prefix-summed 32 groups at a time.
 // ---------------------------------------------------------------------------
-__global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_head, int32_t* work,
-                                 int32_t* nwork) {
+__global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_head, int unit_rows,
+                                 int32_t* work, int32_t* nwork) {
   const int h = blockIdx.x, lane = threadIdx.x;
   const int32_t* oq = off_q + static_cast<size_t>(h) * (Cq + 1);
   int32_t* wl = work + static_cast<size_t>(h) * tiles_per_head;
@@ -620,7 +673,7 @@ __global__ void work_list_kernel(const int32_t* off_q, int Cq, int tiles_per_hea
   for (int g0 = 0; g0 < Cq; g0 += 32) {
     const int g = g0 + lane;
     const int n = (g < Cq) ? oq[g + 1] - oq[g] : 0;
-    const int t = n > 0 ? (n + kUnitRows - 1) / kUnitRows : 0;
+    const int t = n > 0 ? (n + unit_rows - 1) / unit_rows : 0;
     int x = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -760,29 +813,29 @@ __global__ void __launch_bounds__(kSpWarps * 32)
 // unit, thread = (row, 4 columns).
 __global__ void split_combine_kernel(const float* opart, const float* lpart, const int32_t* off_q,
                                      const int32_t* work, const int32_t* nwork, int Cq,
-                                     int tiles_per_head, int units, int splits, int q_rows, int d,
-                                     float* out, float* lse) {
+                                     int tiles_per_head, int units, int splits, int unit_rows,
+                                     int q_rows, int d, float* out, float* lse) {
   const int h = blockIdx.z, wi = blockIdx.y;
   if (wi >= nwork[h]) return;
   const int wcode = work[static_cast<size_t>(h) * tiles_per_head + wi];
   const int g = wcode >> 16, tu = wcode & 0xFFFF;
   const int32_t* offq = off_q + static_cast<size_t>(h) * (Cq + 1);
-  const int row0 = offq[g] + tu * kUnitRows;
-  const int rows = min(kUnitRows, offq[g + 1] - row0);
+  const int row0 = offq[g] + tu * unit_rows;
+  const int rows = min(unit_rows, offq[g + 1] - row0);
   const int cpr = d / 4;  // threads per row
   const int r = blockIdx.x * (blockDim.x / cpr) + threadIdx.x / cpr;
   const int c = (threadIdx.x % cpr) * 4;
   if (r >= rows) return;
   const size_t ub = (static_cast<size_t>(h) * units + wi) * splits;
   float L = -INFINITY;
-  for (int s = 0; s < splits; ++s) L = fmaxf(L, lpart[(ub + s) * kUnitRows + r]);
+  for (int s = 0; s < splits; ++s) L = fmaxf(L, lpart[(ub + s) * unit_rows + r]);
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
   for (int s = 0; s < splits; ++s) {
-    const float ls = lpart[(ub + s) * kUnitRows + r];
+    const float ls = lpart[(ub + s) * unit_rows + r];
     if (ls == -INFINITY) continue;
     const float wgt = exp2f(ls - L);
-    const float4 o = *reinterpret_cast<const float4*>(opart + ((ub + s) * kUnitRows + r) * d + c);
+    const float4 o = *reinterpret_cast<const float4*>(opart + ((ub + s) * unit_rows + r) * d + c);
     num.x = fmaf(wgt, o.x, num.x);
     num.y = fmaf(wgt, o.y, num.y);
     num.z = fmaf(wgt, o.z, num.z);
@@ -835,7 +888,7 @@ bool make_map(CUtensorMap* m, const void* base, size_t rows, int d, int box_rows
   return r == CUDA_SUCCESS;
 }
 
-template <int HD>
+template <int HD, bool DUAL>
 cudaError_t launch_attn_hd(const AttnArgs& a, AttnParams prm, cudaStream_t st) {
   AttnMaps maps;
   const size_t qrows_total = static_cast<size_t>(a.H) * a.q_rows;
@@ -854,28 +907,39 @@ cudaError_t launch_attn_hd(const AttnArgs& a, AttnParams prm, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   const int shb = kAttnSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<HD>,
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<HD, DUAL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, shb);
   if (e != cudaSuccess) return e;
   dim3 grid(a.tiles_per_head * prm.splits, a.H);
-  sparse_attn_kernel<HD><<<grid, kAttnThreads, shb, st>>>(maps, prm);
-  if (prm.splits > 1)
-    split_combine_kernel<<<dim3(kUnitRows / (256 / (HD / 4)), a.units, a.H), 256, 0, st>>>(
-        a.opart, a.lpart, a.off_q, a.work, a.nwork, a.Cq, a.tiles_per_head, a.units, prm.splits,
-        a.q_rows, HD, a.out, a.lse);
+  sparse_attn_kernel<HD, DUAL><<<grid, kAttnThreads, shb, st>>>(maps, prm);
+  if (prm.splits > 1) {
+    const dim3 cg(prm.unit_rows / (256 / (HD / 4)), a.units, a.H);
+    split_combine_kernel<<<cg, 256, 0, st>>>(a.opart, a.lpart, a.off_q, a.work, a.nwork, a.Cq,
+                                             a.tiles_per_head, a.units, prm.splits, prm.unit_rows,
+                                             a.q_rows, HD, a.out, a.lse);
+    if (DUAL)
+      split_combine_kernel<<<cg, 256, 0, st>>>(a.opart2, a.lpart2, a.off_q, a.work, a.nwork, a.Cq,
+                                               a.tiles_per_head, a.units, prm.splits,
+                                               prm.unit_rows, a.q_rows, HD, a.out2, a.lse2);
+  }
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
-  work_list_kernel<<<a.H, 32, 0, st>>>(a.off_q, a.Cq, a.tiles_per_head, a.work, a.nwork);
+cudaError_t launch_attn_meta(const AttnArgs& a, cudaStream_t st) {
+  const int unit_rows = a.dual ? kTileM : kUnitRows;
+  work_list_kernel<<<a.H, 32, 0, st>>>(a.off_q, a.Cq, a.tiles_per_head, unit_rows, a.work, a.nwork);
   if (a.pairs) zero_i64_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H);
   const int n = a.H * a.Cq;
   slots_pairs_kernel<<<(n + kSpWarps - 1) / kSpWarps, kSpWarps * 32, 0, st>>>(
       a.off_q, a.off_k, a.csr, a.kh, a.H, a.N, a.Cq, a.Ck, a.kmax, a.text, a.nslots, a.runs,
       a.nruns, a.pairs, a.stats);
   if (a.pairs) pairs_to_stats_kernel<<<(a.H + 127) / 128, 128, 0, st>>>(a.pairs, a.H, a.stats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_kernel(const AttnArgs& a, cudaStream_t st) {
   AttnParams prm;
   prm.H = a.H;
   prm.N = a.N;
@@ -898,12 +962,31 @@ cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
   prm.opart = a.opart;
   prm.lpart = a.lpart;
   prm.lse = a.lse;
+  prm.unit_rows = a.dual ? kTileM : kUnitRows;
+  prm.out2 = a.out2;
+  prm.opart2 = a.opart2;
+  prm.lpart2 = a.lpart2;
+  prm.lse2 = a.lse2;
+  prm.pgrp = a.pgrp;
+  prm.gruns = a.gruns;
+  prm.gnruns = a.gnruns;
+  prm.gCq = a.gCq;
+  prm.gkmax = a.gkmax;
   if (prm.splits > 1 && (!a.opart || !a.lpart || a.units < 1)) return cudaErrorInvalidValue;
+  if (a.dual && (!a.out2 || !a.pgrp || !a.gruns || !a.gnruns || a.gCq < 1 ||
+                 (prm.splits > 1 && (!a.opart2 || !a.lpart2))))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.d == 128) return launch_attn_hd<128>(a, prm, st);
-  if (a.d == 64) return launch_attn_hd<64>(a, prm, st);
+  if (a.d == 128) return a.dual ? launch_attn_hd<128, true>(a, prm, st) : launch_attn_hd<128, false>(a, prm, st);
+  if (a.d == 64) return a.dual ? launch_attn_hd<64, true>(a, prm, st) : launch_attn_hd<64, false>(a, prm, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st) {
+  const cudaError_t e = launch_attn_meta(a, st);
+  if (e != cudaSuccess) return e;
+  return launch_attn_kernel(a, st);
 }
 
 cudaError_t launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st) {

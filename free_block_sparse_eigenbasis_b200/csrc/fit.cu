@@ -12,7 +12,7 @@ namespace {
 // Probes per query group by largest remainder (ties to the lower group),
 // rows at offsets floor((t + 1/2) n_g / m_g) inside each group.
 __global__ void probe_select_kernel(const int32_t* off_q, int off_stride, int Cq, int M,
-                                    int32_t* probes) {
+                                    int32_t* probes, int32_t* pgrp) {
   extern __shared__ int64_t psm[];
   int64_t* rem = psm;                                  // [Cq]
   int32_t* m = reinterpret_cast<int32_t*>(rem + Cq);   // [Cq]
@@ -54,11 +54,14 @@ __global__ void probe_select_kernel(const int32_t* off_q, int off_stride, int Cq
   }
   __syncthreads();
   int32_t* out = probes + static_cast<size_t>(h) * M;
+  int32_t* grp = pgrp ? pgrp + static_cast<size_t>(h) * M : nullptr;
   for (int g = threadIdx.x; g < Cq; g += blockDim.x) {
     const int64_t n = oq[g + 1] - oq[g];
     const int mg = m[g];
-    for (int t = 0; t < mg; ++t)
+    for (int t = 0; t < mg; ++t) {
       out[start[g] + t] = oq[g] + static_cast<int32_t>(((2LL * t + 1) * n) / (2LL * mg));
+      if (grp) grp[start[g] + t] = g;
+    }
   }
 }
 
@@ -79,13 +82,13 @@ __global__ void gather_probe_rows_kernel(const void* qp, int bf16, const int32_t
   }
 }
 
-// X = O_sparse[probes], R = O_dense - X (fp64), column means xbar, rbar.
-// X = O_sparse[probes], R = O_dense - X (fp64) for a block of probe rows
+// X = O_sparse[probes] (or the probe rows' sparse outputs x_rows [H, M, d]
+// when given), R = O_dense - X (fp64) for a block of probe rows
 // per CTA (thread = column), with the block's column sums of X and R in
 // part [H, nblk, 2, d]; probe_means_kernel adds the blocks in order.
-__global__ void probe_residuals_kernel(const float* o_sparse, const float* od,
-                                       const int32_t* probes, int N, int M, int d, int rows_blk,
-                                       double* xr, double* part) {
+__global__ void probe_residuals_kernel(const float* o_sparse, const float* x_rows,
+                                       const float* od, const int32_t* probes, int N, int M,
+                                       int d, int rows_blk, double* xr, double* part) {
   const int h = blockIdx.y, blk = blockIdx.x, a = threadIdx.x;
   if (a >= d) return;
   double* X = xr + static_cast<size_t>(h) * 2 * M * d;
@@ -94,8 +97,9 @@ __global__ void probe_residuals_kernel(const float* o_sparse, const float* od,
   const int t0 = blk * rows_blk, t1 = min(M, t0 + rows_blk);
 #pragma unroll 4
   for (int t = t0; t < t1; ++t) {
-    const size_t row = static_cast<size_t>(h) * N + probes[static_cast<size_t>(h) * M + t];
-    const double x = o_sparse[row * d + a];
+    const double x =
+        x_rows ? x_rows[(static_cast<size_t>(h) * M + t) * d + a]
+               : o_sparse[(static_cast<size_t>(h) * N + probes[static_cast<size_t>(h) * M + t]) * d + a];
     const double r = static_cast<double>(od[(static_cast<size_t>(h) * M + t) * d + a]) - x;
     X[static_cast<size_t>(t) * d + a] = x;
     R[static_cast<size_t>(t) * d + a] = r;
@@ -407,9 +411,9 @@ __global__ void pairs_exec_kernel(const int64_t* ps, int H, int64_t add, int64_t
 }  // namespace
 
 cudaError_t launch_probe_select(const int32_t* off_q, int off_stride, int H, int Cq, int M,
-                                int32_t* probes, cudaStream_t st) {
+                                int32_t* probes, int32_t* pgrp, cudaStream_t st) {
   const size_t shb = static_cast<size_t>(Cq) * 16;
-  probe_select_kernel<<<H, 256, shb, st>>>(off_q, off_stride, Cq, M, probes);
+  probe_select_kernel<<<H, 256, shb, st>>>(off_q, off_stride, Cq, M, probes, pgrp);
   return cudaGetLastError();
 }
 
@@ -419,9 +423,10 @@ cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* p
   return cudaGetLastError();
 }
 
-cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const int32_t* probes,
-                                   int H, int N, int M, int d, double* xr, double* means,
-                                   double* part, size_t part_doubles, cudaStream_t st) {
+cudaError_t launch_probe_residuals(const float* o_sparse, const float* x_rows, const float* od,
+                                   const int32_t* probes, int H, int N, int M, int d, double* xr,
+                                   double* means, double* part, size_t part_doubles,
+                                   cudaStream_t st) {
   // blocks of >= 16 rows, at most part_doubles / (2 d H) of them
   int nblk = (M + 15) / 16;
   const int cap = static_cast<int>(part_doubles / (2 * static_cast<size_t>(d) * H));
@@ -430,8 +435,8 @@ cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const
   const int rows_blk = (M + nblk - 1) / nblk;
   nblk = (M + rows_blk - 1) / rows_blk;
   if (nblk < 1) nblk = 1;
-  probe_residuals_kernel<<<dim3(nblk, H), d, 0, st>>>(o_sparse, od, probes, N, M, d, rows_blk, xr,
-                                                      part);
+  probe_residuals_kernel<<<dim3(nblk, H), d, 0, st>>>(o_sparse, x_rows, od, probes, N, M, d,
+                                                      rows_blk, xr, part);
   probe_means_kernel<<<H, d, 0, st>>>(part, nblk, M, d, means);
   return cudaGetLastError();
 }

@@ -221,7 +221,26 @@ struct AttnArgs {
   // log2-sum-exp of every row's scaled logits over its kept keys (log2
   // units: m + log2 l), [H, q_rows]; may be null
   float* lse = nullptr;
+  // dual probe pass (dense routes, units of 128 rows): every row is computed
+  // twice over all keys, once densely (out, lse, opart, lpart) and once with
+  // its keys limited to the kept runs of its query group pgrp[h, row] in the
+  // routed pass's run lists gruns [H, gCq, gkmax + 1] / gnruns [H, gCq]
+  // (out2, lse2, opart2, lpart2; partial buffers with 128-row units)
+  int dual = 0;
+  float* out2 = nullptr;
+  float* lse2 = nullptr;
+  float* opart2 = nullptr;
+  float* lpart2 = nullptr;
+  const int32_t* pgrp = nullptr;
+  const int2* gruns = nullptr;
+  const int32_t* gnruns = nullptr;
+  int gCq = 0, gkmax = 0;
 };
+// the work list and the slot / run / pair metadata of a pass
+cudaError_t launch_attn_meta(const AttnArgs& a, cudaStream_t st);
+// the attention kernel (and split-KV combine) over metadata already formed
+cudaError_t launch_attn_kernel(const AttnArgs& a, cudaStream_t st);
+// both, in order
 cudaError_t launch_block_sparse_attn(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t st);
 
@@ -244,14 +263,17 @@ cudaError_t launch_density(const void* q, const void* k, bool bf16, int H, int N
                            unsigned long long* count_sum, double* density, cudaStream_t st);
 
 // ---- fit.cu ----------------------------------------------------------------
+// probes [H, M]; pgrp [H, M] (may be null): the query group of each probe
 cudaError_t launch_probe_select(const int32_t* off_q, int off_stride, int H, int Cq, int M,
-                                int32_t* probes, cudaStream_t st);
+                                int32_t* probes, int32_t* pgrp, cudaStream_t st);
 cudaError_t launch_gather_probe_rows(const void* qp, bool bf16, const int32_t* probes, int H,
                                      int N, int M, int d, __nv_bfloat16* dst, cudaStream_t st);
+// X from o_sparse at the probe rows, or from x_rows [H, M, d] when not null;
 // part: scratch of part_doubles fp64 for per-block column sums.
-cudaError_t launch_probe_residuals(const float* o_sparse, const float* od, const int32_t* probes,
-                                   int H, int N, int M, int d, double* xr, double* means,
-                                   double* part, size_t part_doubles, cudaStream_t st);
+cudaError_t launch_probe_residuals(const float* o_sparse, const float* x_rows, const float* od,
+                                   const int32_t* probes, int H, int N, int M, int d, double* xr,
+                                   double* means, double* part, size_t part_doubles,
+                                   cudaStream_t st);
 cudaError_t launch_ridge_solve(double* gram, int H, int d, double* bmat, double* bvec,
                                const double* means, DeviceStats* stats, cudaStream_t st);
 // B' = (B V_r) V_r^T, b' = (b V_r) V_r^T with vr [H, d, r]; bp32 holds B'^T

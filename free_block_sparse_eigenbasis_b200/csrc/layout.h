@@ -91,6 +91,10 @@ struct Layout {
                    // nruns(1), runs(2 int2: run-list stride kmax + 1 = 2)
   size_t opart;    // [H, punits, kMaxSplits, 256, d] f32 split-KV partial outputs (probes)
   size_t lpart;    // [H, punits, kMaxSplits, 256] f32 split-KV log2-sum-exps
+  size_t opart2;   // [H, punits, kMaxSplits, 256, d] f32: partial sparse outputs of the dual pass
+  size_t lpart2;   // [H, punits, kMaxSplits, 256] f32
+  size_t xp;       // [H, M + 1, d] f32 sparse outputs of the probe rows (dual pass)
+  size_t pgrp;     // [H, M + 1] int32 query group of each probe row
   size_t lse_s;    // [H, N] f32 log2-sum-exp of each row's kept logits (sparse pass, group-major)
   size_t lse_d;    // [H, M + 1] f32 log2-sum-exp of each probe row over all keys (dense pass)
   size_t diag;     // [H, M + 1, 4] f64 per-probe-row residual energies (diagnostics)
@@ -225,6 +229,10 @@ inline void compute_layout(const sparsepr_params& p, Layout* L) {
   L->punits = static_cast<int>(M / 256 + 1);
   L->opart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * d * 4);
   L->lpart = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * 4);
+  L->opart2 = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * d * 4);
+  L->lpart2 = take(H * static_cast<size_t>(L->punits) * kMaxSplits * 256 * 4);
+  L->xp = take(H * (M + 1) * d * 4);
+  L->pgrp = take(H * (M + 1) * 4);
   L->lse_s = take(H * N * 4);
   L->lse_d = take(H * (M + 1) * 4);
   L->diag = take(H * (M + 1) * 4 * 8);

@@ -26,7 +26,7 @@ EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_part
             "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
             "sparsepr_reset_stats", "sparsepr_check_wait_limit", "sparsepr_route_noalloc",
             "sparsepr_workspace_region", "sparsepr_probe_diagnostics",
-            "sparsepr_support_expansion", "sparsepr_density_profile")
+            "sparsepr_support_expansion", "sparsepr_density_profile", "sparsepr_attention")
 
 
 class Params(ctypes.Structure):
@@ -36,6 +36,13 @@ class Params(ctypes.Structure):
                 ("kmeans_iters", ctypes.c_int32), ("M", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("partition", ctypes.c_int32), ("lam", ctypes.c_double), ("scale", ctypes.c_double),
                 ("seed", ctypes.c_uint64), ("keep", ctypes.POINTER(ctypes.c_double))]
+
+
+class CallBuffers(ctypes.Structure):
+    """sparsepr_call_buffers: device pointers of every output of one call."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "label_q", "label_k", "perm_q", "perm_k", "off_q", "off_k", "qp", "kp", "vp", "csr",
+        "k_per_head", "o_sparse", "pairs_sparse", "probes", "pairs_exec", "fit")]
 
 
 class Stats(ctypes.Structure):
@@ -90,6 +97,8 @@ def _load():
     lib.sparsepr_density_profile.argtypes = [P, P, st, PP, ctypes.c_double, ctypes.c_int32, P, V,
                                              sz, V]
     lib.sparsepr_density_profile.restype = st
+    lib.sparsepr_attention.argtypes = [P, P, P, st, PP, ctypes.POINTER(CallBuffers), P, V, sz, V]
+    lib.sparsepr_attention.restype = st
     lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
     lib.sparsepr_reset_stats.argtypes = [V, V]
     lib.sparsepr_check_wait_limit.argtypes = [V, V]
@@ -432,6 +441,38 @@ def attention(q, k, v, p: dict, bufs: Optional[Buffers] = None, stream=None) -> 
                                b.o_sparse, b.pairs_sparse, b.ws, stream)
     sparsepr_probe_correct(b.qp, b.kp, b.vp, p, b.off_q, b.perm_q, b.o_sparse, b.pairs_sparse,
                            b.out, b.probes, b.pairs_exec, b.ws, b.fit, stream)
+    return b
+
+
+def sparsepr_attention(q, k, v, p: dict, bufs: Buffers, stream=None) -> Buffers:
+    """The whole call in one library entry point (sparsepr_attention): the
+    probe fit runs on a side stream beside the attention of all rows. Fills
+    the same buffers as attention(); bufs.out is the output."""
+    prm, keep = make_params(p)
+    H, N, d, oq, ok = _dims(p)
+    (pq, pk, pv), dt = _qkv(p, [("q", q), ("k", k), ("v", v)])
+    b = bufs
+    I32T = torch.int32
+    ptr = lambda t, n, shape, dtype: _arg(t, n, shape, dtype).value  # noqa: E731
+    kmax = route_width(p)
+    M = int(p["M"])
+    cb = CallBuffers(
+        label_q=ptr(b.label_q, "label_q", (H, N), I32T), label_k=ptr(b.label_k, "label_k", (H, N), I32T),
+        perm_q=ptr(b.perm_q, "perm_q", (H, N), I32T), perm_k=ptr(b.perm_k, "perm_k", (H, N), I32T),
+        off_q=ptr(b.off_q, "off_q", (H, oq), I32T), off_k=ptr(b.off_k, "off_k", (H, ok), I32T),
+        qp=ptr(b.qp, "qp", (H, N, d), q.dtype), kp=ptr(b.kp, "kp", (H, N, d), q.dtype),
+        vp=ptr(b.vp, "vp", (H, N, d), q.dtype),
+        csr=ptr(b.csr, "csr", (H, int(p["Cq"]), kmax), I32T),
+        k_per_head=ptr(b.k_per_head, "k_per_head", (H,), I32T),
+        o_sparse=ptr(b.o_sparse, "o_sparse", (H, N, d), torch.float32),
+        pairs_sparse=ptr(b.pairs_sparse, "pairs_sparse", (H,), I64),
+        probes=ptr(b.probes, "probes", (H, max(M, 1)), I32T),
+        pairs_exec=ptr(b.pairs_exec, "pairs_exec", (H,), I64),
+        fit=None if b.fit is None else ptr(b.fit, "fit", (H, d * d + d), torch.float64))
+    out = _arg(b.out, "out", (H, N, d), q.dtype)
+    wp, wb = _ws(b.ws)
+    _check(lib.sparsepr_attention(pq, pk, pv, dt, ctypes.byref(prm), ctypes.byref(cb), out, wp, wb,
+                                  _stream(stream)), "sparsepr_attention")
     return b
 
 

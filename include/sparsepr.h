@@ -263,6 +263,46 @@ sparsepr_status sparsepr_probe_correct(const void* qp, const void* kp, const voi
                                        double* fit, void* ws, size_t ws_bytes,
                                        void* stream);
 
+/* Buffers of sparsepr_attention: every output of the five calls, with the
+ * shapes and types given there (caller-owned device memory). fit may be
+ * NULL; probes may be NULL when M = 0. */
+typedef struct {
+  int32_t* label_q;       /* [H, N] */
+  int32_t* label_k;       /* [H, N] */
+  int32_t* perm_q;        /* [H, N] */
+  int32_t* perm_k;        /* [H, N] */
+  int32_t* off_q;         /* [H, Cq + 1 (+1 with text)] */
+  int32_t* off_k;         /* [H, Ck + 1 (+1 with text)] */
+  void* qp;               /* [H, N, d] input dtype: permuted Q, K, V */
+  void* kp;
+  void* vp;
+  int32_t* csr;           /* [H, Cq, sparsepr_route_width(p)] */
+  int32_t* k_per_head;    /* [H] */
+  float* o_sparse;        /* [H, N, d] fp32 */
+  int64_t* pairs_sparse;  /* [H] */
+  int32_t* probes;        /* [H, M] */
+  int64_t* pairs_exec;    /* [H] */
+  double* fit;            /* [H, d*d + d] or NULL */
+} sparsepr_call_buffers;
+
+/* The whole call [SPR 2.A-2.C] in one entry point: sparsepr_partition,
+ * sparsepr_permute and sparsepr_route as above, then the attention of all
+ * rows while the probe fit of stage 4 runs beside it on a second stream:
+ * the probe rows' dense outputs and their sparse outputs X come from one
+ * pass over all keys (each probe row's keys limited to its query group's
+ * kept runs for X, with the same masking and fp32 arithmetic as
+ * sparsepr_block_sparse_attn, taken over the key tiles in another order),
+ * then the ridge fit and the residual subspace; only the correction waits
+ * for both. Outputs are those of the five calls; integer outputs (labels,
+ * permutations, offsets, routes, pair counts, probes) are identical to
+ * theirs, and X, hence fit and out, may differ from theirs in the rounding
+ * of fp32 sums. q, k, v [H, N, d] in the dtype dt; out [H, N, d] dt, original
+ * token order. Errors: those of the five calls (no work is enqueued after a
+ * host-side error). */
+sparsepr_status sparsepr_attention(const void* q, const void* k, const void* v, sparsepr_dtype dt,
+                                   const sparsepr_params* p, const sparsepr_call_buffers* b,
+                                   void* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Where a stage's intermediate results sit inside `ws`, for stage-level
  * tests and debugging (the workspace layout depends only on the
  * parameters): the byte offset and size of the named region. Contents
