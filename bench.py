@@ -62,8 +62,8 @@ def workload_desc(w):
 # DRAM traffic of the routed attention launch on the 720p workload from one ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
 # attention source it was taken on (hash of attn.cu below).
-ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=724185600 + 449008640,
-                    source_sha256_prefix="d4a872a215d524c3")
+ATTN_TRAFFIC = dict(workload="wan13b_720p", bytes=721397760 + 453008128,
+                    source_sha256_prefix="a016b904110c31fc")
 
 
 def attn_traffic(w):

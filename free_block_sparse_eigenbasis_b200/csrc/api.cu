@@ -352,6 +352,10 @@ __global__ void dense_meta_kernel(int32_t* meta, int H, int M, int N) {
   kh[h] = 1;
 }
 
+// sparsepr_attention overlaps the probe fit with the attention of all rows
+// while the dual pass's extra work stays below this many flop.
+constexpr double kDualFlopMax = 4e11;
+
 // bf16 copies of the permuted Q, K, V for the attention kernels (fp32 inputs
 // are rounded into the workspace; bf16 inputs are used in place).
 struct Bf16Qkv {
@@ -928,7 +932,19 @@ sparsepr_status sparsepr_attention(const void* q, const void* k, const void* v, 
   const AttnArgs a = main_attn_args(c, ws, t, b->off_q, b->off_k, b->csr, b->k_per_head,
                                     b->o_sparse, b->pairs_sparse);
   SPR_TRY(launch_attn_meta(a, c.st));  // the runs the dual probe pass reads
-  if (c.p.M > 0) {
+  // The overlap pays while the dual pass's extra work (the probe rows' masked
+  // pass over all keys, 4 d H M N flop) costs less than the fit latency it
+  // hides (about 0.6 ms, latency-bound on H CTAs): below 4e11 flop (the 720p
+  // 12-head layer: 2.4e11). Wider calls keep the five-call order.
+  const double dual_flop = 4.0 * c.p.d * c.p.H * static_cast<double>(c.p.M) * c.p.N;
+  if (c.p.M > 0 && dual_flop >= kDualFlopMax) {
+    SPR_TRY(launch_attn_kernel(a, c.st));
+    sparsepr_status fs = probe_pass(c, ws, t, b->qp, b->off_q, b->probes, false, c.st);
+    if (fs != SPARSEPR_OK) return fs;
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    fs = probe_solve(c, ws, b->probes, b->o_sparse, b->fit, c.st, side_stream(0));
+    if (fs != SPARSEPR_OK) return fs;
+  } else if (c.p.M > 0) {
     // the probe rows' dense and sparse outputs in one pass (work for every
     // SM, so in order before the attention), then the fit, latency-bound on
     // few SMs, on a side stream beside the attention of all rows; joined on

@@ -287,18 +287,21 @@ typedef struct {
 
 /* The whole call [SPR 2.A-2.C] in one entry point: sparsepr_partition,
  * sparsepr_permute and sparsepr_route as above, then the attention of all
- * rows while the probe fit of stage 4 runs beside it on a second stream:
- * the probe rows' dense outputs and their sparse outputs X come from one
- * pass over all keys (each probe row's keys limited to its query group's
- * kept runs for X, with the same masking and fp32 arithmetic as
- * sparsepr_block_sparse_attn, taken over the key tiles in another order),
- * then the ridge fit and the residual subspace; only the correction waits
- * for both. Outputs are those of the five calls; integer outputs (labels,
- * permutations, offsets, routes, pair counts, probes) are identical to
- * theirs, and X, hence fit and out, may differ from theirs in the rounding
- * of fp32 sums. q, k, v [H, N, d] in the dtype dt; out [H, N, d] dt, original
- * token order. Errors: those of the five calls (no work is enqueued after a
- * host-side error). */
+ * rows while the probe fit of stage 4 runs beside it on a second stream. The
+ * probe rows' dense outputs and their sparse outputs X come from one pass
+ * over all keys (for X each probe row's keys are limited to its query
+ * group's kept runs, with the same masking and fp32 arithmetic as
+ * sparsepr_block_sparse_attn, taken over the key tiles in another order);
+ * then come the ridge fit and the residual subspace, and only the correction
+ * waits for both. The overlap is taken while that extra pass is cheaper than
+ * the fit latency it hides (4 d H M N < 4e11 flop); wider calls run the
+ * probe rows after the attention of all rows, as the five calls do (X =
+ * o_sparse at the probe rows). Outputs are those of the five calls; integer
+ * outputs (labels, permutations, offsets, routes, pair counts, probes) are
+ * identical to theirs, and X, hence fit and out, may differ from theirs in
+ * the rounding of fp32 sums. q, k, v [H, N, d] in the dtype dt; out
+ * [H, N, d] dt, original token order. Errors: those of the five calls (no
+ * work is enqueued after a host-side error). */
 sparsepr_status sparsepr_attention(const void* q, const void* k, const void* v, sparsepr_dtype dt,
                                    const sparsepr_params* p, const sparsepr_call_buffers* b,
                                    void* out, void* ws, size_t ws_bytes, void* stream);

@@ -84,3 +84,18 @@ def test_fused_call_720p_sampled():
     rows = np.arange(7, w.N, 613)
     res = oracle_head(w, q, k, v, 0, rows=rows)
     compare_head(b, res, w, 0, rows)
+
+
+def test_fused_call_wide_layer_keeps_five_call_order():
+    """24 heads of the Wan2.1-14B-shaped layer: the dual pass would cost more
+    than the fit latency it hides (4 d H M N = 4.8e11 flop), so the probe rows
+    follow the attention of all rows as in the five calls, and every output,
+    the float ones included, equals theirs bit for bit."""
+    w = synth.workload("wan14b_720p", heads=24)
+    assert 4.0 * w.d * w.H * w.M * w.N >= 4e11
+    q, k, v = synth.generate(w)
+    five, _ = gpu_run(w, q, k, v)
+    b = _fused(w, q, k, v)
+    for name in ("label_q", "label_k", "perm_q", "off_q", "csr", "probes", "pairs_exec",
+                 "o_sparse", "out", "fit"):
+        assert torch.equal(getattr(b, name), getattr(five, name)), name
