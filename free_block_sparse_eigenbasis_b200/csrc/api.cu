@@ -176,7 +176,7 @@ struct DPass {
 
 cudaError_t dpass_setup(const Ctx& c, void* ws, const void* X, int m, int Cpad, int32_t* labels,
                         int flag_base, float* xnorm, const double* cy, const double* G, int sms,
-                        DPass* P) {
+                        DPass* P, cudaStream_t st) {
   const int H = c.p.H, N = c.p.N, d = c.p.d, Nv = c.L.Nv;
   const long long hs_in = static_cast<long long>(N) * d;
   P->X = X;
@@ -195,7 +195,7 @@ cudaError_t dpass_setup(const Ctx& c, void* ws, const void* X, int m, int Cpad, 
   }
   if (!P->nb) return cudaSuccess;
   const cudaError_t e = launch_split_rows(X, c.kind, hs_in, d, Nv, d, d, 0, H, nullptr, 0, xnorm,
-                                          c.st);
+                                          st);
   if (e != cudaSuccess) return e;
   AssignTC& a = P->a;
   a = assign_common(c, ws, labels, at<int32_t>(ws, c.L.flags), flag_base, sms);
@@ -272,8 +272,10 @@ sparsepr_status partition_alternative(const Ctx& c, const void* q, const void* k
   SPR_TRY(launch_gather_init(k, c.kind, hs_in, d, d, init_k, Ck, H, ck, nullptr, st));
   SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
   DPass pk, pq;
-  SPR_TRY(dpass_setup(c, ws, k, Ck, L.CpadK, lab_k, 0, at<float>(ws, L.xnk), cg, nullptr, sms, &pk));
-  SPR_TRY(dpass_setup(c, ws, q, Cq, L.CpadQ, lab_q, 2, at<float>(ws, L.xnq), cg, nullptr, sms, &pq));
+  SPR_TRY(dpass_setup(c, ws, k, Ck, L.CpadK, lab_k, 0, at<float>(ws, L.xnk), cg, nullptr, sms, &pk,
+                      c.st));
+  SPR_TRY(dpass_setup(c, ws, q, Cq, L.CpadQ, lab_q, 2, at<float>(ws, L.xnq), cg, nullptr, sms, &pq,
+                      c.st));
   if (c.p.partition == SPARSEPR_PARTITION_SEMANTIC) {
     // plain Euclidean Lloyd on each side: the d-space form with G = I
     // (y = centre, cy = |centre|^2)
@@ -704,6 +706,7 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     return partition_alternative(c, q, k, label_q, label_k, ws);
 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
+  DPass pq;  // the query passes (set up beside the key eigen solve)
   {
     // the side stream is joined on every path, also after a failed launch,
     // so that a stream capture in progress stays valid
@@ -711,6 +714,13 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     SideStream* ss = side_stream();
     const cudaStream_t side = fork_side(ss, st);
     cudaError_t err = launch_fy_init(H, Nv, Ck, Cq, c.p.seed, init_k, init_q, side);
+    // the query side's first centroids and row norms need only q: beside the
+    // key metric and its eigen solve (few SMs)
+    if (err == cudaSuccess)
+      err = launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, side);
+    if (err == cudaSuccess)
+      err = dpass_setup(c, ws, q, Cq, L.CpadQ, lab_q, 2, at<float>(ws, L.xnq), cg, G, sm_count(),
+                        &pq, side);
     if (err == cudaSuccess)
       err = launch_metric_mk(q, c.bf16, H, N, Nv, d, c.p.Ms, mk, at<double>(ws, L.gpart), st);
     if (err == cudaSuccess)
@@ -790,11 +800,8 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
   SPR_TRY(launch_gram_f64(ck, ck, nullptr, nullptr, static_cast<long long>(Ck) * d,
                           static_cast<long long>(Ck) * d, d, Ck, H, d, c.scale * c.scale, 0.0, G,
                           static_cast<long long>(d) * d, 0, at<double>(ws, L.gpart), st));
-  // queries: Lloyd passes on logit profiles in the d-space form
-  SPR_TRY(launch_gather_init(q, c.kind, hs_in, d, d, init_q, Cq, H, qbar, nullptr, st));
-  // queries on the tensor cores for bf16 inputs (exact in one bf16 plane)
-  DPass pq;
-  SPR_TRY(dpass_setup(c, ws, q, Cq, L.CpadQ, lab_q, 2, at<float>(ws, L.xnq), cg, G, sms, &pq));
+  // queries: Lloyd passes on logit profiles in the d-space form (on the
+  // tensor cores for bf16 inputs, exact in one bf16 plane)
   for (int t = 0; t < iters; ++t) {
     SPR_TRY(launch_query_metric_apply(G, qbar, Cq, H, d, wg, cg, flags + 3, 4, st));
     SPR_TRY(dpass_run(c, ws, pq, wg, cg));
