@@ -291,12 +291,65 @@ constexpr int kEigWarps = kEigThreads / 32;
 constexpr int kEigMax = kTriEigMax;  // eigenpairs per matrix
 constexpr int kInvBatch = 32;  // eigenvalues in inverse iteration at a time
 
-// One CTA of 512 threads per matrix, ne <= 64 eigenpairs (largest first):
-// multisection by 8-32 threads per eigenvalue (one point each), inverse
-// iteration by thread t (one LU, three solves) for batches of 32 eigenvalues,
-// Gram-Schmidt inside clusters by all warps, then the back-transformation
-// with warp w owning vectors w, w + 16, ... Writes evals [H, ne] and evecs
-// [H, D, ne].
+// The ne largest eigenvalues of the tridiagonal T of each matrix by
+// multisection on Sturm-sequence counts (Golub & Van Loan, sec. 8.4.1): one
+// warp per eigenvalue (rank e_i, ascending index D-1-e_i), each lane
+// evaluating the count at one of 32 interior points of the current interval,
+// which shrinks 33-fold per round, to 4 eps |lambda| + pivmin. A few warps per
+// CTA and several CTAs per matrix, so that the fp64 recurrences of the
+// eigenvalues spread over the SMs instead of sharing one. Writes
+// evals[h, e_i].
+constexpr int kBisWarps = 2;
+
+template <int D>
+__global__ void __launch_bounds__(kBisWarps * 32) multisect_kernel(const double* scratch, int ne,
+                                                                  double* evals) {
+  __shared__ double dg[D], od[D], e2[D];
+  __shared__ double tnorm;
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const double* tau = scratch + static_cast<size_t>(h) * (D * D + 3 * D) + D * D;
+  for (int i = tid; i < D; i += blockDim.x) {
+    dg[i] = tau[D + i];
+    od[i] = tau[2 * D + i];
+    e2[i] = (i < D - 1) ? od[i] * od[i] : 0.0;
+  }
+  __syncthreads();
+  if (tid == 0) {  // the same bound as tri_eig_kernel's
+    double m = 0.0;
+    for (int i = 0; i < D; ++i)
+      m = fmax(m, fabs(dg[i]) + (i > 0 ? fabs(od[i - 1]) : 0.0) + (i < D - 1 ? fabs(od[i]) : 0.0));
+    tnorm = m;
+  }
+  __syncthreads();
+  const int e_i = blockIdx.y * kBisWarps + (tid >> 5);
+  if (e_i >= ne) return;  // the whole warp
+  const double eps = 1.1102230246251565e-16;
+  double emax2 = 0.0;
+  for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
+  const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
+  const int m = D - 1 - e_i;
+  const double inv_parts = 1.0 / 33.0;
+  double lo = -tnorm - 1.0, hi = tnorm + 1.0;
+  for (int it = 0; it < 200; ++it) {
+    const double w = hi - lo;
+    if (!(w > 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin)) break;  // warp-uniform
+    double x[1] = {lo + w * (lane + 1) * inv_parts};
+    int cnt[1] = {D};
+    sturm_counts<D, 1>(dg, e2, x, pivmin, cnt);
+    const int nt = __popc(__ballot_sync(0xffffffffu, cnt[0] <= m));  // points below lambda
+    const double nlo = nt > 0 ? lo + w * nt * inv_parts : lo;
+    const double nhi = nt < 32 ? lo + w * (nt + 1) * inv_parts : hi;
+    lo = nlo;
+    hi = nhi;
+  }
+  if (lane == 0) evals[static_cast<size_t>(h) * ne + e_i] = 0.5 * (lo + hi);
+}
+
+// One CTA of 512 threads per matrix, ne <= 64 eigenpairs (largest first),
+// from the eigenvalues multisect_kernel left in evals: inverse iteration by
+// thread t (one LU, three solves) for batches of 32 eigenvalues, Gram-Schmidt
+// inside clusters by all warps, then the back-transformation with warp w
+// owning vectors w, w + 16, ... Writes evals [H, ne] and evecs [H, D, ne].
 // Dynamic shared memory: the inverse-iteration work arrays of one batch (32
 // threads interleaved; later the staged Householder vectors), then the
 // vectors Y [kEigMax][D + 1].
@@ -318,7 +371,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) tri_eig_kernel(const double* s
                                                        double* evals, double* evecs) {
   extern __shared__ double eig_work[];  // inverse-iteration work arrays, then Y
   double (*Y)[D + 1] = reinterpret_cast<double (*)[D + 1]>(eig_work + eig_work_bytes<D>() / 8);
-  __shared__ double dg[D], od[D], e2[D];
+  __shared__ double dg[D], od[D];
   __shared__ double lam[kEigMax];
   __shared__ double tnorm;
   __shared__ double gdot[kEigMax], gred[kEigWarps];
@@ -330,7 +383,6 @@ __global__ void __launch_bounds__(kEigThreads, 1) tri_eig_kernel(const double* s
     od[i] = tau[2 * D + i];
   }
   __syncthreads();
-  for (int i = tid; i < D; i += blockDim.x) e2[i] = (i < D - 1) ? od[i] * od[i] : 0.0;
   if (tid == 0) {
     double m = 0.0;
     for (int i = 0; i < D; ++i)
@@ -339,40 +391,8 @@ __global__ void __launch_bounds__(kEigThreads, 1) tri_eig_kernel(const double* s
   }
   __syncthreads();
   const double eps = 1.1102230246251565e-16;
-  double emax2 = 0.0;
-  for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
-  const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
-  // multisection: tpe threads per wanted eigenvalue (rank e_i = tid / tpe,
-  // ascending index D-1-e_i; tpe = 32, 16 or 8 for ne <= 16, 32 or 64) each
-  // evaluate the Sturm count at one interior point of the current interval,
-  // which shrinks (tpe + 1)-fold per round (the recurrences are bound by the
-  // fp64 pipe, so more points per thread only add work)
-  {
-    const int tpe = ne <= kEigThreads / 32 ? 32 : (ne <= kEigThreads / 16 ? 16 : 8);
-    const int e_i = tid / tpe, q = tid % tpe;
-    const bool act = e_i < ne;
-    const int m = D - 1 - e_i;
-    const double inv_parts = 1.0 / (tpe + 1);
-    const unsigned gmask = tpe == 32 ? 0xFFFFFFFFu : ((1u << tpe) - 1u);
-    double lo = -tnorm - 1.0, hi = tnorm + 1.0;
-    for (int it = 0; it < 200; ++it) {
-      const double w = hi - lo;
-      const bool done = !(w > 4.0 * eps * fmax(fabs(lo), fabs(hi)) + pivmin);
-      if (__all_sync(0xffffffffu, done || !act)) break;
-      double x[1] = {lo + w * (q + 1) * inv_parts};
-      int cnt[1] = {D};
-      if (act && !done) sturm_counts<D, 1>(dg, e2, x, pivmin, cnt);
-      const unsigned bal = __ballot_sync(0xffffffffu, act && !done && cnt[0] <= m);
-      const int nt = __popc((bal >> ((lane / tpe) * tpe)) & gmask);  // points below lambda
-      if (act && !done) {
-        const double nlo = nt > 0 ? lo + w * nt * inv_parts : lo;
-        const double nhi = nt < tpe ? lo + w * (nt + 1) * inv_parts : hi;
-        lo = nlo;
-        hi = nhi;
-      }
-    }
-    if (act && q == 0) lam[e_i] = 0.5 * (lo + hi);
-  }
+  // the eigenvalues, from multisect_kernel
+  for (int i = tid; i < ne; i += blockDim.x) lam[i] = evals[static_cast<size_t>(h) * ne + i];
   __syncthreads();
   // inverse iteration from a fixed, index-dependent start vector, 32
   // eigenvalues at a time; Gram-Schmidt against the earlier vectors of the
@@ -502,6 +522,8 @@ cudaError_t launch_d(const double* A, int H, int ne, double* evals, double* evec
                                        static_cast<int>(eig_smem_bytes<D>()));
   if (e != cudaSuccess) return e;
   tridiag_kernel<D><<<H, kTriThreads, 0, st>>>(A, scratch);
+  multisect_kernel<D><<<dim3(H, (ne + kBisWarps - 1) / kBisWarps), kBisWarps * 32, 0, st>>>(
+      scratch, ne, evals);
   tri_eig_kernel<D><<<H, kEigThreads, eig_smem_bytes<D>(), st>>>(scratch, ne, evals, evecs);
   return cudaGetLastError();
 }
