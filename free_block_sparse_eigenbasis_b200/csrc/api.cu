@@ -608,6 +608,40 @@ __global__ void wait_limit_kernel(DeviceStats* stats) {
   if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort)) raise_status(stats, SPARSEPR_ERR_TIMEOUT);
 }
 
+// The sorts and the gathers of q and k (and of v when `with_v`; K and V
+// share their permutation and move in one launch).
+sparsepr_status permute_rows(const Ctx& c, const void* q, const void* k, const void* v,
+                             const int32_t* label_q, const int32_t* label_k, int32_t* perm_q,
+                             int32_t* perm_k, int32_t* off_q, int32_t* off_k, void* qp, void* kp,
+                             void* vp, bool with_v, void* ws) {
+  const int H = c.p.H, N = c.p.N, d = c.p.d;
+  const int nchunk = c.L.nchunk;  // chunks of all N tokens
+  int32_t* hist = at<int32_t>(ws, c.L.hist);
+  // with text tokens the last group of each side is the text group
+  SPR_TRY(launch_counting_sort(label_q, H, N, c.L.Cqt, nchunk, hist, perm_q, off_q, nullptr, 0,
+                               c.stats, c.st));
+  SPR_TRY(launch_counting_sort(label_k, H, N, c.L.Ckt, nchunk, hist, perm_k, off_k, nullptr, 0,
+                               c.stats, c.st));
+  const int eb = c.bf16 ? 2 : 4;
+  SPR_TRY(launch_gather_rows(q, qp, nullptr, nullptr, perm_q, H, N, d, eb, c.st));
+  SPR_TRY(launch_gather_rows(k, kp, with_v ? v : nullptr, with_v ? vp : nullptr, perm_k, H, N, d,
+                             eb, c.st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status check_permute_args(const void* q, const void* k, const void* v,
+                                   const int32_t* label_q, const int32_t* label_k,
+                                   const int32_t* perm_q, const int32_t* perm_k,
+                                   const int32_t* off_q, const int32_t* off_k, const void* qp,
+                                   const void* kp, const void* vp) {
+  if (!q || !k || !v || !label_q || !label_k || !perm_q || !perm_k || !off_q || !off_k || !qp ||
+      !kp || !vp)
+    return SPARSEPR_ERR_INVALID_ARG;
+  if (qp == q || kp == k || vp == v) return SPARSEPR_ERR_INVALID_ARG;
+  if (!al16(q, k, v, qp, kp, vp)) return SPARSEPR_ERR_INVALID_ARG;
+  return SPARSEPR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -826,24 +860,10 @@ sparsepr_status sparsepr_permute(const void* q, const void* k, const void* v, sp
   Ctx c;
   sparsepr_status s = setup(&c, p, dt, ws, ws_bytes, stream);
   if (s != SPARSEPR_OK) return s;
-  if (!q || !k || !v || !label_q || !label_k || !perm_q || !perm_k || !off_q || !off_k || !qp ||
-      !kp || !vp)
-    return SPARSEPR_ERR_INVALID_ARG;
-  if (qp == q || kp == k || vp == v) return SPARSEPR_ERR_INVALID_ARG;
-  if (!al16(q, k, v, qp, kp, vp)) return SPARSEPR_ERR_INVALID_ARG;
-  const int H = c.p.H, N = c.p.N, d = c.p.d;
-  const int nchunk = c.L.nchunk;  // chunks of all N tokens
-  int32_t* hist = at<int32_t>(ws, c.L.hist);
-  // with text tokens the last group of each side is the text group
-  SPR_TRY(launch_counting_sort(label_q, H, N, c.L.Cqt, nchunk, hist, perm_q, off_q, nullptr, 0,
-                               c.stats, c.st));
-  SPR_TRY(launch_counting_sort(label_k, H, N, c.L.Ckt, nchunk, hist, perm_k, off_k, nullptr, 0,
-                               c.stats, c.st));
-  const int eb = c.bf16 ? 2 : 4;
-  SPR_TRY(launch_gather_rows(q, qp, perm_q, H, N, d, eb, c.st));
-  SPR_TRY(launch_gather_rows(k, kp, perm_k, H, N, d, eb, c.st));
-  SPR_TRY(launch_gather_rows(v, vp, perm_k, H, N, d, eb, c.st));
-  return SPARSEPR_OK;
+  s = check_permute_args(q, k, v, label_q, label_k, perm_q, perm_k, off_q, off_k, qp, kp, vp);
+  if (s != SPARSEPR_OK) return s;
+  return permute_rows(c, q, k, v, label_q, label_k, perm_q, perm_k, off_q, off_k, qp, kp, vp, true,
+                      ws);
 }
 
 sparsepr_status sparsepr_route(const void* qp, const void* kp, sparsepr_dtype dt,
@@ -922,12 +942,30 @@ sparsepr_status sparsepr_attention(const void* q, const void* k, const void* v, 
   if (!b || !out) return SPARSEPR_ERR_INVALID_ARG;
   sparsepr_status s = sparsepr_partition(q, k, dt, p, b->label_q, b->label_k, ws, ws_bytes, stream);
   if (s != SPARSEPR_OK) return s;
-  s = sparsepr_permute(q, k, v, dt, p, b->label_q, b->label_k, b->perm_q, b->perm_k, b->off_q,
-                       b->off_k, b->qp, b->kp, b->vp, ws, ws_bytes, stream);
-  if (s != SPARSEPR_OK) return s;
-  s = sparsepr_route(b->qp, b->kp, dt, p, b->off_q, b->off_k, b->csr, b->k_per_head, ws, ws_bytes,
-                     stream);
-  if (s != SPARSEPR_OK) return s;
+  {
+    Ctx c;
+    s = setup(&c, p, dt, ws, ws_bytes, stream);
+    if (s != SPARSEPR_OK) return s;
+    s = check_permute_args(q, k, v, b->label_q, b->label_k, b->perm_q, b->perm_k, b->off_q,
+                           b->off_k, b->qp, b->kp, b->vp);
+    if (s != SPARSEPR_OK) return s;
+    s = permute_rows(c, q, k, v, b->label_q, b->label_k, b->perm_q, b->perm_k, b->off_q, b->off_k,
+                     b->qp, b->kp, b->vp, false, ws);
+    if (s != SPARSEPR_OK) return s;
+    // V is read first by the attention: its gather runs beside the routing
+    // (joined on every path)
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStream* ss = side_stream(0);
+    const cudaStream_t side = fork_side(ss, c.st);
+    const cudaError_t ev = launch_gather_rows(v, b->vp, nullptr, nullptr, b->perm_k, c.p.H, c.p.N,
+                                              c.p.d, c.bf16 ? 2 : 4, side);
+    s = sparsepr_route(b->qp, b->kp, dt, p, b->off_q, b->off_k, b->csr, b->k_per_head, ws,
+                       ws_bytes, stream);
+    const cudaError_t ej = join_side(ss, side, c.st);
+    if (s != SPARSEPR_OK) return s;
+    SPR_TRY(ev);
+    SPR_TRY(ej);
+  }
   Ctx c;
   s = setup(&c, p, dt, ws, ws_bytes, stream);
   if (s != SPARSEPR_OK) return s;

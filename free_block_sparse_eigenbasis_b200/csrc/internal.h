@@ -170,8 +170,11 @@ cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals
                             double* scratch, cudaStream_t st);
 
 // ---- permute.cu ------------------------------------------------------------
-cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, int H, int N,
-                               int d, int elem_bytes, cudaStream_t st);
+// dst = src gathered by `perm` (and dst2 = src2, the same rows, when src2 is
+// given; both null otherwise)
+cudaError_t launch_gather_rows(const void* src, void* dst, const void* src2, void* dst2,
+                               const int32_t* perm, int H, int N, int d, int elem_bytes,
+                               cudaStream_t st);
 // Score GEMM + warp top-k, heads in groups whose scores fit in `scores`
 // (route_scores_bytes(H, Cq, Ck) bytes in the workspace).
 size_t route_scores_bytes(int H, int Cq, int Ck);

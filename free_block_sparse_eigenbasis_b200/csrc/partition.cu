@@ -643,6 +643,52 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_kernel(
   }
 }
 
+// 16-byte pieces in flight per thread in the vector and warp forms of the
+// group mean, and the row positions staged in shared memory at a time.
+constexpr int kMeanDepth = 8;
+constexpr int kMeanChunk = 1024;     // per CTA (vector form)
+constexpr int kMeanWarpChunk = 128;  // per warp (warp form)
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Adds to acc, in ascending order, this thread's 16-byte pieces of the rows
+// rows_s[q], q = q0, q0 + RL, ... < nq (row stride ldx, Xh already at the
+// thread's columns). The pieces come through the thread's own kMeanDepth
+// shared-memory slots (slot s at slot0[s * kMeanThreads]), kMeanDepth copies
+// in flight; a slot is refilled only after its piece was added, so the
+// thread reads and writes no other thread's slots.
+template <typename T, int EPT>
+__device__ __forceinline__ void sum_pieces(const T* Xh, int ldx, const int32_t* rows_s, int q0,
+                                           int nq, int RL, uint4* slot0, double (&acc)[EPT]) {
+  const int K = q0 < nq ? (nq - q0 + RL - 1) / RL : 0;
+#pragma unroll
+  for (int s = 0; s < kMeanDepth; ++s) {
+    if (s < K) cp_async16(slot0 + s * kMeanThreads, Xh + static_cast<size_t>(rows_s[q0 + s * RL]) * ldx);
+    cp_async_commit();
+  }
+#pragma unroll 1
+  for (int k = 0; k < K; ++k) {
+    cp_async_wait<kMeanDepth - 1>();  // the piece k has landed
+    uint4* sl = slot0 + (k & (kMeanDepth - 1)) * kMeanThreads;
+    double v[EPT];
+    vwiden16<T>(*sl, v);
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) acc[i] += v[i];
+    if (k + kMeanDepth < K)
+      cp_async16(sl, Xh + static_cast<size_t>(rows_s[q0 + (k + kMeanDepth) * RL]) * ldx);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+}
+
 // Vector form of the group mean for rows of D * sizeof(T) bytes that split
 // into 16-byte pieces: TPR = D * sizeof(T) / 16 threads per row, each summing
 // EPT = 16 / sizeof(T) columns over the rows lo + rl, lo + rl + RL, ...
@@ -655,8 +701,11 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
     const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
     const int32_t* skip, int skip_stride) {
   constexpr int EPT = 16 / sizeof(T);
-  __shared__ double part[kMeanThreads * EPT];
+  static_assert(sizeof(double) * EPT <= sizeof(uint4) * kMeanDepth, "partial sums fit in the slots");
+  __shared__ __align__(16) uint4 slots[kMeanDepth * kMeanThreads];
+  __shared__ int32_t rows_s[kMeanChunk];
   __shared__ double red[kMeanThreads / 32];
+  double* part = reinterpret_cast<double*>(slots);  // after the sums
   const int h = blockIdx.y, c = blockIdx.x;
   if (skip && skip[h * skip_stride]) return;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -669,33 +718,18 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
   double acc[EPT];
 #pragma unroll
   for (int i = 0; i < EPT; ++i) acc[i] = 0.0;
-  // rows p, p + RL, p + 2 RL, p + 3 RL of this row lane in flight together,
-  // summed in ascending position order
-  int p = lo + rl;
+  // the group's rows in chunks of kMeanChunk positions (a multiple of RL, so
+  // that row lane rl sums the rows lo + rl, lo + rl + RL, ... in ascending
+  // order), their row indices staged in shared memory
 #pragma unroll 1
-  for (; p + 3 * RL < hi; p += 4 * RL) {
-    size_t r[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) r[j] = pp ? static_cast<size_t>(pp[p + j * RL]) : static_cast<size_t>(p + j * RL);
-    uint4 u[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) u[j] = *reinterpret_cast<const uint4*>(Xh + r[j] * ldx);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      double v[EPT];
-      vwiden16<T>(u[j], v);
-#pragma unroll
-      for (int i = 0; i < EPT; ++i) acc[i] += v[i];
-    }
+  for (int cb = lo; cb < hi; cb += kMeanChunk) {
+    const int nq = min(kMeanChunk, hi - cb);
+    __syncthreads();  // the previous chunk's positions are no longer read
+    for (int i = threadIdx.x; i < nq; i += kMeanThreads) rows_s[i] = pp ? pp[cb + i] : cb + i;
+    __syncthreads();
+    sum_pieces<T, EPT>(Xh, ldx, rows_s, rl, nq, RL, slots + threadIdx.x, acc);
   }
-#pragma unroll 1
-  for (; p < hi; p += RL) {
-    const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
-    double v0[EPT];
-    vload16(Xh + r0 * ldx, v0);
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
-  }
+  __syncthreads();  // every slot read before the partial sums overwrite them
   // the row lanes of a warp that share columns (lanes TPR apart) first, by
   // shuffles; then the warps' partial rows in shared memory, in warp order
   int prow = rl, npart = RL;
@@ -749,6 +783,9 @@ __global__ void __launch_bounds__(kMeanWarpGroups * 32) group_mean_warp_kernel(
     const int32_t* off, int off_stride, int C, bool keep_prev, double* out, double* norms,
     const int32_t* skip, int skip_stride) {
   constexpr int EPT = 16 / sizeof(T);
+  static_assert(kMeanWarpGroups * 32 == kMeanThreads, "slot stride");
+  __shared__ __align__(16) uint4 slots[kMeanDepth * kMeanThreads];
+  __shared__ int32_t rows_s[kMeanWarpGroups][kMeanWarpChunk];
   const int h = blockIdx.y;
   const int c = blockIdx.x * kMeanWarpGroups + static_cast<int>(threadIdx.x >> 5);
   if (c >= C) return;  // the whole warp
@@ -763,30 +800,17 @@ __global__ void __launch_bounds__(kMeanWarpGroups * 32) group_mean_warp_kernel(
   double acc[EPT];
 #pragma unroll
   for (int i = 0; i < EPT; ++i) acc[i] = 0.0;
-  int p = lo + rl;
+  // the group's rows in chunks of kMeanWarpChunk positions (a multiple of
+  // RL: lane row rl sums the rows lo + rl, lo + rl + RL, ... in ascending
+  // order), their row indices staged in the warp's shared memory
+  int32_t* rw = rows_s[threadIdx.x >> 5];
 #pragma unroll 1
-  for (; p + 3 * RL < hi; p += 4 * RL) {
-    size_t r[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) r[j] = pp ? static_cast<size_t>(pp[p + j * RL]) : static_cast<size_t>(p + j * RL);
-    uint4 u[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) u[j] = *reinterpret_cast<const uint4*>(Xh + r[j] * ldx);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      double v[EPT];
-      vwiden16<T>(u[j], v);
-#pragma unroll
-      for (int i = 0; i < EPT; ++i) acc[i] += v[i];
-    }
-  }
-#pragma unroll 1
-  for (; p < hi; p += RL) {
-    const size_t r0 = pp ? static_cast<size_t>(pp[p]) : static_cast<size_t>(p);
-    double v0[EPT];
-    vload16(Xh + r0 * ldx, v0);
-#pragma unroll
-    for (int i = 0; i < EPT; ++i) acc[i] += v0[i];
+  for (int cb = lo; cb < hi; cb += kMeanWarpChunk) {
+    const int nq = min(kMeanWarpChunk, hi - cb);
+    __syncwarp();  // the previous chunk's positions are no longer read
+    for (int i = lane; i < nq; i += 32) rw[i] = pp ? pp[cb + i] : cb + i;
+    __syncwarp();
+    sum_pieces<T, EPT>(Xh, ldx, rw, rl, nq, RL, slots + threadIdx.x, acc);
   }
   for (int o = TPR; o < 32; o <<= 1)
 #pragma unroll

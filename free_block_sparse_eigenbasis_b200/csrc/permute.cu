@@ -9,17 +9,47 @@
 namespace spr {
 namespace {
 
-// dst[h, i, :] = src[h, perm[h, i], :]; rows are copied with 16-byte vectors.
-__global__ void gather_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                   const int32_t* __restrict__ perm, int N, int vec_per_row,
-                                   size_t total_vec) {
-  const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= total_vec) return;
-  const size_t row = t / vec_per_row;
-  const int v = static_cast<int>(t % vec_per_row);
-  const size_t h = row / N;
-  const size_t srow = h * N + static_cast<size_t>(perm[row]);
-  dst[t] = __ldg(src + srow * vec_per_row + v);
+// dst[h, i, :] = src[h, perm[h, i], :] for one or two (src, dst) pairs that
+// share the permutation (K and V), rows copied in 16-byte pieces. Grid: x over
+// the rows of a head in blocks of kGatherDepth passes, y over heads, so that
+// no index needs a 64-bit division. A thread moves piece v of the rows
+// rr, rr + R, ..., rr + (kGatherDepth - 1) R of its block (R = rows per pass,
+// 256 / pieces per row); all its loads, of both pairs, are issued before its
+// first store, so several are in flight together.
+constexpr int kGatherThreads = 256, kGatherDepth = 4;
+
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
+    const uint4* __restrict__ s0, uint4* __restrict__ d0, const uint4* __restrict__ s1,
+    uint4* __restrict__ d1, const int32_t* __restrict__ perm, int N, int vpr) {
+  const int rpp = kGatherThreads / vpr;
+  const int rr = static_cast<int>(threadIdx.x) / vpr;
+  const int v = static_cast<int>(threadIdx.x) - rr * vpr;
+  if (rr >= rpp) return;
+  const size_t hb = static_cast<size_t>(blockIdx.y) * N;
+  const int r0 = static_cast<int>(blockIdx.x) * rpp * kGatherDepth + rr;
+  int sr[kGatherDepth];
+#pragma unroll
+  for (int j = 0; j < kGatherDepth; ++j) {
+    const int r = r0 + j * rpp;
+    sr[j] = r < N ? __ldg(perm + hb + r) : -1;
+  }
+  uint4 u[kGatherDepth], w[kGatherDepth];
+#pragma unroll
+  for (int j = 0; j < kGatherDepth; ++j)
+    if (sr[j] >= 0) u[j] = __ldcs(s0 + (hb + sr[j]) * vpr + v);
+  if (s1) {
+#pragma unroll
+    for (int j = 0; j < kGatherDepth; ++j)
+      if (sr[j] >= 0) w[j] = __ldcs(s1 + (hb + sr[j]) * vpr + v);
+  }
+#pragma unroll
+  for (int j = 0; j < kGatherDepth; ++j)
+    if (sr[j] >= 0) d0[(hb + r0 + j * rpp) * vpr + v] = u[j];
+  if (s1) {
+#pragma unroll
+    for (int j = 0; j < kGatherDepth; ++j)
+      if (sr[j] >= 0) d1[(hb + r0 + j * rpp) * vpr + v] = w[j];
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -177,12 +207,19 @@ __global__ void write_k_kernel(KhParam kp, int H, int32_t* out) {
 
 }  // namespace
 
-cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* perm, int H, int N,
-                               int d, int elem_bytes, cudaStream_t st) {
-  const int vec = d * elem_bytes / 16;
-  const size_t total = static_cast<size_t>(H) * N * vec;
-  gather_rows_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), perm, N, vec, total);
+cudaError_t launch_gather_rows(const void* src, void* dst, const void* src2, void* dst2,
+                               const int32_t* perm, int H, int N, int d, int elem_bytes,
+                               cudaStream_t st) {
+  const int vpr = d * elem_bytes / 16;
+  if (vpr < 1 || vpr > kGatherThreads || vpr * 16 != d * elem_bytes || (src2 == nullptr) != (dst2 == nullptr))
+    return cudaErrorInvalidValue;
+  if (H < 1 || N < 1) return cudaSuccess;
+  const int rows_per_block = (kGatherThreads / vpr) * kGatherDepth;
+  const dim3 grid(static_cast<unsigned>((N + rows_per_block - 1) / rows_per_block),
+                  static_cast<unsigned>(H));
+  gather_rows_kernel<<<grid, kGatherThreads, 0, st>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), static_cast<const uint4*>(src2),
+      static_cast<uint4*>(dst2), perm, N, vpr);
   return cudaGetLastError();
 }
 
