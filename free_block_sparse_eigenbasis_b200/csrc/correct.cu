@@ -194,33 +194,49 @@ __global__ void __launch_bounds__(kCtThreads, 1)
       for (int j = threadIdx.x; j < D; j += kCtEpi) bvs[j] = p.bv[static_cast<size_t>(h) * D + j];
       named_barrier_sync(kCtBarHead, kCtEpi);
       const int32_t* pr = p.probes + static_cast<size_t>(h) * p.M;
+      const int32_t* pq = p.perm_q + static_cast<size_t>(h) * p.N;
+      int lo = 0;  // first probe >= the row's position (ascending over the tiles)
+      // the row's token index, read one tile ahead so that the load overlaps
+      // the waits of the tile before
+      int tok = (t0 * kTileM + r < p.N) ? pq[t0 * kTileM + r] : 0;
       for (int t = t0; t < t1; ++t, ++u) {
         const int s = u & 1;
+        const int i = t * kTileM + r;  // group-major position in head h
+        const int in = i + kTileM;
+        const int tok_next = (t + 1 < t1 && in < p.N) ? pq[in] : 0;
+        const bool valid = i < p.N;
+        if (valid) {  // probe rows: before the waits too
+          if (t == t0) {  // a binary search at the segment's first tile
+            int hi = p.M;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (pr[mid] < i) lo = mid + 1; else hi = mid;
+            }
+          } else {  // then a forward scan (about M * 128 / N probes per tile)
+            while (lo < p.M && pr[lo] < i) ++lo;
+          }
+        }
+        const bool is_probe = valid && lo < p.M && pr[lo] == i;
         ok = ok && mbar_wait(&bars->acc_full[s], (u >> 1) & 1, abort);
         ok = ok && mbar_wait(&bars->a_full[s], (u >> 1) & 1, abort);  // x tile visible here too
         // tcgen05.ld is warp-collective: the whole warp loads or none of it does
         ok = __all_sync(0xffffffffu, ok);
-        const int i = t * kTileM + r;  // group-major position in head h
         if (ok) {
           tc_fence_after();
-          const bool valid = i < p.N;
-          int lo = 0, hi = valid ? p.M : 0;  // first probe >= i
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (pr[mid] < i) lo = mid + 1; else hi = mid;
-          }
-          const bool is_probe = valid && lo < p.M && pr[lo] == i;
           const bool plain = i >= p.n_corr;  // text row: x itself
-          const size_t dst =
-              valid ? (static_cast<size_t>(h) * p.N + p.perm_q[static_cast<size_t>(h) * p.N + i]) * D : 0;
+          const size_t dst = valid ? (static_cast<size_t>(h) * p.N + tok) * D : 0;
           const float* odr = p.od + (static_cast<size_t>(h) * p.M + lo) * D;
           const uint8_t* xa = As + s * S::kAStage + r * 128;
+          // the half row's accumulators in one round trip
+          uint32_t accs[D / 64][32];
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(s * D + hf * (D / 2) + c * 32), accs[c]);
+          tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
             const int col0 = hf * (D / 2) + c * 32;  // 32 columns = one swizzle atom
-            uint32_t acc[32];
-            tmem_ld32(tmem + lane_base + static_cast<uint32_t>(s * D + col0), acc);
-            tmem_wait_ld();
+            const uint32_t (&acc)[32] = accs[c];
             if (!valid) continue;
             float y[32];
             const uint8_t* xrow = xa + (col0 / 32) * S::kSlabA;
@@ -268,6 +284,7 @@ __global__ void __launch_bounds__(kCtThreads, 1)
         tc_fence_before();
         mbar_arrive(&bars->acc_empty[s]);
         mbar_arrive(&bars->a_empty[s]);
+        tok = tok_next;
       }
     });
   }

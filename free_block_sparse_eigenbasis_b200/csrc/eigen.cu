@@ -183,6 +183,21 @@ __global__ void __launch_bounds__(kTriThreads, 1)
   }
 }
 
+// 1/q for a finite q of normal magnitude: the approximate reciprocal of the
+// PTX instruction set refined by two Newton-Raphson steps for f(y) = 1/y - q,
+// y <- y + y (1 - q y) (each step squares the relative error; Muller et al.,
+// Handbook of Floating-Point Arithmetic, 2nd ed., sec. 4.7), so the result is
+// within a few ulp of 1/q, not correctly rounded. The Sturm counts below keep
+// |q| >= pivmin and |e2 / q| <= 1 / safe-minimum, so q is always in range.
+__device__ __forceinline__ double rcp_newton(double q) {
+  double y;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(q));
+  double r = fma(-q, y, 1.0);
+  y = fma(y, r, y);
+  r = fma(-q, y, 1.0);
+  return fma(y, r, y);
+}
+
 // Number of eigenvalues of T below each of P points x (Sturm sequences of
 // the LDL^T pivots), the P recurrences interleaved.
 template <int D, int P>
@@ -200,7 +215,7 @@ __device__ void sturm_counts(const double* dg, const double* e2, const double (&
     const double d = dg[i], e = e2[i - 1];
 #pragma unroll
     for (int p = 0; p < P; ++p) {
-      q[p] = d - x[p] - e * __drcp_rn(q[p]);
+      q[p] = d - x[p] - e * rcp_newton(q[p]);
       if (fabs(q[p]) < pivmin) q[p] = -pivmin;
       cnt[p] += (q[p] < 0.0);
     }

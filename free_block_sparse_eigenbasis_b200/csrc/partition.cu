@@ -692,7 +692,7 @@ __device__ __forceinline__ void sum_pieces(const T* Xh, int ldx, const int32_t* 
 // Vector form of the group mean for rows of D * sizeof(T) bytes that split
 // into 16-byte pieces: TPR = D * sizeof(T) / 16 threads per row, each summing
 // EPT = 16 / sizeof(T) columns over the rows lo + rl, lo + rl + RL, ...
-// (RL = 256 / TPR row lanes, four rows in flight), then the row lanes' sums
+// (RL = 256 / TPR row lanes, kMeanDepth pieces in flight), then the row lanes' sums
 // are combined in a fixed order (within a warp by shuffles, across warps in
 // shared memory).
 template <typename T>
@@ -770,11 +770,11 @@ __global__ void __launch_bounds__(kMeanThreads) group_mean_vec_kernel(
   }
 }
 
-// Warp form of the group mean for short rows (D * sizeof(T) <= 128 bytes,
-// TPR = D * sizeof(T) / 16 <= 8 threads per row): one warp per group, eight
-// groups per CTA; lane l sums the 16-byte piece l % TPR of the rows
-// lo + l / TPR, lo + l / TPR + 32 / TPR, ... (four rows per lane in flight),
-// then the lanes that share a piece are added by shuffles in a fixed order.
+// Warp form of the group mean (TPR = D * sizeof(T) / 16 <= 32 threads per
+// row): one warp per group, eight groups per CTA; lane l sums the 16-byte
+// piece l % TPR of the rows lo + l / TPR, lo + l / TPR + 32 / TPR, ...
+// (kMeanDepth pieces in flight), then the lanes that share a piece are added
+// by shuffles in a fixed order.
 constexpr int kMeanWarpGroups = 8;
 
 template <typename T>
@@ -1150,7 +1150,13 @@ cudaError_t launch_group_mean(const void* X, int x_kind, long long hsx, int ldx,
   const int es = (x_kind == kXf64) ? 8 : (x_kind == kXbf16 ? 2 : 4);
   const bool vec = (D * es) % 16 == 0 && kMeanThreads % (D * es / 16) == 0 && (ldx * es) % 16 == 0 &&
                    (hsx * es) % 16 == 0 && (reinterpret_cast<uintptr_t>(X) & 15) == 0;
-  if (vec && D * es <= 128) {
+  // the warp form (one warp per group) for short rows, and for rows of up to
+  // 32 pieces when the groups are small on average (at most 256 rows), where
+  // a CTA per group would spend more time on its start and its reduction
+  // than on its rows
+  const int tpr = D * es / 16;
+  const bool small_groups = hsx / ldx <= 256LL * C;
+  if (vec && 32 % tpr == 0 && (D * es <= 128 || small_groups)) {
     const dim3 wgrid((C + kMeanWarpGroups - 1) / kMeanWarpGroups, H);
     if (x_kind == kXf64)
       group_mean_warp_kernel<<<wgrid, kMeanWarpGroups * 32, 0, st>>>(
