@@ -690,6 +690,11 @@ sparsepr_status sparsepr_check_wait_limit(void* ws, void* stream) {
   return cuda_status(cudaGetLastError());
 }
 
+sparsepr_status sparsepr_check_reciprocal(const double* x, int64_t n, double* err, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !err))) return SPARSEPR_ERR_INVALID_ARG;
+  return cuda_status(launch_check_reciprocal(x, n, err, static_cast<cudaStream_t>(stream)));
+}
+
 sparsepr_status sparsepr_reset_stats(void* ws, void* stream) {
   if (!ws) return SPARSEPR_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(ws, 0, sizeof(DeviceStats), static_cast<cudaStream_t>(stream)));
@@ -741,6 +746,15 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
 
   // keys: metric, eigenbasis, response coordinates, Lloyd passes
   DPass pq;  // the query passes (set up beside the key eigen solve)
+  // tensor-core assignment when the centroid planes fit in shared memory
+  // (a 128-row TMA box needs at least 128 rows in the tensor)
+  const bool tc_keys = assign_tc_smem_bytes(3, 3, L.Dpk, L.CpadK) <= kMaxDynSmem &&
+                       static_cast<size_t>(H) * Nv >= static_cast<size_t>(kTileM);
+  __nv_bfloat16* zp = at<__nv_bfloat16>(ws, L.zplanes);
+  const long long zps = static_cast<long long>(H) * Nv * L.Dpk;
+  // the projection writes z's planes and row norms itself when its two-row
+  // form runs
+  const bool zproj_planes = tc_keys && e == 16 && L.Dpk == 16 && d % 8 == 0;
   {
     // the side stream is joined on every path, also after a failed launch,
     // so that a stream capture in progress stays valid
@@ -760,24 +774,21 @@ sparsepr_status sparsepr_partition(const void* q, const void* k, sparsepr_dtype 
     if (err == cudaSuccess)
       err = launch_sym_eigs(mk, H, d, e, evl, evc, at<double>(ws, L.eigscr), st);
     if (err == cudaSuccess) err = launch_scale_columns(evl, evc, H, d, e, wk, st);
-    if (err == cudaSuccess) err = launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, st);
+    if (err == cudaSuccess)
+      err = launch_zproj(k, c.bf16, H, N, Nv, d, e, wk, z, zproj_planes ? zp : nullptr, zps,
+                         zproj_planes ? at<float>(ws, L.xnk) : nullptr, st);
     const cudaError_t ej = join_side(ss, side, st);
     SPR_TRY(err);
     SPR_TRY(ej);
   }
   const long long hs_z = static_cast<long long>(Nv) * e;
   SPR_TRY(launch_gather_init(z, kXf64, hs_z, e, e, init_k, Ck, H, mu, mun, st));
-  // tensor-core assignment when the centroid planes fit in shared memory
   const int sms = sm_count();
-  // (a 128-row TMA box needs at least 128 rows in the tensor)
-  const bool tc_keys = assign_tc_smem_bytes(3, 3, L.Dpk, L.CpadK) <= kMaxDynSmem &&
-                       static_cast<size_t>(H) * Nv >= static_cast<size_t>(kTileM);
   AssignTC ak;
   if (tc_keys) {
-    __nv_bfloat16* zp = at<__nv_bfloat16>(ws, L.zplanes);
-    const long long zps = static_cast<long long>(H) * Nv * L.Dpk;
-    SPR_TRY(launch_split_rows(z, kXf64, hs_z, e, Nv, e, L.Dpk, 3, H, zp, zps,
-                              at<float>(ws, L.xnk), st));
+    if (!zproj_planes)
+      SPR_TRY(launch_split_rows(z, kXf64, hs_z, e, Nv, e, L.Dpk, 3, H, zp, zps,
+                                at<float>(ws, L.xnk), st));
     ak = assign_common(c, ws, lab_k, flags, 0, sms);
     ak.a_planes = zp;
     ak.a_plane_stride = zps;

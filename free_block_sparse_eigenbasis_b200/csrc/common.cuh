@@ -274,6 +274,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Warp / block reductions (fixed order -> deterministic).
 // ---------------------------------------------------------------------------
 // 16 bytes of T (16-byte aligned), widened to fp64
+// 1/q for a finite q of normal magnitude: the approximate reciprocal of the
+// PTX instruction set refined by two Newton-Raphson steps for f(y) = 1/y - q,
+// y <- y + y (1 - q y) (each step squares the relative error; Muller et al.,
+// Handbook of Floating-Point Arithmetic, 2nd ed., sec. 4.7), so the result is
+// within a few ulp of 1/q, not correctly rounded (sparsepr_check_reciprocal
+// measures that against the correctly rounded reciprocal). The Sturm counts
+// keep |q| >= pivmin and |e2 / q| <= 1 / safe-minimum, so q is in range there.
+__device__ __forceinline__ double rcp_newton(double q) {
+  double y;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(q));
+  double r = fma(-q, y, 1.0);
+  y = fma(y, r, y);
+  r = fma(-q, y, 1.0);
+  return fma(y, r, y);
+}
+
 template <typename T>
 __device__ __forceinline__ void vwiden16(const uint4 u, double* out);
 template <>

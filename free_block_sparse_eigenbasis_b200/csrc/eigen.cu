@@ -183,21 +183,6 @@ __global__ void __launch_bounds__(kTriThreads, 1)
   }
 }
 
-// 1/q for a finite q of normal magnitude: the approximate reciprocal of the
-// PTX instruction set refined by two Newton-Raphson steps for f(y) = 1/y - q,
-// y <- y + y (1 - q y) (each step squares the relative error; Muller et al.,
-// Handbook of Floating-Point Arithmetic, 2nd ed., sec. 4.7), so the result is
-// within a few ulp of 1/q, not correctly rounded. The Sturm counts below keep
-// |q| >= pivmin and |e2 / q| <= 1 / safe-minimum, so q is always in range.
-__device__ __forceinline__ double rcp_newton(double q) {
-  double y;
-  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(q));
-  double r = fma(-q, y, 1.0);
-  y = fma(y, r, y);
-  r = fma(-q, y, 1.0);
-  return fma(y, r, y);
-}
-
 // Number of eigenvalues of T below each of P points x (Sturm sequences of
 // the LDL^T pivots), the P recurrences interleaved.
 template <int D, int P>
@@ -230,63 +215,62 @@ __device__ void sturm_counts(const double* dg, const double* e2, const double (&
 template <int D, int S>
 __device__ void tri_factor(const double* dg, const double* od, double lam, double tiny, double* a,
                            double* dl, double* du, double* du2, int* pv) {
-#pragma unroll 4
-  for (int i = 0; i < D; ++i) a[i * S] = dg[i] - lam;
-#pragma unroll 4
+  // the current diagonal entry and superdiagonal entry (as the previous
+  // step's elimination left them) are carried in registers, and each step
+  // picks its pivot row by selects, so that the chain from one step to the
+  // next holds no shared-memory round trip and no divergent branch
+  double a_cur = dg[0] - lam;
+  double du_cur = od[0];
+#pragma unroll 2
   for (int i = 0; i < D - 1; ++i) {
-    dl[i * S] = od[i];
-    du[i * S] = od[i];
-    du2[i * S] = 0.0;
+    const double li = od[i];
+    const double a_nx = dg[i + 1] - lam;
+    const double du_nx = (i < D - 2) ? od[i + 1] : 0.0;
+    const bool sw = !(fabs(a_cur) >= fabs(li));  // pivot on the subdiagonal row
+    const double piv = sw ? li : (a_cur == 0.0 ? tiny : a_cur);
+    const double f = (sw ? a_cur : li) / piv;
+    a[i * S] = piv;
+    dl[i * S] = f;
+    pv[i * S] = sw ? 1 : 0;
+    du[i * S] = sw ? a_nx : du_cur;
+    if (i < D - 2) du2[i * S] = sw ? du_nx : 0.0;
+    a_cur = sw ? fma(-f, a_nx, du_cur) : fma(-f, du_cur, a_nx);
+    du_cur = sw ? -f * du_nx : du_nx;
   }
-#pragma unroll 1
-  for (int i = 0; i < D - 1; ++i) {
-    const double ai = a[i * S], li = dl[i * S];
-    if (fabs(ai) >= fabs(li)) {
-      const double piv = (ai == 0.0) ? tiny : ai;
-      a[i * S] = piv;
-      const double f = li / piv;
-      dl[i * S] = f;
-      a[(i + 1) * S] -= f * du[i * S];
-      pv[i * S] = 0;
-    } else {
-      const double f = ai / li;
-      a[i * S] = li;
-      dl[i * S] = f;
-      const double t = du[i * S];
-      const double an = a[(i + 1) * S];
-      du[i * S] = an;
-      a[(i + 1) * S] = t - f * an;
-      if (i < D - 2) {
-        du2[i * S] = du[(i + 1) * S];
-        du[(i + 1) * S] = -f * du[(i + 1) * S];
-      }
-      pv[i * S] = 1;
-    }
-  }
-  if (a[(D - 1) * S] == 0.0) a[(D - 1) * S] = tiny;
+  a[(D - 1) * S] = (a_cur == 0.0) ? tiny : a_cur;
 #pragma unroll 8
   for (int i = 0; i < D; ++i) a[i * S] = 1.0 / a[i * S];  // independent: unrolled to overlap
 }
 
-// b <- (T - lam I)^-1 b with the factors of tri_factor.
+// b <- (T - lam I)^-1 b with the factors of tri_factor; returns |b|^2 of the
+// result. The element that the next step updates is carried in registers.
 template <int D, int S>
-__device__ void tri_apply(const double* ra, const double* dl, const double* du, const double* du2,
-                          const int* pv, double* b) {
-#pragma unroll 1
+__device__ double tri_apply(const double* ra, const double* dl, const double* du,
+                            const double* du2, const int* pv, double* b) {
+  double cur = b[0];
+#pragma unroll 4
   for (int i = 0; i < D - 1; ++i) {
-    if (pv[i * S] == 0) {
-      b[i + 1] -= dl[i * S] * b[i];
-    } else {
-      const double t = b[i];
-      b[i] = b[i + 1];
-      b[i + 1] = t - dl[i * S] * b[i];
-    }
+    const double nx = b[i + 1];
+    const bool sw = pv[i * S] != 0;
+    const double top = sw ? nx : cur;
+    const double bot = sw ? cur : nx;
+    b[i] = top;
+    cur = fma(-dl[i * S], top, bot);
   }
-  b[D - 1] *= ra[(D - 1) * S];
-  b[D - 2] = (b[D - 2] - du[(D - 2) * S] * b[D - 1]) * ra[(D - 2) * S];
-#pragma unroll 1
-  for (int i = D - 3; i >= 0; --i)
-    b[i] = (b[i] - du[i * S] * b[i + 1] - du2[i * S] * b[i + 2]) * ra[i * S];
+  double x1 = cur * ra[(D - 1) * S];                               // x_{i+2}
+  double x0 = (b[D - 2] - du[(D - 2) * S] * x1) * ra[(D - 2) * S];  // x_{i+1}
+  b[D - 1] = x1;
+  b[D - 2] = x0;
+  double nn = fma(x1, x1, x0 * x0);
+#pragma unroll 4
+  for (int i = D - 3; i >= 0; --i) {
+    const double xi = (b[i] - du[i * S] * x0 - du2[i * S] * x1) * ra[i * S];
+    b[i] = xi;
+    nn = fma(xi, xi, nn);
+    x1 = x0;
+    x0 = xi;
+  }
+  return nn;
 }
 
 // Fixed start vector of inverse iteration: components in [0.5, 1.5) from an
@@ -431,10 +415,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) tri_eig_kernel(const double* s
     for (int it = 0; it < kInvIters; ++it) {
       if (tid < nb) {
         double* bvec = Y[vi];
-        tri_apply<D, kInvBatch>(wa, wdl, wdu, wdu2, pv, bvec);
-        double sacc = 0.0;
-#pragma unroll 4
-        for (int i = 0; i < D; ++i) sacc = fma(bvec[i], bvec[i], sacc);
+        const double sacc = tri_apply<D, kInvBatch>(wa, wdl, wdu, wdu2, pv, bvec);
         const double inv = 1.0 / sqrt(sacc);
 #pragma unroll 4
         for (int i = 0; i < D; ++i) bvec[i] *= inv;
@@ -555,6 +536,26 @@ cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals
   if (d == 128) return launch_d<128>(A, H, ne, evals, evecs, scratch, st);
   if (d == 64) return launch_d<64>(A, H, ne, evals, evecs, scratch, st);
   return cudaErrorInvalidValue;
+}
+
+namespace {
+// err[i] = |rcp_newton(x[i]) - 1/x[i]| in units of the last place of the
+// correctly rounded 1/x[i] (__drcp_rn)
+__global__ void check_reciprocal_kernel(const double* x, long long n, double* err) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const double r = __drcp_rn(x[i]);
+  const double y = rcp_newton(x[i]);
+  int ex = 0;
+  frexp(r, &ex);
+  err[i] = fabs(y - r) / ldexp(1.0, ex - 53);
+}
+}  // namespace
+
+cudaError_t launch_check_reciprocal(const double* x, long long n, double* err, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  check_reciprocal_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(x, n, err);
+  return cudaGetLastError();
 }
 
 }  // namespace spr

@@ -59,8 +59,12 @@ cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
                             int ld, int S, int H, int d, double factor, double diag,
                             double* out, long long out_stride, long long mean_stride,
                             double* part, cudaStream_t st);
+// z = k W_K; with zp given (e = 16, d a multiple of 8, k 16-byte aligned)
+// also z's three bf16 planes (plane stride zps elements) and its row norms
+// rounded up, as launch_split_rows forms them
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
-                         const double* wk, double* z, cudaStream_t st);
+                         const double* wk, double* z, __nv_bfloat16* zp, long long zps,
+                         float* xnorm, cudaStream_t st);
 // dst[h, c, :] = src[h, idx[h, c], :] (as fp64) and norms[h, c] = |dst|^2 (norms may be null)
 cudaError_t launch_gather_init(const void* src, int src_kind, long long head_stride, int ld,
                                int D, const int32_t* idx, int C, int H, double* dst,
@@ -166,6 +170,8 @@ cudaError_t launch_scale_columns(const double* vals, const double* vecs, int H, 
 // bisection and inverse iteration ---------------------------------------------
 size_t sym_eigs_scratch_doubles(int H, int d);
 // evals [H, ne] descending, evecs [H, d, ne].
+// err[i]: distance in ulp of rcp_newton(x[i]) from the correctly rounded 1/x[i]
+cudaError_t launch_check_reciprocal(const double* x, long long n, double* err, cudaStream_t st);
 cudaError_t launch_sym_eigs(const double* A, int H, int d, int ne, double* evals, double* evecs,
                             double* scratch, cudaStream_t st);
 

@@ -266,6 +266,8 @@ inline bool named_region(const sparsepr_params& p, const Layout& L, const char* 
       {"g", L.g, H * d * d * 8},        {"bmat", L.bmat, H * d * d * 8},
       {"bvec", L.bvec, H * d * 8},      {"xr", L.xr, H * 2 * M * d * 8},
       {"vr", p.r <= kTriEigMax ? L.evec : L.gram, H * d * static_cast<size_t>(p.r) * 8},
+      {"zplanes", L.zplanes, 3 * H * Nv * static_cast<size_t>(L.Dpk) * 2},
+      {"xnk", L.xnk, H * Nv * 4},
   };
   for (const R& r : tab) {
     const char* a = r.n;

@@ -65,13 +65,18 @@ __global__ void fy_init_kernel(int Nv, int Ck, int Cq, uint64_t seed, int32_t* i
 // coordinates of each in registers; the rows of k are streamed with 16-byte
 // loads and W [d][16] is read from shared memory as 16-byte broadcasts, so
 // every value of W read serves two rows. Same ascending-column sums as
-// above.
+// above. With `zp` given it also writes what the tensor-core assignment
+// reads of each row: its three bf16 planes (hi, mid, lo: each the bf16
+// rounding of what the planes before it leave) and its norm rounded up, with
+// the squares summed in the order of split_rows_vec_kernel (pairs of
+// columns, then a butterfly over eight of them), so both give the same bits.
 constexpr int kZRowThreads = 128;
 constexpr int kZ16Rows = 2;  // rows per thread
 
 template <typename T>
 __global__ void __launch_bounds__(kZRowThreads)
-    zproj_row16_kernel(const T* k, int N, int Nv, int d, const double* wk, double* z) {
+    zproj_row16_kernel(const T* k, int N, int Nv, int d, const double* wk, double* z,
+                       __nv_bfloat16* zp, long long zps, float* xnorm) {
   constexpr int E = 16, EPT = 16 / sizeof(T);
   extern __shared__ double w16[];  // [d][16]
   const int h = blockIdx.y;
@@ -114,6 +119,27 @@ __global__ void __launch_bounds__(kZRowThreads)
         z + (static_cast<size_t>(h) * Nv + j0 + r * kZRowThreads) * E);
 #pragma unroll
     for (int c2 = 0; c2 < E / 2; ++c2) zr[c2] = make_double2(acc[r][2 * c2], acc[r][2 * c2 + 1]);
+    if (zp) {
+      const size_t row = static_cast<size_t>(h) * Nv + j0 + r * kZRowThreads;
+      double s8[E / 2];
+#pragma unroll
+      for (int t = 0; t < E / 2; ++t)
+        s8[t] = fma(acc[r][2 * t + 1], acc[r][2 * t + 1], acc[r][2 * t] * acc[r][2 * t]);
+      const double ss = ((s8[0] + s8[4]) + (s8[2] + s8[6])) + ((s8[1] + s8[5]) + (s8[3] + s8[7]));
+      xnorm[row] = static_cast<float>(sqrt(ss) * (1.0 + 1e-6));
+#pragma unroll
+      for (int pl = 0; pl < 3; ++pl) {
+        __align__(16) __nv_bfloat16 b[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          b[i] = __double2bfloat16(acc[r][i]);
+          acc[r][i] -= static_cast<double>(__bfloat162float(b[i]));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(zp + pl * zps + row * E);
+        dst[0] = *reinterpret_cast<const uint4*>(b);
+        dst[1] = *reinterpret_cast<const uint4*>(b + 8);
+      }
+    }
   }
 }
 
@@ -1088,16 +1114,21 @@ cudaError_t launch_gram_f64(const double* X, const double* Y, const double* xm,
 }
 
 cudaError_t launch_zproj(const void* k, bool bf16, int H, int N, int Nv, int d, int e,
-                         const double* wk, double* z, cudaStream_t st) {
-  if (e == 16 && d % 8 == 0 && reinterpret_cast<uintptr_t>(k) % 16 == 0) {
+                         const double* wk, double* z, __nv_bfloat16* zp, long long zps,
+                         float* xnorm, cudaStream_t st) {
+  const bool row16 = e == 16 && d % 8 == 0 && reinterpret_cast<uintptr_t>(k) % 16 == 0;
+  // the planes only with the two-row form
+  if (zp && (!row16 || !xnorm || reinterpret_cast<uintptr_t>(zp) % 16 != 0 || zps % 8 != 0))
+    return cudaErrorInvalidValue;
+  if (row16) {
     const size_t shb16 = static_cast<size_t>(d) * 16 * 8;
     dim3 g16((Nv + kZRowThreads * kZ16Rows - 1) / (kZRowThreads * kZ16Rows), H);
     if (bf16)
       zproj_row16_kernel<<<g16, kZRowThreads, shb16, st>>>(static_cast<const __nv_bfloat16*>(k), N, Nv,
-                                                           d, wk, z);
+                                                           d, wk, z, zp, zps, xnorm);
     else
       zproj_row16_kernel<<<g16, kZRowThreads, shb16, st>>>(static_cast<const float*>(k), N, Nv, d,
-                                                           wk, z);
+                                                           wk, z, zp, zps, xnorm);
     return cudaGetLastError();
   }
   const size_t shb = static_cast<size_t>(d) * e * 8 + static_cast<size_t>(kZRows) * (d + 1) * 4;

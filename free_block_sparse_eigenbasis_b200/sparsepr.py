@@ -26,7 +26,8 @@ EXPORTED = ("sparsepr_workspace_bytes", "sparsepr_status_string", "sparsepr_part
             "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
             "sparsepr_reset_stats", "sparsepr_check_wait_limit", "sparsepr_route_noalloc",
             "sparsepr_workspace_region", "sparsepr_probe_diagnostics",
-            "sparsepr_support_expansion", "sparsepr_density_profile", "sparsepr_attention")
+            "sparsepr_support_expansion", "sparsepr_density_profile", "sparsepr_attention",
+            "sparsepr_check_reciprocal")
 
 
 class Params(ctypes.Structure):
@@ -102,6 +103,8 @@ def _load():
     lib.sparsepr_read_stats.argtypes = [V, ctypes.POINTER(Stats)]
     lib.sparsepr_reset_stats.argtypes = [V, V]
     lib.sparsepr_check_wait_limit.argtypes = [V, V]
+    lib.sparsepr_check_reciprocal.argtypes = [P, ctypes.c_int64, P, V]
+    lib.sparsepr_check_reciprocal.restype = st
     for name in ("sparsepr_partition", "sparsepr_permute", "sparsepr_route",
                  "sparsepr_block_sparse_attn", "sparsepr_probe_correct", "sparsepr_read_stats",
                  "sparsepr_reset_stats", "sparsepr_check_wait_limit"):
@@ -345,7 +348,19 @@ def sparsepr_check_wait_limit(ws, stream=None):
     _check(lib.sparsepr_check_wait_limit(_ws(ws)[0], _stream(stream)), "sparsepr_check_wait_limit")
 
 
-_REGION_DTYPES = dict(init_k=torch.int32, init_q=torch.int32)
+def sparsepr_check_reciprocal(x, stream=None):
+    """Distance in ulp of the multisection's reciprocal from the correctly
+    rounded 1/x, for a 1-D fp64 device tensor x; returns a tensor like x."""
+    if x.dtype != torch.float64 or x.dim() != 1 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x: a contiguous 1-D float64 CUDA tensor")
+    err = torch.empty_like(x)
+    _check(lib.sparsepr_check_reciprocal(x.data_ptr(), x.numel(), err.data_ptr(), _stream(stream)),
+           "sparsepr_check_reciprocal")
+    return err
+
+
+_REGION_DTYPES = dict(init_k=torch.int32, init_q=torch.int32, zplanes=torch.bfloat16,
+                      xnk=torch.float32)
 
 
 def sparsepr_workspace_region(p: dict, name: str):
@@ -359,8 +374,9 @@ def sparsepr_workspace_region(p: dict, name: str):
 
 
 def workspace_view(ws, p: dict, name: str) -> torch.Tensor:
-    """The named region of `ws` as a flat tensor of its element type (fp64,
-    or int32 for the initial centroid rows); a view, no copy."""
+    """The named region of `ws` as a flat tensor of its element type (fp64;
+    int32 for the initial centroid rows, bf16 for the key planes, fp32 for
+    the key row norms); a view, no copy."""
     off, nb = sparsepr_workspace_region(p, name)
     return ws[off:off + nb].view(_REGION_DTYPES.get(name, torch.float64))
 

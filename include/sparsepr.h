@@ -323,6 +323,11 @@ sparsepr_status sparsepr_attention(const void* q, const void* k, const void* v, 
  *     "ck"     [H, Ck, d] fp64: K group means in the original space over the
  *             final key labels (the zero vector for an empty group)
  *     "g"      [H, d, d] fp64: query metric G = scale^2 C_K^T C_K
+ *     "zplanes" [3, H, Nv, Dp] bf16 (Dp = 16 for n_eig <= 16, else 64): z
+ *             split into three bf16 planes (each the rounding of what the
+ *             planes before it leave of z; zero padded to Dp columns), the
+ *             operands of the tensor-core key assignment
+ *     "xnk"    [H, Nv] fp32: |z_j| rounded up, for the assignment's bound
  *   written by sparsepr_probe_correct [SPR 2.B] (M > 0; it also reuses
  *   "mk", "eval" and "evec" for R^T R and its eigenpairs):
  *     "bmat"   [H, d, d] fp64, "bvec" [H, d] fp64: the ridge solution B, b
@@ -408,6 +413,16 @@ sparsepr_status sparsepr_reset_stats(void* ws, void* stream);
  * synchronising. Errors: INVALID_ARG for a NULL or not 256-byte-aligned `ws`,
  * CUDA for a failed launch. */
 sparsepr_status sparsepr_check_wait_limit(void* ws, void* stream);
+
+/* Check of the reciprocal the eigenvalue multisection uses in its Sturm
+ * counts (Golub & Van Loan, Matrix Computations, sec. 8.4.1): the PTX
+ * approximate reciprocal refined by two Newton-Raphson steps, which is not
+ * correctly rounded. For n device doubles x (finite, nonzero, of normal
+ * magnitude) it writes to the device array err[n] the distance of that
+ * reciprocal from the correctly rounded 1/x, in units of the last place of
+ * the latter. Enqueued on `stream`. Errors: INVALID_ARG for n < 0 or a NULL
+ * array with n > 0, CUDA for a failed launch. */
+sparsepr_status sparsepr_check_reciprocal(const double* x, int64_t n, double* err, void* stream);
 
 #ifdef __cplusplus
 }

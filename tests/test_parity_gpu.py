@@ -272,3 +272,29 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable():
     assert S.sparsepr_read_stats(b.ws)["status"] == 0
     res = oracle_head(w, q, k, v, 0)
     compare_head(b, res, w, 0, None)
+
+
+def test_multisection_reciprocal_within_two_ulp():
+    """The reciprocal in the eigenvalue multisection's Sturm counts (an
+    approximate reciprocal refined by two Newton-Raphson steps, not correctly
+    rounded) against CUDA's correctly rounded one: within 2 ulp over random
+    mantissas across the normal range, both signs, powers of two and the
+    magnitudes the counts meet (pivots down to the safe minimum times the
+    largest squared off-diagonal)."""
+    S = _S()
+    g = torch.Generator().manual_seed(7)
+    n = 1 << 20
+    mant = 1.0 + torch.rand(n, generator=g, dtype=torch.float64)
+    expo = torch.randint(-1020, 1020, (n,), generator=g)
+    sign = torch.where(torch.rand(n, generator=g) < 0.5, -1.0, 1.0).double()
+    x = sign * torch.ldexp(mant, expo)
+    special = torch.tensor([1.0, -1.0, 2.0, 0.5, 3.0, 1.0 / 3.0, 2.2250738585072014e-308,
+                            -2.2250738585072014e-308, 4.0 * 2.2250738585072014e-308,
+                            1.7976931348623157e+308 / 4.0, 0.1, -7.0, 1e-300, 1e300],
+                           dtype=torch.float64)
+    xd = torch.cat([x, special]).cuda()
+    err = S.sparsepr_check_reciprocal(xd)
+    torch.cuda.synchronize()
+    e = err.cpu()
+    assert torch.isfinite(e).all()
+    assert e.max().item() <= 2.0, e.max().item()

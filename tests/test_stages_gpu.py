@@ -115,3 +115,46 @@ def test_partition_stages_match_oracle(w):
         CK = O.group_means(kv, labels, Ck)
         check_rel(R["ck"].reshape(H, Ck, d)[h], CK, 1e-12, "C_K head %d" % h)
         check_rel(R["g"].reshape(H, d, d)[h], scale * scale * (CK.T @ CK), 1e-12, "G head %d" % h)
+
+
+def _bf16_rne(x):
+    """fp64 -> nearest bf16 value (ties to even), as fp64; normal range."""
+    b = np.ascontiguousarray(x, dtype=np.float64).view(np.uint64)
+    half = np.uint64((1 << 44) - 1) + ((b >> np.uint64(45)) & np.uint64(1))
+    r = (b + half) & ~np.uint64((1 << 45) - 1)
+    return r.view(np.float64)
+
+
+PLANE_CASES = [
+    synth.custom("planes_bf16_d128_e16", 2, (4, 16, 32), 128, "bf16", Ck=64, Cq=16, Ms=256,
+                 n_eig=16, M=64, r=16, keep=0.3, seed=13),
+    synth.workload("wan13b_480p"),
+]
+
+
+@pytest.mark.parametrize("w", PLANE_CASES, ids=[x.name for x in PLANE_CASES])
+def test_key_planes_and_norms_from_z(w):
+    """The bf16 planes of the key coordinates (written by the projection
+    itself for e = 16) are z split exactly: plane 1 is the nearest bf16 of
+    z, plane 2 of what it leaves, plane 3 of what both leave; the stored row
+    norms bound |z| from above by at most 1e-6 relative plus float rounding."""
+    S = _S()
+    b, q, k, p, R = run_partition(w)
+    H, Nv, e = w.H, w.Nv, w.n_eig
+    assert e == 16
+    z = R["z"].reshape(H * Nv, e)
+    planes = S.workspace_view(b.ws, p, "zplanes").float().cpu().numpy().astype(np.float64)
+    planes = planes.reshape(3, H * Nv, 16)
+    rest = z.copy()
+    for pl in range(3):
+        want = _bf16_rne(rest)
+        assert np.array_equal(planes[pl], want), ("plane", pl, np.abs(planes[pl] - want).max())
+        rest = rest - want
+    # a planted one-ulp change of one element in the first plane is seen
+    bad = planes[0].copy()
+    bad[0, 0] = np.nextafter(np.float32(bad[0, 0]), np.float32(np.inf))
+    assert not np.array_equal(bad, _bf16_rne(z))
+    xn = S.workspace_view(b.ws, p, "xnk").cpu().numpy().astype(np.float64)
+    nz = np.sqrt((z * z).sum(axis=1))
+    assert (xn >= nz * (1 - 1e-12)).all()
+    assert (xn <= nz * (1 + 1e-6) * (1 + 2.0 ** -23) + 1e-300).all()
