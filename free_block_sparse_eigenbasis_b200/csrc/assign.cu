@@ -500,10 +500,18 @@ __global__ void __launch_bounds__(kRcThreads)
   const double* Yh = yT + static_cast<size_t>(h) * D * m;
   const double* ch = DIRECT ? nullptr : c + static_cast<size_t>(h) * m;
   const double* Gh = (!DIRECT && G) ? G + static_cast<size_t>(h) * D * D : nullptr;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0) {  // trace of G, for the near-tie test (blocks with rows)
     double t = 0.0;
-    if (Gh)
-      for (int a = 0; a < D; ++a) t += Gh[static_cast<size_t>(a) * D + a];
+    if (Gh && static_cast<long long>(blockIdx.x) * R < cnt) {
+#pragma unroll 1
+      for (int a0 = 0; a0 < D; a0 += 8) {  // eight loads in flight, summed in order
+        double g[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) g[q] = (a0 + q < D) ? Gh[static_cast<size_t>(a0 + q) * (D + 1)] : 0.0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) t += g[q];
+      }
+    }
     gtr = t;
   }
   int ties = 0;

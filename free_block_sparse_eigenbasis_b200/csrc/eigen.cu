@@ -183,6 +183,28 @@ __global__ void __launch_bounds__(kTriThreads, 1)
   }
 }
 
+// Gershgorin bound max_i |d_i| + |e_{i-1}| + |e_i| of T and the largest
+// squared off-diagonal entry, by the calling warp (lanes over the rows, then
+// a max over the lanes: the result does not depend on the order).
+template <int D>
+__device__ __forceinline__ void tri_bounds(const double* dg, const double* od, int lane,
+                                           double* tnorm, double* emax2) {
+  double m = 0.0, e = 0.0;
+  for (int i = lane; i < D; i += 32) {
+    m = fmax(m, fabs(dg[i]) + (i > 0 ? fabs(od[i - 1]) : 0.0) + (i < D - 1 ? fabs(od[i]) : 0.0));
+    if (i < D - 1) e = fmax(e, od[i] * od[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    e = fmax(e, __shfl_xor_sync(0xffffffffu, e, o));
+  }
+  if (lane == 0) {
+    *tnorm = m;
+    if (emax2) *emax2 = e;
+  }
+}
+
 // Number of eigenvalues of T below each of P points x (Sturm sequences of
 // the LDL^T pivots), the P recurrences interleaved.
 template <int D, int P>
@@ -304,7 +326,7 @@ template <int D>
 __global__ void __launch_bounds__(kBisWarps * 32) multisect_kernel(const double* scratch, int ne,
                                                                   double* evals) {
   __shared__ double dg[D], od[D], e2[D];
-  __shared__ double tnorm;
+  __shared__ double tnorm, emax2_s;
   const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   const double* tau = scratch + static_cast<size_t>(h) * (D * D + 3 * D) + D * D;
   for (int i = tid; i < D; i += blockDim.x) {
@@ -313,18 +335,12 @@ __global__ void __launch_bounds__(kBisWarps * 32) multisect_kernel(const double*
     e2[i] = (i < D - 1) ? od[i] * od[i] : 0.0;
   }
   __syncthreads();
-  if (tid == 0) {  // the same bound as tri_eig_kernel's
-    double m = 0.0;
-    for (int i = 0; i < D; ++i)
-      m = fmax(m, fabs(dg[i]) + (i > 0 ? fabs(od[i - 1]) : 0.0) + (i < D - 1 ? fabs(od[i]) : 0.0));
-    tnorm = m;
-  }
+  if (tid < 32) tri_bounds<D>(dg, od, lane, &tnorm, &emax2_s);  // the same bound as tri_eig_kernel's
   __syncthreads();
   const int e_i = blockIdx.y * kBisWarps + (tid >> 5);
   if (e_i >= ne) return;  // the whole warp
   const double eps = 1.1102230246251565e-16;
-  double emax2 = 0.0;
-  for (int i = 0; i < D - 1; ++i) emax2 = fmax(emax2, e2[i]);
+  const double emax2 = emax2_s;
   const double pivmin = 2.2250738585072014e-308 * fmax(1.0, emax2);
   const int m = D - 1 - e_i;
   const double inv_parts = 1.0 / 33.0;
@@ -382,12 +398,7 @@ __global__ void __launch_bounds__(kEigThreads, 1) tri_eig_kernel(const double* s
     od[i] = tau[2 * D + i];
   }
   __syncthreads();
-  if (tid == 0) {
-    double m = 0.0;
-    for (int i = 0; i < D; ++i)
-      m = fmax(m, fabs(dg[i]) + (i > 0 ? fabs(od[i - 1]) : 0.0) + (i < D - 1 ? fabs(od[i]) : 0.0));
-    tnorm = m;
-  }
+  if (tid < 32) tri_bounds<D>(dg, od, lane, &tnorm, nullptr);
   __syncthreads();
   const double eps = 1.1102230246251565e-16;
   // the eigenvalues, from multisect_kernel

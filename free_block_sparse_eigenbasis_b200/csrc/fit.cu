@@ -9,6 +9,46 @@
 namespace spr {
 namespace {
 
+// Exclusive prefix sums of v[0..n) into out (out may be v), and the total,
+// by the whole block (blockDim.x a multiple of 32): chunks of blockDim.x
+// values, a warp scan by shuffles, then the warp totals. Integer sums, so
+// the result does not depend on the order.
+__device__ int32_t block_exclusive_scan(const int32_t* v, int32_t* out, int n) {
+  __shared__ int32_t warp_tot[32];
+  __shared__ int32_t carry;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int c = base + threadIdx.x;
+    const int32_t x0 = (c < n) ? v[c] : 0;
+    int32_t x = x0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int32_t t = (lane < nw) ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      if (lane < nw) warp_tot[lane] = t;
+    }
+    __syncthreads();
+    const int32_t before = carry + (wid > 0 ? warp_tot[wid - 1] : 0) + (x - x0);
+    __syncthreads();  // every thread has read carry and warp_tot
+    if (c < n) out[c] = before;
+    if (threadIdx.x == blockDim.x - 1) carry = before + x0;
+    __syncthreads();
+  }
+  return carry;
+}
+
 // Probes per query group by largest remainder (ties to the lower group),
 // rows at offsets floor((t + 1/2) n_g / m_g) inside each group.
 __global__ void probe_select_kernel(const int32_t* off_q, int off_stride, int Cq, int M,
@@ -27,11 +67,10 @@ __global__ void probe_select_kernel(const int32_t* off_q, int off_stride, int Cq
     m[g] = static_cast<int32_t>(Nt > 0 ? num / Nt : 0);
     rem[g] = Nt > 0 ? num % Nt : 0;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int64_t s = 0;
-    for (int g = 0; g < Cq; ++g) s += m[g];
-    left = static_cast<int32_t>(M - s);
+  {
+    // the floors' total (start is free here); each m[g] <= M, so it fits
+    const int32_t s = block_exclusive_scan(m, start, Cq);
+    if (threadIdx.x == 0) left = M - s;
   }
   __syncthreads();
   // rank of each remainder (larger first, lower group on ties)
@@ -45,13 +84,7 @@ __global__ void probe_select_kernel(const int32_t* off_q, int off_stride, int Cq
   for (int g = threadIdx.x; g < Cq; g += blockDim.x)
     if (start[g] < left) m[g] += 1;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t s = 0;
-    for (int g = 0; g < Cq; ++g) {
-      start[g] = s;
-      s += m[g];
-    }
-  }
+  block_exclusive_scan(m, start, Cq);
   __syncthreads();
   int32_t* out = probes + static_cast<size_t>(h) * M;
   int32_t* grp = pgrp ? pgrp + static_cast<size_t>(h) * M : nullptr;

@@ -74,7 +74,7 @@ constexpr int kZRowThreads = 128;
 constexpr int kZ16Rows = 2;  // rows per thread
 
 template <typename T>
-__global__ void __launch_bounds__(kZRowThreads)
+__global__ void __launch_bounds__(kZRowThreads, 4)
     zproj_row16_kernel(const T* k, int N, int Nv, int d, const double* wk, double* z,
                        __nv_bfloat16* zp, long long zps, float* xnorm) {
   constexpr int E = 16, EPT = 16 / sizeof(T);
@@ -93,11 +93,21 @@ __global__ void __launch_bounds__(kZRowThreads)
   for (int r = 0; r < kZ16Rows; ++r)
 #pragma unroll
     for (int c = 0; c < E; ++c) acc[r][c] = 0.0;
+  // the next 16-byte pieces of both rows are loaded while the current ones
+  // are multiplied
+  uint4 u0 = *reinterpret_cast<const uint4*>(kr0), u1 = *reinterpret_cast<const uint4*>(kr1);
 #pragma unroll 1
   for (int a0 = 0; a0 < d; a0 += EPT) {
+    uint4 n0 = u0, n1 = u1;
+    if (a0 + EPT < d) {
+      n0 = *reinterpret_cast<const uint4*>(kr0 + a0 + EPT);
+      n1 = *reinterpret_cast<const uint4*>(kr1 + a0 + EPT);
+    }
     double kv[kZ16Rows][EPT];
-    vload16(kr0 + a0, kv[0]);
-    vload16(kr1 + a0, kv[1]);
+    vwiden16<T>(u0, kv[0]);
+    vwiden16<T>(u1, kv[1]);
+    u0 = n0;
+    u1 = n1;
 #pragma unroll
     for (int i = 0; i < EPT; ++i) {
       const double2* wa = reinterpret_cast<const double2*>(w16 + (a0 + i) * E);
