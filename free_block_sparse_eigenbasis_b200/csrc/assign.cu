@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(kRcThreads)
                    const double* yT, const double* c, int m, int32_t* labels, int32_t* flags,
                    int flag_base, const int32_t* recheck, const int32_t* nrecheck,
                    const double* G, DeviceStats* stats) {
-  __shared__ double xs[R][kRcMaxD];
+  __shared__ __align__(16) double xs[R][kRcMaxD];
   __shared__ double wb1[R][kRcWarps], wb2[R][kRcWarps];
   __shared__ int wbi[R][kRcWarps];
   __shared__ int rows_s[R], cand_s[R];
@@ -545,7 +545,30 @@ __global__ void __launch_bounds__(kRcThreads)
           }
         }
       };
-      if (DT > 0 && DT <= 16) {
+      // columns t and t + 1 (t even) with one 16-byte shared load per row:
+      // the same FMAs in the same order as two steps
+      auto step2 = [&](int t, double y0, double y1) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const double2 xv = *reinterpret_cast<const double2*>(&xs[r][t]);
+          if (DIRECT) {
+            const double e0 = xv.x - y0;
+            acc[r] = fma(e0, e0, acc[r]);
+            const double e1 = xv.y - y1;
+            acc[r] = fma(e1, e1, acc[r]);
+          } else {
+            acc[r] = fma(xv.x, y0, acc[r]);
+            acc[r] = fma(xv.y, y1, acc[r]);
+          }
+        }
+      };
+      if (DT > 0 && DT <= 16 && DT % 2 == 0) {
+        double y[DT > 0 ? DT : 1];
+#pragma unroll
+        for (int t = 0; t < DT; ++t) y[t] = Yh[static_cast<size_t>(t) * m + j];
+#pragma unroll
+        for (int t = 0; t < DT; t += 2) step2(t, y[t], y[t + 1]);
+      } else if (DT > 0 && DT <= 16) {
 #pragma unroll
         for (int t = 0; t < DT; ++t) step(t, Yh[static_cast<size_t>(t) * m + j]);
       } else if (DT > 0) {
@@ -559,12 +582,12 @@ __global__ void __launch_bounds__(kRcThreads)
 #pragma unroll
           for (int q = 0; q < 8; ++q) yb[q] = Yh[static_cast<size_t>(t + 8 + q) * m + j];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) step(t + q, ya[q]);
+          for (int q = 0; q < 8; q += 2) step2(t + q, ya[q], ya[q + 1]);
           if (t + 16 < DT)
 #pragma unroll
             for (int q = 0; q < 8; ++q) ya[q] = Yh[static_cast<size_t>(t + 16 + q) * m + j];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) step(t + 8 + q, yb[q]);
+          for (int q = 0; q < 8; q += 2) step2(t + 8 + q, yb[q], yb[q + 1]);
         }
       } else {
         int t = 0;
