@@ -679,22 +679,28 @@ __global__ void __launch_bounds__(kRcThreads)
 
 template <bool DIRECT>
 void launch_recheck_d(const AssignTC& a, cudaStream_t st) {
-  // short rows (D <= 16): one row per block over 128 blocks per head;
-  // longer rows: batches of kRcRows over 64 blocks per head
+  // short rows (D <= 16): one row per block at a time over at most 128
+  // blocks per head; longer rows: batches of kRcRows over at most 64 blocks
+  // per head. In all no more blocks than two per SM (one wave at two
+  // resident blocks of 256 threads at up to 128 registers), so that the
+  // blocks with rows do not wait behind waves of blocks without.
+  const int nb_all = 2 * (a.sm_count > 0 ? a.sm_count : 148) / (a.H > 0 ? a.H : 1);
+  const int nb1 = nb_all > 128 ? 128 : (nb_all < 1 ? 1 : nb_all);
+  const int nb8 = nb_all > 64 ? 64 : (nb_all < 1 ? 1 : nb_all);
 #define SPR_RC(DT, R, NB)                                                                       \
   recheck_kernel<DT, DIRECT, R><<<dim3(NB, a.H), kRcThreads, 0, st>>>(                        \
       a.x_exact, a.x_kind, a.x_hs, a.x_ld, a.n, a.D, a.y_tr, a.c_exact, a.m, a.labels, a.flags, \
       a.flag_base, a.recheck, a.nrecheck, a.metric, a.stats)
   if (a.D == 16)
-    SPR_RC(16, 1, 128);
+    SPR_RC(16, 1, nb1);
   else if (a.D == 64)
-    SPR_RC(64, kRcRows, 64);
+    SPR_RC(64, kRcRows, nb8);
   else if (a.D == 128)
-    SPR_RC(128, kRcRows, 64);
+    SPR_RC(128, kRcRows, nb8);
   else if (a.D < 16)
-    SPR_RC(0, 1, 128);
+    SPR_RC(0, 1, nb1);
   else
-    SPR_RC(0, kRcRows, 64);
+    SPR_RC(0, kRcRows, nb8);
 #undef SPR_RC
 }
 
