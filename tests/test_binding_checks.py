@@ -116,3 +116,13 @@ def test_host_tensors_are_rejected():
         S.sparsepr_partition(q, q, p, b.label_q, b.label_k, b.ws, _Stream())
     with pytest.raises(ValueError, match="CUDA tensor"):
         S.sparsepr_read_stats(b.ws)
+
+
+def test_reciprocal_check_rejects_tensors_it_cannot_pass():
+    """The reciprocal self-check takes a contiguous 1-D fp64 CUDA tensor only;
+    anything else is refused in the binding, before the library is called."""
+    for bad in (torch.zeros(4, dtype=torch.float64),                 # host memory
+                torch.zeros(4, dtype=torch.float32),
+                torch.zeros((2, 2), dtype=torch.float64)):
+        with pytest.raises(ValueError):
+            S.sparsepr_check_reciprocal(bad)
