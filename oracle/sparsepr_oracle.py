@@ -135,9 +135,10 @@ NEAR_TIE_REL = 1e-12
 def count_near_ties(D: np.ndarray) -> int:
     """Rows of a distance matrix whose two smallest squared distances
     d1 <= d2 satisfy d2 - d1 <= 1e-12 d2: rows whose nearest centroid is
-    decided by rounding rather than by the data (reading: the survey's
-    "several correct results" point; exact ties, e.g. two identical
-    centroids, count, and the lowest index wins them)."""
+    decided by rounding rather than by the data (reading: such a row has
+    more than one correct label, so it is counted and reported rather than
+    compared; exact ties, e.g. two identical centroids, count, and the
+    lowest index wins them)."""
     if D.shape[1] < 2:
         return 0
     two = np.partition(D, 1, axis=1)[:, :2]
