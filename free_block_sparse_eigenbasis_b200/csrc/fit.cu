@@ -12,7 +12,8 @@ namespace {
 // Exclusive prefix sums of v[0..n) into out (out may be v), and the total,
 // by the whole block (blockDim.x a multiple of 32): chunks of blockDim.x
 // values, a warp scan by shuffles, then the warp totals. Integer sums, so
-// the result does not depend on the order.
+// the result does not depend on the order. Every thread reads the total from
+// shared memory on return, so two calls must be separated by a barrier.
 __device__ int32_t block_exclusive_scan(const int32_t* v, int32_t* out, int n) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
